@@ -1,0 +1,191 @@
+/*
+ * cqsa.h -- C ABI of the CQS-decomposed exact attention library (libcqsa.so).
+ *
+ * The library computes exact softmax attention over one sequence by the CQS
+ * Divide of Stream-CQSA: the N tokens are split into c = l(l-1)+1 chunks; the
+ * c cyclic subsequences S_k = {(x + k) mod c : x in D} (D a perfect
+ * difference set) each run masked attention so that every ordered chunk pair
+ * is computed exactly once; each task emits local softmax statistics and a
+ * log-sum-exp merge recomposes them into the full output.  Subsequences can
+ * be divided again (recursion), and inputs held in pinned host memory are
+ * streamed through a bounded device working set.
+ *
+ * Sources (page title, section):
+ *   [A] "Stream-CQSA: Exact Out-of-Memory Recovery for Attention" (arXiv
+ *       abstract page): recursive partition into independent subsequence
+ *       tasks, recomposition of local statistics, exact output.
+ *   [B] "Stream-CQSA: Breaking the Billion-Token Barrier on a Single GPU"
+ *       (wispaper.ai blog): section "The CQS Divide" (c = l(l-1)+1, every
+ *       chunk pair exactly once, Steiner system S(2,l,c)); section "The
+ *       Recursive Benefit" (divide again until it fits); section
+ *       "Implementation" (CQS mask, stream Q_i/K_i/V_i to the GPU, local
+ *       numerators and denominators, aggregate); section "Performance"
+ *       (host-device transfer overhead).
+ *   [C] layerthelatestinalattice.com summary: subproblems sized to fit a
+ *       stated memory budget; recomposition equals full attention.
+ *
+ * Conventions for every call:
+ *   - Tensors q, k, v, out are [N, H, d] contiguous (one sequence, B = 1) in
+ *     the plan's dtype; lse is fp32 [H, N], the natural log of the sum of
+ *     exp(score) with score = <q_i, k_j> / sqrt(d).
+ *   - The caller owns every tensor.  The plan owns its device arena, its
+ *     streams and events; it never allocates device memory after the first
+ *     forward call, and its arena never exceeds mem_budget_bytes when a
+ *     budget is given.
+ *   - No call aborts or exits.  Each returns a status; on failure
+ *     cqsa_last_error() holds a message (thread-local).
+ */
+#ifndef CQSA_H
+#define CQSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct cqsa_plan cqsa_plan_t; /* opaque; created by cqsa_plan*, freed by cqsa_plan_destroy */
+
+typedef enum {
+    CQSA_OK = 0,
+    CQSA_ERR_INVALID_ARG = 1,       /* null pointer, bad size, N not divisible by the chunk product */
+    CQSA_ERR_NO_DIFFERENCE_SET = 2, /* no perfect difference set of size l mod l(l-1)+1 (e.g. l = 7) */
+    CQSA_ERR_BUDGET = 3,            /* no working set fits mem_budget_bytes */
+    CQSA_ERR_NOT_PINNED = 4,        /* host mode given a pointer that is not page-locked host memory */
+    CQSA_ERR_CUDA = 5,              /* a CUDA runtime call failed; message names it */
+    CQSA_ERR_TIMEOUT = 6,           /* a bounded device-side wait ran out; the kernel stopped early */
+    CQSA_ERR_UNSUPPORTED = 7,       /* valid request this build does not implement (e.g. d not 64/128) */
+    CQSA_ERR_NO_DEVICE = 8          /* no usable sm_100 device */
+} cqsa_status_t;
+
+typedef enum { CQSA_BF16 = 0, CQSA_FP32 = 1 } cqsa_dtype_t;
+
+enum { CQSA_DEVICE = 0, CQSA_HOST = 1 };
+
+#define CQSA_MAX_LEVELS 4
+#define CQSA_MAX_L 16
+
+/* Full plan description.  levels >= 1 and l[0..levels-1] each >= 2; the
+ * leaf block is N / prod_i (l_i (l_i - 1) + 1) tokens.  mem_budget_bytes = 0
+ * means unlimited. */
+typedef struct {
+    int64_t N;
+    int H;
+    int d;
+    int levels;
+    int l[CQSA_MAX_LEVELS];
+    int causal;
+    int dtype; /* cqsa_dtype_t */
+    size_t mem_budget_bytes;
+} cqsa_plan_desc_t;
+
+/* What a plan decided (for logging, tests and the benchmark). */
+typedef struct {
+    int64_t N;
+    int H, d, levels, causal, dtype;
+    int l[CQSA_MAX_LEVELS];
+    int c[CQSA_MAX_LEVELS];
+    int D[CQSA_MAX_LEVELS][CQSA_MAX_L]; /* difference set of each level */
+    int64_t num_blocks;                 /* prod c_i */
+    int64_t block_tokens;               /* N / num_blocks */
+    int64_t num_tasks;                  /* leaf tasks = prod c_i */
+    int64_t num_entries;                /* (leaf task, query block) pairs with >= 1 allowed key */
+    int64_t max_slots;                  /* most partials any query block receives */
+    int64_t max_task_rows;              /* tokens in the largest leaf task */
+    int head_group;                     /* heads per streamed group in host mode */
+    size_t device_arena_bytes;          /* arena of a device-mode forward */
+    size_t host_arena_bytes;            /* arena of a host-mode forward (<= budget) */
+    size_t h2d_bytes;                   /* planned host->device bytes of one host-mode forward */
+    size_t d2h_bytes;                   /* planned device->host bytes of one host-mode forward */
+    double useful_flops;                /* 4 N^2 H d, halved when causal */
+} cqsa_plan_info_t;
+
+/* One (leaf task, query block) entry of the work list, in global blocks. */
+typedef struct {
+    int64_t task;       /* leaf task index, planner order */
+    int64_t q_block;    /* global query block */
+    int64_t slot;       /* partial index of this entry among the query block's entries */
+    int64_t num_runs;   /* runs of consecutive allowed key blocks */
+} cqsa_entry_t;
+
+/*
+ * cqsa_plan -- plan attention over N tokens, H heads, head dim d, bf16.
+ * Level 0 uses l; each further level uses max(3, l_prev - 1) ([B] "The
+ * Recursive Benefit").  levels = 0 picks the fewest levels (<= 4) whose
+ * host-mode working set fits mem_budget_bytes.  causal != 0 keeps keys at
+ * or before the query position.  On success *out owns a new plan.
+ * Host-only: touches no GPU.  Errors: INVALID_ARG, NO_DIFFERENCE_SET,
+ * BUDGET, UNSUPPORTED.
+ */
+cqsa_status_t cqsa_plan(int64_t N, int H, int d, int l, int levels, int causal,
+                        size_t mem_budget_bytes, cqsa_plan_t **out);
+
+/* cqsa_plan_ex -- as cqsa_plan with per-level l and a dtype (bf16 or fp32). */
+cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out);
+
+/*
+ * cqsa_forward -- run the planned attention ([A]; [B] "Implementation").
+ *   host_or_device = CQSA_DEVICE: q, k, v, out, lse are device pointers on the
+ *     current device.  Every task runs from HBM; partials go to the plan's
+ *     arena and one merge writes out and lse.
+ *   host_or_device = CQSA_HOST: all five are page-locked host pointers
+ *     (cudaHostAlloc / pinned torch tensors).  Tasks are streamed: each
+ *     task's Q/K/V blocks are copied in on a copy stream, double buffered,
+ *     computed, merged into device-resident accumulators of the current head
+ *     group, and finished blocks are copied back.
+ *   stream: a cudaStream_t (0 = legacy default stream) the call is ordered
+ *     after and that is ordered after all of its work.
+ * Asynchronous: returns once all work is enqueued.  The first call on a plan
+ * allocates its arena (one cudaMalloc, sized by the plan).  One forward at a
+ * time per plan.  Errors: INVALID_ARG, NOT_PINNED, CUDA, NO_DEVICE, BUDGET.
+ * Device-side timeouts are reported by cqsa_plan_sync.
+ */
+cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,
+                           const void *v, void *out, float *lse,
+                           int host_or_device, void *stream);
+
+/* cqsa_plan_sync -- wait for the plan's work on `stream` and report any
+ * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync. */
+cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream);
+
+/* cqsa_plan_info -- copy what the plan decided into *info. */
+cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info);
+
+/* cqsa_plan_task_blocks -- global blocks of leaf task t in increasing order
+ * (its token sequence) and its subsequence index per level.  blocks must
+ * hold max_blocks entries, path CQSA_MAX_LEVELS; *num_blocks gets the
+ * count.  INVALID_ARG when t is out of range or max_blocks is too small. */
+cqsa_status_t cqsa_plan_task_blocks(const cqsa_plan_t *plan, int64_t t, int64_t *blocks,
+                                    int64_t max_blocks, int64_t *num_blocks, int *path);
+
+/* cqsa_plan_entry -- entry i (0 <= i < num_entries) of the work list and its
+ * key runs: runs[2r], runs[2r+1] are the first and last global key block of
+ * run r (inclusive).  runs must hold 2 * max_runs values. */
+cqsa_status_t cqsa_plan_entry(const cqsa_plan_t *plan, int64_t i, cqsa_entry_t *entry,
+                              int64_t *runs, int64_t max_runs);
+
+/* cqsa_difference_set -- the lexicographically first perfect difference set
+ * of size l modulo l(l-1)+1 that contains 0 and 1 ([B] "The CQS Divide";
+ * [A] cyclic quorum sets).  D must hold l ints.  NO_DIFFERENCE_SET if none. */
+cqsa_status_t cqsa_difference_set(int l, int *D);
+
+/* cqsa_plan_debug -- failure-detection hooks for tests.  timeout_ns bounds
+ * every device-side wait (0 restores the default of 4 s); stall_mma != 0
+ * makes the bf16 kernel's MMA issuer issue nothing, so that the other
+ * warps' bounded waits run out and the next cqsa_plan_sync reports
+ * CQSA_ERR_TIMEOUT.  Never needed in normal use. */
+cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_mma);
+
+/* cqsa_plan_destroy -- free the plan, its arena, streams and events.  Waits
+ * for the plan's outstanding work first.  Null is ignored. */
+void cqsa_plan_destroy(cqsa_plan_t *plan);
+
+/* cqsa_last_error -- message of the last failing call on this thread. */
+const char *cqsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CQSA_H */

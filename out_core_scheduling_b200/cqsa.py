@@ -1,0 +1,230 @@
+"""ctypes binding of libcqsa.so (C ABI in include/cqsa.h).
+
+Argument marshalling only: every step of the attention path runs in the
+library's CUDA kernels and host scheduler.  The functions keep the C names:
+``cqsa_plan``, ``cqsa_plan_ex``, ``cqsa_forward``, ``cqsa_plan_sync`` ...
+If the library is missing this module raises; there is no other path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcqsa.so")
+
+CQSA_OK = 0
+CQSA_ERR_INVALID_ARG = 1
+CQSA_ERR_NO_DIFFERENCE_SET = 2
+CQSA_ERR_BUDGET = 3
+CQSA_ERR_NOT_PINNED = 4
+CQSA_ERR_CUDA = 5
+CQSA_ERR_TIMEOUT = 6
+CQSA_ERR_UNSUPPORTED = 7
+CQSA_ERR_NO_DEVICE = 8
+
+CQSA_BF16 = 0
+CQSA_FP32 = 1
+CQSA_DEVICE = 0
+CQSA_HOST = 1
+MAX_LEVELS = 4
+MAX_L = 16
+
+# Every symbol include/cqsa.h declares.
+EXPORTS = (
+    "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_plan_sync", "cqsa_plan_info",
+    "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
+    "cqsa_plan_destroy", "cqsa_last_error",
+)
+
+
+class CqsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"cqsa status {status}: {message}")
+        self.status = status
+
+
+class PlanDesc(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
+                ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("mem_budget_bytes", ctypes.c_size_t)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("levels", ctypes.c_int), ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("l", ctypes.c_int * MAX_LEVELS), ("c", ctypes.c_int * MAX_LEVELS),
+                ("D", (ctypes.c_int * MAX_L) * MAX_LEVELS),
+                ("num_blocks", ctypes.c_int64), ("block_tokens", ctypes.c_int64),
+                ("num_tasks", ctypes.c_int64), ("num_entries", ctypes.c_int64),
+                ("max_slots", ctypes.c_int64), ("max_task_rows", ctypes.c_int64),
+                ("head_group", ctypes.c_int), ("device_arena_bytes", ctypes.c_size_t),
+                ("host_arena_bytes", ctypes.c_size_t), ("h2d_bytes", ctypes.c_size_t),
+                ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double)]
+
+    def as_dict(self) -> dict:
+        out = {}
+        for name, _ in self._fields_:
+            val = getattr(self, name)
+            if name in ("l", "c"):
+                val = list(val)[: self.levels]
+            elif name == "D":
+                val = [list(val[i])[: self.l[i]] for i in range(self.levels)]
+            out[name] = val
+        return out
+
+
+class Entry(ctypes.Structure):
+    _fields_ = [("task", ctypes.c_int64), ("q_block", ctypes.c_int64),
+                ("slot", ctypes.c_int64), ("num_runs", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libcqsa.so; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m out_core_scheduling_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    st = ctypes.c_int
+    sig = {
+        "cqsa_plan": (st, [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                           ctypes.c_int, ctypes.c_size_t, ctypes.POINTER(P)]),
+        "cqsa_plan_ex": (st, [ctypes.POINTER(PlanDesc), ctypes.POINTER(P)]),
+        "cqsa_forward": (st, [P, P, P, P, P, P, ctypes.c_int, P]),
+        "cqsa_plan_sync": (st, [P, P]),
+        "cqsa_plan_info": (st, [P, ctypes.POINTER(PlanInfo)]),
+        "cqsa_plan_task_blocks": (st, [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]),
+        "cqsa_plan_entry": (st, [P, ctypes.c_int64, ctypes.POINTER(Entry), ctypes.POINTER(ctypes.c_int64),
+                                 ctypes.c_int64]),
+        "cqsa_difference_set": (st, [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
+        "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
+        "cqsa_plan_destroy": (None, [P]),
+        "cqsa_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != CQSA_OK:
+        msg = load_library().cqsa_last_error()
+        raise CqsaError(status, msg.decode() if msg else "")
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Plan:
+    """Owns a cqsa_plan_t handle."""
+
+    def __init__(self, handle: int):
+        self.handle = ctypes.c_void_p(handle)
+
+    def info(self) -> dict:
+        inf = PlanInfo()
+        _check(load_library().cqsa_plan_info(self.handle, ctypes.byref(inf)))
+        return inf.as_dict()
+
+    def task_blocks(self, t: int):
+        lib = load_library()
+        n = ctypes.c_int64()
+        path = (ctypes.c_int * MAX_LEVELS)()
+        _check(lib.cqsa_plan_task_blocks(self.handle, t, None, 0, ctypes.byref(n), path))
+        buf = (ctypes.c_int64 * max(1, n.value))()
+        _check(lib.cqsa_plan_task_blocks(self.handle, t, buf, n.value, ctypes.byref(n), path))
+        return list(buf)[: n.value], [p for p in path if p >= 0]
+
+    def entry(self, i: int):
+        lib = load_library()
+        e = Entry()
+        _check(lib.cqsa_plan_entry(self.handle, i, ctypes.byref(e), None, 0))
+        runs = (ctypes.c_int64 * (2 * max(1, e.num_runs)))()
+        _check(lib.cqsa_plan_entry(self.handle, i, ctypes.byref(e), runs, e.num_runs))
+        pairs = [(runs[2 * r], runs[2 * r + 1]) for r in range(e.num_runs)]
+        return {"task": e.task, "q_block": e.q_block, "slot": e.slot, "runs": pairs}
+
+    def sync(self, stream=None):
+        _check(load_library().cqsa_plan_sync(self.handle, ctypes.c_void_p(_stream_ptr(stream))))
+
+    def debug(self, timeout_ns: int = 0, stall_mma: bool = False):
+        _check(load_library().cqsa_plan_debug(self.handle, timeout_ns, int(bool(stall_mma))))
+
+    def destroy(self):
+        if self.handle and self.handle.value:
+            load_library().cqsa_plan_destroy(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = False,
+              mem_budget_bytes: int = 0) -> Plan:
+    h = ctypes.c_void_p()
+    _check(load_library().cqsa_plan(N, H, d, l, levels, int(bool(causal)), mem_budget_bytes, ctypes.byref(h)))
+    return Plan(h.value)
+
+
+def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
+                 mem_budget_bytes: int = 0) -> Plan:
+    desc = PlanDesc()
+    desc.N, desc.H, desc.d = N, H, d
+    desc.levels = len(ls)
+    for i, x in enumerate(ls):
+        desc.l[i] = x
+    desc.causal = int(bool(causal))
+    desc.dtype = dtype
+    desc.mem_budget_bytes = mem_budget_bytes
+    h = ctypes.c_void_p()
+    _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
+    return Plan(h.value)
+
+
+def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVICE, stream=None):
+    """q, k, v, out: [N, H, d] contiguous torch tensors in the plan's dtype;
+    lse: fp32 [H, N].  Device tensors for CQSA_DEVICE, pinned CPU tensors
+    for CQSA_HOST.  Asynchronous on ``stream`` (default: torch's current)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
+        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous torch tensor")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be float32")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share a dtype")
+    if not (q.shape == k.shape == v.shape == out.shape) or q.dim() != 3:
+        raise ValueError("q, k, v, out must all be [N, H, d]")
+    N, H, _ = q.shape
+    if tuple(lse.shape) != (H, N):
+        raise ValueError("lse must be [H, N]")
+    _check(load_library().cqsa_forward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       out.data_ptr(), lse.data_ptr(), host_or_device,
+                                       ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_difference_set(l: int):
+    D = (ctypes.c_int * l)()
+    _check(load_library().cqsa_difference_set(l, D))
+    return list(D)

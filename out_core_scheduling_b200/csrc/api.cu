@@ -1,0 +1,697 @@
+// api.cu -- the C ABI (cqsa.h): plans, the device-resident path and the
+// streamed out-of-core scheduler.
+//
+// Streamed path ("Stream-CQSA: Breaking the Billion-Token Barrier on a
+// Single GPU", section "Implementation": decompose, stream Q_i/K_i/V_i to the
+// GPU, compute local statistics, aggregate; section "Performance": the cost
+// is host-device transfer).  For each head group and each leaf task, in
+// planner order:
+//   copy stream     H2D of the task's needed Q/K/V blocks into stage i%2
+//   compute stream  tile attention on stage i%2 -> task partials, then the
+//                   log-sum-exp merge into the device-resident accumulator
+//                   of the head group; blocks seen for the last time are
+//                   finished into out stage i%2
+//   copy-out stream D2H of the finished rows and their lse
+// Events order the three streams; stage reuse waits on the work two tasks
+// back, so copies of task i+1 and i-1 overlap the compute of task i.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "cqsa.h"
+#include "kernels.h"
+#include "planner.h"
+#include "worklist.h"
+
+using namespace cqsa;
+
+namespace {
+
+thread_local std::string g_err;
+
+cqsa_status_t fail(cqsa_status_t code, const char *fmt, ...) {
+    char buf[1024];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+#define CK(call)                                                                                  \
+    do {                                                                                          \
+        cudaError_t e_ = (call);                                                                  \
+        if (e_ != cudaSuccess)                                                                    \
+            return fail(CQSA_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),    \
+                        __FILE__, __LINE__);                                                      \
+    } while (0)
+
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [rows, heads, d] bf16 tensor, box {64 columns, 1 head, 128 rows}, 128-byte
+// swizzle: the shared-memory image the tensor-core descriptors expect.
+cqsa_status_t make_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int d) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(CQSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    if ((reinterpret_cast<uintptr_t>(base) & 15) != 0)
+        return fail(CQSA_ERR_INVALID_ARG, "tensor base %p is not 16-byte aligned", base);
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CQSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return CQSA_OK;
+}
+
+struct DevWl {
+    WlEntry *entries = nullptr;
+    WlRun *runs = nullptr;
+    WlUnit *units = nullptr;
+    int num_units = 0;
+};
+
+// Places a work list inside an arena region laid out as the planner sized it.
+DevWl place_wl(char *base, const WorkList &wl) {
+    ArenaLayout sub;
+    const size_t oe = sub.take(wl.entries.size() * sizeof(WlEntry));
+    const size_t orr = sub.take(wl.runs.size() * sizeof(WlRun));
+    const size_t ou = sub.take(wl.units.size() * sizeof(WlUnit));
+    DevWl d;
+    d.entries = reinterpret_cast<WlEntry *>(base + oe);
+    d.runs = reinterpret_cast<WlRun *>(base + orr);
+    d.units = reinterpret_cast<WlUnit *>(base + ou);
+    d.num_units = (int)wl.units.size();
+    return d;
+}
+
+size_t wl_region(const WorkList &wl) {
+    ArenaLayout sub;
+    sub.take(wl.entries.size() * sizeof(WlEntry));
+    sub.take(wl.runs.size() * sizeof(WlRun));
+    sub.take(wl.units.size() * sizeof(WlUnit));
+    return sub.total;
+}
+
+std::vector<char> pack_wl(const WorkList &wl) {
+    ArenaLayout sub;
+    const size_t oe = sub.take(wl.entries.size() * sizeof(WlEntry));
+    const size_t orr = sub.take(wl.runs.size() * sizeof(WlRun));
+    const size_t ou = sub.take(wl.units.size() * sizeof(WlUnit));
+    std::vector<char> buf(sub.total, 0);
+    if (!wl.entries.empty()) memcpy(buf.data() + oe, wl.entries.data(), wl.entries.size() * sizeof(WlEntry));
+    if (!wl.runs.empty()) memcpy(buf.data() + orr, wl.runs.data(), wl.runs.size() * sizeof(WlRun));
+    if (!wl.units.empty()) memcpy(buf.data() + ou, wl.units.data(), wl.units.size() * sizeof(WlUnit));
+    return buf;
+}
+
+struct LeafState {
+    DevWl wl;
+    MergeSeg *segs = nullptr;
+    std::vector<MergeSeg> host_segs;
+    std::vector<char> need_q, need_kv;
+};
+
+}  // namespace
+
+struct cqsa_plan {
+    Planner pl;
+    int dtype = CQSA_BF16;
+    int elem = 2;
+    int device = -1;
+    uint64_t timeout_ns = kDefaultTimeoutNs;
+    int stall_test = 0;
+
+    // Device-resident path.
+    char *dev_arena = nullptr;
+    size_t dev_bytes = 0;
+    int *dev_err = nullptr;
+    float *dev_part_o = nullptr, *dev_part_lse = nullptr;
+    int32_t *dev_nslots = nullptr;
+    DevWl dev_wl;
+
+    // Streamed path.
+    char *host_arena = nullptr;
+    size_t host_bytes = 0;
+    int g = 0;
+    int *h_err = nullptr;
+    float *acc_o = nullptr, *acc_lse = nullptr;
+    char *in_q[2] = {}, *in_k[2] = {}, *in_v[2] = {}, *out_st[2] = {};
+    float *lse_st[2] = {};
+    float *h_part_o = nullptr, *h_part_lse = nullptr;
+    std::vector<LeafState> leaves;
+    CUtensorMap mq[2], mk[2], mv[2];
+    cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+    cudaEvent_t ev_in_ready[2] = {}, ev_in_free[2] = {}, ev_merged[2] = {}, ev_out_free[2] = {};
+    cudaEvent_t ev_start = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
+};
+
+namespace {
+
+cqsa_status_t check_device(cqsa_plan_t *P) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(CQSA_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+    }
+    int major = 0, minor = 0;
+    CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    CK(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (major != 10 || minor != 0)
+        return fail(CQSA_ERR_NO_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
+                    minor);
+    if (P->device >= 0 && P->device != dev)
+        return fail(CQSA_ERR_INVALID_ARG, "plan is bound to device %d but device %d is current", P->device, dev);
+    P->device = dev;
+    return CQSA_OK;
+}
+
+cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
+    if (P->dev_arena) return CQSA_OK;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    if (pl.max_slots > 32) return fail(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
+    WorkList wl = pl.device_worklist(unit_rows_for(P->elem), key_tile_for(P->elem), H);
+    ArenaLayout a;
+    const size_t o_err = a.take(256);
+    const size_t o_po = a.take((size_t)pl.max_slots * N * H * d * sizeof(float));
+    const size_t o_pl = a.take((size_t)pl.max_slots * H * N * sizeof(float));
+    const size_t o_ns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+    const size_t o_wl = a.take(wl_region(wl));
+    if (a.total != pl.sizing.device_arena)
+        return fail(CQSA_ERR_CUDA, "internal: device arena layout mismatch (%zu vs %zu)", a.total,
+                    pl.sizing.device_arena);
+    if (pl.spec.budget && a.total > pl.spec.budget)
+        return fail(CQSA_ERR_BUDGET, "device-resident path needs %zu bytes, budget is %zu", a.total, pl.spec.budget);
+    char *arena = nullptr;
+    CK(cudaMalloc(&arena, a.total));
+    P->dev_arena = arena;
+    P->dev_bytes = a.total;
+    CK(cudaMemset(arena, 0, a.total));
+    P->dev_err = reinterpret_cast<int *>(arena + o_err);
+    P->dev_part_o = reinterpret_cast<float *>(arena + o_po);
+    P->dev_part_lse = reinterpret_cast<float *>(arena + o_pl);
+    P->dev_nslots = reinterpret_cast<int32_t *>(arena + o_ns);
+    CK(cudaMemcpy(P->dev_nslots, pl.slots_per_block.data(), pl.slots_per_block.size() * sizeof(int32_t),
+                  cudaMemcpyHostToDevice));
+    std::vector<char> buf = pack_wl(wl);
+    if (!buf.empty()) CK(cudaMemcpy(arena + o_wl, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+    P->dev_wl = place_wl(arena + o_wl, wl);
+    return CQSA_OK;
+}
+
+cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
+    if (P->host_arena) return CQSA_OK;
+    const Planner &pl = P->pl;
+    const int g = pl.sizing.head_group;
+    if (g <= 0)
+        return fail(CQSA_ERR_BUDGET, "no head group of the streamed path fits the budget of %zu bytes",
+                    pl.spec.budget);
+    const int64_t N = pl.spec.N, R = pl.max_task_rows;
+    const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
+    ArenaLayout a;
+    const size_t o_err = a.take(256);
+    const size_t o_acc = a.take((size_t)N * g * dd * sizeof(float));
+    const size_t o_accl = a.take((size_t)g * N * sizeof(float));
+    size_t o_q[2], o_k[2], o_v[2], o_out[2], o_lse[2];
+    for (int s = 0; s < 2; ++s) {
+        o_q[s] = a.take((size_t)R * g * dd * e);
+        o_k[s] = a.take((size_t)R * g * dd * e);
+        o_v[s] = a.take((size_t)R * g * dd * e);
+        o_out[s] = a.take((size_t)R * g * dd * e);
+        o_lse[s] = a.take((size_t)g * R * sizeof(float));
+    }
+    const size_t o_po = a.take((size_t)R * g * dd * sizeof(float));
+    const size_t o_pl = a.take((size_t)g * R * sizeof(float));
+    std::vector<WorkList> wls(pl.leaves.size());
+    std::vector<size_t> o_wl(pl.leaves.size()), o_seg(pl.leaves.size());
+    P->leaves.assign(pl.leaves.size(), LeafState());
+    for (size_t t = 0; t < pl.leaves.size(); ++t) {
+        wls[t] = pl.leaf_worklist((int64_t)t, unit_rows_for(P->elem), key_tile_for(P->elem), g);
+        o_wl[t] = a.take(wl_region(wls[t]));
+        P->leaves[t].host_segs = pl.leaf_merge_segments((int64_t)t);
+        o_seg[t] = a.take(P->leaves[t].host_segs.size() * sizeof(MergeSeg));
+        pl.leaf_needs((int64_t)t, &P->leaves[t].need_q, &P->leaves[t].need_kv);
+    }
+    if (a.total != pl.sizing.host_arena)
+        return fail(CQSA_ERR_CUDA, "internal: host-mode arena layout mismatch (%zu vs %zu)", a.total,
+                    pl.sizing.host_arena);
+    char *arena = nullptr;
+    CK(cudaMalloc(&arena, a.total));
+    P->host_arena = arena;
+    P->host_bytes = a.total;
+    P->g = g;
+    // Zeroed once, so rows a partial key tile reads past its run are finite.
+    CK(cudaMemset(arena, 0, a.total));
+    P->h_err = reinterpret_cast<int *>(arena + o_err);
+    P->acc_o = reinterpret_cast<float *>(arena + o_acc);
+    P->acc_lse = reinterpret_cast<float *>(arena + o_accl);
+    for (int s = 0; s < 2; ++s) {
+        P->in_q[s] = arena + o_q[s];
+        P->in_k[s] = arena + o_k[s];
+        P->in_v[s] = arena + o_v[s];
+        P->out_st[s] = arena + o_out[s];
+        P->lse_st[s] = reinterpret_cast<float *>(arena + o_lse[s]);
+    }
+    P->h_part_o = reinterpret_cast<float *>(arena + o_po);
+    P->h_part_lse = reinterpret_cast<float *>(arena + o_pl);
+    for (size_t t = 0; t < pl.leaves.size(); ++t) {
+        std::vector<char> buf = pack_wl(wls[t]);
+        if (!buf.empty()) CK(cudaMemcpy(arena + o_wl[t], buf.data(), buf.size(), cudaMemcpyHostToDevice));
+        P->leaves[t].wl = place_wl(arena + o_wl[t], wls[t]);
+        P->leaves[t].segs = reinterpret_cast<MergeSeg *>(arena + o_seg[t]);
+        const auto &hs = P->leaves[t].host_segs;
+        if (!hs.empty())
+            CK(cudaMemcpy(P->leaves[t].segs, hs.data(), hs.size() * sizeof(MergeSeg), cudaMemcpyHostToDevice));
+    }
+    if (P->dtype == CQSA_BF16) {
+        for (int s = 0; s < 2; ++s) {
+            cqsa_status_t st;
+            if ((st = make_map(&P->mq[s], P->in_q[s], R, g, pl.spec.d)) != CQSA_OK) return st;
+            if ((st = make_map(&P->mk[s], P->in_k[s], R, g, pl.spec.d)) != CQSA_OK) return st;
+            if ((st = make_map(&P->mv[s], P->in_v[s], R, g, pl.spec.d)) != CQSA_OK) return st;
+        }
+    }
+    CK(cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&P->s_out, cudaStreamNonBlocking));
+    for (int s = 0; s < 2; ++s) {
+        CK(cudaEventCreateWithFlags(&P->ev_in_ready[s], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&P->ev_in_free[s], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&P->ev_merged[s], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&P->ev_out_free[s], cudaEventDisableTiming));
+    }
+    CK(cudaEventCreateWithFlags(&P->ev_start, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_done_comp, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_done_out, cudaEventDisableTiming));
+    return CQSA_OK;
+}
+
+AttnParams base_params(const cqsa_plan_t *P, int *err) {
+    AttnParams ap{};
+    ap.causal = P->pl.spec.causal;
+    ap.scale = 1.0f / std::sqrt((float)P->pl.spec.d);
+    ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)P->pl.spec.d));
+    ap.timeout_ns = P->timeout_ns;
+    ap.err = err;
+    ap.stall_test = P->stall_test;
+    return ap;
+}
+
+cqsa_status_t check_ptr(const void *p, bool want_host, const char *name) {
+    if (!p) return fail(CQSA_ERR_INVALID_ARG, "%s is null", name);
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(want_host ? CQSA_ERR_NOT_PINNED : CQSA_ERR_INVALID_ARG, "%s: cudaPointerGetAttributes: %s",
+                    name, cudaGetErrorString(e));
+    }
+    if (want_host) {
+        if (at.type != cudaMemoryTypeHost)
+            return fail(CQSA_ERR_NOT_PINNED, "%s is not page-locked host memory", name);
+    } else {
+        if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+            return fail(CQSA_ERR_INVALID_ARG, "%s is not device memory", name);
+    }
+    return CQSA_OK;
+}
+
+cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const void *v, void *out, float *lse,
+                             cudaStream_t stream) {
+    cqsa_status_t st = setup_device_mode(P);
+    if (st != CQSA_OK) return st;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    AttnParams ap = base_params(P, P->dev_err);
+    ap.entries = P->dev_wl.entries;
+    ap.runs = P->dev_wl.runs;
+    ap.units = P->dev_wl.units;
+    ap.part_o = P->dev_part_o;
+    ap.part_lse = P->dev_part_lse;
+    ap.part_rows = N;
+    ap.H = H;
+    if (P->dtype == CQSA_BF16) {
+        CUtensorMap mq, mk, mv;
+        if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mk, k, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mv, v, N, H, d)) != CQSA_OK) return st;
+        CK(launch_attn_tc(d, mq, mk, mv, ap, P->dev_wl.num_units, stream));
+    } else {
+        CK(launch_attn_simt(d, P->elem, q, k, v, ap, P->dev_wl.num_units, stream));
+    }
+    CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H, out, lse,
+                          stream));
+    return CQSA_OK;
+}
+
+// Copies `rows` token rows of heads [h0, h0+g) between a full [*, H, d]
+// tensor and a compact [*, g, d] one.
+cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width, size_t rows,
+                      cudaMemcpyKind kind, cudaStream_t s) {
+    if (dpitch == width && spitch == width) return cudaMemcpyAsync(dst, src, width * rows, kind, s);
+    return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, kind, s);
+}
+
+cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const void *v, void *out, float *lse,
+                           cudaStream_t stream) {
+    cqsa_status_t st = setup_host_mode(P);
+    if (st != CQSA_OK) return st;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N, R = pl.max_task_rows, B = pl.block;
+    const int H = pl.spec.H, d = pl.spec.d, g = P->g;
+    const size_t e = (size_t)P->elem;
+    const size_t full_row = (size_t)H * d * e, grp_row = (size_t)g * d * e;
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
+               *hv = static_cast<const char *>(v);
+    char *ho = static_cast<char *>(out);
+    CK(cudaEventRecord(P->ev_start, stream));
+    CK(cudaStreamWaitEvent(P->s_in, P->ev_start, 0));
+    CK(cudaStreamWaitEvent(P->s_comp, P->ev_start, 0));
+    CK(cudaStreamWaitEvent(P->s_out, P->ev_start, 0));
+    int64_t it = 0;
+    for (int h0 = 0; h0 < H; h0 += g) {
+        for (size_t t = 0; t < P->leaves.size(); ++t, ++it) {
+            const LeafState &L = P->leaves[t];
+            const Leaf &leaf = pl.leaves[t];
+            const int s = (int)(it & 1);
+            // -- H2D of the task's blocks (runs of consecutive needed members).
+            if (it >= 2) CK(cudaStreamWaitEvent(P->s_in, P->ev_in_free[s], 0));
+            const char *srcs[3] = {hq, hk, hv};
+            char *dsts[3] = {P->in_q[s], P->in_k[s], P->in_v[s]};
+            for (int x = 0; x < 3; ++x) {
+                const std::vector<char> &need = (x == 0) ? L.need_q : L.need_kv;
+                size_t m = 0;
+                while (m < need.size()) {
+                    if (!need[m]) { ++m; continue; }
+                    size_t m1 = m;
+                    while (m1 + 1 < need.size() && need[m1 + 1] && leaf.blocks[m1 + 1] == leaf.blocks[m1] + 1) ++m1;
+                    const size_t rows = (m1 - m + 1) * (size_t)B;
+                    char *dst = dsts[x] + (size_t)m * B * grp_row;
+                    const char *src = srcs[x] + ((size_t)leaf.blocks[m] * B * H + h0) * d * e;
+                    CK(copy_rows(dst, grp_row, src, full_row, grp_row, rows, cudaMemcpyHostToDevice, P->s_in));
+                    m = m1 + 1;
+                }
+            }
+            CK(cudaEventRecord(P->ev_in_ready[s], P->s_in));
+            // -- tile attention on the staged task.
+            CK(cudaStreamWaitEvent(P->s_comp, P->ev_in_ready[s], 0));
+            AttnParams ap = base_params(P, P->h_err);
+            ap.entries = L.wl.entries;
+            ap.runs = L.wl.runs;
+            ap.units = L.wl.units;
+            ap.part_o = P->h_part_o;
+            ap.part_lse = P->h_part_lse;
+            ap.part_rows = R;
+            ap.H = g;
+            if (P->dtype == CQSA_BF16)
+                CK(launch_attn_tc(d, P->mq[s], P->mk[s], P->mv[s], ap, L.wl.num_units, P->s_comp));
+            else
+                CK(launch_attn_simt(d, P->elem, P->in_q[s], P->in_k[s], P->in_v[s], ap, L.wl.num_units,
+                                    P->s_comp));
+            CK(cudaEventRecord(P->ev_in_free[s], P->s_comp));
+            // -- merge into the accumulator; finished rows go to out stage s.
+            if (it >= 2) CK(cudaStreamWaitEvent(P->s_comp, P->ev_out_free[s], 0));
+            CK(launch_merge_stream(d, P->elem, L.segs, (int)L.host_segs.size(), (int)B, P->h_part_o,
+                                   P->h_part_lse, R, P->acc_o, P->acc_lse, N, g, P->out_st[s], P->lse_st[s],
+                                   P->s_comp));
+            CK(cudaEventRecord(P->ev_merged[s], P->s_comp));
+            // -- D2H of finished rows.
+            CK(cudaStreamWaitEvent(P->s_out, P->ev_merged[s], 0));
+            for (const MergeSeg &sg : L.host_segs) {
+                if (!(sg.flags & SEG_LAST)) continue;
+                CK(copy_rows(ho + ((size_t)sg.global_lo * H + h0) * d * e, full_row,
+                             P->out_st[s] + (size_t)sg.local_lo * grp_row, grp_row, grp_row, (size_t)sg.rows,
+                             cudaMemcpyDeviceToHost, P->s_out));
+                CK(cudaMemcpy2DAsync(lse + (size_t)h0 * N + sg.global_lo, (size_t)N * sizeof(float),
+                                     P->lse_st[s] + sg.local_lo, (size_t)R * sizeof(float),
+                                     (size_t)sg.rows * sizeof(float), (size_t)g, cudaMemcpyDeviceToHost, P->s_out));
+            }
+            CK(cudaEventRecord(P->ev_out_free[s], P->s_out));
+        }
+    }
+    CK(cudaEventRecord(P->ev_done_comp, P->s_comp));
+    CK(cudaEventRecord(P->ev_done_out, P->s_out));
+    CK(cudaStreamWaitEvent(stream, P->ev_done_comp, 0));
+    CK(cudaStreamWaitEvent(stream, P->ev_done_out, 0));
+    return CQSA_OK;
+}
+
+cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
+    cqsa_plan_t *P = new cqsa_plan_t();
+    P->dtype = dtype;
+    P->elem = spec.elem_bytes;
+    int code = 0;
+    std::string msg = P->pl.build(spec, &code);
+    if (!msg.empty()) {
+        delete P;
+        return fail((cqsa_status_t)code, "%s", msg.c_str());
+    }
+    *out = P;
+    return CQSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
+    if (!desc || !out) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    *out = nullptr;
+    if (desc->dtype != CQSA_BF16 && desc->dtype != CQSA_FP32)
+        return fail(CQSA_ERR_INVALID_ARG, "dtype must be CQSA_BF16 or CQSA_FP32");
+    if (desc->d != 64 && desc->d != 128) return fail(CQSA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", desc->d);
+    if (desc->levels < 1 || desc->levels > CQSA_MAX_LEVELS)
+        return fail(CQSA_ERR_INVALID_ARG, "levels must be in 1..%d", CQSA_MAX_LEVELS);
+    PlanSpec s;
+    s.N = desc->N;
+    s.H = desc->H;
+    s.d = desc->d;
+    s.levels = desc->levels;
+    for (int i = 0; i < desc->levels; ++i) s.l[i] = desc->l[i];
+    s.causal = desc->causal ? 1 : 0;
+    s.elem_bytes = desc->dtype == CQSA_BF16 ? 2 : 4;
+    s.budget = desc->mem_budget_bytes;
+    cqsa_plan_t *P = nullptr;
+    cqsa_status_t st = build_plan(s, desc->dtype, &P);
+    if (st != CQSA_OK) return st;
+    if (s.budget && P->pl.sizing.head_group == 0 && P->pl.sizing.device_arena > s.budget) {
+        delete P;
+        return fail(CQSA_ERR_BUDGET, "neither path fits the budget of %zu bytes", s.budget);
+    }
+    *out = P;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan(int64_t N, int H, int d, int l, int levels, int causal, size_t mem_budget_bytes,
+                        cqsa_plan_t **out) {
+    if (!out) return fail(CQSA_ERR_INVALID_ARG, "null out");
+    *out = nullptr;
+    if (levels < 0 || levels > CQSA_MAX_LEVELS) return fail(CQSA_ERR_INVALID_ARG, "levels must be in 0..4");
+    cqsa_plan_desc_t desc{};
+    desc.N = N;
+    desc.H = H;
+    desc.d = d;
+    desc.causal = causal;
+    desc.dtype = CQSA_BF16;
+    desc.mem_budget_bytes = mem_budget_bytes;
+    const int lo = levels == 0 ? 1 : levels, hi = levels == 0 ? CQSA_MAX_LEVELS : levels;
+    cqsa_status_t last = CQSA_ERR_INVALID_ARG;
+    std::string last_msg;
+    for (int L = lo; L <= hi; ++L) {
+        desc.levels = L;
+        desc.l[0] = l;
+        for (int i = 1; i < L; ++i) desc.l[i] = std::max(3, desc.l[i - 1] - 1);
+        cqsa_plan_t *P = nullptr;
+        last = cqsa_plan_ex(&desc, &P);
+        if (last == CQSA_OK) {
+            if (levels == 0 && mem_budget_bytes && P->pl.sizing.head_group == 0) {
+                cqsa_plan_destroy(P);
+                last = fail(CQSA_ERR_BUDGET, "streamed path does not fit %zu bytes at %d levels", mem_budget_bytes, L);
+                last_msg = g_err;
+                continue;
+            }
+            *out = P;
+            return CQSA_OK;
+        }
+        last_msg = g_err;
+    }
+    g_err = last_msg;
+    return last;
+}
+
+cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, void *out, float *lse,
+                           int host_or_device, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    if (host_or_device != CQSA_DEVICE && host_or_device != CQSA_HOST)
+        return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be CQSA_DEVICE or CQSA_HOST");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const bool host = host_or_device == CQSA_HOST;
+    const void *ptrs[5] = {q, k, v, out, lse};
+    const char *names[5] = {"q", "k", "v", "out", "lse"};
+    for (int i = 0; i < 5; ++i)
+        if ((st = check_ptr(ptrs[i], host, names[i])) != CQSA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return host ? forward_host(plan, q, k, v, out, lse, s) : forward_device(plan, q, k, v, out, lse, s);
+}
+
+cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    if (plan->device < 0) return CQSA_OK;
+    CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int *words[2] = {plan->dev_err, plan->h_err};
+    int bad = 0;
+    for (int *w : words) {
+        if (!w) continue;
+        int v = 0;
+        CK(cudaMemcpy(&v, w, sizeof v, cudaMemcpyDeviceToHost));
+        if (v) {
+            bad = v;
+            CK(cudaMemset(w, 0, sizeof v));
+        }
+    }
+    if (bad) return fail(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d); output is incomplete", bad);
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_mma) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    plan->timeout_ns = timeout_ns ? timeout_ns : kDefaultTimeoutNs;
+    plan->stall_test = stall_mma ? 1 : 0;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
+    if (!plan || !info) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    memset(info, 0, sizeof *info);
+    info->N = pl.spec.N;
+    info->H = pl.spec.H;
+    info->d = pl.spec.d;
+    info->levels = pl.spec.levels;
+    info->causal = pl.spec.causal;
+    info->dtype = plan->dtype;
+    for (int i = 0; i < pl.spec.levels; ++i) {
+        info->l[i] = pl.levels[i].l;
+        info->c[i] = pl.levels[i].c;
+        for (int j = 0; j < pl.levels[i].l && j < CQSA_MAX_L; ++j) info->D[i][j] = pl.levels[i].D[j];
+    }
+    info->num_blocks = pl.num_blocks;
+    info->block_tokens = pl.block;
+    info->num_tasks = (int64_t)pl.leaves.size();
+    info->num_entries = (int64_t)pl.entries.size();
+    info->max_slots = pl.max_slots;
+    info->max_task_rows = pl.max_task_rows;
+    info->head_group = pl.sizing.head_group;
+    info->device_arena_bytes = pl.sizing.device_arena;
+    info->host_arena_bytes = pl.sizing.host_arena;
+    info->h2d_bytes = pl.sizing.h2d;
+    info->d2h_bytes = pl.sizing.d2h;
+    const double n = (double)pl.spec.N;
+    info->useful_flops = 4.0 * n * n * pl.spec.H * pl.spec.d * (pl.spec.causal ? 0.5 : 1.0);
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_task_blocks(const cqsa_plan_t *plan, int64_t t, int64_t *blocks, int64_t max_blocks,
+                                    int64_t *num_blocks, int *path) {
+    if (!plan || !num_blocks) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    if (t < 0 || t >= (int64_t)pl.leaves.size()) return fail(CQSA_ERR_INVALID_ARG, "task %lld out of range", (long long)t);
+    const Leaf &lf = pl.leaves[t];
+    *num_blocks = (int64_t)lf.blocks.size();
+    if (blocks) {
+        if (max_blocks < (int64_t)lf.blocks.size()) return fail(CQSA_ERR_INVALID_ARG, "blocks buffer too small");
+        for (size_t i = 0; i < lf.blocks.size(); ++i) blocks[i] = lf.blocks[i];
+    }
+    if (path)
+        for (int i = 0; i < CQSA_MAX_LEVELS; ++i) path[i] = i < (int)lf.path.size() ? lf.path[i] : -1;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_entry(const cqsa_plan_t *plan, int64_t i, cqsa_entry_t *entry, int64_t *runs,
+                              int64_t max_runs) {
+    if (!plan || !entry) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    if (i < 0 || i >= (int64_t)pl.entries.size()) return fail(CQSA_ERR_INVALID_ARG, "entry %lld out of range", (long long)i);
+    const Entry &e = pl.entries[i];
+    entry->task = e.task;
+    entry->q_block = e.qb;
+    entry->slot = e.slot;
+    entry->num_runs = (int64_t)e.runs.size();
+    if (runs) {
+        if (max_runs < (int64_t)e.runs.size()) return fail(CQSA_ERR_INVALID_ARG, "runs buffer too small");
+        for (size_t r = 0; r < e.runs.size(); ++r) {
+            runs[2 * r] = e.runs[r].b0;
+            runs[2 * r + 1] = e.runs[r].b1;
+        }
+    }
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_difference_set(int l, int *D) {
+    if (!D) return fail(CQSA_ERR_INVALID_ARG, "null D");
+    std::vector<int> v;
+    if (!find_difference_set(l, &v))
+        return fail(CQSA_ERR_NO_DIFFERENCE_SET, "no perfect difference set of size %d mod %d", l, l * (l - 1) + 1);
+    for (size_t i = 0; i < v.size(); ++i) D[i] = v[i];
+    return CQSA_OK;
+}
+
+void cqsa_plan_destroy(cqsa_plan_t *plan) {
+    if (!plan) return;
+    if (plan->device >= 0) {
+        cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
+        for (cudaStream_t s : ss)
+            if (s) cudaStreamSynchronize(s);
+        if (plan->dev_arena) cudaDeviceSynchronize();
+        for (int s = 0; s < 2; ++s) {
+            if (plan->ev_in_ready[s]) cudaEventDestroy(plan->ev_in_ready[s]);
+            if (plan->ev_in_free[s]) cudaEventDestroy(plan->ev_in_free[s]);
+            if (plan->ev_merged[s]) cudaEventDestroy(plan->ev_merged[s]);
+            if (plan->ev_out_free[s]) cudaEventDestroy(plan->ev_out_free[s]);
+        }
+        if (plan->ev_start) cudaEventDestroy(plan->ev_start);
+        if (plan->ev_done_comp) cudaEventDestroy(plan->ev_done_comp);
+        if (plan->ev_done_out) cudaEventDestroy(plan->ev_done_out);
+        for (cudaStream_t s : ss)
+            if (s) cudaStreamDestroy(s);
+        if (plan->dev_arena) cudaFree(plan->dev_arena);
+        if (plan->host_arena) cudaFree(plan->host_arena);
+        cudaGetLastError();
+    }
+    delete plan;
+}
+
+const char *cqsa_last_error(void) { return g_err.c_str(); }
+
+}  // extern "C"

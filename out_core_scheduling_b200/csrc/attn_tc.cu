@@ -1,0 +1,402 @@
+// attn_tc.cu -- masked tile attention on the sm_100a tensor cores (bf16 in,
+// fp32 accumulate): the per-task compute of the CQS Divide.
+//
+// Each CTA takes one work unit: one (task, query block) entry of the CQS
+// work list, 2 x 128 query rows of it, one head.  It visits only the key
+// tiles the CQS mask allows (the entry's key runs), so masked chunk pairs
+// cost nothing, and emits the task's local softmax statistics for its rows:
+// the normalised partial output O_j and lse_j = m_j + ln(l_j)
+// ("Stream-CQSA: Breaking the Billion-Token Barrier on a Single GPU",
+// section "Implementation", step 3: local numerators and denominators).
+//
+// Warp roles (320 threads, one CTA per SM):
+//   warps 0-3  softmax for query tile 0 (TMEM lanes 0-127, one row per thread)
+//   warps 4-7  softmax for query tile 1
+//   warp 8     TMA producer: Q tiles once, then K and V tiles (2-stage rings)
+//   warp 9     MMA issuer: S_t = Q_t K^T and O_t += P_t V with tcgen05.mma
+// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0, O_1 after.
+// P_t (bf16) is written over the first 64 columns of S_t and fed to the PV
+// MMA straight from tensor memory.  The MMA order per key tile j is
+// PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one warpgroup does the
+// softmax of its tile, the tensor core works on the other tile.
+//
+// Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, drains
+// its own copies and MMAs, frees its tensor memory and returns.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "worklist.h"
+
+namespace cqsa {
+namespace tc {
+
+constexpr int BM = 128;       // query rows per tile (one warpgroup)
+constexpr int QT = 2;         // query tiles per CTA
+constexpr int BN = 128;       // keys per tile
+constexpr int STAGES = 2;     // K and V ring depth
+constexpr int THREADS = 320;
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizzle
+constexpr float LOG2_RESCALE_THRESHOLD = 8.0f;
+
+template <int D>
+struct Smem {
+    static constexpr int KB = D / 64;
+    alignas(1024) uint8_t q[QT][KB][BOX_BYTES];
+    alignas(1024) uint8_t k[STAGES][KB][BOX_BYTES];
+    alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
+    uint64_t bar_q;
+    uint64_t k_full[STAGES], k_empty[STAGES], v_full[STAGES], v_empty[STAGES];
+    uint64_t s_full[QT], p_full[QT], o_full, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Keeps the compiler from using registers filled by tcgen05.ld before the
+// matching tcgen05.wait::ld.
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// Warp-uniform bounded wait: every lane polls, then the warp agrees.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t timeout_ns) {
+    bool ok = mbar_wait(bar, parity, abort, timeout_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace tc
+
+template <int D>
+__global__ void __launch_bounds__(tc::THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    using namespace tc;
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    constexpr int KB = D / 64;
+    constexpr uint32_t TILE_BYTES = KB * BOX_BYTES;
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    Smem<D> &s = *reinterpret_cast<Smem<D> *>(smem_raw + pad);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const WlUnit u = p.units[blockIdx.x];
+    const WlEntry e = p.entries[u.entry];
+    const int32_t q0 = u.q0;
+    const int head = u.head;
+    const int32_t q_end = min(q0 + QT * BM, e.q_hi);
+    const int causal = p.causal;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.bar_q, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.k_full[i], 1);
+            mbar_init(&s.k_empty[i], 1);
+            mbar_init(&s.v_full[i], 1);
+            mbar_init(&s.v_empty[i], 1);
+        }
+        for (int t = 0; t < QT; ++t) {
+            mbar_init(&s.s_full[t], 1);
+            mbar_init(&s.p_full[t], BM);
+        }
+        mbar_init(&s.o_full, 1);
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(&s.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    volatile int *abort = &s.abort;
+    const int ntiles = unit_key_tiles(e, p.runs, q0, QT * BM, causal, BN);
+
+    if (warp == WARP_TMA) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_expect_tx(&s.bar_q, QT * TILE_BYTES);
+            for (int t = 0; t < QT; ++t)
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_3d(s.q[t][kb], &tmQ, &s.bar_q, kb * 64, head, q0 + t * BM);
+            int jk = 0, jv = 0;
+            bool ok = true;
+            for (int r = 0; r < e.run_count && ok; ++r) {
+                int32_t lo, hi;
+                clip_run(e, p.runs[e.run_begin + r], q_end, causal, &lo, &hi);
+                for (int32_t ks = lo; ks < hi; ks += BN) {
+                    const int st = jk % STAGES;
+                    const uint32_t ph = (uint32_t)(jk / STAGES) & 1u;
+                    if (!mbar_wait(&s.k_empty[st], ph ^ 1u, abort, tmo)) { ok = false; break; }
+                    mbar_expect_tx(&s.k_full[st], TILE_BYTES);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_3d(s.k[st][kb], &tmK, &s.k_full[st], kb * 64, head, ks);
+                    ++jk;
+                    if (!mbar_wait(&s.v_empty[st], ph ^ 1u, abort, tmo)) { ok = false; break; }
+                    mbar_expect_tx(&s.v_full[st], TILE_BYTES);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_3d(s.v[st][kb], &tmV, &s.v_full[st], kb * 64, head, ks);
+                    ++jv;
+                }
+            }
+            if (!ok) {
+                atomicExch(p.err, DEV_TIMEOUT);
+                // Let the copies already issued land before the CTA exits.
+                int zero = 0;
+                mbar_wait(&s.bar_q, 0, (volatile int *)&zero, tmo);
+                for (int i = max(0, jk - STAGES); i < jk; ++i)
+                    mbar_wait(&s.k_full[i % STAGES], (uint32_t)(i / STAGES) & 1u,
+                              (volatile int *)&zero, tmo);
+                for (int i = max(0, jv - STAGES); i < jv; ++i)
+                    mbar_wait(&s.v_full[i % STAGES], (uint32_t)(i / STAGES) & 1u,
+                              (volatile int *)&zero, tmo);
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && !p.stall_test) {
+            bool ok = mbar_wait(&s.bar_q, 0, abort, tmo);
+            auto issue_qk = [&](int t, int st) {
+                const uint32_t qa = smem_u32(s.q[t][0]);
+                const uint32_t ka = smem_u32(s.k[st][0]);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
+                    mma_ss(tmem + (uint32_t)t * 128u, smem_desc_sw128(qa + off, 16, 1024),
+                           smem_desc_sw128(ka + off, 16, 1024), IDESC_QK, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int t, int st, bool acc) {
+                const uint32_t va = smem_u32(s.v[st][0]);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    mma_ts(tmem + 256u + (uint32_t)(t * D), tmem + (uint32_t)t * 128u + (uint32_t)kk * 8u,
+                           smem_desc_sw128(va + (uint32_t)kk * 2048u, BOX_BYTES, 1024), IDESC_PV,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            if (ok && ntiles > 0) {
+                ok = mbar_wait(&s.k_full[0], 0, abort, tmo);
+                if (ok) {
+                    tc_fence_after();
+                    for (int t = 0; t < QT; ++t) {
+                        issue_qk(t, 0);
+                        mma_commit(&s.s_full[t]);
+                    }
+                    mma_commit(&s.k_empty[0]);
+                }
+            }
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int st = j % STAGES;
+                const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
+                const bool has_next = (j + 1) < ntiles;
+                const int st1 = (j + 1) % STAGES;
+                const uint32_t ph1 = (uint32_t)((j + 1) / STAGES) & 1u;
+                if (!mbar_wait(&s.v_full[st], ph, abort, tmo)) { ok = false; break; }
+                if (has_next && !mbar_wait(&s.k_full[st1], ph1, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                for (int t = 0; t < QT; ++t) {
+                    if (!mbar_wait(&s.p_full[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv(t, st, j > 0);
+                    if (t == QT - 1) mma_commit(&s.v_empty[st]);
+                    if (has_next) {
+                        issue_qk(t, st1);
+                        mma_commit(&s.s_full[t]);
+                    }
+                }
+                if (ok && has_next) mma_commit(&s.k_empty[st1]);
+            }
+            if (ok) {
+                mma_commit(&s.o_full);
+            } else {
+                atomicExch(p.err, DEV_TIMEOUT);
+            }
+            // Every MMA issued above must finish before tensor memory is freed.
+            mma_commit(&s.drain);
+            int zero = 0;
+            mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int t = warp >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int32_t q_local = q0 + t * BM + row;
+        const int64_t q_glob = (int64_t)q_local + e.q_goff;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t s_addr = lane_base + (uint32_t)t * 128u;
+        const uint32_t o_addr = lane_base + 256u + (uint32_t)(t * D);
+        const float sl2 = p.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        int j = 0;
+        for (int r = 0; r < e.run_count && ok; ++r) {
+            const WlRun run = p.runs[e.run_begin + r];
+            int32_t lo, hi;
+            clip_run(e, run, q_end, causal, &lo, &hi);
+            for (int32_t ks = lo; ks < hi; ks += BN, ++j) {
+                if (!warp_wait(&s.s_full[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                float sv[BN];
+                {
+                    uint32_t a[32], b[32], c[32], d[32];
+                    tmem_ld32(s_addr + 0, a);
+                    tmem_ld32(s_addr + 32, b);
+                    tmem_ld32(s_addr + 64, c);
+                    tmem_ld32(s_addr + 96, d);
+                    tmem_wait_ld();
+                    reg_fence32(a);
+                    reg_fence32(b);
+                    reg_fence32(c);
+                    reg_fence32(d);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        sv[i] = __uint_as_float(a[i]);
+                        sv[32 + i] = __uint_as_float(b[i]);
+                        sv[64 + i] = __uint_as_float(c[i]);
+                        sv[96 + i] = __uint_as_float(d[i]);
+                    }
+                }
+                // CQS mask inside a tile: the end of a key run (ragged
+                // blocks) and the causal triangle on the diagonal block.
+                const int64_t kg0 = (int64_t)ks + run.k_goff;
+                const bool need_mask = (ks + BN > run.k_hi) || (causal && kg0 + BN - 1 > q_glob);
+                if (need_mask) {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) {
+                        const bool keep = (ks + c < run.k_hi) && (!causal || kg0 + c <= q_glob);
+                        if (!keep) sv[c] = -INFINITY;
+                    }
+                }
+                float mx = sv[0];
+#pragma unroll
+                for (int c = 1; c < BN; ++c) mx = fmaxf(mx, sv[c]);
+                const float xm = mx * sl2;
+                // Online softmax with a lazy rescale: the running max only
+                // moves when the tile max exceeds it by 2^8, so most tiles
+                // skip the O correction; values stay below 2^8 meanwhile.
+                const float m_new = (xm > m_run + LOG2_RESCALE_THRESHOLD) ? xm : m_run;
+                const float alpha = (m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
+                l_run *= alpha;
+                m_run = m_new;
+                const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+                float sum = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float p0 = ex2_approx(fmaf(sv[half * 64 + 2 * i], sl2, -mu));
+                        const float p1 = ex2_approx(fmaf(sv[half * 64 + 2 * i + 1], sl2, -mu));
+                        sum += p0 + p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(s_addr + (uint32_t)(half * 32), pk);
+                }
+                // O correction after P is out of registers (lower pressure);
+                // PV_t(j) waits for p_full, so it sees the corrected O.
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
+                        tmem_wait_ld();
+                        reg_fence32(o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(o_addr + (uint32_t)(cc * 32), o);
+                    }
+                }
+                l_run += sum;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&s.p_full[t]);
+            }
+        }
+        if (ok) ok = warp_wait(&s.o_full, 0, abort, tmo);
+        if (ok) {
+            tc_fence_after();
+            const bool valid = q_local < e.q_hi;
+            const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+            float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + q_local) * p.H + head) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
+                tmem_wait_ld();
+                reg_fence32(o);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 v4 = make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                        *reinterpret_cast<float4 *>(dst + cc * 32 + i) = v4;
+                    }
+                }
+            }
+            if (valid) {
+                const float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+                p.part_lse[((int64_t)e.slot * p.H + head) * p.part_rows + q_local] = lse;
+            }
+        } else {
+            if (lane == 0) atomicExch(p.err, DEV_TIMEOUT);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int D>
+static size_t tc_smem_bytes() {
+    return sizeof(tc::Smem<D>) + 1024;
+}
+
+template <int D>
+static cudaError_t launch_tc(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const AttnParams &p, int num_units, cudaStream_t stream) {
+    const size_t smem = tc_smem_bytes<D>();
+    cudaError_t err = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+    if (err != cudaSuccess) return err;
+    attn_tc_kernel<D><<<num_units, tc::THREADS, smem, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attn_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const AttnParams &p, int num_units, cudaStream_t stream) {
+    if (num_units <= 0) return cudaSuccess;
+    if (d == 128) return launch_tc<128>(mq, mk, mv, p, num_units, stream);
+    if (d == 64) return launch_tc<64>(mq, mk, mv, p, num_units, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace cqsa

@@ -1,0 +1,356 @@
+// planner.cpp -- CQS planner (see planner.h for the sources it follows).
+#include "planner.h"
+
+#include <algorithm>
+#include <numeric>
+
+namespace cqsa {
+
+// ---------------------------------------------------------------------------
+// Perfect difference sets ("The CQS Divide"; arXiv abstract: cyclic quorum
+// sets).  D of size l mod c = l(l-1)+1 such that every nonzero residue is a
+// difference of two members exactly once.  Depth-first search in increasing
+// order, so the first set found is the lexicographically first one that
+// starts 0, 1.
+// ---------------------------------------------------------------------------
+static bool pds_search(int c, int l, std::vector<int> *cur, std::vector<char> *used) {
+    if ((int)cur->size() == l) return true;
+    for (int x = cur->back() + 1; x < c; ++x) {
+        // Remaining slots must still fit below c.
+        if (c - x < l - (int)cur->size()) break;
+        std::vector<int> added;
+        bool ok = true;
+        for (int y : *cur) {
+            const int a = ((x - y) % c + c) % c;
+            const int b = (c - a) % c;
+            if ((*used)[a] || (*used)[b] || a == b) { ok = false; break; }
+            (*used)[a] = (*used)[b] = 1;
+            added.push_back(a);
+            added.push_back(b);
+        }
+        if (ok) {
+            cur->push_back(x);
+            if (pds_search(c, l, cur, used)) return true;
+            cur->pop_back();
+        }
+        for (int a : added) (*used)[a] = 0;
+    }
+    return false;
+}
+
+bool find_difference_set(int l, std::vector<int> *D) {
+    D->clear();
+    if (l < 2 || l > 64) return false;
+    const int c = l * (l - 1) + 1;
+    std::vector<int> cur = {0, 1};
+    std::vector<char> used(c, 0);
+    used[1] = used[c - 1] = 1;
+    if (l == 2) { *D = cur; return true; }
+    if (!pds_search(c, l, &cur, &used)) return false;
+    *D = cur;
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// Plan construction.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct Node {
+    std::vector<int> path;
+    std::vector<int64_t> blocks;
+    std::vector<std::vector<int>> chunk;  // [level][member] chunk index at that level
+};
+
+}  // namespace
+
+std::string Planner::build(const PlanSpec &s, int *code) {
+    spec = s;
+    *code = 1;  // INVALID_ARG unless changed
+    if (s.N <= 0 || s.H <= 0 || s.d <= 0) return "N, H and d must be positive";
+    if (s.levels < 1 || s.levels > kMaxLevels) return "levels must be in 1..4";
+    if (s.N > (int64_t)INT32_MAX) return "N must be below 2^31";
+    levels.clear();
+    num_blocks = 1;
+    for (int i = 0; i < s.levels; ++i) {
+        Level L;
+        L.l = s.l[i];
+        if (L.l < 2 || L.l > 16) return "each level's l must be in 2..16";
+        L.c = L.l * (L.l - 1) + 1;
+        if (!find_difference_set(L.l, &L.D)) {
+            *code = 2;
+            return "no perfect difference set of size " + std::to_string(L.l) + " mod " +
+                   std::to_string(L.c);
+        }
+        num_blocks *= L.c;
+        levels.push_back(L);
+    }
+    if (s.N % num_blocks != 0)
+        return "N (" + std::to_string(s.N) + ") must be divisible by the product of chunk counts (" +
+               std::to_string(num_blocks) + ")";
+    block = s.N / num_blocks;
+
+    // Recursive division ("The Recursive Benefit"): level i divides each
+    // parent's token sequence (its blocks in increasing order) into c_i equal
+    // chunks and forms the c_i subsequences {(x + k) mod c_i : x in D_i}.
+    std::vector<Node> frontier(1);
+    frontier[0].blocks.resize(num_blocks);
+    std::iota(frontier[0].blocks.begin(), frontier[0].blocks.end(), 0);
+    for (int i = 0; i < s.levels; ++i) {
+        const Level &L = levels[i];
+        std::vector<Node> next;
+        next.reserve(frontier.size() * L.c);
+        for (const Node &p : frontier) {
+            const int64_t n = (int64_t)p.blocks.size();
+            const int64_t per = n / L.c;
+            for (int k = 0; k < L.c; ++k) {
+                std::vector<char> in(L.c, 0);
+                for (int x : L.D) in[(x + k) % L.c] = 1;
+                Node ch;
+                ch.path = p.path;
+                ch.path.push_back(k);
+                ch.chunk.resize(i + 1);
+                for (int64_t m = 0; m < n; ++m) {
+                    const int a = (int)(m / per);
+                    if (!in[a]) continue;
+                    ch.blocks.push_back(p.blocks[m]);
+                    for (int j = 0; j < i; ++j) ch.chunk[j].push_back(p.chunk[j][m]);
+                    ch.chunk[i].push_back(a);
+                }
+                next.push_back(std::move(ch));
+            }
+        }
+        frontier.swap(next);
+    }
+
+    // CQS mask of a leaf ("Implementation"): at every level, a pair of
+    // distinct chunks is allowed; the diagonal pair (a, a) only in the
+    // subsequence that owns it, k = (a - D[0]) mod c.  Causal keeps key
+    // blocks at or before the query block (the diagonal block's upper
+    // triangle is removed inside the kernel).
+    leaves.clear();
+    entries.clear();
+    entry_begin_of_leaf_.clear();
+    slots_per_block.assign(num_blocks, 0);
+    first_leaf_.assign(num_blocks, -1);
+    last_leaf_.assign(num_blocks, -1);
+    max_task_rows = 0;
+    for (int64_t t = 0; t < (int64_t)frontier.size(); ++t) {
+        const Node &nd = frontier[t];
+        const int64_t n = (int64_t)nd.blocks.size();
+        max_task_rows = std::max<int64_t>(max_task_rows, n * block);
+        entry_begin_of_leaf_.push_back((int64_t)entries.size());
+        for (int64_t mq = 0; mq < n; ++mq) {
+            Entry e;
+            e.task = t;
+            e.qb = nd.blocks[mq];
+            e.mq = (int32_t)mq;
+            for (int64_t mk = 0; mk < n; ++mk) {
+                bool ok = true;
+                for (int i = 0; i < s.levels && ok; ++i) {
+                    const Level &L = levels[i];
+                    const int a = nd.chunk[i][mq], b = nd.chunk[i][mk];
+                    if (a == b) {
+                        const int owner = ((a - L.D[0]) % L.c + L.c) % L.c;
+                        ok = (owner == nd.path[i]);
+                    }
+                }
+                if (ok && s.causal && nd.blocks[mk] > nd.blocks[mq]) ok = false;
+                if (!ok) continue;
+                const int64_t kb = nd.blocks[mk];
+                if (!e.runs.empty() && e.runs.back().b1 + 1 == kb &&
+                    e.runs.back().m0 + (e.runs.back().b1 - e.runs.back().b0) + 1 == mk) {
+                    e.runs.back().b1 = kb;
+                } else {
+                    e.runs.push_back(KeyRun{kb, kb, (int32_t)mk});
+                }
+            }
+            if (e.runs.empty()) continue;
+            e.slot = slots_per_block[e.qb]++;
+            if (first_leaf_[e.qb] < 0) first_leaf_[e.qb] = (int32_t)t;
+            last_leaf_[e.qb] = (int32_t)t;
+            entries.push_back(std::move(e));
+        }
+        Leaf lf;
+        lf.path = nd.path;
+        lf.blocks = nd.blocks;
+        leaves.push_back(std::move(lf));
+    }
+    entry_begin_of_leaf_.push_back((int64_t)entries.size());
+    max_slots = 0;
+    for (int32_t v : slots_per_block) max_slots = std::max<int64_t>(max_slots, v);
+    size_plan();
+    *code = 0;
+    return "";
+}
+
+// ---------------------------------------------------------------------------
+// Work lists.
+// ---------------------------------------------------------------------------
+static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int causal) {
+    std::vector<WlUnit> u;
+    for (int32_t ei = 0; ei < (int32_t)wl->entries.size(); ++ei) {
+        const WlEntry &e = wl->entries[ei];
+        for (int h = 0; h < heads; ++h)
+            for (int32_t q0 = e.q_lo; q0 < e.q_hi; q0 += rows_per_unit) {
+                WlUnit x;
+                x.entry = ei;
+                x.q0 = q0;
+                x.head = h;
+                x.ntiles = unit_key_tiles(e, wl->runs.data(), q0, rows_per_unit, causal, bn);
+                if (x.ntiles > 0) u.push_back(x);
+            }
+    }
+    // Longest units first (LPT order) so the tail of the grid is short;
+    // the stable sort keeps units of one entry and head together.
+    std::stable_sort(u.begin(), u.end(),
+                     [](const WlUnit &a, const WlUnit &b) { return a.ntiles > b.ntiles; });
+    wl->units.swap(u);
+}
+
+WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
+    WorkList wl;
+    for (const Entry &e : entries) {
+        WlEntry w{};
+        w.q_lo = (int32_t)(e.qb * block);
+        w.q_hi = (int32_t)((e.qb + 1) * block);
+        w.q_goff = 0;
+        w.slot = (int32_t)e.slot;
+        w.run_begin = (int32_t)wl.runs.size();
+        w.run_count = (int32_t)e.runs.size();
+        for (const KeyRun &r : e.runs) {
+            WlRun x{};
+            x.k_lo = (int32_t)(r.b0 * block);
+            x.k_hi = (int32_t)((r.b1 + 1) * block);
+            x.k_goff = 0;
+            wl.runs.push_back(x);
+        }
+        wl.entries.push_back(w);
+    }
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal);
+    return wl;
+}
+
+WorkList Planner::leaf_worklist(int64_t t, int rows_per_unit, int bn, int heads) const {
+    WorkList wl;
+    for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+        const Entry &e = entries[i];
+        WlEntry w{};
+        w.q_lo = (int32_t)(e.mq * block);
+        w.q_hi = (int32_t)((e.mq + 1) * block);
+        w.q_goff = (int32_t)((e.qb - e.mq) * block);
+        w.slot = 0;
+        w.run_begin = (int32_t)wl.runs.size();
+        w.run_count = (int32_t)e.runs.size();
+        for (const KeyRun &r : e.runs) {
+            WlRun x{};
+            x.k_lo = (int32_t)(r.m0 * block);
+            x.k_hi = (int32_t)((r.m0 + (r.b1 - r.b0) + 1) * block);
+            x.k_goff = (int32_t)((r.b0 - r.m0) * block);
+            wl.runs.push_back(x);
+        }
+        wl.entries.push_back(w);
+    }
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal);
+    return wl;
+}
+
+std::vector<MergeSeg> Planner::leaf_merge_segments(int64_t t) const {
+    std::vector<MergeSeg> segs;
+    for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+        const Entry &e = entries[i];
+        MergeSeg s{};
+        s.local_lo = (int32_t)(e.mq * block);
+        s.rows = (int32_t)block;
+        s.global_lo = (int32_t)(e.qb * block);
+        s.flags = (first_leaf_[e.qb] == t ? SEG_FIRST : 0) | (last_leaf_[e.qb] == t ? SEG_LAST : 0);
+        segs.push_back(s);
+    }
+    return segs;
+}
+
+void Planner::leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char> *need_kv) const {
+    const size_t n = leaves[t].blocks.size();
+    need_q->assign(n, 0);
+    need_kv->assign(n, 0);
+    for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+        const Entry &e = entries[i];
+        (*need_q)[e.mq] = 1;
+        for (const KeyRun &r : e.runs)
+            for (int64_t b = r.b0; b <= r.b1; ++b) (*need_kv)[r.m0 + (b - r.b0)] = 1;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Memory sizing (layerthelatestinalattice.com summary: subproblems fit a
+// stated memory budget).  Every byte the library holds on the device lives
+// in one arena whose layout the runtime rebuilds with the same ArenaLayout
+// steps, so these totals are exact.
+// ---------------------------------------------------------------------------
+static size_t wl_bytes(const WorkList &wl) {
+    ArenaLayout a;
+    a.take(wl.entries.size() * sizeof(WlEntry));
+    a.take(wl.runs.size() * sizeof(WlRun));
+    a.take(wl.units.size() * sizeof(WlUnit));
+    return a.total;
+}
+
+size_t Planner::device_arena_bytes() const {
+    const int64_t N = spec.N;
+    ArenaLayout a;
+    a.take(256);                                                    // error word
+    a.take((size_t)max_slots * N * spec.H * spec.d * sizeof(float)); // partial O
+    a.take((size_t)max_slots * spec.H * N * sizeof(float));          // partial lse
+    a.take((size_t)num_blocks * sizeof(int32_t));                    // slots per block
+    WorkList wl = device_worklist(unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), spec.H);
+    a.take(wl_bytes(wl));
+    return a.total;
+}
+
+size_t Planner::host_arena_bytes(int g) const {
+    const int64_t N = spec.N, R = max_task_rows;
+    const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
+    ArenaLayout a;
+    a.take(256);                                        // error word
+    a.take((size_t)N * g * dd * sizeof(float));         // accumulator O
+    a.take((size_t)g * N * sizeof(float));              // accumulator lse
+    for (int s = 0; s < 2; ++s) {
+        for (int x = 0; x < 3; ++x) a.take((size_t)R * g * dd * e);   // staged q, k, v
+        a.take((size_t)R * g * dd * e);                 // finished out rows
+        a.take((size_t)g * R * sizeof(float));          // finished lse rows
+    }
+    a.take((size_t)R * g * dd * sizeof(float));         // task partial O
+    a.take((size_t)g * R * sizeof(float));              // task partial lse
+    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+        WorkList wl = leaf_worklist(t, unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
+        a.take(wl_bytes(wl));
+        a.take(leaf_merge_segments(t).size() * sizeof(MergeSeg));
+    }
+    return a.total;
+}
+
+void Planner::size_plan() {
+    sizing = Sizing{};
+    sizing.device_arena = device_arena_bytes();
+    for (int g = spec.H; g >= 1; --g) {
+        if (spec.H % g) continue;
+        const size_t b = host_arena_bytes(g);
+        if (spec.budget == 0 || b <= spec.budget) {
+            sizing.head_group = g;
+            sizing.host_arena = b;
+            break;
+        }
+    }
+    const size_t row_bytes = (size_t)spec.H * spec.d * spec.elem_bytes;
+    size_t h2d = 0;
+    std::vector<char> nq, nkv;
+    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+        leaf_needs(t, &nq, &nkv);
+        for (size_t m = 0; m < nq.size(); ++m)
+            h2d += (size_t)(nq[m] + 2 * nkv[m]) * block * row_bytes;
+    }
+    sizing.h2d = h2d;
+    sizing.d2h = (size_t)spec.N * row_bytes + (size_t)spec.H * spec.N * sizeof(float);
+}
+
+}  // namespace cqsa

@@ -1,0 +1,122 @@
+// planner.h -- host-side CQS planner: difference sets, subsequence tasks,
+// CQS masks, recursion, work lists and memory sizing.  Pure C++ (no CUDA).
+//
+// Follows "Stream-CQSA: Breaking the Billion-Token Barrier on a Single GPU"
+// (wispaper.ai blog): section "The CQS Divide" (c = l(l-1)+1 chunks, c
+// subsequences of l chunks, every chunk pair exactly once), section "The
+// Recursive Benefit" (divide a subsequence again), section "Implementation"
+// (CQS mask against redundant work in overlapping chunks; stream each task's
+// Q_i, K_i, V_i), and the layerthelatestinalattice.com summary (subproblems
+// sized to a memory budget).
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "worklist.h"
+
+namespace cqsa {
+
+constexpr int kMaxLevels = 4;
+
+struct Level {
+    int l = 0;            // chunks per subsequence
+    int c = 0;            // chunks = l(l-1)+1
+    std::vector<int> D;   // perfect difference set mod c
+};
+
+struct Leaf {
+    std::vector<int> path;                  // subsequence index per level
+    std::vector<int64_t> blocks;            // global blocks, increasing
+};
+
+struct KeyRun {
+    int64_t b0, b1;                         // global key blocks, inclusive
+    int32_t m0;                             // leaf member index of b0
+};
+
+struct Entry {
+    int64_t task;                           // leaf index
+    int64_t qb;                             // global query block
+    int32_t mq;                             // leaf member index of qb
+    int64_t slot;                           // partial index for qb
+    std::vector<KeyRun> runs;
+};
+
+// Work list for one launch domain (device mode: the whole sequence; host
+// mode: one leaf task in its local buffers).
+struct WorkList {
+    std::vector<WlEntry> entries;
+    std::vector<WlRun> runs;
+    std::vector<WlUnit> units;
+};
+
+struct PlanSpec {
+    int64_t N = 0;
+    int H = 0, d = 0;
+    int levels = 0;
+    int l[kMaxLevels] = {0, 0, 0, 0};
+    int causal = 0;
+    int elem_bytes = 2;                     // 2 = bf16, 4 = fp32
+    size_t budget = 0;                      // 0 = unlimited
+};
+
+struct Sizing {
+    int head_group = 0;
+    size_t host_arena = 0;
+    size_t device_arena = 0;
+    size_t h2d = 0, d2h = 0;
+};
+
+class Planner {
+public:
+    // Returns "" on success, else an error message; *code gets a status.
+    std::string build(const PlanSpec &spec, int *code);
+
+    PlanSpec spec;
+    std::vector<Level> levels;
+    int64_t num_blocks = 0;     // prod c_i
+    int64_t block = 0;          // tokens per block
+    std::vector<Leaf> leaves;
+    std::vector<Entry> entries; // ordered by (task, qb)
+    std::vector<int32_t> slots_per_block;
+    int64_t max_slots = 0;
+    int64_t max_task_rows = 0;
+    Sizing sizing;
+
+    // rows_per_unit: query rows one CTA covers; bn: key tile width.
+    WorkList device_worklist(int rows_per_unit, int bn, int heads) const;
+    WorkList leaf_worklist(int64_t t, int rows_per_unit, int bn, int heads) const;
+    // Merge segments of leaf t in host mode (one per query block with an
+    // entry), with first/last-touch flags in leaf order.
+    std::vector<MergeSeg> leaf_merge_segments(int64_t t) const;
+    // Members of leaf t whose Q (resp. K/V) rows a streamed task needs.
+    void leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char> *need_kv) const;
+
+    // Arena bytes of each mode for a head group g (host) / all heads (device).
+    size_t host_arena_bytes(int g) const;
+    size_t device_arena_bytes() const;
+
+private:
+    std::vector<int64_t> entry_begin_of_leaf_;  // first entry index of each leaf
+    std::vector<int32_t> first_leaf_, last_leaf_; // per query block
+    void size_plan();
+};
+
+// Lexicographically first perfect difference set of size l mod l(l-1)+1
+// containing {0, 1}; false if none exists.
+bool find_difference_set(int l, std::vector<int> *D);
+
+// Byte offsets of the sub-buffers of an arena, 256-byte aligned.
+struct ArenaLayout {
+    size_t total = 0;
+    size_t take(size_t bytes) {
+        size_t off = total;
+        total += (bytes + 255) & ~size_t(255);
+        return off;
+    }
+};
+
+}  // namespace cqsa

@@ -1,0 +1,167 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every
+symbol include/cqsa.h declares, and its planner matches the CQS reference in
+the oracle bit for bit (integer work)."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import cqs_ref
+from out_core_scheduling_b200 import cqsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    from out_core_scheduling_b200 import build
+    build.build()
+    cqsa.load_library()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "cqsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(cqsa_[a-z_]+)\s*\(", src))
+
+
+def test_exports_every_declared_symbol():
+    declared = header_functions()
+    assert declared == set(cqsa.EXPORTS)
+    lib = cqsa.load_library()
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+@pytest.mark.parametrize("l", [2, 3, 4, 5, 6, 8])
+def test_difference_set_matches_reference(l):
+    assert cqsa.cqsa_difference_set(l) == cqs_ref.perfect_difference_set(l)
+
+
+def test_no_difference_set_error():
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_difference_set(7)
+    assert ei.value.status == cqsa.CQSA_ERR_NO_DIFFERENCE_SET
+
+
+def plan_pairs(plan):
+    info = plan.info()
+    pairs = set()
+    for i in range(info["num_entries"]):
+        e = plan.entry(i)
+        for b0, b1 in e["runs"]:
+            for kb in range(b0, b1 + 1):
+                pairs.add((e["task"], e["q_block"], kb))
+    return pairs
+
+
+def reference_pairs(P, ls, causal):
+    out = set()
+    for t, leaf in enumerate(cqs_ref.leaf_tasks(P, ls)):
+        ps = cqs_ref.causal_pairs(leaf.pairs) if causal else leaf.pairs
+        out |= {(t, qb, kb) for (qb, kb) in ps}
+    return out
+
+
+CASES = [((3,), 7), ((4,), 13), ((5,), 21), ((6,), 31), ((4, 3), 91), ((3, 3), 49)]
+
+
+@pytest.mark.parametrize("ls,P", CASES, ids=lambda x: str(x))
+@pytest.mark.parametrize("causal", [False, True])
+def test_planner_matches_reference(ls, P, causal):
+    B = 3
+    plan = cqsa.cqsa_plan_ex(P * B, 2, 64, list(ls), causal=causal)
+    info = plan.info()
+    assert info["num_tasks"] == P and info["num_blocks"] == P and info["block_tokens"] == B
+    ref = cqs_ref.leaf_tasks(P, ls)
+    for t, leaf in enumerate(ref):
+        blocks, path = plan.task_blocks(t)
+        assert blocks == leaf.blocks and tuple(path) == leaf.path
+    assert plan_pairs(plan) == reference_pairs(P, ls, causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_slots_number_each_query_block(causal):
+    plan = cqsa.cqsa_plan_ex(91 * 2, 1, 64, [4, 3], causal=causal)
+    info = plan.info()
+    seen = {}
+    for i in range(info["num_entries"]):
+        e = plan.entry(i)
+        seen.setdefault(e["q_block"], []).append(e["slot"])
+    for qb, slots in seen.items():
+        assert slots == list(range(len(slots)))
+    assert info["max_slots"] == max(len(s) for s in seen.values())
+    if not causal:
+        assert info["max_slots"] == 12  # l * l' partials per block
+
+
+def test_runs_are_maximal_and_sorted():
+    plan = cqsa.cqsa_plan_ex(13 * 4, 1, 64, [4])
+    for i in range(plan.info()["num_entries"]):
+        runs = plan.entry(i)["runs"]
+        for (a0, a1), (b0, b1) in zip(runs, runs[1:]):
+            assert a1 + 1 < b0
+
+
+def test_configs_plan():
+    """The five workloads plan with the sizes and partitions they name."""
+    GiB = 1 << 30
+    p1 = cqsa.cqsa_plan_ex(3584, 1, 64, [3], dtype=cqsa.CQSA_FP32)
+    assert p1.info()["block_tokens"] == 512 and p1.info()["D"] == [[0, 1, 3]]
+    p2 = cqsa.cqsa_plan(53248, 8, 128, 4, 1, False, 0)
+    i2 = p2.info()
+    assert i2["block_tokens"] == 4096 and i2["num_tasks"] == 13 and i2["head_group"] == 8
+    assert i2["useful_flops"] == 4.0 * 53248 ** 2 * 8 * 128
+    p3 = cqsa.cqsa_plan(688128, 8, 128, 5, 1, False, 2 * GiB)
+    i3 = p3.info()
+    assert i3["num_tasks"] == 21 and 0 < i3["head_group"] < 8 and i3["host_arena_bytes"] <= 2 * GiB
+    p4 = cqsa.cqsa_plan_ex(1490944, 4, 128, [4, 3], causal=True, mem_budget_bytes=4 * GiB)
+    i4 = p4.info()
+    assert i4["num_tasks"] == 91 and i4["block_tokens"] == 16384 and i4["host_arena_bytes"] <= 4 * GiB
+    p5 = cqsa.cqsa_plan(2031616, 1, 128, 6, 1, False, 2 * GiB)
+    i5 = p5.info()
+    assert i5["num_tasks"] == 31 and i5["head_group"] == 1 and i5["host_arena_bytes"] <= 2 * GiB
+    assert i5["D"] == [[0, 1, 3, 8, 12, 18]]
+
+
+def test_h2d_bytes_count_needed_blocks():
+    """Non-causal: every block is a query and key block of each of its l
+    tasks, so the streamed path moves each of Q, K, V l times."""
+    p = cqsa.cqsa_plan(13 * 256, 2, 128, 4, 1, False, 0)
+    i = p.info()
+    assert i["h2d_bytes"] == 4 * 3 * 13 * 256 * 2 * 128 * 2
+    assert i["d2h_bytes"] == 13 * 256 * 2 * 128 * 2 + 2 * 13 * 256 * 4
+
+
+def test_auto_levels_recurse_until_it_fits():
+    GiB = 1 << 30
+    one = cqsa.cqsa_plan(7 * 7 * 4096, 1, 128, 3, 1, False, 0).info()
+    p = cqsa.cqsa_plan(7 * 7 * 4096, 1, 128, 3, 0, False, one["host_arena_bytes"] - 1)
+    assert p.info()["levels"] == 2
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1000, 1, 64, 3, 1, False, 0), cqsa.CQSA_ERR_INVALID_ARG),       # 1000 % 7 != 0
+    ((43 * 4, 1, 64, 7, 1, False, 0), cqsa.CQSA_ERR_NO_DIFFERENCE_SET),
+    ((7 * 4, 1, 96, 3, 1, False, 0), cqsa.CQSA_ERR_UNSUPPORTED),
+    ((7 * 4096, 8, 128, 3, 1, False, 1 << 20), cqsa.CQSA_ERR_BUDGET),
+    ((0, 1, 64, 3, 1, False, 0), cqsa.CQSA_ERR_INVALID_ARG),
+])
+def test_plan_errors(args, status):
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_plan(*args)
+    assert ei.value.status == status
+    assert cqsa.load_library().cqsa_last_error()
+
+
+def test_forward_without_device_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    plan = cqsa.cqsa_plan(7 * 4, 1, 64, 3)
+    x = torch.zeros(28, 1, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 28)
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_forward(plan, x, x, x, x.clone(), lse, cqsa.CQSA_DEVICE, stream=0)
+    assert ei.value.status == cqsa.CQSA_ERR_NO_DEVICE

@@ -1,0 +1,170 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs.  Small cases compare every output row; the full-size
+workloads compare 256 seeded query rows computed exactly against all keys."""
+import numpy as np
+import pytest
+import torch
+
+from out_core_scheduling_b200 import cqsa
+from out_core_scheduling_b200.inputs import make_qkv, sample_rows
+
+from parity import check, run
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+GiB = 1 << 30
+
+
+def _inputs(N, H, d, dtype, seed=0, dist="normal", host=False):
+    q, k, v = make_qkv(N, H, d, dtype=dtype, seed=seed, device=DEV, dist=dist)
+    if host:
+        q, k, v = (x.cpu().pin_memory() for x in (q, k, v))
+        torch.cuda.empty_cache()
+    return q, k, v
+
+
+# ---------------------------------------------------------------- device mode
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp32_l3_n3584_d64(causal):
+    """The fp32 workload: l=3, 7 chunks of 512, H=1, d=64; every row."""
+    q, k, v = _inputs(3584, 1, 64, torch.float32)
+    plan = cqsa.cqsa_plan_ex(3584, 1, 64, [3], causal=causal, dtype=cqsa.CQSA_FP32)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(3584), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_small_every_row(causal, d):
+    N, H = 7 * 256, 2
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=1)
+    plan = cqsa.cqsa_plan(N, H, d, 3, 1, causal, 0)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ragged_blocks(causal, dtype):
+    """Blocks of 200 tokens: tiles straddle block ends (ragged tails)."""
+    N, H, d = 7 * 200, 2, 128
+    q, k, v = _inputs(N, H, d, dtype, seed=2)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal,
+                             dtype=cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_l4_multi_tile(causal):
+    N, H, d = 13 * 384, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=3)
+    plan = cqsa.cqsa_plan(N, H, d, 4, 1, causal, 0)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_two_level_device(causal):
+    N, H, d = 91 * 128, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=4)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3], causal=causal)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, sample_rows(N, 512), causal)
+
+
+def test_tiny_blocks_smaller_than_a_tile():
+    """Blocks of 3 tokens: every tile is ragged; a 256-row unit spans many blocks."""
+    N, H, d = 7 * 3, 1, 64
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=5)
+    for causal in (False, True):
+        plan = cqsa.cqsa_plan(N, H, d, 3, 1, causal, 0)
+        out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+        check(out, lse, q, k, v, np.arange(N), causal)
+
+
+def test_repeated_forward_is_deterministic():
+    N, H, d = 7 * 256, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=6)
+    plan = cqsa.cqsa_plan(N, H, d, 3, 1, False, 0)
+    a, la = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    b, lb = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+# ---------------------------------------------------------------- streamed
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_streamed_head_groups(causal, dtype):
+    """Host-resident inputs under a budget that forces head groups < H."""
+    N, H, d = 7 * 256, 4, 128
+    q, k, v = _inputs(N, H, d, dtype, seed=7, host=True)
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    full = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt).info()["host_arena_bytes"]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt, mem_budget_bytes=full // 2)
+    assert plan.info()["head_group"] < H
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_streamed_two_level(causal):
+    N, H, d = 91 * 128, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=8, host=True)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3], causal=causal)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, sample_rows(N, 512), causal)
+
+
+def test_streamed_equals_device():
+    N, H, d = 13 * 256, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=9)
+    plan = cqsa.cqsa_plan(N, H, d, 4, 1, True, 0)
+    a, la = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    b, lb = run(plan, hq, hk, hv, cqsa.CQSA_HOST)
+    # Same kernels, same partial order per block: identical up to merge order.
+    assert (a.cpu().float() - b.float()).abs().max().item() <= 2e-2
+    assert (la.cpu() - lb).abs().max().item() <= 1e-4
+
+
+# ---------------------------------------------------------------- errors
+def test_host_mode_rejects_pageable_memory():
+    N, H, d = 7 * 128, 1, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0)  # pageable CPU tensors
+    plan = cqsa.cqsa_plan(N, H, d, 3)
+    out = torch.empty_like(q)
+    lse = torch.empty(H, N)
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_HOST)
+    assert ei.value.status == cqsa.CQSA_ERR_NOT_PINNED
+
+
+def test_device_mode_rejects_host_pointers():
+    N, H, d = 7 * 128, 1, 128
+    q, k, v = (x.pin_memory() for x in make_qkv(N, H, d, dtype=torch.bfloat16, seed=0))
+    plan = cqsa.cqsa_plan(N, H, d, 3)
+    out = torch.empty_like(q).pin_memory()
+    lse = torch.empty(H, N).pin_memory()
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+
+
+def test_bounded_wait_reports_timeout_and_recovers():
+    """The MMA issuer is told to issue nothing: every other warp's bounded
+    wait runs out, the kernel returns, and sync reports CQSA_ERR_TIMEOUT.
+    The context stays usable: the next forward is correct."""
+    N, H, d = 7 * 256, 1, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=10)
+    plan = cqsa.cqsa_plan(N, H, d, 3)
+    plan.debug(timeout_ns=20_000_000, stall_mma=True)
+    out = torch.empty_like(q)
+    lse = torch.empty(H, N, device=DEV)
+    cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    with pytest.raises(cqsa.CqsaError) as ei:
+        plan.sync()
+    assert ei.value.status == cqsa.CQSA_ERR_TIMEOUT
+    plan.debug(timeout_ns=0, stall_mma=False)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), False)
