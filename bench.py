@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the CQS-decomposed exact attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 oracle on host cores
+
+One step = one pass of the whole path over the workload's synthetic input.
+The default workload is CQS l=4 (13 chunks of 4096), N=53248, H=8, d=128,
+bf16, device-resident, run non-causal and causal: a step is both forwards.
+Metric: useful TFLOP/s, 4 N^2 H d per forward (halved when causal).
+
+Rank 0 prints one JSON line.  Under torchrun every rank runs its own
+independent problem (weak scaling, no collective on the data path); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GiB = 1 << 30
+L2_BYTES = 126 * 1000 * 1000
+
+# name -> workload.  "variants" are the causal settings one step runs.
+WORKLOADS = {
+    "cqs-l4-n53248-h8-d128-bf16-device": dict(
+        N=53248, H=8, d=128, ls=[4], dtype="bf16", mode="device", variants=[False, True],
+        dist="normal", budget=0),
+    "cqs-l3-n3584-h1-d64-fp32-device": dict(
+        N=3584, H=1, d=64, ls=[3], dtype="fp32", mode="device", variants=[False],
+        dist="normal", budget=0),
+    "cqs-l5-n688128-h8-d128-bf16-host-2gib": dict(
+        N=688128, H=8, d=128, ls=[5], dtype="bf16", mode="host", variants=[False],
+        dist="normal", budget=2 * GiB),
+    "cqs-l4l3-n1490944-h4-d128-bf16-host-4gib-causal": dict(
+        N=1490944, H=4, d=128, ls=[4, 3], dtype="bf16", mode="host", variants=[True],
+        dist="normal", budget=4 * GiB),
+    "cqs-l6-n2031616-h1-d128-bf16-host-2gib": dict(
+        N=2031616, H=1, d=128, ls=[6], dtype="bf16", mode="host", variants=[False],
+        dist="half_normal_uniform_v", budget=2 * GiB),
+}
+DEFAULT_WORKLOAD = "cqs-l4-n53248-h8-d128-bf16-device"
+METRIC = "exact-attention TFLOP/s (4*N^2*H*d, halved for causal)"
+
+
+# ------------------------------------------------------------------ helpers
+def useful_flops(N: int, H: int, d: int, causal: bool) -> float:
+    return 4.0 * N * N * H * d * (0.5 if causal else 1.0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def profile_traffic(kernel_file: str, summary: str):
+    """Per-launch DRAM bytes recorded in a committed ncu summary, or None when
+    the kernel source has changed since the counters were taken."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
+        src = open(os.path.join(ROOT, "out_core_scheduling_b200", "csrc", kernel_file), "rb").read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with nvidia-smi."""
+
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.device_id],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for_smi(torch, dev: int) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [x for x in vis.split(",") if x.strip()]
+        return ids[dev] if dev < len(ids) else str(dev)
+
+
+# ------------------------------------------------------------------ distributed
+class Dist:
+    """Rank bookkeeping; torch.distributed only when launched by torchrun."""
+
+    def __init__(self, backend: str | None = None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.on = self.world > 1
+        if self.on and not dist.is_initialized():
+            import datetime
+            dist.init_process_group(backend=backend or "nccl",
+                                    timeout=datetime.timedelta(seconds=120))
+
+    def barrier(self, device=None):
+        if self.on:
+            if device is not None and self.dist.get_backend() == "nccl":
+                self.dist.barrier(device_ids=[device])
+            else:
+                self.dist.barrier()
+
+    def max(self, x: float, device="cpu") -> float:
+        if not self.on:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.on and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, W):
+    import torch
+    from out_core_scheduling_b200 import cqsa
+    from out_core_scheduling_b200.inputs import make_qkv
+
+    D = Dist()
+    dev = D.local_rank
+    torch.cuda.set_device(dev)
+    torch_dev = f"cuda:{dev}"
+    cqsa.load_library()  # fails loudly when the library is missing
+    N, H, d = W["N"], W["H"], W["d"]
+    tdt = torch.bfloat16 if W["dtype"] == "bf16" else torch.float32
+    cdt = cqsa.CQSA_BF16 if W["dtype"] == "bf16" else cqsa.CQSA_FP32
+    ebytes = 2 if W["dtype"] == "bf16" else 4
+    seed = D.rank  # each rank: its own independent problem
+
+    plans = [cqsa.cqsa_plan_ex(N, H, d, W["ls"], causal=c, dtype=cdt, mem_budget_bytes=W["budget"])
+             for c in W["variants"]]
+    infos = [p.info() for p in plans]
+    flops_step = sum(useful_flops(N, H, d, c) for c in W["variants"])
+    stream = torch.cuda.current_stream()
+
+    free_before, _ = torch.cuda.mem_get_info()
+    if W["mode"] == "device":
+        q, k, v = make_qkv(N, H, d, dtype=tdt, seed=seed, device=torch_dev, dist=W["dist"])
+        outs = [torch.empty_like(q) for _ in plans]
+        lses = [torch.empty(H, N, device=torch_dev, dtype=torch.float32) for _ in plans]
+        mode = cqsa.CQSA_DEVICE
+        io_bytes = (3 + len(plans)) * q.numel() * ebytes + sum(x.numel() * 4 for x in lses)
+    else:
+        gq, gk, gv = make_qkv(N, H, d, dtype=tdt, seed=seed, device=torch_dev, dist=W["dist"])
+        q, k, v = (x.cpu().pin_memory() for x in (gq, gk, gv))
+        del gq, gk, gv
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        free_before, _ = torch.cuda.mem_get_info()
+        outs = [torch.empty(q.shape, dtype=tdt).pin_memory() for _ in plans]
+        lses = [torch.empty(H, N, dtype=torch.float32).pin_memory() for _ in plans]
+        mode = cqsa.CQSA_HOST
+        io_bytes = 0
+
+    def step():
+        for p, o, l in zip(plans, outs, lses):
+            cqsa.cqsa_forward(p, q, k, v, o, l, mode, stream)
+
+    for _ in range(args.warmup):
+        step()
+    for p in plans:
+        p.sync(stream)
+    free_after, _ = torch.cuda.mem_get_info()
+
+    if args.profile_run:
+        for _ in range(args.steps):
+            step()
+        for p in plans:
+            p.sync(stream)
+        D.close()
+        return
+
+    sampler = ClockSampler(gpu_id_for_smi(torch, dev))
+    for p in plans:
+        p.kernel_stats(reset=True)
+        p.profile(True)
+    sampler.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(dev)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    D.barrier(dev)
+    clocks = sampler.stop()
+    for p in plans:
+        p.profile(False)
+        p.sync(stream)
+    ms = D.max(ev0.elapsed_time(ev1), torch_dev)
+    stats = [p.kernel_stats(reset=True) for p in plans]
+
+    value = flops_step * args.steps * D.world / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+
+    # Roofline of the dominant kernel: the tile-attention launch of the first
+    # variant (non-causal for the default workload), its useful flops over
+    # its mean event-timed duration on the stream it was launched on.
+    attn_ms = sum(s["attn_ms"] for s in stats)
+    attn_launches = sum(s["attn_launches"] for s in stats)
+    s0 = stats[0]
+    launch_ms = s0["attn_ms"] / max(1, s0["attn_launches"])
+    flops_per_forward = useful_flops(N, H, d, W["variants"][0])
+    if W["mode"] == "device":
+        achieved = flops_per_forward / (launch_ms * 1e-3) / 1e12 if launch_ms > 0 else None
+    else:  # one launch per task: all the forward's flops over all its launches
+        achieved = flops_per_forward * args.steps / (s0["attn_ms"] * 1e-3) / 1e12 if s0["attn_ms"] else None
+    if W["dtype"] == "bf16":
+        peak = peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak if achieved else None,
+                    "peak_source": peaks["source"] + " bf16 dense (burst)",
+                    "traffic": (profile_traffic("attn_tc.cu", "attn_tc_l4_n53248_h8_d128.md")
+                                if args.workload == DEFAULT_WORKLOAD else None),
+                    "kernel": f"attn_tc_kernel<{d}> (causal={W['variants'][0]})",
+                    "avg_launch_ms": launch_ms}
+    else:
+        # fp32 FFMA on the CUDA cores: 148 SMs x 128 FMA/clk x 2 flops x max clock.
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak if achieved else None,
+                    "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz",
+                    "traffic": None, "kernel": f"attn_simt_kernel<{d}>",
+                    "avg_launch_ms": launch_ms}
+    merge = None
+    merge_ms = sum(s["merge_ms"] for s in stats)
+    merge_launches = sum(s["merge_launches"] for s in stats)
+    if W["mode"] == "device" and merge_ms > 0:
+        mb = 0.0
+        for info, s in zip(infos, stats):
+            S = info["max_slots"]
+            mb += N * H * (S * (4 * d + 4) + ebytes * d + 4) * s["merge_launches"]
+        merge = {"bound": "hbm", "achieved": mb / (merge_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                 "unit": "GB/s", "frac": mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "bytes_per_launch": mb / max(1, merge_launches), "kernel": "merge_slots_kernel",
+                 "note": "upper bound: assumes every block holds max_slots partials"}
+
+    arena = sum(i["device_arena_bytes"] if W["mode"] == "device" else i["host_arena_bytes"] for i in infos)
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": D.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": W["dtype"], "data": "synthetic (seeded torch.Generator, see inputs.py)",
+        "config": {"workload": args.workload, "N": N, "H": H, "d": d, "l": W["ls"],
+                   "c": [info["c"] for info in infos[:1]][0], "D": infos[0]["D"],
+                   "causal": W["variants"], "mode": W["mode"],
+                   "mem_budget_bytes": W["budget"] or None,
+                   "parallelism": f"independent problem per GPU x{D.world}",
+                   "l2": f"inputs larger than L2 ({3 * N * H * d * ebytes / 1e6:.0f} MB > 126 MB); no flush"},
+        "roofline": roofline,
+        "roofline_merge": merge,
+        "clocks": clocks,
+        "gpu_launches": attn_launches + merge_launches,
+        "per_variant": [{"causal": c, "tflops_kernel": useful_flops(N, H, d, c) * args.steps
+                         / (s["attn_ms"] * 1e-3) / 1e12 if s["attn_ms"] else None,
+                         "attn_ms_per_launch": s["attn_ms"] / max(1, s["attn_launches"]),
+                         "merge_ms_per_launch": s["merge_ms"] / max(1, s["merge_launches"])}
+                        for c, s in zip(W["variants"], stats)],
+        "peak_hbm_gib": {"library_arena": arena / GiB, "inputs_outputs": io_bytes / GiB,
+                         "device_free_delta": (free_before - free_after) / GiB},
+        "wall_ms_timed": (wall1 - wall0) * 1e3,
+    }
+
+    # ---- end to end through the public API from pinned host memory.
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream)
+
+    # ---- oracle on the host cores (rank 0, N = 1 only).
+    if D.rank == 0 and D.world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(W, q, k, v, args.cpu_rows)
+
+    if D.rank == 0:
+        print(json.dumps(result), flush=True)
+    del plans
+    D.close()
+
+
+def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream):
+    import torch
+    from out_core_scheduling_b200 import cqsa
+
+    N, H = W["N"], W["H"]
+    if W["mode"] == "host":
+        hq, hk, hv = q, k, v
+    else:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    outs = [torch.empty(hq.shape, dtype=hq.dtype).pin_memory() for _ in plans]
+    lses = [torch.empty(H, N, dtype=torch.float32).pin_memory() for _ in plans]
+
+    def step():
+        for p, o, l in zip(plans, outs, lses):
+            cqsa.cqsa_forward(p, hq, hk, hv, o, l, cqsa.CQSA_HOST, stream)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, args.e2e_steps))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(D.local_rank)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier(D.local_rank)
+    for p in plans:
+        p.sync(stream)
+    ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}")
+    return {"value": flops_step * steps * D.world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(sum(i["h2d_bytes"] for i in infos)),
+            "d2h_bytes_per_step": int(sum(i["d2h_bytes"] for i in infos)),
+            "steps": steps, "ms_per_step": ms / steps,
+            "path": "cqsa_forward(CQSA_HOST): pinned host q,k,v -> streamed tasks -> pinned host out,lse"}
+
+
+def oracle_sample(W, q, k, v, rows_per_variant, seed):
+    """Time the fp64 oracle on a row sample of each variant; returns
+    (useful flops of the sample, seconds, threads, description)."""
+    import numpy as np
+    import torch
+    import oracle
+    from out_core_scheduling_b200.inputs import sample_rows
+
+    N, H, d = W["N"], W["H"], W["d"]
+    qc, kc, vc = (x.cpu() if x.is_cuda else x for x in (q, k, v))
+    flops, secs = 0.0, 0.0
+    for i, causal in enumerate(W["variants"]):
+        rows = sample_rows(N, rows_per_variant, seed=seed + i).numpy()
+        keys = (rows + 1).sum() if causal else rows.size * N
+        t0 = time.perf_counter()
+        oracle.attention_rows(qc, kc, vc, rows=rows, causal=causal)
+        secs += time.perf_counter() - t0
+        flops += 4.0 * d * H * float(keys)
+    desc = (f"{rows_per_variant} seeded query rows x {H} heads per variant "
+            f"(causal={W['variants']}) against all allowed keys of the workload")
+    return flops, secs, oracle.num_threads(), desc
+
+
+def cpu_baseline(W, q, k, v, rows):
+    flops, secs, threads, desc = oracle_sample(W, q, k, v, rows, seed=1234)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": desc, "seconds": secs}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, W):
+    """The fp64 oracle, as it stands, on the host cores: each step a bounded
+    row sample of the workload.  Rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from out_core_scheduling_b200.inputs import make_qkv
+
+    tdt = torch.bfloat16 if W["dtype"] == "bf16" else torch.float32
+    q, k, v = make_qkv(W["N"], W["H"], W["d"], dtype=tdt, seed=0, device="cpu", dist=W["dist"])
+    for i in range(args.warmup):
+        oracle_sample(W, q, k, v, args.ref_rows, seed=100 + i)
+    flops, secs, threads, desc = 0.0, 0.0, 1, ""
+    for i in range(args.steps):
+        f, s, threads, desc = oracle_sample(W, q, k, v, args.ref_rows, seed=1000 + i)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded torch.Generator, see inputs.py)",
+        "config": {"workload": args.workload, "N": W["N"], "H": W["H"], "d": W["d"],
+                   "l": W["ls"], "causal": W["variants"], "mode": "host cores (oracle)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per variant for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=16, help="oracle rows per variant per reference step")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only warm-up + steps of the device path (for ncu captures)")
+    args = ap.parse_args(argv)
+    if args.warmup < 0 or args.steps < 1:
+        ap.error("need --steps >= 1 and --warmup >= 0")
+    W = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, W)
+    else:
+        run_ours(args, W)
+
+
+if __name__ == "__main__":
+    main()

@@ -177,6 +177,25 @@ cqsa_status_t cqsa_difference_set(int l, int *D);
  * CQSA_ERR_TIMEOUT.  Never needed in normal use. */
 cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_mma);
 
+/* Per-kernel device time of a plan's launches, from CUDA events recorded
+ * on the stream each kernel is launched on. */
+typedef struct {
+    int64_t attn_launches;  /* tile-attention kernel launches */
+    int64_t merge_launches; /* log-sum-exp merge kernel launches */
+    double attn_ms;         /* summed device time of those launches */
+    double merge_ms;
+} cqsa_kernel_stats_t;
+
+/* cqsa_plan_profile -- enable != 0: from the next forward on, record a CUDA
+ * event pair around every kernel the plan launches (a few microseconds per
+ * launch).  enable = 0 stops recording. */
+cqsa_status_t cqsa_plan_profile(cqsa_plan_t *plan, int enable);
+
+/* cqsa_plan_kernel_stats -- wait for the recorded events, add their times to
+ * the plan's totals and copy the totals into *stats; reset != 0 then clears
+ * the totals.  CUDA on an event failure. */
+cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *stats, int reset);
+
 /* cqsa_plan_destroy -- free the plan, its arena, streams and events.  Waits
  * for the plan's outstanding work first.  Null is ignored. */
 void cqsa_plan_destroy(cqsa_plan_t *plan);

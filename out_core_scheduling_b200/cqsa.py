@@ -34,7 +34,7 @@ MAX_L = 16
 EXPORTS = (
     "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_plan_sync", "cqsa_plan_info",
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
-    "cqsa_plan_destroy", "cqsa_last_error",
+    "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_plan_destroy", "cqsa_last_error",
 )
 
 
@@ -75,6 +75,11 @@ class PlanInfo(ctypes.Structure):
         return out
 
 
+class KernelStats(ctypes.Structure):
+    _fields_ = [("attn_launches", ctypes.c_int64), ("merge_launches", ctypes.c_int64),
+                ("attn_ms", ctypes.c_double), ("merge_ms", ctypes.c_double)]
+
+
 class Entry(ctypes.Structure):
     _fields_ = [("task", ctypes.c_int64), ("q_block", ctypes.c_int64),
                 ("slot", ctypes.c_int64), ("num_runs", ctypes.c_int64)]
@@ -107,6 +112,8 @@ def load_library():
                                  ctypes.c_int64]),
         "cqsa_difference_set": (st, [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
         "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
+        "cqsa_plan_profile": (st, [P, ctypes.c_int]),
+        "cqsa_plan_kernel_stats": (st, [P, ctypes.POINTER(KernelStats), ctypes.c_int]),
         "cqsa_plan_destroy": (None, [P]),
         "cqsa_last_error": (ctypes.c_char_p, []),
     }
@@ -167,6 +174,15 @@ class Plan:
 
     def debug(self, timeout_ns: int = 0, stall_mma: bool = False):
         _check(load_library().cqsa_plan_debug(self.handle, timeout_ns, int(bool(stall_mma))))
+
+    def profile(self, enable: bool = True):
+        _check(load_library().cqsa_plan_profile(self.handle, int(bool(enable))))
+
+    def kernel_stats(self, reset: bool = False) -> dict:
+        ks = KernelStats()
+        _check(load_library().cqsa_plan_kernel_stats(self.handle, ctypes.byref(ks), int(bool(reset))))
+        return {"attn_launches": ks.attn_launches, "merge_launches": ks.merge_launches,
+                "attn_ms": ks.attn_ms, "merge_ms": ks.merge_ms}
 
     def destroy(self):
         if self.handle and self.handle.value:

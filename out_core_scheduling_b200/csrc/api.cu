@@ -170,9 +170,46 @@ struct cqsa_plan {
     cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
     cudaEvent_t ev_in_ready[2] = {}, ev_in_free[2] = {}, ev_merged[2] = {}, ev_out_free[2] = {};
     cudaEvent_t ev_start = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
+
+    // Kernel timing (cqsa_plan_profile): event pairs not yet read, a pool of
+    // spare events, and the totals read so far.
+    int profiling = 0;
+    struct Timed { cudaEvent_t a, b; int kind; };
+    std::vector<Timed> pending;
+    std::vector<cudaEvent_t> spare;
+    cqsa_kernel_stats_t totals{};
 };
 
 namespace {
+
+// Event pair around one launch when profiling is on (kind 0 attention, 1 merge).
+struct LaunchTimer {
+    cqsa_plan_t *P;
+    cudaStream_t s;
+    int kind;
+    cudaEvent_t a = nullptr, b = nullptr;
+    static cudaEvent_t get(cqsa_plan_t *P) {
+        if (!P->spare.empty()) {
+            cudaEvent_t e = P->spare.back();
+            P->spare.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        return cudaEventCreate(&e) == cudaSuccess ? e : nullptr;
+    }
+    LaunchTimer(cqsa_plan_t *P_, cudaStream_t s_, int kind_) : P(P_), s(s_), kind(kind_) {
+        if (!P->profiling) return;
+        a = get(P);
+        b = get(P);
+        if (a && b) cudaEventRecord(a, s);
+    }
+    void stop() {
+        if (!P->profiling || !a || !b) return;
+        cudaEventRecord(b, s);
+        P->pending.push_back({a, b, kind});
+        a = b = nullptr;
+    }
+};
 
 cqsa_status_t check_device(cqsa_plan_t *P) {
     int dev = -1;
@@ -365,12 +402,18 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
         if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
         if ((st = make_map(&mk, k, N, H, d)) != CQSA_OK) return st;
         if ((st = make_map(&mv, v, N, H, d)) != CQSA_OK) return st;
+        LaunchTimer tm(P, stream, 0);
         CK(launch_attn_tc(d, mq, mk, mv, ap, P->dev_wl.num_units, stream));
+        tm.stop();
     } else {
+        LaunchTimer tm(P, stream, 0);
         CK(launch_attn_simt(d, P->elem, q, k, v, ap, P->dev_wl.num_units, stream));
+        tm.stop();
     }
+    LaunchTimer tm(P, stream, 1);
     CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H, out, lse,
                           stream));
+    tm.stop();
     return CQSA_OK;
 }
 
@@ -433,17 +476,25 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
             ap.part_lse = P->h_part_lse;
             ap.part_rows = R;
             ap.H = g;
-            if (P->dtype == CQSA_BF16)
-                CK(launch_attn_tc(d, P->mq[s], P->mk[s], P->mv[s], ap, L.wl.num_units, P->s_comp));
-            else
-                CK(launch_attn_simt(d, P->elem, P->in_q[s], P->in_k[s], P->in_v[s], ap, L.wl.num_units,
-                                    P->s_comp));
+            {
+                LaunchTimer tm(P, P->s_comp, 0);
+                if (P->dtype == CQSA_BF16)
+                    CK(launch_attn_tc(d, P->mq[s], P->mk[s], P->mv[s], ap, L.wl.num_units, P->s_comp));
+                else
+                    CK(launch_attn_simt(d, P->elem, P->in_q[s], P->in_k[s], P->in_v[s], ap, L.wl.num_units,
+                                        P->s_comp));
+                tm.stop();
+            }
             CK(cudaEventRecord(P->ev_in_free[s], P->s_comp));
             // -- merge into the accumulator; finished rows go to out stage s.
             if (it >= 2) CK(cudaStreamWaitEvent(P->s_comp, P->ev_out_free[s], 0));
-            CK(launch_merge_stream(d, P->elem, L.segs, (int)L.host_segs.size(), (int)B, P->h_part_o,
-                                   P->h_part_lse, R, P->acc_o, P->acc_lse, N, g, P->out_st[s], P->lse_st[s],
-                                   P->s_comp));
+            {
+                LaunchTimer tm(P, P->s_comp, 1);
+                CK(launch_merge_stream(d, P->elem, L.segs, (int)L.host_segs.size(), (int)B, P->h_part_o,
+                                       P->h_part_lse, R, P->acc_o, P->acc_lse, N, g, P->out_st[s], P->lse_st[s],
+                                       P->s_comp));
+                tm.stop();
+            }
             CK(cudaEventRecord(P->ev_merged[s], P->s_comp));
             // -- D2H of finished rows.
             CK(cudaStreamWaitEvent(P->s_out, P->ev_merged[s], 0));
@@ -591,6 +642,34 @@ cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_
     return CQSA_OK;
 }
 
+cqsa_status_t cqsa_plan_profile(cqsa_plan_t *plan, int enable) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    plan->profiling = enable ? 1 : 0;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *stats, int reset) {
+    if (!plan || !stats) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    for (const auto &t : plan->pending) {
+        CK(cudaEventSynchronize(t.b));
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, t.a, t.b));
+        if (t.kind == 0) {
+            plan->totals.attn_launches++;
+            plan->totals.attn_ms += ms;
+        } else {
+            plan->totals.merge_launches++;
+            plan->totals.merge_ms += ms;
+        }
+        plan->spare.push_back(t.a);
+        plan->spare.push_back(t.b);
+    }
+    plan->pending.clear();
+    *stats = plan->totals;
+    if (reset) plan->totals = cqsa_kernel_stats_t{};
+    return CQSA_OK;
+}
+
 cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     if (!plan || !info) return fail(CQSA_ERR_INVALID_ARG, "null argument");
     const Planner &pl = plan->pl;
@@ -680,6 +759,11 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
             if (plan->ev_merged[s]) cudaEventDestroy(plan->ev_merged[s]);
             if (plan->ev_out_free[s]) cudaEventDestroy(plan->ev_out_free[s]);
         }
+        for (const auto &t : plan->pending) {
+            cudaEventDestroy(t.a);
+            cudaEventDestroy(t.b);
+        }
+        for (cudaEvent_t e : plan->spare) cudaEventDestroy(e);
         if (plan->ev_start) cudaEventDestroy(plan->ev_start);
         if (plan->ev_done_comp) cudaEventDestroy(plan->ev_done_comp);
         if (plan->ev_done_out) cudaEventDestroy(plan->ev_done_out);
