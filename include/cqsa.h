@@ -196,6 +196,36 @@ cqsa_status_t cqsa_plan_profile(cqsa_plan_t *plan, int enable);
  * the totals.  CUDA on an event failure. */
 cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *stats, int reset);
 
+/* Size of the fixed device scratch array behind cqsa_forward_noalloc. */
+#define CQSA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * cqsa_forward_noalloc -- the device-resident forward without any device
+ * allocation.  The pages have no counterpart: this is a convenience of this
+ * library for callers that must not call cudaMalloc at call time (a
+ * framework whose caching allocator already reserved the free device
+ * memory, a process at its device-memory cap, or a loop that cannot afford
+ * cudaMalloc's implicit device synchronisation).
+ *   q, k, v, out: device pointers, [N, H, d] in the plan's dtype; lse: fp32
+ *   [H, N] on the device.  The caller owns them.  The task partials, work
+ *   list and error word live in one file-scope device array of
+ *   CQSA_NOALLOC_SCRATCH_BYTES (64 MiB), placed by the module loader on each
+ *   device that uses it and held until the process exits.
+ *   Limits: the plan's partials (max_slots * N * H * d * 4 bytes, plus lse)
+ *   and work list must fit the array; otherwise CQSA_ERR_BUDGET with the
+ *   sizes in the message, and cqsa_forward is the way.
+ *   The first call on a device looks up the array's address
+ *   (cudaGetSymbolAddress) and loads the library's device code; make it
+ *   before any stream capture.  Calls share the array and keep the last
+ *   call's contents; host callers are serialised, but work of two calls that
+ *   overlaps on the GPU would race, so the call waits until its own work on
+ *   `stream` has finished and then reports CQSA_ERR_TIMEOUT if a bounded
+ *   device wait ran out.  Calls no cudaMalloc, cudaFree or other allocating
+ *   routine.  Errors: INVALID_ARG, NO_DEVICE, BUDGET, CUDA, TIMEOUT.
+ */
+cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, const void *k,
+                                   const void *v, void *out, float *lse, void *stream);
+
 /* cqsa_plan_destroy -- free the plan, its arena, streams and events.  Waits
  * for the plan's outstanding work first.  Null is ignored. */
 void cqsa_plan_destroy(cqsa_plan_t *plan);

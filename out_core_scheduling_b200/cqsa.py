@@ -34,7 +34,8 @@ MAX_L = 16
 EXPORTS = (
     "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_plan_sync", "cqsa_plan_info",
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
-    "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_plan_destroy", "cqsa_last_error",
+    "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
+    "cqsa_last_error",
 )
 
 
@@ -114,6 +115,7 @@ def load_library():
         "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
         "cqsa_plan_profile": (st, [P, ctypes.c_int]),
         "cqsa_plan_kernel_stats": (st, [P, ctypes.POINTER(KernelStats), ctypes.c_int]),
+        "cqsa_forward_noalloc": (st, [P, P, P, P, P, P, P]),
         "cqsa_plan_destroy": (None, [P]),
         "cqsa_last_error": (ctypes.c_char_p, []),
     }
@@ -238,6 +240,24 @@ def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVIC
     _check(load_library().cqsa_forward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                        out.data_ptr(), lse.data_ptr(), host_or_device,
                                        ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_forward_noalloc(plan: Plan, q, k, v, out, lse, stream=None):
+    """Device-resident forward whose scratch is the library's fixed device
+    array (no device allocation at call time).  Same tensors as
+    ``cqsa_forward`` in CQSA_DEVICE mode; returns after the work on
+    ``stream`` has finished."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
+        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous torch tensor")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be float32")
+    if not (q.shape == k.shape == v.shape == out.shape) or q.dim() != 3:
+        raise ValueError("q, k, v, out must all be [N, H, d]")
+    _check(load_library().cqsa_forward_noalloc(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               out.data_ptr(), lse.data_ptr(),
+                                               ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def cqsa_difference_set(l: int):

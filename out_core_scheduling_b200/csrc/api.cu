@@ -533,6 +533,19 @@ cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
 
 }  // namespace
 
+namespace cqsa {
+
+// Read-only views of a plan for other translation units of this library.
+const Planner &plan_planner(const cqsa_plan_t *P) { return P->pl; }
+int plan_dtype(const cqsa_plan_t *P) { return P->dtype; }
+uint64_t plan_timeout_ns(const cqsa_plan_t *P) { return P->timeout_ns; }
+cqsa_status_t plan_make_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int d) {
+    return make_map(m, base, rows, heads, d);
+}
+cqsa_status_t set_error(cqsa_status_t code, const char *msg) { return fail(code, "%s", msg); }
+
+}  // namespace cqsa
+
 extern "C" {
 
 cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
