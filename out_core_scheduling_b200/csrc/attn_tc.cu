@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "exp2_poly.h"
 #include "kernels.h"
 #include "worklist.h"
 
@@ -68,6 +69,28 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                  :
                  : "memory");
 }
+
+// 2^x on the FMA pipe: Cody-Waite split x = j + f (j = round(x) taken from
+// the low mantissa bits of x + 1.5 * 2^23), 2^f by the degree-3 minimax
+// polynomial of exp2_poly.h, and 2^j added to the exponent field.  Inputs
+// are clamped at -125 so the exponent never wraps (2^-125 is zero for the
+// softmax); masked -inf scores therefore give a negligible positive value.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float y = x + 12582912.f;
+    const float f = x - (y - 12582912.f);
+    float p = fmaf(CQSA_EXP2_C3, f, CQSA_EXP2_C2);
+    p = fmaf(p, f, CQSA_EXP2_C1);
+    p = fmaf(p, f, CQSA_EXP2_C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+
+// Which column pairs of a 128-wide score row take the polynomial instead of
+// the MUFU ex2: POLY_PAIRS_PER_8 of every 8 pairs.  Measured on B200 the
+// softmax is issue- and latency-bound rather than MUFU-bound, where the
+// polynomial's extra instructions cost more than they save, so it is off.
+constexpr int POLY_PAIRS_PER_8 = 0;
+__device__ __forceinline__ constexpr bool poly_pair(int pair) { return (pair & 7) >= 8 - POLY_PAIRS_PER_8; }
 
 // Warp-uniform bounded wait: every lane polls, then the warp agrees.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -113,7 +136,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         for (int t = 0; t < QT; ++t) {
             mbar_init(&s.s_full[t], 1);
-            mbar_init(&s.p_full[t], BM);
+            mbar_init(&s.p_full[t], BM / 32);  // one arrival per softmax warp
         }
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
@@ -176,36 +199,44 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && !p.stall_test) {
-            bool ok = mbar_wait(&s.bar_q, 0, abort, tmo);
+        // The whole warp runs this loop with warp-uniform values; one elected
+        // lane issues each tcgen05 instruction.  Descriptors are built once:
+        // a K step of 16 columns moves the start address by 32 bytes (+2 in
+        // the >>4 field) inside the 128-byte swizzle row, the second 64-column
+        // box is BOX_BYTES further, and a V step of 16 keys is 2048 bytes.
+        if (!p.stall_test) {
+            bool ok = warp_wait(&s.bar_q, 0, abort, tmo);
+            uint64_t qdesc[QT], kdesc[STAGES], vdesc[STAGES];
+            for (int t = 0; t < QT; ++t) qdesc[t] = smem_desc_sw128(smem_u32(s.q[t][0]), 16, 1024);
+            for (int i = 0; i < STAGES; ++i) {
+                kdesc[i] = smem_desc_sw128(smem_u32(s.k[i][0]), 16, 1024);
+                vdesc[i] = smem_desc_sw128(smem_u32(s.v[i][0]), BOX_BYTES, 1024);
+            }
             auto issue_qk = [&](int t, int st) {
-                const uint32_t qa = smem_u32(s.q[t][0]);
-                const uint32_t ka = smem_u32(s.k[st][0]);
+                const uint64_t qa = qdesc[t], kb = kdesc[st];
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
-                    mma_ss(tmem + (uint32_t)t * 128u, smem_desc_sw128(qa + off, 16, 1024),
-                           smem_desc_sw128(ka + off, 16, 1024), IDESC_QK, kk > 0);
+                    const uint64_t off = (uint64_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+                    mma_ss_elect(tmem + (uint32_t)t * 128u, qa + off, kb + off, IDESC_QK, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int t, int st, bool acc) {
-                const uint32_t va = smem_u32(s.v[st][0]);
+                const uint64_t vb = vdesc[st];
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    mma_ts(tmem + 256u + (uint32_t)(t * D), tmem + (uint32_t)t * 128u + (uint32_t)kk * 8u,
-                           smem_desc_sw128(va + (uint32_t)kk * 2048u, BOX_BYTES, 1024), IDESC_PV,
-                           (acc || kk > 0) ? 1u : 0u);
+                    mma_ts_elect(tmem + 256u + (uint32_t)(t * D), tmem + (uint32_t)t * 128u + (uint32_t)kk * 8u,
+                                 vb + (uint64_t)(kk * (2048 >> 4)), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                 }
             };
             if (ok && ntiles > 0) {
-                ok = mbar_wait(&s.k_full[0], 0, abort, tmo);
+                ok = warp_wait(&s.k_full[0], 0, abort, tmo);
                 if (ok) {
                     tc_fence_after();
                     for (int t = 0; t < QT; ++t) {
                         issue_qk(t, 0);
-                        mma_commit(&s.s_full[t]);
+                        mma_commit_elect(&s.s_full[t]);
                     }
-                    mma_commit(&s.k_empty[0]);
+                    mma_commit_elect(&s.k_empty[0]);
                 }
             }
             for (int j = 0; j < ntiles && ok; ++j) {
@@ -214,30 +245,31 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 const bool has_next = (j + 1) < ntiles;
                 const int st1 = (j + 1) % STAGES;
                 const uint32_t ph1 = (uint32_t)((j + 1) / STAGES) & 1u;
-                if (!mbar_wait(&s.v_full[st], ph, abort, tmo)) { ok = false; break; }
-                if (has_next && !mbar_wait(&s.k_full[st1], ph1, abort, tmo)) { ok = false; break; }
+                if (!warp_wait(&s.v_full[st], ph, abort, tmo)) { ok = false; break; }
+                if (has_next && !warp_wait(&s.k_full[st1], ph1, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
                 for (int t = 0; t < QT; ++t) {
-                    if (!mbar_wait(&s.p_full[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                    if (!warp_wait(&s.p_full[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
                     tc_fence_after();
                     issue_pv(t, st, j > 0);
-                    if (t == QT - 1) mma_commit(&s.v_empty[st]);
+                    if (t == QT - 1) mma_commit_elect(&s.v_empty[st]);
                     if (has_next) {
                         issue_qk(t, st1);
-                        mma_commit(&s.s_full[t]);
+                        mma_commit_elect(&s.s_full[t]);
                     }
                 }
-                if (ok && has_next) mma_commit(&s.k_empty[st1]);
+                if (ok && has_next) mma_commit_elect(&s.k_empty[st1]);
             }
             if (ok) {
-                mma_commit(&s.o_full);
-            } else {
+                mma_commit_elect(&s.o_full);
+            } else if (lane == 0) {
                 atomicExch(p.err, DEV_TIMEOUT);
             }
             // Every MMA issued above must finish before tensor memory is freed.
-            mma_commit(&s.drain);
+            mma_commit_elect(&s.drain);
             int zero = 0;
             mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ softmax
@@ -291,9 +323,18 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                         if (!keep) sv[c] = -INFINITY;
                     }
                 }
-                float mx = sv[0];
+                // Row max in 8 independent chains (a single chain would be a
+                // 128-deep dependency).
+                float mx;
+                {
+                    float m8[8];
 #pragma unroll
-                for (int c = 1; c < BN; ++c) mx = fmaxf(mx, sv[c]);
+                    for (int c = 0; c < 8; ++c) m8[c] = sv[c];
+#pragma unroll
+                    for (int c = 8; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
+                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                }
                 const float xm = mx * sl2;
                 // Online softmax with a lazy rescale: the running max only
                 // moves when the tile max exceeds it by 2^8, so most tiles
@@ -303,19 +344,29 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 l_run *= alpha;
                 m_run = m_new;
                 const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-                float sum = 0.f;
+                float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float p0 = ex2_approx(fmaf(sv[half * 64 + 2 * i], sl2, -mu));
-                        const float p1 = ex2_approx(fmaf(sv[half * 64 + 2 * i + 1], sl2, -mu));
-                        sum += p0 + p1;
+                        const int pair = half * 32 + i;
+                        const float x0 = fmaf(sv[2 * pair], sl2, -mu);
+                        const float x1 = fmaf(sv[2 * pair + 1], sl2, -mu);
+                        float p0, p1;
+                        if (poly_pair(pair)) {
+                            p0 = exp2_poly(x0);
+                            p1 = exp2_poly(x1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        s8[i & 7] += p0 + p1;
                         pk[i] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(s_addr + (uint32_t)(half * 32), pk);
                 }
+                const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
                 // O correction after P is out of registers (lower pressure);
                 // PV_t(j) waits for p_full, so it sees the corrected O.
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -333,7 +384,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 l_run += sum;
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&s.p_full[t]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.p_full[t]);
             }
         }
         if (ok) ok = warp_wait(&s.o_full, 0, abort, tmo);
