@@ -351,12 +351,23 @@ def run_ours(args, W):
     }
 
     # ---- end to end through the public API from pinned host memory.
-    if not args.no_e2e:
+    if W["mode"] == "host":
+        # The timed path already starts and ends in pinned host memory.
+        h2d = int(sum(i["h2d_bytes"] for i in infos))
+        d2h = int(sum(i["d2h_bytes"] for i in infos))
+        result["e2e"] = {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps,
+                         "path": "cqsa_forward(CQSA_HOST), the timed path itself"}
+        result["streaming"] = streaming_report(W, infos, flops_step, ms / args.steps, peaks,
+                                               free_before, torch)
+    elif not args.no_e2e:
         result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream)
 
     # ---- oracle on the host cores (rank 0, N = 1 only).
     if D.rank == 0 and D.world == 1 and not args.no_cpu:
-        result["cpu_baseline"] = cpu_baseline(W, q, k, v, args.cpu_rows)
+        # About 10-20 s of fp64 work on the host cores, whatever the workload.
+        rows = args.cpu_rows or max(8, min(512, int(2.5e11 / (W["H"] * W["N"] * 4 * W["d"]))))
+        result["cpu_baseline"] = cpu_baseline(W, q, k, v, rows)
 
     if D.rank == 0:
         print(json.dumps(result), flush=True)
@@ -401,6 +412,51 @@ def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream):
             "d2h_bytes_per_step": int(sum(i["d2h_bytes"] for i in infos)),
             "steps": steps, "ms_per_step": ms / steps,
             "path": "cqsa_forward(CQSA_HOST): pinned host q,k,v -> streamed tasks -> pinned host out,lse"}
+
+
+def host_link_gbs(torch, nbytes=1 << 30):
+    """Pinned host <-> device copy bandwidth (GB/s), 1 GiB each way, best of 3."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name, dst, src in (("h2d", d, h), ("d2h", h, d)):
+        best = None
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            dst.copy_(src, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1)
+            best = t if best is None else min(best, t)
+        out[name] = nbytes / (best * 1e-3) / 1e9
+    del h, d
+    torch.cuda.empty_cache()
+    return out
+
+
+def streaming_report(W, infos, flops_step, ms_step, peaks, free_before, torch):
+    """Streamed workloads: time bound = the slowest of compute at the bf16
+    peak and each direction of the host link at its measured bandwidth;
+    efficiency = bound / measured time; device memory against the budget."""
+    free_after, _ = torch.cuda.mem_get_info()
+    link = host_link_gbs(torch)
+    h2d = sum(i["h2d_bytes"] for i in infos)
+    d2h = sum(i["d2h_bytes"] for i in infos)
+    t_compute = flops_step / (peaks["bf16_tflops"] * 1e12) * 1e3
+    t_h2d = h2d / (link["h2d"] * 1e9) * 1e3
+    t_d2h = d2h / (link["d2h"] * 1e9) * 1e3
+    bound = max(t_compute, t_h2d, t_d2h)
+    which = ("compute" if bound == t_compute else "h2d" if bound == t_h2d else "d2h")
+    min_in = 3 * W["N"] * W["H"] * W["d"] * 2
+    return {"h2d_gbs": link["h2d"], "d2h_gbs": link["d2h"], "h2d_bytes": h2d, "d2h_bytes": d2h,
+            "h2d_bytes_minimum": min_in, "t_compute_at_peak_ms": t_compute, "t_h2d_ms": t_h2d,
+            "t_d2h_ms": t_d2h, "t_bound_ms": bound, "bound": which, "t_wall_ms": ms_step,
+            "efficiency": bound / ms_step,
+            "budget_gib": W["budget"] / GiB,
+            "library_arena_gib": max(i["host_arena_bytes"] for i in infos) / GiB,
+            "device_free_delta_gib": (free_before - free_after) / GiB,
+            "head_group": infos[0]["head_group"], "tasks": infos[0]["num_tasks"]}
 
 
 def oracle_sample(W, q, k, v, rows_per_variant, seed):
@@ -474,7 +530,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--cpu-rows", type=int, default=512, help="oracle rows per variant for cpu_baseline")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="oracle rows per variant for cpu_baseline (0: sized to about 15 s)")
     ap.add_argument("--ref-rows", type=int, default=16, help="oracle rows per variant per reference step")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
