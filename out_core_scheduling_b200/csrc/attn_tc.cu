@@ -70,27 +70,35 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                  : "memory");
 }
 
-// 2^x on the FMA pipe: Cody-Waite split x = j + f (j = round(x) taken from
-// the low mantissa bits of x + 1.5 * 2^23), 2^f by the degree-3 minimax
-// polynomial of exp2_poly.h, and 2^j added to the exponent field.  Inputs
-// are clamped at -125 so the exponent never wraps (2^-125 is zero for the
-// softmax); masked -inf scores therefore give a negligible positive value.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.f);
-    const float y = x + 12582912.f;
-    const float f = x - (y - 12582912.f);
-    float p = fmaf(CQSA_EXP2_C3, f, CQSA_EXP2_C2);
-    p = fmaf(p, f, CQSA_EXP2_C1);
-    p = fmaf(p, f, CQSA_EXP2_C0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+// 2^x for a pair of arguments on the FMA and ALU pipes (Cody-Waite split
+// x = j + f with j = floor(x)): adding 1.5 * 2^23 with round-down leaves j in
+// the low mantissa bits, f = x - j lies in [0, 1), 2^f comes from the
+// degree-3 minimax polynomial of exp2_poly.h by packed Horner steps, and j
+// is added to the exponent field.  Arguments are clamped at -126 so the
+// exponent never wraps (2^-126 is zero for the softmax), which also maps the
+// -inf of masked scores to a negligible positive value.
+__device__ __forceinline__ void exp2_emulated_pair(float x0, float x1, float &p0, float &p1) {
+    const uint64_t X = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t MAG = f2_pack(12582912.f, 12582912.f);
+    uint64_t Y, YB, F;
+    asm("add.rm.ftz.f32x2 %0, %1, %2;" : "=l"(Y) : "l"(X), "l"(MAG));
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(YB) : "l"(Y), "l"(MAG));
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(F) : "l"(X), "l"(YB));
+    uint64_t P = f2_fma(f2_pack(CQSA_EXP2_C3, CQSA_EXP2_C3), F, f2_pack(CQSA_EXP2_C2, CQSA_EXP2_C2));
+    P = f2_fma(P, F, f2_pack(CQSA_EXP2_C1, CQSA_EXP2_C1));
+    P = f2_fma(P, F, f2_pack(CQSA_EXP2_C0, CQSA_EXP2_C0));
+    float y0, y1, q0, q1;
+    f2_unpack(Y, y0, y1);
+    f2_unpack(P, q0, q1);
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(y0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(y1) << 23));
 }
 
-// Which column pairs of a 128-wide score row take the polynomial instead of
-// the MUFU ex2: POLY_PAIRS_PER_8 of every 8 pairs.  Measured on B200 the
-// softmax is issue- and latency-bound rather than MUFU-bound, where the
-// polynomial's extra instructions cost more than they save, so it is off.
-constexpr int POLY_PAIRS_PER_8 = 0;
-__device__ __forceinline__ constexpr bool poly_pair(int pair) { return (pair & 7) >= 8 - POLY_PAIRS_PER_8; }
+// Which column pairs of a 128-wide score row use the emulated exponential
+// instead of the MUFU ex2: EMU_PAIRS_PER_8 of every 8 (measured on B200:
+// one in eight balances the MUFU against the FMA/ALU pipes best).
+constexpr int EMU_PAIRS_PER_8 = 1;
+__device__ __forceinline__ constexpr bool emu_pair(int pair) { return (pair & 7) >= 8 - EMU_PAIRS_PER_8; }
 
 // Warp-uniform bounded wait: every lane polls, then the warp agrees.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -327,13 +335,17 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 // 128-deep dependency).
                 float mx;
                 {
-                    float m8[8];
+                    float m4[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) m8[c] = sv[c];
-#pragma unroll
-                    for (int c = 8; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
-                    mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                    for (int c = 4; c + 8 <= BN; c += 8) {
+                        m4[0] = fmax3(m4[0], sv[c], sv[c + 1]);
+                        m4[1] = fmax3(m4[1], sv[c + 2], sv[c + 3]);
+                        m4[2] = fmax3(m4[2], sv[c + 4], sv[c + 5]);
+                        m4[3] = fmax3(m4[3], sv[c + 6], sv[c + 7]);
+                    }
+                    m4[0] = fmax3(m4[0], sv[BN - 4], sv[BN - 3]);
+                    m4[1] = fmax3(m4[1], sv[BN - 2], sv[BN - 1]);
+                    mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
                 }
                 const float xm = mx * sl2;
                 // Online softmax with a lazy rescale: the running max only
@@ -344,29 +356,37 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 l_run *= alpha;
                 m_run = m_new;
                 const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-                float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // Scale and shift two scores per instruction, exponentiate
+                // (MUFU ex2, or the emulation for some pairs), accumulate the
+                // row sum two lanes at a time and write P as bf16 pairs.
+                const uint64_t SL2 = f2_pack(sl2, sl2), NMU = f2_pack(-mu, -mu);
+                uint64_t s4[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int pair = half * 32 + i;
-                        const float x0 = fmaf(sv[2 * pair], sl2, -mu);
-                        const float x1 = fmaf(sv[2 * pair + 1], sl2, -mu);
-                        float p0, p1;
-                        if (poly_pair(pair)) {
-                            p0 = exp2_poly(x0);
-                            p1 = exp2_poly(x1);
+                        float x0, x1, p0, p1;
+                        f2_unpack(f2_fma(f2_pack(sv[2 * pair], sv[2 * pair + 1]), SL2, NMU), x0, x1);
+                        if (emu_pair(pair)) {
+                            exp2_emulated_pair(x0, x1, p0, p1);
                         } else {
                             p0 = ex2_approx(x0);
                             p1 = ex2_approx(x1);
                         }
-                        s8[i & 7] += p0 + p1;
+                        s4[i & 3] = f2_add(s4[i & 3], f2_pack(p0, p1));
                         pk[i] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(s_addr + (uint32_t)(half * 32), pk);
                 }
-                const float sum = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+                float sum;
+                {
+                    float a0, a1, b0, b1;
+                    f2_unpack(f2_add(s4[0], s4[1]), a0, a1);
+                    f2_unpack(f2_add(s4[2], s4[3]), b0, b1);
+                    sum = (a0 + a1) + (b0 + b1);
+                }
                 // O correction after P is out of registers (lower pressure);
                 // PV_t(j) waits for p_full, so it sees the corrected O.
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {

@@ -17,10 +17,13 @@ def coeffs():
 
 
 def exp2_poly_f32(x):
+    """The kernel's steps: clamp at -126, y = x + 1.5*2^23 rounded down (the
+    low mantissa bits hold floor(x)), f = x - (y - 1.5*2^23) in [0, 1), the
+    polynomial by Horner in fp32, then floor(x) added to the exponent field."""
     c0, c1, c2, c3 = coeffs()
     f32 = np.float32
-    x = np.maximum(x.astype(f32), f32(-125.0))
-    y = (x + f32(12582912.0)).astype(f32)
+    x = np.maximum(x.astype(f32), f32(-126.0))
+    y = (f32(12582912.0) + np.floor(x)).astype(f32)      # exact: an integer below 2^24
     f = (x - (y - f32(12582912.0)).astype(f32)).astype(f32)
     p = (c3 * f + c2).astype(f32)
     p = (p * f + c1).astype(f32)
@@ -40,7 +43,7 @@ def test_relative_error_over_softmax_range():
 
 
 def test_masked_and_tiny_arguments_are_negligible():
-    x = np.float32([-np.inf, -1e30, -200.0, -125.0, -126.0])
+    x = np.float32([-np.inf, -1e30, -200.0, -127.0, -126.0, -125.5])
     got = exp2_poly_f32(x)
     assert np.all(got >= 0) and np.all(got < 1e-37)
 
