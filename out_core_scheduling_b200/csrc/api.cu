@@ -135,7 +135,6 @@ struct LeafState {
     DevWl wl;
     MergeSeg *segs = nullptr;
     std::vector<MergeSeg> host_segs;
-    std::vector<char> need_q, need_kv;
 };
 
 }  // namespace
@@ -162,11 +161,12 @@ struct cqsa_plan {
     int g = 0;
     int *h_err = nullptr;
     float *acc_o = nullptr, *acc_lse = nullptr;
-    char *in_q[2] = {}, *in_k[2] = {}, *in_v[2] = {}, *out_st[2] = {};
+    char *pool_q = nullptr, *pool_k = nullptr, *pool_v = nullptr;  // block caches
+    char *out_st[2] = {};
     float *lse_st[2] = {};
     float *h_part_o = nullptr, *h_part_lse = nullptr;
     std::vector<LeafState> leaves;
-    CUtensorMap mq[2], mk[2], mv[2];
+    CUtensorMap mq, mk, mv;  // over the block pools
     cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
     cudaEvent_t ev_in_ready[2] = {}, ev_in_free[2] = {}, ev_merged[2] = {}, ev_out_free[2] = {};
     cudaEvent_t ev_start = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
@@ -274,15 +274,18 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
                     pl.spec.budget);
     const int64_t N = pl.spec.N, R = pl.max_task_rows;
     const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
+    const size_t blk = (size_t)pl.block * g * dd * e;
+    const PoolPlan &pp = pl.pool;
+    // Same layout steps as Planner::host_arena_bytes.
     ArenaLayout a;
     const size_t o_err = a.take(256);
     const size_t o_acc = a.take((size_t)N * g * dd * sizeof(float));
     const size_t o_accl = a.take((size_t)g * N * sizeof(float));
-    size_t o_q[2], o_k[2], o_v[2], o_out[2], o_lse[2];
+    const size_t o_pq = a.take((size_t)pp.q_slots * blk);
+    const size_t o_pk = a.take((size_t)pp.kv_slots * blk);
+    const size_t o_pv = a.take((size_t)pp.kv_slots * blk);
+    size_t o_out[2], o_lse[2];
     for (int s = 0; s < 2; ++s) {
-        o_q[s] = a.take((size_t)R * g * dd * e);
-        o_k[s] = a.take((size_t)R * g * dd * e);
-        o_v[s] = a.take((size_t)R * g * dd * e);
         o_out[s] = a.take((size_t)R * g * dd * e);
         o_lse[s] = a.take((size_t)g * R * sizeof(float));
     }
@@ -292,11 +295,10 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     std::vector<size_t> o_wl(pl.leaves.size()), o_seg(pl.leaves.size());
     P->leaves.assign(pl.leaves.size(), LeafState());
     for (size_t t = 0; t < pl.leaves.size(); ++t) {
-        wls[t] = pl.leaf_worklist((int64_t)t, unit_rows_for(P->elem), key_tile_for(P->elem), g);
+        wls[t] = pl.leaf_worklist((int64_t)t, pp, unit_rows_for(P->elem), key_tile_for(P->elem), g);
         o_wl[t] = a.take(wl_region(wls[t]));
         P->leaves[t].host_segs = pl.leaf_merge_segments((int64_t)t);
         o_seg[t] = a.take(P->leaves[t].host_segs.size() * sizeof(MergeSeg));
-        pl.leaf_needs((int64_t)t, &P->leaves[t].need_q, &P->leaves[t].need_kv);
     }
     if (a.total != pl.sizing.host_arena)
         return fail(CQSA_ERR_CUDA, "internal: host-mode arena layout mismatch (%zu vs %zu)", a.total,
@@ -306,15 +308,15 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     P->host_arena = arena;
     P->host_bytes = a.total;
     P->g = g;
-    // Zeroed once, so rows a partial key tile reads past its run are finite.
+    // Zeroed once, so rows a partial key tile reads past its block are finite.
     CK(cudaMemset(arena, 0, a.total));
     P->h_err = reinterpret_cast<int *>(arena + o_err);
     P->acc_o = reinterpret_cast<float *>(arena + o_acc);
     P->acc_lse = reinterpret_cast<float *>(arena + o_accl);
+    P->pool_q = arena + o_pq;
+    P->pool_k = arena + o_pk;
+    P->pool_v = arena + o_pv;
     for (int s = 0; s < 2; ++s) {
-        P->in_q[s] = arena + o_q[s];
-        P->in_k[s] = arena + o_k[s];
-        P->in_v[s] = arena + o_v[s];
         P->out_st[s] = arena + o_out[s];
         P->lse_st[s] = reinterpret_cast<float *>(arena + o_lse[s]);
     }
@@ -330,12 +332,10 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
             CK(cudaMemcpy(P->leaves[t].segs, hs.data(), hs.size() * sizeof(MergeSeg), cudaMemcpyHostToDevice));
     }
     if (P->dtype == CQSA_BF16) {
-        for (int s = 0; s < 2; ++s) {
-            cqsa_status_t st;
-            if ((st = make_map(&P->mq[s], P->in_q[s], R, g, pl.spec.d)) != CQSA_OK) return st;
-            if ((st = make_map(&P->mk[s], P->in_k[s], R, g, pl.spec.d)) != CQSA_OK) return st;
-            if ((st = make_map(&P->mv[s], P->in_v[s], R, g, pl.spec.d)) != CQSA_OK) return st;
-        }
+        cqsa_status_t st;
+        if ((st = make_map(&P->mq, P->pool_q, pp.q_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mk, P->pool_k, pp.kv_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mv, P->pool_v, pp.kv_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
     }
     CK(cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
@@ -442,31 +442,33 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     CK(cudaStreamWaitEvent(P->s_comp, P->ev_start, 0));
     CK(cudaStreamWaitEvent(P->s_out, P->ev_start, 0));
     int64_t it = 0;
+    const size_t blk_rows = (size_t)B;
     for (int h0 = 0; h0 < H; h0 += g) {
         for (size_t t = 0; t < P->leaves.size(); ++t, ++it) {
             const LeafState &L = P->leaves[t];
-            const Leaf &leaf = pl.leaves[t];
             const int s = (int)(it & 1);
-            // -- H2D of the task's blocks (runs of consecutive needed members).
+            // -- H2D of the blocks this task misses in the device block cache.
+            // The cache plan never evicts a block of the previous task, so a
+            // copy only waits for the kernel two tasks back; at a head-group
+            // boundary every slot changes meaning, so it also waits for the
+            // previous task's kernel.
             if (it >= 2) CK(cudaStreamWaitEvent(P->s_in, P->ev_in_free[s], 0));
-            const char *srcs[3] = {hq, hk, hv};
-            char *dsts[3] = {P->in_q[s], P->in_k[s], P->in_v[s]};
-            for (int x = 0; x < 3; ++x) {
-                const std::vector<char> &need = (x == 0) ? L.need_q : L.need_kv;
-                size_t m = 0;
-                while (m < need.size()) {
-                    if (!need[m]) { ++m; continue; }
-                    size_t m1 = m;
-                    while (m1 + 1 < need.size() && need[m1 + 1] && leaf.blocks[m1 + 1] == leaf.blocks[m1] + 1) ++m1;
-                    const size_t rows = (m1 - m + 1) * (size_t)B;
-                    char *dst = dsts[x] + (size_t)m * B * grp_row;
-                    const char *src = srcs[x] + ((size_t)leaf.blocks[m] * B * H + h0) * d * e;
-                    CK(copy_rows(dst, grp_row, src, full_row, grp_row, rows, cudaMemcpyHostToDevice, P->s_in));
-                    m = m1 + 1;
+            if (t == 0 && it >= 1) CK(cudaStreamWaitEvent(P->s_in, P->ev_in_free[1 - s], 0));
+            for (const PoolCopy &c : pl.pool.copies[t]) {
+                const size_t src_off = ((size_t)c.block * B * H + h0) * d * e;
+                const size_t dst_off = (size_t)c.slot * blk_rows * grp_row;
+                if (c.kind == 0) {
+                    CK(copy_rows(P->pool_q + dst_off, grp_row, hq + src_off, full_row, grp_row, blk_rows,
+                                 cudaMemcpyHostToDevice, P->s_in));
+                } else {
+                    CK(copy_rows(P->pool_k + dst_off, grp_row, hk + src_off, full_row, grp_row, blk_rows,
+                                 cudaMemcpyHostToDevice, P->s_in));
+                    CK(copy_rows(P->pool_v + dst_off, grp_row, hv + src_off, full_row, grp_row, blk_rows,
+                                 cudaMemcpyHostToDevice, P->s_in));
                 }
             }
             CK(cudaEventRecord(P->ev_in_ready[s], P->s_in));
-            // -- tile attention on the staged task.
+            // -- tile attention on the task's cached blocks.
             CK(cudaStreamWaitEvent(P->s_comp, P->ev_in_ready[s], 0));
             AttnParams ap = base_params(P, P->h_err);
             ap.entries = L.wl.entries;
@@ -479,9 +481,9 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
             {
                 LaunchTimer tm(P, P->s_comp, 0);
                 if (P->dtype == CQSA_BF16)
-                    CK(launch_attn_tc(d, P->mq[s], P->mk[s], P->mv[s], ap, L.wl.num_units, P->s_comp));
+                    CK(launch_attn_tc(d, P->mq, P->mk, P->mv, ap, L.wl.num_units, P->s_comp));
                 else
-                    CK(launch_attn_simt(d, P->elem, P->in_q[s], P->in_k[s], P->in_v[s], ap, L.wl.num_units,
+                    CK(launch_attn_simt(d, P->elem, P->pool_q, P->pool_k, P->pool_v, ap, L.wl.num_units,
                                         P->s_comp));
                 tm.stop();
             }

@@ -148,11 +148,12 @@ __global__ void __launch_bounds__(simt::THREADS)
         const int32_t row = q0 + ty * 4 + i;
         if (row >= q_end) continue;
         const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
-        float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + row) * H + h) * D;
+        const int64_t out_row = (int64_t)e.out_lo + (row - e.q_lo);
+        float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * H + h) * D;
 #pragma unroll
         for (int jj = 0; jj < NJ; ++jj) dst[tx + 16 * jj] = o[i][jj] * inv;
         if (tx == 0)
-            p.part_lse[((int64_t)e.slot * H + h) * p.part_rows + row] =
+            p.part_lse[((int64_t)e.slot * H + h) * p.part_rows + out_row] =
                 (m[i] + log2f(l[i])) * 0.69314718055994531f;
     }
 }

@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             tc_fence_after();
             const bool valid = q_local < e.q_hi;
             const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + q_local) * p.H + head) * D;
+            const int64_t out_row = (int64_t)e.out_lo + (q_local - e.q_lo);
+            float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * p.H + head) * D;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
             if (valid) {
                 const float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-                p.part_lse[((int64_t)e.slot * p.H + head) * p.part_rows + q_local] = lse;
+                p.part_lse[((int64_t)e.slot * p.H + head) * p.part_rows + out_row] = lse;
             }
         } else {
             if (lane == 0) atomicExch(p.err, DEV_TIMEOUT);

@@ -10,7 +10,8 @@ namespace cqsa {
 
 // Parameters shared by both attention kernels.  Partial outputs are laid
 // out [slot][part_rows][H][d] (fp32, normalised by the task's own softmax
-// denominator) and partial lse [slot][H][part_rows] (natural log).
+// denominator) and partial lse [slot][H][part_rows] (natural log); query row
+// q of an entry goes to partial row out_lo + (q - q_lo).
 struct AttnParams {
     const WlEntry *entries;
     const WlRun *runs;

@@ -2,7 +2,9 @@
 #include "planner.h"
 
 #include <algorithm>
+#include <map>
 #include <numeric>
+#include <unordered_map>
 
 namespace cqsa {
 
@@ -216,6 +218,7 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
         w.q_hi = (int32_t)((e.qb + 1) * block);
         w.q_goff = 0;
         w.slot = (int32_t)e.slot;
+        w.out_lo = w.q_lo;
         w.run_begin = (int32_t)wl.runs.size();
         w.run_count = (int32_t)e.runs.size();
         for (const KeyRun &r : e.runs) {
@@ -231,24 +234,37 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     return wl;
 }
 
-WorkList Planner::leaf_worklist(int64_t t, int rows_per_unit, int bn, int heads) const {
+WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const {
+    // Q rows come from Q slot q_slot * block, K and V rows from KV slot
+    // kv_slot * block; partial outputs go to the task's local rows mq * block.
     WorkList wl;
     for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
         const Entry &e = entries[i];
+        const int64_t qs = pool.q_slot[t][e.mq];
         WlEntry w{};
-        w.q_lo = (int32_t)(e.mq * block);
-        w.q_hi = (int32_t)((e.mq + 1) * block);
-        w.q_goff = (int32_t)((e.qb - e.mq) * block);
+        w.q_lo = (int32_t)(qs * block);
+        w.q_hi = (int32_t)((qs + 1) * block);
+        w.q_goff = (int32_t)((e.qb - qs) * block);
         w.slot = 0;
+        w.out_lo = (int32_t)(e.mq * block);
         w.run_begin = (int32_t)wl.runs.size();
-        w.run_count = (int32_t)e.runs.size();
         for (const KeyRun &r : e.runs) {
-            WlRun x{};
-            x.k_lo = (int32_t)(r.m0 * block);
-            x.k_hi = (int32_t)((r.m0 + (r.b1 - r.b0) + 1) * block);
-            x.k_goff = (int32_t)((r.b0 - r.m0) * block);
-            wl.runs.push_back(x);
+            for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
+                const int64_t ks = pool.kv_slot[t][r.m0 + (kb - r.b0)];
+                const int32_t lo = (int32_t)(ks * block), goff = (int32_t)((kb - ks) * block);
+                if ((int32_t)wl.runs.size() > w.run_begin && wl.runs.back().k_hi == lo &&
+                    wl.runs.back().k_goff == goff) {
+                    wl.runs.back().k_hi = lo + (int32_t)block;   // contiguous slots: one run
+                } else {
+                    WlRun x{};
+                    x.k_lo = lo;
+                    x.k_hi = lo + (int32_t)block;
+                    x.k_goff = goff;
+                    wl.runs.push_back(x);
+                }
+            }
         }
+        w.run_count = (int32_t)wl.runs.size() - w.run_begin;
         wl.entries.push_back(w);
     }
     add_units(&wl, heads, rows_per_unit, bn, spec.causal);
@@ -282,6 +298,110 @@ void Planner::leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char>
 }
 
 // ---------------------------------------------------------------------------
+// Block cache of the streamed path (Belady; see planner.h).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Blocks each leaf task needs as Q and as K/V, in member order.
+void task_needs(const Planner &pl, std::vector<std::vector<int64_t>> *nq, std::vector<std::vector<int64_t>> *nkv) {
+    const size_t T = pl.leaves.size();
+    nq->assign(T, {});
+    nkv->assign(T, {});
+    std::vector<char> q, kv;
+    for (size_t t = 0; t < T; ++t) {
+        pl.leaf_needs((int64_t)t, &q, &kv);
+        for (size_t m = 0; m < q.size(); ++m) {
+            if (q[m]) (*nq)[t].push_back(pl.leaves[t].blocks[m]);
+            if (kv[m]) (*nkv)[t].push_back(pl.leaves[t].blocks[m]);
+        }
+    }
+}
+
+// One cache of `cap` slots over the task sequence; fills slot_of[t][block]
+// and the copies.  False when a task and its predecessor need more than cap.
+bool simulate(const std::vector<std::vector<int64_t>> &need, int64_t cap, int kind,
+              std::vector<std::unordered_map<int64_t, int32_t>> *slot_of, std::vector<std::vector<PoolCopy>> *copies,
+              int64_t *ncopies) {
+    const size_t T = need.size();
+    std::map<int64_t, std::vector<int64_t>> uses;  // block -> tasks using it, increasing
+    for (size_t t = 0; t < T; ++t)
+        for (int64_t b : need[t]) uses[b].push_back((int64_t)t);
+    auto next_use = [&](int64_t b, int64_t t) -> int64_t {
+        const std::vector<int64_t> &u = uses[b];
+        auto it = std::upper_bound(u.begin(), u.end(), t);
+        return it == u.end() ? INT64_MAX : *it;
+    };
+    std::vector<int64_t> slot_block(cap, -1);
+    std::unordered_map<int64_t, int32_t> where;
+    slot_of->assign(T, {});
+    for (size_t t = 0; t < T; ++t) {
+        std::vector<int64_t> protect = need[t];
+        if (t > 0) protect.insert(protect.end(), need[t - 1].begin(), need[t - 1].end());
+        std::sort(protect.begin(), protect.end());
+        for (int64_t b : need[t]) {
+            auto hit = where.find(b);
+            if (hit == where.end()) {
+                int32_t slot = -1;
+                for (int64_t sl = 0; sl < cap; ++sl)
+                    if (slot_block[sl] < 0) { slot = (int32_t)sl; break; }
+                if (slot < 0) {
+                    int64_t best = -1;
+                    for (int64_t sl = 0; sl < cap; ++sl) {
+                        const int64_t ob = slot_block[sl];
+                        if (std::binary_search(protect.begin(), protect.end(), ob)) continue;
+                        const int64_t nu = next_use(ob, (int64_t)t);
+                        if (nu > best) { best = nu; slot = (int32_t)sl; }
+                    }
+                    if (slot < 0) return false;
+                    where.erase(slot_block[slot]);
+                }
+                slot_block[slot] = b;
+                where[b] = slot;
+                (*copies)[t].push_back(PoolCopy{kind, b, slot});
+                ++*ncopies;
+                hit = where.find(b);
+            }
+            (*slot_of)[t][b] = hit->second;
+        }
+    }
+    return true;
+}
+
+}  // namespace
+
+bool Planner::plan_pool(int64_t q_slots, int64_t kv_slots, PoolPlan *out) const {
+    std::vector<std::vector<int64_t>> nq, nkv;
+    task_needs(*this, &nq, &nkv);
+    PoolPlan pp;
+    pp.q_slots = q_slots;
+    pp.kv_slots = kv_slots;
+    const size_t T = leaves.size();
+    pp.copies.assign(T, {});
+    std::vector<std::unordered_map<int64_t, int32_t>> sq, skv;
+    if (!simulate(nq, q_slots, 0, &sq, &pp.copies, &pp.q_copies)) return false;
+    // K/V copies after the task's Q copies (one list per task).
+    std::vector<std::vector<PoolCopy>> kvc(T);
+    if (!simulate(nkv, kv_slots, 1, &skv, &kvc, &pp.kv_copies)) return false;
+    pp.q_slot.assign(T, {});
+    pp.kv_slot.assign(T, {});
+    for (size_t t = 0; t < T; ++t) {
+        pp.copies[t].insert(pp.copies[t].end(), kvc[t].begin(), kvc[t].end());
+        const size_t n = leaves[t].blocks.size();
+        pp.q_slot[t].assign(n, -1);
+        pp.kv_slot[t].assign(n, -1);
+        for (size_t m = 0; m < n; ++m) {
+            const int64_t b = leaves[t].blocks[m];
+            auto a = sq[t].find(b);
+            if (a != sq[t].end()) pp.q_slot[t][m] = a->second;
+            auto k = skv[t].find(b);
+            if (k != skv[t].end()) pp.kv_slot[t][m] = k->second;
+        }
+    }
+    *out = std::move(pp);
+    return true;
+}
+
+// ---------------------------------------------------------------------------
 // Memory sizing (layerthelatestinalattice.com summary: subproblems fit a
 // stated memory budget).  Every byte the library holds on the device lives
 // in one arena whose layout the runtime rebuilds with the same ArenaLayout
@@ -307,22 +427,25 @@ size_t Planner::device_arena_bytes() const {
     return a.total;
 }
 
-size_t Planner::host_arena_bytes(int g) const {
+size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
     const int64_t N = spec.N, R = max_task_rows;
     const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
+    const size_t blk = (size_t)block * g * dd * e;
     ArenaLayout a;
     a.take(256);                                        // error word
     a.take((size_t)N * g * dd * sizeof(float));         // accumulator O
     a.take((size_t)g * N * sizeof(float));              // accumulator lse
+    a.take((size_t)pl.q_slots * blk);                   // Q block pool
+    a.take((size_t)pl.kv_slots * blk);                  // K block pool
+    a.take((size_t)pl.kv_slots * blk);                  // V block pool
     for (int s = 0; s < 2; ++s) {
-        for (int x = 0; x < 3; ++x) a.take((size_t)R * g * dd * e);   // staged q, k, v
         a.take((size_t)R * g * dd * e);                 // finished out rows
         a.take((size_t)g * R * sizeof(float));          // finished lse rows
     }
     a.take((size_t)R * g * dd * sizeof(float));         // task partial O
     a.take((size_t)g * R * sizeof(float));              // task partial lse
     for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
-        WorkList wl = leaf_worklist(t, unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
+        WorkList wl = leaf_worklist(t, pl, unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
         a.take(wl_bytes(wl));
         a.take(leaf_merge_segments(t).size() * sizeof(MergeSeg));
     }
@@ -332,25 +455,60 @@ size_t Planner::host_arena_bytes(int g) const {
 void Planner::size_plan() {
     sizing = Sizing{};
     sizing.device_arena = device_arena_bytes();
+    // Smallest and largest useful pools (a task and its predecessor must fit).
+    std::vector<std::vector<int64_t>> nq, nkv;
+    task_needs(*this, &nq, &nkv);
+    auto span = [](const std::vector<std::vector<int64_t>> &need, int64_t *mn, int64_t *full) {
+        std::vector<int64_t> all;
+        *mn = 0;
+        for (size_t t = 0; t < need.size(); ++t) {
+            std::vector<int64_t> u = need[t];
+            if (t > 0) u.insert(u.end(), need[t - 1].begin(), need[t - 1].end());
+            std::sort(u.begin(), u.end());
+            u.erase(std::unique(u.begin(), u.end()), u.end());
+            *mn = std::max<int64_t>(*mn, (int64_t)u.size());
+            all.insert(all.end(), need[t].begin(), need[t].end());
+        }
+        std::sort(all.begin(), all.end());
+        all.erase(std::unique(all.begin(), all.end()), all.end());
+        *full = (int64_t)all.size();
+    };
+    span(nq, &min_q_slots, &full_q_slots);
+    span(nkv, &min_kv_slots, &full_kv_slots);
+
     for (int g = spec.H; g >= 1; --g) {
         if (spec.H % g) continue;
-        const size_t b = host_arena_bytes(g);
-        if (spec.budget == 0 || b <= spec.budget) {
-            sizing.head_group = g;
-            sizing.host_arena = b;
-            break;
+        const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
+        int64_t qs = full_q_slots, kvs = full_kv_slots;
+        PoolPlan pp;
+        if (!plan_pool(qs, kvs, &pp)) continue;
+        size_t bytes = host_arena_bytes(g, pp);
+        if (spec.budget) {
+            // Shrink the pools (K/V first, they take two blocks per slot)
+            // until the arena fits, never below what a task pair needs.
+            while (bytes > spec.budget && (qs > min_q_slots || kvs > min_kv_slots)) {
+                const size_t over = bytes - spec.budget;
+                int64_t drop_kv = std::min<int64_t>(kvs - min_kv_slots, (int64_t)((over + 2 * blk - 1) / (2 * blk)));
+                int64_t drop_q = 0;
+                if (drop_kv <= 0) drop_q = std::min<int64_t>(qs - min_q_slots, (int64_t)((over + blk - 1) / blk));
+                if (drop_kv <= 0 && drop_q <= 0) break;
+                kvs -= std::max<int64_t>(drop_kv, 0);
+                qs -= std::max<int64_t>(drop_q, 0);
+                if (!plan_pool(qs, kvs, &pp)) { bytes = SIZE_MAX; break; }
+                bytes = host_arena_bytes(g, pp);
+            }
+            if (bytes > spec.budget) continue;
         }
+        sizing.head_group = g;
+        sizing.host_arena = bytes;
+        sizing.q_slots = qs;
+        sizing.kv_slots = kvs;
+        const size_t groups = (size_t)(spec.H / g);
+        sizing.h2d = ((size_t)pp.q_copies + 2 * (size_t)pp.kv_copies) * blk * groups;
+        pool = std::move(pp);
+        break;
     }
-    const size_t row_bytes = (size_t)spec.H * spec.d * spec.elem_bytes;
-    size_t h2d = 0;
-    std::vector<char> nq, nkv;
-    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
-        leaf_needs(t, &nq, &nkv);
-        for (size_t m = 0; m < nq.size(); ++m)
-            h2d += (size_t)(nq[m] + 2 * nkv[m]) * block * row_bytes;
-    }
-    sizing.h2d = h2d;
-    sizing.d2h = (size_t)spec.N * row_bytes + (size_t)spec.H * spec.N * sizeof(float);
+    sizing.d2h = (size_t)spec.N * spec.H * spec.d * spec.elem_bytes + (size_t)spec.H * spec.N * sizeof(float);
 }
 
 }  // namespace cqsa

@@ -63,11 +63,32 @@ struct PlanSpec {
     size_t budget = 0;                      // 0 = unlimited
 };
 
+// Device block cache of the streamed path.  A Q slot holds one query block
+// of the current head group ([block, g, d]); a KV slot holds its K and V
+// blocks (same slot index in the K pool and the V pool, so one key
+// coordinate addresses both).  The task order is fixed, so the cache is
+// simulated at plan time with Belady's rule (evict the block whose next use
+// is farthest away); blocks of the current and the previous task are never
+// evicted, because the previous task's kernel may still be reading them.
+struct PoolCopy {
+    int32_t kind;     // 0: Q block, 1: K and V blocks
+    int64_t block;    // global block
+    int32_t slot;
+};
+
+struct PoolPlan {
+    int64_t q_slots = 0, kv_slots = 0;
+    std::vector<std::vector<PoolCopy>> copies;          // per leaf task, in copy order
+    std::vector<std::vector<int32_t>> q_slot, kv_slot;  // per leaf task, per member; -1: unused
+    int64_t q_copies = 0, kv_copies = 0;                // per head group
+};
+
 struct Sizing {
     int head_group = 0;
     size_t host_arena = 0;
     size_t device_arena = 0;
     size_t h2d = 0, d2h = 0;
+    int64_t q_slots = 0, kv_slots = 0;
 };
 
 class Planner {
@@ -88,15 +109,22 @@ public:
 
     // rows_per_unit: query rows one CTA covers; bn: key tile width.
     WorkList device_worklist(int rows_per_unit, int bn, int heads) const;
-    WorkList leaf_worklist(int64_t t, int rows_per_unit, int bn, int heads) const;
+    // Work list of leaf t reading Q, K, V from the block pools of `pool`.
+    WorkList leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const;
     // Merge segments of leaf t in host mode (one per query block with an
     // entry), with first/last-touch flags in leaf order.
     std::vector<MergeSeg> leaf_merge_segments(int64_t t) const;
     // Members of leaf t whose Q (resp. K/V) rows a streamed task needs.
     void leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char> *need_kv) const;
 
+    // Simulate the block cache with the given capacities; false if some
+    // task (with its predecessor) needs more slots than there are.
+    bool plan_pool(int64_t q_slots, int64_t kv_slots, PoolPlan *out) const;
+    PoolPlan pool;                  // cache plan of the chosen sizing
+    int64_t min_q_slots = 0, min_kv_slots = 0, full_q_slots = 0, full_kv_slots = 0;
+
     // Arena bytes of each mode for a head group g (host) / all heads (device).
-    size_t host_arena_bytes(int g) const;
+    size_t host_arena_bytes(int g, const PoolPlan &pool) const;
     size_t device_arena_bytes() const;
 
 private:

@@ -27,7 +27,8 @@ struct WlEntry {
     int32_t slot;         // partial index (device mode); 0 in host mode
     int32_t run_begin;    // first WlRun of this entry
     int32_t run_count;    // number of runs (>= 1)
-    int32_t pad0, pad1;
+    int32_t out_lo;       // partial-output row of query row q_lo
+    int32_t pad;
 };
 
 struct WlRun {

@@ -125,20 +125,51 @@ def test_configs_plan():
     assert i5["D"] == [[0, 1, 3, 8, 12, 18]]
 
 
-def test_h2d_bytes_count_needed_blocks():
-    """Non-causal: every block is a query and key block of each of its l
-    tasks, so the streamed path moves each of Q, K, V l times."""
-    p = cqsa.cqsa_plan(13 * 256, 2, 128, 4, 1, False, 0)
+def test_h2d_bytes_with_block_cache():
+    """Unlimited budget: the device block cache holds every block, so each
+    of Q, K, V crosses the host link once.  A tight budget forces evictions:
+    more traffic, but never more than one copy of every block per task."""
+    N, H, d = 13 * 256, 2, 128
+    once = 3 * N * H * d * 2
+    p = cqsa.cqsa_plan(N, H, d, 4, 1, False, 0)
     i = p.info()
-    assert i["h2d_bytes"] == 4 * 3 * 13 * 256 * 2 * 128 * 2
-    assert i["d2h_bytes"] == 13 * 256 * 2 * 128 * 2 + 2 * 13 * 256 * 4
+    assert i["h2d_bytes"] == once
+    assert i["d2h_bytes"] == N * H * d * 2 + H * N * 4
+    per_task = 4 * once  # every block is in l = 4 tasks
+    tight = cqsa.cqsa_plan(N, H, d, 4, 1, False, int(i["host_arena_bytes"] * 0.55))
+    t = tight.info()
+    assert t["host_arena_bytes"] <= int(i["host_arena_bytes"] * 0.55)
+    assert once <= t["h2d_bytes"] <= per_task
+
+
+@pytest.mark.parametrize("budget_frac", [1.0, 0.6, 0.45])
+def test_streamed_budgets_hold(budget_frac):
+    GiB = 1 << 30
+    full = cqsa.cqsa_plan_ex(91 * 256, 4, 128, [4, 3], causal=True).info()["host_arena_bytes"]
+    budget = int(full * budget_frac)
+    try:
+        p = cqsa.cqsa_plan_ex(91 * 256, 4, 128, [4, 3], causal=True, mem_budget_bytes=budget)
+    except cqsa.CqsaError as e:
+        assert e.status == cqsa.CQSA_ERR_BUDGET
+        return
+    assert p.info()["host_arena_bytes"] <= budget
 
 
 def test_auto_levels_recurse_until_it_fits():
-    GiB = 1 << 30
-    one = cqsa.cqsa_plan(7 * 7 * 4096, 1, 128, 3, 1, False, 0).info()
-    p = cqsa.cqsa_plan(7 * 7 * 4096, 1, 128, 3, 0, False, one["host_arena_bytes"] - 1)
-    assert p.info()["levels"] == 2
+    """Below the smallest one-level working set, levels = 0 divides again."""
+    N = 7 * 7 * 4096
+    lo, hi = 1 << 20, cqsa.cqsa_plan(N, 1, 128, 3, 1, False, 0).info()["host_arena_bytes"]
+    while hi - lo > (1 << 20):       # smallest budget one level accepts
+        mid = (lo + hi) // 2
+        try:
+            cqsa.cqsa_plan(N, 1, 128, 3, 1, False, mid)
+            hi = mid
+        except cqsa.CqsaError:
+            lo = mid
+    with pytest.raises(cqsa.CqsaError):
+        cqsa.cqsa_plan(N, 1, 128, 3, 1, False, lo)
+    p = cqsa.cqsa_plan(N, 1, 128, 3, 0, False, lo)
+    assert p.info()["levels"] == 2 and p.info()["host_arena_bytes"] <= lo
 
 
 @pytest.mark.parametrize("args,status", [

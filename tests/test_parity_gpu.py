@@ -116,6 +116,33 @@ def test_streamed_two_level(causal):
     check(out, lse, q, k, v, sample_rows(N, 512), causal)
 
 
+def _min_budget(N, H, d, ls, causal):
+    lo, hi = 1 << 20, cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal).info()["host_arena_bytes"]
+    while hi - lo > (1 << 18):
+        mid = (lo + hi) // 2
+        try:
+            cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, mem_budget_bytes=mid)
+            hi = mid
+        except cqsa.CqsaError:
+            lo = mid
+    return hi
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_streamed_block_cache_evicts(causal):
+    """A budget near the smallest the streamed path accepts: the device block
+    cache keeps little more than two tasks' blocks, so blocks are evicted and
+    copied again; the result must not change."""
+    N, H, d = 13 * 256, 1, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=12, host=True)
+    budget = _min_budget(N, H, d, [4], causal)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, mem_budget_bytes=budget)
+    info = plan.info()
+    assert info["h2d_bytes"] > 3 * N * H * d * 2  # some blocks travel twice
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
 def test_streamed_equals_device():
     N, H, d = 13 * 256, 2, 128
     q, k, v = _inputs(N, H, d, torch.bfloat16, seed=9)
