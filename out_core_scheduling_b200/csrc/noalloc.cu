@@ -104,6 +104,7 @@ WlEntry entry_record(const Planner &pl, const Entry &e, int32_t run_begin) {
     w.q_hi = (int32_t)((e.qb + 1) * pl.block);
     w.q_goff = 0;
     w.slot = (int32_t)e.slot;
+    w.out_lo = w.q_lo;
     w.run_begin = run_begin;
     w.run_count = (int32_t)e.runs.size();
     return w;
