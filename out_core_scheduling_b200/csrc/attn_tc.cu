@@ -18,7 +18,11 @@
 // P_t (bf16) is written over the first 64 columns of S_t and fed to the PV
 // MMA straight from tensor memory.  The MMA order per key tile j is
 // PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while one warpgroup does the
-// softmax of its tile, the tensor core works on the other tile.
+// softmax of its tile, the tensor core works on the other tile.  P_t(j) is
+// handed over in two halves of 64 keys, so the first half of PV_t(j) runs
+// while the softmax still computes the second; only half a PV and the next
+// QK separate a tile's last P column from its next S.  The row sum is taken
+// after the hand-off, off that path.
 //
 // Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, drains
 // its own copies and MMAs, frees its tensor memory and returns.
@@ -42,6 +46,7 @@ constexpr int WARP_MMA = 9;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizzle
 constexpr float LOG2_RESCALE_THRESHOLD = 8.0f;
+constexpr int P_HALF_LEAD = 8;  // pairs of the second P half computed before the p_half arrival
 
 template <int D>
 struct Smem {
@@ -51,7 +56,7 @@ struct Smem {
     alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
     uint64_t bar_q;
     uint64_t k_full[STAGES], k_empty[STAGES], v_full[STAGES], v_empty[STAGES];
-    uint64_t s_full[QT], p_full[QT], o_full, drain;
+    uint64_t s_full[QT], p_half[QT], p_full[QT], o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -144,7 +149,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         }
         for (int t = 0; t < QT; ++t) {
             mbar_init(&s.s_full[t], 1);
-            mbar_init(&s.p_full[t], BM / 32);  // one arrival per softmax warp
+            mbar_init(&s.p_half[t], BM / 32);  // one arrival per softmax warp
+            mbar_init(&s.p_full[t], BM / 32);
         }
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
@@ -228,10 +234,11 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     mma_ss_elect(tmem + (uint32_t)t * 128u, qa + off, kb + off, IDESC_QK, kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int t, int st, bool acc) {
+            // O_t += P_t V for the keys [64 h, 64 h + 64) of the tile.
+            auto issue_pv_half = [&](int t, int st, bool acc, int h) {
                 const uint64_t vb = vdesc[st];
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
+                for (int kk = h * BN / 32; kk < (h + 1) * BN / 32; ++kk) {
                     mma_ts_elect(tmem + 256u + (uint32_t)(t * D), tmem + (uint32_t)t * 128u + (uint32_t)kk * 8u,
                                  vb + (uint64_t)(kk * (2048 >> 4)), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                 }
@@ -257,9 +264,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 if (has_next && !warp_wait(&s.k_full[st1], ph1, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
                 for (int t = 0; t < QT; ++t) {
+                    // P_t(j) arrives in two halves of 64 keys: the first half
+                    // of PV_t(j) runs while the softmax finishes the second.
+                    if (!warp_wait(&s.p_half[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                    tc_fence_after();
+                    issue_pv_half(t, st, j > 0, 0);
                     if (!warp_wait(&s.p_full[t], (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
                     tc_fence_after();
-                    issue_pv(t, st, j > 0);
+                    issue_pv_half(t, st, true, 1);
                     if (t == QT - 1) mma_commit_elect(&s.v_empty[st]);
                     if (has_next) {
                         issue_qk(t, st1);
@@ -356,56 +368,75 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 l_run *= alpha;
                 m_run = m_new;
                 const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-                // Scale and shift two scores per instruction, exponentiate
-                // (MUFU ex2, or the emulation for some pairs), accumulate the
-                // row sum two lanes at a time and write P as bf16 pairs.
-                const uint64_t SL2 = f2_pack(sl2, sl2), NMU = f2_pack(-mu, -mu);
-                uint64_t s4[4] = {0, 0, 0, 0};
+                // O correction before any of P_t(j) is handed over: the first
+                // half of PV_t(j) starts at the p_half arrival.  PV_t(j-1) is
+                // done (S_t(j) was committed after it).
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // Eight columns at a time: the scores of the row are live.
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 8; ++cc) {
+                        uint32_t o[8];
+                        tmem_ld8(o_addr + (uint32_t)(cc * 8), o);
+                        tmem_wait_ld();
+                        asm volatile("" : "+r"(o[0]), "+r"(o[1]), "+r"(o[2]), "+r"(o[3]), "+r"(o[4]), "+r"(o[5]),
+                                          "+r"(o[6]), "+r"(o[7]) :: "memory");
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                        for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st8(o_addr + (uint32_t)(cc * 8), o);
+                    }
+                }
+                // Scale and shift two scores per instruction, exponentiate
+                // (MUFU ex2, or the emulation for some pairs), keep the fp32
+                // values for the row sum and write P as bf16 pairs: keys 0..63
+                // to columns 0..31, keys 64..127 to columns 32..63.  The first
+                // half is announced (p_half) once its store has landed, after
+                // a quarter of the second half's exponentials hid the wait.
+                const uint64_t SL2 = f2_pack(sl2, sl2), NMU = f2_pack(-mu, -mu);
+                auto exp_pair = [&](int pair) -> uint32_t {
+                    float x0, x1, p0, p1;
+                    f2_unpack(f2_fma(f2_pack(sv[2 * pair], sv[2 * pair + 1]), SL2, NMU), x0, x1);
+                    if (emu_pair(pair)) {
+                        exp2_emulated_pair(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    sv[2 * pair] = p0;
+                    sv[2 * pair + 1] = p1;
+                    return pack_bf16x2(p0, p1);
+                };
+                {
                     uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int pair = half * 32 + i;
-                        float x0, x1, p0, p1;
-                        f2_unpack(f2_fma(f2_pack(sv[2 * pair], sv[2 * pair + 1]), SL2, NMU), x0, x1);
-                        if (emu_pair(pair)) {
-                            exp2_emulated_pair(x0, x1, p0, p1);
-                        } else {
-                            p0 = ex2_approx(x0);
-                            p1 = ex2_approx(x1);
-                        }
-                        s4[i & 3] = f2_add(s4[i & 3], f2_pack(p0, p1));
-                        pk[i] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st32(s_addr + (uint32_t)(half * 32), pk);
+                    for (int i = 0; i < 32; ++i) pk[i] = exp_pair(i);
+                    tmem_st32(s_addr, pk);
                 }
-                float sum;
                 {
-                    float a0, a1, b0, b1;
-                    f2_unpack(f2_add(s4[0], s4[1]), a0, a1);
-                    f2_unpack(f2_add(s4[2], s4[3]), b0, b1);
-                    sum = (a0 + a1) + (b0 + b1);
-                }
-                // O correction after P is out of registers (lower pressure);
-                // PV_t(j) waits for p_full, so it sees the corrected O.
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
-                        tmem_wait_ld();
-                        reg_fence32(o);
+                    for (int i = 0; i < P_HALF_LEAD; ++i) pk[i] = exp_pair(32 + i);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.p_half[t]);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(o_addr + (uint32_t)(cc * 32), o);
-                    }
+                    for (int i = P_HALF_LEAD; i < 32; ++i) pk[i] = exp_pair(32 + i);
+                    tmem_st32(s_addr + 32u, pk);
                 }
-                l_run += sum;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.p_full[t]);
+                // The row sum is off the hand-off path: P is already out.
+                {
+                    uint64_t s4[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int i = 0; i < BN / 2; ++i) s4[i & 3] = f2_add(s4[i & 3], f2_pack(sv[2 * i], sv[2 * i + 1]));
+                    float a0, a1, b0, b1;
+                    f2_unpack(f2_add(s4[0], s4[1]), a0, a1);
+                    f2_unpack(f2_add(s4[2], s4[3]), b0, b1);
+                    l_run += (a0 + a1) + (b0 + b1);
+                }
             }
         }
         if (ok) ok = warp_wait(&s.o_full, 0, abort, tmo);
