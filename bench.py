@@ -295,10 +295,14 @@ def run_ours(args, W):
     else:  # one launch per task: all the forward's flops over all its launches
         achieved = flops_per_forward * args.steps / (s0["attn_ms"] * 1e-3) / 1e12 if s0["attn_ms"] else None
     if W["dtype"] == "bf16":
-        peak = peaks["bf16_tflops"]
+        # A device-mode launch is timed alone (burst peak); a streamed step
+        # runs the tensor cores for seconds (sustained peak).
+        sustained = W["mode"] != "device"
+        peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak if achieved else None,
-                    "peak_source": peaks["source"] + " bf16 dense (burst)",
+                    "peak_source": peaks["source"] + (" bf16 dense (sustained)" if sustained
+                                                      else " bf16 dense (burst)"),
                     "traffic": (profile_traffic("attn_tc.cu", "attn_tc_l4_n53248_h8_d128.md")
                                 if args.workload == DEFAULT_WORKLOAD else None),
                     "kernel": f"attn_tc_kernel<{d}> (causal={W['variants'][0]})",
@@ -438,12 +442,16 @@ def host_link_gbs(torch, nbytes=1 << 30):
 def streaming_report(W, infos, flops_step, ms_step, peaks, free_before, torch):
     """Streamed workloads: time bound = the slowest of compute at the bf16
     peak and each direction of the host link at its measured bandwidth;
-    efficiency = bound / measured time; device memory against the budget."""
+    efficiency = bound / measured time; device memory against the budget.
+    A streamed step keeps the tensor cores busy for seconds, so the compute
+    bound uses the sustained peak; the burst-peak figure is reported beside
+    it."""
     free_after, _ = torch.cuda.mem_get_info()
     link = host_link_gbs(torch)
     h2d = sum(i["h2d_bytes"] for i in infos)
     d2h = sum(i["d2h_bytes"] for i in infos)
-    t_compute = flops_step / (peaks["bf16_tflops"] * 1e12) * 1e3
+    t_compute = flops_step / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3
+    t_compute_burst = flops_step / (peaks["bf16_tflops"] * 1e12) * 1e3
     t_h2d = h2d / (link["h2d"] * 1e9) * 1e3
     t_d2h = d2h / (link["d2h"] * 1e9) * 1e3
     bound = max(t_compute, t_h2d, t_d2h)
@@ -452,7 +460,9 @@ def streaming_report(W, infos, flops_step, ms_step, peaks, free_before, torch):
     return {"h2d_gbs": link["h2d"], "d2h_gbs": link["d2h"], "h2d_bytes": h2d, "d2h_bytes": d2h,
             "h2d_bytes_minimum": min_in, "t_compute_at_peak_ms": t_compute, "t_h2d_ms": t_h2d,
             "t_d2h_ms": t_d2h, "t_bound_ms": bound, "bound": which, "t_wall_ms": ms_step,
-            "efficiency": bound / ms_step,
+            "efficiency": bound / ms_step, "peak_tflops": peaks["bf16_tflops_sustained"],
+            "peak_source": "sustained bf16 dense",
+            "efficiency_at_burst_peak": max(t_compute_burst, t_h2d, t_d2h) / ms_step,
             "budget_gib": W["budget"] / GiB,
             "library_arena_gib": max(i["host_arena_bytes"] for i in infos) / GiB,
             "device_free_delta_gib": (free_before - free_after) / GiB,
