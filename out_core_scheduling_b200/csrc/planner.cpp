@@ -189,7 +189,10 @@ std::string Planner::build(const PlanSpec &s, int *code) {
 // ---------------------------------------------------------------------------
 // Work lists.
 // ---------------------------------------------------------------------------
-static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int causal) {
+// group[ei]: the task of entry ei (units of one task and head read the same
+// key and value blocks).
+static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int causal,
+                      const std::vector<int64_t> &group) {
     std::vector<WlUnit> u;
     for (int32_t ei = 0; ei < (int32_t)wl->entries.size(); ++ei) {
         const WlEntry &e = wl->entries[ei];
@@ -203,16 +206,25 @@ static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int ca
                 if (x.ntiles > 0) u.push_back(x);
             }
     }
-    // Longest units first (LPT order) so the tail of the grid is short;
-    // the stable sort keeps units of one entry and head together.
-    std::stable_sort(u.begin(), u.end(),
-                     [](const WlUnit &a, const WlUnit &b) { return a.ntiles > b.ntiles; });
+    // Longest units first, in classes of 32 key tiles (coarse LPT order, so
+    // the tail of the grid is short), and inside a class by head, then task:
+    // the CTAs in flight at one time then share a few tasks' key and value
+    // blocks of one head, which stay in L2 instead of being fetched again
+    // from HBM for every (entry, head).
+    std::stable_sort(u.begin(), u.end(), [&](const WlUnit &a, const WlUnit &b) {
+        const int ca = a.ntiles / 32, cb = b.ntiles / 32;
+        if (ca != cb) return ca > cb;
+        if (a.head != b.head) return a.head < b.head;
+        return group[a.entry] < group[b.entry];
+    });
     wl->units.swap(u);
 }
 
 WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     WorkList wl;
+    std::vector<int64_t> task_of;
     for (const Entry &e : entries) {
+        task_of.push_back(e.task);
         WlEntry w{};
         w.q_lo = (int32_t)(e.qb * block);
         w.q_hi = (int32_t)((e.qb + 1) * block);
@@ -230,7 +242,7 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
         }
         wl.entries.push_back(w);
     }
-    add_units(&wl, heads, rows_per_unit, bn, spec.causal);
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, task_of);
     return wl;
 }
 
@@ -267,7 +279,7 @@ WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_un
         w.run_count = (int32_t)wl.runs.size() - w.run_begin;
         wl.entries.push_back(w);
     }
-    add_units(&wl, heads, rows_per_unit, bn, spec.causal);
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, std::vector<int64_t>(wl.entries.size(), t));
     return wl;
 }
 
