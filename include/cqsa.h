@@ -63,6 +63,18 @@ typedef enum { CQSA_BF16 = 0, CQSA_FP32 = 1 } cqsa_dtype_t;
 
 enum { CQSA_DEVICE = 0, CQSA_HOST = 1 };
 
+/* How a device-mode forward recomposes the tasks' local statistics ([A]
+ * recomposition; [B] "Implementation" step 4).
+ *   CQSA_MERGE_SLOTS: every (task, query block) writes its partial O_j and
+ *     lse_j to a slot; a merge kernel then takes the log-sum-exp over the
+ *     slots.  The tasks' results are materialised as the pages describe.
+ *   CQSA_MERGE_FUSED: one CTA walks the allowed key blocks of all the tasks
+ *     of its query rows; its online softmax is the merge, and it writes the
+ *     output directly (no slots, no merge launch).
+ * The streamed (host-mode) path always folds each task into a running
+ * accumulator in the attention kernel's epilogue. */
+typedef enum { CQSA_MERGE_SLOTS = 0, CQSA_MERGE_FUSED = 1 } cqsa_merge_t;
+
 #define CQSA_MAX_LEVELS 4
 #define CQSA_MAX_L 16
 
@@ -78,6 +90,7 @@ typedef struct {
     int causal;
     int dtype; /* cqsa_dtype_t */
     size_t mem_budget_bytes;
+    int merge; /* cqsa_merge_t; 0 (slots) when zero-initialised */
 } cqsa_plan_desc_t;
 
 /* What a plan decided (for logging, tests and the benchmark). */
@@ -99,6 +112,7 @@ typedef struct {
     size_t h2d_bytes;                   /* planned host->device bytes of one host-mode forward */
     size_t d2h_bytes;                   /* planned device->host bytes of one host-mode forward */
     double useful_flops;                /* 4 N^2 H d, halved when causal */
+    int merge;                          /* cqsa_merge_t of device-mode forwards */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */

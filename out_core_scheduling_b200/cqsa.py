@@ -27,6 +27,8 @@ CQSA_BF16 = 0
 CQSA_FP32 = 1
 CQSA_DEVICE = 0
 CQSA_HOST = 1
+CQSA_MERGE_SLOTS = 0
+CQSA_MERGE_FUSED = 1
 MAX_LEVELS = 4
 MAX_L = 16
 
@@ -49,7 +51,7 @@ class PlanDesc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
                 ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("mem_budget_bytes", ctypes.c_size_t)]
+                ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -62,7 +64,8 @@ class PlanInfo(ctypes.Structure):
                 ("max_slots", ctypes.c_int64), ("max_task_rows", ctypes.c_int64),
                 ("head_group", ctypes.c_int), ("device_arena_bytes", ctypes.c_size_t),
                 ("host_arena_bytes", ctypes.c_size_t), ("h2d_bytes", ctypes.c_size_t),
-                ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double)]
+                ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double),
+                ("merge", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -206,7 +209,7 @@ def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = Fa
 
 
 def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
-                 mem_budget_bytes: int = 0) -> Plan:
+                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS) -> Plan:
     desc = PlanDesc()
     desc.N, desc.H, desc.d = N, H, d
     desc.levels = len(ls)
@@ -215,6 +218,7 @@ def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = 
     desc.causal = int(bool(causal))
     desc.dtype = dtype
     desc.mem_budget_bytes = mem_budget_bytes
+    desc.merge = merge
     h = ctypes.c_void_p()
     _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
     return Plan(h.value)

@@ -133,8 +133,7 @@ std::vector<char> pack_wl(const WorkList &wl) {
 
 struct LeafState {
     DevWl wl;
-    MergeSeg *segs = nullptr;
-    std::vector<MergeSeg> host_segs;
+    std::vector<MergeSeg> host_segs;  // query blocks of the task; SEG_LAST ones are copied out after it
 };
 
 }  // namespace
@@ -164,7 +163,6 @@ struct cqsa_plan {
     char *pool_q = nullptr, *pool_k = nullptr, *pool_v = nullptr;  // block caches
     char *out_st[2] = {};
     float *lse_st[2] = {};
-    float *h_part_o = nullptr, *h_part_lse = nullptr;
     std::vector<LeafState> leaves;
     CUtensorMap mq, mk, mv;  // over the block pools
     cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
@@ -235,13 +233,17 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
-    if (pl.max_slots > 32) return fail(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
+    const bool fused = pl.spec.fused != 0;
+    if (!fused && pl.max_slots > 32) return fail(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
     WorkList wl = pl.device_worklist(unit_rows_for(P->elem), key_tile_for(P->elem), H);
     ArenaLayout a;
     const size_t o_err = a.take(256);
-    const size_t o_po = a.take((size_t)pl.max_slots * N * H * d * sizeof(float));
-    const size_t o_pl = a.take((size_t)pl.max_slots * H * N * sizeof(float));
-    const size_t o_ns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+    size_t o_po = 0, o_pl = 0, o_ns = 0;
+    if (!fused) {
+        o_po = a.take((size_t)pl.max_slots * N * H * d * sizeof(float));
+        o_pl = a.take((size_t)pl.max_slots * H * N * sizeof(float));
+        o_ns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+    }
     const size_t o_wl = a.take(wl_region(wl));
     if (a.total != pl.sizing.device_arena)
         return fail(CQSA_ERR_CUDA, "internal: device arena layout mismatch (%zu vs %zu)", a.total,
@@ -254,11 +256,13 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
     P->dev_bytes = a.total;
     CK(cudaMemset(arena, 0, a.total));
     P->dev_err = reinterpret_cast<int *>(arena + o_err);
-    P->dev_part_o = reinterpret_cast<float *>(arena + o_po);
-    P->dev_part_lse = reinterpret_cast<float *>(arena + o_pl);
-    P->dev_nslots = reinterpret_cast<int32_t *>(arena + o_ns);
-    CK(cudaMemcpy(P->dev_nslots, pl.slots_per_block.data(), pl.slots_per_block.size() * sizeof(int32_t),
-                  cudaMemcpyHostToDevice));
+    if (!fused) {
+        P->dev_part_o = reinterpret_cast<float *>(arena + o_po);
+        P->dev_part_lse = reinterpret_cast<float *>(arena + o_pl);
+        P->dev_nslots = reinterpret_cast<int32_t *>(arena + o_ns);
+        CK(cudaMemcpy(P->dev_nslots, pl.slots_per_block.data(), pl.slots_per_block.size() * sizeof(int32_t),
+                      cudaMemcpyHostToDevice));
+    }
     std::vector<char> buf = pack_wl(wl);
     if (!buf.empty()) CK(cudaMemcpy(arena + o_wl, buf.data(), buf.size(), cudaMemcpyHostToDevice));
     P->dev_wl = place_wl(arena + o_wl, wl);
@@ -289,16 +293,13 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
         o_out[s] = a.take((size_t)R * g * dd * e);
         o_lse[s] = a.take((size_t)g * R * sizeof(float));
     }
-    const size_t o_po = a.take((size_t)R * g * dd * sizeof(float));
-    const size_t o_pl = a.take((size_t)g * R * sizeof(float));
     std::vector<WorkList> wls(pl.leaves.size());
-    std::vector<size_t> o_wl(pl.leaves.size()), o_seg(pl.leaves.size());
+    std::vector<size_t> o_wl(pl.leaves.size());
     P->leaves.assign(pl.leaves.size(), LeafState());
     for (size_t t = 0; t < pl.leaves.size(); ++t) {
         wls[t] = pl.leaf_worklist((int64_t)t, pp, unit_rows_for(P->elem), key_tile_for(P->elem), g);
         o_wl[t] = a.take(wl_region(wls[t]));
         P->leaves[t].host_segs = pl.leaf_merge_segments((int64_t)t);
-        o_seg[t] = a.take(P->leaves[t].host_segs.size() * sizeof(MergeSeg));
     }
     if (a.total != pl.sizing.host_arena)
         return fail(CQSA_ERR_CUDA, "internal: host-mode arena layout mismatch (%zu vs %zu)", a.total,
@@ -320,16 +321,10 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
         P->out_st[s] = arena + o_out[s];
         P->lse_st[s] = reinterpret_cast<float *>(arena + o_lse[s]);
     }
-    P->h_part_o = reinterpret_cast<float *>(arena + o_po);
-    P->h_part_lse = reinterpret_cast<float *>(arena + o_pl);
     for (size_t t = 0; t < pl.leaves.size(); ++t) {
         std::vector<char> buf = pack_wl(wls[t]);
         if (!buf.empty()) CK(cudaMemcpy(arena + o_wl[t], buf.data(), buf.size(), cudaMemcpyHostToDevice));
         P->leaves[t].wl = place_wl(arena + o_wl[t], wls[t]);
-        P->leaves[t].segs = reinterpret_cast<MergeSeg *>(arena + o_seg[t]);
-        const auto &hs = P->leaves[t].host_segs;
-        if (!hs.empty())
-            CK(cudaMemcpy(P->leaves[t].segs, hs.data(), hs.size() * sizeof(MergeSeg), cudaMemcpyHostToDevice));
     }
     if (P->dtype == CQSA_BF16) {
         cqsa_status_t st;
@@ -397,6 +392,15 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     ap.part_lse = P->dev_part_lse;
     ap.part_rows = N;
     ap.H = H;
+    const bool fused = pl.spec.fused != 0;
+    if (fused) {
+        // Every entry is the first and last partial of its rows: the kernel
+        // writes out and lse itself.
+        ap.epi = EPI_MERGE;
+        ap.out = out;
+        ap.out_lse = lse;
+        ap.out_rows = N;
+    }
     if (P->dtype == CQSA_BF16) {
         CUtensorMap mq, mk, mv;
         if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
@@ -410,6 +414,7 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
         CK(launch_attn_simt(d, P->elem, q, k, v, ap, P->dev_wl.num_units, stream));
         tm.stop();
     }
+    if (fused) return CQSA_OK;
     LaunchTimer tm(P, stream, 1);
     CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H, out, lse,
                           stream));
@@ -468,16 +473,24 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
                 }
             }
             CK(cudaEventRecord(P->ev_in_ready[s], P->s_in));
-            // -- tile attention on the task's cached blocks.
+            // -- tile attention on the task's cached blocks; its epilogue
+            // folds the task into the accumulator and writes the rows the
+            // task finishes to out stage s (free once the D2H of the task two
+            // back has read it).
             CK(cudaStreamWaitEvent(P->s_comp, P->ev_in_ready[s], 0));
+            if (it >= 2) CK(cudaStreamWaitEvent(P->s_comp, P->ev_out_free[s], 0));
             AttnParams ap = base_params(P, P->h_err);
             ap.entries = L.wl.entries;
             ap.runs = L.wl.runs;
             ap.units = L.wl.units;
-            ap.part_o = P->h_part_o;
-            ap.part_lse = P->h_part_lse;
-            ap.part_rows = R;
             ap.H = g;
+            ap.epi = EPI_MERGE;
+            ap.acc_o = P->acc_o;
+            ap.acc_lse = P->acc_lse;
+            ap.acc_rows = N;
+            ap.out = P->out_st[s];
+            ap.out_lse = P->lse_st[s];
+            ap.out_rows = R;
             {
                 LaunchTimer tm(P, P->s_comp, 0);
                 if (P->dtype == CQSA_BF16)
@@ -488,15 +501,6 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
                 tm.stop();
             }
             CK(cudaEventRecord(P->ev_in_free[s], P->s_comp));
-            // -- merge into the accumulator; finished rows go to out stage s.
-            if (it >= 2) CK(cudaStreamWaitEvent(P->s_comp, P->ev_out_free[s], 0));
-            {
-                LaunchTimer tm(P, P->s_comp, 1);
-                CK(launch_merge_stream(d, P->elem, L.segs, (int)L.host_segs.size(), (int)B, P->h_part_o,
-                                       P->h_part_lse, R, P->acc_o, P->acc_lse, N, g, P->out_st[s], P->lse_st[s],
-                                       P->s_comp));
-                tm.stop();
-            }
             CK(cudaEventRecord(P->ev_merged[s], P->s_comp));
             // -- D2H of finished rows.
             CK(cudaStreamWaitEvent(P->s_out, P->ev_merged[s], 0));
@@ -567,6 +571,9 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
     s.causal = desc->causal ? 1 : 0;
     s.elem_bytes = desc->dtype == CQSA_BF16 ? 2 : 4;
     s.budget = desc->mem_budget_bytes;
+    if (desc->merge != CQSA_MERGE_SLOTS && desc->merge != CQSA_MERGE_FUSED)
+        return fail(CQSA_ERR_INVALID_ARG, "merge must be CQSA_MERGE_SLOTS or CQSA_MERGE_FUSED");
+    s.fused = desc->merge == CQSA_MERGE_FUSED;
     cqsa_plan_t *P = nullptr;
     cqsa_status_t st = build_plan(s, desc->dtype, &P);
     if (st != CQSA_OK) return st;
@@ -713,6 +720,7 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->d2h_bytes = pl.sizing.d2h;
     const double n = (double)pl.spec.N;
     info->useful_flops = 4.0 * n * n * pl.spec.H * pl.spec.d * (pl.spec.causal ? 0.5 : 1.0);
+    info->merge = pl.spec.fused ? CQSA_MERGE_FUSED : CQSA_MERGE_SLOTS;
     return CQSA_OK;
 }
 

@@ -15,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 #include "worklist.h"
 
@@ -148,13 +149,39 @@ __global__ void __launch_bounds__(simt::THREADS)
         const int32_t row = q0 + ty * 4 + i;
         if (row >= q_end) continue;
         const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
+        const float lse_n = (m[i] + log2f(l[i])) * 0.69314718055994531f;
         const int64_t out_row = (int64_t)e.out_lo + (row - e.q_lo);
-        float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * H + h) * D;
+        if (p.epi == EPI_MERGE) {
+            // Fold into the running accumulator or write the finished row
+            // (see epilogue.cuh).
+            const bool first = (e.flags & SEG_FIRST) != 0, last = (e.flags & SEG_LAST) != 0;
+            const int64_t grow = (int64_t)row + e.q_goff;
+            FoldWeights w{0.f, 1.f, lse_n};
+            if (!first) w = fold_weights(p.acc_lse[(int64_t)h * p.acc_rows + grow], lse_n);
+            float *acc = p.acc_o + (grow * H + h) * D;
+            T *dst = static_cast<T *>(p.out) + (out_row * H + h) * D;
 #pragma unroll
-        for (int jj = 0; jj < NJ; ++jj) dst[tx + 16 * jj] = o[i][jj] * inv;
-        if (tx == 0)
-            p.part_lse[((int64_t)e.slot * H + h) * p.part_rows + out_row] =
-                (m[i] + log2f(l[i])) * 0.69314718055994531f;
+            for (int jj = 0; jj < NJ; ++jj) {
+                const int c = tx + 16 * jj;
+                float v = o[i][jj] * inv;
+                if (!first) v = w.wa * acc[c] + w.wn * v;
+                if (last)
+                    store_out(dst + c, v);
+                else
+                    acc[c] = v;
+            }
+            if (tx == 0) {
+                if (last)
+                    p.out_lse[(int64_t)h * p.out_rows + out_row] = w.lse;
+                else
+                    p.acc_lse[(int64_t)h * p.acc_rows + grow] = w.lse;
+            }
+        } else {
+            float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * H + h) * D;
+#pragma unroll
+            for (int jj = 0; jj < NJ; ++jj) dst[tx + 16 * jj] = o[i][jj] * inv;
+            if (tx == 0) p.part_lse[((int64_t)e.slot * H + h) * p.part_rows + out_row] = lse_n;
+        }
     }
 }
 

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "exp2_poly.h"
 #include "kernels.h"
 #include "worklist.h"
@@ -440,7 +441,56 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
         }
         if (ok) ok = warp_wait(&s.o_full, 0, abort, tmo);
-        if (ok) {
+        if (ok && p.epi == EPI_MERGE) {
+            // Fold this task's row into the running accumulator, or write
+            // the finished row (see epilogue.cuh).
+            tc_fence_after();
+            const bool valid = q_local < e.q_hi;
+            const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+            const float lse_n = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+            const bool first = (e.flags & SEG_FIRST) != 0, last = (e.flags & SEG_LAST) != 0;
+            const int64_t grow = (int64_t)q_local + e.q_goff;
+            const int64_t orow = (int64_t)e.out_lo + (q_local - e.q_lo);
+            FoldWeights w{0.f, 1.f, lse_n};
+            if (valid && !first) w = fold_weights(p.acc_lse[(int64_t)head * p.acc_rows + grow], lse_n);
+            float *acc = p.acc_o + (grow * p.H + head) * D;
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + (orow * p.H + head) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
+                tmem_wait_ld();
+                reg_fence32(o);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 v4 = make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                        if (!first) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(acc + cc * 32 + i);
+                            v4.x = w.wa * a4.x + w.wn * v4.x;
+                            v4.y = w.wa * a4.y + w.wn * v4.y;
+                            v4.z = w.wa * a4.z + w.wn * v4.z;
+                            v4.w = w.wa * a4.w + w.wn * v4.w;
+                        }
+                        if (last) {
+                            uint2 u;
+                            u.x = pack_bf16x2(v4.x, v4.y);
+                            u.y = pack_bf16x2(v4.z, v4.w);
+                            *reinterpret_cast<uint2 *>(dst + cc * 32 + i) = u;
+                        } else {
+                            *reinterpret_cast<float4 *>(acc + cc * 32 + i) = v4;
+                        }
+                    }
+                }
+            }
+            if (valid) {
+                if (last)
+                    p.out_lse[(int64_t)head * p.out_rows + orow] = w.lse;
+                else
+                    p.acc_lse[(int64_t)head * p.acc_rows + grow] = w.lse;
+            }
+        } else if (ok) {
             tc_fence_after();
             const bool valid = q_local < e.q_hi;
             const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;

@@ -8,10 +8,18 @@
 
 namespace cqsa {
 
-// Parameters shared by both attention kernels.  Partial outputs are laid
-// out [slot][part_rows][H][d] (fp32, normalised by the task's own softmax
-// denominator) and partial lse [slot][H][part_rows] (natural log); query row
-// q of an entry goes to partial row out_lo + (q - q_lo).
+// Epilogue of the attention kernels.
+//   EPI_SLOTS: write the task's partial (O_j normalised by its own softmax
+//     denominator, fp32, [slot][part_rows][H][d]; lse_j [slot][H][part_rows],
+//     natural log) at partial row out_lo + (q - q_lo) for the merge kernel.
+//   EPI_MERGE: recompose in place.  The entry's flags say whether the
+//     partial is the first of its query block (it initialises the running
+//     accumulator acc_o [acc_rows][H][d] fp32 / acc_lse [H][acc_rows] at the
+//     global row q + q_goff) and whether it is the last (the merged row goes
+//     to out [out_rows][H][d] in the input dtype and out_lse [H][out_rows] at
+//     row out_lo + (q - q_lo)).  An entry that is both writes out directly.
+enum { EPI_SLOTS = 0, EPI_MERGE = 1 };
+
 struct AttnParams {
     const WlEntry *entries;
     const WlRun *runs;
@@ -26,6 +34,13 @@ struct AttnParams {
     uint64_t timeout_ns;
     int *err;           // device error word
     int stall_test;     // test hook: the MMA issuer issues nothing (waits run out)
+    int epi;            // EPI_SLOTS or EPI_MERGE
+    float *acc_o;
+    float *acc_lse;
+    int64_t acc_rows;
+    void *out;
+    float *out_lse;
+    int64_t out_rows;
 };
 
 // bf16 tensor-core kernel (attn_tc.cu).  Maps describe [rows, H, d] bf16
@@ -43,15 +58,5 @@ cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k
 cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const float *part_lse,
                                const int32_t *nslots, int64_t block, int64_t N, int H, void *out,
                                float *lse, cudaStream_t stream);
-
-// Streamed recomposition: merge one task's partial rows (local layout
-// [R][g][d], lse [g][R]) into the running accumulator (global rows
-// [N][g][d], lse [g][N]) segment by segment; a segment's first partial
-// initialises the accumulator, its last writes the finished rows to out
-// ([R][g][d] in the input dtype) and lse_out ([g][R]).
-cudaError_t launch_merge_stream(int d, int elem_bytes, const MergeSeg *segs, int nsegs, int max_rows,
-                                const float *part_o, const float *part_lse, int64_t R, float *acc_o,
-                                float *acc_lse, int64_t N, int g, void *out, float *lse_out,
-                                cudaStream_t stream);
 
 }  // namespace cqsa

@@ -107,50 +107,6 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Streamed mode: one task's partials [R][g][D] / [g][R] merged into the
-// running accumulator [N][g][D] / [g][N], segment by segment.
-template <int D, typename TO>
-__global__ void __launch_bounds__(256)
-    merge_stream_kernel(const MergeSeg *__restrict__ segs, const float *__restrict__ part_o,
-                        const float *__restrict__ part_lse, int64_t R, float *__restrict__ acc_o,
-                        float *__restrict__ acc_lse, int64_t N, int g, TO *__restrict__ out,
-                        float *__restrict__ lse_out) {
-    constexpr int V = D / 32;
-    const MergeSeg sg = segs[blockIdx.y];
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    const int64_t total = (int64_t)sg.rows * g;
-    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-        const int64_t i = w / g;
-        const int h = (int)(w - i * g);
-        const int64_t lr = sg.local_lo + i;
-        const int64_t gr = sg.global_lo + i;
-        float o[V];
-        load_vec<V>(part_o + (lr * g + h) * D + lane * V, o);
-        float l = part_lse[(int64_t)h * R + lr];
-        if (!(sg.flags & SEG_FIRST)) {
-            float a[V];
-            load_vec<V>(acc_o + (gr * g + h) * D + lane * V, a);
-            const float la = acc_lse[(int64_t)h * N + gr];
-            const float M = fmaxf(la, l);
-            const float wa = (la == -INFINITY) ? 0.f : __expf(la - M);
-            const float wp = (l == -INFINITY) ? 0.f : __expf(l - M);
-            const float W = wa + wp;
-            const float inv = 1.f / W;
-#pragma unroll
-            for (int t = 0; t < V; ++t) o[t] = (wa * a[t] + wp * o[t]) * inv;
-            l = M + __logf(W);
-        }
-        if (sg.flags & SEG_LAST) {
-            store_vec<V>(out + (lr * g + h) * D + lane * V, o);
-            if (lane == 0) lse_out[(int64_t)h * R + lr] = l;
-        } else {
-            store_vec<V>(acc_o + (gr * g + h) * D + lane * V, o);
-            if (lane == 0) acc_lse[(int64_t)h * N + gr] = l;
-        }
-    }
-}
-
 static int merge_grid(int64_t warps_needed) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -178,41 +134,6 @@ cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const
             return merge_slots_t<64, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
         if (d == 128)
             return merge_slots_t<128, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
-    }
-    return cudaErrorInvalidValue;
-}
-
-template <int D, typename TO>
-static cudaError_t merge_stream_t(const MergeSeg *segs, int nsegs, int max_rows, const float *po,
-                                  const float *pl, int64_t R, float *ao, float *al, int64_t N, int g,
-                                  void *out, float *lo, cudaStream_t st) {
-    int gx = merge_grid((int64_t)max_rows * g);
-    gx = (gx + nsegs - 1) / nsegs;
-    if (gx < 1) gx = 1;
-    dim3 grid(gx, nsegs);
-    merge_stream_kernel<D, TO><<<grid, 256, 0, st>>>(segs, po, pl, R, ao, al, N, g, static_cast<TO *>(out), lo);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_merge_stream(int d, int elem_bytes, const MergeSeg *segs, int nsegs, int max_rows,
-                                const float *part_o, const float *part_lse, int64_t R, float *acc_o,
-                                float *acc_lse, int64_t N, int g, void *out, float *lse_out,
-                                cudaStream_t stream) {
-    if (nsegs <= 0) return cudaSuccess;
-    if (elem_bytes == 4) {
-        if (d == 64)
-            return merge_stream_t<64, float>(segs, nsegs, max_rows, part_o, part_lse, R, acc_o, acc_lse, N, g, out,
-                                             lse_out, stream);
-        if (d == 128)
-            return merge_stream_t<128, float>(segs, nsegs, max_rows, part_o, part_lse, R, acc_o, acc_lse, N, g, out,
-                                              lse_out, stream);
-    } else if (elem_bytes == 2) {
-        if (d == 64)
-            return merge_stream_t<64, __nv_bfloat16>(segs, nsegs, max_rows, part_o, part_lse, R, acc_o, acc_lse, N,
-                                                     g, out, lse_out, stream);
-        if (d == 128)
-            return merge_stream_t<128, __nv_bfloat16>(segs, nsegs, max_rows, part_o, part_lse, R, acc_o, acc_lse, N,
-                                                      g, out, lse_out, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -222,9 +222,43 @@ static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int ca
 
 WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     WorkList wl;
-    std::vector<int64_t> task_of;
+    std::vector<int64_t> group;
+    if (spec.fused) {
+        // The tasks of a query block own disjoint sets of its allowed key
+        // blocks; their union, as maximal runs, is one entry.
+        std::vector<std::vector<int64_t>> keys(num_blocks);
+        for (const Entry &e : entries)
+            for (const KeyRun &r : e.runs)
+                for (int64_t b = r.b0; b <= r.b1; ++b) keys[e.qb].push_back(b);
+        for (int64_t qb = 0; qb < num_blocks; ++qb) {
+            std::vector<int64_t> &kb = keys[qb];
+            if (kb.empty()) continue;
+            std::sort(kb.begin(), kb.end());
+            WlEntry w{};
+            w.q_lo = (int32_t)(qb * block);
+            w.q_hi = (int32_t)((qb + 1) * block);
+            w.out_lo = w.q_lo;
+            w.flags = SEG_FIRST | SEG_LAST;
+            w.run_begin = (int32_t)wl.runs.size();
+            for (size_t i = 0; i < kb.size(); ++i) {
+                if (i > 0 && kb[i] == kb[i - 1] + 1) {
+                    wl.runs.back().k_hi = (int32_t)((kb[i] + 1) * block);
+                } else {
+                    WlRun x{};
+                    x.k_lo = (int32_t)(kb[i] * block);
+                    x.k_hi = (int32_t)((kb[i] + 1) * block);
+                    wl.runs.push_back(x);
+                }
+            }
+            w.run_count = (int32_t)wl.runs.size() - w.run_begin;
+            wl.entries.push_back(w);
+            group.push_back(0);
+        }
+        add_units(&wl, heads, rows_per_unit, bn, spec.causal, group);
+        return wl;
+    }
     for (const Entry &e : entries) {
-        task_of.push_back(e.task);
+        group.push_back(e.task);
         WlEntry w{};
         w.q_lo = (int32_t)(e.qb * block);
         w.q_hi = (int32_t)((e.qb + 1) * block);
@@ -242,7 +276,7 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
         }
         wl.entries.push_back(w);
     }
-    add_units(&wl, heads, rows_per_unit, bn, spec.causal, task_of);
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, group);
     return wl;
 }
 
@@ -259,6 +293,7 @@ WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_un
         w.q_goff = (int32_t)((e.qb - qs) * block);
         w.slot = 0;
         w.out_lo = (int32_t)(e.mq * block);
+        w.flags = (first_leaf_[e.qb] == t ? SEG_FIRST : 0) | (last_leaf_[e.qb] == t ? SEG_LAST : 0);
         w.run_begin = (int32_t)wl.runs.size();
         for (const KeyRun &r : e.runs) {
             for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
@@ -430,10 +465,12 @@ static size_t wl_bytes(const WorkList &wl) {
 size_t Planner::device_arena_bytes() const {
     const int64_t N = spec.N;
     ArenaLayout a;
-    a.take(256);                                                    // error word
-    a.take((size_t)max_slots * N * spec.H * spec.d * sizeof(float)); // partial O
-    a.take((size_t)max_slots * spec.H * N * sizeof(float));          // partial lse
-    a.take((size_t)num_blocks * sizeof(int32_t));                    // slots per block
+    a.take(256);                                                        // error word
+    if (!spec.fused) {
+        a.take((size_t)max_slots * N * spec.H * spec.d * sizeof(float)); // partial O
+        a.take((size_t)max_slots * spec.H * N * sizeof(float));          // partial lse
+        a.take((size_t)num_blocks * sizeof(int32_t));                    // slots per block
+    }
     WorkList wl = device_worklist(unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), spec.H);
     a.take(wl_bytes(wl));
     return a.total;
@@ -454,12 +491,9 @@ size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
         a.take((size_t)R * g * dd * e);                 // finished out rows
         a.take((size_t)g * R * sizeof(float));          // finished lse rows
     }
-    a.take((size_t)R * g * dd * sizeof(float));         // task partial O
-    a.take((size_t)g * R * sizeof(float));              // task partial lse
     for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
         WorkList wl = leaf_worklist(t, pl, unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
         a.take(wl_bytes(wl));
-        a.take(leaf_merge_segments(t).size() * sizeof(MergeSeg));
     }
     return a.total;
 }

@@ -61,6 +61,7 @@ struct PlanSpec {
     int causal = 0;
     int elem_bytes = 2;                     // 2 = bf16, 4 = fp32
     size_t budget = 0;                      // 0 = unlimited
+    int fused = 0;                          // device mode: merge in the kernel, no partial slots
 };
 
 // Device block cache of the streamed path.  A Q slot holds one query block
@@ -107,12 +108,17 @@ public:
     int64_t max_task_rows = 0;
     Sizing sizing;
 
-    // rows_per_unit: query rows one CTA covers; bn: key tile width.
+    // rows_per_unit: query rows one CTA covers; bn: key tile width.  With
+    // spec.fused, one entry per query block holds the allowed key blocks of
+    // all its tasks (the kernel's online softmax merges them) and writes the
+    // output directly; otherwise one entry per (task, query block) with a
+    // partial slot.
     WorkList device_worklist(int rows_per_unit, int bn, int heads) const;
     // Work list of leaf t reading Q, K, V from the block pools of `pool`.
     WorkList leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const;
     // Merge segments of leaf t in host mode (one per query block with an
-    // entry), with first/last-touch flags in leaf order.
+    // entry), with first/last-touch flags in leaf order; the D2H copies of
+    // finished rows follow them.
     std::vector<MergeSeg> leaf_merge_segments(int64_t t) const;
     // Members of leaf t whose Q (resp. K/V) rows a streamed task needs.
     void leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char> *need_kv) const;

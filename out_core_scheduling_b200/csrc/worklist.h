@@ -27,8 +27,8 @@ struct WlEntry {
     int32_t slot;         // partial index (device mode); 0 in host mode
     int32_t run_begin;    // first WlRun of this entry
     int32_t run_count;    // number of runs (>= 1)
-    int32_t out_lo;       // partial-output row of query row q_lo
-    int32_t pad;
+    int32_t out_lo;       // output row of query row q_lo
+    int32_t flags;        // merge in the epilogue: SEG_FIRST / SEG_LAST
 };
 
 struct WlRun {
@@ -53,6 +53,8 @@ struct MergeSeg {
     int32_t flags;        // bit 0: first partial of the block, bit 1: last
 };
 
+// SEG_FIRST: the first partial of its query block (nothing to merge with);
+// SEG_LAST: the last (the merged rows are final).
 enum { SEG_FIRST = 1, SEG_LAST = 2 };
 
 // Tile shapes of the two attention kernels.  The planner sizes work lists

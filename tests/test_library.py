@@ -172,6 +172,22 @@ def test_auto_levels_recurse_until_it_fits():
     assert p.info()["levels"] == 2 and p.info()["host_arena_bytes"] <= lo
 
 
+def test_fused_merge_plan():
+    """The fused recomposition needs no partial slots: a smaller device arena,
+    the same tasks and the same host-mode plan."""
+    args = (13 * 256, 2, 128, [4])
+    slots = cqsa.cqsa_plan_ex(*args).info()
+    fused = cqsa.cqsa_plan_ex(*args, merge=cqsa.CQSA_MERGE_FUSED).info()
+    assert slots["merge"] == cqsa.CQSA_MERGE_SLOTS and fused["merge"] == cqsa.CQSA_MERGE_FUSED
+    assert fused["num_tasks"] == slots["num_tasks"] and fused["num_entries"] == slots["num_entries"]
+    partials = slots["max_slots"] * 13 * 256 * 2 * (128 + 1) * 4
+    assert fused["device_arena_bytes"] + partials <= slots["device_arena_bytes"]
+    assert fused["host_arena_bytes"] == slots["host_arena_bytes"]
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_plan_ex(*args, merge=7)
+    assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("args,status", [
     ((1000, 1, 64, 3, 1, False, 0), cqsa.CQSA_ERR_INVALID_ARG),       # 1000 % 7 != 0
     ((43 * 4, 1, 64, 7, 1, False, 0), cqsa.CQSA_ERR_NO_DIFFERENCE_SET),

@@ -195,3 +195,43 @@ def test_bounded_wait_reports_timeout_and_recovers():
     plan.debug(timeout_ns=0, stall_mma=False)
     out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
     check(out, lse, q, k, v, np.arange(N), False)
+
+
+# ---------------------------------------------------------------- fused merge
+FUSED_CASES = [
+    # (N, H, d, levels, dtype, sample)
+    (7 * 256, 2, 128, [3], torch.bfloat16, None),
+    (7 * 256, 2, 64, [3], torch.bfloat16, None),
+    (7 * 200, 2, 128, [3], torch.bfloat16, None),      # ragged tiles
+    (13 * 384, 2, 128, [4], torch.bfloat16, None),
+    (91 * 128, 2, 128, [4, 3], torch.bfloat16, 512),   # two levels
+    (7 * 3, 1, 64, [3], torch.bfloat16, None),         # blocks smaller than a tile
+    (3584, 1, 64, [3], torch.float32, None),
+    (7 * 200, 2, 128, [3], torch.float32, None),
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: f"n{c[0]}-h{c[1]}-d{c[2]}-l{c[3]}-{str(c[4])[6:]}")
+def test_fused_merge_device(case, causal):
+    """CQSA_MERGE_FUSED: one CTA walks all the tasks' key runs of its rows
+    and writes out / lse itself; same oracle, same tolerances."""
+    N, H, d, ls, dtype, sample = case
+    q, k, v = _inputs(N, H, d, dtype, seed=20)
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, merge=cqsa.CQSA_MERGE_FUSED)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    rows = np.arange(N) if sample is None else sample_rows(N, sample)
+    check(out, lse, q, k, v, rows, causal)
+
+
+def test_fused_equals_slots():
+    """Both recompositions of the same forward agree to rounding."""
+    N, H, d = 13 * 256, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=21)
+    for causal in (False, True):
+        a, la = run(cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal), q, k, v, cqsa.CQSA_DEVICE)
+        b, lb = run(cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, merge=cqsa.CQSA_MERGE_FUSED), q, k, v,
+                    cqsa.CQSA_DEVICE)
+        assert (a.float() - b.float()).abs().max().item() <= 2e-2
+        assert (la - lb).abs().max().item() <= 1e-4

@@ -24,11 +24,12 @@ def _host_inputs(N, H, d, dist="normal"):
     return hq, hk, hv
 
 
+@pytest.mark.parametrize("merge", [0, 1], ids=["slots", "fused"])
 @pytest.mark.parametrize("causal", [False, True])
-def test_l4_n53248_h8_device(causal):
+def test_l4_n53248_h8_device(causal, merge):
     N, H, d = 53248, 8, 128
     q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
-    plan = cqsa.cqsa_plan(N, H, d, 4, 1, causal, 0)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, merge=merge)
     out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
     check(out, lse, q, k, v, sample_rows(N), causal)
 
