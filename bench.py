@@ -354,6 +354,11 @@ def run_ours(args, W):
         "wall_ms_timed": (wall1 - wall0) * 1e3,
     }
 
+    # ---- the fused recomposition on the same device inputs (no slots, no
+    # merge launch), timed the same way; the headline stays the slots path.
+    if W["mode"] == "device" and not args.no_fused:
+        result["fused_merge"] = run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, value)
+
     # ---- end to end through the public API from pinned host memory.
     if W["mode"] == "host":
         # The timed path already starts and ends in pinned host memory.
@@ -377,6 +382,42 @@ def run_ours(args, W):
         print(json.dumps(result), flush=True)
     del plans
     D.close()
+
+
+def run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, slots_value):
+    import torch
+    from out_core_scheduling_b200 import cqsa
+
+    N, H, d = W["N"], W["H"], W["d"]
+    cdt = cqsa.CQSA_BF16 if W["dtype"] == "bf16" else cqsa.CQSA_FP32
+    plans = [cqsa.cqsa_plan_ex(N, H, d, W["ls"], causal=c, dtype=cdt, merge=cqsa.CQSA_MERGE_FUSED)
+             for c in W["variants"]]
+
+    def step():
+        for p, o, l in zip(plans, outs, lses):
+            cqsa.cqsa_forward(p, q, k, v, o, l, cqsa.CQSA_DEVICE, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(D.local_rank)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier(D.local_rank)
+    for p in plans:
+        p.sync(stream)
+    ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}")
+    value = flops_step * args.steps * D.world / (ms * 1e-3) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms / args.steps,
+            "vs_slots": value / slots_value if slots_value else None,
+            "gpu_launches": len(plans) * args.steps,
+            "path": "cqsa_plan_ex(merge=CQSA_MERGE_FUSED): one CTA per 256 query rows walks the allowed "
+                    "key runs of all the tasks of its rows and writes out and lse; no slots, no merge launch"}
 
 
 def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream):
@@ -546,6 +587,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused-merge timing of device workloads")
     ap.add_argument("--profile-run", action="store_true",
                     help="only warm-up + steps of the device path (for ncu captures)")
     args = ap.parse_args(argv)
