@@ -7,6 +7,8 @@ never does, and this package imports nothing from the product.
   * ``attention_rows``  - fp64 exact softmax attention (C, OpenMP) for chosen
     query rows, from ``oracle_attention.c``.
   * ``attention_probs`` - the full weight matrix for tiny problems.
+  * ``attention_backward_dq`` / ``attention_backward_dkdv`` - fp64 gradients
+    of the same definition for chosen query / key rows.
   * ``cqs_ref``         - plain-Python CQS Divide reference (difference sets,
     subsequences, masks, recursion, decomposed fp64 simulation).
 """
@@ -52,6 +54,17 @@ def _load():
         lib.oracle_attention_probs.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_void_p]
+        for name in ("oracle_attention_backward_dq", "oracle_attention_backward_dkdv"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+        lib.oracle_attention_backward_dq.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_attention_backward_dkdv.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -130,3 +143,58 @@ def attention_probs(q, k, causal=False, scale=None):
     if rc != 0:
         raise ValueError("oracle_attention_probs rejected its arguments")
     return probs
+
+
+def _four(q, k, v, dout):
+    qa, tq = _as_stored(q)
+    ka, tk = _as_stored(k)
+    va, tv = _as_stored(v)
+    da, td = _as_stored(dout)
+    if not (tq == tk == tv == td):
+        raise TypeError("q, k, v, dout must share a dtype")
+    N, H, d = qa.shape
+    for x in (ka, va, da):
+        if x.shape != (N, H, d):
+            raise ValueError("q, k, v, dout must all be [N, H, d]")
+    return qa, ka, va, da, tq, N, H, d
+
+
+def attention_backward_dq(q, k, v, dout, rows=None, causal=False, scale=None):
+    """fp64 dq for query rows ``rows`` (default all), every head, given the
+    output gradient ``dout``.  Returns (dq [R, H, d], lse [R, H], D [R, H])
+    with D_i = <dout_i, out_i>."""
+    lib = _load()
+    qa, ka, va, da, t, N, H, d = _four(q, k, v, dout)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    rows = np.arange(N, dtype=np.int64) if rows is None else rows
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dq = np.empty((rows.size, H, d), dtype=np.float64)
+    lse = np.empty((rows.size, H), dtype=np.float64)
+    D = np.empty((rows.size, H), dtype=np.float64)
+    rc = lib.oracle_attention_backward_dq(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data,
+                                          t, N, H, d, int(bool(causal)), float(scale),
+                                          rows.ctypes.data, rows.size, dq.ctypes.data,
+                                          lse.ctypes.data, D.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_attention_backward_dq rejected its arguments")
+    return dq, lse, D
+
+
+def attention_backward_dkdv(q, k, v, dout, keys=None, causal=False, scale=None):
+    """fp64 dk, dv for key rows ``keys`` (default all), every head.
+    Returns (dk [K, H, d], dv [K, H, d]).  Costs O(N^2 H d)."""
+    lib = _load()
+    qa, ka, va, da, t, N, H, d = _four(q, k, v, dout)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    keys = np.arange(N, dtype=np.int64) if keys is None else keys
+    keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+    dk = np.empty((keys.size, H, d), dtype=np.float64)
+    dv = np.empty((keys.size, H, d), dtype=np.float64)
+    rc = lib.oracle_attention_backward_dkdv(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data,
+                                            t, N, H, d, int(bool(causal)), float(scale),
+                                            keys.ctypes.data, keys.size, dk.ctypes.data, dv.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle_attention_backward_dkdv rejected its arguments")
+    return dk, dv

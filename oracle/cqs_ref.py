@@ -197,3 +197,43 @@ def decomposed_attention(q, k, v, ls, causal: bool, scale: float):
         lse_out[r] = M + np.log(tot)
         out[r] = np.einsum("sh,shd->hd", W / tot, np.stack(partial_o[r]))
     return out, lse_out
+
+
+def decomposed_backward(q, k, v, dout, ls, causal: bool, scale: float):
+    """fp64 CQS-decomposed backward: the merged statistics of the whole row
+    (lse_i, and D_i = <dout_i, out_i> from the decomposed forward), then, task
+    by task, the gradient terms of the chunk pairs the task's CQS mask allows
+    (P recomputed from the merged lse), summed over tasks.
+
+    Returns (dq, dk, dv), each [N, H, d] float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    N, H, d = q.shape
+    out, lse = decomposed_attention(q, k, v, ls, causal, scale)
+    D = np.einsum("ihd,ihd->ih", dout, out)                      # [N, H]
+    P = 1
+    for l in ls:
+        P *= cqs_chunk_count(l)
+    B = N // P
+    pos = np.arange(N)
+    dq = np.zeros((N, H, d))
+    dk = np.zeros((N, H, d))
+    dv = np.zeros((N, H, d))
+    for t in leaf_tasks(P, ls):
+        ps = causal_pairs(t.pairs) if causal else t.pairs
+        for (qb, kb) in ps:
+            rows = pos[qb * B:(qb + 1) * B]
+            keys = pos[kb * B:(kb + 1) * B]
+            s = np.einsum("ihd,jhd->hij", q[rows], k[keys]) * scale
+            p = np.exp(s - lse[rows].T[:, :, None])             # [H, rows, keys]
+            if causal:
+                p = np.where((keys[None, :] <= rows[:, None])[None], p, 0.0)
+            dp = np.einsum("ihd,jhd->hij", dout[rows], v[keys])
+            ds = p * (dp - D[rows].T[:, :, None])
+            dq[rows] += scale * np.einsum("hij,jhd->ihd", ds, k[keys])
+            dk[keys] += scale * np.einsum("hij,ihd->jhd", ds, q[rows])
+            dv[keys] += np.einsum("hij,ihd->jhd", p, dout[rows])
+    return dq, dk, dv
