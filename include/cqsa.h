@@ -141,13 +141,15 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out);
 /*
  * cqsa_forward -- run the planned attention ([A]; [B] "Implementation").
  *   host_or_device = CQSA_DEVICE: q, k, v, out, lse are device pointers on the
- *     current device.  Every task runs from HBM; partials go to the plan's
- *     arena and one merge writes out and lse.
+ *     current device.  Every task runs from HBM.  CQSA_MERGE_SLOTS plans write
+ *     the tasks' partials to the plan's arena and one merge writes out and
+ *     lse; CQSA_MERGE_FUSED plans write out and lse from the tile kernel.
  *   host_or_device = CQSA_HOST: all five are page-locked host pointers
  *     (cudaHostAlloc / pinned torch tensors).  Tasks are streamed: each
- *     task's Q/K/V blocks are copied in on a copy stream, double buffered,
- *     computed, merged into device-resident accumulators of the current head
- *     group, and finished blocks are copied back.
+ *     task's missing Q/K/V blocks are copied into a device block cache on a
+ *     copy stream, computed, folded into device-resident accumulators of the
+ *     current head group in the kernel's epilogue, and finished blocks are
+ *     copied back.
  *   stream: a cudaStream_t (0 = legacy default stream) the call is ordered
  *     after and that is ordered after all of its work.
  * Asynchronous: returns once all work is enqueued.  The first call on a plan
@@ -158,6 +160,32 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out);
 cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,
                            const void *v, void *out, float *lse,
                            int host_or_device, void *stream);
+
+/*
+ * cqsa_backward -- gradients of the planned attention with respect to q, k,
+ * v, given the forward's out and lse and the gradient dout of the loss with
+ * respect to out.  The pages report the method's backward-gradient error and
+ * forward-backward runtime ([A]) and backward memory ([B] "Precise
+ * Scaling"); they do not spell the backward out.  Reading used here: with
+ * the merged row statistics lse_i and D_i = <dout_i, out_i>, every allowed
+ * (query, key) pair lies in exactly one task and contributes
+ *     P = exp(s - lse_i),  dS = P (<dout_i, v_j> - D_i),
+ *     dq_i += dS k_j / sqrt(d),  dk_j += dS q_i / sqrt(d),  dv_j += P dout_i
+ * independently of the other pairs, so the tasks' partial gradients sum to
+ * the exact gradients.
+ *   Layouts: q, k, v, out, dout, dq, dk, dv [N, H, d] contiguous in the plan
+ *     dtype; lse fp32 [H, N] as cqsa_forward wrote it.  The caller owns all.
+ *   host_or_device: CQSA_DEVICE only (all ten pointers on the current
+ *     device); CQSA_HOST returns UNSUPPORTED.
+ *   CQSA_MERGE_SLOTS plans write each (task, query block) dq partial and
+ *     each (task, key block) dk / dv partial to slots of a backward arena
+ *     (allocated on the first call) and sum them; CQSA_MERGE_FUSED plans
+ *     walk all the tasks of a block in one CTA and write dq, dk, dv directly.
+ * Asynchronous on stream.  Errors: INVALID_ARG, UNSUPPORTED, CUDA, NO_DEVICE.
+ */
+cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
+                            const void *out, const float *lse, const void *dout, void *dq, void *dk,
+                            void *dv, int host_or_device, void *stream);
 
 /* cqsa_plan_sync -- wait for the plan's work on `stream` and report any
  * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync. */
@@ -198,6 +226,8 @@ typedef struct {
     int64_t merge_launches; /* log-sum-exp merge kernel launches */
     double attn_ms;         /* summed device time of those launches */
     double merge_ms;
+    int64_t bwd_launches;   /* backward gradient kernel launches (dq and dk/dv) */
+    double bwd_ms;
 } cqsa_kernel_stats_t;
 
 /* cqsa_plan_profile -- enable != 0: from the next forward on, record a CUDA

@@ -34,7 +34,7 @@ MAX_L = 16
 
 # Every symbol include/cqsa.h declares.
 EXPORTS = (
-    "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_plan_sync", "cqsa_plan_info",
+    "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_backward", "cqsa_plan_sync", "cqsa_plan_info",
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error",
@@ -81,7 +81,8 @@ class PlanInfo(ctypes.Structure):
 
 class KernelStats(ctypes.Structure):
     _fields_ = [("attn_launches", ctypes.c_int64), ("merge_launches", ctypes.c_int64),
-                ("attn_ms", ctypes.c_double), ("merge_ms", ctypes.c_double)]
+                ("attn_ms", ctypes.c_double), ("merge_ms", ctypes.c_double),
+                ("bwd_launches", ctypes.c_int64), ("bwd_ms", ctypes.c_double)]
 
 
 class Entry(ctypes.Structure):
@@ -108,6 +109,7 @@ def load_library():
                            ctypes.c_int, ctypes.c_size_t, ctypes.POINTER(P)]),
         "cqsa_plan_ex": (st, [ctypes.POINTER(PlanDesc), ctypes.POINTER(P)]),
         "cqsa_forward": (st, [P, P, P, P, P, P, ctypes.c_int, P]),
+        "cqsa_backward": (st, [P, P, P, P, P, P, P, P, P, P, ctypes.c_int, P]),
         "cqsa_plan_sync": (st, [P, P]),
         "cqsa_plan_info": (st, [P, ctypes.POINTER(PlanInfo)]),
         "cqsa_plan_task_blocks": (st, [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64,
@@ -187,7 +189,8 @@ class Plan:
         ks = KernelStats()
         _check(load_library().cqsa_plan_kernel_stats(self.handle, ctypes.byref(ks), int(bool(reset))))
         return {"attn_launches": ks.attn_launches, "merge_launches": ks.merge_launches,
-                "attn_ms": ks.attn_ms, "merge_ms": ks.merge_ms}
+                "attn_ms": ks.attn_ms, "merge_ms": ks.merge_ms,
+                "bwd_launches": ks.bwd_launches, "bwd_ms": ks.bwd_ms}
 
     def destroy(self):
         if self.handle and self.handle.value:
@@ -244,6 +247,29 @@ def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVIC
     _check(load_library().cqsa_forward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                        out.data_ptr(), lse.data_ptr(), host_or_device,
                                        ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_backward(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, host_or_device: int = CQSA_DEVICE,
+                  stream=None):
+    """Gradients dq, dk, dv of the planned attention given the forward's out
+    and lse and the output gradient dout.  All [N, H, d] contiguous device
+    tensors in the plan's dtype except lse (fp32 [H, N]).  Asynchronous on
+    ``stream``."""
+    import torch
+    named = (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv))
+    for name, t in named + (("lse", lse),):
+        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous torch tensor")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be float32")
+    if len({t.dtype for _, t in named}) != 1 or len({tuple(t.shape) for _, t in named}) != 1 or q.dim() != 3:
+        raise ValueError("q, k, v, out, dout, dq, dk, dv must share a dtype and an [N, H, d] shape")
+    N, H, _ = q.shape
+    if tuple(lse.shape) != (H, N):
+        raise ValueError("lse must be [H, N]")
+    _check(load_library().cqsa_backward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                        dv.data_ptr(), host_or_device, ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def cqsa_forward_noalloc(plan: Plan, q, k, v, out, lse, stream=None):

@@ -154,6 +154,13 @@ struct cqsa_plan {
     int32_t *dev_nslots = nullptr;
     DevWl dev_wl;
 
+    // Backward (device mode): D, partial-gradient slots, work lists.
+    char *bwd_arena = nullptr;
+    size_t bwd_bytes = 0;
+    float *bwd_delta = nullptr, *bwd_dq = nullptr, *bwd_dk = nullptr, *bwd_dv = nullptr;
+    int32_t *bwd_q_nslots = nullptr, *bwd_kv_nslots = nullptr;
+    DevWl bwd_qwl, bwd_kvwl;
+
     // Streamed path.
     char *host_arena = nullptr;
     size_t host_bytes = 0;
@@ -180,7 +187,8 @@ struct cqsa_plan {
 
 namespace {
 
-// Event pair around one launch when profiling is on (kind 0 attention, 1 merge).
+// Event pair around one launch when profiling is on (kind 0 attention, 1 merge
+// or slot sum, 2 backward gradients).
 struct LaunchTimer {
     cqsa_plan_t *P;
     cudaStream_t s;
@@ -422,6 +430,111 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     return CQSA_OK;
 }
 
+cqsa_status_t setup_backward(cqsa_plan_t *P) {
+    if (P->bwd_arena) return CQSA_OK;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    const bool fused = pl.spec.fused != 0;
+    WorkList qwl = pl.device_worklist(64, 64, H);
+    int64_t max_kv = 0;
+    WorkList kvwl = pl.device_worklist_kv(64, 64, H, &max_kv);
+    std::vector<int32_t> kv_ns(pl.num_blocks, 0);
+    for (const WlEntry &e : kvwl.entries) {
+        const int64_t kb = e.q_lo / pl.block;
+        kv_ns[kb] = std::max<int32_t>(kv_ns[kb], e.slot + 1);
+    }
+    const size_t slot = (size_t)N * H * d * sizeof(float);
+    ArenaLayout a;
+    const size_t o_delta = a.take((size_t)H * N * sizeof(float));
+    size_t o_dq = 0, o_dk = 0, o_dv = 0, o_qns = 0, o_kvns = 0;
+    if (!fused) {
+        o_dq = a.take((size_t)pl.max_slots * slot);
+        o_dk = a.take((size_t)max_kv * slot);
+        o_dv = a.take((size_t)max_kv * slot);
+        o_qns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+        o_kvns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+    }
+    const size_t o_qwl = a.take(wl_region(qwl));
+    const size_t o_kvwl = a.take(wl_region(kvwl));
+    char *arena = nullptr;
+    CK(cudaMalloc(&arena, a.total));
+    P->bwd_arena = arena;
+    P->bwd_bytes = a.total;
+    P->bwd_delta = reinterpret_cast<float *>(arena + o_delta);
+    if (!fused) {
+        P->bwd_dq = reinterpret_cast<float *>(arena + o_dq);
+        P->bwd_dk = reinterpret_cast<float *>(arena + o_dk);
+        P->bwd_dv = reinterpret_cast<float *>(arena + o_dv);
+        P->bwd_q_nslots = reinterpret_cast<int32_t *>(arena + o_qns);
+        P->bwd_kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
+        CK(cudaMemcpy(P->bwd_q_nslots, pl.slots_per_block.data(), pl.num_blocks * sizeof(int32_t),
+                      cudaMemcpyHostToDevice));
+        CK(cudaMemcpy(P->bwd_kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
+    }
+    std::vector<char> b1 = pack_wl(qwl), b2 = pack_wl(kvwl);
+    if (!b1.empty()) CK(cudaMemcpy(arena + o_qwl, b1.data(), b1.size(), cudaMemcpyHostToDevice));
+    if (!b2.empty()) CK(cudaMemcpy(arena + o_kvwl, b2.data(), b2.size(), cudaMemcpyHostToDevice));
+    P->bwd_qwl = place_wl(arena + o_qwl, qwl);
+    P->bwd_kvwl = place_wl(arena + o_kvwl, kvwl);
+    return CQSA_OK;
+}
+
+cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, const void *v, const void *out,
+                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              cudaStream_t stream) {
+    cqsa_status_t st = setup_backward(P);
+    if (st != CQSA_OK) return st;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    const bool fused = pl.spec.fused != 0;
+    CK(launch_bwd_delta(d, P->elem, out, dout, N, H, P->bwd_delta, stream));
+    BwdParams bp{};
+    bp.q = q;
+    bp.k = k;
+    bp.v = v;
+    bp.dout = dout;
+    bp.lse = lse;
+    bp.delta = P->bwd_delta;
+    bp.N = N;
+    bp.H = H;
+    bp.causal = pl.spec.causal;
+    bp.scale = 1.0f / std::sqrt((float)d);
+    {
+        BwdParams p = bp;
+        p.entries = P->bwd_qwl.entries;
+        p.runs = P->bwd_qwl.runs;
+        p.units = P->bwd_qwl.units;
+        p.part_a = P->bwd_dq;
+        p.out_a = dq;
+        LaunchTimer tm(P, stream, 2);
+        CK(launch_bwd_dq(d, P->elem, p, P->bwd_qwl.num_units, stream));
+        tm.stop();
+    }
+    {
+        BwdParams p = bp;
+        p.entries = P->bwd_kvwl.entries;
+        p.runs = P->bwd_kvwl.runs;
+        p.units = P->bwd_kvwl.units;
+        p.part_a = P->bwd_dk;
+        p.part_b = P->bwd_dv;
+        p.out_a = dk;
+        p.out_b = dv;
+        LaunchTimer tm(P, stream, 2);
+        CK(launch_bwd_dkdv(d, P->elem, p, P->bwd_kvwl.num_units, stream));
+        tm.stop();
+    }
+    if (!fused) {
+        LaunchTimer tm(P, stream, 1);
+        CK(launch_sum_slots(d, P->elem, P->bwd_dq, P->bwd_q_nslots, pl.block, N, H, dq, stream));
+        CK(launch_sum_slots(d, P->elem, P->bwd_dk, P->bwd_kv_nslots, pl.block, N, H, dk, stream));
+        CK(launch_sum_slots(d, P->elem, P->bwd_dv, P->bwd_kv_nslots, pl.block, N, H, dv, stream));
+        tm.stop();
+    }
+    return CQSA_OK;
+}
+
 // Copies `rows` token rows of heads [h0, h0+g) between a full [*, H, d]
 // tensor and a compact [*, g, d] one.
 cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width, size_t rows,
@@ -638,6 +751,22 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
     return host ? forward_host(plan, q, k, v, out, lse, s) : forward_device(plan, q, k, v, out, lse, s);
 }
 
+cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, const void *out,
+                            const float *lse, const void *dout, void *dq, void *dk, void *dv, int host_or_device,
+                            void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    if (host_or_device == CQSA_HOST)
+        return fail(CQSA_ERR_UNSUPPORTED, "the backward runs in device mode only");
+    if (host_or_device != CQSA_DEVICE) return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be 0 or 1");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+    const char *names[] = {"q", "k", "v", "out", "lse", "dout", "dq", "dk", "dv"};
+    for (int i = 0; i < 9; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    return backward_device(plan, q, k, v, out, lse, dout, dq, dk, dv, static_cast<cudaStream_t>(stream));
+}
+
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
@@ -679,6 +808,9 @@ cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *sta
         if (t.kind == 0) {
             plan->totals.attn_launches++;
             plan->totals.attn_ms += ms;
+        } else if (t.kind == 2) {
+            plan->totals.bwd_launches++;
+            plan->totals.bwd_ms += ms;
         } else {
             plan->totals.merge_launches++;
             plan->totals.merge_ms += ms;
@@ -775,7 +907,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
         cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);
-        if (plan->dev_arena) cudaDeviceSynchronize();
+        if (plan->dev_arena || plan->bwd_arena) cudaDeviceSynchronize();
         for (int s = 0; s < 2; ++s) {
             if (plan->ev_in_ready[s]) cudaEventDestroy(plan->ev_in_ready[s]);
             if (plan->ev_in_free[s]) cudaEventDestroy(plan->ev_in_free[s]);
@@ -794,6 +926,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
             if (s) cudaStreamDestroy(s);
         if (plan->dev_arena) cudaFree(plan->dev_arena);
         if (plan->host_arena) cudaFree(plan->host_arena);
+        if (plan->bwd_arena) cudaFree(plan->bwd_arena);
         cudaGetLastError();
     }
     delete plan;

@@ -52,6 +52,39 @@ cudaError_t launch_attn_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, 
 cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k, const void *v,
                              const AttnParams &p, int num_units, cudaStream_t stream);
 
+// Backward (attn_bwd.cu).  The gradients of each task's allowed pairs, with
+// P recomputed from the merged lse: D_i = <dO_i, O_i>, P = exp(s - lse_i),
+// dS = P (dP - D_i), dq_i += scale dS k_j, dk_j += scale dS q_i,
+// dv_j += P dO_i.  Partial gradients of a task go to slot e.slot of
+// part_* ([slot][N][H][d] fp32); an entry flagged SEG_FIRST | SEG_LAST
+// (fused plans) writes its finished rows to out* in the input dtype.
+struct BwdParams {
+    const WlEntry *entries;
+    const WlRun *runs;
+    const WlUnit *units;
+    const void *q, *k, *v, *dout;
+    const float *lse;    // [H][N], natural log
+    const float *delta;  // [H][N]
+    int64_t N;
+    int H;
+    int causal;
+    float scale;         // 1 / sqrt(d)
+    float *part_a;       // dq, or dk
+    float *part_b;       // dv
+    void *out_a;         // dq, or dk (input dtype)
+    void *out_b;         // dv
+};
+
+cudaError_t launch_bwd_delta(int d, int elem_bytes, const void *out, const void *dout, int64_t N, int H,
+                             float *delta, cudaStream_t stream);
+// Query-stationary: 64 query rows per unit, key tiles of 64.
+cudaError_t launch_bwd_dq(int d, int elem_bytes, const BwdParams &p, int num_units, cudaStream_t stream);
+// Key-stationary: 64 key rows per unit, query tiles of 64.
+cudaError_t launch_bwd_dkdv(int d, int elem_bytes, const BwdParams &p, int num_units, cudaStream_t stream);
+// out[r][h][:] = sum over the nslots[r / block] slots of part[s][r][h][:].
+cudaError_t launch_sum_slots(int d, int elem_bytes, const float *part, const int32_t *nslots, int64_t block,
+                             int64_t N, int H, void *out, cudaStream_t stream);
+
 // Log-sum-exp recomposition of a query block's partials (merge.cu).
 //   out[r][h][:] = sum_j exp(lse_j - lse) O_j,  lse = log sum_j exp(lse_j)
 // over the nslots[r / block] partials of row r.  out in the input dtype.

@@ -280,6 +280,72 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     return wl;
 }
 
+WorkList Planner::device_worklist_kv(int rows_per_unit, int bn, int heads, int64_t *max_kv_slots) const {
+    // kb -> (task, query blocks) in task order; pairs come from the forward
+    // entries, whose key runs already carry every level's CQS mask.
+    std::vector<std::vector<std::pair<int64_t, std::vector<int64_t>>>> by_kb(num_blocks);
+    for (const Entry &e : entries)
+        for (const KeyRun &r : e.runs)
+            for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
+                auto &lst = by_kb[kb];
+                if (spec.fused) {
+                    if (lst.empty()) lst.push_back({0, {}});
+                    lst.back().second.push_back(e.qb);
+                } else {
+                    if (lst.empty() || lst.back().first != e.task) lst.push_back({e.task, {}});
+                    lst.back().second.push_back(e.qb);
+                }
+            }
+    WorkList wl;
+    std::vector<int64_t> group;
+    *max_kv_slots = 0;
+    for (int64_t kb = 0; kb < num_blocks; ++kb) {
+        int32_t slot = 0;
+        for (auto &tq : by_kb[kb]) {
+            std::vector<int64_t> &qs = tq.second;
+            std::sort(qs.begin(), qs.end());
+            WlEntry w{};
+            w.q_lo = (int32_t)(kb * block);
+            w.q_hi = (int32_t)((kb + 1) * block);
+            w.slot = slot++;
+            w.out_lo = w.q_lo;
+            w.flags = spec.fused ? (SEG_FIRST | SEG_LAST) : 0;
+            w.run_begin = (int32_t)wl.runs.size();
+            for (size_t i = 0; i < qs.size(); ++i) {
+                if (i > 0 && qs[i] == qs[i - 1] + 1) {
+                    wl.runs.back().k_hi = (int32_t)((qs[i] + 1) * block);
+                } else {
+                    WlRun x{};
+                    x.k_lo = (int32_t)(qs[i] * block);
+                    x.k_hi = (int32_t)((qs[i] + 1) * block);
+                    wl.runs.push_back(x);
+                }
+            }
+            w.run_count = (int32_t)wl.runs.size() - w.run_begin;
+            wl.entries.push_back(w);
+            group.push_back(tq.first);
+        }
+        *max_kv_slots = std::max<int64_t>(*max_kv_slots, slot);
+    }
+    std::vector<WlUnit> u;
+    for (int32_t ei = 0; ei < (int32_t)wl.entries.size(); ++ei) {
+        const WlEntry &e = wl.entries[ei];
+        for (int h = 0; h < heads; ++h)
+            for (int32_t k0 = e.q_lo; k0 < e.q_hi; k0 += rows_per_unit) {
+                WlUnit x{ei, k0, h, unit_query_tiles(e, wl.runs.data(), k0, spec.causal, bn)};
+                if (x.ntiles > 0) u.push_back(x);
+            }
+    }
+    std::stable_sort(u.begin(), u.end(), [&](const WlUnit &a, const WlUnit &b) {
+        const int ca = a.ntiles / 32, cb = b.ntiles / 32;
+        if (ca != cb) return ca > cb;
+        if (a.head != b.head) return a.head < b.head;
+        return group[a.entry] < group[b.entry];
+    });
+    wl.units.swap(u);
+    return wl;
+}
+
 WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const {
     // Q rows come from Q slot q_slot * block, K and V rows from KV slot
     // kv_slot * block; partial outputs go to the task's local rows mq * block.

@@ -114,6 +114,12 @@ public:
     // output directly; otherwise one entry per (task, query block) with a
     // partial slot.
     WorkList device_worklist(int rows_per_unit, int bn, int heads) const;
+    // Key-stationary work list for the key and value gradients: one entry
+    // per (task, key block) with the runs of query blocks the task's mask
+    // allows (with spec.fused: one entry per key block over all tasks).
+    // kv_slot of each entry numbers the tasks of a key block (partial slots);
+    // *max_kv_slots gets the most any block has.
+    WorkList device_worklist_kv(int rows_per_unit, int bn, int heads, int64_t *max_kv_slots) const;
     // Work list of leaf t reading Q, K, V from the block pools of `pool`.
     WorkList leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const;
     // Merge segments of leaf t in host mode (one per query block with an

@@ -94,4 +94,28 @@ CQSA_HD int32_t unit_key_tiles(const WlEntry &e, const WlRun *runs, int32_t q0,
     return n;
 }
 
+// Transposed work lists (key-stationary, for the key and value gradients):
+// an entry's rows [q_lo, q_hi) are key rows with offset q_goff, and its runs
+// are query rows.  Under the causal rule a query before the unit's first key
+// attends to none of the unit's keys, so runs start at that key.
+CQSA_HD void clip_run_t(const WlEntry &e, const WlRun &r, int32_t k0, int causal, int32_t *lo,
+                        int32_t *hi) {
+    *lo = r.k_lo;
+    *hi = r.k_hi;
+    if (causal) {
+        const int64_t lim = (int64_t)k0 + e.q_goff - r.k_goff;  // first local query row kept
+        if (lim > *lo) *lo = (int32_t)(lim < *hi ? lim : *hi);
+    }
+}
+
+CQSA_HD int32_t unit_query_tiles(const WlEntry &e, const WlRun *runs, int32_t k0, int causal, int32_t bm) {
+    int32_t n = 0;
+    for (int32_t r = 0; r < e.run_count; ++r) {
+        int32_t lo, hi;
+        clip_run_t(e, runs[e.run_begin + r], k0, causal, &lo, &hi);
+        if (hi > lo) n += (hi - lo + bm - 1) / bm;
+    }
+    return n;
+}
+
 }  // namespace cqsa

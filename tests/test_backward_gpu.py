@@ -1,0 +1,109 @@
+"""GPU parity of the backward: cqsa_backward through the C ABI (fed the
+library's own forward out and lse, as a caller would) against the fp64
+oracle's gradients on the same seeded inputs and output gradient.
+
+Tolerances (a reading; the benchmark spec states none for gradients), relative
+to the largest reference gradient entry g_max of each tensor:
+  fp32 inputs: max|err| <= 1e-4 g_max + 1e-6 (fp32 arithmetic throughout).
+  bf16 inputs: max|err| <= 2e-2 g_max and relative Frobenius error <= 1e-2:
+  the forward's bf16 out enters D_i = <dout_i, out_i> (2^-9 relative) and the
+  gradients are rounded to bf16 (2^-9 relative)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from out_core_scheduling_b200 import cqsa
+from out_core_scheduling_b200.inputs import make_qkv
+
+from parity import run
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+GTOL = {torch.float32: dict(rel_max=1e-4, abs_max=1e-6, rel_fro=None),
+        torch.bfloat16: dict(rel_max=2e-2, abs_max=0.0, rel_fro=1e-2)}
+
+
+def _grads(plan, q, k, v, dout):
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    plan.sync()
+    return dq, dk, dv
+
+
+def _compare(got, ref, dtype, name):
+    tol = GTOL[dtype]
+    g = got.cpu().double().numpy()
+    assert np.all(np.isfinite(g)), name
+    gmax = np.abs(ref).max()
+    err = np.abs(g - ref)
+    assert err.max() <= tol["rel_max"] * gmax + tol["abs_max"], (name, err.max(), gmax)
+    if tol["rel_fro"] is not None:
+        fro = np.linalg.norm(g - ref) / np.linalg.norm(ref)
+        assert fro <= tol["rel_fro"], (name, fro)
+
+
+def _check_all(N, H, d, ls, dtype, causal, merge, seed):
+    q, k, v = make_qkv(N, H, d, dtype=dtype, seed=seed, device=DEV)
+    dout = make_qkv(N, H, d, dtype=dtype, seed=seed + 1000, device=DEV)[0]
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, merge=merge)
+    dq, dk, dv = _grads(plan, q, k, v, dout)
+    qc, kc, vc, dc = (x.cpu() for x in (q, k, v, dout))
+    ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
+    ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, causal=causal)
+    _compare(dq, ref_dq, dtype, "dq")
+    _compare(dk, ref_dk, dtype, "dk")
+    _compare(dv, ref_dv, dtype, "dv")
+
+
+CASES = [
+    # (N, H, d, levels, dtype)
+    (7 * 128, 2, 128, [3], torch.bfloat16),
+    (7 * 128, 2, 64, [3], torch.bfloat16),
+    (7 * 100, 2, 128, [3], torch.bfloat16),      # blocks not a multiple of the tile
+    (13 * 64, 2, 128, [4], torch.bfloat16),
+    (91 * 16, 1, 64, [4, 3], torch.bfloat16),    # two levels
+    (7 * 3, 1, 64, [3], torch.bfloat16),         # blocks smaller than a tile
+    (7 * 128, 1, 64, [3], torch.float32),
+    (7 * 100, 2, 128, [3], torch.float32),
+]
+
+
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"n{c[0]}-h{c[1]}-d{c[2]}-l{c[3]}-{str(c[4])[6:]}")
+def test_backward_matches_oracle(case, causal, merge):
+    N, H, d, ls, dtype = case
+    _check_all(N, H, d, ls, dtype, causal, merge, seed=30)
+
+
+def test_backward_gradient_identities_full_size():
+    """At the l=4, N=53248, H=8, d=128 workload: sum_j dk_j = 0 and
+    sum_j dv_j = sum_i dout_i per head and feature (softmax rows sum to one),
+    to the rounding of the bf16 gradients."""
+    N, H, d = 53248, 8, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
+    dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=1000, device=DEV)[0]
+    for causal in (False, True):
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal)
+        dq, dk, dv = _grads(plan, q, k, v, dout)
+        sk = dk.double().sum(0)
+        sv = dv.double().sum(0)
+        sd = dout.double().sum(0)
+        scale_k = dk.double().abs().sum(0)
+        assert (sk.abs() <= 1e-2 * scale_k + 1e-3).all()
+        assert ((sv - sd).abs() <= 1e-2 * dv.double().abs().sum(0) + 1e-3).all()
+        assert torch.isfinite(dq.float()).all()
+
+
+def test_backward_rejects_host_mode():
+    N, H, d = 7 * 64, 1, 64
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
+    plan = cqsa.cqsa_plan(N, H, d, 3)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    g = [torch.empty_like(q) for _ in range(3)]
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_backward(plan, q, k, v, out, lse, q, *g, host_or_device=cqsa.CQSA_HOST)
+    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
