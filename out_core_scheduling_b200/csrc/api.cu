@@ -157,6 +157,7 @@ struct cqsa_plan {
     // Backward (device mode): D, partial-gradient slots, work lists.
     char *bwd_arena = nullptr;
     size_t bwd_bytes = 0;
+    int *bwd_err = nullptr;
     float *bwd_delta = nullptr, *bwd_dq = nullptr, *bwd_dk = nullptr, *bwd_dv = nullptr;
     int32_t *bwd_q_nslots = nullptr, *bwd_kv_nslots = nullptr;
     DevWl bwd_qwl, bwd_kvwl;
@@ -436,9 +437,11 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
     const bool fused = pl.spec.fused != 0;
-    WorkList qwl = pl.device_worklist(64, 64, H);
+    // bf16: tensor-core kernels on 128-row tiles; fp32: CUDA-core kernels on 64.
+    const int rows = P->dtype == CQSA_BF16 ? 128 : 64;
+    WorkList qwl = pl.device_worklist(rows, rows, H);
     int64_t max_kv = 0;
-    WorkList kvwl = pl.device_worklist_kv(64, 64, H, &max_kv);
+    WorkList kvwl = pl.device_worklist_kv(rows, rows, H, &max_kv);
     std::vector<int32_t> kv_ns(pl.num_blocks, 0);
     for (const WlEntry &e : kvwl.entries) {
         const int64_t kb = e.q_lo / pl.block;
@@ -446,6 +449,7 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     }
     const size_t slot = (size_t)N * H * d * sizeof(float);
     ArenaLayout a;
+    const size_t o_err = a.take(256);
     const size_t o_delta = a.take((size_t)H * N * sizeof(float));
     size_t o_dq = 0, o_dk = 0, o_dv = 0, o_qns = 0, o_kvns = 0;
     if (!fused) {
@@ -461,6 +465,8 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     CK(cudaMalloc(&arena, a.total));
     P->bwd_arena = arena;
     P->bwd_bytes = a.total;
+    CK(cudaMemset(arena, 0, 256));
+    P->bwd_err = reinterpret_cast<int *>(arena + o_err);
     P->bwd_delta = reinterpret_cast<float *>(arena + o_delta);
     if (!fused) {
         P->bwd_dq = reinterpret_cast<float *>(arena + o_dq);
@@ -489,6 +495,13 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
     const bool fused = pl.spec.fused != 0;
+    CUtensorMap mq{}, mk{}, mv{}, mo{};
+    if (P->dtype == CQSA_BF16) {
+        if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mk, k, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mv, v, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mo, dout, N, H, d)) != CQSA_OK) return st;
+    }
     CK(launch_bwd_delta(d, P->elem, out, dout, N, H, P->bwd_delta, stream));
     BwdParams bp{};
     bp.q = q;
@@ -509,7 +522,10 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
         p.part_a = P->bwd_dq;
         p.out_a = dq;
         LaunchTimer tm(P, stream, 2);
-        CK(launch_bwd_dq(d, P->elem, p, P->bwd_qwl.num_units, stream));
+        if (P->dtype == CQSA_BF16)
+            CK(launch_bwd_dq_tc(d, mq, mk, mv, mo, p, P->bwd_qwl.num_units, P->timeout_ns, P->bwd_err, stream));
+        else
+            CK(launch_bwd_dq(d, P->elem, p, P->bwd_qwl.num_units, stream));
         tm.stop();
     }
     {
@@ -522,7 +538,11 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
         p.out_a = dk;
         p.out_b = dv;
         LaunchTimer tm(P, stream, 2);
-        CK(launch_bwd_dkdv(d, P->elem, p, P->bwd_kvwl.num_units, stream));
+        if (P->dtype == CQSA_BF16)
+            CK(launch_bwd_dkdv_tc(d, mq, mk, mv, mo, p, P->bwd_kvwl.num_units, P->timeout_ns, P->bwd_err,
+                                  stream));
+        else
+            CK(launch_bwd_dkdv(d, P->elem, p, P->bwd_kvwl.num_units, stream));
         tm.stop();
     }
     if (!fused) {
@@ -771,7 +791,7 @@ cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
     CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-    int *words[2] = {plan->dev_err, plan->h_err};
+    int *words[3] = {plan->dev_err, plan->h_err, plan->bwd_err};
     int bad = 0;
     for (int *w : words) {
         if (!w) continue;

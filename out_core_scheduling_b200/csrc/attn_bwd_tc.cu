@@ -1,0 +1,614 @@
+// attn_bwd_tc.cu -- backward gradients on the sm_100a tensor cores (bf16 in,
+// fp32 accumulate): the per-task gradient terms of the CQS Divide.
+//
+// Same arithmetic as attn_bwd.cu (P = exp(s - lse_i), dS = P (dP - D_i);
+// dq += scale dS K, dk += scale dS^T Q, dv += P^T dO, with the merged row
+// statistics), on 128 x 128 tiles:
+//   bwd_dq_tc_kernel   one CTA per 128 query rows of a (task, query block)
+//                      entry; per allowed key tile: S = Q K^T and
+//                      dP = dO V^T (tcgen05, operands in shared memory by
+//                      TMA), dS in bf16 written over S in tensor memory,
+//                      then dQ += dS K with dS as the TMEM operand.
+//   bwd_dkdv_tc_kernel one CTA per 128 key rows of a (task, key block)
+//                      entry; per allowed query tile: S^T = K Q^T and
+//                      dP^T = V dO^T, P^T and dS^T in bf16 written over
+//                      them, then dV += P^T dO and dK += dS^T Q.
+// Warp roles (192 threads): warps 0-3 the elementwise step (one TMEM lane,
+// i.e. one stationary row, per thread), warp 4 TMA, warp 5 MMA.  Every wait
+// is bounded; on a timeout the CTA records DEV_TIMEOUT, drains its copies and
+// MMAs, frees its tensor memory and returns.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "worklist.h"
+
+namespace cqsa {
+namespace btc {
+
+constexpr int BM = 128;           // stationary rows per CTA
+constexpr int BN = 128;           // rows of an iterated tile
+constexpr int STAGES = 2;
+constexpr int THREADS = 192;
+constexpr int WARP_TMA = 4;
+constexpr int WARP_MMA = 5;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizzle
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int D>
+struct SmemDq {
+    static constexpr int KB = D / 64;
+    alignas(1024) uint8_t q[KB][BOX_BYTES];
+    alignas(1024) uint8_t dout[KB][BOX_BYTES];
+    alignas(1024) uint8_t k[STAGES][KB][BOX_BYTES];
+    alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
+    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, p_full, o_full, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int D>
+struct SmemKv {
+    static constexpr int KB = D / 64;
+    alignas(1024) uint8_t k[KB][BOX_BYTES];
+    alignas(1024) uint8_t v[KB][BOX_BYTES];
+    alignas(1024) uint8_t q[STAGES][KB][BOX_BYTES];
+    alignas(1024) uint8_t dout[STAGES][KB][BOX_BYTES];
+    float lse2[STAGES][BN];  // lse * log2(e) of the tile's query rows (+inf outside the run)
+    float dl[STAGES][BN];    // D of the tile's query rows
+    uint64_t bar_kv, qd_full[STAGES], qd_empty[STAGES], s_full, p_full, o_full, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ bool warp_wait_b(uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t tmo) {
+    bool ok = mbar_wait(bar, parity, abort, tmo);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void fence_regs32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive columns store.
+__device__ __forceinline__ void tmem_st16_b(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// SS MMA D[128 x 128] = A[128 x D] B[128 x D]^T, both K-major tiles.
+template <int D>
+__device__ __forceinline__ void mma_rows_dot(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+        mma_ss_elect(d_tmem, adesc + off, bdesc + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// TS MMA D[128 x D] (+)= A[128 x 128] (bf16 in TMEM at a_tmem, 2 per column)
+// times B[128 x D] with B's rows the K dimension, stored [rows][D] (MN-major).
+__device__ __forceinline__ void mma_tmem_rows(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              bool acc) {
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+        mma_ts_elect(d_tmem, a_tmem + (uint32_t)kk * 8u, bdesc + (uint64_t)(kk * (2048 >> 4)), idesc,
+                     (acc || kk > 0) ? 1u : 0u);
+}
+
+}  // namespace btc
+
+// ------------------------------------------------------------------ dq
+template <int D>
+__global__ void __launch_bounds__(btc::THREADS, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const BwdParams p, uint64_t tmo, int *err) {
+    using namespace btc;
+    constexpr int KB = D / 64;
+    constexpr uint32_t TILE = KB * BOX_BYTES;
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_TS = idesc_bf16_f32(BM, D, 0, 1);
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    SmemDq<D> &s = *reinterpret_cast<SmemDq<D> *>(smem_raw + pad);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WlUnit u = p.units[blockIdx.x];
+    const WlEntry e = p.entries[u.entry];
+    const int32_t q0 = u.q0;
+    const int head = u.head;
+    const int32_t q_end = min(q0 + BM, e.q_hi);
+    const int causal = p.causal;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.bar_q, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.kv_full[i], 1);
+            mbar_init(&s.kv_empty[i], 1);
+        }
+        mbar_init(&s.s_full, 1);
+        mbar_init(&s.p_full, 4);
+        mbar_init(&s.o_full, 1);
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(&s.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    volatile int *abort = &s.abort;
+    const int ntiles = unit_key_tiles(e, p.runs, q0, BM, causal, BN);
+
+    if (warp == WARP_TMA) {
+        if (lane == 0) {
+            mbar_expect_tx(&s.bar_q, 2 * TILE);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_3d(s.q[kb], &tmQ, &s.bar_q, kb * 64, head, q0);
+                tma_load_3d(s.dout[kb], &tmO, &s.bar_q, kb * 64, head, q0);
+            }
+            int j = 0;
+            bool ok = true;
+            for (int r = 0; r < e.run_count && ok; ++r) {
+                int32_t lo, hi;
+                clip_run(e, p.runs[e.run_begin + r], q_end, causal, &lo, &hi);
+                for (int32_t ks = lo; ks < hi; ks += BN, ++j) {
+                    const int st = j % STAGES;
+                    if (!mbar_wait(&s.kv_empty[st], ((uint32_t)(j / STAGES) & 1u) ^ 1u, abort, tmo)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&s.kv_full[st], 2 * TILE);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_load_3d(s.k[st][kb], &tmK, &s.kv_full[st], kb * 64, head, ks);
+                        tma_load_3d(s.v[st][kb], &tmV, &s.kv_full[st], kb * 64, head, ks);
+                    }
+                }
+            }
+            if (!ok) {
+                atomicExch(err, DEV_TIMEOUT);
+                int zero = 0;
+                mbar_wait(&s.bar_q, 0, (volatile int *)&zero, tmo);
+                for (int i = max(0, j - STAGES); i < j; ++i)
+                    mbar_wait(&s.kv_full[i % STAGES], (uint32_t)(i / STAGES) & 1u, (volatile int *)&zero, tmo);
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        bool ok = warp_wait_b(&s.bar_q, 0, abort, tmo);
+        const uint64_t qdesc = smem_desc_sw128(smem_u32(s.q[0]), 16, 1024);
+        const uint64_t odesc = smem_desc_sw128(smem_u32(s.dout[0]), 16, 1024);
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int st = j % STAGES;
+            if (!warp_wait_b(&s.kv_full[st], (uint32_t)(j / STAGES) & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            if (j > 0) {
+                // dQ += dS(j-1) K(j-1): dS was written over S.
+                if (!warp_wait_b(&s.p_full, (uint32_t)(j - 1) & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                const int sp = (j - 1) % STAGES;
+                mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[sp][0]), BOX_BYTES, 1024), IDESC_TS,
+                              j > 1);
+                mma_commit_elect(&s.kv_empty[sp]);
+            }
+            mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[st][0]), 16, 1024), IDESC_SS);
+            mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[st][0]), 16, 1024), IDESC_SS);
+            mma_commit_elect(&s.s_full);
+        }
+        if (ok && ntiles > 0) {
+            ok = warp_wait_b(&s.p_full, (uint32_t)(ntiles - 1) & 1u, abort, tmo);
+            if (ok) {
+                tc_fence_after();
+                const int sp = (ntiles - 1) % STAGES;
+                mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[sp][0]), BOX_BYTES, 1024), IDESC_TS,
+                              ntiles > 1);
+                mma_commit_elect(&s.kv_empty[sp]);
+            }
+        }
+        if (ok) {
+            mma_commit_elect(&s.o_full);
+        } else if (lane == 0) {
+            atomicExch(err, DEV_TIMEOUT);
+        }
+        mma_commit_elect(&s.drain);
+        int zero = 0;
+        mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
+        __syncwarp();
+    } else {
+        // Elementwise: thread = query row.
+        const int row = warp * 32 + lane;
+        const int32_t q_local = q0 + row;
+        const bool valid = q_local < q_end;
+        const int64_t q_glob = (int64_t)q_local + e.q_goff;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float sl2 = p.scale * LOG2E;
+        const float lse2 = valid ? p.lse[(int64_t)head * p.N + q_glob] * LOG2E : INFINITY;
+        const float dl = valid ? p.delta[(int64_t)head * p.N + q_glob] : 0.f;
+        bool ok = true;
+        int j = 0;
+        for (int r = 0; r < e.run_count && ok; ++r) {
+            const WlRun run = p.runs[e.run_begin + r];
+            int32_t lo, hi;
+            clip_run(e, run, q_end, causal, &lo, &hi);
+            for (int32_t ks = lo; ks < hi; ks += BN, ++j) {
+                if (!warp_wait_b(&s.s_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                int lim = min(BN, run.k_hi - ks);
+                if (causal) {
+                    const int64_t diag = q_glob - ((int64_t)ks + run.k_goff) + 1;
+                    if (diag < (int64_t)lim) lim = diag < 0 ? 0 : (int)diag;
+                }
+                if (!valid) lim = 0;
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    uint32_t sv[32], dp[32];
+                    tmem_ld32(lane_base + (uint32_t)(cc * 32), sv);
+                    tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp);
+                    tmem_wait_ld();
+                    fence_regs32(sv);
+                    fence_regs32(dp);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const int c = cc * 32 + t;
+                        const float p0 = c < lim ? ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, -lse2)) : 0.f;
+                        const float p1 =
+                            c + 1 < lim ? ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, -lse2)) : 0.f;
+                        pk[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[t]) - dl),
+                                                p1 * (__uint_as_float(dp[t + 1]) - dl));
+                    }
+                    tmem_st16_b(lane_base + (uint32_t)(cc * 16), pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.p_full);
+            }
+        }
+        if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
+        if (ok) {
+            tc_fence_after();
+            const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
+            const int64_t orow = (int64_t)e.out_lo + (q_local - e.q_lo);
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + 256u + (uint32_t)(cc * 32), o);
+                tmem_wait_ld();
+                fence_regs32(o);
+                if (valid) {
+                    if (fused) {
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out_a) + (orow * p.H + head) * D;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            uint2 w;
+                            w.x = pack_bf16x2(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale);
+                            w.y = pack_bf16x2(__uint_as_float(o[i + 2]) * p.scale,
+                                              __uint_as_float(o[i + 3]) * p.scale);
+                            *reinterpret_cast<uint2 *>(dst + cc * 32 + i) = w;
+                        }
+                    } else {
+                        float *dst = p.part_a + (((int64_t)e.slot * p.N + orow) * p.H + head) * D;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(dst + cc * 32 + i) =
+                                make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                            __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            atomicExch(err, DEV_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ dk, dv
+template <int D>
+__global__ void __launch_bounds__(btc::THREADS, 1)
+    bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       const BwdParams p, uint64_t tmo, int *err) {
+    using namespace btc;
+    constexpr int KB = D / 64;
+    constexpr uint32_t TILE = KB * BOX_BYTES;
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_TS = idesc_bf16_f32(BM, D, 0, 1);
+    constexpr uint32_t COL_DV = 256u, COL_DK = 256u + (uint32_t)D;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    SmemKv<D> &s = *reinterpret_cast<SmemKv<D> *>(smem_raw + pad);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WlUnit u = p.units[blockIdx.x];
+    const WlEntry e = p.entries[u.entry];
+    const int32_t k0 = u.q0;
+    const int head = u.head;
+    const int32_t k_end = min(k0 + BM, e.q_hi);
+    const int causal = p.causal;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.bar_kv, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.qd_full[i], 1);
+            mbar_init(&s.qd_empty[i], 1);
+        }
+        mbar_init(&s.s_full, 1);
+        mbar_init(&s.p_full, 4);
+        mbar_init(&s.o_full, 1);
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(&s.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    volatile int *abort = &s.abort;
+    const int ntiles = unit_query_tiles(e, p.runs, k0, causal, BN);
+
+    if (warp == WARP_TMA) {
+        // The whole warp stages each tile's lse and D; lane 0 issues the TMA.
+        if (lane == 0) {
+            mbar_expect_tx(&s.bar_kv, 2 * TILE);
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_3d(s.k[kb], &tmK, &s.bar_kv, kb * 64, head, k0);
+                tma_load_3d(s.v[kb], &tmV, &s.bar_kv, kb * 64, head, k0);
+            }
+        }
+        int i = 0;
+        bool ok = true;
+        for (int r = 0; r < e.run_count && ok; ++r) {
+            const WlRun run = p.runs[e.run_begin + r];
+            int32_t lo, hi;
+            clip_run_t(e, run, k0, causal, &lo, &hi);
+            for (int32_t qs = lo; qs < hi; qs += BN, ++i) {
+                const int st = i % STAGES;
+                if (!warp_wait_b(&s.qd_empty[st], ((uint32_t)(i / STAGES) & 1u) ^ 1u, abort, tmo)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int c = lane; c < BN; c += 32) {
+                    const int32_t row = qs + c;
+                    const bool in = row < run.k_hi;
+                    const int64_t g = (int64_t)row + run.k_goff;
+                    s.lse2[st][c] = in ? p.lse[(int64_t)head * p.N + g] * LOG2E : INFINITY;
+                    s.dl[st][c] = in ? p.delta[(int64_t)head * p.N + g] : 0.f;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_expect_tx(&s.qd_full[st], 2 * TILE);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_load_3d(s.q[st][kb], &tmQ, &s.qd_full[st], kb * 64, head, qs);
+                        tma_load_3d(s.dout[st][kb], &tmO, &s.qd_full[st], kb * 64, head, qs);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok && lane == 0) {
+            atomicExch(err, DEV_TIMEOUT);
+            int zero = 0;
+            mbar_wait(&s.bar_kv, 0, (volatile int *)&zero, tmo);
+            for (int x = max(0, i - STAGES); x < i; ++x)
+                mbar_wait(&s.qd_full[x % STAGES], (uint32_t)(x / STAGES) & 1u, (volatile int *)&zero, tmo);
+        }
+    } else if (warp == WARP_MMA) {
+        bool ok = warp_wait_b(&s.bar_kv, 0, abort, tmo);
+        const uint64_t kdesc = smem_desc_sw128(smem_u32(s.k[0]), 16, 1024);
+        const uint64_t vdesc = smem_desc_sw128(smem_u32(s.v[0]), 16, 1024);
+        auto grads = [&](int it) {
+            // dV += P^T dO, dK += dS^T Q for query tile `it` (P^T over S^T,
+            // dS^T over dP^T in tensor memory).
+            const int sp = it % STAGES;
+            mma_tmem_rows(tmem + COL_DV, tmem, smem_desc_sw128(smem_u32(s.dout[sp][0]), BOX_BYTES, 1024), IDESC_TS,
+                          it > 0);
+            mma_tmem_rows(tmem + COL_DK, tmem + 128u, smem_desc_sw128(smem_u32(s.q[sp][0]), BOX_BYTES, 1024),
+                          IDESC_TS, it > 0);
+            mma_commit_elect(&s.qd_empty[sp]);
+        };
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int st = i % STAGES;
+            if (!warp_wait_b(&s.qd_full[st], (uint32_t)(i / STAGES) & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            if (i > 0) {
+                if (!warp_wait_b(&s.p_full, (uint32_t)(i - 1) & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                grads(i - 1);
+            }
+            mma_rows_dot<D>(tmem, kdesc, smem_desc_sw128(smem_u32(s.q[st][0]), 16, 1024), IDESC_SS);
+            mma_rows_dot<D>(tmem + 128u, vdesc, smem_desc_sw128(smem_u32(s.dout[st][0]), 16, 1024), IDESC_SS);
+            mma_commit_elect(&s.s_full);
+        }
+        if (ok && ntiles > 0) {
+            ok = warp_wait_b(&s.p_full, (uint32_t)(ntiles - 1) & 1u, abort, tmo);
+            if (ok) {
+                tc_fence_after();
+                grads(ntiles - 1);
+            }
+        }
+        if (ok) {
+            mma_commit_elect(&s.o_full);
+        } else if (lane == 0) {
+            atomicExch(err, DEV_TIMEOUT);
+        }
+        mma_commit_elect(&s.drain);
+        int zero = 0;
+        mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
+        __syncwarp();
+    } else {
+        // Elementwise: thread = key row; columns are the tile's query rows.
+        const int row = warp * 32 + lane;
+        const int32_t k_local = k0 + row;
+        const bool valid = k_local < k_end;
+        const int64_t k_glob = (int64_t)k_local + e.q_goff;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float sl2 = p.scale * LOG2E;
+        bool ok = true;
+        int i = 0;
+        for (int r = 0; r < e.run_count && ok; ++r) {
+            const WlRun run = p.runs[e.run_begin + r];
+            int32_t lo, hi;
+            clip_run_t(e, run, k0, causal, &lo, &hi);
+            for (int32_t qs = lo; qs < hi; qs += BN, ++i) {
+                const int st = i % STAGES;
+                // qd_full makes the TMA warp's lse / D stores of this stage
+                // visible here (it completed before S^T was issued).
+                if (!warp_wait_b(&s.qd_full[st], (uint32_t)(i / STAGES) & 1u, abort, tmo)) { ok = false; break; }
+                if (!warp_wait_b(&s.s_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                // Query column c is kept iff c >= first (causal: at or after
+                // this key) and the row is inside the run (lse2 = +inf
+                // outside, so its P is 0).
+                int first = 0;
+                if (causal) {
+                    const int64_t f = k_glob - ((int64_t)qs + run.k_goff);
+                    first = f <= 0 ? 0 : (f > BN ? BN : (int)f);
+                }
+                if (!valid) first = BN;
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) {
+                    uint32_t sv[32], dp[32];
+                    tmem_ld32(lane_base + (uint32_t)(cc * 32), sv);
+                    tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp);
+                    tmem_wait_ld();
+                    fence_regs32(sv);
+                    fence_regs32(dp);
+                    uint32_t pp[16], pd[16];
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const int c = cc * 32 + t;
+                        const float p0 =
+                            c >= first ? ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, -s.lse2[st][c])) : 0.f;
+                        const float p1 = c + 1 >= first
+                                             ? ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, -s.lse2[st][c + 1]))
+                                             : 0.f;
+                        pp[t / 2] = pack_bf16x2(p0, p1);
+                        pd[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[t]) - s.dl[st][c]),
+                                                p1 * (__uint_as_float(dp[t + 1]) - s.dl[st][c + 1]));
+                    }
+                    tmem_st16_b(lane_base + (uint32_t)(cc * 16), pp);
+                    tmem_st16_b(lane_base + 128u + (uint32_t)(cc * 16), pd);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.p_full);
+            }
+        }
+        if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
+        if (ok) {
+            tc_fence_after();
+            const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
+            const int64_t orow = (int64_t)e.out_lo + (k_local - e.q_lo);
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? COL_DK : COL_DV;
+                const float mul = which == 0 ? p.scale : 1.f;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + col + (uint32_t)(cc * 32), o);
+                    tmem_wait_ld();
+                    fence_regs32(o);
+                    if (!valid) continue;
+                    if (fused) {
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? p.out_a : p.out_b) +
+                                             (orow * p.H + head) * D;
+#pragma unroll
+                        for (int x = 0; x < 32; x += 4) {
+                            uint2 w;
+                            w.x = pack_bf16x2(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul);
+                            w.y = pack_bf16x2(__uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
+                            *reinterpret_cast<uint2 *>(dst + cc * 32 + x) = w;
+                        }
+                    } else {
+                        float *dst = (which == 0 ? p.part_a : p.part_b) +
+                                     (((int64_t)e.slot * p.N + orow) * p.H + head) * D;
+#pragma unroll
+                        for (int x = 0; x < 32; x += 4)
+                            *reinterpret_cast<float4 *>(dst + cc * 32 + x) =
+                                make_float4(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul,
+                                            __uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            atomicExch(err, DEV_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int D, template <int> class SMEM, typename K>
+static cudaError_t launch_btc(K kernel, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                              const CUtensorMap &mo, const BwdParams &p, int units, uint64_t tmo, int *err,
+                              cudaStream_t st) {
+    const size_t smem = sizeof(SMEM<D>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<units, btc::THREADS, smem, st>>>(mq, mk, mv, mo, p, tmo, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dq_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const CUtensorMap &mo, const BwdParams &p, int num_units, uint64_t timeout_ns,
+                             int *err, cudaStream_t stream) {
+    if (num_units <= 0) return cudaSuccess;
+    if (d == 128)
+        return launch_btc<128, btc::SmemDq>(bwd_dq_tc_kernel<128>, mq, mk, mv, mo, p, num_units, timeout_ns, err,
+                                            stream);
+    if (d == 64)
+        return launch_btc<64, btc::SmemDq>(bwd_dq_tc_kernel<64>, mq, mk, mv, mo, p, num_units, timeout_ns, err,
+                                           stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dkdv_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                               const CUtensorMap &mo, const BwdParams &p, int num_units, uint64_t timeout_ns,
+                               int *err, cudaStream_t stream) {
+    if (num_units <= 0) return cudaSuccess;
+    if (d == 128)
+        return launch_btc<128, btc::SmemKv>(bwd_dkdv_tc_kernel<128>, mq, mk, mv, mo, p, num_units, timeout_ns,
+                                            err, stream);
+    if (d == 64)
+        return launch_btc<64, btc::SmemKv>(bwd_dkdv_tc_kernel<64>, mq, mk, mv, mo, p, num_units, timeout_ns, err,
+                                           stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace cqsa

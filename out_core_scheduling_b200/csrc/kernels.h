@@ -81,6 +81,15 @@ cudaError_t launch_bwd_delta(int d, int elem_bytes, const void *out, const void 
 cudaError_t launch_bwd_dq(int d, int elem_bytes, const BwdParams &p, int num_units, cudaStream_t stream);
 // Key-stationary: 64 key rows per unit, query tiles of 64.
 cudaError_t launch_bwd_dkdv(int d, int elem_bytes, const BwdParams &p, int num_units, cudaStream_t stream);
+// Tensor-core versions for bf16 (attn_bwd_tc.cu): 128 stationary rows per
+// unit, tiles of 128; maps describe q, k, v, dout as [rows, H, d] bf16 with a
+// {64, 1, 128} box.  Bounded waits report DEV_TIMEOUT in *err.
+cudaError_t launch_bwd_dq_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const CUtensorMap &mo, const BwdParams &p, int num_units, uint64_t timeout_ns,
+                             int *err, cudaStream_t stream);
+cudaError_t launch_bwd_dkdv_tc(int d, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                               const CUtensorMap &mo, const BwdParams &p, int num_units, uint64_t timeout_ns,
+                               int *err, cudaStream_t stream);
 // out[r][h][:] = sum over the nslots[r / block] slots of part[s][r][h][:].
 cudaError_t launch_sum_slots(int d, int elem_bytes, const float *part, const int32_t *nslots, int64_t block,
                              int64_t N, int H, void *out, cudaStream_t stream);
