@@ -358,6 +358,9 @@ def run_ours(args, W):
     # merge launch), timed the same way; the headline stays the slots path.
     if W["mode"] == "device" and not args.no_fused:
         result["fused_merge"] = run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, value)
+    # ---- the backward of the same problems (device mode).
+    if W["mode"] == "device" and not args.no_backward:
+        result["backward"] = run_backward(args, W, D, plans, q, k, v, outs, lses, flops_step, stream, peaks)
 
     # ---- end to end through the public API from pinned host memory.
     if W["mode"] == "host":
@@ -382,6 +385,58 @@ def run_ours(args, W):
         print(json.dumps(result), flush=True)
     del plans
     D.close()
+
+
+def run_backward(args, W, D, plans, q, k, v, outs, lses, flops_step, stream, peaks):
+    """cqsa_backward after each variant's forward outputs, with a seeded
+    output gradient; useful flops 2.5x the forward's (S, dP, dQ, dK, dV
+    against S, PV)."""
+    import torch
+    from out_core_scheduling_b200 import cqsa
+    from out_core_scheduling_b200.inputs import make_qkv
+
+    N, H, d = W["N"], W["H"], W["d"]
+    tdt = q.dtype
+    dout = make_qkv(N, H, d, dtype=tdt, seed=1000 + D.rank, device=q.device, dist=W["dist"])[0]
+    grads = [tuple(torch.empty_like(q) for _ in range(3)) for _ in plans]
+
+    def step():
+        for p, o, l, g in zip(plans, outs, lses, grads):
+            cqsa.cqsa_backward(p, q, k, v, o, l, dout, *g, stream=stream)
+
+    for p, o, l in zip(plans, outs, lses):
+        cqsa.cqsa_forward(p, q, k, v, o, l, cqsa.CQSA_DEVICE, stream)
+    for _ in range(args.warmup):
+        step()
+    for p in plans:
+        p.sync(stream)
+        p.kernel_stats(reset=True)
+        p.profile(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(D.local_rank)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier(D.local_rank)
+    for p in plans:
+        p.profile(False)
+        p.sync(stream)
+    stats = [p.kernel_stats(reset=True) for p in plans]
+    ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}")
+    bflops = 2.5 * flops_step
+    value = bflops * args.steps * D.world / (ms * 1e-3) / 1e12
+    bwd_ms = sum(s["bwd_ms"] for s in stats)
+    kern = bflops * args.steps / (bwd_ms * 1e-3) / 1e12 if bwd_ms else None
+    peak = peaks["bf16_tflops"] if W["dtype"] == "bf16" else 148 * 128 * 2 * 1.965e9 / 1e12
+    return {"value": value, "unit": "TFLOP/s", "ms_per_step": ms / args.steps,
+            "useful_flops_per_step": bflops,
+            "gradient_kernels_tflops": kern, "frac_of_peak": kern / peak if kern else None,
+            "peak": peak, "gpu_launches": sum(s["bwd_launches"] + s["merge_launches"] for s in stats),
+            "path": "cqsa_backward: D = rowsum(dout * out); dq kernel over the (task, query block) list, "
+                    "dk/dv kernel over the (task, key block) list, slot sums"}
 
 
 def run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, slots_value):
@@ -588,6 +643,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-fused", action="store_true", help="skip the fused-merge timing of device workloads")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing of device workloads")
     ap.add_argument("--profile-run", action="store_true",
                     help="only warm-up + steps of the device path (for ncu captures)")
     args = ap.parse_args(argv)
