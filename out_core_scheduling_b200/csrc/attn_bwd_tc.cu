@@ -43,7 +43,7 @@ struct SmemDq {
     alignas(1024) uint8_t dout[KB][BOX_BYTES];
     alignas(1024) uint8_t k[STAGES][KB][BOX_BYTES];
     alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
-    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, p_full, o_full, drain;
+    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, dp_free, p_full, o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             mbar_init(&s.kv_empty[i], 1);
         }
         mbar_init(&s.s_full, 1);
+        mbar_init(&s.dp_free, 4);
         mbar_init(&s.p_full, 4);
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
@@ -191,34 +192,38 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             }
         }
     } else if (warp == WARP_MMA) {
+        // Per key tile j: dP(j+1) = dO V(j+1)^T goes in as soon as the
+        // elementwise warps hold dP(j) in registers (its own TMEM columns);
+        // dQ += dS(j) K(j) and S(j+1) = Q K(j+1)^T follow dS(j), in that order
+        // because S(j+1) overwrites the columns dS(j) occupies.
         bool ok = warp_wait_b(&s.bar_q, 0, abort, tmo);
         const uint64_t qdesc = smem_desc_sw128(smem_u32(s.q[0]), 16, 1024);
         const uint64_t odesc = smem_desc_sw128(smem_u32(s.dout[0]), 16, 1024);
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int st = j % STAGES;
-            if (!warp_wait_b(&s.kv_full[st], (uint32_t)(j / STAGES) & 1u, abort, tmo)) { ok = false; break; }
-            tc_fence_after();
-            if (j > 0) {
-                // dQ += dS(j-1) K(j-1): dS was written over S.
-                if (!warp_wait_b(&s.p_full, (uint32_t)(j - 1) & 1u, abort, tmo)) { ok = false; break; }
-                tc_fence_after();
-                const int sp = (j - 1) % STAGES;
-                mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[sp][0]), BOX_BYTES, 1024), IDESC_TS,
-                              j > 1);
-                mma_commit_elect(&s.kv_empty[sp]);
-            }
-            mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[st][0]), 16, 1024), IDESC_SS);
-            mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[st][0]), 16, 1024), IDESC_SS);
-            mma_commit_elect(&s.s_full);
-        }
         if (ok && ntiles > 0) {
-            ok = warp_wait_b(&s.p_full, (uint32_t)(ntiles - 1) & 1u, abort, tmo);
+            ok = warp_wait_b(&s.kv_full[0], 0, abort, tmo);
             if (ok) {
                 tc_fence_after();
-                const int sp = (ntiles - 1) % STAGES;
-                mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[sp][0]), BOX_BYTES, 1024), IDESC_TS,
-                              ntiles > 1);
-                mma_commit_elect(&s.kv_empty[sp]);
+                mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[0][0]), 16, 1024), IDESC_SS);
+                mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[0][0]), 16, 1024), IDESC_SS);
+                mma_commit_elect(&s.s_full);
+            }
+        }
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int st = j % STAGES, st1 = (j + 1) % STAGES;
+            const bool has_next = j + 1 < ntiles;
+            if (has_next) {
+                if (!warp_wait_b(&s.kv_full[st1], (uint32_t)((j + 1) / STAGES) & 1u, abort, tmo)) { ok = false; break; }
+                if (!warp_wait_b(&s.dp_free, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[st1][0]), 16, 1024), IDESC_SS);
+            }
+            if (!warp_wait_b(&s.p_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[st][0]), BOX_BYTES, 1024), IDESC_TS, j > 0);
+            mma_commit_elect(&s.kv_empty[st]);
+            if (has_next) {
+                mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[st1][0]), 16, 1024), IDESC_SS);
+                mma_commit_elect(&s.s_full);
             }
         }
         if (ok) {
@@ -255,14 +260,23 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     if (diag < (int64_t)lim) lim = diag < 0 ? 0 : (int)diag;
                 }
                 if (!valid) lim = 0;
+                // All of dP(j) into registers first, so dP(j+1) can be computed
+                // into the same columns while this tile finishes.
+                uint32_t dp[4][32];
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp[cc]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < BN / 32; ++cc) fence_regs32(dp[cc]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.dp_free);
 #pragma unroll
                 for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t sv[32], dp[32];
+                    uint32_t sv[32];
                     tmem_ld32(lane_base + (uint32_t)(cc * 32), sv);
-                    tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp);
                     tmem_wait_ld();
                     fence_regs32(sv);
-                    fence_regs32(dp);
                     uint32_t pk[16];
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
@@ -270,8 +284,8 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                         const float p0 = c < lim ? ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, -lse2)) : 0.f;
                         const float p1 =
                             c + 1 < lim ? ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, -lse2)) : 0.f;
-                        pk[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[t]) - dl),
-                                                p1 * (__uint_as_float(dp[t + 1]) - dl));
+                        pk[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[cc][t]) - dl),
+                                                p1 * (__uint_as_float(dp[cc][t + 1]) - dl));
                     }
                     tmem_st16_b(lane_base + (uint32_t)(cc * 16), pk);
                 }
