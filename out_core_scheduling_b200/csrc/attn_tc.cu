@@ -101,9 +101,11 @@ __device__ __forceinline__ void exp2_emulated_pair(float x0, float x1, float &p0
 }
 
 // Which column pairs of a 128-wide score row use the emulated exponential
-// instead of the MUFU ex2: EMU_PAIRS_PER_8 of every 8 (measured on B200:
-// one in eight balances the MUFU against the FMA/ALU pipes best).
-constexpr int EMU_PAIRS_PER_8 = 1;
+// instead of the MUFU ex2: EMU_PAIRS_PER_8 of every 8.  Measured on B200
+// with the split P hand-off and the row sum after it: none (0) is 2-3 %
+// faster than one in eight (10 % fewer instructions; the MUFU is not the
+// binding limit of this loop), so the emulation stays a compile-time option.
+constexpr int EMU_PAIRS_PER_8 = 0;
 __device__ __forceinline__ constexpr bool emu_pair(int pair) { return (pair & 7) >= 8 - EMU_PAIRS_PER_8; }
 
 // Warp-uniform bounded wait: every lane polls, then the warp agrees.
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     }
                 }
                 // Scale and shift two scores per instruction, exponentiate
-                // (MUFU ex2, or the emulation for some pairs), keep the fp32
+                // (MUFU ex2, or the emulation for the pairs emu_pair picks), keep the fp32
                 // values for the row sum and write P as bf16 pairs: keys 0..63
                 // to columns 0..31, keys 64..127 to columns 32..63.  The first
                 // half is announced (p_half) once its store has landed, after
