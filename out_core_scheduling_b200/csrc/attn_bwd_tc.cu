@@ -43,7 +43,7 @@ struct SmemDq {
     alignas(1024) uint8_t dout[KB][BOX_BYTES];
     alignas(1024) uint8_t k[STAGES][KB][BOX_BYTES];
     alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
-    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, dp_free, p_full, o_full, drain;
+    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, dp_free, p_half, p_full, o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -57,7 +57,7 @@ struct SmemKv {
     alignas(1024) uint8_t dout[STAGES][KB][BOX_BYTES];
     float lse2[STAGES][BN];  // lse * log2(e) of the tile's query rows (+inf outside the run)
     float dl[STAGES][BN];    // D of the tile's query rows
-    uint64_t bar_kv, qd_full[STAGES], qd_empty[STAGES], s_full, p_full, o_full, drain;
+    uint64_t bar_kv, qd_full[STAGES], qd_empty[STAGES], s_full, p_half, p_full, o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -101,9 +101,9 @@ __device__ __forceinline__ void mma_rows_dot(uint32_t d_tmem, uint64_t adesc, ui
 // TS MMA D[128 x D] (+)= A[128 x 128] (bf16 in TMEM at a_tmem, 2 per column)
 // times B[128 x D] with B's rows the K dimension, stored [rows][D] (MN-major).
 __device__ __forceinline__ void mma_tmem_rows(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                              bool acc) {
+                                              bool acc, int k0 = 0, int k1 = BN / 16) {
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
+    for (int kk = k0; kk < k1; ++kk)
         mma_ts_elect(d_tmem, a_tmem + (uint32_t)kk * 8u, bdesc + (uint64_t)(kk * (2048 >> 4)), idesc,
                      (acc || kk > 0) ? 1u : 0u);
 }
@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         }
         mbar_init(&s.s_full, 1);
         mbar_init(&s.dp_free, 4);
+        mbar_init(&s.p_half, 4);
         mbar_init(&s.p_full, 4);
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
@@ -217,9 +218,15 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 tc_fence_after();
                 mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[st1][0]), 16, 1024), IDESC_SS);
             }
+            // dS(j) arrives in two halves of 64 keys: the first half of dQ
+            // runs while the elementwise warps finish the second.
+            const uint64_t kb = smem_desc_sw128(smem_u32(s.k[st][0]), BOX_BYTES, 1024);
+            if (!warp_wait_b(&s.p_half, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            mma_tmem_rows(tmem + 256u, tmem, kb, IDESC_TS, j > 0, 0, BN / 32);
             if (!warp_wait_b(&s.p_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
-            mma_tmem_rows(tmem + 256u, tmem, smem_desc_sw128(smem_u32(s.k[st][0]), BOX_BYTES, 1024), IDESC_TS, j > 0);
+            mma_tmem_rows(tmem + 256u, tmem, kb, IDESC_TS, true, BN / 32, BN / 16);
             mma_commit_elect(&s.kv_empty[st]);
             if (has_next) {
                 mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[st1][0]), 16, 1024), IDESC_SS);
@@ -288,6 +295,12 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                                                 p1 * (__uint_as_float(dp[cc][t + 1]) - dl));
                     }
                     tmem_st16_b(lane_base + (uint32_t)(cc * 16), pk);
+                    if (cc == 1) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.p_half);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -371,6 +384,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             mbar_init(&s.qd_empty[i], 1);
         }
         mbar_init(&s.s_full, 1);
+        mbar_init(&s.p_half, 4);
         mbar_init(&s.p_full, 4);
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
@@ -439,36 +453,34 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         bool ok = warp_wait_b(&s.bar_kv, 0, abort, tmo);
         const uint64_t kdesc = smem_desc_sw128(smem_u32(s.k[0]), 16, 1024);
         const uint64_t vdesc = smem_desc_sw128(smem_u32(s.v[0]), 16, 1024);
-        auto grads = [&](int it) {
+        auto grads = [&](int it) -> bool {
             // dV += P^T dO, dK += dS^T Q for query tile `it` (P^T over S^T,
-            // dS^T over dP^T in tensor memory).
+            // dS^T over dP^T in tensor memory), in two halves of 64 queries:
+            // the first runs while the elementwise warps finish the second.
             const int sp = it % STAGES;
-            mma_tmem_rows(tmem + COL_DV, tmem, smem_desc_sw128(smem_u32(s.dout[sp][0]), BOX_BYTES, 1024), IDESC_TS,
-                          it > 0);
-            mma_tmem_rows(tmem + COL_DK, tmem + 128u, smem_desc_sw128(smem_u32(s.q[sp][0]), BOX_BYTES, 1024),
-                          IDESC_TS, it > 0);
+            const uint64_t ob = smem_desc_sw128(smem_u32(s.dout[sp][0]), BOX_BYTES, 1024);
+            const uint64_t qb = smem_desc_sw128(smem_u32(s.q[sp][0]), BOX_BYTES, 1024);
+            if (!warp_wait_b(&s.p_half, (uint32_t)it & 1u, abort, tmo)) return false;
+            tc_fence_after();
+            mma_tmem_rows(tmem + COL_DV, tmem, ob, IDESC_TS, it > 0, 0, BN / 32);
+            mma_tmem_rows(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, it > 0, 0, BN / 32);
+            if (!warp_wait_b(&s.p_full, (uint32_t)it & 1u, abort, tmo)) return false;
+            tc_fence_after();
+            mma_tmem_rows(tmem + COL_DV, tmem, ob, IDESC_TS, true, BN / 32, BN / 16);
+            mma_tmem_rows(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, true, BN / 32, BN / 16);
             mma_commit_elect(&s.qd_empty[sp]);
+            return true;
         };
         for (int i = 0; i < ntiles && ok; ++i) {
             const int st = i % STAGES;
             if (!warp_wait_b(&s.qd_full[st], (uint32_t)(i / STAGES) & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
-            if (i > 0) {
-                if (!warp_wait_b(&s.p_full, (uint32_t)(i - 1) & 1u, abort, tmo)) { ok = false; break; }
-                tc_fence_after();
-                grads(i - 1);
-            }
+            if (i > 0 && !grads(i - 1)) { ok = false; break; }
             mma_rows_dot<D>(tmem, kdesc, smem_desc_sw128(smem_u32(s.q[st][0]), 16, 1024), IDESC_SS);
             mma_rows_dot<D>(tmem + 128u, vdesc, smem_desc_sw128(smem_u32(s.dout[st][0]), 16, 1024), IDESC_SS);
             mma_commit_elect(&s.s_full);
         }
-        if (ok && ntiles > 0) {
-            ok = warp_wait_b(&s.p_full, (uint32_t)(ntiles - 1) & 1u, abort, tmo);
-            if (ok) {
-                tc_fence_after();
-                grads(ntiles - 1);
-            }
-        }
+        if (ok && ntiles > 0) ok = grads(ntiles - 1);
         if (ok) {
             mma_commit_elect(&s.o_full);
         } else if (lane == 0) {
@@ -531,6 +543,12 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     }
                     tmem_st16_b(lane_base + (uint32_t)(cc * 16), pp);
                     tmem_st16_b(lane_base + 128u + (uint32_t)(cc * 16), pd);
+                    if (cc == 1) {
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.p_half);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
