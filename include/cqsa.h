@@ -49,7 +49,7 @@ typedef struct cqsa_plan cqsa_plan_t; /* opaque; created by cqsa_plan*, freed by
 
 typedef enum {
     CQSA_OK = 0,
-    CQSA_ERR_INVALID_ARG = 1,       /* null pointer, bad size, N not divisible by the chunk product */
+    CQSA_ERR_INVALID_ARG = 1,       /* null pointer, bad size or option */
     CQSA_ERR_NO_DIFFERENCE_SET = 2, /* no perfect difference set of size l mod l(l-1)+1 (e.g. l = 7) */
     CQSA_ERR_BUDGET = 3,            /* no working set fits mem_budget_bytes */
     CQSA_ERR_NOT_PINNED = 4,        /* host mode given a pointer that is not page-locked host memory */
@@ -79,7 +79,8 @@ typedef enum { CQSA_MERGE_SLOTS = 0, CQSA_MERGE_FUSED = 1 } cqsa_merge_t;
 #define CQSA_MAX_L 16
 
 /* Full plan description.  levels >= 1 and l[0..levels-1] each >= 2; the
- * leaf block is N / prod_i (l_i (l_i - 1) + 1) tokens.  mem_budget_bytes = 0
+ * leaf block is ceil(N / prod_i (l_i (l_i - 1) + 1)) tokens (positions at or
+ * past N belong to no pair, so N need not divide evenly).  mem_budget_bytes = 0
  * means unlimited. */
 typedef struct {
     int64_t N;

@@ -580,7 +580,7 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     CK(cudaStreamWaitEvent(P->s_comp, P->ev_start, 0));
     CK(cudaStreamWaitEvent(P->s_out, P->ev_start, 0));
     int64_t it = 0;
-    const size_t blk_rows = (size_t)B;
+    const size_t blk_stride = (size_t)B;  // pool rows per slot
     for (int h0 = 0; h0 < H; h0 += g) {
         for (size_t t = 0; t < P->leaves.size(); ++t, ++it) {
             const LeafState &L = P->leaves[t];
@@ -594,7 +594,8 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
             if (t == 0 && it >= 1) CK(cudaStreamWaitEvent(P->s_in, P->ev_in_free[1 - s], 0));
             for (const PoolCopy &c : pl.pool.copies[t]) {
                 const size_t src_off = ((size_t)c.block * B * H + h0) * d * e;
-                const size_t dst_off = (size_t)c.slot * blk_rows * grp_row;
+                const size_t dst_off = (size_t)c.slot * blk_stride * grp_row;
+                const size_t blk_rows = (size_t)pl.block_rows(c.block);  // the last block may be short
                 if (c.kind == 0) {
                     CK(copy_rows(P->pool_q + dst_off, grp_row, hq + src_off, full_row, grp_row, blk_rows,
                                  cudaMemcpyHostToDevice, P->s_in));

@@ -90,7 +90,7 @@ int32_t entry_unit_tiles(const Planner &pl, const Entry &e, const WlEntry &w, in
     for (const KeyRun &kr : e.runs) {
         WlRun x{};
         x.k_lo = (int32_t)(kr.b0 * pl.block);
-        x.k_hi = (int32_t)((kr.b1 + 1) * pl.block);
+        x.k_hi = (int32_t)pl.block_end(kr.b1);
         int32_t lo, hi;
         clip_run(w, x, qb, pl.spec.causal, &lo, &hi);
         if (hi > lo) n += (hi - lo + bn - 1) / bn;
@@ -101,7 +101,7 @@ int32_t entry_unit_tiles(const Planner &pl, const Entry &e, const WlEntry &w, in
 WlEntry entry_record(const Planner &pl, const Entry &e, int32_t run_begin) {
     WlEntry w{};
     w.q_lo = (int32_t)(e.qb * pl.block);
-    w.q_hi = (int32_t)((e.qb + 1) * pl.block);
+    w.q_hi = (int32_t)pl.block_end(e.qb);
     w.q_goff = 0;
     w.slot = (int32_t)e.slot;
     w.out_lo = w.q_lo;
@@ -134,7 +134,7 @@ void write_list(const Planner &pl, int rows_per_unit, int bn, const ListSizes &n
         for (const KeyRun &kr : e.runs) {
             WlRun x{};
             x.k_lo = (int32_t)(kr.b0 * pl.block);
-            x.k_hi = (int32_t)((kr.b1 + 1) * pl.block);
+            x.k_hi = (int32_t)pl.block_end(kr.b1);
             x.k_goff = 0;
             R[r++] = x;
         }

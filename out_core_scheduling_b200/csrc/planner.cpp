@@ -87,10 +87,9 @@ std::string Planner::build(const PlanSpec &s, int *code) {
         num_blocks *= L.c;
         levels.push_back(L);
     }
-    if (s.N % num_blocks != 0)
-        return "N (" + std::to_string(s.N) + ") must be divisible by the product of chunk counts (" +
-               std::to_string(num_blocks) + ")";
-    block = s.N / num_blocks;
+    // N need not be a multiple of the block count: blocks of ceil(N / P)
+    // tokens, and positions at or past N belong to no pair.
+    block = (s.N + num_blocks - 1) / num_blocks;
 
     // Recursive division ("The Recursive Benefit"): level i divides each
     // parent's token sequence (its blocks in increasing order) into c_i equal
@@ -143,6 +142,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
         max_task_rows = std::max<int64_t>(max_task_rows, n * block);
         entry_begin_of_leaf_.push_back((int64_t)entries.size());
         for (int64_t mq = 0; mq < n; ++mq) {
+            if (block_rows(nd.blocks[mq]) == 0) continue;  // no query row in this block
             Entry e;
             e.task = t;
             e.qb = nd.blocks[mq];
@@ -158,6 +158,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
                     }
                 }
                 if (ok && s.causal && nd.blocks[mk] > nd.blocks[mq]) ok = false;
+                if (ok && block_rows(nd.blocks[mk]) == 0) ok = false;
                 if (!ok) continue;
                 const int64_t kb = nd.blocks[mk];
                 if (!e.runs.empty() && e.runs.back().b1 + 1 == kb &&
@@ -236,17 +237,17 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
             std::sort(kb.begin(), kb.end());
             WlEntry w{};
             w.q_lo = (int32_t)(qb * block);
-            w.q_hi = (int32_t)((qb + 1) * block);
+            w.q_hi = (int32_t)block_end(qb);
             w.out_lo = w.q_lo;
             w.flags = SEG_FIRST | SEG_LAST;
             w.run_begin = (int32_t)wl.runs.size();
             for (size_t i = 0; i < kb.size(); ++i) {
                 if (i > 0 && kb[i] == kb[i - 1] + 1) {
-                    wl.runs.back().k_hi = (int32_t)((kb[i] + 1) * block);
+                    wl.runs.back().k_hi = (int32_t)block_end(kb[i]);
                 } else {
                     WlRun x{};
                     x.k_lo = (int32_t)(kb[i] * block);
-                    x.k_hi = (int32_t)((kb[i] + 1) * block);
+                    x.k_hi = (int32_t)block_end(kb[i]);
                     wl.runs.push_back(x);
                 }
             }
@@ -261,7 +262,7 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
         group.push_back(e.task);
         WlEntry w{};
         w.q_lo = (int32_t)(e.qb * block);
-        w.q_hi = (int32_t)((e.qb + 1) * block);
+        w.q_hi = (int32_t)block_end(e.qb);
         w.q_goff = 0;
         w.slot = (int32_t)e.slot;
         w.out_lo = w.q_lo;
@@ -270,7 +271,7 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
         for (const KeyRun &r : e.runs) {
             WlRun x{};
             x.k_lo = (int32_t)(r.b0 * block);
-            x.k_hi = (int32_t)((r.b1 + 1) * block);
+            x.k_hi = (int32_t)block_end(r.b1);
             x.k_goff = 0;
             wl.runs.push_back(x);
         }
@@ -306,18 +307,18 @@ WorkList Planner::device_worklist_kv(int rows_per_unit, int bn, int heads, int64
             std::sort(qs.begin(), qs.end());
             WlEntry w{};
             w.q_lo = (int32_t)(kb * block);
-            w.q_hi = (int32_t)((kb + 1) * block);
+            w.q_hi = (int32_t)block_end(kb);
             w.slot = slot++;
             w.out_lo = w.q_lo;
             w.flags = spec.fused ? (SEG_FIRST | SEG_LAST) : 0;
             w.run_begin = (int32_t)wl.runs.size();
             for (size_t i = 0; i < qs.size(); ++i) {
                 if (i > 0 && qs[i] == qs[i - 1] + 1) {
-                    wl.runs.back().k_hi = (int32_t)((qs[i] + 1) * block);
+                    wl.runs.back().k_hi = (int32_t)block_end(qs[i]);
                 } else {
                     WlRun x{};
                     x.k_lo = (int32_t)(qs[i] * block);
-                    x.k_hi = (int32_t)((qs[i] + 1) * block);
+                    x.k_hi = (int32_t)block_end(qs[i]);
                     wl.runs.push_back(x);
                 }
             }
@@ -355,7 +356,7 @@ WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_un
         const int64_t qs = pool.q_slot[t][e.mq];
         WlEntry w{};
         w.q_lo = (int32_t)(qs * block);
-        w.q_hi = (int32_t)((qs + 1) * block);
+        w.q_hi = (int32_t)(qs * block + block_rows(e.qb));
         w.q_goff = (int32_t)((e.qb - qs) * block);
         w.slot = 0;
         w.out_lo = (int32_t)(e.mq * block);
@@ -367,11 +368,13 @@ WorkList Planner::leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_un
                 const int32_t lo = (int32_t)(ks * block), goff = (int32_t)((kb - ks) * block);
                 if ((int32_t)wl.runs.size() > w.run_begin && wl.runs.back().k_hi == lo &&
                     wl.runs.back().k_goff == goff) {
-                    wl.runs.back().k_hi = lo + (int32_t)block;   // contiguous slots: one run
+                    // Contiguous slots: one run.  A partial last block ends its
+                    // run short, so nothing is ever appended past it.
+                    wl.runs.back().k_hi = lo + (int32_t)block_rows(kb);
                 } else {
                     WlRun x{};
                     x.k_lo = lo;
-                    x.k_hi = lo + (int32_t)block;
+                    x.k_hi = lo + (int32_t)block_rows(kb);
                     x.k_goff = goff;
                     wl.runs.push_back(x);
                 }
@@ -390,7 +393,7 @@ std::vector<MergeSeg> Planner::leaf_merge_segments(int64_t t) const {
         const Entry &e = entries[i];
         MergeSeg s{};
         s.local_lo = (int32_t)(e.mq * block);
-        s.rows = (int32_t)block;
+        s.rows = (int32_t)block_rows(e.qb);
         s.global_lo = (int32_t)(e.qb * block);
         s.flags = (first_leaf_[e.qb] == t ? SEG_FIRST : 0) | (last_leaf_[e.qb] == t ? SEG_LAST : 0);
         segs.push_back(s);

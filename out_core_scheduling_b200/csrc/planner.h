@@ -12,6 +12,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <string>
 #include <vector>
 
@@ -100,7 +101,11 @@ public:
     PlanSpec spec;
     std::vector<Level> levels;
     int64_t num_blocks = 0;     // prod c_i
-    int64_t block = 0;          // tokens per block
+    int64_t block = 0;          // tokens per block: ceil(N / num_blocks)
+    // Token rows of block b: [b * block, block_end(b)); blocks at or past N
+    // hold none (N need not be a multiple of num_blocks).
+    int64_t block_end(int64_t b) const { return std::min<int64_t>((b + 1) * block, spec.N); }
+    int64_t block_rows(int64_t b) const { return std::max<int64_t>(0, block_end(b) - b * block); }
     std::vector<Leaf> leaves;
     std::vector<Entry> entries; // ordered by (task, qb)
     std::vector<int32_t> slots_per_block;

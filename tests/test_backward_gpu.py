@@ -107,3 +107,13 @@ def test_backward_rejects_host_mode():
     with pytest.raises(cqsa.CqsaError) as ei:
         cqsa.cqsa_backward(plan, q, k, v, out, lse, q, *g, host_or_device=cqsa.CQSA_HOST)
     assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", [(1000, 2, 128, [3], torch.bfloat16), (91 * 12 + 5, 1, 64, [4, 3], torch.bfloat16),
+                                  (700 - 9, 1, 64, [3], torch.float32)],
+                         ids=lambda c: f"n{c[0]}-l{c[3]}-{str(c[4])[6:]}")
+def test_backward_ragged_n(case, causal, merge):
+    N, H, d, ls, dtype = case
+    _check_all(N, H, d, ls, dtype, causal, merge, seed=31)

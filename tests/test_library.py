@@ -81,6 +81,24 @@ def test_planner_matches_reference(ls, P, causal):
     assert plan_pairs(plan) == reference_pairs(P, ls, causal)
 
 
+@pytest.mark.parametrize("N,ls", [(1000, [3]), (13 * 100 - 37, [4]), (5, [3]), (91 * 9 + 50, [4, 3])])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ragged_n_plans(N, ls, causal):
+    """N need not be a multiple of the block count: blocks of ceil(N / P)
+    tokens; blocks holding no token get no entry and appear in no run; the
+    pairs among the others are exactly the reference's."""
+    P = 1
+    for l in ls:
+        P *= l * (l - 1) + 1
+    plan = cqsa.cqsa_plan_ex(N, 1, 64, ls, causal=causal)
+    info = plan.info()
+    B = -(-N // P)
+    assert info["block_tokens"] == B and info["num_blocks"] == P
+    live = {b for b in range(P) if b * B < N}
+    ref = {(t, qb, kb) for (t, qb, kb) in reference_pairs(P, tuple(ls), causal) if qb in live and kb in live}
+    assert plan_pairs(plan) == ref
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_slots_number_each_query_block(causal):
     plan = cqsa.cqsa_plan_ex(91 * 2, 1, 64, [4, 3], causal=causal)
@@ -189,7 +207,7 @@ def test_fused_merge_plan():
 
 
 @pytest.mark.parametrize("args,status", [
-    ((1000, 1, 64, 3, 1, False, 0), cqsa.CQSA_ERR_INVALID_ARG),       # 1000 % 7 != 0
+    ((-7, 1, 64, 3, 1, False, 0), cqsa.CQSA_ERR_INVALID_ARG),
     ((43 * 4, 1, 64, 7, 1, False, 0), cqsa.CQSA_ERR_NO_DIFFERENCE_SET),
     ((7 * 4, 1, 96, 3, 1, False, 0), cqsa.CQSA_ERR_UNSUPPORTED),
     ((7 * 4096, 8, 128, 3, 1, False, 1 << 20), cqsa.CQSA_ERR_BUDGET),

@@ -116,14 +116,21 @@ def test_streamed_two_level(causal):
     check(out, lse, q, k, v, sample_rows(N, 512), causal)
 
 
-def _min_budget(N, H, d, ls, causal):
-    lo, hi = 1 << 20, cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal).info()["host_arena_bytes"]
+def _min_budget(N, H, d, ls, causal, dtype=cqsa.CQSA_BF16):
+    """Smallest budget (to 256 KB) the streamed path accepts for this plan."""
+    lo, hi = 0, cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dtype).info()["host_arena_bytes"]
     while hi - lo > (1 << 18):
         mid = (lo + hi) // 2
         try:
-            cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, mem_budget_bytes=mid)
-            hi = mid
+            # A plan can also be accepted because its device-resident path
+            # fits; the streamed path needs a head group.
+            ok = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dtype,
+                                   mem_budget_bytes=mid).info()["head_group"] > 0
         except cqsa.CqsaError:
+            ok = False
+        if ok:
+            hi = mid
+        else:
             lo = mid
     return hi
 
@@ -235,3 +242,40 @@ def test_fused_equals_slots():
                     cqsa.CQSA_DEVICE)
         assert (a.float() - b.float()).abs().max().item() <= 2e-2
         assert (la - lb).abs().max().item() <= 1e-4
+
+
+# ---------------------------------------------------------------- ragged N
+RAGGED = [
+    # (N, H, d, levels, dtype): N not a multiple of the block count
+    (1000, 2, 128, [3], torch.bfloat16),
+    (13 * 300 - 77, 2, 64, [4], torch.bfloat16),
+    (91 * 40 + 13, 1, 128, [4, 3], torch.bfloat16),
+    (5, 1, 64, [3], torch.bfloat16),                 # fewer tokens than blocks
+    (1000, 1, 64, [3], torch.float32),
+]
+
+
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", RAGGED, ids=lambda c: f"n{c[0]}-h{c[1]}-d{c[2]}-l{c[3]}-{str(c[4])[6:]}")
+def test_ragged_n_device(case, causal, merge):
+    N, H, d, ls, dtype = case
+    q, k, v = _inputs(N, H, d, dtype, seed=40)
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, merge=merge)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", RAGGED[:3] + RAGGED[4:], ids=lambda c: f"n{c[0]}-l{c[3]}-{str(c[4])[6:]}")
+def test_ragged_n_streamed(case, causal):
+    """Streamed at the smallest budget the plan accepts (block cache
+    evictions, a short last block)."""
+    N, H, d, ls, dtype = case
+    q, k, v = _inputs(N, H, d, dtype, seed=41, host=True)
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    budget = _min_budget(N, H, d, ls, causal, dt)
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, mem_budget_bytes=budget)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), causal)

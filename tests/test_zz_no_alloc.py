@@ -32,6 +32,7 @@ CASES = [
     (torch.bfloat16, cqsa.CQSA_BF16, 7 * 256, 2, 128, [3], False),
     (torch.bfloat16, cqsa.CQSA_BF16, 13 * 200, 2, 128, [4], True),
     (torch.float32, cqsa.CQSA_FP32, 7 * 512, 1, 64, [3], False),
+    (torch.bfloat16, cqsa.CQSA_BF16, 1000, 2, 64, [3], True),      # N not a multiple of the blocks
 ]
 
 
