@@ -92,6 +92,9 @@ typedef struct {
     int dtype; /* cqsa_dtype_t */
     size_t mem_budget_bytes;
     int merge; /* cqsa_merge_t; 0 (slots) when zero-initialised */
+    int H_kv;  /* key/value heads (grouped-query attention): H must be a
+                  multiple; query head h reads key/value head h / (H / H_kv).
+                  0 = H.  k, v (and dk, dv) are then [N, H_kv, d]. */
 } cqsa_plan_desc_t;
 
 /* What a plan decided (for logging, tests and the benchmark). */
@@ -114,6 +117,7 @@ typedef struct {
     size_t d2h_bytes;                   /* planned device->host bytes of one host-mode forward */
     double useful_flops;                /* 4 N^2 H d, halved when causal */
     int merge;                          /* cqsa_merge_t of device-mode forwards */
+    int H_kv;                           /* key/value heads */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */

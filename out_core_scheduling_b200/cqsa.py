@@ -51,7 +51,7 @@ class PlanDesc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
                 ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int)]
+                ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int), ("H_kv", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -65,7 +65,7 @@ class PlanInfo(ctypes.Structure):
                 ("head_group", ctypes.c_int), ("device_arena_bytes", ctypes.c_size_t),
                 ("host_arena_bytes", ctypes.c_size_t), ("h2d_bytes", ctypes.c_size_t),
                 ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double),
-                ("merge", ctypes.c_int)]
+                ("merge", ctypes.c_int), ("H_kv", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -212,7 +212,7 @@ def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = Fa
 
 
 def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
-                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS) -> Plan:
+                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0) -> Plan:
     desc = PlanDesc()
     desc.N, desc.H, desc.d = N, H, d
     desc.levels = len(ls)
@@ -222,28 +222,42 @@ def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = 
     desc.dtype = dtype
     desc.mem_budget_bytes = mem_budget_bytes
     desc.merge = merge
+    desc.H_kv = H_kv
     h = ctypes.c_void_p()
     _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
     return Plan(h.value)
 
 
-def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVICE, stream=None):
-    """q, k, v, out: [N, H, d] contiguous torch tensors in the plan's dtype;
-    lse: fp32 [H, N].  Device tensors for CQSA_DEVICE, pinned CPU tensors
-    for CQSA_HOST.  Asynchronous on ``stream`` (default: torch's current)."""
+def _check_shapes(plan: Plan, qlike, kvlike, lse):
+    """Tensors against the plan: query-shaped [N, H, d], key/value-shaped
+    [N, H_kv, d] (H_kv = H without grouped-query attention), lse [H, N]."""
     import torch
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
+    info = plan.info()
+    N, H, d, Hkv = info["N"], info["H"], info["d"], info["H_kv"]
+    named = list(qlike) + list(kvlike) + [("lse", lse)]
+    for name, t in named:
         if not isinstance(t, torch.Tensor) or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous torch tensor")
     if lse.dtype != torch.float32:
         raise ValueError("lse must be float32")
-    if not (q.dtype == k.dtype == v.dtype == out.dtype):
-        raise ValueError("q, k, v, out must share a dtype")
-    if not (q.shape == k.shape == v.shape == out.shape) or q.dim() != 3:
-        raise ValueError("q, k, v, out must all be [N, H, d]")
-    N, H, _ = q.shape
+    if len({t.dtype for _, t in list(qlike) + list(kvlike)}) != 1:
+        raise ValueError(", ".join(n for n, _ in list(qlike) + list(kvlike)) + " must share a dtype")
+    for name, t in qlike:
+        if tuple(t.shape) != (N, H, d):
+            raise ValueError(f"{name} must be [N, H, d] = {(N, H, d)}")
+    for name, t in kvlike:
+        if tuple(t.shape) != (N, Hkv, d):
+            raise ValueError(f"{name} must be [N, H_kv, d] = {(N, Hkv, d)}")
     if tuple(lse.shape) != (H, N):
         raise ValueError("lse must be [H, N]")
+
+
+def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVICE, stream=None):
+    """q, out: [N, H, d]; k, v: [N, H_kv, d] (H_kv = H without grouped-query
+    attention); contiguous torch tensors in the plan's dtype; lse: fp32
+    [H, N].  Device tensors for CQSA_DEVICE, pinned CPU tensors for
+    CQSA_HOST.  Asynchronous on ``stream`` (default: torch's current)."""
+    _check_shapes(plan, (("q", q), ("out", out)), (("k", k), ("v", v)), lse)
     _check(load_library().cqsa_forward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                        out.data_ptr(), lse.data_ptr(), host_or_device,
                                        ctypes.c_void_p(_stream_ptr(stream))))
@@ -252,21 +266,11 @@ def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVIC
 def cqsa_backward(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, host_or_device: int = CQSA_DEVICE,
                   stream=None):
     """Gradients dq, dk, dv of the planned attention given the forward's out
-    and lse and the output gradient dout.  All [N, H, d] contiguous device
-    tensors in the plan's dtype except lse (fp32 [H, N]).  Asynchronous on
-    ``stream``."""
-    import torch
-    named = (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv))
-    for name, t in named + (("lse", lse),):
-        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous torch tensor")
-    if lse.dtype != torch.float32:
-        raise ValueError("lse must be float32")
-    if len({t.dtype for _, t in named}) != 1 or len({tuple(t.shape) for _, t in named}) != 1 or q.dim() != 3:
-        raise ValueError("q, k, v, out, dout, dq, dk, dv must share a dtype and an [N, H, d] shape")
-    N, H, _ = q.shape
-    if tuple(lse.shape) != (H, N):
-        raise ValueError("lse must be [H, N]")
+    and lse and the output gradient dout.  q, out, dout, dq: [N, H, d];
+    k, v, dk, dv: [N, H_kv, d]; contiguous device tensors in the plan's dtype;
+    lse fp32 [H, N].  Asynchronous on ``stream``."""
+    _check_shapes(plan, (("q", q), ("out", out), ("dout", dout), ("dq", dq)),
+                  (("k", k), ("v", v), ("dk", dk), ("dv", dv)), lse)
     _check(load_library().cqsa_backward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                         lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                                         dv.data_ptr(), host_or_device, ctypes.c_void_p(_stream_ptr(stream))))
@@ -277,14 +281,7 @@ def cqsa_forward_noalloc(plan: Plan, q, k, v, out, lse, stream=None):
     array (no device allocation at call time).  Same tensors as
     ``cqsa_forward`` in CQSA_DEVICE mode; returns after the work on
     ``stream`` has finished."""
-    import torch
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
-        if not isinstance(t, torch.Tensor) or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous torch tensor")
-    if lse.dtype != torch.float32:
-        raise ValueError("lse must be float32")
-    if not (q.shape == k.shape == v.shape == out.shape) or q.dim() != 3:
-        raise ValueError("q, k, v, out must all be [N, H, d]")
+    _check_shapes(plan, (("q", q), ("out", out)), (("k", k), ("v", v)), lse)
     _check(load_library().cqsa_forward_noalloc(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                                out.data_ptr(), lse.data_ptr(),
                                                ctypes.c_void_p(_stream_ptr(stream))))

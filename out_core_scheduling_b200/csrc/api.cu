@@ -288,6 +288,8 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     const int64_t N = pl.spec.N, R = pl.max_task_rows;
     const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
     const size_t blk = (size_t)pl.block * g * dd * e;
+    const int gk = pl.spec.kv_heads_of(g);  // key/value heads of a head group
+    const size_t blk_kv = (size_t)pl.block * gk * dd * e;
     const PoolPlan &pp = pl.pool;
     // Same layout steps as Planner::host_arena_bytes.
     ArenaLayout a;
@@ -295,8 +297,8 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     const size_t o_acc = a.take((size_t)N * g * dd * sizeof(float));
     const size_t o_accl = a.take((size_t)g * N * sizeof(float));
     const size_t o_pq = a.take((size_t)pp.q_slots * blk);
-    const size_t o_pk = a.take((size_t)pp.kv_slots * blk);
-    const size_t o_pv = a.take((size_t)pp.kv_slots * blk);
+    const size_t o_pk = a.take((size_t)pp.kv_slots * blk_kv);
+    const size_t o_pv = a.take((size_t)pp.kv_slots * blk_kv);
     size_t o_out[2], o_lse[2];
     for (int s = 0; s < 2; ++s) {
         o_out[s] = a.take((size_t)R * g * dd * e);
@@ -338,8 +340,8 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     if (P->dtype == CQSA_BF16) {
         cqsa_status_t st;
         if ((st = make_map(&P->mq, P->pool_q, pp.q_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
-        if ((st = make_map(&P->mk, P->pool_k, pp.kv_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
-        if ((st = make_map(&P->mv, P->pool_v, pp.kv_slots * pl.block, g, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mk, P->pool_k, pp.kv_slots * pl.block, gk, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mv, P->pool_v, pp.kv_slots * pl.block, gk, pl.spec.d)) != CQSA_OK) return st;
     }
     CK(cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
@@ -364,6 +366,8 @@ AttnParams base_params(const cqsa_plan_t *P, int *err) {
     ap.timeout_ns = P->timeout_ns;
     ap.err = err;
     ap.stall_test = P->stall_test;
+    ap.Hkv = P->pl.spec.Hkv;
+    ap.kv_group = P->pl.spec.kv_group();
     return ap;
 }
 
@@ -413,8 +417,8 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     if (P->dtype == CQSA_BF16) {
         CUtensorMap mq, mk, mv;
         if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
-        if ((st = make_map(&mk, k, N, H, d)) != CQSA_OK) return st;
-        if ((st = make_map(&mv, v, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mk, k, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mv, v, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
         LaunchTimer tm(P, stream, 0);
         CK(launch_attn_tc(d, mq, mk, mv, ap, P->dev_wl.num_units, stream));
         tm.stop();
@@ -442,21 +446,28 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     WorkList qwl = pl.device_worklist(rows, rows, H);
     int64_t max_kv = 0;
     WorkList kvwl = pl.device_worklist_kv(rows, rows, H, &max_kv);
+    // Key/value partial slots: per (task, key block) entry, and per query
+    // head of a key/value group (grouped-query attention).
+    const int kvg = pl.spec.kv_group(), Hkv = pl.spec.Hkv;
     std::vector<int32_t> kv_ns(pl.num_blocks, 0);
     for (const WlEntry &e : kvwl.entries) {
         const int64_t kb = e.q_lo / pl.block;
-        kv_ns[kb] = std::max<int32_t>(kv_ns[kb], e.slot + 1);
+        kv_ns[kb] = std::max<int32_t>(kv_ns[kb], (e.slot + 1) * kvg);
     }
+    const bool kv_slots = !fused || kvg > 1;
     const size_t slot = (size_t)N * H * d * sizeof(float);
+    const size_t kv_slot = (size_t)N * Hkv * d * sizeof(float);
     ArenaLayout a;
     const size_t o_err = a.take(256);
     const size_t o_delta = a.take((size_t)H * N * sizeof(float));
     size_t o_dq = 0, o_dk = 0, o_dv = 0, o_qns = 0, o_kvns = 0;
     if (!fused) {
         o_dq = a.take((size_t)pl.max_slots * slot);
-        o_dk = a.take((size_t)max_kv * slot);
-        o_dv = a.take((size_t)max_kv * slot);
         o_qns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
+    }
+    if (kv_slots) {
+        o_dk = a.take((size_t)max_kv * kvg * kv_slot);
+        o_dv = a.take((size_t)max_kv * kvg * kv_slot);
         o_kvns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
     }
     const size_t o_qwl = a.take(wl_region(qwl));
@@ -470,12 +481,14 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     P->bwd_delta = reinterpret_cast<float *>(arena + o_delta);
     if (!fused) {
         P->bwd_dq = reinterpret_cast<float *>(arena + o_dq);
-        P->bwd_dk = reinterpret_cast<float *>(arena + o_dk);
-        P->bwd_dv = reinterpret_cast<float *>(arena + o_dv);
         P->bwd_q_nslots = reinterpret_cast<int32_t *>(arena + o_qns);
-        P->bwd_kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
         CK(cudaMemcpy(P->bwd_q_nslots, pl.slots_per_block.data(), pl.num_blocks * sizeof(int32_t),
                       cudaMemcpyHostToDevice));
+    }
+    if (kv_slots) {
+        P->bwd_dk = reinterpret_cast<float *>(arena + o_dk);
+        P->bwd_dv = reinterpret_cast<float *>(arena + o_dv);
+        P->bwd_kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
         CK(cudaMemcpy(P->bwd_kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
     }
     std::vector<char> b1 = pack_wl(qwl), b2 = pack_wl(kvwl);
@@ -498,8 +511,8 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
     CUtensorMap mq{}, mk{}, mv{}, mo{};
     if (P->dtype == CQSA_BF16) {
         if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
-        if ((st = make_map(&mk, k, N, H, d)) != CQSA_OK) return st;
-        if ((st = make_map(&mv, v, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mk, k, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mv, v, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
         if ((st = make_map(&mo, dout, N, H, d)) != CQSA_OK) return st;
     }
     CK(launch_bwd_delta(d, P->elem, out, dout, N, H, P->bwd_delta, stream));
@@ -512,6 +525,8 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
     bp.delta = P->bwd_delta;
     bp.N = N;
     bp.H = H;
+    bp.Hkv = pl.spec.Hkv;
+    bp.kv_group = pl.spec.kv_group();
     bp.causal = pl.spec.causal;
     bp.scale = 1.0f / std::sqrt((float)d);
     {
@@ -545,11 +560,13 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
             CK(launch_bwd_dkdv(d, P->elem, p, P->bwd_kvwl.num_units, stream));
         tm.stop();
     }
-    if (!fused) {
+    if (!fused || P->bwd_dk) {
         LaunchTimer tm(P, stream, 1);
-        CK(launch_sum_slots(d, P->elem, P->bwd_dq, P->bwd_q_nslots, pl.block, N, H, dq, stream));
-        CK(launch_sum_slots(d, P->elem, P->bwd_dk, P->bwd_kv_nslots, pl.block, N, H, dk, stream));
-        CK(launch_sum_slots(d, P->elem, P->bwd_dv, P->bwd_kv_nslots, pl.block, N, H, dv, stream));
+        if (!fused) CK(launch_sum_slots(d, P->elem, P->bwd_dq, P->bwd_q_nslots, pl.block, N, H, dq, stream));
+        if (P->bwd_dk) {
+            CK(launch_sum_slots(d, P->elem, P->bwd_dk, P->bwd_kv_nslots, pl.block, N, pl.spec.Hkv, dk, stream));
+            CK(launch_sum_slots(d, P->elem, P->bwd_dv, P->bwd_kv_nslots, pl.block, N, pl.spec.Hkv, dv, stream));
+        }
         tm.stop();
     }
     return CQSA_OK;
@@ -572,6 +589,8 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     const int H = pl.spec.H, d = pl.spec.d, g = P->g;
     const size_t e = (size_t)P->elem;
     const size_t full_row = (size_t)H * d * e, grp_row = (size_t)g * d * e;
+    const int Hkv = pl.spec.Hkv, kvg = pl.spec.kv_group(), gk = pl.spec.kv_heads_of(g);
+    const size_t full_kv_row = (size_t)Hkv * d * e, grp_kv_row = (size_t)gk * d * e;
     const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
                *hv = static_cast<const char *>(v);
     char *ho = static_cast<char *>(out);
@@ -594,15 +613,17 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
             if (t == 0 && it >= 1) CK(cudaStreamWaitEvent(P->s_in, P->ev_in_free[1 - s], 0));
             for (const PoolCopy &c : pl.pool.copies[t]) {
                 const size_t src_off = ((size_t)c.block * B * H + h0) * d * e;
+                const size_t src_kv = ((size_t)c.block * B * Hkv + h0 / kvg) * d * e;
                 const size_t dst_off = (size_t)c.slot * blk_stride * grp_row;
+                const size_t dst_kv = (size_t)c.slot * blk_stride * grp_kv_row;
                 const size_t blk_rows = (size_t)pl.block_rows(c.block);  // the last block may be short
                 if (c.kind == 0) {
                     CK(copy_rows(P->pool_q + dst_off, grp_row, hq + src_off, full_row, grp_row, blk_rows,
                                  cudaMemcpyHostToDevice, P->s_in));
                 } else {
-                    CK(copy_rows(P->pool_k + dst_off, grp_row, hk + src_off, full_row, grp_row, blk_rows,
+                    CK(copy_rows(P->pool_k + dst_kv, grp_kv_row, hk + src_kv, full_kv_row, grp_kv_row, blk_rows,
                                  cudaMemcpyHostToDevice, P->s_in));
-                    CK(copy_rows(P->pool_v + dst_off, grp_row, hv + src_off, full_row, grp_row, blk_rows,
+                    CK(copy_rows(P->pool_v + dst_kv, grp_kv_row, hv + src_kv, full_kv_row, grp_kv_row, blk_rows,
                                  cudaMemcpyHostToDevice, P->s_in));
                 }
             }
@@ -618,6 +639,9 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
             ap.runs = L.wl.runs;
             ap.units = L.wl.units;
             ap.H = g;
+            ap.Hkv = gk;
+            ap.hq_off = h0;
+            ap.hk_off = h0 / kvg;
             ap.epi = EPI_MERGE;
             ap.acc_o = P->acc_o;
             ap.acc_lse = P->acc_lse;
@@ -705,6 +729,7 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
     s.causal = desc->causal ? 1 : 0;
     s.elem_bytes = desc->dtype == CQSA_BF16 ? 2 : 4;
     s.budget = desc->mem_budget_bytes;
+    s.Hkv = desc->H_kv;
     if (desc->merge != CQSA_MERGE_SLOTS && desc->merge != CQSA_MERGE_FUSED)
         return fail(CQSA_ERR_INVALID_ARG, "merge must be CQSA_MERGE_SLOTS or CQSA_MERGE_FUSED");
     s.fused = desc->merge == CQSA_MERGE_FUSED;
@@ -874,6 +899,7 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     const double n = (double)pl.spec.N;
     info->useful_flops = 4.0 * n * n * pl.spec.H * pl.spec.d * (pl.spec.causal ? 0.5 : 1.0);
     info->merge = pl.spec.fused ? CQSA_MERGE_FUSED : CQSA_MERGE_SLOTS;
+    info->H_kv = pl.spec.Hkv;
     return CQSA_OK;
 }
 

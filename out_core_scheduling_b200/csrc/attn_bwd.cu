@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dq_kernel(const BwdParams p)
     const WlUnit u = p.units[blockIdx.x];
     const WlEntry e = p.entries[u.entry];
     const int H = p.H, h = u.head;
+    const int Hkv = p.Hkv, hkv = h / p.kv_group;  // grouped-query attention
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int32_t q0 = u.q0;
     const int32_t q_end = min(q0 + BM, e.q_hi);
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dq_kernel(const BwdParams p)
                 const int rr = idx / D, c = idx % D;
                 const int32_t key = ks + rr;
                 const bool in = key < run.k_hi;
-                const int64_t off = ((int64_t)key * H + h) * D + c;
+                const int64_t off = ((int64_t)key * Hkv + hkv) * D + c;
                 Ks[rr * DP + c] = in ? ld_f32(k, off) : 0.f;
                 Vs[rr * DP + c] = in ? ld_f32(v, off) : 0.f;
             }
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
     const WlUnit u = p.units[blockIdx.x];
     const WlEntry e = p.entries[u.entry];
     const int H = p.H, h = u.head;
+    const int Hkv = p.Hkv, hkv = h / p.kv_group;  // grouped-query attention
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int32_t k0 = u.q0;
     const int32_t k_end = min(k0 + BN, e.q_hi);
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
     for (int idx = tid; idx < BN * D; idx += THREADS) {
         const int r = idx / D, c = idx % D;
         const int32_t row = k0 + r;
-        const int64_t off = ((int64_t)row * H + h) * D + c;
+        const int64_t off = ((int64_t)row * Hkv + hkv) * D + c;
         Ks[r * DP + c] = row < k_end ? ld_f32(k, off) : 0.f;
         Vs[r * DP + c] = row < k_end ? ld_f32(v, off) : 0.f;
     }
@@ -310,7 +312,9 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
         }
     }
 
-    const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
+    // Direct writes only when one query head owns the key/value head.
+    const bool direct = p.kv_group == 1 && (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
+    const int64_t slot = (int64_t)e.slot * p.kv_group + h % p.kv_group;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int32_t row = k0 + ty * 4 + i;
@@ -319,12 +323,12 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
 #pragma unroll
         for (int jj = 0; jj < NJ; ++jj) {
             const int c = tx + 16 * jj;
-            const int64_t o = (orow * H + h) * D + c;
-            if (fused) {
+            const int64_t o = (orow * Hkv + hkv) * D + c;
+            if (direct) {
                 st_out(static_cast<T *>(p.out_a), o, gk[i][jj] * p.scale);
                 st_out(static_cast<T *>(p.out_b), o, gv[i][jj]);
             } else {
-                const int64_t po = (int64_t)e.slot * p.N * H * D + o;
+                const int64_t po = slot * p.N * Hkv * D + o;
                 p.part_a[po] = gk[i][jj] * p.scale;
                 p.part_b[po] = gv[i][jj];
             }

@@ -179,8 +179,8 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     }
                     mbar_expect_tx(&s.kv_full[st], 2 * TILE);
                     for (int kb = 0; kb < KB; ++kb) {
-                        tma_load_3d(s.k[st][kb], &tmK, &s.kv_full[st], kb * 64, head, ks);
-                        tma_load_3d(s.v[st][kb], &tmV, &s.kv_full[st], kb * 64, head, ks);
+                        tma_load_3d(s.k[st][kb], &tmK, &s.kv_full[st], kb * 64, head / p.kv_group, ks);
+                        tma_load_3d(s.v[st][kb], &tmV, &s.kv_full[st], kb * 64, head / p.kv_group, ks);
                     }
                 }
             }
@@ -407,8 +407,8 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         if (lane == 0) {
             mbar_expect_tx(&s.bar_kv, 2 * TILE);
             for (int kb = 0; kb < KB; ++kb) {
-                tma_load_3d(s.k[kb], &tmK, &s.bar_kv, kb * 64, head, k0);
-                tma_load_3d(s.v[kb], &tmV, &s.bar_kv, kb * 64, head, k0);
+                tma_load_3d(s.k[kb], &tmK, &s.bar_kv, kb * 64, head / p.kv_group, k0);
+                tma_load_3d(s.v[kb], &tmV, &s.bar_kv, kb * 64, head / p.kv_group, k0);
             }
         }
         int i = 0;
@@ -559,8 +559,12 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
         if (ok) {
             tc_fence_after();
-            const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
+            // Direct writes only when one query head owns the key/value head;
+            // otherwise each query head of the group has its own slot.
+            const bool fused = p.kv_group == 1 && (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
             const int64_t orow = (int64_t)e.out_lo + (k_local - e.q_lo);
+            const int hkv = head / p.kv_group;
+            const int64_t slot = (int64_t)e.slot * p.kv_group + head % p.kv_group;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t col = which == 0 ? COL_DK : COL_DV;
@@ -574,7 +578,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     if (!valid) continue;
                     if (fused) {
                         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? p.out_a : p.out_b) +
-                                             (orow * p.H + head) * D;
+                                             (orow * p.Hkv + hkv) * D;
 #pragma unroll
                         for (int x = 0; x < 32; x += 4) {
                             uint2 w;
@@ -583,8 +587,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                             *reinterpret_cast<uint2 *>(dst + cc * 32 + x) = w;
                         }
                     } else {
-                        float *dst = (which == 0 ? p.part_a : p.part_b) +
-                                     (((int64_t)e.slot * p.N + orow) * p.H + head) * D;
+                        float *dst = (which == 0 ? p.part_a : p.part_b) + ((slot * p.N + orow) * p.Hkv + hkv) * D;
 #pragma unroll
                         for (int x = 0; x < 32; x += 4)
                             *reinterpret_cast<float4 *>(dst + cc * 32 + x) =

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(simt::THREADS)
     const WlEntry e = p.entries[u.entry];
     const int H = p.H;
     const int h = u.head;
+    const int hkv = (h + p.hq_off) / p.kv_group - p.hk_off;  // grouped-query attention
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const int32_t q0 = u.q0;
     const int32_t q_end = min(q0 + BM, e.q_hi);
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(simt::THREADS)
                 const int rr = idx / D, c = idx % D;
                 const int32_t key = ks + rr;
                 const bool in = key < run.k_hi;
-                const int64_t off = ((int64_t)key * H + h) * D + c;
+                const int64_t off = ((int64_t)key * p.Hkv + hkv) * D + c;
                 Ks[rr * DP + c] = in ? to_f32(k[off]) : 0.f;
                 Vs[rr * D + c] = in ? to_f32(v[off]) : 0.f;
             }

@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const WlEntry e = p.entries[u.entry];
     const int32_t q0 = u.q0;
     const int head = u.head;
+    const int kv_head = (head + p.hq_off) / p.kv_group - p.hk_off;  // grouped-query attention
     const int32_t q_end = min(q0 + QT * BM, e.q_hi);
     const int causal = p.causal;
     const uint64_t tmo = p.timeout_ns;
@@ -192,12 +193,12 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     if (!mbar_wait(&s.k_empty[st], ph ^ 1u, abort, tmo)) { ok = false; break; }
                     mbar_expect_tx(&s.k_full[st], TILE_BYTES);
                     for (int kb = 0; kb < KB; ++kb)
-                        tma_load_3d(s.k[st][kb], &tmK, &s.k_full[st], kb * 64, head, ks);
+                        tma_load_3d(s.k[st][kb], &tmK, &s.k_full[st], kb * 64, kv_head, ks);
                     ++jk;
                     if (!mbar_wait(&s.v_empty[st], ph ^ 1u, abort, tmo)) { ok = false; break; }
                     mbar_expect_tx(&s.v_full[st], TILE_BYTES);
                     for (int kb = 0; kb < KB; ++kb)
-                        tma_load_3d(s.v[st][kb], &tmV, &s.v_full[st], kb * 64, head, ks);
+                        tma_load_3d(s.v[st][kb], &tmV, &s.v_full[st], kb * 64, kv_head, ks);
                     ++jv;
                 }
             }

@@ -27,7 +27,15 @@ struct AttnParams {
     float *part_o;
     float *part_lse;
     int64_t part_rows;
-    int H;              // heads of the tensors the kernel reads
+    int H;              // query heads of the tensors the kernel reads
+    // Grouped-query attention: query head h reads key/value head
+    // (h + hq_off) / kv_group - hk_off of tensors with Hkv heads (device
+    // mode: hq_off = hk_off = 0; a streamed head group: its first query head
+    // and the pool's first key/value head).  kv_group = 1, Hkv = H without.
+    int Hkv;
+    int kv_group;
+    int hq_off;
+    int hk_off;
     int causal;
     float scale_log2;   // log2(e) / sqrt(d)
     float scale;        // 1 / sqrt(d)
@@ -59,6 +67,11 @@ cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k
 // part_* ([slot][N][H][d] fp32); an entry flagged SEG_FIRST | SEG_LAST
 // (fused plans) writes its finished rows to out* in the input dtype.
 struct BwdParams {
+    // Grouped-query attention: query head h uses key/value head h / kv_group
+    // of Hkv; dk / dv partials of the group's query heads go to slots
+    // e.slot * kv_group + h % kv_group ([slot][N][Hkv][d]).
+    int Hkv;
+    int kv_group;
     const WlEntry *entries;
     const WlRun *runs;
     const WlUnit *units;

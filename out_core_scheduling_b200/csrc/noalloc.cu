@@ -185,6 +185,8 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     const int H = pl.spec.H, d = pl.spec.d;
     const int rows = unit_rows_for(elem), bn = key_tile_for(elem);
     if (pl.max_slots > 32) return err(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
+    if (pl.spec.Hkv != pl.spec.H)
+        return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes as many key/value heads as query heads");
 
     // Layout inside the scratch array; reject what does not fit.
     const ListSizes n = count_list(pl, rows, bn);
@@ -230,6 +232,8 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     NA_CK(cudaMemcpyAsync(scratch + o_wl, g_host_list, list_bytes, cudaMemcpyHostToDevice, s));
 
     AttnParams ap{};
+    ap.Hkv = H;        // one key/value head per query head (checked above)
+    ap.kv_group = 1;
     ap.entries = reinterpret_cast<const WlEntry *>(scratch + o_wl + list_e);
     ap.runs = reinterpret_cast<const WlRun *>(scratch + o_wl + list_r);
     ap.units = reinterpret_cast<const WlUnit *>(scratch + o_wl + list_u);

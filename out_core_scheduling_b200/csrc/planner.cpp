@@ -72,6 +72,9 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     if (s.N <= 0 || s.H <= 0 || s.d <= 0) return "N, H and d must be positive";
     if (s.levels < 1 || s.levels > kMaxLevels) return "levels must be in 1..4";
     if (s.N > (int64_t)INT32_MAX) return "N must be below 2^31";
+    if (s.Hkv < 0 || (s.Hkv > 0 && s.H % s.Hkv != 0))
+        return "the query heads must be a multiple of the key/value heads";
+    if (spec.Hkv == 0) spec.Hkv = s.H;
     levels.clear();
     num_blocks = 1;
     for (int i = 0; i < s.levels; ++i) {
@@ -549,13 +552,14 @@ size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
     const int64_t N = spec.N, R = max_task_rows;
     const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
     const size_t blk = (size_t)block * g * dd * e;
+    const size_t blk_kv = (size_t)block * spec.kv_heads_of(g) * dd * e;  // fewer heads under GQA
     ArenaLayout a;
     a.take(256);                                        // error word
     a.take((size_t)N * g * dd * sizeof(float));         // accumulator O
     a.take((size_t)g * N * sizeof(float));              // accumulator lse
     a.take((size_t)pl.q_slots * blk);                   // Q block pool
-    a.take((size_t)pl.kv_slots * blk);                  // K block pool
-    a.take((size_t)pl.kv_slots * blk);                  // V block pool
+    a.take((size_t)pl.kv_slots * blk_kv);               // K block pool
+    a.take((size_t)pl.kv_slots * blk_kv);               // V block pool
     for (int s = 0; s < 2; ++s) {
         a.take((size_t)R * g * dd * e);                 // finished out rows
         a.take((size_t)g * R * sizeof(float));          // finished lse rows
@@ -591,9 +595,13 @@ void Planner::size_plan() {
     span(nq, &min_q_slots, &full_q_slots);
     span(nkv, &min_kv_slots, &full_kv_slots);
 
+    const int kvg = spec.kv_group();
     for (int g = spec.H; g >= 1; --g) {
         if (spec.H % g) continue;
+        // A head group covers whole key/value groups, or lies inside one.
+        if (g % kvg != 0 && kvg % g != 0) continue;
         const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
+        const size_t blk_kv = (size_t)block * spec.kv_heads_of(g) * spec.d * spec.elem_bytes;
         int64_t qs = full_q_slots, kvs = full_kv_slots;
         PoolPlan pp;
         if (!plan_pool(qs, kvs, &pp)) continue;
@@ -603,7 +611,8 @@ void Planner::size_plan() {
             // until the arena fits, never below what a task pair needs.
             while (bytes > spec.budget && (qs > min_q_slots || kvs > min_kv_slots)) {
                 const size_t over = bytes - spec.budget;
-                int64_t drop_kv = std::min<int64_t>(kvs - min_kv_slots, (int64_t)((over + 2 * blk - 1) / (2 * blk)));
+                int64_t drop_kv =
+                    std::min<int64_t>(kvs - min_kv_slots, (int64_t)((over + 2 * blk_kv - 1) / (2 * blk_kv)));
                 int64_t drop_q = 0;
                 if (drop_kv <= 0) drop_q = std::min<int64_t>(qs - min_q_slots, (int64_t)((over + blk - 1) / blk));
                 if (drop_kv <= 0 && drop_q <= 0) break;
@@ -619,7 +628,7 @@ void Planner::size_plan() {
         sizing.q_slots = qs;
         sizing.kv_slots = kvs;
         const size_t groups = (size_t)(spec.H / g);
-        sizing.h2d = ((size_t)pp.q_copies + 2 * (size_t)pp.kv_copies) * blk * groups;
+        sizing.h2d = ((size_t)pp.q_copies * blk + 2 * (size_t)pp.kv_copies * blk_kv) * groups;
         pool = std::move(pp);
         break;
     }

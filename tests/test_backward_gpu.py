@@ -117,3 +117,32 @@ def test_backward_rejects_host_mode():
 def test_backward_ragged_n(case, causal, merge):
     N, H, d, ls, dtype = case
     _check_all(N, H, d, ls, dtype, causal, merge, seed=31)
+
+
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", [(7 * 128, 4, 2, 128, [3], torch.bfloat16), (13 * 64, 4, 1, 64, [4], torch.bfloat16),
+                                  (700, 4, 2, 64, [3], torch.float32)],
+                         ids=lambda c: f"n{c[0]}-h{c[1]}-kv{c[2]}-d{c[3]}-{str(c[5])[6:]}")
+def test_backward_grouped_query(case, causal, merge):
+    """dk, dv of a key/value head sum the gradients of its query heads."""
+    N, H, Hkv, d, ls, dtype = case
+    g = H // Hkv
+    q = make_qkv(N, H, d, dtype=dtype, seed=60, device=DEV)[0]
+    _, k, v = make_qkv(N, Hkv, d, dtype=dtype, seed=61, device=DEV)
+    dout = make_qkv(N, H, d, dtype=dtype, seed=62, device=DEV)[0]
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, merge=merge, H_kv=Hkv)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    dq = torch.empty_like(q)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    plan.sync()
+    ke = k.repeat_interleave(g, dim=1).contiguous()
+    ve = v.repeat_interleave(g, dim=1).contiguous()
+    qc, kc, vc, dc = (x.cpu() for x in (q, ke, ve, dout))
+    ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
+    ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, causal=causal)
+    _compare(dq, ref_dq, dtype, "dq")
+    _compare(dk, ref_dk.reshape(N, Hkv, g, d).sum(2), dtype, "dk")
+    _compare(dv, ref_dv.reshape(N, Hkv, g, d).sum(2), dtype, "dv")

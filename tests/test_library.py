@@ -230,3 +230,25 @@ def test_forward_without_device_reports_no_device():
     with pytest.raises(cqsa.CqsaError) as ei:
         cqsa.cqsa_forward(plan, x, x, x, x.clone(), lse, cqsa.CQSA_DEVICE, stream=0)
     assert ei.value.status == cqsa.CQSA_ERR_NO_DEVICE
+
+
+def test_grouped_query_plans():
+    """H_kv key/value heads: head groups cover whole key/value groups or lie
+    inside one, and the streamed path copies only the groups' K/V heads."""
+    N, H, d = 13 * 256, 8, 128
+    mha = cqsa.cqsa_plan_ex(N, H, d, [4]).info()
+    gqa = cqsa.cqsa_plan_ex(N, H, d, [4], H_kv=2).info()
+    assert gqa["H_kv"] == 2 and mha["H_kv"] == H
+    # Each input once: Q with H heads, K and V with 2.
+    assert gqa["h2d_bytes"] == N * H * d * 2 + 2 * N * 2 * d * 2
+    assert gqa["host_arena_bytes"] < mha["host_arena_bytes"]
+    for budget_frac in (0.5, 0.3):
+        try:
+            p = cqsa.cqsa_plan_ex(N, H, d, [4], H_kv=2, mem_budget_bytes=int(gqa["host_arena_bytes"] * budget_frac))
+        except cqsa.CqsaError:
+            continue
+        g = p.info()["head_group"]
+        assert g == 0 or g % 4 == 0 or 4 % g == 0
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_plan_ex(N, H, d, [4], H_kv=3)
+    assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG

@@ -279,3 +279,50 @@ def test_ragged_n_streamed(case, causal):
     plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, mem_budget_bytes=budget)
     out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
     check(out, lse, q, k, v, np.arange(N), causal)
+
+
+# ---------------------------------------------------------------- grouped-query attention
+def _expand(x, group):
+    return x.repeat_interleave(group, dim=1).contiguous()
+
+
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", [(7 * 256, 4, 2, 128, [3], torch.bfloat16), (13 * 200, 8, 1, 64, [4], torch.bfloat16),
+                                  (1000, 4, 2, 64, [3], torch.float32)],
+                         ids=lambda c: f"n{c[0]}-h{c[1]}-kv{c[2]}-d{c[3]}-{str(c[5])[6:]}")
+def test_grouped_query_device(case, causal, merge):
+    N, H, Hkv, d, ls, dtype = case
+    q = make_qkv(N, H, d, dtype=dtype, seed=50, device=DEV)[0]
+    _, k, v = make_qkv(N, Hkv, d, dtype=dtype, seed=51, device=DEV)
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, merge=merge, H_kv=Hkv)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, _expand(k, H // Hkv), _expand(v, H // Hkv), np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("frac", [1.0, 0.0], ids=["full", "tight"])
+def test_grouped_query_streamed(causal, frac):
+    """Head groups larger than a key/value group (full budget) and inside one
+    (tightest budget)."""
+    N, H, Hkv, d = 13 * 256, 8, 2, 128
+    q = make_qkv(N, H, d, dtype=torch.bfloat16, seed=52, device=DEV)[0]
+    _, k, v = make_qkv(N, Hkv, d, dtype=torch.bfloat16, seed=53, device=DEV)
+    q, k, v = (x.cpu().pin_memory() for x in (q, k, v))
+    torch.cuda.empty_cache()
+    if frac == 1.0:
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, H_kv=Hkv)
+    else:
+        lo, hi = 0, cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, H_kv=Hkv).info()["host_arena_bytes"]
+        while hi - lo > (1 << 18):
+            mid = (lo + hi) // 2
+            try:
+                ok = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, H_kv=Hkv, mem_budget_bytes=mid).info()["head_group"] > 0
+            except cqsa.CqsaError:
+                ok = False
+            lo, hi = (lo, mid) if ok else (mid, hi)
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, H_kv=Hkv, mem_budget_bytes=hi)
+        assert plan.info()["head_group"] < H // Hkv  # inside one key/value group
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, _expand(k, H // Hkv), _expand(v, H // Hkv), np.arange(N), causal)
