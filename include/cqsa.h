@@ -95,6 +95,9 @@ typedef struct {
     int H_kv;  /* key/value heads (grouped-query attention): H must be a
                   multiple; query head h reads key/value head h / (H / H_kv).
                   0 = H.  k, v (and dk, dv) are then [N, H_kv, d]. */
+    int B;     /* independent sequences per call (0 or 1: one): tensors are
+                  [B, N, heads, d] and lse [B, H, N]; the sequences run one
+                  after another through the plan on the call's stream. */
 } cqsa_plan_desc_t;
 
 /* What a plan decided (for logging, tests and the benchmark). */
@@ -118,6 +121,7 @@ typedef struct {
     double useful_flops;                /* 4 N^2 H d, halved when causal */
     int merge;                          /* cqsa_merge_t of device-mode forwards */
     int H_kv;                           /* key/value heads */
+    int B;                              /* sequences per call */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */

@@ -51,7 +51,8 @@ class PlanDesc(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
                 ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int), ("H_kv", ctypes.c_int)]
+                ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int), ("H_kv", ctypes.c_int),
+                ("B", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -65,7 +66,7 @@ class PlanInfo(ctypes.Structure):
                 ("head_group", ctypes.c_int), ("device_arena_bytes", ctypes.c_size_t),
                 ("host_arena_bytes", ctypes.c_size_t), ("h2d_bytes", ctypes.c_size_t),
                 ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double),
-                ("merge", ctypes.c_int), ("H_kv", ctypes.c_int)]
+                ("merge", ctypes.c_int), ("H_kv", ctypes.c_int), ("B", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -212,7 +213,7 @@ def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = Fa
 
 
 def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
-                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0) -> Plan:
+                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0, B: int = 1) -> Plan:
     desc = PlanDesc()
     desc.N, desc.H, desc.d = N, H, d
     desc.levels = len(ls)
@@ -223,17 +224,20 @@ def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = 
     desc.mem_budget_bytes = mem_budget_bytes
     desc.merge = merge
     desc.H_kv = H_kv
+    desc.B = B
     h = ctypes.c_void_p()
     _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
     return Plan(h.value)
 
 
 def _check_shapes(plan: Plan, qlike, kvlike, lse):
-    """Tensors against the plan: query-shaped [N, H, d], key/value-shaped
-    [N, H_kv, d] (H_kv = H without grouped-query attention), lse [H, N]."""
+    """Tensors against the plan: query-shaped [B, N, H, d], key/value-shaped
+    [B, N, H_kv, d] (H_kv = H without grouped-query attention), lse
+    [B, H, N]; with B = 1 the leading dimension may be left out."""
     import torch
     info = plan.info()
-    N, H, d, Hkv = info["N"], info["H"], info["d"], info["H_kv"]
+    N, H, d, Hkv, B = info["N"], info["H"], info["d"], info["H_kv"], info["B"]
+    lead = (B,) if B > 1 else ()
     named = list(qlike) + list(kvlike) + [("lse", lse)]
     for name, t in named:
         if not isinstance(t, torch.Tensor) or not t.is_contiguous():
@@ -242,14 +246,16 @@ def _check_shapes(plan: Plan, qlike, kvlike, lse):
         raise ValueError("lse must be float32")
     if len({t.dtype for _, t in list(qlike) + list(kvlike)}) != 1:
         raise ValueError(", ".join(n for n, _ in list(qlike) + list(kvlike)) + " must share a dtype")
+    def shape_ok(t, want):
+        return tuple(t.shape) == lead + want or (B == 1 and tuple(t.shape) == (1,) + want)
     for name, t in qlike:
-        if tuple(t.shape) != (N, H, d):
-            raise ValueError(f"{name} must be [N, H, d] = {(N, H, d)}")
+        if not shape_ok(t, (N, H, d)):
+            raise ValueError(f"{name} must be {lead + (N, H, d)}")
     for name, t in kvlike:
-        if tuple(t.shape) != (N, Hkv, d):
-            raise ValueError(f"{name} must be [N, H_kv, d] = {(N, Hkv, d)}")
-    if tuple(lse.shape) != (H, N):
-        raise ValueError("lse must be [H, N]")
+        if not shape_ok(t, (N, Hkv, d)):
+            raise ValueError(f"{name} must be {lead + (N, Hkv, d)}")
+    if not shape_ok(lse, (H, N)):
+        raise ValueError(f"lse must be {lead + (H, N)}")
 
 
 def cqsa_forward(plan: Plan, q, k, v, out, lse, host_or_device: int = CQSA_DEVICE, stream=None):

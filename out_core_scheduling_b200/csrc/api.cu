@@ -730,6 +730,7 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
     s.elem_bytes = desc->dtype == CQSA_BF16 ? 2 : 4;
     s.budget = desc->mem_budget_bytes;
     s.Hkv = desc->H_kv;
+    s.B = desc->B > 0 ? desc->B : 1;
     if (desc->merge != CQSA_MERGE_SLOTS && desc->merge != CQSA_MERGE_FUSED)
         return fail(CQSA_ERR_INVALID_ARG, "merge must be CQSA_MERGE_SLOTS or CQSA_MERGE_FUSED");
     s.fused = desc->merge == CQSA_MERGE_FUSED;
@@ -794,7 +795,20 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
     for (int i = 0; i < 5; ++i)
         if ((st = check_ptr(ptrs[i], host, names[i])) != CQSA_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return host ? forward_host(plan, q, k, v, out, lse, s) : forward_device(plan, q, k, v, out, lse, s);
+    // A batch is B independent sequences; each runs through the plan in
+    // turn on the caller's stream (the arena is reused).
+    const Planner &pl = plan->pl;
+    const size_t e = (size_t)plan->elem, N = (size_t)pl.spec.N, d = (size_t)pl.spec.d;
+    const size_t qs = N * pl.spec.H * d * e, kvs = N * pl.spec.Hkv * d * e, ls = N * pl.spec.H;
+    for (int b = 0; b < pl.spec.B; ++b) {
+        const char *qb = static_cast<const char *>(q) + b * qs, *kb = static_cast<const char *>(k) + b * kvs,
+                   *vb = static_cast<const char *>(v) + b * kvs;
+        char *ob = static_cast<char *>(out) + b * qs;
+        float *lb = lse + b * ls;
+        st = host ? forward_host(plan, qb, kb, vb, ob, lb, s) : forward_device(plan, qb, kb, vb, ob, lb, s);
+        if (st != CQSA_OK) return st;
+    }
+    return CQSA_OK;
 }
 
 cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, const void *out,
@@ -810,7 +824,17 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
     const char *names[] = {"q", "k", "v", "out", "lse", "dout", "dq", "dk", "dv"};
     for (int i = 0; i < 9; ++i)
         if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
-    return backward_device(plan, q, k, v, out, lse, dout, dq, dk, dv, static_cast<cudaStream_t>(stream));
+    const Planner &pl = plan->pl;
+    const size_t e = (size_t)plan->elem, N = (size_t)pl.spec.N, d = (size_t)pl.spec.d;
+    const size_t qs = N * pl.spec.H * d * e, kvs = N * pl.spec.Hkv * d * e, ls = N * pl.spec.H;
+    for (int b = 0; b < pl.spec.B; ++b) {
+        auto at = [&](const void *p, size_t stride) { return static_cast<const char *>(p) + b * stride; };
+        auto atw = [&](void *p, size_t stride) { return static_cast<char *>(p) + b * stride; };
+        st = backward_device(plan, at(q, qs), at(k, kvs), at(v, kvs), at(out, qs), lse + b * ls, at(dout, qs),
+                             atw(dq, qs), atw(dk, kvs), atw(dv, kvs), static_cast<cudaStream_t>(stream));
+        if (st != CQSA_OK) return st;
+    }
+    return CQSA_OK;
 }
 
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
@@ -897,9 +921,10 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->h2d_bytes = pl.sizing.h2d;
     info->d2h_bytes = pl.sizing.d2h;
     const double n = (double)pl.spec.N;
-    info->useful_flops = 4.0 * n * n * pl.spec.H * pl.spec.d * (pl.spec.causal ? 0.5 : 1.0);
+    info->useful_flops = 4.0 * n * n * pl.spec.H * pl.spec.d * (pl.spec.causal ? 0.5 : 1.0) * pl.spec.B;
     info->merge = pl.spec.fused ? CQSA_MERGE_FUSED : CQSA_MERGE_SLOTS;
     info->H_kv = pl.spec.Hkv;
+    info->B = pl.spec.B;
     return CQSA_OK;
 }
 

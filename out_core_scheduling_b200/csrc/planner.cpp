@@ -75,6 +75,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     if (s.Hkv < 0 || (s.Hkv > 0 && s.H % s.Hkv != 0))
         return "the query heads must be a multiple of the key/value heads";
     if (spec.Hkv == 0) spec.Hkv = s.H;
+    if (s.B < 1) return "the batch B must be at least 1";
     levels.clear();
     num_blocks = 1;
     for (int i = 0; i < s.levels; ++i) {
@@ -633,6 +634,9 @@ void Planner::size_plan() {
         break;
     }
     sizing.d2h = (size_t)spec.N * spec.H * spec.d * spec.elem_bytes + (size_t)spec.H * spec.N * sizeof(float);
+    // A call runs the B sequences one after another on the same plan.
+    sizing.h2d *= (size_t)spec.B;
+    sizing.d2h *= (size_t)spec.B;
 }
 
 }  // namespace cqsa

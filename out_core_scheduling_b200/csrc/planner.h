@@ -64,6 +64,7 @@ struct PlanSpec {
     size_t budget = 0;                      // 0 = unlimited
     int fused = 0;                          // device mode: merge in the kernel, no partial slots
     int Hkv = 0;                            // key/value heads (grouped-query attention); 0 = H
+    int B = 1;                              // independent sequences of N tokens per call
     int kv_group() const { return H / (Hkv > 0 ? Hkv : H); }
     // Key/value heads a streamed head group of g query heads reads.
     int kv_heads_of(int g) const { return g >= kv_group() ? g / kv_group() : 1; }

@@ -146,3 +146,25 @@ def test_backward_grouped_query(case, causal, merge):
     _compare(dq, ref_dq, dtype, "dq")
     _compare(dk, ref_dk.reshape(N, Hkv, g, d).sum(2), dtype, "dk")
     _compare(dv, ref_dv.reshape(N, Hkv, g, d).sum(2), dtype, "dv")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_batch_of_sequences(causal):
+    B, N, H, d = 2, 7 * 96, 2, 64
+    q = torch.stack([make_qkv(N, H, d, dtype=torch.bfloat16, seed=90 + b, device=DEV)[0] for b in range(B)])
+    k = torch.stack([make_qkv(N, H, d, dtype=torch.bfloat16, seed=92 + b, device=DEV)[1] for b in range(B)])
+    v = torch.stack([make_qkv(N, H, d, dtype=torch.bfloat16, seed=94 + b, device=DEV)[2] for b in range(B)])
+    dout = torch.stack([make_qkv(N, H, d, dtype=torch.bfloat16, seed=96 + b, device=DEV)[0] for b in range(B)])
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, B=B)
+    out, lse = torch.empty_like(q), torch.empty(B, H, N, device=DEV)
+    cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    plan.sync()
+    for b in range(B):
+        qc, kc, vc, dc = (x[b].cpu() for x in (q, k, v, dout))
+        ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
+        ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, causal=causal)
+        _compare(dq[b], ref_dq, torch.bfloat16, "dq")
+        _compare(dk[b], ref_dk, torch.bfloat16, "dk")
+        _compare(dv[b], ref_dv, torch.bfloat16, "dv")

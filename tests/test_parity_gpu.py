@@ -326,3 +326,33 @@ def test_grouped_query_streamed(causal, frac):
         assert plan.info()["head_group"] < H // Hkv  # inside one key/value group
     out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
     check(out, lse, q, _expand(k, H // Hkv), _expand(v, H // Hkv), np.arange(N), causal)
+
+
+# ---------------------------------------------------------------- batches
+@pytest.mark.parametrize("mode,merge", [(cqsa.CQSA_DEVICE, cqsa.CQSA_MERGE_SLOTS), (cqsa.CQSA_DEVICE, cqsa.CQSA_MERGE_FUSED),
+                                        (cqsa.CQSA_HOST, cqsa.CQSA_MERGE_SLOTS)], ids=["slots", "fused", "streamed"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_batch_of_sequences(mode, merge, causal):
+    """B independent sequences in one call; each equals its own attention."""
+    B, N, H, Hkv, d = 3, 7 * 100, 4, 2, 128
+    qs, ks, vs = [], [], []
+    for b in range(B):
+        qs.append(make_qkv(N, H, d, dtype=torch.bfloat16, seed=70 + b, device=DEV)[0])
+        _, kb, vb = make_qkv(N, Hkv, d, dtype=torch.bfloat16, seed=80 + b, device=DEV)
+        ks.append(kb)
+        vs.append(vb)
+    q, k, v = torch.stack(qs), torch.stack(ks), torch.stack(vs)
+    if mode == cqsa.CQSA_HOST:
+        q, k, v = (x.cpu().pin_memory() for x in (q, k, v))
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, merge=merge, H_kv=Hkv, B=B)
+    assert plan.info()["B"] == B
+    if mode == cqsa.CQSA_DEVICE:
+        out = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device=DEV)
+    else:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        lse = torch.empty(B, H, N).pin_memory()
+    cqsa.cqsa_forward(plan, q, k, v, out, lse, mode)
+    plan.sync()
+    for b in range(B):
+        check(out[b], lse[b], q[b], _expand(k[b], H // Hkv), _expand(v[b], H // Hkv), np.arange(N), causal)
