@@ -250,6 +250,11 @@ def run_ours(args, W):
     if args.profile_run:
         for _ in range(args.steps):
             step()
+        if args.profile_backward and mode == cqsa.CQSA_DEVICE:
+            dout = make_qkv(N, H, d, dtype=tdt, seed=1000 + D.rank, device=q.device, dist=W["dist"])[0]
+            grads = tuple(torch.empty_like(q) for _ in range(3))
+            for _ in range(args.steps):  # first variant only: one backward arena on the device
+                cqsa.cqsa_backward(plans[0], q, k, v, outs[0], lses[0], dout, *grads, stream=stream)
         for p in plans:
             p.sync(stream)
         D.close()
@@ -646,6 +651,8 @@ def main(argv=None):
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing of device workloads")
     ap.add_argument("--profile-run", action="store_true",
                     help="only warm-up + steps of the device path (for ncu captures)")
+    ap.add_argument("--profile-backward", action="store_true",
+                    help="with --profile-run: the first variant's backward after the forward steps")
     args = ap.parse_args(argv)
     if args.warmup < 0 or args.steps < 1:
         ap.error("need --steps >= 1 and --warmup >= 0")
