@@ -13,10 +13,13 @@
 //                      entry; per allowed query tile: S^T = K Q^T and
 //                      dP^T = V dO^T, P^T and dS^T in bf16 written over
 //                      them, then dV += P^T dO and dK += dS^T Q.
-// Warp roles (192 threads): warps 0-3 the elementwise step (one TMEM lane,
-// i.e. one stationary row, per thread), warp 4 TMA, warp 5 MMA.  Every wait
-// is bounded; on a timeout the CTA records DEV_TIMEOUT, drains its copies and
-// MMAs, frees its tensor memory and returns.
+// Warp roles (320 threads): warps 0-7 the elementwise step (one TMEM lane,
+// i.e. one stationary row, per thread; the two warps of a lane quarter take
+// the tile's columns 0-63 and 64-127), warp 8 TMA, warp 9 MMA.  Each warp
+// writes its packed bf16 results over its own half of the fp32 columns, so
+// the two never touch each other's columns.  Every wait is bounded; on a
+// timeout the CTA records DEV_TIMEOUT, drains its copies and MMAs, frees its
+// tensor memory and returns.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -29,24 +32,35 @@ namespace btc {
 constexpr int BM = 128;           // stationary rows per CTA
 constexpr int BN = 128;           // rows of an iterated tile
 constexpr int STAGES = 2;
-constexpr int THREADS = 192;
-constexpr int WARP_TMA = 4;
-constexpr int WARP_MMA = 5;
+constexpr int EW_WARPS = 8;       // elementwise warps, two per TMEM lane quarter
+constexpr int THREADS = (EW_WARPS + 2) * 32;
+constexpr int WARP_TMA = EW_WARPS;
+constexpr int WARP_MMA = EW_WARPS + 1;
+constexpr int HALF = BN / 2;      // columns of a tile per elementwise warp
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizzle
 constexpr float LOG2E = 1.4426950408889634f;
+
+// K and V of the dq kernel have their own stages: V(j) is free once dP(j) is
+// done, K(j) only after dQ(j), so K gets one stage more to keep its copy off
+// the critical path.
+constexpr int KST = 3;
+constexpr int VST = 2;
 
 template <int D>
 struct SmemDq {
     static constexpr int KB = D / 64;
     alignas(1024) uint8_t q[KB][BOX_BYTES];
     alignas(1024) uint8_t dout[KB][BOX_BYTES];
-    alignas(1024) uint8_t k[STAGES][KB][BOX_BYTES];
-    alignas(1024) uint8_t v[STAGES][KB][BOX_BYTES];
-    uint64_t bar_q, kv_full[STAGES], kv_empty[STAGES], s_full, dp_free, p_half, p_full, o_full, drain;
+    alignas(1024) uint8_t k[KST][KB][BOX_BYTES];
+    alignas(1024) uint8_t v[VST][KB][BOX_BYTES];
+    uint64_t bar_q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full, dp_free, p_half, p_full, o_full,
+        drain;
     uint32_t tmem_base;
     int abort;
 };
+
+static_assert(sizeof(SmemDq<128>) + 1024 <= 232448, "dq shared memory (with alignment slack) over 227 KB");
 
 template <int D>
 struct SmemKv {
@@ -55,12 +69,25 @@ struct SmemKv {
     alignas(1024) uint8_t v[KB][BOX_BYTES];
     alignas(1024) uint8_t q[STAGES][KB][BOX_BYTES];
     alignas(1024) uint8_t dout[STAGES][KB][BOX_BYTES];
-    float lse2[STAGES][BN];  // lse * log2(e) of the tile's query rows (+inf outside the run)
-    float dl[STAGES][BN];    // D of the tile's query rows
-    uint64_t bar_kv, qd_full[STAGES], qd_empty[STAGES], s_full, p_half, p_full, o_full, drain;
+    alignas(16) float lse2[STAGES][BN];  // lse * log2(e) of the tile's query rows (+inf outside the run)
+    alignas(16) float dl[STAGES][BN];    // D of the tile's query rows
+    uint64_t bar_kv, qd_full[STAGES], qd_empty[STAGES], st_full, dp_full, pt_full, ds_full, o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
+
+// Four floats from shared memory, kept in program order (not hoisted ahead
+// of the arithmetic that precedes them, which would raise register pressure).
+__device__ __forceinline__ float4 lds_f4(const float *p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+// TMEM column of S for the dq kernel's key tile j (double-buffered).
+__device__ __forceinline__ uint32_t s_col(int j) { return (j & 1) ? 384u : 0u; }
 
 __device__ __forceinline__ bool warp_wait_b(uint64_t *bar, uint32_t parity, volatile int *abort, uint64_t tmo) {
     bool ok = mbar_wait(bar, parity, abort, tmo);
@@ -98,14 +125,23 @@ __device__ __forceinline__ void mma_rows_dot(uint32_t d_tmem, uint64_t adesc, ui
     }
 }
 
-// TS MMA D[128 x D] (+)= A[128 x 128] (bf16 in TMEM at a_tmem, 2 per column)
-// times B[128 x D] with B's rows the K dimension, stored [rows][D] (MN-major).
-__device__ __forceinline__ void mma_tmem_rows(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                              bool acc, int k0 = 0, int k1 = BN / 16) {
+// TMEM column of the packed bf16 operand for K step kk (16 of the tile's
+// 128 columns): the warp of columns 0-63 packs them into columns 0-31, the
+// warp of columns 64-127 into columns 64-95.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)(kk * 8 + (kk >= 4 ? 32 : 0)); }
+
+// TS MMA D[128 x D] (+)= A B over half h of the K dimension: A[128 x 128]
+// bf16 in TMEM at a_tmem (packed as above), B[128 x D] with B's rows the K
+// dimension, stored [rows][D] (MN-major).  Half 0 is each elementwise warp's
+// first 32 columns (K steps 0, 1, 4, 5), half 1 their second (2, 3, 6, 7).
+__device__ __forceinline__ void mma_tmem_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                              bool acc, int h) {
 #pragma unroll
-    for (int kk = k0; kk < k1; ++kk)
-        mma_ts_elect(d_tmem, a_tmem + (uint32_t)kk * 8u, bdesc + (uint64_t)(kk * (2048 >> 4)), idesc,
-                     (acc || kk > 0) ? 1u : 0u);
+    for (int i = 0; i < 4; ++i) {
+        const int kk = (i >> 1) * 4 + 2 * h + (i & 1);
+        mma_ts_elect(d_tmem, a_tmem + packed_col(kk), bdesc + (uint64_t)(kk * (2048 >> 4)), idesc,
+                     (acc || i > 0) ? 1u : 0u);
+    }
 }
 
 }  // namespace btc
@@ -135,14 +171,18 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&s.bar_q, 1);
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&s.kv_full[i], 1);
-            mbar_init(&s.kv_empty[i], 1);
+        for (int i = 0; i < KST; ++i) {
+            mbar_init(&s.k_full[i], 1);
+            mbar_init(&s.k_empty[i], 1);
+        }
+        for (int i = 0; i < VST; ++i) {
+            mbar_init(&s.v_full[i], 1);
+            mbar_init(&s.v_empty[i], 1);
         }
         mbar_init(&s.s_full, 1);
-        mbar_init(&s.dp_free, 4);
-        mbar_init(&s.p_half, 4);
-        mbar_init(&s.p_full, 4);
+        mbar_init(&s.dp_free, EW_WARPS);
+        mbar_init(&s.p_half, EW_WARPS);
+        mbar_init(&s.p_full, EW_WARPS);
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
         s.abort = 0;
@@ -166,72 +206,88 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 tma_load_3d(s.q[kb], &tmQ, &s.bar_q, kb * 64, head, q0);
                 tma_load_3d(s.dout[kb], &tmO, &s.bar_q, kb * 64, head, q0);
             }
-            int j = 0;
+            int nk = 0, nv = 0;  // K and V tiles requested
             bool ok = true;
             for (int r = 0; r < e.run_count && ok; ++r) {
                 int32_t lo, hi;
                 clip_run(e, p.runs[e.run_begin + r], q_end, causal, &lo, &hi);
-                for (int32_t ks = lo; ks < hi; ks += BN, ++j) {
-                    const int st = j % STAGES;
-                    if (!mbar_wait(&s.kv_empty[st], ((uint32_t)(j / STAGES) & 1u) ^ 1u, abort, tmo)) {
+                for (int32_t ks = lo; ks < hi; ks += BN) {
+                    const int kst = nk % KST, vst = nv % VST;
+                    if (!mbar_wait(&s.k_empty[kst], ((uint32_t)(nk / KST) & 1u) ^ 1u, abort, tmo)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&s.kv_full[st], 2 * TILE);
-                    for (int kb = 0; kb < KB; ++kb) {
-                        tma_load_3d(s.k[st][kb], &tmK, &s.kv_full[st], kb * 64, head / p.kv_group, ks);
-                        tma_load_3d(s.v[st][kb], &tmV, &s.kv_full[st], kb * 64, head / p.kv_group, ks);
+                    mbar_expect_tx(&s.k_full[kst], TILE);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_3d(s.k[kst][kb], &tmK, &s.k_full[kst], kb * 64, head / p.kv_group, ks);
+                    ++nk;
+                    if (!mbar_wait(&s.v_empty[vst], ((uint32_t)(nv / VST) & 1u) ^ 1u, abort, tmo)) {
+                        ok = false;
+                        break;
                     }
+                    mbar_expect_tx(&s.v_full[vst], TILE);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_3d(s.v[vst][kb], &tmV, &s.v_full[vst], kb * 64, head / p.kv_group, ks);
+                    ++nv;
                 }
             }
             if (!ok) {
+                // Wait for the copies in flight (the latest phase of each stage).
                 atomicExch(err, DEV_TIMEOUT);
                 int zero = 0;
                 mbar_wait(&s.bar_q, 0, (volatile int *)&zero, tmo);
-                for (int i = max(0, j - STAGES); i < j; ++i)
-                    mbar_wait(&s.kv_full[i % STAGES], (uint32_t)(i / STAGES) & 1u, (volatile int *)&zero, tmo);
+                for (int x = max(0, nk - KST); x < nk; ++x)
+                    mbar_wait(&s.k_full[x % KST], (uint32_t)(x / KST) & 1u, (volatile int *)&zero, tmo);
+                for (int x = max(0, nv - VST); x < nv; ++x)
+                    mbar_wait(&s.v_full[x % VST], (uint32_t)(x / VST) & 1u, (volatile int *)&zero, tmo);
             }
         }
     } else if (warp == WARP_MMA) {
-        // Per key tile j: dP(j+1) = dO V(j+1)^T goes in as soon as the
-        // elementwise warps hold dP(j) in registers (its own TMEM columns);
-        // dQ += dS(j) K(j) and S(j+1) = Q K(j+1)^T follow dS(j), in that order
-        // because S(j+1) overwrites the columns dS(j) occupies.
+        // S(j) alternates between TMEM columns 0 and 384, so S(j+1) = Q K(j+1)^T
+        // is computed while the elementwise warps still work on tile j; dP(j+1)
+        // = dO V(j+1)^T goes into the dP columns as soon as they hold dP(j) in
+        // registers.  dQ += dS(j) K(j) reads dS(j) in bf16 over S(j), in two
+        // halves.  S(j+1) lands in the columns of dS(j-1), whose dQ MMAs were
+        // issued before it.
         bool ok = warp_wait_b(&s.bar_q, 0, abort, tmo);
         const uint64_t qdesc = smem_desc_sw128(smem_u32(s.q[0]), 16, 1024);
         const uint64_t odesc = smem_desc_sw128(smem_u32(s.dout[0]), 16, 1024);
         if (ok && ntiles > 0) {
-            ok = warp_wait_b(&s.kv_full[0], 0, abort, tmo);
+            ok = warp_wait_b(&s.k_full[0], 0, abort, tmo) && warp_wait_b(&s.v_full[0], 0, abort, tmo);
             if (ok) {
                 tc_fence_after();
                 mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[0][0]), 16, 1024), IDESC_SS);
                 mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[0][0]), 16, 1024), IDESC_SS);
+                mma_commit_elect(&s.v_empty[0]);
                 mma_commit_elect(&s.s_full);
             }
         }
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int st = j % STAGES, st1 = (j + 1) % STAGES;
-            const bool has_next = j + 1 < ntiles;
-            if (has_next) {
-                if (!warp_wait_b(&s.kv_full[st1], (uint32_t)((j + 1) / STAGES) & 1u, abort, tmo)) { ok = false; break; }
-                if (!warp_wait_b(&s.dp_free, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            const int j1 = j + 1;
+            if (j1 < ntiles) {
+                if (!warp_wait_b(&s.k_full[j1 % KST], (uint32_t)(j1 / KST) & 1u, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
-                mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[st1][0]), 16, 1024), IDESC_SS);
-            }
-            // dS(j) arrives in two halves of 64 keys: the first half of dQ
-            // runs while the elementwise warps finish the second.
-            const uint64_t kb = smem_desc_sw128(smem_u32(s.k[st][0]), BOX_BYTES, 1024);
-            if (!warp_wait_b(&s.p_half, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
-            tc_fence_after();
-            mma_tmem_rows(tmem + 256u, tmem, kb, IDESC_TS, j > 0, 0, BN / 32);
-            if (!warp_wait_b(&s.p_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
-            tc_fence_after();
-            mma_tmem_rows(tmem + 256u, tmem, kb, IDESC_TS, true, BN / 32, BN / 16);
-            mma_commit_elect(&s.kv_empty[st]);
-            if (has_next) {
-                mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[st1][0]), 16, 1024), IDESC_SS);
+                mma_rows_dot<D>(tmem + s_col(j1), qdesc, smem_desc_sw128(smem_u32(s.k[j1 % KST][0]), 16, 1024),
+                                IDESC_SS);
+                if (!warp_wait_b(&s.v_full[j1 % VST], (uint32_t)(j1 / VST) & 1u, abort, tmo) ||
+                    !warp_wait_b(&s.dp_free, (uint32_t)j & 1u, abort, tmo)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[j1 % VST][0]), 16, 1024),
+                                IDESC_SS);
+                mma_commit_elect(&s.v_empty[j1 % VST]);
                 mma_commit_elect(&s.s_full);
             }
+            const uint64_t kb = smem_desc_sw128(smem_u32(s.k[j % KST][0]), BOX_BYTES, 1024);
+            if (!warp_wait_b(&s.p_half, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            mma_tmem_half(tmem + 256u, tmem + s_col(j), kb, IDESC_TS, j > 0, 0);
+            if (!warp_wait_b(&s.p_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            tc_fence_after();
+            mma_tmem_half(tmem + 256u, tmem + s_col(j), kb, IDESC_TS, true, 1);
+            mma_commit_elect(&s.k_empty[j % KST]);
         }
         if (ok) {
             mma_commit_elect(&s.o_full);
@@ -243,15 +299,18 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
         __syncwarp();
     } else {
-        // Elementwise: thread = query row.
-        const int row = warp * 32 + lane;
+        // Elementwise: thread = query row (TMEM lane); this warp's key columns
+        // are c0 .. c0 + 63 of each tile.
+        const int quarter = warp & 3, hf = warp >> 2;
+        const int row = quarter * 32 + lane;
         const int32_t q_local = q0 + row;
         const bool valid = q_local < q_end;
         const int64_t q_glob = (int64_t)q_local + e.q_goff;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.scale * LOG2E;
         const float lse2 = valid ? p.lse[(int64_t)head * p.N + q_glob] * LOG2E : INFINITY;
         const float dl = valid ? p.delta[(int64_t)head * p.N + q_glob] : 0.f;
+        const int c0 = hf * HALF;
         bool ok = true;
         int j = 0;
         for (int r = 0; r < e.run_count && ok; ++r) {
@@ -267,45 +326,44 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     if (diag < (int64_t)lim) lim = diag < 0 ? 0 : (int)diag;
                 }
                 if (!valid) lim = 0;
-                // All of dP(j) into registers first, so dP(j+1) can be computed
-                // into the same columns while this tile finishes.
-                uint32_t dp[4][32];
+                lim -= c0;  // in this warp's columns
+                const uint32_t sb = lane_base + s_col(j) + (uint32_t)c0;
+                // This warp's halves of dP(j) and S(j) into registers with one
+                // wait, so dP(j+1) can be computed into the dP columns while the
+                // tile finishes.
+                uint32_t dp[HALF / 32][32], sv[HALF / 32][32];
 #pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp[cc]);
+                for (int cc = 0; cc < HALF / 32; ++cc) {
+                    tmem_ld32(lane_base + 128u + (uint32_t)(c0 + cc * 32), dp[cc]);
+                    tmem_ld32(sb + (uint32_t)(cc * 32), sv[cc]);
+                }
                 tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) fence_regs32(dp[cc]);
+                for (int cc = 0; cc < HALF / 32; ++cc) {
+                    fence_regs32(dp[cc]);
+                    fence_regs32(sv[cc]);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.dp_free);
 #pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t sv[32];
-                    tmem_ld32(lane_base + (uint32_t)(cc * 32), sv);
-                    tmem_wait_ld();
-                    fence_regs32(sv);
+                for (int cc = 0; cc < HALF / 32; ++cc) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int t = 0; t < 32; t += 2) {
                         const int c = cc * 32 + t;
-                        const float p0 = c < lim ? ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, -lse2)) : 0.f;
+                        const float p0 = c < lim ? ex2_approx(fmaf(__uint_as_float(sv[cc][t]), sl2, -lse2)) : 0.f;
                         const float p1 =
-                            c + 1 < lim ? ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, -lse2)) : 0.f;
+                            c + 1 < lim ? ex2_approx(fmaf(__uint_as_float(sv[cc][t + 1]), sl2, -lse2)) : 0.f;
                         pk[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[cc][t]) - dl),
                                                 p1 * (__uint_as_float(dp[cc][t + 1]) - dl));
                     }
-                    tmem_st16_b(lane_base + (uint32_t)(cc * 16), pk);
-                    if (cc == 1) {
-                        tmem_wait_st();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&s.p_half);
-                    }
+                    tmem_st16_b(sb + (uint32_t)(cc * 16), pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(cc == 0 ? &s.p_half : &s.p_full);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.p_full);
             }
         }
         if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
@@ -313,8 +371,10 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             tc_fence_after();
             const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
             const int64_t orow = (int64_t)e.out_lo + (q_local - e.q_lo);
+            // This warp writes features hf * D/2 .. of its row.
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
+            for (int ch = 0; ch < D / 64; ++ch) {
+                const int cc = hf * (D / 64) + ch;
                 uint32_t o[32];
                 tmem_ld32(lane_base + 256u + (uint32_t)(cc * 32), o);
                 tmem_wait_ld();
@@ -383,9 +443,10 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             mbar_init(&s.qd_full[i], 1);
             mbar_init(&s.qd_empty[i], 1);
         }
-        mbar_init(&s.s_full, 1);
-        mbar_init(&s.p_half, 4);
-        mbar_init(&s.p_full, 4);
+        mbar_init(&s.st_full, 1);
+        mbar_init(&s.dp_full, 1);
+        mbar_init(&s.pt_full, EW_WARPS);
+        mbar_init(&s.ds_full, EW_WARPS);
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
         s.abort = 0;
@@ -453,34 +514,56 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         bool ok = warp_wait_b(&s.bar_kv, 0, abort, tmo);
         const uint64_t kdesc = smem_desc_sw128(smem_u32(s.k[0]), 16, 1024);
         const uint64_t vdesc = smem_desc_sw128(smem_u32(s.v[0]), 16, 1024);
-        auto grads = [&](int it) -> bool {
-            // dV += P^T dO, dK += dS^T Q for query tile `it` (P^T over S^T,
-            // dS^T over dP^T in tensor memory), in two halves of 64 queries:
-            // the first runs while the elementwise warps finish the second.
-            const int sp = it % STAGES;
+        // Per query tile i: S^T(i) = K Q^T and dP^T(i) = V dO^T; the elementwise
+        // warps form P^T over S^T (phase A, pt_full), then dS^T over dP^T
+        // (phase B, ds_full).  dV(i) += P^T dO goes in after phase A, then
+        // S^T(i+1), which overwrites the P^T columns dV(i) read before it, so
+        // phase A of tile i+1 can start while phase B of tile i, dK(i) +=
+        // dS^T Q and dP^T(i+1) are still running.
+        auto ss_tiles = [&](int it, bool which_dp) {
+            const int st = it % STAGES;
+            if (!which_dp)
+                mma_rows_dot<D>(tmem, kdesc, smem_desc_sw128(smem_u32(s.q[st][0]), 16, 1024), IDESC_SS);
+            else
+                mma_rows_dot<D>(tmem + 128u, vdesc, smem_desc_sw128(smem_u32(s.dout[st][0]), 16, 1024), IDESC_SS);
+        };
+        if (ok && ntiles > 0) {
+            ok = warp_wait_b(&s.qd_full[0], 0, abort, tmo);
+            if (ok) {
+                tc_fence_after();
+                ss_tiles(0, false);
+                mma_commit_elect(&s.st_full);
+                ss_tiles(0, true);
+                mma_commit_elect(&s.dp_full);
+            }
+        }
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int sp = i % STAGES, i1 = i + 1;
             const uint64_t ob = smem_desc_sw128(smem_u32(s.dout[sp][0]), BOX_BYTES, 1024);
             const uint64_t qb = smem_desc_sw128(smem_u32(s.q[sp][0]), BOX_BYTES, 1024);
-            if (!warp_wait_b(&s.p_half, (uint32_t)it & 1u, abort, tmo)) return false;
+            if (!warp_wait_b(&s.pt_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
-            mma_tmem_rows(tmem + COL_DV, tmem, ob, IDESC_TS, it > 0, 0, BN / 32);
-            mma_tmem_rows(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, it > 0, 0, BN / 32);
-            if (!warp_wait_b(&s.p_full, (uint32_t)it & 1u, abort, tmo)) return false;
+            mma_tmem_half(tmem + COL_DV, tmem, ob, IDESC_TS, i > 0, 0);
+            mma_tmem_half(tmem + COL_DV, tmem, ob, IDESC_TS, true, 1);
+            if (i1 < ntiles) {
+                if (!warp_wait_b(&s.qd_full[i1 % STAGES], (uint32_t)(i1 / STAGES) & 1u, abort, tmo)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                ss_tiles(i1, false);
+                mma_commit_elect(&s.st_full);
+            }
+            if (!warp_wait_b(&s.ds_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
-            mma_tmem_rows(tmem + COL_DV, tmem, ob, IDESC_TS, true, BN / 32, BN / 16);
-            mma_tmem_rows(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, true, BN / 32, BN / 16);
+            mma_tmem_half(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, i > 0, 0);
+            mma_tmem_half(tmem + COL_DK, tmem + 128u, qb, IDESC_TS, true, 1);
             mma_commit_elect(&s.qd_empty[sp]);
-            return true;
-        };
-        for (int i = 0; i < ntiles && ok; ++i) {
-            const int st = i % STAGES;
-            if (!warp_wait_b(&s.qd_full[st], (uint32_t)(i / STAGES) & 1u, abort, tmo)) { ok = false; break; }
-            tc_fence_after();
-            if (i > 0 && !grads(i - 1)) { ok = false; break; }
-            mma_rows_dot<D>(tmem, kdesc, smem_desc_sw128(smem_u32(s.q[st][0]), 16, 1024), IDESC_SS);
-            mma_rows_dot<D>(tmem + 128u, vdesc, smem_desc_sw128(smem_u32(s.dout[st][0]), 16, 1024), IDESC_SS);
-            mma_commit_elect(&s.s_full);
+            if (i1 < ntiles) {
+                ss_tiles(i1, true);
+                mma_commit_elect(&s.dp_full);
+            }
         }
-        if (ok && ntiles > 0) ok = grads(ntiles - 1);
         if (ok) {
             mma_commit_elect(&s.o_full);
         } else if (lane == 0) {
@@ -491,13 +574,16 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         mbar_wait(&s.drain, 0, (volatile int *)&zero, tmo);
         __syncwarp();
     } else {
-        // Elementwise: thread = key row; columns are the tile's query rows.
-        const int row = warp * 32 + lane;
+        // Elementwise: thread = key row (TMEM lane); columns are the tile's
+        // query rows, this warp's c0 .. c0 + 63.
+        const int quarter = warp & 3, hf = warp >> 2;
+        const int row = quarter * 32 + lane;
         const int32_t k_local = k0 + row;
         const bool valid = k_local < k_end;
         const int64_t k_glob = (int64_t)k_local + e.q_goff;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = p.scale * LOG2E;
+        const int c0 = hf * HALF;
         bool ok = true;
         int i = 0;
         for (int r = 0; r < e.run_count && ok; ++r) {
@@ -509,51 +595,76 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 // qd_full makes the TMA warp's lse / D stores of this stage
                 // visible here (it completed before S^T was issued).
                 if (!warp_wait_b(&s.qd_full[st], (uint32_t)(i / STAGES) & 1u, abort, tmo)) { ok = false; break; }
-                if (!warp_wait_b(&s.s_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
+                if (!warp_wait_b(&s.st_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
                 // Query column c is kept iff c >= first (causal: at or after
                 // this key) and the row is inside the run (lse2 = +inf
-                // outside, so its P is 0).
+                // outside, so its P is 0); first is in this warp's columns.
                 int first = 0;
                 if (causal) {
                     const int64_t f = k_glob - ((int64_t)qs + run.k_goff);
                     first = f <= 0 ? 0 : (f > BN ? BN : (int)f);
                 }
                 if (!valid) first = BN;
-#pragma unroll
-                for (int cc = 0; cc < BN / 32; ++cc) {
-                    uint32_t sv[32], dp[32];
-                    tmem_ld32(lane_base + (uint32_t)(cc * 32), sv);
-                    tmem_ld32(lane_base + 128u + (uint32_t)(cc * 32), dp);
+                first -= c0;
+                const float *lse2 = &s.lse2[st][c0];
+                const float *dl = &s.dl[st][c0];
+                static_assert(HALF == 64, "two 32-column chunks per warp");
+                // Phase A: P^T of this warp's 64 columns, kept in fp32 for dS.
+                float pv[2][32];
+                {
+                    uint32_t sv[2][32];
+                    tmem_ld32(lane_base + (uint32_t)c0, sv[0]);
+                    tmem_ld32(lane_base + (uint32_t)(c0 + 32), sv[1]);
                     tmem_wait_ld();
-                    fence_regs32(sv);
-                    fence_regs32(dp);
-                    uint32_t pp[16], pd[16];
+                    fence_regs32(sv[0]);
+                    fence_regs32(sv[1]);
 #pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const int c = cc * 32 + t;
-                        const float p0 =
-                            c >= first ? ex2_approx(fmaf(__uint_as_float(sv[t]), sl2, -s.lse2[st][c])) : 0.f;
-                        const float p1 = c + 1 >= first
-                                             ? ex2_approx(fmaf(__uint_as_float(sv[t + 1]), sl2, -s.lse2[st][c + 1]))
-                                             : 0.f;
-                        pp[t / 2] = pack_bf16x2(p0, p1);
-                        pd[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[t]) - s.dl[st][c]),
-                                                p1 * (__uint_as_float(dp[t + 1]) - s.dl[st][c + 1]));
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t pp[16];
+#pragma unroll
+                        for (int t = 0; t < 32; t += 4) {
+                            const float4 l4 = lds_f4(lse2 + cc * 32 + t);
+                            const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int c = cc * 32 + t + u;
+                                pv[cc][t + u] =
+                                    c >= first ? ex2_approx(fmaf(__uint_as_float(sv[cc][t + u]), sl2, -la[u])) : 0.f;
+                            }
+                            pp[t / 2] = pack_bf16x2(pv[cc][t], pv[cc][t + 1]);
+                            pp[t / 2 + 1] = pack_bf16x2(pv[cc][t + 2], pv[cc][t + 3]);
+                        }
+                        tmem_st16_b(lane_base + (uint32_t)(c0 + cc * 16), pp);
                     }
-                    tmem_st16_b(lane_base + (uint32_t)(cc * 16), pp);
-                    tmem_st16_b(lane_base + 128u + (uint32_t)(cc * 16), pd);
-                    if (cc == 1) {
-                        tmem_wait_st();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&s.p_half);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.pt_full);
+                }
+                // Phase B: dS^T = P^T (dP^T - D) over dP^T.
+                if (!warp_wait_b(&s.dp_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t dp[32], pd[16];
+                    tmem_ld32(lane_base + 128u + (uint32_t)(c0 + cc * 32), dp);
+                    tmem_wait_ld();
+                    fence_regs32(dp);
+#pragma unroll
+                    for (int t = 0; t < 32; t += 4) {
+                        const float4 d4 = lds_f4(dl + cc * 32 + t);
+                        pd[t / 2] = pack_bf16x2(pv[cc][t] * (__uint_as_float(dp[t]) - d4.x),
+                                                pv[cc][t + 1] * (__uint_as_float(dp[t + 1]) - d4.y));
+                        pd[t / 2 + 1] = pack_bf16x2(pv[cc][t + 2] * (__uint_as_float(dp[t + 2]) - d4.z),
+                                                    pv[cc][t + 3] * (__uint_as_float(dp[t + 3]) - d4.w));
                     }
+                    tmem_st16_b(lane_base + 128u + (uint32_t)(c0 + cc * 16), pd);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s.p_full);
+                if (lane == 0) mbar_arrive(&s.ds_full);
             }
         }
         if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
@@ -565,8 +676,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             const int64_t orow = (int64_t)e.out_lo + (k_local - e.q_lo);
             const int hkv = head / p.kv_group;
             const int64_t slot = (int64_t)e.slot * p.kv_group + head % p.kv_group;
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
+            // Warps of columns 0-63 write dK, those of 64-127 dV.
+            {
+                const int which = hf;
                 const uint32_t col = which == 0 ? COL_DK : COL_DV;
                 const float mul = which == 0 ? p.scale : 1.f;
 #pragma unroll
