@@ -98,6 +98,13 @@ typedef struct {
     int B;     /* independent sequences per call (0 or 1: one): tensors are
                   [B, N, heads, d] and lse [B, H, N]; the sequences run one
                   after another through the plan on the call's stream. */
+    int shard_rank;  /* task sharding over shard_count processes (0 or 1:
+                        none): the plan's entries (leaf task, query block) go
+                        to ranks by longest-first assignment of their allowed
+                        pair counts, the same on every rank, and this plan
+                        computes the entries of shard_rank with
+                        cqsa_forward_partial (see there). */
+    int shard_count;
 } cqsa_plan_desc_t;
 
 /* What a plan decided (for logging, tests and the benchmark). */
@@ -122,6 +129,10 @@ typedef struct {
     int merge;                          /* cqsa_merge_t of device-mode forwards */
     int H_kv;                           /* key/value heads */
     int B;                              /* sequences per call */
+    int shard_rank, shard_count;        /* task sharding (count 1: none) */
+    int64_t shard_entries;              /* entries this rank computes */
+    double shard_pairs;                 /* allowed (query, key) pairs of those entries, per head */
+    double total_pairs;                 /* allowed pairs of all entries, per head */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */
@@ -130,6 +141,7 @@ typedef struct {
     int64_t q_block;    /* global query block */
     int64_t slot;       /* partial index of this entry among the query block's entries */
     int64_t num_runs;   /* runs of consecutive allowed key blocks */
+    int64_t shard;      /* rank that computes this entry in a sharded plan (0 otherwise) */
 } cqsa_entry_t;
 
 /*
@@ -195,6 +207,49 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,
 cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
                             const void *out, const float *lse, const void *dout, void *dq, void *dk,
                             void *dv, int host_or_device, void *stream);
+
+/*
+ * Task sharding across processes (one GPU each).  The tasks of the CQS
+ * Divide are independent ([A]; [B] "Implementation": each task's partial
+ * result is aggregated afterwards), so a plan with shard_count = G splits
+ * one problem's (task, query block) entries over G ranks and the ranks
+ * exchange their log-sum-exp partials once:
+ *   1. cqsa_forward_partial on every rank: o_r, lse_r of its entries.
+ *   2. lse_max = max over ranks of lse_r          (all-reduce MAX, caller)
+ *   3. cqsa_partial_rescale: w_r = exp(lse_r - lse_max), o_r *= w_r.
+ *   4. o = sum over ranks of o_r, w = sum of w_r  (all-reduce SUM, caller)
+ *   5. cqsa_partial_finish: out = o / w, lse = lse_max + ln w.
+ * The collectives are the caller's (the Python binding uses NCCL through
+ * torch.distributed); all arithmetic runs in this library's kernels.  Any
+ * plan may run steps 1, 3 and 5 (with one rank they reproduce
+ * cqsa_forward); cqsa_forward and cqsa_backward reject a plan with
+ * shard_count > 1.  Device mode only; B sequences are handled as in
+ * cqsa_forward (each buffer gains a leading B).
+ */
+
+/* cqsa_forward_partial -- this rank's part of the forward.  q, k, v as in
+ * cqsa_forward (device pointers).  o_part fp32 [N, H, d] gets, for every row,
+ * the attention over this rank's allowed keys normalised by its own
+ * denominator (0 where it has none) and lse_part fp32 [H, N] the natural-log
+ * denominator (-inf where it has none).  Caller-owned device buffers; the
+ * first call allocates a small arena (work list, error word).  Asynchronous
+ * on stream.  Errors: INVALID_ARG, CUDA, NO_DEVICE, UNSUPPORTED. */
+cqsa_status_t cqsa_forward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
+                                   float *o_part, float *lse_part, void *stream);
+
+/* cqsa_partial_rescale -- w[h][n] = exp(lse_part[h][n] - lse_max[h][n]) (0
+ * when lse_part is -inf) and o_part[n][h][:] *= w[h][n], in place.  All fp32
+ * device buffers laid out as in cqsa_forward_partial; w may not alias the
+ * others.  Asynchronous on stream.  Errors: INVALID_ARG, CUDA. */
+cqsa_status_t cqsa_partial_rescale(cqsa_plan_t *plan, float *o_part, const float *lse_part,
+                                   const float *lse_max, float *w, void *stream);
+
+/* cqsa_partial_finish -- out[n][h][:] = o_sum[n][h][:] / w_sum[h][n] in the
+ * plan dtype and lse[h][n] = lse_max[h][n] + ln w_sum[h][n] (0 and -inf
+ * where w_sum is 0).  Device buffers; out and lse as cqsa_forward writes
+ * them.  Asynchronous on stream.  Errors: INVALID_ARG, CUDA. */
+cqsa_status_t cqsa_partial_finish(cqsa_plan_t *plan, const float *o_sum, const float *w_sum,
+                                  const float *lse_max, void *out, float *lse, void *stream);
 
 /* cqsa_plan_sync -- wait for the plan's work on `stream` and report any
  * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync. */

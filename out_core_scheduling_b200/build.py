@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcqsa.so")
-SOURCES = ["planner.cpp", "api.cu", "attn_tc.cu", "attn_simt.cu", "attn_bwd.cu", "attn_bwd_tc.cu", "merge.cu", "noalloc.cu"]
+SOURCES = ["planner.cpp", "api.cu", "attn_tc.cu", "attn_simt.cu", "attn_bwd.cu", "attn_bwd_tc.cu", "merge.cu", "partial.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -37,7 +37,7 @@ EXPORTS = (
     "cqsa_plan", "cqsa_plan_ex", "cqsa_forward", "cqsa_backward", "cqsa_plan_sync", "cqsa_plan_info",
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
-    "cqsa_last_error",
+    "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
 )
 
 
@@ -52,7 +52,7 @@ class PlanDesc(ctypes.Structure):
                 ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
                 ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int), ("H_kv", ctypes.c_int),
-                ("B", ctypes.c_int)]
+                ("B", ctypes.c_int), ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -66,7 +66,9 @@ class PlanInfo(ctypes.Structure):
                 ("head_group", ctypes.c_int), ("device_arena_bytes", ctypes.c_size_t),
                 ("host_arena_bytes", ctypes.c_size_t), ("h2d_bytes", ctypes.c_size_t),
                 ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double),
-                ("merge", ctypes.c_int), ("H_kv", ctypes.c_int), ("B", ctypes.c_int)]
+                ("merge", ctypes.c_int), ("H_kv", ctypes.c_int), ("B", ctypes.c_int),
+                ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int), ("shard_entries", ctypes.c_int64),
+                ("shard_pairs", ctypes.c_double), ("total_pairs", ctypes.c_double)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -88,7 +90,7 @@ class KernelStats(ctypes.Structure):
 
 class Entry(ctypes.Structure):
     _fields_ = [("task", ctypes.c_int64), ("q_block", ctypes.c_int64),
-                ("slot", ctypes.c_int64), ("num_runs", ctypes.c_int64)]
+                ("slot", ctypes.c_int64), ("num_runs", ctypes.c_int64), ("shard", ctypes.c_int64)]
 
 
 _lib = None
@@ -122,6 +124,9 @@ def load_library():
         "cqsa_plan_profile": (st, [P, ctypes.c_int]),
         "cqsa_plan_kernel_stats": (st, [P, ctypes.POINTER(KernelStats), ctypes.c_int]),
         "cqsa_forward_noalloc": (st, [P, P, P, P, P, P, P]),
+        "cqsa_forward_partial": (st, [P, P, P, P, P, P, P]),
+        "cqsa_partial_rescale": (st, [P, P, P, P, P, P]),
+        "cqsa_partial_finish": (st, [P, P, P, P, P, P, P]),
         "cqsa_plan_destroy": (None, [P]),
         "cqsa_last_error": (ctypes.c_char_p, []),
     }
@@ -175,7 +180,7 @@ class Plan:
         runs = (ctypes.c_int64 * (2 * max(1, e.num_runs)))()
         _check(lib.cqsa_plan_entry(self.handle, i, ctypes.byref(e), runs, e.num_runs))
         pairs = [(runs[2 * r], runs[2 * r + 1]) for r in range(e.num_runs)]
-        return {"task": e.task, "q_block": e.q_block, "slot": e.slot, "runs": pairs}
+        return {"task": e.task, "q_block": e.q_block, "slot": e.slot, "runs": pairs, "shard": e.shard}
 
     def sync(self, stream=None):
         _check(load_library().cqsa_plan_sync(self.handle, ctypes.c_void_p(_stream_ptr(stream))))
@@ -213,7 +218,8 @@ def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = Fa
 
 
 def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
-                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0, B: int = 1) -> Plan:
+                 mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0, B: int = 1,
+                 shard_rank: int = 0, shard_count: int = 1) -> Plan:
     desc = PlanDesc()
     desc.N, desc.H, desc.d = N, H, d
     desc.levels = len(ls)
@@ -225,6 +231,7 @@ def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = 
     desc.merge = merge
     desc.H_kv = H_kv
     desc.B = B
+    desc.shard_rank, desc.shard_count = shard_rank, shard_count
     h = ctypes.c_void_p()
     _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
     return Plan(h.value)
@@ -291,6 +298,49 @@ def cqsa_forward_noalloc(plan: Plan, q, k, v, out, lse, stream=None):
     _check(load_library().cqsa_forward_noalloc(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                                out.data_ptr(), lse.data_ptr(),
                                                ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def _check_partials(plan: Plan, named_o, named_l):
+    """fp32 device tensors: o-like [B, N, H, d], lse-like [B, H, N] (B = 1:
+    the leading dimension may be left out)."""
+    import torch
+    info = plan.info()
+    N, H, d, B = info["N"], info["H"], info["d"], info["B"]
+    lead = (B,) if B > 1 else ()
+    for names, want in ((named_o, (N, H, d)), (named_l, (H, N))):
+        for name, t in names:
+            if not isinstance(t, torch.Tensor) or not t.is_contiguous() or t.dtype != torch.float32:
+                raise ValueError(f"{name} must be a contiguous float32 torch tensor")
+            if tuple(t.shape) != lead + want and not (B == 1 and tuple(t.shape) == (1,) + want):
+                raise ValueError(f"{name} must be {lead + want}")
+
+
+def cqsa_forward_partial(plan: Plan, q, k, v, o_part, lse_part, stream=None):
+    """This rank's part of a sharded forward: o_part fp32 [N, H, d] (the
+    attention over this rank's allowed keys, normalised by its own
+    denominator) and lse_part fp32 [H, N] (-inf where it has no key)."""
+    _check_shapes(plan, (("q", q),), (("k", k), ("v", v)), lse_part)
+    _check_partials(plan, (("o_part", o_part),), (("lse_part", lse_part),))
+    _check(load_library().cqsa_forward_partial(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               o_part.data_ptr(), lse_part.data_ptr(),
+                                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_partial_rescale(plan: Plan, o_part, lse_part, lse_max, w, stream=None):
+    """w = exp(lse_part - lse_max) (0 where lse_part is -inf), o_part *= w."""
+    _check_partials(plan, (("o_part", o_part),), (("lse_part", lse_part), ("lse_max", lse_max), ("w", w)))
+    _check(load_library().cqsa_partial_rescale(plan.handle, o_part.data_ptr(), lse_part.data_ptr(),
+                                               lse_max.data_ptr(), w.data_ptr(),
+                                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_partial_finish(plan: Plan, o_sum, w_sum, lse_max, out, lse, stream=None):
+    """out = o_sum / w_sum in the plan dtype, lse = lse_max + ln w_sum."""
+    _check_partials(plan, (("o_sum", o_sum),), (("w_sum", w_sum), ("lse_max", lse_max), ("lse", lse)))
+    _check_shapes(plan, (("out", out),), (), lse)
+    _check(load_library().cqsa_partial_finish(plan.handle, o_sum.data_ptr(), w_sum.data_ptr(),
+                                              lse_max.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                              ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def cqsa_difference_set(l: int):

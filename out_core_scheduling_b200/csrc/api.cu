@@ -162,6 +162,11 @@ struct cqsa_plan {
     int32_t *bwd_q_nslots = nullptr, *bwd_kv_nslots = nullptr;
     DevWl bwd_qwl, bwd_kvwl;
 
+    // Sharded forward (cqsa_forward_partial): this rank's work list.
+    char *part_arena = nullptr;
+    int *part_err = nullptr;
+    DevWl part_wl;
+
     // Streamed path.
     char *host_arena = nullptr;
     size_t host_bytes = 0;
@@ -432,6 +437,62 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H, out, lse,
                           stream));
     tm.stop();
+    return CQSA_OK;
+}
+
+cqsa_status_t setup_partial(cqsa_plan_t *P) {
+    if (P->part_arena) return CQSA_OK;
+    const Planner &pl = P->pl;
+    WorkList wl = pl.partial_worklist(unit_rows_for(P->elem), key_tile_for(P->elem), pl.spec.H);
+    ArenaLayout a;
+    const size_t o_err = a.take(256);
+    const size_t o_wl = a.take(wl_region(wl));
+    char *arena = nullptr;
+    CK(cudaMalloc(&arena, a.total));
+    P->part_arena = arena;
+    CK(cudaMemset(arena, 0, a.total));
+    P->part_err = reinterpret_cast<int *>(arena + o_err);
+    std::vector<char> buf = pack_wl(wl);
+    if (!buf.empty()) CK(cudaMemcpy(arena + o_wl, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+    P->part_wl = place_wl(arena + o_wl, wl);
+    return CQSA_OK;
+}
+
+// This rank's entries of a sharded plan: every query block it has an entry
+// for is one work-list entry flagged SEG_FIRST only, so the epilogue leaves
+// the normalised partial and its lse in o_part / lse_part at the global row.
+cqsa_status_t forward_partial_device(cqsa_plan_t *P, const void *q, const void *k, const void *v, float *o_part,
+                                     float *lse_part, cudaStream_t stream) {
+    cqsa_status_t st = setup_partial(P);
+    if (st != CQSA_OK) return st;
+    const Planner &pl = P->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    CK(launch_partial_init(o_part, N * H * d, lse_part, (int64_t)H * N, stream));
+    if (P->part_wl.num_units == 0) return CQSA_OK;
+    AttnParams ap = base_params(P, P->part_err);
+    ap.entries = P->part_wl.entries;
+    ap.runs = P->part_wl.runs;
+    ap.units = P->part_wl.units;
+    ap.part_rows = N;
+    ap.H = H;
+    ap.epi = EPI_MERGE;
+    ap.acc_o = o_part;
+    ap.acc_lse = lse_part;
+    ap.acc_rows = N;
+    if (P->dtype == CQSA_BF16) {
+        CUtensorMap mq, mk, mv;
+        if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mk, k, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
+        if ((st = make_map(&mv, v, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
+        LaunchTimer tm(P, stream, 0);
+        CK(launch_attn_tc(d, mq, mk, mv, ap, P->part_wl.num_units, stream));
+        tm.stop();
+    } else {
+        LaunchTimer tm(P, stream, 0);
+        CK(launch_attn_simt(d, P->elem, q, k, v, ap, P->part_wl.num_units, stream));
+        tm.stop();
+    }
     return CQSA_OK;
 }
 
@@ -731,6 +792,8 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
     s.budget = desc->mem_budget_bytes;
     s.Hkv = desc->H_kv;
     s.B = desc->B > 0 ? desc->B : 1;
+    s.shard_count = desc->shard_count > 0 ? desc->shard_count : 1;
+    s.shard_rank = desc->shard_rank;
     if (desc->merge != CQSA_MERGE_SLOTS && desc->merge != CQSA_MERGE_FUSED)
         return fail(CQSA_ERR_INVALID_ARG, "merge must be CQSA_MERGE_SLOTS or CQSA_MERGE_FUSED");
     s.fused = desc->merge == CQSA_MERGE_FUSED;
@@ -787,6 +850,9 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (host_or_device != CQSA_DEVICE && host_or_device != CQSA_HOST)
         return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be CQSA_DEVICE or CQSA_HOST");
+    if (plan->pl.spec.shard_count > 1)
+        return fail(CQSA_ERR_UNSUPPORTED, "a sharded plan runs cqsa_forward_partial (shard_count = %d)",
+                    plan->pl.spec.shard_count);
     cqsa_status_t st = check_device(plan);
     if (st != CQSA_OK) return st;
     const bool host = host_or_device == CQSA_HOST;
@@ -818,6 +884,8 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
     if (host_or_device == CQSA_HOST)
         return fail(CQSA_ERR_UNSUPPORTED, "the backward runs in device mode only");
     if (host_or_device != CQSA_DEVICE) return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be 0 or 1");
+    if (plan->pl.spec.shard_count > 1)
+        return fail(CQSA_ERR_UNSUPPORTED, "the backward of a sharded plan is not supported");
     cqsa_status_t st = check_device(plan);
     if (st != CQSA_OK) return st;
     const void *ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
@@ -837,11 +905,73 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
     return CQSA_OK;
 }
 
+cqsa_status_t cqsa_forward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
+                                   float *o_part, float *lse_part, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[5] = {q, k, v, o_part, lse_part};
+    const char *names[5] = {"q", "k", "v", "o_part", "lse_part"};
+    for (int i = 0; i < 5; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    const Planner &pl = plan->pl;
+    const size_t e = (size_t)plan->elem, N = (size_t)pl.spec.N, d = (size_t)pl.spec.d;
+    const size_t qs = N * pl.spec.H * d * e, kvs = N * pl.spec.Hkv * d * e, os = N * pl.spec.H * d,
+                 ls = N * pl.spec.H;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int b = 0; b < pl.spec.B; ++b) {
+        st = forward_partial_device(plan, static_cast<const char *>(q) + b * qs,
+                                    static_cast<const char *>(k) + b * kvs, static_cast<const char *>(v) + b * kvs,
+                                    o_part + b * os, lse_part + b * ls, s);
+        if (st != CQSA_OK) return st;
+    }
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_partial_rescale(cqsa_plan_t *plan, float *o_part, const float *lse_part, const float *lse_max,
+                                   float *w, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[4] = {o_part, lse_part, lse_max, w};
+    const char *names[4] = {"o_part", "lse_part", "lse_max", "w"};
+    for (int i = 0; i < 4; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    const Planner &pl = plan->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    const size_t os = (size_t)N * H * d, ls = (size_t)N * H;  // per sequence: o [N][H][d], lse-like [H][N]
+    for (int b = 0; b < pl.spec.B; ++b)
+        CK(launch_partial_rescale(d, o_part + b * os, lse_part + b * ls, lse_max + b * ls, w + b * ls, N, H,
+                                  static_cast<cudaStream_t>(stream)));
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_partial_finish(cqsa_plan_t *plan, const float *o_sum, const float *w_sum, const float *lse_max,
+                                  void *out, float *lse, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[5] = {o_sum, w_sum, lse_max, out, lse};
+    const char *names[5] = {"o_sum", "w_sum", "lse_max", "out", "lse"};
+    for (int i = 0; i < 5; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    const Planner &pl = plan->pl;
+    const int64_t N = pl.spec.N;
+    const int H = pl.spec.H, d = pl.spec.d;
+    const size_t os = (size_t)N * H * d, ls = (size_t)N * H;
+    for (int b = 0; b < pl.spec.B; ++b)
+        CK(launch_partial_finish(d, plan->elem, o_sum + b * os, w_sum + b * ls, lse_max + b * ls,
+                                 static_cast<char *>(out) + b * os * plan->elem, lse + b * ls, N, H,
+                                 static_cast<cudaStream_t>(stream)));
+    return CQSA_OK;
+}
+
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
     CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-    int *words[3] = {plan->dev_err, plan->h_err, plan->bwd_err};
+    int *words[4] = {plan->dev_err, plan->h_err, plan->bwd_err, plan->part_err};
     int bad = 0;
     for (int *w : words) {
         if (!w) continue;
@@ -925,6 +1055,11 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->merge = pl.spec.fused ? CQSA_MERGE_FUSED : CQSA_MERGE_SLOTS;
     info->H_kv = pl.spec.Hkv;
     info->B = pl.spec.B;
+    info->shard_rank = pl.spec.shard_rank;
+    info->shard_count = pl.spec.shard_count;
+    info->shard_entries = pl.shard_entries;
+    info->shard_pairs = pl.shard_pairs;
+    info->total_pairs = pl.total_pairs;
     return CQSA_OK;
 }
 
@@ -954,6 +1089,7 @@ cqsa_status_t cqsa_plan_entry(const cqsa_plan_t *plan, int64_t i, cqsa_entry_t *
     entry->q_block = e.qb;
     entry->slot = e.slot;
     entry->num_runs = (int64_t)e.runs.size();
+    entry->shard = pl.entry_rank.empty() ? 0 : pl.entry_rank[i];
     if (runs) {
         if (max_runs < (int64_t)e.runs.size()) return fail(CQSA_ERR_INVALID_ARG, "runs buffer too small");
         for (size_t r = 0; r < e.runs.size(); ++r) {
@@ -979,7 +1115,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
         cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);
-        if (plan->dev_arena || plan->bwd_arena) cudaDeviceSynchronize();
+        if (plan->dev_arena || plan->bwd_arena || plan->part_arena) cudaDeviceSynchronize();
         for (int s = 0; s < 2; ++s) {
             if (plan->ev_in_ready[s]) cudaEventDestroy(plan->ev_in_ready[s]);
             if (plan->ev_in_free[s]) cudaEventDestroy(plan->ev_in_free[s]);
@@ -999,6 +1135,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
         if (plan->dev_arena) cudaFree(plan->dev_arena);
         if (plan->host_arena) cudaFree(plan->host_arena);
         if (plan->bwd_arena) cudaFree(plan->bwd_arena);
+        if (plan->part_arena) cudaFree(plan->part_arena);
         cudaGetLastError();
     }
     delete plan;

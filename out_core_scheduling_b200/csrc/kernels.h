@@ -114,4 +114,13 @@ cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const
                                const int32_t *nslots, int64_t block, int64_t N, int H, void *out,
                                float *lse, cudaStream_t stream);
 
+// Cross-rank exchange of a sharded forward (partial.cu).  o [N][H][d] fp32,
+// lse-like arrays [H][N] fp32.
+cudaError_t launch_partial_init(float *o, int64_t n, float *lse, int64_t nl, cudaStream_t stream);
+cudaError_t launch_partial_rescale(int d, float *o, const float *lse_part, const float *lse_max, float *w,
+                                   int64_t N, int H, cudaStream_t stream);
+cudaError_t launch_partial_finish(int d, int elem_bytes, const float *o_sum, const float *w_sum,
+                                  const float *lse_max, void *out, float *lse, int64_t N, int H,
+                                  cudaStream_t stream);
+
 }  // namespace cqsa

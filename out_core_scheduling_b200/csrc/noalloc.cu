@@ -186,6 +186,7 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     const int rows = unit_rows_for(elem), bn = key_tile_for(elem);
     if (pl.max_slots > 32) return err(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
     if (pl.spec.B != 1) return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes one sequence (B = 1)");
+    if (pl.spec.shard_count != 1) return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes no sharded plan");
     if (pl.spec.Hkv != pl.spec.H)
         return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes as many key/value heads as query heads");
 

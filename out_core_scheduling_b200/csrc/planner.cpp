@@ -76,6 +76,8 @@ std::string Planner::build(const PlanSpec &s, int *code) {
         return "the query heads must be a multiple of the key/value heads";
     if (spec.Hkv == 0) spec.Hkv = s.H;
     if (s.B < 1) return "the batch B must be at least 1";
+    if (s.shard_count < 1 || s.shard_rank < 0 || s.shard_rank >= s.shard_count)
+        return "the shard rank must be in 0..shard_count-1 (shard_count >= 1)";
     levels.clear();
     num_blocks = 1;
     for (int i = 0; i < s.levels; ++i) {
@@ -186,6 +188,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     entry_begin_of_leaf_.push_back((int64_t)entries.size());
     max_slots = 0;
     for (int32_t v : slots_per_block) max_slots = std::max<int64_t>(max_slots, v);
+    assign_shards();
     size_plan();
     *code = 0;
     return "";
@@ -225,43 +228,98 @@ static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int ca
     wl->units.swap(u);
 }
 
+double Planner::entry_pairs(const Entry &e) const {
+    const double qr = (double)block_rows(e.qb);
+    double n = 0;
+    for (const KeyRun &r : e.runs)
+        for (int64_t b = r.b0; b <= r.b1; ++b)
+            n += (spec.causal && b == e.qb) ? qr * (qr + 1) / 2 : qr * (double)block_rows(b);
+    return n;
+}
+
+void Planner::assign_shards() {
+    const int G = std::max(1, spec.shard_count);
+    entry_rank.assign(entries.size(), 0);
+    std::vector<double> cost(entries.size());
+    total_pairs = 0;
+    for (size_t i = 0; i < entries.size(); ++i) {
+        cost[i] = entry_pairs(entries[i]);
+        total_pairs += cost[i];
+    }
+    if (G > 1) {
+        std::vector<size_t> order(entries.size());
+        for (size_t i = 0; i < order.size(); ++i) order[i] = i;
+        std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return cost[a] > cost[b]; });
+        std::vector<double> load(G, 0.0);
+        for (size_t i : order) {
+            int r = 0;
+            for (int x = 1; x < G; ++x)
+                if (load[x] < load[r]) r = x;
+            entry_rank[i] = r;
+            load[r] += cost[i];
+        }
+    }
+    shard_pairs = 0;
+    shard_entries = 0;
+    for (size_t i = 0; i < entries.size(); ++i)
+        if (entry_rank[i] == spec.shard_rank) {
+            shard_pairs += cost[i];
+            ++shard_entries;
+        }
+}
+
+WorkList Planner::union_worklist(const std::vector<char> &use, int32_t flags, int rows_per_unit, int bn,
+                                 int heads) const {
+    // The tasks of a query block own disjoint sets of its allowed key
+    // blocks; their union, as maximal runs, is one entry.
+    WorkList wl;
+    std::vector<int64_t> group;
+    std::vector<std::vector<int64_t>> keys(num_blocks);
+    for (size_t i = 0; i < entries.size(); ++i) {
+        if (!use[i]) continue;
+        const Entry &e = entries[i];
+        for (const KeyRun &r : e.runs)
+            for (int64_t b = r.b0; b <= r.b1; ++b) keys[e.qb].push_back(b);
+    }
+    for (int64_t qb = 0; qb < num_blocks; ++qb) {
+        std::vector<int64_t> &kb = keys[qb];
+        if (kb.empty()) continue;
+        std::sort(kb.begin(), kb.end());
+        WlEntry w{};
+        w.q_lo = (int32_t)(qb * block);
+        w.q_hi = (int32_t)block_end(qb);
+        w.out_lo = w.q_lo;
+        w.flags = flags;
+        w.run_begin = (int32_t)wl.runs.size();
+        for (size_t i = 0; i < kb.size(); ++i) {
+            if (i > 0 && kb[i] == kb[i - 1] + 1) {
+                wl.runs.back().k_hi = (int32_t)block_end(kb[i]);
+            } else {
+                WlRun x{};
+                x.k_lo = (int32_t)(kb[i] * block);
+                x.k_hi = (int32_t)block_end(kb[i]);
+                wl.runs.push_back(x);
+            }
+        }
+        w.run_count = (int32_t)wl.runs.size() - w.run_begin;
+        wl.entries.push_back(w);
+        group.push_back(0);
+    }
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, group);
+    return wl;
+}
+
+WorkList Planner::partial_worklist(int rows_per_unit, int bn, int heads) const {
+    std::vector<char> use(entries.size());
+    for (size_t i = 0; i < entries.size(); ++i) use[i] = entry_rank[i] == spec.shard_rank;
+    return union_worklist(use, SEG_FIRST, rows_per_unit, bn, heads);
+}
+
 WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     WorkList wl;
     std::vector<int64_t> group;
-    if (spec.fused) {
-        // The tasks of a query block own disjoint sets of its allowed key
-        // blocks; their union, as maximal runs, is one entry.
-        std::vector<std::vector<int64_t>> keys(num_blocks);
-        for (const Entry &e : entries)
-            for (const KeyRun &r : e.runs)
-                for (int64_t b = r.b0; b <= r.b1; ++b) keys[e.qb].push_back(b);
-        for (int64_t qb = 0; qb < num_blocks; ++qb) {
-            std::vector<int64_t> &kb = keys[qb];
-            if (kb.empty()) continue;
-            std::sort(kb.begin(), kb.end());
-            WlEntry w{};
-            w.q_lo = (int32_t)(qb * block);
-            w.q_hi = (int32_t)block_end(qb);
-            w.out_lo = w.q_lo;
-            w.flags = SEG_FIRST | SEG_LAST;
-            w.run_begin = (int32_t)wl.runs.size();
-            for (size_t i = 0; i < kb.size(); ++i) {
-                if (i > 0 && kb[i] == kb[i - 1] + 1) {
-                    wl.runs.back().k_hi = (int32_t)block_end(kb[i]);
-                } else {
-                    WlRun x{};
-                    x.k_lo = (int32_t)(kb[i] * block);
-                    x.k_hi = (int32_t)block_end(kb[i]);
-                    wl.runs.push_back(x);
-                }
-            }
-            w.run_count = (int32_t)wl.runs.size() - w.run_begin;
-            wl.entries.push_back(w);
-            group.push_back(0);
-        }
-        add_units(&wl, heads, rows_per_unit, bn, spec.causal, group);
-        return wl;
-    }
+    if (spec.fused) return union_worklist(std::vector<char>(entries.size(), 1), SEG_FIRST | SEG_LAST,
+                                          rows_per_unit, bn, heads);
     for (const Entry &e : entries) {
         group.push_back(e.task);
         WlEntry w{};

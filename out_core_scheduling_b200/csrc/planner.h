@@ -65,6 +65,7 @@ struct PlanSpec {
     int fused = 0;                          // device mode: merge in the kernel, no partial slots
     int Hkv = 0;                            // key/value heads (grouped-query attention); 0 = H
     int B = 1;                              // independent sequences of N tokens per call
+    int shard_rank = 0, shard_count = 1;    // task sharding over processes
     int kv_group() const { return H / (Hkv > 0 ? Hkv : H); }
     // Key/value heads a streamed head group of g query heads reads.
     int kv_heads_of(int g) const { return g >= kv_group() ? g / kv_group() : 1; }
@@ -117,6 +118,15 @@ public:
     int64_t max_slots = 0;
     int64_t max_task_rows = 0;
     Sizing sizing;
+    // Task sharding: the rank of each entry (longest-first assignment of
+    // the entries' allowed pair counts to the least-loaded rank, ties to the
+    // lower rank and entry), and the pairs (per head) this rank and all
+    // ranks compute.
+    std::vector<int32_t> entry_rank;
+    double shard_pairs = 0, total_pairs = 0;
+    int64_t shard_entries = 0;
+    // Allowed (query, key) pairs of entry e, per head.
+    double entry_pairs(const Entry &e) const;
 
     // rows_per_unit: query rows one CTA covers; bn: key tile width.  With
     // spec.fused, one entry per query block holds the allowed key blocks of
@@ -124,6 +134,11 @@ public:
     // output directly; otherwise one entry per (task, query block) with a
     // partial slot.
     WorkList device_worklist(int rows_per_unit, int bn, int heads) const;
+    // This rank's part of a sharded forward: one entry per query block with
+    // the union of the key runs of this rank's entries, flagged SEG_FIRST
+    // only, so that the kernel leaves the rank's normalised partial and its
+    // lse in the fp32 accumulator at the global row.
+    WorkList partial_worklist(int rows_per_unit, int bn, int heads) const;
     // Key-stationary work list for the key and value gradients: one entry
     // per (task, key block) with the runs of query blocks the task's mask
     // allows (with spec.fused: one entry per key block over all tasks).
@@ -138,6 +153,15 @@ public:
     std::vector<MergeSeg> leaf_merge_segments(int64_t t) const;
     // Members of leaf t whose Q (resp. K/V) rows a streamed task needs.
     void leaf_needs(int64_t t, std::vector<char> *need_q, std::vector<char> *need_kv) const;
+
+private:
+    // One entry per query block over the key blocks of the entries `use`
+    // selects, as maximal runs.
+    WorkList union_worklist(const std::vector<char> &use, int32_t flags, int rows_per_unit, int bn,
+                            int heads) const;
+    void assign_shards();
+
+public:
 
     // Simulate the block cache with the given capacities; false if some
     // task (with its predecessor) needs more slots than there are.

@@ -1,0 +1,204 @@
+"""Task sharding on CPU: the planner's assignment of (task, query block)
+entries to ranks, and the exchange of out_core_scheduling_b200.sharded over
+gloo with 2 and 3 processes.  The three per-rank steps are replaced by fp64
+host stand-ins built from the plan's own entry list, so the tests check the
+host logic (every allowed pair on exactly one rank, the two collectives and
+the buffer packing) against the oracle's full attention."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from out_core_scheduling_b200 import cqsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CONFIGS = [
+    # (N, H, d, levels, causal)
+    (7 * 64, 2, 64, [3], False),
+    (7 * 64, 2, 64, [3], True),
+    (13 * 32, 1, 64, [4], True),
+    (91 * 8, 1, 64, [4, 3], False),
+    (91 * 8 + 5, 1, 64, [4, 3], True),   # ragged N
+    (1000, 1, 128, [4], False),           # ragged N
+]
+
+
+def _total_pairs(N, causal):
+    return N * (N + 1) / 2 if causal else float(N) * N
+
+
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: f"n{c[0]}-l{c[3]}-{'c' if c[4] else 'nc'}")
+def test_every_pair_on_exactly_one_rank(cfg, G):
+    """The ranks' entries partition the plan's entries; their allowed pairs
+    sum to N^2 (N (N + 1) / 2 causal), whatever the ragged tail."""
+    N, H, d, ls, causal = cfg
+    plans = [cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, shard_rank=r, shard_count=G) for r in range(G)]
+    infos = [p.info() for p in plans]
+    assert sum(i["shard_pairs"] for i in infos) == _total_pairs(N, causal)
+    assert all(i["total_pairs"] == _total_pairs(N, causal) for i in infos)
+    assert sum(i["shard_entries"] for i in infos) == infos[0]["num_entries"]
+    # Every rank's plan agrees on the owner of every entry.
+    owners = [[p.entry(i)["shard"] for i in range(infos[0]["num_entries"])] for p in plans]
+    assert all(o == owners[0] for o in owners)
+    assert all(0 <= x < G for x in owners[0])
+    for r, i in enumerate(infos):
+        assert i["shard_entries"] == owners[0].count(r)
+
+
+@pytest.mark.parametrize("G", [2, 3, 8])
+def test_longest_first_balance(G):
+    """Longest-first assignment: no rank is loaded above the mean by more
+    than the largest entry."""
+    N, H, d, ls, causal = 13 * 64, 1, 64, [4], True
+    plans = [cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, shard_rank=r, shard_count=G) for r in range(G)]
+    loads = [p.info()["shard_pairs"] for p in plans]
+    p0 = plans[0]
+    blk = p0.info()["block_tokens"]
+    biggest = 0.0
+    for i in range(p0.info()["num_entries"]):
+        e = p0.entry(i)
+        n = 0.0
+        for b0, b1 in e["runs"]:
+            for b in range(b0, b1 + 1):
+                n += blk * (blk + 1) / 2 if (causal and b == e["q_block"]) else blk * blk
+        biggest = max(biggest, n)
+    assert max(loads) <= sum(loads) / G + biggest
+
+
+def test_shard_plan_errors():
+    for rank, count in ((2, 2), (-1, 2), (3, 1)):
+        with pytest.raises(cqsa.CqsaError) as ei:
+            cqsa.cqsa_plan_ex(7 * 64, 1, 64, [3], shard_rank=rank, shard_count=count)
+        assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------ exchange (gloo)
+class HostOps:
+    """fp64 host stand-ins of the three per-rank library steps, for CPU
+    ranks only (the product path is the library; see sharded.LibraryOps)."""
+
+    @staticmethod
+    def forward_partial(plan, q, k, v, o_part, lse_part):
+        import torch
+        info = plan.info()
+        N, H, d, blk, causal = info["N"], info["H"], info["d"], info["block_tokens"], info["causal"]
+        qn, kn, vn = (x.double().numpy() for x in (q, k, v))
+        o_acc = np.zeros((N, H, d))
+        l_acc = np.full((H, N), -np.inf)
+        for i in range(info["num_entries"]):
+            e = plan.entry(i)
+            if e["shard"] != info["shard_rank"]:
+                continue
+            rows = np.arange(e["q_block"] * blk, min((e["q_block"] + 1) * blk, N))
+            keys = np.concatenate([np.arange(b0 * blk, min((b1 + 1) * blk, N)) for b0, b1 in e["runs"]])
+            if rows.size == 0 or keys.size == 0:
+                continue
+            s = np.einsum("ihd,jhd->hij", qn[rows], kn[keys]) / np.sqrt(d)
+            if causal:
+                s = np.where((keys[None, :] <= rows[:, None])[None], s, -np.inf)
+            m = s.max(axis=2, keepdims=True)
+            lse_e = m[..., 0] + np.log(np.exp(s - m).sum(axis=2))          # [H, rows]
+            o_e = np.einsum("hij,jhd->ihd", np.exp(s - lse_e[..., None]), vn[keys])
+            la = l_acc[:, rows]
+            M = np.maximum(la, lse_e)
+            wa = np.where(np.isinf(la), 0.0, np.exp(la - M))
+            we = np.exp(lse_e - M)
+            W = wa + we
+            o_acc[rows] = (wa.T[..., None] * o_acc[rows] + we.T[..., None] * o_e) / W.T[..., None]
+            l_acc[:, rows] = M + np.log(W)
+        o_part.copy_(torch.from_numpy(o_acc).float())
+        lse_part.copy_(torch.from_numpy(l_acc).float())
+
+    @staticmethod
+    def partial_rescale(plan, o_part, lse_part, lse_max, w):
+        import torch
+        lp, lm = lse_part.double().numpy(), lse_max.double().numpy()
+        wr = np.where(np.isinf(lp), 0.0, np.exp(lp - lm))                    # [H, N]
+        w.copy_(torch.from_numpy(wr).float())
+        o_part.copy_(torch.from_numpy(o_part.double().numpy() * wr.T[..., None]).float())
+
+    @staticmethod
+    def partial_finish(plan, o_sum, w_sum, lse_max, out, lse):
+        import torch
+        W = w_sum.double().numpy()
+        out.copy_(torch.from_numpy(o_sum.double().numpy() / W.T[..., None]).to(out.dtype))
+        lse.copy_(torch.from_numpy(lse_max.double().numpy() + np.log(W)).float())
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, cfg, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from out_core_scheduling_b200 import cqsa as lib
+    from out_core_scheduling_b200.inputs import make_qkv
+    from out_core_scheduling_b200.sharded import forward_sharded
+    from test_sharded import HostOps
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        N, H, d, ls, causal = cfg
+        qt, kt, vt = make_qkv(N, H, d, dtype=torch.float32, seed=11)
+        plan = lib.cqsa_plan_ex(N, H, d, ls, causal=causal, shard_rank=rank, shard_count=world)
+        out = torch.empty(N, H, d)
+        lse = torch.empty(H, N)
+        forward_sharded(plan, qt, kt, vt, out, lse, ops=HostOps)
+        ref_o, ref_l = oracle.attention_rows(qt, kt, vt, causal=causal)
+        e_o = float(np.abs(out.double().numpy() - ref_o).max())
+        e_l = float(np.abs(lse.double().numpy().T - ref_l).max())
+        q.put((rank, e_o, e_l))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("cfg", [CONFIGS[1], CONFIGS[3], CONFIGS[4]], ids=["l3-c", "l43-nc", "l43-ragged-c"])
+def test_forward_sharded_gloo(cfg, world):
+    """Every rank ends with the full attention (fp32 buffers: 1e-5)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, cfg, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, e_o, e_l in res:
+        assert e_o <= 1e-5 and e_l <= 1e-5, (rank, e_o, e_l)
+
+
+def test_plan_rank_must_match_group():
+    """forward_sharded refuses a plan made for another rank or world size."""
+    from out_core_scheduling_b200.sharded import forward_sharded
+
+    plan = cqsa.cqsa_plan_ex(7 * 64, 1, 64, [3], shard_rank=1, shard_count=2)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        import torch
+        x = torch.zeros(7 * 64, 1, 64)
+        with pytest.raises(ValueError):
+            forward_sharded(plan, x, x, x, x.clone(), torch.zeros(1, 7 * 64), ops=HostOps)
+    finally:
+        dist.destroy_process_group()

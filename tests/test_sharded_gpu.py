@@ -1,0 +1,168 @@
+"""GPU parity of the sharded forward.  The G ranks of a shard are run one
+after another on one GPU (each rank's kernels are independent: nothing
+waits on another rank), with the two collectives of the exchange stood in
+for by torch reductions over the ranks' buffers; the library's partial
+forward, rescale and finish kernels do the rest, and the result is compared
+with the fp64 oracle.  One test runs out_core_scheduling_b200.sharded over a
+real NCCL group of one process."""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+from out_core_scheduling_b200 import cqsa
+from out_core_scheduling_b200.inputs import make_qkv, sample_rows
+
+from parity import check, run
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _expand(x, g):
+    return x.repeat_interleave(g, dim=1).contiguous() if g > 1 else x
+
+
+def _sharded(N, H, d, ls, causal, dtype, G, Hkv=0, B=1, seed=0):
+    cdt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    Hk = Hkv or H
+    lead = (B,) if B > 1 else ()
+    qs, ks, vs = [], [], []
+    for b in range(B):
+        qs.append(make_qkv(N, H, d, dtype=dtype, seed=seed + b, device=DEV)[0])
+        _, kb, vb = make_qkv(N, Hk, d, dtype=dtype, seed=seed + 100 + b, device=DEV)
+        ks.append(kb)
+        vs.append(vb)
+    q, k, v = (torch.stack(x) if B > 1 else x[0] for x in (qs, ks, vs))
+    o_parts, l_parts = [], []
+    plans = [cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, H_kv=Hkv, B=B, shard_rank=r, shard_count=G)
+             for r in range(G)]
+    for p in plans:
+        o = torch.empty(lead + (N, H, d), device=DEV)
+        l = torch.empty(lead + (H, N), device=DEV)
+        cqsa.cqsa_forward_partial(p, q, k, v, o, l)
+        o_parts.append(o)
+        l_parts.append(l)
+    lse_max = torch.stack(l_parts).amax(0)                       # all-reduce MAX
+    ws = []
+    for p, o, l in zip(plans, o_parts, l_parts):
+        w = torch.empty_like(l)
+        cqsa.cqsa_partial_rescale(p, o, l, lse_max, w)
+        ws.append(w)
+    o_sum, w_sum = torch.stack(o_parts).sum(0), torch.stack(ws).sum(0)  # all-reduce SUM
+    out = torch.empty(lead + (N, H, d), device=DEV, dtype=dtype)
+    lse = torch.empty(lead + (H, N), device=DEV)
+    cqsa.cqsa_partial_finish(plans[0], o_sum, w_sum, lse_max, out, lse)
+    for p in plans:
+        p.sync()
+    return q, k, v, out, lse, plans
+
+
+CASES = [
+    # (N, H, d, levels, causal, dtype, G)
+    (7 * 256, 2, 128, [3], False, torch.bfloat16, 2),
+    (7 * 256, 2, 128, [3], True, torch.bfloat16, 3),
+    (13 * 128, 2, 64, [4], True, torch.bfloat16, 8),
+    (13 * 128, 2, 128, [4], False, torch.bfloat16, 5),
+    (91 * 32, 1, 128, [4, 3], True, torch.bfloat16, 4),
+    (1000, 2, 128, [4], True, torch.bfloat16, 3),          # ragged N
+    (7 * 200, 1, 64, [3], False, torch.float32, 2),
+    (7 * 200, 1, 128, [3], True, torch.float32, 3),
+    (7 * 128, 2, 128, [3], True, torch.bfloat16, 1),       # one rank = the plain forward
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"n{c[0]}-d{c[2]}-l{c[3]}-{'c' if c[4] else 'nc'}-"
+                                                      f"{str(c[5])[6:]}-g{c[6]}")
+def test_sharded_forward_matches_oracle(case):
+    N, H, d, ls, causal, dtype, G = case
+    q, k, v, out, lse, _ = _sharded(N, H, d, ls, causal, dtype, G)
+    check(out, lse, q, k, v, np.arange(N) if N <= 3000 else sample_rows(N, 512), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sharded_grouped_query_and_batch(causal):
+    N, H, Hkv, d, B, G = 7 * 128, 4, 2, 128, 2, 3
+    q, k, v, out, lse, _ = _sharded(N, H, d, [3], causal, torch.bfloat16, G, Hkv=Hkv, B=B, seed=20)
+    for b in range(B):
+        check(out[b], lse[b], q[b], _expand(k[b], H // Hkv), _expand(v[b], H // Hkv), np.arange(N), causal)
+
+
+def test_one_rank_partial_is_the_forward():
+    """With one rank the partial is the whole attention: o_part matches the
+    plain forward's out within the bf16 output tolerance (the two sum the
+    tasks in different orders) and lse_part its lse."""
+    N, H, d = 13 * 128, 2, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=30, device=DEV)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    o = torch.empty(N, H, d, device=DEV)
+    l = torch.empty(H, N, device=DEV)
+    cqsa.cqsa_forward_partial(plan, q, k, v, o, l)
+    plan.sync()
+    assert (o - out.float()).abs().max().item() <= 2e-2
+    assert (l - lse).abs().max().item() <= 1e-4
+
+
+def test_rank_without_entries_leaves_neutral_rows():
+    """More ranks than entries: the idle rank's partial is o = 0, lse = -inf
+    everywhere, and the exchange still gives the full attention."""
+    N, H, d = 7 * 64, 1, 64
+    p0 = cqsa.cqsa_plan_ex(N, H, d, [3], shard_rank=0, shard_count=64)
+    E = p0.info()["num_entries"]
+    G = E + 2
+    q, k, v, out, lse, plans = _sharded(N, H, d, [3], False, torch.bfloat16, G, seed=40)
+    idle = [p for p in plans if p.info()["shard_entries"] == 0]
+    assert idle
+    o = torch.full((N, H, d), 7.0, device=DEV)
+    l = torch.zeros(H, N, device=DEV)
+    cqsa.cqsa_forward_partial(idle[0], q, k, v, o, l)
+    idle[0].sync()
+    assert o.abs().max().item() == 0.0 and torch.isinf(l).all() and (l < 0).all()
+    check(out, lse, q, k, v, np.arange(N), False)
+
+
+def test_sharded_plan_rejects_forward_and_backward():
+    N, H, d = 7 * 64, 1, 64
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], shard_rank=0, shard_count=2)
+    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+    g = [torch.empty_like(q) for _ in range(3)]
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_backward(plan, q, k, v, out, lse, q, *g)
+    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_forward_sharded_over_nccl_one_rank():
+    """out_core_scheduling_b200.sharded with a one-process NCCL group: the
+    library kernels and the two NCCL all-reduces on the current stream."""
+    import torch.distributed as dist
+    from out_core_scheduling_b200.sharded import forward_sharded
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device(DEV))
+    try:
+        N, H, d = 13 * 128, 2, 128
+        q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=50, device=DEV)
+        for causal in (False, True):
+            plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, shard_rank=0, shard_count=1)
+            out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+            forward_sharded(plan, q, k, v, out, lse)
+            plan.sync()
+            check(out, lse, q, k, v, np.arange(N), causal)
+    finally:
+        dist.destroy_process_group()
