@@ -195,6 +195,102 @@ class Dist:
             self.dist.destroy_process_group()
 
 
+# ------------------------------------------------------------ sharded arm
+def run_sharded(args, W):
+    """--shard: ONE problem of the workload split over the ranks (strong
+    scaling): every rank plans with shard_rank = its rank, computes its
+    (task, query block) entries with cqsa_forward_partial, and the ranks
+    exchange their log-sum-exp partials with two NCCL all-reduces
+    (out_core_scheduling_b200.sharded).  Launched without torchrun it runs
+    on a one-process NCCL group.  Device workloads only."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+    from out_core_scheduling_b200 import cqsa
+    from out_core_scheduling_b200.inputs import make_qkv
+    from out_core_scheduling_b200.sharded import forward_sharded
+
+    if W["mode"] != "device":
+        raise SystemExit("--shard takes a device workload")
+    D = Dist()
+    dev = D.local_rank
+    torch.cuda.set_device(dev)
+    torch_dev = f"cuda:{dev}"
+    cqsa.load_library()
+    if not dist.is_initialized():
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(port))
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(torch_dev))
+    rank, world = dist.get_rank(), dist.get_world_size()
+    N, H, d = W["N"], W["H"], W["d"]
+    tdt = torch.bfloat16 if W["dtype"] == "bf16" else torch.float32
+    cdt = cqsa.CQSA_BF16 if W["dtype"] == "bf16" else cqsa.CQSA_FP32
+    q, k, v = make_qkv(N, H, d, dtype=tdt, seed=0, device=torch_dev, dist=W["dist"])  # the same problem everywhere
+    plans = [cqsa.cqsa_plan_ex(N, H, d, W["ls"], causal=c, dtype=cdt, shard_rank=rank, shard_count=world)
+             for c in W["variants"]]
+    outs = [torch.empty_like(q) for _ in plans]
+    lses = [torch.empty(H, N, device=torch_dev) for _ in plans]
+    flops_step = sum(useful_flops(N, H, d, c) for c in W["variants"])
+
+    def step():
+        for p, o, l in zip(plans, outs, lses):
+            forward_sharded(p, q, k, v, o, l)
+
+    for _ in range(args.warmup):
+        step()
+    for p in plans:
+        p.sync()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(gpu_id_for_smi(torch, dev))
+    for p in plans:
+        p.kernel_stats(reset=True)
+        p.profile(True)
+    sampler.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(dev)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier(dev)
+    clocks = sampler.stop()
+    for p in plans:
+        p.profile(False)
+        p.sync()
+    stats = [p.kernel_stats(reset=True) for p in plans]
+    ms = D.max(ev0.elapsed_time(ev1), torch_dev)
+    value = flops_step * args.steps / (ms * 1e-3) / 1e12
+    infos = [p.info() for p in plans]
+    exch = sum(N * H * (d + 2) * 4 for _ in plans)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": W["dtype"], "data": "synthetic (seeded torch.Generator, see inputs.py)",
+        "config": {"workload": args.workload, "N": N, "H": H, "d": d, "l": W["ls"], "causal": W["variants"],
+                   "mode": "device, task shards", "parallelism": f"one problem in {world} task shards",
+                   "l2": "inputs larger than L2; no flush"},
+        "shard": {"rank0_entries": [i["shard_entries"] for i in infos],
+                  "rank0_pair_share": [i["shard_pairs"] / i["total_pairs"] for i in infos],
+                  "exchange_bytes_per_rank_per_step": exch,
+                  "collectives_per_step": 2 * len(plans)},
+        "clocks": clocks,
+        # attention (none on a rank without entries) + partial init, rescale and finish
+        "gpu_launches": sum(s["attn_launches"] for s in stats) + 3 * len(plans) * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, W):
     import torch
@@ -653,12 +749,16 @@ def main(argv=None):
                     help="only warm-up + steps of the device path (for ncu captures)")
     ap.add_argument("--profile-backward", action="store_true",
                     help="with --profile-run: the first variant's backward after the forward steps")
+    ap.add_argument("--shard", action="store_true",
+                    help="one problem split over the ranks in task shards (strong scaling; not the default line)")
     args = ap.parse_args(argv)
     if args.warmup < 0 or args.steps < 1:
         ap.error("need --steps >= 1 and --warmup >= 0")
     W = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, W)
+    elif args.shard:
+        run_sharded(args, W)
     else:
         run_ours(args, W)
 
