@@ -56,7 +56,8 @@ typedef enum {
     CQSA_ERR_CUDA = 5,              /* a CUDA runtime call failed; message names it */
     CQSA_ERR_TIMEOUT = 6,           /* a bounded device-side wait ran out; the kernel stopped early */
     CQSA_ERR_UNSUPPORTED = 7,       /* valid request this build does not implement (e.g. d not 64/128) */
-    CQSA_ERR_NO_DEVICE = 8          /* no usable sm_100 device */
+    CQSA_ERR_NO_DEVICE = 8,         /* no usable sm_100 device */
+    CQSA_ERR_INTERNAL = 9           /* a consistency check failed (CQSA_DEBUG plan checks, injected faults) */
 } cqsa_status_t;
 
 typedef enum { CQSA_BF16 = 0, CQSA_FP32 = 1 } cqsa_dtype_t;
@@ -131,6 +132,7 @@ typedef struct {
     int B;                              /* sequences per call */
     int shard_rank, shard_count;        /* task sharding (count 1: none) */
     int64_t shard_entries;              /* entries this rank computes */
+    int debug_checked;                  /* CQSA_DEBUG set: the plan passed the brute-force checks */
     double shard_pairs;                 /* allowed (query, key) pairs of those entries, per head */
     double total_pairs;                 /* allowed pairs of all entries, per head */
 } cqsa_plan_info_t;
@@ -282,6 +284,17 @@ cqsa_status_t cqsa_difference_set(int l, int *D);
  * warps' bounded waits run out and the next cqsa_plan_sync reports
  * CQSA_ERR_TIMEOUT.  Never needed in normal use. */
 cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_mma);
+
+/* cqsa_debug_inject -- host-side fault injection for tests.  kind =
+ * CQSA_FAULT_ALLOC: the nth following device allocation of the library
+ * (plan arenas) fails as if cudaMalloc had run out of memory; kind =
+ * CQSA_FAULT_COPY: the nth following host<->device copy of a streamed
+ * forward fails.  The failing call returns CQSA_ERR_CUDA without touching
+ * the GPU; work already enqueued completes, and the plan stays usable (a
+ * failed allocation is retried by the next call).  nth = 0 clears; the
+ * setting is process-wide and fires once.  Errors: INVALID_ARG. */
+enum { CQSA_FAULT_ALLOC = 1, CQSA_FAULT_COPY = 2 };
+cqsa_status_t cqsa_debug_inject(int kind, int64_t nth);
 
 /* Per-kernel device time of a plan's launches, from CUDA events recorded
  * on the stream each kernel is launched on. */

@@ -199,6 +199,30 @@ def decomposed_attention(q, k, v, ls, causal: bool, scale: float):
     return out, lse_out
 
 
+def lse_merge(outs, lses):
+    """Log-sum-exp recomposition of partial attention results over disjoint
+    key sets (arXiv abstract "Stream-CQSA: Exact Out-of-Memory Recovery for
+    Attention": local statistics are recomposed into the full output;
+    wispaper.ai blog, section "Implementation", step 4: aggregate).
+
+    outs: sequence of [R, H, d] partial outputs, each normalised by its own
+    softmax denominator; lses: the matching [R, H] natural-log denominators,
+    -inf where a partial saw no key.  With M the largest lse of a row and
+    w_s = exp(lse_s - M), the row is sum_s w_s o_s / sum_s w_s and its lse
+    M + ln sum_s w_s (0 and -inf for a row no partial saw).
+    Returns (out [R, H, d], lse [R, H]) in float64."""
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])     # [S, R, H]
+    O = np.stack([np.asarray(x, dtype=np.float64) for x in outs])     # [S, R, H, d]
+    M = L.max(axis=0)
+    Ms = np.where(np.isfinite(M), M, 0.0)
+    W = np.where(np.isfinite(L), np.exp(np.where(np.isfinite(L), L, 0.0) - Ms), 0.0)
+    tot = W.sum(axis=0)
+    seen = tot > 0
+    lse = np.where(seen, Ms + np.log(np.where(seen, tot, 1.0)), -np.inf)
+    out = np.einsum("srh,srhd->rhd", W, O) / np.where(seen, tot, 1.0)[..., None]
+    return out, lse
+
+
 def decomposed_backward(q, k, v, dout, ls, causal: bool, scale: float):
     """fp64 CQS-decomposed backward: the merged statistics of the whole row
     (lse_i, and D_i = <dout_i, out_i> from the decomposed forward), then, task

@@ -22,6 +22,9 @@ CQSA_ERR_CUDA = 5
 CQSA_ERR_TIMEOUT = 6
 CQSA_ERR_UNSUPPORTED = 7
 CQSA_ERR_NO_DEVICE = 8
+CQSA_ERR_INTERNAL = 9
+CQSA_FAULT_ALLOC = 1
+CQSA_FAULT_COPY = 2
 
 CQSA_BF16 = 0
 CQSA_FP32 = 1
@@ -38,6 +41,7 @@ EXPORTS = (
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
+    "cqsa_debug_inject",
 )
 
 
@@ -68,6 +72,7 @@ class PlanInfo(ctypes.Structure):
                 ("d2h_bytes", ctypes.c_size_t), ("useful_flops", ctypes.c_double),
                 ("merge", ctypes.c_int), ("H_kv", ctypes.c_int), ("B", ctypes.c_int),
                 ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int), ("shard_entries", ctypes.c_int64),
+                ("debug_checked", ctypes.c_int),
                 ("shard_pairs", ctypes.c_double), ("total_pairs", ctypes.c_double)]
 
     def as_dict(self) -> dict:
@@ -127,6 +132,7 @@ def load_library():
         "cqsa_forward_partial": (st, [P, P, P, P, P, P, P]),
         "cqsa_partial_rescale": (st, [P, P, P, P, P, P]),
         "cqsa_partial_finish": (st, [P, P, P, P, P, P, P]),
+        "cqsa_debug_inject": (st, [ctypes.c_int, ctypes.c_int64]),
         "cqsa_plan_destroy": (None, [P]),
         "cqsa_last_error": (ctypes.c_char_p, []),
     }
@@ -341,6 +347,12 @@ def cqsa_partial_finish(plan: Plan, o_sum, w_sum, lse_max, out, lse, stream=None
     _check(load_library().cqsa_partial_finish(plan.handle, o_sum.data_ptr(), w_sum.data_ptr(),
                                               lse_max.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_debug_inject(kind: int, nth: int):
+    """Test hook: the nth following library allocation (CQSA_FAULT_ALLOC)
+    or streamed copy (CQSA_FAULT_COPY) fails on the host; 0 clears."""
+    _check(load_library().cqsa_debug_inject(kind, nth))
 
 
 def cqsa_difference_set(l: int):

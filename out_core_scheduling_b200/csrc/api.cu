@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -35,6 +36,23 @@ using namespace cqsa;
 namespace {
 
 thread_local std::string g_err;
+
+// Host-side fault injection for tests (cqsa_debug_inject): the n-th next
+// device allocation or streamed copy of the library reports a failure
+// instead of calling CUDA.  Process-wide, one-shot.
+std::atomic<int64_t> g_fail_alloc{0}, g_fail_copy{0};
+
+bool injected(std::atomic<int64_t> &c) {
+    int64_t v = c.load();
+    while (v > 0)
+        if (c.compare_exchange_weak(v, v - 1)) return v == 1;
+    return false;
+}
+
+cudaError_t lib_malloc(void **ptr, size_t bytes) {
+    if (injected(g_fail_alloc)) return cudaErrorMemoryAllocation;
+    return cudaMalloc(ptr, bytes);
+}
 
 cqsa_status_t fail(cqsa_status_t code, const char *fmt, ...) {
     char buf[1024];
@@ -265,7 +283,7 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
     if (pl.spec.budget && a.total > pl.spec.budget)
         return fail(CQSA_ERR_BUDGET, "device-resident path needs %zu bytes, budget is %zu", a.total, pl.spec.budget);
     char *arena = nullptr;
-    CK(cudaMalloc(&arena, a.total));
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
     P->dev_arena = arena;
     P->dev_bytes = a.total;
     CK(cudaMemset(arena, 0, a.total));
@@ -321,7 +339,7 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
         return fail(CQSA_ERR_CUDA, "internal: host-mode arena layout mismatch (%zu vs %zu)", a.total,
                     pl.sizing.host_arena);
     char *arena = nullptr;
-    CK(cudaMalloc(&arena, a.total));
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
     P->host_arena = arena;
     P->host_bytes = a.total;
     P->g = g;
@@ -448,7 +466,7 @@ cqsa_status_t setup_partial(cqsa_plan_t *P) {
     const size_t o_err = a.take(256);
     const size_t o_wl = a.take(wl_region(wl));
     char *arena = nullptr;
-    CK(cudaMalloc(&arena, a.total));
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
     P->part_arena = arena;
     CK(cudaMemset(arena, 0, a.total));
     P->part_err = reinterpret_cast<int *>(arena + o_err);
@@ -534,7 +552,7 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     const size_t o_qwl = a.take(wl_region(qwl));
     const size_t o_kvwl = a.take(wl_region(kvwl));
     char *arena = nullptr;
-    CK(cudaMalloc(&arena, a.total));
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
     P->bwd_arena = arena;
     P->bwd_bytes = a.total;
     CK(cudaMemset(arena, 0, 256));
@@ -637,6 +655,7 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
 // tensor and a compact [*, g, d] one.
 cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width, size_t rows,
                       cudaMemcpyKind kind, cudaStream_t s) {
+    if (injected(g_fail_copy)) return cudaErrorUnknown;
     if (dpitch == width && spitch == width) return cudaMemcpyAsync(dst, src, width * rows, kind, s);
     return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, kind, s);
 }
@@ -740,6 +759,19 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     CK(cudaStreamWaitEvent(stream, P->ev_done_comp, 0));
     CK(cudaStreamWaitEvent(stream, P->ev_done_out, 0));
     return CQSA_OK;
+}
+
+// After a streamed forward failed part-way: order the caller's stream after
+// everything the plan's internal streams already hold, so the next call
+// cannot overlap the abandoned one.  Best effort; the original error stands.
+void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
+    if (!P->s_in || !P->s_comp || !P->s_out) return;
+    cudaEventRecord(P->ev_start, P->s_in);
+    cudaEventRecord(P->ev_done_comp, P->s_comp);
+    cudaEventRecord(P->ev_done_out, P->s_out);
+    cudaStreamWaitEvent(stream, P->ev_start, 0);
+    cudaStreamWaitEvent(stream, P->ev_done_comp, 0);
+    cudaStreamWaitEvent(stream, P->ev_done_out, 0);
 }
 
 cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
@@ -872,7 +904,10 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
         char *ob = static_cast<char *>(out) + b * qs;
         float *lb = lse + b * ls;
         st = host ? forward_host(plan, qb, kb, vb, ob, lb, s) : forward_device(plan, qb, kb, vb, ob, lb, s);
-        if (st != CQSA_OK) return st;
+        if (st != CQSA_OK) {
+            if (host) join_after_error(plan, s);
+            return st;
+        }
     }
     return CQSA_OK;
 }
@@ -993,6 +1028,18 @@ cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_
     return CQSA_OK;
 }
 
+cqsa_status_t cqsa_debug_inject(int kind, int64_t nth) {
+    if (nth < 0) return fail(CQSA_ERR_INVALID_ARG, "nth must be >= 0");
+    if (kind == CQSA_FAULT_ALLOC) {
+        g_fail_alloc.store(nth);
+    } else if (kind == CQSA_FAULT_COPY) {
+        g_fail_copy.store(nth);
+    } else {
+        return fail(CQSA_ERR_INVALID_ARG, "kind must be CQSA_FAULT_ALLOC or CQSA_FAULT_COPY");
+    }
+    return CQSA_OK;
+}
+
 cqsa_status_t cqsa_plan_profile(cqsa_plan_t *plan, int enable) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     plan->profiling = enable ? 1 : 0;
@@ -1058,6 +1105,7 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->shard_rank = pl.spec.shard_rank;
     info->shard_count = pl.spec.shard_count;
     info->shard_entries = pl.shard_entries;
+    info->debug_checked = pl.debug_checked ? 1 : 0;
     info->shard_pairs = pl.shard_pairs;
     info->total_pairs = pl.total_pairs;
     return CQSA_OK;

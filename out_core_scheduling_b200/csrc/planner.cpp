@@ -1,6 +1,8 @@
 // planner.cpp -- CQS planner (see planner.h for the sources it follows).
 #include "planner.h"
 
+#include <stdlib.h>
+
 #include <algorithm>
 #include <map>
 #include <numeric>
@@ -190,7 +192,63 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     for (int32_t v : slots_per_block) max_slots = std::max<int64_t>(max_slots, v);
     assign_shards();
     size_plan();
+    const char *dbg = getenv("CQSA_DEBUG");
+    if (dbg && dbg[0] && !(dbg[0] == '0' && dbg[1] == 0)) {
+        const std::string bad = verify();
+        if (!bad.empty()) {
+            *code = 9;  // CQSA_ERR_INTERNAL
+            return "CQSA_DEBUG: plan invariant violated: " + bad;
+        }
+        debug_checked = true;
+    }
     *code = 0;
+    return "";
+}
+
+std::string Planner::verify() const {
+    const int64_t P = num_blocks;
+    // Runs: sorted, disjoint, in range; slots: 0..n-1 per query block.
+    std::vector<int32_t> seen_slots(P, 0);
+    for (const Entry &e : entries) {
+        if (e.qb < 0 || e.qb >= P) return "query block out of range";
+        int64_t prev = -1;
+        for (const KeyRun &r : e.runs) {
+            if (r.b0 > r.b1 || r.b0 <= prev || r.b1 >= P) return "key runs not sorted, disjoint and in range";
+            prev = r.b1;
+        }
+        if (e.slot != seen_slots[e.qb]++) return "slots do not number a query block's entries in order";
+    }
+    for (int64_t b = 0; b < P; ++b)
+        if (seen_slots[b] != slots_per_block[b]) return "slot count mismatch";
+    // Exactly-once coverage of the allowed block pairs.
+    if (P <= 4096) {
+        std::vector<uint8_t> hits((size_t)P * P, 0);
+        for (const Entry &e : entries)
+            for (const KeyRun &r : e.runs)
+                for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
+                    uint8_t &h = hits[(size_t)e.qb * P + kb];
+                    if (h == 255) return "pair counted 255 times";
+                    ++h;
+                }
+        for (int64_t qb = 0; qb < P; ++qb)
+            for (int64_t kb = 0; kb < P; ++kb) {
+                const bool allowed = block_rows(qb) > 0 && block_rows(kb) > 0 && (!spec.causal || kb <= qb);
+                if (hits[(size_t)qb * P + kb] != (allowed ? 1 : 0)) return "a block pair is not covered exactly once";
+            }
+    }
+    // Device work list: the units of each entry cover its rows once per head.
+    const int rows = unit_rows_for(spec.elem_bytes);
+    WorkList wl = device_worklist(rows, key_tile_for(spec.elem_bytes), spec.H);
+    std::vector<int64_t> covered(wl.entries.size(), 0);
+    for (const WlUnit &u : wl.units) {
+        if (u.entry < 0 || u.entry >= (int32_t)wl.entries.size()) return "unit entry out of range";
+        const WlEntry &e = wl.entries[u.entry];
+        if (u.q0 < e.q_lo || u.q0 >= e.q_hi || u.head < 0 || u.head >= spec.H) return "unit outside its entry";
+        covered[u.entry] += std::min<int64_t>(rows, e.q_hi - u.q0);
+    }
+    for (size_t i = 0; i < wl.entries.size(); ++i)
+        if (covered[i] != (int64_t)(wl.entries[i].q_hi - wl.entries[i].q_lo) * spec.H)
+            return "device units do not cover an entry's rows once per head";
     return "";
 }
 

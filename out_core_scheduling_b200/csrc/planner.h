@@ -127,6 +127,14 @@ public:
     int64_t shard_entries = 0;
     // Allowed (query, key) pairs of entry e, per head.
     double entry_pairs(const Entry &e) const;
+    // With the environment variable CQSA_DEBUG set (not "0"), build() also
+    // re-checks the plan by brute force (verify()); debug_checked says so.
+    bool debug_checked = false;
+    // Every allowed ordered block pair lies in exactly one entry; runs are
+    // sorted, disjoint and in range; slots number each query block's
+    // entries 0..n-1; the device work lists cover each entry's rows once.
+    // Returns "" or what is violated.  Pair check up to 4096 blocks.
+    std::string verify() const;
 
     // rows_per_unit: query rows one CTA covers; bn: key tile width.  With
     // spec.fused, one entry per query block holds the allowed key blocks of

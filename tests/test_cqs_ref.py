@@ -110,3 +110,57 @@ def test_decomposition_detects_a_dropped_owner():
         assert np.abs(dec - full).max() > 1e-3
     finally:
         cqs_ref.diagonal_owner = orig
+
+
+# ------------------------------------------------------------------ lse_merge
+def _subset_partial(q, k, v, keys):
+    """fp64 softmax attention of every query row over the key rows `keys`
+    (the plain definition; an input to the merge, not its expected value)."""
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    d = q.shape[2]
+    if len(keys) == 0:
+        return np.zeros(q.shape), np.full(q.shape[:2], -np.inf)
+    s = np.einsum("ihd,jhd->ihj", q, k[keys]) / np.sqrt(d)
+    m = s.max(axis=2, keepdims=True)
+    lse = m[..., 0] + np.log(np.exp(s - m).sum(axis=2))
+    o = np.einsum("ihj,jhd->ihd", np.exp(s - lse[..., None]), v[keys])
+    return o, lse
+
+
+@pytest.mark.parametrize("parts", [1, 2, 5])
+def test_lse_merge_of_key_subsets_is_full_attention(parts):
+    """Partials over a random partition of the keys (one part may be empty)
+    merge to the C oracle's attention over all keys."""
+    import oracle
+    rng = np.random.default_rng(parts)
+    N, H, d = 40, 2, 16
+    q, k, v = (rng.standard_normal((N, H, d)).astype(np.float32) for _ in range(3))
+    owner = rng.integers(0, parts, size=N)
+    subsets = [np.flatnonzero(owner == s) for s in range(parts)] + [np.array([], dtype=np.int64)]
+    outs, lses = zip(*(_subset_partial(q, k, v, ks) for ks in subsets))
+    got_o, got_l = cqs_ref.lse_merge(outs, lses)
+    ref_o, ref_l = oracle.attention_rows(q, k, v)
+    assert np.abs(got_o - ref_o).max() <= 1e-12 and np.abs(got_l - ref_l).max() <= 1e-12
+
+
+def test_lse_merge_special_cases():
+    rng = np.random.default_rng(9)
+    o = rng.standard_normal((3, 2, 4))
+    l = rng.standard_normal((3, 2))
+    # One partial is returned unchanged.
+    mo, ml = cqs_ref.lse_merge([o], [l])
+    assert np.allclose(mo, o, atol=1e-15) and np.allclose(ml, l, atol=1e-15)
+    # Two equal partials: same output, lse + ln 2.
+    mo, ml = cqs_ref.lse_merge([o, o], [l, l])
+    assert np.allclose(mo, o, atol=1e-15) and np.allclose(ml, l + np.log(2.0), atol=1e-15)
+    # A row no partial saw: 0 and -inf.
+    ninf = np.full((3, 2), -np.inf)
+    mo, ml = cqs_ref.lse_merge([np.zeros_like(o), np.zeros_like(o)], [ninf, ninf])
+    assert np.all(mo == 0) and np.all(np.isneginf(ml))
+    # A planted mistake (weights not normalised) is caught by the subset pin.
+    import oracle
+    q, k, v = (rng.standard_normal((12, 1, 8)).astype(np.float32) for _ in range(3))
+    outs, lses = zip(*(_subset_partial(q, k, v, ks) for ks in (np.arange(0, 5), np.arange(5, 12))))
+    L = np.stack(lses)
+    wrong = np.einsum("srh,srhd->rhd", np.exp(L - L.max(axis=0)), np.stack(outs))
+    assert np.abs(wrong - oracle.attention_rows(q, k, v)[0]).max() > 1e-3

@@ -252,3 +252,30 @@ def test_grouped_query_plans():
     with pytest.raises(cqsa.CqsaError) as ei:
         cqsa.cqsa_plan_ex(N, H, d, [4], H_kv=3)
     assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args", [
+    (7 * 64, 2, 64, [3], False, 0), (13 * 32, 1, 64, [4], True, 0), (91 * 8 + 5, 1, 64, [4, 3], True, 0),
+    (1000, 1, 128, [4], False, 0), (31 * 16, 1, 64, [6], True, 0), (21 * 13 * 8, 1, 64, [5, 4], False, 0),
+    (7 * 64, 4, 64, [3], True, 2), (57 * 4 + 3, 2, 64, [8], True, 1)])
+def test_debug_plan_checks(monkeypatch, args):
+    """CQSA_DEBUG=1: every plan re-checks itself by brute force (each allowed
+    block pair in exactly one entry, runs and slots well formed, device units
+    covering every entry's rows once per head) and reports that it did."""
+    N, H, d, ls, causal, Hkv = args
+    monkeypatch.setenv("CQSA_DEBUG", "1")
+    for merge in (cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED):
+        for dtype in (cqsa.CQSA_BF16, cqsa.CQSA_FP32):
+            p = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dtype, merge=merge, H_kv=Hkv)
+            assert p.info()["debug_checked"] == 1
+    monkeypatch.setenv("CQSA_DEBUG", "0")
+    assert cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, H_kv=Hkv).info()["debug_checked"] == 0
+
+
+def test_fault_injection_arguments():
+    for kind, nth in ((0, 1), (3, 1), (cqsa.CQSA_FAULT_ALLOC, -1)):
+        with pytest.raises(cqsa.CqsaError) as ei:
+            cqsa.cqsa_debug_inject(kind, nth)
+        assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_ALLOC, 0)
+    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, 0)

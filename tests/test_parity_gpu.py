@@ -356,3 +356,44 @@ def test_batch_of_sequences(mode, merge, causal):
     plan.sync()
     for b in range(B):
         check(out[b], lse[b], q[b], _expand(k[b], H // Hkv), _expand(v[b], H // Hkv), np.arange(N), causal)
+
+
+# ------------------------------------------------------- injected host faults
+def test_injected_allocation_failure_is_recoverable():
+    """The first arena allocation fails (host-side injection): the forward
+    reports CQSA_ERR_CUDA, allocates on the next call and is correct."""
+    N, H, d = 7 * 128, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=60)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True)
+    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_ALLOC, 1)
+    try:
+        with pytest.raises(cqsa.CqsaError) as ei:
+            cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+        assert ei.value.status == cqsa.CQSA_ERR_CUDA
+    finally:
+        cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_ALLOC, 0)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), True)
+
+
+@pytest.mark.parametrize("nth", [1, 7, 40])
+def test_injected_copy_failure_is_recoverable(nth):
+    """A host<->device copy of a streamed forward fails part-way: the call
+    reports CQSA_ERR_CUDA, the work already enqueued completes, and the next
+    forward on the same plan is correct."""
+    N, H, d = 13 * 256, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=61, host=True)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=False, mem_budget_bytes=int(_min_budget(N, H, d, [4], False) * 1.3))
+    out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lse = torch.empty(H, N).pin_memory()
+    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, nth)
+    try:
+        with pytest.raises(cqsa.CqsaError) as ei:
+            cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_HOST)
+        assert ei.value.status == cqsa.CQSA_ERR_CUDA
+    finally:
+        cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, 0)
+    plan.sync()
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), False)

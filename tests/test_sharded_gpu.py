@@ -166,3 +166,47 @@ def test_forward_sharded_over_nccl_one_rank():
             check(out, lse, q, k, v, np.arange(N), causal)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 128), (torch.bfloat16, 64), (torch.bfloat16, 128)])
+def test_exchange_kernels_against_oracle_merge(dtype, d):
+    """cqsa_partial_rescale / cqsa_partial_finish on random partials of 4
+    ranks (lse in [-6, 6], some rows -inf on some ranks, one row on none)
+    against the oracle's fp64 log-sum-exp merge."""
+    from oracle import cqs_ref
+    N, H, R = 7 * 40, 2, 4
+    g = torch.Generator(device="cpu").manual_seed(70 + d)
+    cdt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], dtype=cdt)
+    o = [torch.randn(N, H, d, generator=g) for _ in range(R)]
+    l = [torch.rand(H, N, generator=g) * 12 - 6 for _ in range(R)]
+    for r in range(R):
+        miss = torch.rand(H, N, generator=g) < 0.3
+        l[r][miss] = -float("inf")
+        o[r][miss.T] = 0.0
+    l[0][:, 5] = 3.0                                   # row 5 seen by rank 0 only
+    for r in range(1, R):
+        l[r][:, 5] = -float("inf")
+        o[r][5] = 0.0
+    for r in range(R):
+        l[r][:, 7] = -float("inf")                     # row 7 seen by no rank
+        o[r][7] = 0.0
+    ref_o, ref_l = cqs_ref.lse_merge([x.numpy() for x in o], [x.numpy().T for x in l])
+    od = [x.to(DEV) for x in o]
+    ld = [x.to(DEV) for x in l]
+    lse_max = torch.stack(ld).amax(0)
+    ws = []
+    for r in range(R):
+        w = torch.empty_like(ld[r])
+        cqsa.cqsa_partial_rescale(plan, od[r], ld[r], lse_max, w)
+        ws.append(w)
+    out = torch.empty(N, H, d, device=DEV, dtype=dtype)
+    lse = torch.empty(H, N, device=DEV)
+    cqsa.cqsa_partial_finish(plan, torch.stack(od).sum(0), torch.stack(ws).sum(0), lse_max, out, lse)
+    plan.sync()
+    got_o, got_l = out.float().cpu().double().numpy(), lse.cpu().double().numpy().T
+    seen = np.isfinite(ref_l)
+    assert np.all(np.isneginf(got_l[~seen])) and np.all(got_o[~seen] == 0)
+    tol = 1e-5 if dtype == torch.float32 else 2e-2
+    assert np.abs(got_o - ref_o).max() <= tol * max(1.0, np.abs(ref_o).max())
+    assert np.abs(got_l[seen] - ref_l[seen]).max() <= 1e-5
