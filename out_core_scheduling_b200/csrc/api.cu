@@ -16,6 +16,7 @@
 // back, so copies of task i+1 and i-1 overlap the compute of task i.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -48,6 +49,27 @@ bool injected(std::atomic<int64_t> &c) {
         if (c.compare_exchange_weak(v, v - 1)) return v == 1;
     return false;
 }
+
+// NVTX range around a host-side step, for timeline profilers; a few
+// instructions when no tool is attached.  payload >= 0 is attached as an
+// integer (the task index of a streamed forward).
+struct NvtxRange {
+    explicit NvtxRange(const char *name, int64_t payload = -1) {
+        nvtxEventAttributes_t a{};
+        a.version = NVTX_VERSION;
+        a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+        a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+        a.message.ascii = name;
+        if (payload >= 0) {
+            a.payloadType = NVTX_PAYLOAD_TYPE_INT64;
+            a.payload.llValue = payload;
+        }
+        nvtxRangePushEx(&a);
+    }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 cudaError_t lib_malloc(void **ptr, size_t bytes) {
     if (injected(g_fail_alloc)) return cudaErrorMemoryAllocation;
@@ -682,6 +704,7 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     const size_t blk_stride = (size_t)B;  // pool rows per slot
     for (int h0 = 0; h0 < H; h0 += g) {
         for (size_t t = 0; t < P->leaves.size(); ++t, ++it) {
+            NvtxRange nvtx_task("cqsa streamed task", (int64_t)t);
             const LeafState &L = P->leaves[t];
             const int s = (int)(it & 1);
             // -- H2D of the blocks this task misses in the device block cache.
@@ -879,6 +902,7 @@ cqsa_status_t cqsa_plan(int64_t N, int H, int d, int l, int levels, int causal, 
 
 cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, void *out, float *lse,
                            int host_or_device, void *stream) {
+    NvtxRange nvtx(host_or_device == CQSA_HOST ? "cqsa_forward (host)" : "cqsa_forward (device)");
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (host_or_device != CQSA_DEVICE && host_or_device != CQSA_HOST)
         return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be CQSA_DEVICE or CQSA_HOST");
@@ -915,6 +939,7 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
 cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, const void *out,
                             const float *lse, const void *dout, void *dq, void *dk, void *dv, int host_or_device,
                             void *stream) {
+    NvtxRange nvtx("cqsa_backward");
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (host_or_device == CQSA_HOST)
         return fail(CQSA_ERR_UNSUPPORTED, "the backward runs in device mode only");
@@ -942,6 +967,7 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
 
 cqsa_status_t cqsa_forward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
                                    float *o_part, float *lse_part, void *stream) {
+    NvtxRange nvtx("cqsa_forward_partial");
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     cqsa_status_t st = check_device(plan);
     if (st != CQSA_OK) return st;
