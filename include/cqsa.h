@@ -253,6 +253,26 @@ cqsa_status_t cqsa_partial_rescale(cqsa_plan_t *plan, float *o_part, const float
 cqsa_status_t cqsa_partial_finish(cqsa_plan_t *plan, const float *o_sum, const float *w_sum,
                                   const float *lse_max, void *out, float *lse, void *stream);
 
+/* cqsa_backward_partial -- this rank's part of the backward of a sharded
+ * plan (any plan: with one rank it is the whole backward).  Every allowed
+ * pair's gradient terms depend only on the pair and the row statistics
+ * (see cqsa_backward), so each rank sums the terms of its own entries and
+ * one all-reduce SUM over ranks gives the gradients:
+ *   q, k, v, out, lse, dout as for cqsa_backward (out and lse the full
+ *   forward's, e.g. from the sharded exchange, on every rank);
+ *   dq_part fp32 [N, H, d], dk_part, dv_part fp32 [N, H_kv, d]: this rank's
+ *   sums (0 where it has no pair).  Device buffers owned by the caller.
+ * The first call allocates the rank's backward arena.  Asynchronous on
+ * stream.  Errors: INVALID_ARG, CUDA, NO_DEVICE. */
+cqsa_status_t cqsa_backward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
+                                    const void *out, const float *lse, const void *dout, float *dq_part,
+                                    float *dk_part, float *dv_part, void *stream);
+
+/* cqsa_partial_cast -- count fp32 values (e.g. all-reduced gradient sums) to
+ * the plan dtype, rounded to nearest even.  Device buffers; asynchronous on
+ * stream.  Errors: INVALID_ARG, CUDA. */
+cqsa_status_t cqsa_partial_cast(cqsa_plan_t *plan, const float *src, void *dst, int64_t count, void *stream);
+
 /* cqsa_plan_sync -- wait for the plan's work on `stream` and report any
  * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync. */
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream);

@@ -41,7 +41,7 @@ EXPORTS = (
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
-    "cqsa_debug_inject",
+    "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast",
 )
 
 
@@ -133,6 +133,8 @@ def load_library():
         "cqsa_partial_rescale": (st, [P, P, P, P, P, P]),
         "cqsa_partial_finish": (st, [P, P, P, P, P, P, P]),
         "cqsa_debug_inject": (st, [ctypes.c_int, ctypes.c_int64]),
+        "cqsa_backward_partial": (st, [P, P, P, P, P, P, P, P, P, P, P]),
+        "cqsa_partial_cast": (st, [P, P, P, ctypes.c_int64, P]),
         "cqsa_plan_destroy": (None, [P]),
         "cqsa_last_error": (ctypes.c_char_p, []),
     }
@@ -347,6 +349,35 @@ def cqsa_partial_finish(plan: Plan, o_sum, w_sum, lse_max, out, lse, stream=None
     _check(load_library().cqsa_partial_finish(plan.handle, o_sum.data_ptr(), w_sum.data_ptr(),
                                               lse_max.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_backward_partial(plan: Plan, q, k, v, out, lse, dout, dq_part, dk_part, dv_part, stream=None):
+    """This rank's sums of the gradient terms of a sharded plan: dq_part fp32
+    [N, H, d], dk_part / dv_part fp32 [N, H_kv, d] (out, lse: the full
+    forward's).  An all-reduce SUM over ranks gives the gradients."""
+    import torch
+    _check_shapes(plan, (("q", q), ("out", out), ("dout", dout)), (("k", k), ("v", v)), lse)
+    info = plan.info()
+    lead = (info["B"],) if info["B"] > 1 else ()
+    for name, t, heads in (("dq_part", dq_part, info["H"]), ("dk_part", dk_part, info["H_kv"]),
+                           ("dv_part", dv_part, info["H_kv"])):
+        want = (info["N"], heads, info["d"])
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_contiguous()
+                or tuple(t.shape) not in (lead + want, (1,) + want)):
+            raise ValueError(f"{name} must be a contiguous float32 tensor of shape {lead + want}")
+    _check(load_library().cqsa_backward_partial(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                                                dq_part.data_ptr(), dk_part.data_ptr(), dv_part.data_ptr(),
+                                                ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_partial_cast(plan: Plan, src, dst, stream=None):
+    """dst (plan dtype) = src (fp32), same number of elements, contiguous."""
+    import torch
+    if src.dtype != torch.float32 or src.numel() != dst.numel() or not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("src must be contiguous float32 with as many elements as the contiguous dst")
+    _check(load_library().cqsa_partial_cast(plan.handle, src.data_ptr(), dst.data_ptr(), src.numel(),
+                                            ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def cqsa_debug_inject(kind: int, nth: int):

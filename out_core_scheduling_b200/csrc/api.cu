@@ -171,6 +171,18 @@ std::vector<char> pack_wl(const WorkList &wl) {
     return buf;
 }
 
+// Backward of a plan: D, partial-gradient slots, work lists (one for the
+// plan's own backward, one for this rank's share of a sharded plan).
+struct BwdState {
+    char *arena = nullptr;
+    size_t bytes = 0;
+    int *err = nullptr;
+    float *delta = nullptr, *dq = nullptr, *dk = nullptr, *dv = nullptr;
+    int32_t *q_nslots = nullptr, *kv_nslots = nullptr;
+    DevWl qwl, kvwl;
+    bool fused = false;
+};
+
 struct LeafState {
     DevWl wl;
     std::vector<MergeSeg> host_segs;  // query blocks of the task; SEG_LAST ones are copied out after it
@@ -194,13 +206,9 @@ struct cqsa_plan {
     int32_t *dev_nslots = nullptr;
     DevWl dev_wl;
 
-    // Backward (device mode): D, partial-gradient slots, work lists.
-    char *bwd_arena = nullptr;
-    size_t bwd_bytes = 0;
-    int *bwd_err = nullptr;
-    float *bwd_delta = nullptr, *bwd_dq = nullptr, *bwd_dk = nullptr, *bwd_dv = nullptr;
-    int32_t *bwd_q_nslots = nullptr, *bwd_kv_nslots = nullptr;
-    DevWl bwd_qwl, bwd_kvwl;
+    // Backward (device mode): the plan's own, and this rank's share of a
+    // sharded plan (cqsa_backward_partial).
+    BwdState bwd, bwd_shard;
 
     // Sharded forward (cqsa_forward_partial): this rank's work list.
     char *part_arena = nullptr;
@@ -536,17 +544,28 @@ cqsa_status_t forward_partial_device(cqsa_plan_t *P, const void *q, const void *
     return CQSA_OK;
 }
 
-cqsa_status_t setup_backward(cqsa_plan_t *P) {
-    if (P->bwd_arena) return CQSA_OK;
+cqsa_status_t setup_backward(cqsa_plan_t *P, BwdState &B, bool shard) {
+    if (B.arena) return CQSA_OK;
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
-    const bool fused = pl.spec.fused != 0;
+    const bool fused = !shard && pl.spec.fused != 0;
     // bf16: tensor-core kernels on 128-row tiles; fp32: CUDA-core kernels on 64.
     const int rows = P->dtype == CQSA_BF16 ? 128 : 64;
-    WorkList qwl = pl.device_worklist(rows, rows, H);
-    int64_t max_kv = 0;
-    WorkList kvwl = pl.device_worklist_kv(rows, rows, H, &max_kv);
+    std::vector<int32_t> q_ns;
+    int64_t max_q = 0, max_kv = 0;
+    WorkList qwl, kvwl;
+    if (shard) {
+        const std::vector<char> use = pl.shard_use();
+        qwl = pl.device_worklist_sel(rows, rows, H, use, &q_ns);
+        kvwl = pl.device_worklist_kv_sel(rows, rows, H, use, &max_kv);
+        for (int32_t v : q_ns) max_q = std::max<int64_t>(max_q, v);
+    } else {
+        qwl = pl.device_worklist(rows, rows, H);
+        kvwl = pl.device_worklist_kv(rows, rows, H, &max_kv);
+        q_ns = pl.slots_per_block;
+        max_q = pl.max_slots;
+    }
     // Key/value partial slots: per (task, key block) entry, and per query
     // head of a key/value group (grouped-query attention).
     const int kvg = pl.spec.kv_group(), Hkv = pl.spec.Hkv;
@@ -563,52 +582,54 @@ cqsa_status_t setup_backward(cqsa_plan_t *P) {
     const size_t o_delta = a.take((size_t)H * N * sizeof(float));
     size_t o_dq = 0, o_dk = 0, o_dv = 0, o_qns = 0, o_kvns = 0;
     if (!fused) {
-        o_dq = a.take((size_t)pl.max_slots * slot);
+        o_dq = a.take((size_t)std::max<int64_t>(1, max_q) * slot);
         o_qns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
     }
     if (kv_slots) {
-        o_dk = a.take((size_t)max_kv * kvg * kv_slot);
-        o_dv = a.take((size_t)max_kv * kvg * kv_slot);
+        o_dk = a.take((size_t)std::max<int64_t>(1, max_kv) * kvg * kv_slot);
+        o_dv = a.take((size_t)std::max<int64_t>(1, max_kv) * kvg * kv_slot);
         o_kvns = a.take((size_t)pl.num_blocks * sizeof(int32_t));
     }
     const size_t o_qwl = a.take(wl_region(qwl));
     const size_t o_kvwl = a.take(wl_region(kvwl));
     char *arena = nullptr;
     CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
-    P->bwd_arena = arena;
-    P->bwd_bytes = a.total;
+    B.arena = arena;
+    B.bytes = a.total;
+    B.fused = fused;
     CK(cudaMemset(arena, 0, 256));
-    P->bwd_err = reinterpret_cast<int *>(arena + o_err);
-    P->bwd_delta = reinterpret_cast<float *>(arena + o_delta);
+    B.err = reinterpret_cast<int *>(arena + o_err);
+    B.delta = reinterpret_cast<float *>(arena + o_delta);
     if (!fused) {
-        P->bwd_dq = reinterpret_cast<float *>(arena + o_dq);
-        P->bwd_q_nslots = reinterpret_cast<int32_t *>(arena + o_qns);
-        CK(cudaMemcpy(P->bwd_q_nslots, pl.slots_per_block.data(), pl.num_blocks * sizeof(int32_t),
-                      cudaMemcpyHostToDevice));
+        B.dq = reinterpret_cast<float *>(arena + o_dq);
+        B.q_nslots = reinterpret_cast<int32_t *>(arena + o_qns);
+        CK(cudaMemcpy(B.q_nslots, q_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
     }
     if (kv_slots) {
-        P->bwd_dk = reinterpret_cast<float *>(arena + o_dk);
-        P->bwd_dv = reinterpret_cast<float *>(arena + o_dv);
-        P->bwd_kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
-        CK(cudaMemcpy(P->bwd_kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
+        B.dk = reinterpret_cast<float *>(arena + o_dk);
+        B.dv = reinterpret_cast<float *>(arena + o_dv);
+        B.kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
+        CK(cudaMemcpy(B.kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
     }
     std::vector<char> b1 = pack_wl(qwl), b2 = pack_wl(kvwl);
     if (!b1.empty()) CK(cudaMemcpy(arena + o_qwl, b1.data(), b1.size(), cudaMemcpyHostToDevice));
     if (!b2.empty()) CK(cudaMemcpy(arena + o_kvwl, b2.data(), b2.size(), cudaMemcpyHostToDevice));
-    P->bwd_qwl = place_wl(arena + o_qwl, qwl);
-    P->bwd_kvwl = place_wl(arena + o_kvwl, kvwl);
+    B.qwl = place_wl(arena + o_qwl, qwl);
+    B.kvwl = place_wl(arena + o_kvwl, kvwl);
     return CQSA_OK;
 }
 
-cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, const void *v, const void *out,
-                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
-                              cudaStream_t stream) {
-    cqsa_status_t st = setup_backward(P);
+// out_elem: element bytes of dq, dk, dv (the plan's, or 4 for the fp32
+// partial sums of cqsa_backward_partial).
+cqsa_status_t backward_device(cqsa_plan_t *P, BwdState &B, bool shard, const void *q, const void *k, const void *v,
+                              const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              int out_elem, cudaStream_t stream) {
+    cqsa_status_t st = setup_backward(P, B, shard);
     if (st != CQSA_OK) return st;
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
-    const bool fused = pl.spec.fused != 0;
+    const bool fused = B.fused;
     CUtensorMap mq{}, mk{}, mv{}, mo{};
     if (P->dtype == CQSA_BF16) {
         if ((st = make_map(&mq, q, N, H, d)) != CQSA_OK) return st;
@@ -616,14 +637,14 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
         if ((st = make_map(&mv, v, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
         if ((st = make_map(&mo, dout, N, H, d)) != CQSA_OK) return st;
     }
-    CK(launch_bwd_delta(d, P->elem, out, dout, N, H, P->bwd_delta, stream));
+    CK(launch_bwd_delta(d, P->elem, out, dout, N, H, B.delta, stream));
     BwdParams bp{};
     bp.q = q;
     bp.k = k;
     bp.v = v;
     bp.dout = dout;
     bp.lse = lse;
-    bp.delta = P->bwd_delta;
+    bp.delta = B.delta;
     bp.N = N;
     bp.H = H;
     bp.Hkv = pl.spec.Hkv;
@@ -632,41 +653,41 @@ cqsa_status_t backward_device(cqsa_plan_t *P, const void *q, const void *k, cons
     bp.scale = 1.0f / std::sqrt((float)d);
     {
         BwdParams p = bp;
-        p.entries = P->bwd_qwl.entries;
-        p.runs = P->bwd_qwl.runs;
-        p.units = P->bwd_qwl.units;
-        p.part_a = P->bwd_dq;
+        p.entries = B.qwl.entries;
+        p.runs = B.qwl.runs;
+        p.units = B.qwl.units;
+        p.part_a = B.dq;
         p.out_a = dq;
         LaunchTimer tm(P, stream, 2);
         if (P->dtype == CQSA_BF16)
-            CK(launch_bwd_dq_tc(d, mq, mk, mv, mo, p, P->bwd_qwl.num_units, P->timeout_ns, P->bwd_err, stream));
+            CK(launch_bwd_dq_tc(d, mq, mk, mv, mo, p, B.qwl.num_units, P->timeout_ns, B.err, stream));
         else
-            CK(launch_bwd_dq(d, P->elem, p, P->bwd_qwl.num_units, stream));
+            CK(launch_bwd_dq(d, P->elem, p, B.qwl.num_units, stream));
         tm.stop();
     }
     {
         BwdParams p = bp;
-        p.entries = P->bwd_kvwl.entries;
-        p.runs = P->bwd_kvwl.runs;
-        p.units = P->bwd_kvwl.units;
-        p.part_a = P->bwd_dk;
-        p.part_b = P->bwd_dv;
+        p.entries = B.kvwl.entries;
+        p.runs = B.kvwl.runs;
+        p.units = B.kvwl.units;
+        p.part_a = B.dk;
+        p.part_b = B.dv;
         p.out_a = dk;
         p.out_b = dv;
         LaunchTimer tm(P, stream, 2);
         if (P->dtype == CQSA_BF16)
-            CK(launch_bwd_dkdv_tc(d, mq, mk, mv, mo, p, P->bwd_kvwl.num_units, P->timeout_ns, P->bwd_err,
+            CK(launch_bwd_dkdv_tc(d, mq, mk, mv, mo, p, B.kvwl.num_units, P->timeout_ns, B.err,
                                   stream));
         else
-            CK(launch_bwd_dkdv(d, P->elem, p, P->bwd_kvwl.num_units, stream));
+            CK(launch_bwd_dkdv(d, P->elem, p, B.kvwl.num_units, stream));
         tm.stop();
     }
-    if (!fused || P->bwd_dk) {
+    if (!fused || B.dk) {
         LaunchTimer tm(P, stream, 1);
-        if (!fused) CK(launch_sum_slots(d, P->elem, P->bwd_dq, P->bwd_q_nslots, pl.block, N, H, dq, stream));
-        if (P->bwd_dk) {
-            CK(launch_sum_slots(d, P->elem, P->bwd_dk, P->bwd_kv_nslots, pl.block, N, pl.spec.Hkv, dk, stream));
-            CK(launch_sum_slots(d, P->elem, P->bwd_dv, P->bwd_kv_nslots, pl.block, N, pl.spec.Hkv, dv, stream));
+        if (!fused) CK(launch_sum_slots(d, out_elem, B.dq, B.q_nslots, pl.block, N, H, dq, stream));
+        if (B.dk) {
+            CK(launch_sum_slots(d, out_elem, B.dk, B.kv_nslots, pl.block, N, pl.spec.Hkv, dk, stream));
+            CK(launch_sum_slots(d, out_elem, B.dv, B.kv_nslots, pl.block, N, pl.spec.Hkv, dv, stream));
         }
         tm.stop();
     }
@@ -936,6 +957,42 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k, cons
     return CQSA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// The backward over B sequences: the plan's own (gradients in the plan
+// dtype) or this rank's share of a sharded plan (fp32 partial sums).
+cqsa_status_t backward_call(cqsa_plan_t *plan, bool shard, const void *q, const void *k, const void *v,
+                            const void *out, const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                            void *stream) {
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+    const char *names[] = {"q", "k", "v", "out", "lse", "dout", "dq", "dk", "dv"};
+    for (int i = 0; i < 9; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    const Planner &pl = plan->pl;
+    const int out_elem = shard ? 4 : plan->elem;
+    const size_t e = (size_t)plan->elem, N = (size_t)pl.spec.N, d = (size_t)pl.spec.d;
+    const size_t qs = N * pl.spec.H * d * e, kvs = N * pl.spec.Hkv * d * e, ls = N * pl.spec.H;
+    const size_t gqs = N * pl.spec.H * d * out_elem, gkvs = N * pl.spec.Hkv * d * out_elem;
+    BwdState &B = shard ? plan->bwd_shard : plan->bwd;
+    for (int b = 0; b < pl.spec.B; ++b) {
+        auto at = [&](const void *p, size_t stride) { return static_cast<const char *>(p) + b * stride; };
+        auto atw = [&](void *p, size_t stride) { return static_cast<char *>(p) + b * stride; };
+        st = backward_device(plan, B, shard, at(q, qs), at(k, kvs), at(v, kvs), at(out, qs), lse + b * ls,
+                             at(dout, qs), atw(dq, gqs), atw(dk, gkvs), atw(dv, gkvs), out_elem,
+                             static_cast<cudaStream_t>(stream));
+        if (st != CQSA_OK) return st;
+    }
+    return CQSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v, const void *out,
                             const float *lse, const void *dout, void *dq, void *dk, void *dv, int host_or_device,
                             void *stream) {
@@ -945,23 +1002,27 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
         return fail(CQSA_ERR_UNSUPPORTED, "the backward runs in device mode only");
     if (host_or_device != CQSA_DEVICE) return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be 0 or 1");
     if (plan->pl.spec.shard_count > 1)
-        return fail(CQSA_ERR_UNSUPPORTED, "the backward of a sharded plan is not supported");
+        return fail(CQSA_ERR_UNSUPPORTED, "a sharded plan runs cqsa_backward_partial (shard_count = %d)",
+                    plan->pl.spec.shard_count);
+    return backward_call(plan, false, q, k, v, out, lse, dout, dq, dk, dv, stream);
+}
+
+cqsa_status_t cqsa_backward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
+                                    const void *out, const float *lse, const void *dout, float *dq_part,
+                                    float *dk_part, float *dv_part, void *stream) {
+    NvtxRange nvtx("cqsa_backward_partial");
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    return backward_call(plan, true, q, k, v, out, lse, dout, dq_part, dk_part, dv_part, stream);
+}
+
+cqsa_status_t cqsa_partial_cast(cqsa_plan_t *plan, const float *src, void *dst, int64_t count, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    if (count < 0) return fail(CQSA_ERR_INVALID_ARG, "count must be >= 0");
+    if (count == 0) return CQSA_OK;
     cqsa_status_t st = check_device(plan);
     if (st != CQSA_OK) return st;
-    const void *ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
-    const char *names[] = {"q", "k", "v", "out", "lse", "dout", "dq", "dk", "dv"};
-    for (int i = 0; i < 9; ++i)
-        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
-    const Planner &pl = plan->pl;
-    const size_t e = (size_t)plan->elem, N = (size_t)pl.spec.N, d = (size_t)pl.spec.d;
-    const size_t qs = N * pl.spec.H * d * e, kvs = N * pl.spec.Hkv * d * e, ls = N * pl.spec.H;
-    for (int b = 0; b < pl.spec.B; ++b) {
-        auto at = [&](const void *p, size_t stride) { return static_cast<const char *>(p) + b * stride; };
-        auto atw = [&](void *p, size_t stride) { return static_cast<char *>(p) + b * stride; };
-        st = backward_device(plan, at(q, qs), at(k, kvs), at(v, kvs), at(out, qs), lse + b * ls, at(dout, qs),
-                             atw(dq, qs), atw(dk, kvs), atw(dv, kvs), static_cast<cudaStream_t>(stream));
-        if (st != CQSA_OK) return st;
-    }
+    if ((st = check_ptr(src, false, "src")) != CQSA_OK || (st = check_ptr(dst, false, "dst")) != CQSA_OK) return st;
+    CK(launch_cast_out(plan->elem, src, dst, count, static_cast<cudaStream_t>(stream)));
     return CQSA_OK;
 }
 
@@ -1032,7 +1093,7 @@ cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
     CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-    int *words[4] = {plan->dev_err, plan->h_err, plan->bwd_err, plan->part_err};
+    int *words[5] = {plan->dev_err, plan->h_err, plan->bwd.err, plan->bwd_shard.err, plan->part_err};
     int bad = 0;
     for (int *w : words) {
         if (!w) continue;
@@ -1189,7 +1250,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
         cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);
-        if (plan->dev_arena || plan->bwd_arena || plan->part_arena) cudaDeviceSynchronize();
+        if (plan->dev_arena || plan->bwd.arena || plan->bwd_shard.arena || plan->part_arena) cudaDeviceSynchronize();
         for (int s = 0; s < 2; ++s) {
             if (plan->ev_in_ready[s]) cudaEventDestroy(plan->ev_in_ready[s]);
             if (plan->ev_in_free[s]) cudaEventDestroy(plan->ev_in_free[s]);
@@ -1208,7 +1269,8 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
             if (s) cudaStreamDestroy(s);
         if (plan->dev_arena) cudaFree(plan->dev_arena);
         if (plan->host_arena) cudaFree(plan->host_arena);
-        if (plan->bwd_arena) cudaFree(plan->bwd_arena);
+        if (plan->bwd.arena) cudaFree(plan->bwd.arena);
+        if (plan->bwd_shard.arena) cudaFree(plan->bwd_shard.arena);
         if (plan->part_arena) cudaFree(plan->part_arena);
         cudaGetLastError();
     }

@@ -119,6 +119,7 @@ cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const
 cudaError_t launch_partial_init(float *o, int64_t n, float *lse, int64_t nl, cudaStream_t stream);
 cudaError_t launch_partial_rescale(int d, float *o, const float *lse_part, const float *lse_max, float *w,
                                    int64_t N, int H, cudaStream_t stream);
+cudaError_t launch_cast_out(int elem_bytes, const float *src, void *dst, int64_t n, cudaStream_t stream);
 cudaError_t launch_partial_finish(int d, int elem_bytes, const float *o_sum, const float *w_sum,
                                   const float *lse_max, void *out, float *lse, int64_t N, int H,
                                   cudaStream_t stream);

@@ -91,7 +91,26 @@ __global__ void partial_finish_kernel(const float *o_sum, const float *w_sum, co
     }
 }
 
+template <typename T>
+__global__ void cast_out_kernel(const float *src, T *dst, int64_t n) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) store_out(dst + i, src[i]);
+}
+
 }  // namespace
+
+// fp32 values (the all-reduced gradient sums of a sharded backward) to the
+// plan dtype, rounded to nearest even.
+cudaError_t launch_cast_out(int elem_bytes, const float *src, void *dst, int64_t n, cudaStream_t stream) {
+    if (elem_bytes == 2)
+        cast_out_kernel<__nv_bfloat16><<<grid_for(n, kThreads), kThreads, 0, stream>>>(
+            src, static_cast<__nv_bfloat16 *>(dst), n);
+    else if (elem_bytes == 4)
+        cast_out_kernel<float><<<grid_for(n, kThreads), kThreads, 0, stream>>>(src, static_cast<float *>(dst), n);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
 
 cudaError_t launch_partial_init(float *o, int64_t n, float *lse, int64_t nl, cudaStream_t stream) {
     if (n % 4 != 0) return cudaErrorInvalidValue;

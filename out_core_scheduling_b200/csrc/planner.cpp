@@ -401,15 +401,62 @@ WorkList Planner::device_worklist(int rows_per_unit, int bn, int heads) const {
     return wl;
 }
 
+std::vector<char> Planner::shard_use() const {
+    std::vector<char> use(entries.size());
+    for (size_t i = 0; i < entries.size(); ++i) use[i] = entry_rank[i] == spec.shard_rank;
+    return use;
+}
+
 WorkList Planner::device_worklist_kv(int rows_per_unit, int bn, int heads, int64_t *max_kv_slots) const {
+    return kv_worklist(rows_per_unit, bn, heads, std::vector<char>(entries.size(), 1), spec.fused != 0,
+                       max_kv_slots);
+}
+
+WorkList Planner::device_worklist_kv_sel(int rows_per_unit, int bn, int heads, const std::vector<char> &use,
+                                         int64_t *max_kv_slots) const {
+    return kv_worklist(rows_per_unit, bn, heads, use, false, max_kv_slots);
+}
+
+WorkList Planner::device_worklist_sel(int rows_per_unit, int bn, int heads, const std::vector<char> &use,
+                                      std::vector<int32_t> *nslots) const {
+    WorkList wl;
+    std::vector<int64_t> group;
+    nslots->assign(num_blocks, 0);
+    for (size_t i = 0; i < entries.size(); ++i) {
+        if (!use[i]) continue;
+        const Entry &e = entries[i];
+        group.push_back(e.task);
+        WlEntry w{};
+        w.q_lo = (int32_t)(e.qb * block);
+        w.q_hi = (int32_t)block_end(e.qb);
+        w.slot = (*nslots)[e.qb]++;
+        w.out_lo = w.q_lo;
+        w.run_begin = (int32_t)wl.runs.size();
+        w.run_count = (int32_t)e.runs.size();
+        for (const KeyRun &r : e.runs) {
+            WlRun x{};
+            x.k_lo = (int32_t)(r.b0 * block);
+            x.k_hi = (int32_t)block_end(r.b1);
+            wl.runs.push_back(x);
+        }
+        wl.entries.push_back(w);
+    }
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, group);
+    return wl;
+}
+
+WorkList Planner::kv_worklist(int rows_per_unit, int bn, int heads, const std::vector<char> &use, bool fused,
+                              int64_t *max_kv_slots) const {
     // kb -> (task, query blocks) in task order; pairs come from the forward
     // entries, whose key runs already carry every level's CQS mask.
     std::vector<std::vector<std::pair<int64_t, std::vector<int64_t>>>> by_kb(num_blocks);
-    for (const Entry &e : entries)
+    for (size_t i = 0; i < entries.size(); ++i) {
+        if (!use[i]) continue;
+        const Entry &e = entries[i];
         for (const KeyRun &r : e.runs)
             for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
                 auto &lst = by_kb[kb];
-                if (spec.fused) {
+                if (fused) {
                     if (lst.empty()) lst.push_back({0, {}});
                     lst.back().second.push_back(e.qb);
                 } else {
@@ -417,6 +464,7 @@ WorkList Planner::device_worklist_kv(int rows_per_unit, int bn, int heads, int64
                     lst.back().second.push_back(e.qb);
                 }
             }
+    }
     WorkList wl;
     std::vector<int64_t> group;
     *max_kv_slots = 0;
@@ -430,7 +478,7 @@ WorkList Planner::device_worklist_kv(int rows_per_unit, int bn, int heads, int64
             w.q_hi = (int32_t)block_end(kb);
             w.slot = slot++;
             w.out_lo = w.q_lo;
-            w.flags = spec.fused ? (SEG_FIRST | SEG_LAST) : 0;
+            w.flags = fused ? (SEG_FIRST | SEG_LAST) : 0;
             w.run_begin = (int32_t)wl.runs.size();
             for (size_t i = 0; i < qs.size(); ++i) {
                 if (i > 0 && qs[i] == qs[i - 1] + 1) {

@@ -153,6 +153,15 @@ public:
     // kv_slot of each entry numbers the tasks of a key block (partial slots);
     // *max_kv_slots gets the most any block has.
     WorkList device_worklist_kv(int rows_per_unit, int bn, int heads, int64_t *max_kv_slots) const;
+    // The same two lists (partial slots, never fused) over only the entries
+    // `use` selects, e.g. this rank's of a sharded plan: query-block slots
+    // are renumbered among them, *nslots gets their count per block.
+    WorkList device_worklist_sel(int rows_per_unit, int bn, int heads, const std::vector<char> &use,
+                                 std::vector<int32_t> *nslots) const;
+    WorkList device_worklist_kv_sel(int rows_per_unit, int bn, int heads, const std::vector<char> &use,
+                                    int64_t *max_kv_slots) const;
+    // Entries of this rank (all entries when the plan is not sharded).
+    std::vector<char> shard_use() const;
     // Work list of leaf t reading Q, K, V from the block pools of `pool`.
     WorkList leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const;
     // Merge segments of leaf t in host mode (one per query block with an
@@ -167,6 +176,8 @@ private:
     // selects, as maximal runs.
     WorkList union_worklist(const std::vector<char> &use, int32_t flags, int rows_per_unit, int bn,
                             int heads) const;
+    WorkList kv_worklist(int rows_per_unit, int bn, int heads, const std::vector<char> &use, bool fused,
+                         int64_t *max_kv_slots) const;
     void assign_shards();
 
 public:

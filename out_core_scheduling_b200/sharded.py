@@ -18,6 +18,7 @@ The collectives go through torch.distributed (NCCL for CUDA tensors); all
 arithmetic runs in the library's kernels.  ``ops`` replaces the three
 library calls (tests on CPU ranks pass a host implementation); the default
 is the CUDA library, which fails loudly when it is not built.
+``backward_sharded`` does the same for the gradients with one all-reduce SUM.
 """
 from __future__ import annotations
 
@@ -25,10 +26,12 @@ from . import cqsa
 
 
 class LibraryOps:
-    """The library's kernels for the three per-rank steps."""
+    """The library's kernels for the per-rank steps."""
     forward_partial = staticmethod(cqsa.cqsa_forward_partial)
     partial_rescale = staticmethod(cqsa.cqsa_partial_rescale)
     partial_finish = staticmethod(cqsa.cqsa_partial_finish)
+    backward_partial = staticmethod(cqsa.cqsa_backward_partial)
+    partial_cast = staticmethod(cqsa.cqsa_partial_cast)
 
 
 def forward_sharded(plan, q, k, v, out, lse, group=None, ops=None):
@@ -60,3 +63,34 @@ def forward_sharded(plan, q, k, v, out, lse, group=None, ops=None):
     ops.partial_rescale(plan, o_part, lse_part, lse_max, w)
     dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
     ops.partial_finish(plan, o_part, w, lse_max, out, lse)
+
+
+def backward_sharded(plan, q, k, v, out, lse, dout, dq, dk, dv, group=None, ops=None):
+    """dq, dk, dv of the full attention on every rank of ``group``.
+
+    Tensors as for ``cqsa_backward``; out and lse are the full forward's
+    (``forward_sharded`` leaves them on every rank).  Each rank sums the
+    gradient terms of its own entries in fp32 (every allowed pair's terms
+    depend only on the pair and the row statistics), one all-reduce SUM over
+    [dq | dk | dv] adds the ranks' sums, and the library casts them to the
+    plan dtype.  Moves N * (H + 2 H_kv) * d fp32 values per rank."""
+    import torch
+    import torch.distributed as dist
+
+    ops = ops or LibraryOps
+    info = plan.info()
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if info["shard_count"] != world or info["shard_rank"] != rank:
+        raise ValueError(f"plan is shard {info['shard_rank']} of {info['shard_count']}, "
+                         f"but this is rank {rank} of {world}")
+    nq, nk = dq.numel(), dk.numel()
+    buf = torch.empty(nq + 2 * nk, dtype=torch.float32, device=dq.device)
+    gq = buf[:nq].view(dq.shape)
+    gk = buf[nq:nq + nk].view(dk.shape)
+    gv = buf[nq + nk:].view(dv.shape)
+    ops.backward_partial(plan, q, k, v, out, lse, dout, gq, gk, gv)
+    dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
+    ops.partial_cast(plan, gq, dq)
+    ops.partial_cast(plan, gk, dk)
+    ops.partial_cast(plan, gv, dv)

@@ -130,6 +130,40 @@ class HostOps:
         lse.copy_(torch.from_numpy(lse_max.double().numpy() + np.log(W)).float())
 
 
+def _host_backward_partial(plan, q, k, v, out, lse, dout, dq_part, dk_part, dv_part):
+    """fp64 sums of the gradient terms of this rank's entries, from the
+    plan's entry list (P from the full lse, dS = P (dP - D))."""
+    import torch
+    info = plan.info()
+    N, H, d, blk, causal = info["N"], info["H"], info["d"], info["block_tokens"], info["causal"]
+    qn, kn, vn, on, dn = (x.double().numpy() for x in (q, k, v, out, dout))
+    ln = lse.double().numpy()                                        # [H, N]
+    Dl = (dn * on).sum(-1)                                           # [N, H]
+    sc = 1.0 / np.sqrt(d)
+    gq, gk, gv = np.zeros((N, H, d)), np.zeros((N, H, d)), np.zeros((N, H, d))
+    for i in range(info["num_entries"]):
+        e = plan.entry(i)
+        if e["shard"] != info["shard_rank"]:
+            continue
+        rows = np.arange(e["q_block"] * blk, min((e["q_block"] + 1) * blk, N))
+        keys = np.concatenate([np.arange(b0 * blk, min((b1 + 1) * blk, N)) for b0, b1 in e["runs"]])
+        s = np.einsum("ihd,jhd->hij", qn[rows], kn[keys]) * sc
+        if causal:
+            s = np.where((keys[None, :] <= rows[:, None])[None], s, -np.inf)
+        P = np.exp(s - ln[:, rows][..., None])
+        dP = np.einsum("ihd,jhd->hij", dn[rows], vn[keys])
+        dS = P * (dP - Dl[rows].T[..., None])
+        gq[rows] += np.einsum("hij,jhd->ihd", dS, kn[keys]) * sc
+        gk[keys] += np.einsum("hij,ihd->jhd", dS, qn[rows]) * sc
+        gv[keys] += np.einsum("hij,ihd->jhd", P, dn[rows])
+    for t, g in ((dq_part, gq), (dk_part, gk), (dv_part, gv)):
+        t.copy_(torch.from_numpy(g).float())
+
+
+HostOps.backward_partial = staticmethod(_host_backward_partial)
+HostOps.partial_cast = staticmethod(lambda plan, src, dst: dst.copy_(src.to(dst.dtype)))
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -148,7 +182,7 @@ def _rank_main(rank, world, port, cfg, q):
     import oracle
     from out_core_scheduling_b200 import cqsa as lib
     from out_core_scheduling_b200.inputs import make_qkv
-    from out_core_scheduling_b200.sharded import forward_sharded
+    from out_core_scheduling_b200.sharded import backward_sharded, forward_sharded
     from test_sharded import HostOps
 
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -162,7 +196,15 @@ def _rank_main(rank, world, port, cfg, q):
         ref_o, ref_l = oracle.attention_rows(qt, kt, vt, causal=causal)
         e_o = float(np.abs(out.double().numpy() - ref_o).max())
         e_l = float(np.abs(lse.double().numpy().T - ref_l).max())
-        q.put((rank, e_o, e_l))
+        # The backward from the exchanged out and lse.
+        dout = make_qkv(N, H, d, dtype=torch.float32, seed=12)[0]
+        dq, dk, dv = (torch.empty(N, H, d) for _ in range(3))
+        backward_sharded(plan, qt, kt, vt, out, lse, dout, dq, dk, dv, ops=HostOps)
+        ref_dq, _, _ = oracle.attention_backward_dq(qt, kt, vt, dout, causal=causal)
+        ref_dk, ref_dv = oracle.attention_backward_dkdv(qt, kt, vt, dout, causal=causal)
+        e_g = max(float(np.abs(g.double().numpy() - r).max() / max(1.0, np.abs(r).max()))
+                  for g, r in ((dq, ref_dq), (dk, ref_dk), (dv, ref_dv)))
+        q.put((rank, e_o, e_l, e_g))
     finally:
         dist.destroy_process_group()
 
@@ -170,7 +212,8 @@ def _rank_main(rank, world, port, cfg, q):
 @pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("cfg", [CONFIGS[1], CONFIGS[3], CONFIGS[4]], ids=["l3-c", "l43-nc", "l43-ragged-c"])
 def test_forward_sharded_gloo(cfg, world):
-    """Every rank ends with the full attention (fp32 buffers: 1e-5)."""
+    """Every rank ends with the full attention (fp32 buffers: 1e-5) and,
+    after backward_sharded, the full gradients (1e-4 of the largest)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -181,8 +224,8 @@ def test_forward_sharded_gloo(cfg, world):
         p.join(300)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(world))
-    for rank, e_o, e_l in res:
-        assert e_o <= 1e-5 and e_l <= 1e-5, (rank, e_o, e_l)
+    for rank, e_o, e_l, e_g in res:
+        assert e_o <= 1e-5 and e_l <= 1e-5 and e_g <= 1e-4, (rank, e_o, e_l, e_g)
 
 
 def test_plan_rank_must_match_group():

@@ -210,3 +210,113 @@ def test_exchange_kernels_against_oracle_merge(dtype, d):
     tol = 1e-5 if dtype == torch.float32 else 2e-2
     assert np.abs(got_o - ref_o).max() <= tol * max(1.0, np.abs(ref_o).max())
     assert np.abs(got_l[seen] - ref_l[seen]).max() <= 1e-5
+
+
+# ------------------------------------------------------------------ backward
+def _grad_compare(got, ref, dtype, name):
+    """Same bar as the plain backward's parity tests."""
+    g = got.float().cpu().double().numpy()
+    gmax = np.abs(ref).max()
+    err = np.abs(g - ref)
+    if dtype == torch.float32:
+        assert err.max() <= 1e-4 * gmax + 1e-6, (name, err.max(), gmax)
+    else:
+        assert err.max() <= 2e-2 * gmax, (name, err.max(), gmax)
+        assert np.linalg.norm(g - ref) / np.linalg.norm(ref) <= 1e-2, name
+
+
+BWD_CASES = [
+    # (N, H, Hkv, d, levels, causal, dtype, G)
+    (7 * 128, 2, 0, 128, [3], False, torch.bfloat16, 2),
+    (7 * 128, 2, 0, 128, [3], True, torch.bfloat16, 3),
+    (13 * 64, 2, 0, 64, [4], True, torch.bfloat16, 8),
+    (1000, 2, 0, 128, [4], False, torch.bfloat16, 3),      # ragged N
+    (7 * 128, 4, 2, 128, [3], True, torch.bfloat16, 2),    # grouped-query
+    (700, 1, 0, 64, [3], True, torch.float32, 2),
+    (7 * 128, 2, 0, 128, [3], True, torch.bfloat16, 1),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: f"n{c[0]}-h{c[1]}-kv{c[2]}-d{c[3]}-{'c' if c[5] else 'nc'}-"
+                                                          f"{str(c[6])[6:]}-g{c[7]}")
+def test_sharded_backward_matches_oracle(case):
+    """Each emulated rank sums its entries' gradient terms
+    (cqsa_backward_partial), a torch sum stands in for the all-reduce, and
+    cqsa_partial_cast gives the gradients: against the fp64 oracle."""
+    import oracle
+    N, H, Hkv, d, ls, causal, dtype, G = case
+    Hk = Hkv or H
+    g = H // Hk
+    q = make_qkv(N, H, d, dtype=dtype, seed=80, device=DEV)[0]
+    _, k, v = make_qkv(N, Hk, d, dtype=dtype, seed=81, device=DEV)
+    dout = make_qkv(N, H, d, dtype=dtype, seed=82, device=DEV)[0]
+    cdt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    # The full forward's out and lse, as forward_sharded leaves them.
+    fplan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, H_kv=Hkv)
+    out, lse = run(fplan, q, k, v, cqsa.CQSA_DEVICE)
+    parts = []
+    for r in range(G):
+        p = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, H_kv=Hkv, shard_rank=r, shard_count=G)
+        gq = torch.empty(N, H, d, device=DEV)
+        gk = torch.empty(N, Hk, d, device=DEV)
+        gv = torch.empty(N, Hk, d, device=DEV)
+        cqsa.cqsa_backward_partial(p, q, k, v, out, lse, dout, gq, gk, gv)
+        p.sync()
+        parts.append((gq, gk, gv))
+    sums = [torch.stack([x[i] for x in parts]).sum(0) for i in range(3)]   # all-reduce SUM
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for src, dst in zip(sums, (dq, dk, dv)):
+        cqsa.cqsa_partial_cast(fplan, src, dst)
+    fplan.sync()
+    ke, ve = _expand(k, g), _expand(v, g)
+    qc, kc, vc, dc = (x.cpu() for x in (q, ke, ve, dout))
+    ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
+    ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, causal=causal)
+    _grad_compare(dq, ref_dq, dtype, "dq")
+    _grad_compare(dk, ref_dk.reshape(N, Hk, g, d).sum(2), dtype, "dk")
+    _grad_compare(dv, ref_dv.reshape(N, Hk, g, d).sum(2), dtype, "dv")
+
+
+def test_one_rank_backward_partial_is_the_backward():
+    N, H, d = 13 * 128, 2, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=83, device=DEV)
+    dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=84, device=DEV)[0]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    g = [torch.empty(N, H, d, device=DEV) for _ in range(3)]
+    cqsa.cqsa_backward_partial(plan, q, k, v, out, lse, dout, *g)
+    plan.sync()
+    for a, b in zip(g, (dq, dk, dv)):
+        # Same slot sums in fp32 against their bf16 rounding.
+        assert (a - b.float()).abs().max().item() <= 2 ** -8 * max(1.0, a.abs().max().item())
+
+
+def test_backward_sharded_over_nccl_one_rank():
+    import torch.distributed as dist
+    from out_core_scheduling_b200.sharded import backward_sharded, forward_sharded
+    import oracle
+    if dist.is_initialized():
+        pytest.skip("a process group is already initialised")
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device(DEV))
+    try:
+        N, H, d = 7 * 128, 2, 128
+        q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=85, device=DEV)
+        dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=86, device=DEV)[0]
+        plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True, shard_rank=0, shard_count=1)
+        out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+        forward_sharded(plan, q, k, v, out, lse)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        backward_sharded(plan, q, k, v, out, lse, dout, dq, dk, dv)
+        plan.sync()
+        qc, kc, vc, dc = (x.cpu() for x in (q, k, v, dout))
+        ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=True)
+        ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, causal=True)
+        _grad_compare(dq, ref_dq, torch.bfloat16, "dq")
+        _grad_compare(dk, ref_dk, torch.bfloat16, "dk")
+        _grad_compare(dv, ref_dv, torch.bfloat16, "dv")
+    finally:
+        dist.destroy_process_group()
