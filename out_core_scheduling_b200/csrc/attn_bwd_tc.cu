@@ -54,8 +54,10 @@ struct SmemDq {
     alignas(1024) uint8_t dout[KB][BOX_BYTES];
     alignas(1024) uint8_t k[KST][KB][BOX_BYTES];
     alignas(1024) uint8_t v[VST][KB][BOX_BYTES];
-    uint64_t bar_q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full, dp_free, p_half, p_full, o_full,
-        drain;
+    // s_ready[b]: S of a tile in TMEM buffer b (tiles b, b + 2, ...): a phase
+    // cannot run ahead of the elementwise warps, since S(j + 2) follows dQ(j).
+    uint64_t bar_q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_ready[2], dp_ready, dp_free, p_half,
+        p_full, o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -179,7 +181,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             mbar_init(&s.v_full[i], 1);
             mbar_init(&s.v_empty[i], 1);
         }
-        mbar_init(&s.s_full, 1);
+        mbar_init(&s.s_ready[0], 1);
+        mbar_init(&s.s_ready[1], 1);
+        mbar_init(&s.dp_ready, 1);
         mbar_init(&s.dp_free, EW_WARPS);
         mbar_init(&s.p_half, EW_WARPS);
         mbar_init(&s.p_full, EW_WARPS);
@@ -248,7 +252,8 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         // = dO V(j+1)^T goes into the dP columns as soon as they hold dP(j) in
         // registers.  dQ += dS(j) K(j) reads dS(j) in bf16 over S(j), in two
         // halves.  S(j+1) lands in the columns of dS(j-1), whose dQ MMAs were
-        // issued before it.
+        // issued before it.  S and dP have their own completion barriers, so
+        // the elementwise warps form P(j+1) while dP(j+1) is still running.
         bool ok = warp_wait_b(&s.bar_q, 0, abort, tmo);
         const uint64_t qdesc = smem_desc_sw128(smem_u32(s.q[0]), 16, 1024);
         const uint64_t odesc = smem_desc_sw128(smem_u32(s.dout[0]), 16, 1024);
@@ -257,9 +262,10 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             if (ok) {
                 tc_fence_after();
                 mma_rows_dot<D>(tmem, qdesc, smem_desc_sw128(smem_u32(s.k[0][0]), 16, 1024), IDESC_SS);
+                mma_commit_elect(&s.s_ready[0]);
                 mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[0][0]), 16, 1024), IDESC_SS);
                 mma_commit_elect(&s.v_empty[0]);
-                mma_commit_elect(&s.s_full);
+                mma_commit_elect(&s.dp_ready);
             }
         }
         for (int j = 0; j < ntiles && ok; ++j) {
@@ -269,6 +275,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 tc_fence_after();
                 mma_rows_dot<D>(tmem + s_col(j1), qdesc, smem_desc_sw128(smem_u32(s.k[j1 % KST][0]), 16, 1024),
                                 IDESC_SS);
+                mma_commit_elect(&s.s_ready[j1 & 1]);
                 if (!warp_wait_b(&s.v_full[j1 % VST], (uint32_t)(j1 / VST) & 1u, abort, tmo) ||
                     !warp_wait_b(&s.dp_free, (uint32_t)j & 1u, abort, tmo)) {
                     ok = false;
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 mma_rows_dot<D>(tmem + 128u, odesc, smem_desc_sw128(smem_u32(s.v[j1 % VST][0]), 16, 1024),
                                 IDESC_SS);
                 mma_commit_elect(&s.v_empty[j1 % VST]);
-                mma_commit_elect(&s.s_full);
+                mma_commit_elect(&s.dp_ready);
             }
             const uint64_t kb = smem_desc_sw128(smem_u32(s.k[j % KST][0]), BOX_BYTES, 1024);
             if (!warp_wait_b(&s.p_half, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
@@ -318,7 +325,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             int32_t lo, hi;
             clip_run(e, run, q_end, causal, &lo, &hi);
             for (int32_t ks = lo; ks < hi; ks += BN, ++j) {
-                if (!warp_wait_b(&s.s_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                // Phase A: P of this warp's 64 columns from S(j), as soon as
+                // S(j) is in (dP(j) may still be computing).
+                if (!warp_wait_b(&s.s_ready[j & 1], (uint32_t)(j >> 1) & 1u, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
                 int lim = min(BN, run.k_hi - ks);
                 if (causal) {
@@ -328,21 +337,31 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 if (!valid) lim = 0;
                 lim -= c0;  // in this warp's columns
                 const uint32_t sb = lane_base + s_col(j) + (uint32_t)c0;
-                // This warp's halves of dP(j) and S(j) into registers with one
-                // wait, so dP(j+1) can be computed into the dP columns while the
-                // tile finishes.
-                uint32_t dp[HALF / 32][32], sv[HALF / 32][32];
+                float pv[HALF / 32][32];
+                {
+                    uint32_t sv[HALF / 32][32];
 #pragma unroll
-                for (int cc = 0; cc < HALF / 32; ++cc) {
-                    tmem_ld32(lane_base + 128u + (uint32_t)(c0 + cc * 32), dp[cc]);
-                    tmem_ld32(sb + (uint32_t)(cc * 32), sv[cc]);
+                    for (int cc = 0; cc < HALF / 32; ++cc) tmem_ld32(sb + (uint32_t)(cc * 32), sv[cc]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < HALF / 32; ++cc) {
+                        fence_regs32(sv[cc]);
+#pragma unroll
+                        for (int t = 0; t < 32; ++t)
+                            pv[cc][t] = cc * 32 + t < lim ? ex2_approx(fmaf(__uint_as_float(sv[cc][t]), sl2, -lse2))
+                                                          : 0.f;
+                    }
                 }
+                // Phase B: dP(j) into registers (its columns then take
+                // dP(j+1)), dS = P (dP - D) in bf16 over S(j), in two halves.
+                if (!warp_wait_b(&s.dp_ready, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t dp[HALF / 32][32];
+#pragma unroll
+                for (int cc = 0; cc < HALF / 32; ++cc) tmem_ld32(lane_base + 128u + (uint32_t)(c0 + cc * 32), dp[cc]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < HALF / 32; ++cc) {
-                    fence_regs32(dp[cc]);
-                    fence_regs32(sv[cc]);
-                }
+                for (int cc = 0; cc < HALF / 32; ++cc) fence_regs32(dp[cc]);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.dp_free);
@@ -350,14 +369,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 for (int cc = 0; cc < HALF / 32; ++cc) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const int c = cc * 32 + t;
-                        const float p0 = c < lim ? ex2_approx(fmaf(__uint_as_float(sv[cc][t]), sl2, -lse2)) : 0.f;
-                        const float p1 =
-                            c + 1 < lim ? ex2_approx(fmaf(__uint_as_float(sv[cc][t + 1]), sl2, -lse2)) : 0.f;
-                        pk[t / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[cc][t]) - dl),
-                                                p1 * (__uint_as_float(dp[cc][t + 1]) - dl));
-                    }
+                    for (int t = 0; t < 32; t += 2)
+                        pk[t / 2] = pack_bf16x2(pv[cc][t] * (__uint_as_float(dp[cc][t]) - dl),
+                                                pv[cc][t + 1] * (__uint_as_float(dp[cc][t + 1]) - dl));
                     tmem_st16_b(sb + (uint32_t)(cc * 16), pk);
                     tmem_wait_st();
                     tc_fence_before();
