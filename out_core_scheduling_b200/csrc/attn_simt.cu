@@ -7,12 +7,17 @@
 // output and its log-sum-exp ("Stream-CQSA: Breaking the Billion-Token
 // Barrier on a Single GPU", section "Implementation", step 3).
 //
-// 256 threads as 16 x 16: thread (ty, tx) owns query rows 4ty..4ty+3 and key
-// columns tx + 16jj of each 64-key tile, and output columns tx + 16jj of d.
-// Row maxima and sums are reduced over the 16 threads of a row with warp
-// shuffles.
+// 256 threads as 16 x 16: thread (ty, tx) owns query rows 4ty..4ty+3, key
+// columns 4tx..4tx+3 of each 64-key tile, and output features
+// 64g + 4tx .. 64g + 4tx + 3 (g < d / 64).  Q, K and P are kept transposed in
+// shared memory ([feature or key][row], rows padded to 68 floats, 16-byte
+// aligned), so every step of both products reads one float4 per operand;
+// the tile's K and V are fetched with one vector load per four features,
+// all issued before any store.  Row maxima and sums are reduced over the 16
+// threads of a row with warp shuffles.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -24,23 +29,37 @@ namespace simt {
 constexpr int BM = 64;
 constexpr int BN = 64;
 constexpr int THREADS = 256;
+constexpr int LD = 68;  // padded row of the transposed tiles, in floats
 }  // namespace simt
 
-__device__ __forceinline__ float to_f32(float x) { return x; }
-__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+// Four consecutive elements as fp32 (16-byte fp32 or 8-byte bf16 load).
+__device__ __forceinline__ float4 load4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void f4_split(const float4 v, float (&a)[4]) {
+    a[0] = v.x;
+    a[1] = v.y;
+    a[2] = v.z;
+    a[3] = v.w;
+}
 
 template <int D, typename T>
 __global__ void __launch_bounds__(simt::THREADS)
     attn_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                      const AttnParams p) {
     using namespace simt;
-    constexpr int DP = D + 1;
-    constexpr int NJ = D / 16;
-    extern __shared__ float smf[];
-    float *Qs = smf;              // [BM][D+1]
-    float *Ks = Qs + BM * DP;     // [BN][D+1]
-    float *Vs = Ks + BN * DP;     // [BN][D]
-    float *Ps = Vs + BN * D;      // [BM][BN+1]
+    constexpr int G = D / 64;                 // float4 groups of output features per thread
+    constexpr int NL = BN * D / 4 / THREADS;  // vector loads per thread per K (or V) tile
+    extern __shared__ __align__(16) float smf[];
+    float *Qt = smf;            // [D][LD]   Q transposed
+    float *Kt = Qt + D * LD;    // [D][LD]   K transposed
+    float *Vs = Kt + D * LD;    // [BN][D]
+    float *Pt = Vs + BN * D;    // [BN][LD]  P transposed
 
     const WlUnit u = p.units[blockIdx.x];
     const WlEntry e = p.entries[u.entry];
@@ -52,12 +71,18 @@ __global__ void __launch_bounds__(simt::THREADS)
     const int32_t q_end = min(q0 + BM, e.q_hi);
     const float sl2 = p.scale_log2;
 
-    for (int idx = tid; idx < BM * D; idx += THREADS) {
+#pragma unroll
+    for (int j = 0; j < BM * D / 4 / THREADS; ++j) {
+        const int idx = 4 * (tid + j * THREADS);
         const int r = idx / D, c = idx % D;
         const int32_t row = q0 + r;
-        Qs[r * DP + c] = row < q_end ? to_f32(q[((int64_t)row * H + h) * D + c]) : 0.f;
+        const float4 x = row < q_end ? load4(q + ((int64_t)row * H + h) * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        Qt[(c + 0) * LD + r] = x.x;
+        Qt[(c + 1) * LD + r] = x.y;
+        Qt[(c + 2) * LD + r] = x.z;
+        Qt[(c + 3) * LD + r] = x.w;
     }
-    float m[4], l[4], o[4][NJ];
+    float m[4], l[4], o[4][G][4];
     int64_t qg[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -65,7 +90,9 @@ __global__ void __launch_bounds__(simt::THREADS)
         l[i] = 0.f;
         qg[i] = (int64_t)(q0 + ty * 4 + i) + e.q_goff;
 #pragma unroll
-        for (int jj = 0; jj < NJ; ++jj) o[i][jj] = 0.f;
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = 0.f;
     }
 
     for (int r = 0; r < e.run_count; ++r) {
@@ -74,13 +101,26 @@ __global__ void __launch_bounds__(simt::THREADS)
         clip_run(e, run, q_end, p.causal, &lo, &hi);
         for (int32_t ks = lo; ks < hi; ks += BN) {
             __syncthreads();
-            for (int idx = tid; idx < BN * D; idx += THREADS) {
+            float4 kr[NL], vr[NL];
+#pragma unroll
+            for (int j = 0; j < NL; ++j) {
+                const int idx = 4 * (tid + j * THREADS);
                 const int rr = idx / D, c = idx % D;
                 const int32_t key = ks + rr;
-                const bool in = key < run.k_hi;
                 const int64_t off = ((int64_t)key * p.Hkv + hkv) * D + c;
-                Ks[rr * DP + c] = in ? to_f32(k[off]) : 0.f;
-                Vs[rr * D + c] = in ? to_f32(v[off]) : 0.f;
+                const bool in = key < run.k_hi;
+                kr[j] = in ? load4(k + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+                vr[j] = in ? load4(v + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < NL; ++j) {
+                const int idx = 4 * (tid + j * THREADS);
+                const int rr = idx / D, c = idx % D;
+                Kt[(c + 0) * LD + rr] = kr[j].x;
+                Kt[(c + 1) * LD + rr] = kr[j].y;
+                Kt[(c + 2) * LD + rr] = kr[j].z;
+                Kt[(c + 3) * LD + rr] = kr[j].w;
+                *reinterpret_cast<float4 *>(Vs + rr * D + c) = vr[j];
             }
             __syncthreads();
             float sacc[4][4];
@@ -90,23 +130,22 @@ __global__ void __launch_bounds__(simt::THREADS)
                 for (int jj = 0; jj < 4; ++jj) sacc[i][jj] = 0.f;
 #pragma unroll 8
             for (int kk = 0; kk < D; ++kk) {
-                float qv[4], kv[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) qv[i] = Qs[(ty * 4 + i) * DP + kk];
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) kv[jj] = Ks[(tx + 16 * jj) * DP + kk];
+                float qa[4], ka[4];
+                f4_split(*reinterpret_cast<const float4 *>(Qt + kk * LD + 4 * ty), qa);
+                f4_split(*reinterpret_cast<const float4 *>(Kt + kk * LD + 4 * tx), ka);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) sacc[i][jj] = fmaf(qv[i], kv[jj], sacc[i][jj]);
+                    for (int jj = 0; jj < 4; ++jj) sacc[i][jj] = fmaf(qa[i], ka[jj], sacc[i][jj]);
             }
+            float pm[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 float x[4];
                 float mx = -INFINITY;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int32_t key = ks + tx + 16 * jj;
+                    const int32_t key = ks + 4 * tx + jj;
                     const bool keep = key < run.k_hi && (!p.causal || (int64_t)key + run.k_goff <= qg[i]);
                     x[jj] = keep ? sacc[i][jj] * sl2 : -INFINITY;
                     mx = fmaxf(mx, x[jj]);
@@ -118,29 +157,36 @@ __global__ void __launch_bounds__(simt::THREADS)
                 float sum = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const float pv = (m_new == -INFINITY) ? 0.f : exp2f(x[jj] - m_new);
-                    sum += pv;
-                    Ps[(ty * 4 + i) * (BN + 1) + tx + 16 * jj] = pv;
+                    pm[i][jj] = (m_new == -INFINITY) ? 0.f : exp2f(x[jj] - m_new);
+                    sum += pm[i][jj];
                 }
 #pragma unroll
                 for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
                 l[i] = l[i] * alpha + sum;
                 m[i] = m_new;
 #pragma unroll
-                for (int jj = 0; jj < NJ; ++jj) o[i][jj] *= alpha;
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) o[i][g][jj] *= alpha;
             }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                *reinterpret_cast<float4 *>(Pt + (4 * tx + jj) * LD + 4 * ty) =
+                    make_float4(pm[0][jj], pm[1][jj], pm[2][jj], pm[3][jj]);
             __syncthreads();
 #pragma unroll 4
             for (int c = 0; c < BN; ++c) {
-                float pv[4], vv[NJ];
+                float pa[4];
+                f4_split(*reinterpret_cast<const float4 *>(Pt + c * LD + 4 * ty), pa);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pv[i] = Ps[(ty * 4 + i) * (BN + 1) + c];
+                for (int g = 0; g < G; ++g) {
+                    float va[4];
+                    f4_split(*reinterpret_cast<const float4 *>(Vs + c * D + 64 * g + 4 * tx), va);
 #pragma unroll
-                for (int jj = 0; jj < NJ; ++jj) vv[jj] = Vs[c * D + tx + 16 * jj];
+                    for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int jj = 0; jj < NJ; ++jj) o[i][jj] = fmaf(pv[i], vv[jj], o[i][jj]);
+                        for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = fmaf(pa[i], va[jj], o[i][g][jj]);
+                }
             }
         }
     }
@@ -162,15 +208,17 @@ __global__ void __launch_bounds__(simt::THREADS)
             float *acc = p.acc_o + (grow * H + h) * D;
             T *dst = static_cast<T *>(p.out) + (out_row * H + h) * D;
 #pragma unroll
-            for (int jj = 0; jj < NJ; ++jj) {
-                const int c = tx + 16 * jj;
-                float v = o[i][jj] * inv;
-                if (!first) v = w.wa * acc[c] + w.wn * v;
-                if (last)
-                    store_out(dst + c, v);
-                else
-                    acc[c] = v;
-            }
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int c = 64 * g + 4 * tx + jj;
+                    float val = o[i][g][jj] * inv;
+                    if (!first) val = w.wa * acc[c] + w.wn * val;
+                    if (last)
+                        store_out(dst + c, val);
+                    else
+                        acc[c] = val;
+                }
             if (tx == 0) {
                 if (last)
                     p.out_lse[(int64_t)h * p.out_rows + out_row] = w.lse;
@@ -180,7 +228,9 @@ __global__ void __launch_bounds__(simt::THREADS)
         } else {
             float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * H + h) * D;
 #pragma unroll
-            for (int jj = 0; jj < NJ; ++jj) dst[tx + 16 * jj] = o[i][jj] * inv;
+            for (int g = 0; g < G; ++g)
+                *reinterpret_cast<float4 *>(dst + 64 * g + 4 * tx) =
+                    make_float4(o[i][g][0] * inv, o[i][g][1] * inv, o[i][g][2] * inv, o[i][g][3] * inv);
             if (tx == 0) p.part_lse[((int64_t)e.slot * H + h) * p.part_rows + out_row] = lse_n;
         }
     }
@@ -190,7 +240,7 @@ template <int D, typename T>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const AttnParams &p,
                                  int num_units, cudaStream_t stream) {
     using namespace simt;
-    const size_t smem = sizeof(float) * (size_t)(BM * (D + 1) + BN * (D + 1) + BN * D + BM * (BN + 1));
+    const size_t smem = sizeof(float) * (size_t)(D * LD + D * LD + BN * D + BN * LD);
     cudaError_t err = cudaFuncSetAttribute(attn_simt_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
@@ -202,6 +252,10 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
 cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k, const void *v,
                              const AttnParams &p, int num_units, cudaStream_t stream) {
     if (num_units <= 0) return cudaSuccess;
+    // The kernel reads four consecutive elements per load.
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                           reinterpret_cast<uintptr_t>(v)) & (uintptr_t)(4 * elem_bytes - 1);
+    if (mis) return cudaErrorMisalignedAddress;
     if (elem_bytes == 4) {
         if (d == 64) return launch_simt_t<64, float>(q, k, v, p, num_units, stream);
         if (d == 128) return launch_simt_t<128, float>(q, k, v, p, num_units, stream);
