@@ -81,8 +81,9 @@ typedef enum { CQSA_MERGE_SLOTS = 0, CQSA_MERGE_FUSED = 1 } cqsa_merge_t;
 
 /* Full plan description.  levels >= 1 and l[0..levels-1] each >= 2; the
  * leaf block is ceil(N / prod_i (l_i (l_i - 1) + 1)) tokens (positions at or
- * past N belong to no pair, so N need not divide evenly).  mem_budget_bytes = 0
- * means unlimited. */
+ * past N belong to no pair, so N need not divide evenly).  1 <= N <=
+ * 2^31 - 4096 (rows are 32-bit on the device).  mem_budget_bytes = 0 means
+ * unlimited. */
 typedef struct {
     int64_t N;
     int H;

@@ -24,6 +24,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <new>
+#include <stdexcept>
 #include <string>
 #include <vector>
 
@@ -84,6 +86,19 @@ cqsa_status_t fail(cqsa_status_t code, const char *fmt, ...) {
     va_end(ap);
     g_err = buf;
     return code;
+}
+
+// Host-side C++ failures (a work list too large for host memory, say)
+// become status codes: no call of this library lets an exception out.
+template <typename F>
+cqsa_status_t guarded(F &&f) {
+    try {
+        return f();
+    } catch (const std::bad_alloc &) {
+        return fail(CQSA_ERR_BUDGET, "host memory ran out while building the plan's work lists");
+    } catch (const std::exception &ex) {
+        return fail(CQSA_ERR_INTERNAL, "internal error: %s", ex.what());
+    }
 }
 
 #define CK(call)                                                                                  \
@@ -290,7 +305,7 @@ cqsa_status_t check_device(cqsa_plan_t *P) {
     return CQSA_OK;
 }
 
-cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
+cqsa_status_t setup_device_mode_impl(cqsa_plan_t *P) {
     if (P->dev_arena) return CQSA_OK;
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N;
@@ -331,7 +346,9 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
     return CQSA_OK;
 }
 
-cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
+cqsa_status_t setup_device_mode(cqsa_plan_t *P) { return guarded([&] { return setup_device_mode_impl(P); }); }
+
+cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     if (P->host_arena) return CQSA_OK;
     const Planner &pl = P->pl;
     const int g = pl.sizing.head_group;
@@ -411,6 +428,8 @@ cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
     return CQSA_OK;
 }
 
+cqsa_status_t setup_host_mode(cqsa_plan_t *P) { return guarded([&] { return setup_host_mode_impl(P); }); }
+
 AttnParams base_params(const cqsa_plan_t *P, int *err) {
     AttnParams ap{};
     ap.causal = P->pl.spec.causal;
@@ -488,7 +507,7 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     return CQSA_OK;
 }
 
-cqsa_status_t setup_partial(cqsa_plan_t *P) {
+cqsa_status_t setup_partial_impl(cqsa_plan_t *P) {
     if (P->part_arena) return CQSA_OK;
     const Planner &pl = P->pl;
     WorkList wl = pl.partial_worklist(unit_rows_for(P->elem), key_tile_for(P->elem), pl.spec.H);
@@ -505,6 +524,8 @@ cqsa_status_t setup_partial(cqsa_plan_t *P) {
     P->part_wl = place_wl(arena + o_wl, wl);
     return CQSA_OK;
 }
+
+cqsa_status_t setup_partial(cqsa_plan_t *P) { return guarded([&] { return setup_partial_impl(P); }); }
 
 // This rank's entries of a sharded plan: every query block it has an entry
 // for is one work-list entry flagged SEG_FIRST only, so the epilogue leaves
@@ -544,7 +565,7 @@ cqsa_status_t forward_partial_device(cqsa_plan_t *P, const void *q, const void *
     return CQSA_OK;
 }
 
-cqsa_status_t setup_backward(cqsa_plan_t *P, BwdState &B, bool shard) {
+cqsa_status_t setup_backward_impl(cqsa_plan_t *P, BwdState &B, bool shard) {
     if (B.arena) return CQSA_OK;
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N;
@@ -617,6 +638,10 @@ cqsa_status_t setup_backward(cqsa_plan_t *P, BwdState &B, bool shard) {
     B.qwl = place_wl(arena + o_qwl, qwl);
     B.kvwl = place_wl(arena + o_kvwl, kvwl);
     return CQSA_OK;
+}
+
+cqsa_status_t setup_backward(cqsa_plan_t *P, BwdState &B, bool shard) {
+    return guarded([&] { return setup_backward_impl(P, B, shard); });
 }
 
 // out_elem: element bytes of dq, dk, dv (the plan's, or 4 for the fp32
@@ -818,7 +843,7 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
     cudaStreamWaitEvent(stream, P->ev_done_out, 0);
 }
 
-cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
+cqsa_status_t build_plan_impl(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
     cqsa_plan_t *P = new cqsa_plan_t();
     P->dtype = dtype;
     P->elem = spec.elem_bytes;
@@ -830,6 +855,10 @@ cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
     }
     *out = P;
     return CQSA_OK;
+}
+
+cqsa_status_t build_plan(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
+    return guarded([&] { return build_plan_impl(spec, dtype, out); });
 }
 
 }  // namespace

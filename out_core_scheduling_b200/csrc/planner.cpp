@@ -73,7 +73,9 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     *code = 1;  // INVALID_ARG unless changed
     if (s.N <= 0 || s.H <= 0 || s.d <= 0) return "N, H and d must be positive";
     if (s.levels < 1 || s.levels > kMaxLevels) return "levels must be in 1..4";
-    if (s.N > (int64_t)INT32_MAX) return "N must be below 2^31";
+    // Rows are 32-bit in the work lists and kernels, which add a tile or
+    // unit width (at most 256) to a row: keep that below 2^31.
+    if (s.N > (int64_t)kMaxN) return "N must be at most 2^31 - 4096";
     if (s.Hkv < 0 || (s.Hkv > 0 && s.H % s.Hkv != 0))
         return "the query heads must be a multiple of the key/value heads";
     if (spec.Hkv == 0) spec.Hkv = s.H;
@@ -263,12 +265,12 @@ static void add_units(WorkList *wl, int heads, int rows_per_unit, int bn, int ca
     for (int32_t ei = 0; ei < (int32_t)wl->entries.size(); ++ei) {
         const WlEntry &e = wl->entries[ei];
         for (int h = 0; h < heads; ++h)
-            for (int32_t q0 = e.q_lo; q0 < e.q_hi; q0 += rows_per_unit) {
+            for (int64_t q0 = e.q_lo; q0 < e.q_hi; q0 += rows_per_unit) {
                 WlUnit x;
                 x.entry = ei;
-                x.q0 = q0;
+                x.q0 = (int32_t)q0;  // < N <= kMaxN
                 x.head = h;
-                x.ntiles = unit_key_tiles(e, wl->runs.data(), q0, rows_per_unit, causal, bn);
+                x.ntiles = unit_key_tiles(e, wl->runs.data(), x.q0, rows_per_unit, causal, bn);
                 if (x.ntiles > 0) u.push_back(x);
             }
     }
@@ -500,8 +502,9 @@ WorkList Planner::kv_worklist(int rows_per_unit, int bn, int heads, const std::v
     for (int32_t ei = 0; ei < (int32_t)wl.entries.size(); ++ei) {
         const WlEntry &e = wl.entries[ei];
         for (int h = 0; h < heads; ++h)
-            for (int32_t k0 = e.q_lo; k0 < e.q_hi; k0 += rows_per_unit) {
-                WlUnit x{ei, k0, h, unit_query_tiles(e, wl.runs.data(), k0, spec.causal, bn)};
+            for (int64_t k0 = e.q_lo; k0 < e.q_hi; k0 += rows_per_unit) {
+                const int32_t r0 = (int32_t)k0;  // < N <= kMaxN
+                WlUnit x{ei, r0, h, unit_query_tiles(e, wl.runs.data(), r0, spec.causal, bn)};
                 if (x.ntiles > 0) u.push_back(x);
             }
     }

@@ -21,6 +21,7 @@
 namespace cqsa {
 
 constexpr int kMaxLevels = 4;
+constexpr int64_t kMaxN = (1LL << 31) - 4096;  // 32-bit rows plus a unit or tile width
 
 struct Level {
     int l = 0;            // chunks per subsequence

@@ -36,10 +36,12 @@ def _compare(got, ref, dtype, name):
     tol = GTOL[dtype]
     g = got.cpu().double().numpy()
     assert np.all(np.isfinite(g)), name
-    gmax = np.abs(ref).max()
+    # A gradient that vanishes exactly (one key per row: dS = 0) is compared
+    # against a floor of 1e-2 instead of its zero maximum.
+    gmax = max(np.abs(ref).max(), 1e-2)
     err = np.abs(g - ref)
     assert err.max() <= tol["rel_max"] * gmax + tol["abs_max"], (name, err.max(), gmax)
-    if tol["rel_fro"] is not None:
+    if tol["rel_fro"] is not None and np.linalg.norm(ref) > 1e-2:
         fro = np.linalg.norm(g - ref) / np.linalg.norm(ref)
         assert fro <= tol["rel_fro"], (name, fro)
 
@@ -112,7 +114,9 @@ def test_backward_rejects_host_mode():
 @pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("case", [(1000, 2, 128, [3], torch.bfloat16), (91 * 12 + 5, 1, 64, [4, 3], torch.bfloat16),
-                                  (700 - 9, 1, 64, [3], torch.float32)],
+                                  (700 - 9, 1, 64, [3], torch.float32), (1, 1, 64, [3], torch.bfloat16),
+                                  (5, 1, 64, [3], torch.bfloat16), (3 * 128, 2, 128, [2], torch.bfloat16),
+                                  (7, 1, 64, [2], torch.float32)],
                          ids=lambda c: f"n{c[0]}-l{c[3]}-{str(c[4])[6:]}")
 def test_backward_ragged_n(case, causal, merge):
     N, H, d, ls, dtype = case

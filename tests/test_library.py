@@ -64,7 +64,7 @@ def reference_pairs(P, ls, causal):
     return out
 
 
-CASES = [((3,), 7), ((4,), 13), ((5,), 21), ((6,), 31), ((4, 3), 91), ((3, 3), 49)]
+CASES = [((2,), 3), ((3,), 7), ((4,), 13), ((5,), 21), ((6,), 31), ((4, 3), 91), ((3, 3), 49), ((2, 2), 9)]
 
 
 @pytest.mark.parametrize("ls,P", CASES, ids=lambda x: str(x))
@@ -279,3 +279,31 @@ def test_fault_injection_arguments():
         assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
     cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_ALLOC, 0)
     cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, 0)
+
+
+def test_n_limit():
+    """Rows are 32-bit on the device and kernels add up to a unit width to a
+    row: N is capped at 2^31 - 4096, and a plan at the cap builds."""
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_plan_ex(2 ** 31 - 4095, 1, 64, [3])
+    assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+    info = cqsa.cqsa_plan_ex(2 ** 31 - 4096, 1, 64, [3]).info()
+    assert info["block_tokens"] == -(-(2 ** 31 - 4096) // 7)
+
+
+@pytest.mark.parametrize("N", [1, 2, 3, 5])
+@pytest.mark.parametrize("ls", [[2], [3], [4, 3]])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_n_plans(N, ls, causal):
+    """Fewer tokens than chunks: blocks of one token, the rest empty; the
+    live pairs are exactly the reference's and cover N^2 (N (N+1)/2)."""
+    P = 1
+    for l in ls:
+        P *= l * (l - 1) + 1
+    plan = cqsa.cqsa_plan_ex(N, 1, 64, ls, causal=causal)
+    info = plan.info()
+    assert info["block_tokens"] == -(-N // P)
+    live = {b for b in range(P) if b * info["block_tokens"] < N}
+    ref = {(t, qb, kb) for (t, qb, kb) in reference_pairs(P, tuple(ls), causal) if qb in live and kb in live}
+    assert plan_pairs(plan) == ref
+    assert info["total_pairs"] == (N * (N + 1) / 2 if causal else float(N * N))

@@ -397,3 +397,24 @@ def test_injected_copy_failure_is_recoverable(nth):
     plan.sync()
     out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
     check(out, lse, q, k, v, np.arange(N), False)
+
+
+# ------------------------------------------------------------- degenerate sizes
+@pytest.mark.parametrize("N,ls", [(1, [3]), (2, [3]), (5, [3]), (3, [2]), (7, [2]), (3 * 256, [2]), (4, [4, 3])])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_degenerate_sizes(N, ls, causal, dtype):
+    """N smaller than the chunk count (one-token and empty blocks), N = 1,
+    and l = 2 (three chunks, D = {0, 1}), on the device (slots and fused)
+    and streamed paths: every row against the oracle."""
+    H, d = 2, 64
+    cdt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    q, k, v = _inputs(N, H, d, dtype, seed=90 + N)
+    for merge in (cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED):
+        plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, merge=merge)
+        out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+        check(out, lse, q, k, v, np.arange(N), causal)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, mem_budget_bytes=1 << 30)
+    out, lse = run(plan, qh, kh, vh, cqsa.CQSA_HOST)
+    check(out, lse, qh, kh, vh, np.arange(N), causal)
