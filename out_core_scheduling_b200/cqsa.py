@@ -261,6 +261,12 @@ def _check_shapes(plan: Plan, qlike, kvlike, lse):
         raise ValueError("lse must be float32")
     if len({t.dtype for _, t in list(qlike) + list(kvlike)}) != 1:
         raise ValueError(", ".join(n for n, _ in list(qlike) + list(kvlike)) + " must share a dtype")
+    want = torch.bfloat16 if info["dtype"] == CQSA_BF16 else torch.float32
+    for name, t in list(qlike) + list(kvlike):
+        if t.dtype != want:
+            # The library reads element sizes from the plan: another dtype
+            # would be misread, or read past the end of the tensor.
+            raise ValueError(f"{name} is {t.dtype}, the plan's dtype is {want}")
     def shape_ok(t, want):
         return tuple(t.shape) == lead + want or (B == 1 and tuple(t.shape) == (1,) + want)
     for name, t in qlike:

@@ -307,3 +307,19 @@ def test_tiny_n_plans(N, ls, causal):
     ref = {(t, qb, kb) for (t, qb, kb) in reference_pairs(P, tuple(ls), causal) if qb in live and kb in live}
     assert plan_pairs(plan) == ref
     assert info["total_pairs"] == (N * (N + 1) / 2 if causal else float(N * N))
+
+
+def test_tensor_dtype_must_match_the_plan():
+    """The ABI reads element sizes from the plan: the binding refuses tensors
+    of another dtype before any pointer reaches the library."""
+    import torch
+    N, H, d = 7 * 4, 1, 64
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], dtype=cqsa.CQSA_FP32)
+    x = torch.zeros(N, H, d, dtype=torch.bfloat16)
+    lse = torch.zeros(H, N)
+    with pytest.raises(ValueError, match="dtype"):
+        cqsa.cqsa_forward(plan, x, x, x, x.clone(), lse)
+    plan16 = cqsa.cqsa_plan_ex(N, H, d, [3])
+    y = torch.zeros(N, H, d)
+    with pytest.raises(ValueError, match="dtype"):
+        cqsa.cqsa_forward(plan16, y, y, y, y.clone(), lse)
