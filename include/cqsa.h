@@ -178,7 +178,11 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out);
  *     after and that is ordered after all of its work.
  * Asynchronous: returns once all work is enqueued.  The first call on a plan
  * allocates its arena (one cudaMalloc, sized by the plan).  One forward at a
- * time per plan.  Errors: INVALID_ARG, NOT_PINNED, CUDA, NO_DEVICE, BUDGET.
+ * time per plan.  After that first call a device-mode forward (and likewise
+ * cqsa_backward) enqueues only kernel launches on `stream`, so it may be
+ * captured in a CUDA graph and replayed with new contents in the same
+ * buffers; the streamed mode's internal streams and events are not for
+ * capture.  Errors: INVALID_ARG, NOT_PINNED, CUDA, NO_DEVICE, BUDGET.
  * Device-side timeouts are reported by cqsa_plan_sync.
  */
 cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,

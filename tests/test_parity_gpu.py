@@ -418,3 +418,44 @@ def test_degenerate_sizes(N, ls, causal, dtype):
     plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, mem_budget_bytes=1 << 30)
     out, lse = run(plan, qh, kh, vh, cqsa.CQSA_HOST)
     check(out, lse, qh, kh, vh, np.arange(N), causal)
+
+
+# ------------------------------------------------------------------ CUDA graphs
+@pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])
+def test_forward_and_backward_in_a_cuda_graph(merge):
+    """After the first call has allocated the plan's arenas, device-mode
+    forward and backward are plain launches on the caller's stream: they can
+    be captured in a CUDA graph and replayed on new inputs in the same
+    buffers."""
+    import oracle
+    N, H, d = 7 * 128, 2, 128
+    causal = True
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=100)
+    dout = _inputs(N, H, d, torch.bfloat16, seed=101)[0]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, merge=merge)
+    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up: arenas allocated outside the capture
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+        cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+        cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, dq, dk, dv)
+    for seed in (102, 103):
+        nq, nk, nv = _inputs(N, H, d, torch.bfloat16, seed=seed)
+        q.copy_(nq)
+        k.copy_(nk)
+        v.copy_(nv)
+        g.replay()
+        torch.cuda.synchronize()
+        plan.sync()
+        check(out, lse, q, k, v, np.arange(N), causal)
+        qc, kc, vc, dc = (x.cpu() for x in (q, k, v, dout))
+        ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
+        g_dq = dq.cpu().double().numpy()
+        assert np.abs(g_dq - ref_dq).max() <= 2e-2 * np.abs(ref_dq).max()
