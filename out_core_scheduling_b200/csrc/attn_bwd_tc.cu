@@ -54,10 +54,16 @@ struct SmemDq {
     alignas(1024) uint8_t dout[KB][BOX_BYTES];
     alignas(1024) uint8_t k[KST][KB][BOX_BYTES];
     alignas(1024) uint8_t v[VST][KB][BOX_BYTES];
-    // s_ready[b]: S of a tile in TMEM buffer b (tiles b, b + 2, ...): a phase
-    // cannot run ahead of the elementwise warps, since S(j + 2) follows dQ(j).
-    uint64_t bar_q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_ready[2], dp_ready, dp_free, p_half,
-        p_full, o_full, drain;
+    // s_ready[b], p_half[b], p_full[b]: tiles b, b + 2, ... (TMEM buffer b).
+    // No phase of them can complete while a waiter has yet to see the one
+    // before: S(j + 2) is issued only after the MMA warp has seen p_full(j),
+    // and the elementwise warps arrive on p_half / p_full of tile j + 2 only
+    // after S(j + 2).  With a single p_half / p_full, the warps could finish
+    // tile j + 1 (its S and dP are issued before the MMA warp waits on tile
+    // j's halves) and complete a second phase before the MMA warp polled the
+    // first, which then waits for good.
+    uint64_t bar_q, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_ready[2], dp_ready, dp_free, p_half[2],
+        p_full[2], o_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -185,8 +191,10 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         mbar_init(&s.s_ready[1], 1);
         mbar_init(&s.dp_ready, 1);
         mbar_init(&s.dp_free, EW_WARPS);
-        mbar_init(&s.p_half, EW_WARPS);
-        mbar_init(&s.p_full, EW_WARPS);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s.p_half[b], EW_WARPS);
+            mbar_init(&s.p_full[b], EW_WARPS);
+        }
         mbar_init(&s.o_full, 1);
         mbar_init(&s.drain, 1);
         s.abort = 0;
@@ -288,10 +296,10 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 mma_commit_elect(&s.dp_ready);
             }
             const uint64_t kb = smem_desc_sw128(smem_u32(s.k[j % KST][0]), BOX_BYTES, 1024);
-            if (!warp_wait_b(&s.p_half, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            if (!warp_wait_b(&s.p_half[j & 1], (uint32_t)(j >> 1) & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
             mma_tmem_half(tmem + 256u, tmem + s_col(j), kb, IDESC_TS, j > 0, 0);
-            if (!warp_wait_b(&s.p_full, (uint32_t)j & 1u, abort, tmo)) { ok = false; break; }
+            if (!warp_wait_b(&s.p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort, tmo)) { ok = false; break; }
             tc_fence_after();
             mma_tmem_half(tmem + 256u, tmem + s_col(j), kb, IDESC_TS, true, 1);
             mma_commit_elect(&s.k_empty[j % KST]);
@@ -376,7 +384,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(cc == 0 ? &s.p_half : &s.p_full);
+                    if (lane == 0) mbar_arrive(cc == 0 ? &s.p_half[j & 1] : &s.p_full[j & 1]);
                 }
             }
         }
@@ -659,19 +667,22 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 // Phase B: dS^T = P^T (dP^T - D) over dP^T.
                 if (!warp_wait_b(&s.dp_full, (uint32_t)i & 1u, abort, tmo)) { ok = false; break; }
                 tc_fence_after();
+                uint32_t dp[2][32];
+                tmem_ld32(lane_base + 128u + (uint32_t)c0, dp[0]);
+                tmem_ld32(lane_base + 128u + (uint32_t)(c0 + 32), dp[1]);
+                tmem_wait_ld();
+                fence_regs32(dp[0]);
+                fence_regs32(dp[1]);
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    uint32_t dp[32], pd[16];
-                    tmem_ld32(lane_base + 128u + (uint32_t)(c0 + cc * 32), dp);
-                    tmem_wait_ld();
-                    fence_regs32(dp);
+                    uint32_t pd[16];
 #pragma unroll
                     for (int t = 0; t < 32; t += 4) {
                         const float4 d4 = lds_f4(dl + cc * 32 + t);
-                        pd[t / 2] = pack_bf16x2(pv[cc][t] * (__uint_as_float(dp[t]) - d4.x),
-                                                pv[cc][t + 1] * (__uint_as_float(dp[t + 1]) - d4.y));
-                        pd[t / 2 + 1] = pack_bf16x2(pv[cc][t + 2] * (__uint_as_float(dp[t + 2]) - d4.z),
-                                                    pv[cc][t + 3] * (__uint_as_float(dp[t + 3]) - d4.w));
+                        pd[t / 2] = pack_bf16x2(pv[cc][t] * (__uint_as_float(dp[cc][t]) - d4.x),
+                                                pv[cc][t + 1] * (__uint_as_float(dp[cc][t + 1]) - d4.y));
+                        pd[t / 2 + 1] = pack_bf16x2(pv[cc][t + 2] * (__uint_as_float(dp[cc][t + 2]) - d4.z),
+                                                    pv[cc][t + 3] * (__uint_as_float(dp[cc][t + 3]) - d4.w));
                     }
                     tmem_st16_b(lane_base + 128u + (uint32_t)(c0 + cc * 16), pd);
                 }
