@@ -20,6 +20,8 @@
 // the two never touch each other's columns.  Every wait is bounded; on a
 // timeout the CTA records DEV_TIMEOUT, drains its copies and MMAs, frees its
 // tensor memory and returns.
+// The barrier hand-offs of both kernels are modelled warp role by warp role
+// in tests/barrier_model.py, whose explorer checks every interleaving.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
