@@ -26,8 +26,6 @@
 //
 // Every wait is bounded; on a timeout the CTA records DEV_TIMEOUT, drains
 // its own copies and MMAs, frees its tensor memory and returns.
-// The barrier hand-offs are modelled warp role by warp role in
-// tests/barrier_model.py, whose explorer checks every interleaving.
 #include <cuda_runtime.h>
 
 #include "common.cuh"

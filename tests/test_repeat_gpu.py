@@ -1,0 +1,46 @@
+"""Back-to-back calls of the tensor-core paths never run out of their
+bounded waits, and repeated calls give identical results.
+
+A barrier hand-off that lets a phase run ahead of its waiter hangs only
+when the warps' timing lines up, which back-to-back launches at a working
+size make likely within a few hundred calls (the dq kernel's former shared
+P-half / P-full pair hung about one call in 250 at l = 4, N = 53248).  The
+exhaustive check of the hand-offs is the CPU model in barrier_model.py;
+this is its end-to-end counterpart on the device."""
+import pytest
+import torch
+
+from out_core_scheduling_b200 import cqsa
+from out_core_scheduling_b200.inputs import make_qkv
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+N, H, d = 13 * 2048, 8, 128
+
+
+def _repeat(plan, fn, calls, per_sync=25):
+    for _ in range(calls // per_sync):
+        for _ in range(per_sync):
+            fn()
+        plan.sync()  # raises CqsaError(CQSA_ERR_TIMEOUT) if any wait ran out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_repeated_forward_and_backward(causal):
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=41, device=DEV)
+    dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=42, device=DEV)[0]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal)
+    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+    cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    plan.sync()
+    out0, lse0 = out.clone(), lse.clone()
+    _repeat(plan, lambda: cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE), 300)
+    assert torch.equal(out, out0) and torch.equal(lse, lse0)
+
+    g = [torch.empty_like(q) for _ in range(3)]
+    cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, *g)
+    plan.sync()
+    g0 = [x.clone() for x in g]
+    _repeat(plan, lambda: cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, *g), 300)
+    for a, b in zip(g, g0):
+        assert torch.equal(a, b)
