@@ -279,7 +279,9 @@ cqsa_status_t cqsa_backward_partial(cqsa_plan_t *plan, const void *q, const void
 cqsa_status_t cqsa_partial_cast(cqsa_plan_t *plan, const float *src, void *dst, int64_t count, void *stream);
 
 /* cqsa_plan_sync -- wait for the plan's work on `stream` and report any
- * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync. */
+ * device-side error word (CQSA_ERR_TIMEOUT) raised since the last sync; the
+ * message (cqsa_last_error) names the kernels whose wait ran out: device
+ * forward, streamed forward, backward, partial forward or partial backward. */
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream);
 
 /* cqsa_plan_info -- copy what the plan decided into *info. */

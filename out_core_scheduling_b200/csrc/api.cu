@@ -1123,17 +1123,23 @@ cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (plan->device < 0) return CQSA_OK;
     CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     int *words[5] = {plan->dev_err, plan->h_err, plan->bwd.err, plan->bwd_shard.err, plan->part_err};
+    static const char *const where[5] = {"device forward", "streamed forward", "backward", "partial backward",
+                                         "partial forward"};
     int bad = 0;
-    for (int *w : words) {
-        if (!w) continue;
+    std::string sites;
+    for (int i = 0; i < 5; ++i) {
+        if (!words[i]) continue;
         int v = 0;
-        CK(cudaMemcpy(&v, w, sizeof v, cudaMemcpyDeviceToHost));
+        CK(cudaMemcpy(&v, words[i], sizeof v, cudaMemcpyDeviceToHost));
         if (v) {
             bad = v;
-            CK(cudaMemset(w, 0, sizeof v));
+            sites += sites.empty() ? where[i] : std::string(", ") + where[i];
+            CK(cudaMemset(words[i], 0, sizeof v));
         }
     }
-    if (bad) return fail(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d); output is incomplete", bad);
+    if (bad)
+        return fail(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d, in the %s kernels); output is incomplete",
+                    bad, sites.c_str());
     return CQSA_OK;
 }
 

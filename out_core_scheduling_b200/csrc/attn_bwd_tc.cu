@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(&s.bar_kv, 1);
         for (int i = 0; i < STAGES; ++i) {
-            mbar_init(&s.qd_full[i], 1);
+            mbar_init(&s.qd_full[i], 2);  // the copy's expect_tx, then the lse / D staging
             mbar_init(&s.qd_empty[i], 1);
         }
         mbar_init(&s.st_full, 1);
@@ -488,7 +488,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
     const int ntiles = unit_query_tiles(e, p.runs, k0, causal, BN);
 
     if (warp == WARP_TMA) {
-        // The whole warp stages each tile's lse and D; lane 0 issues the TMA.
+        // Lane 0 issues each tile's Q / dO copy first; the whole warp then stages
+        // the tile's lse and D, and lane 0 arrives again, so the stage's full
+        // barrier waits for both while the two latencies overlap.
         if (lane == 0) {
             mbar_expect_tx(&s.bar_kv, 2 * TILE);
             for (int kb = 0; kb < KB; ++kb) {
@@ -508,6 +510,13 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     ok = false;
                     break;
                 }
+                if (lane == 0) {
+                    mbar_expect_tx(&s.qd_full[st], 2 * TILE);
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_load_3d(s.q[st][kb], &tmQ, &s.qd_full[st], kb * 64, head, qs);
+                        tma_load_3d(s.dout[st][kb], &tmO, &s.qd_full[st], kb * 64, head, qs);
+                    }
+                }
 #pragma unroll
                 for (int c = lane; c < BN; c += 32) {
                     const int32_t row = qs + c;
@@ -517,13 +526,7 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     s.dl[st][c] = in ? p.delta[(int64_t)head * p.N + g] : 0.f;
                 }
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_expect_tx(&s.qd_full[st], 2 * TILE);
-                    for (int kb = 0; kb < KB; ++kb) {
-                        tma_load_3d(s.q[st][kb], &tmQ, &s.qd_full[st], kb * 64, head, qs);
-                        tma_load_3d(s.dout[st][kb], &tmO, &s.qd_full[st], kb * 64, head, qs);
-                    }
-                }
+                if (lane == 0) mbar_arrive(&s.qd_full[st]);
                 __syncwarp();
             }
         }

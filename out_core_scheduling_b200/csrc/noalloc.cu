@@ -265,6 +265,7 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     NA_CK(cudaStreamSynchronize(s));
     int word = 0;
     NA_CK(cudaMemcpy(&word, err_word, sizeof word, cudaMemcpyDeviceToHost));
-    if (word) return err(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d)", word);
+    if (word)
+        return err(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d, in the allocation-free forward)", word);
     return CQSA_OK;
 }

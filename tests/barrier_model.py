@@ -231,10 +231,13 @@ def dq_model(n, warps=2, kst=3, vst=2, split_handoff=True):
 
 
 def dkdv_model(n, warps=2, stages=2):
-    """dk/dv gradient kernel (the loop runs over query tiles)."""
+    """dk/dv gradient kernel (the loop runs over query tiles).  A Q / dO
+    stage completes on two arrivals: the copy's expect_tx (issued first) and
+    the TMA warp's arrival once it has stored the tile's lse and D."""
     tma = [("tma", "bar_kv")]
     for i in range(n):
-        tma += [("wait", f"qd_empty{i % stages}", i // stages - 1), ("tma", f"qd_full{i % stages}")]
+        tma += [("wait", f"qd_empty{i % stages}", i // stages - 1), ("tma", f"qd_full{i % stages}"),
+                ("arrive", f"qd_full{i % stages}")]
     mma = [("wait", "bar_kv", 0)]
     if n > 0:
         mma += [("wait", "qd_full0", 0), ("commit", "st_full"), ("commit", "dp_full")]
@@ -255,5 +258,6 @@ def dkdv_model(n, warps=2, stages=2):
     counts = {"bar_kv": 1, "st_full": 1, "dp_full": 1, "pt_full": warps, "ds_full": warps, "o_full": 1,
               "drain": 1}
     for s in range(stages):
-        counts[f"qd_full{s}"] = counts[f"qd_empty{s}"] = 1
+        counts[f"qd_full{s}"] = 2
+        counts[f"qd_empty{s}"] = 1
     return [("tma", tma, 1), ("mma", mma, 1), ("elementwise", ew, warps)], counts

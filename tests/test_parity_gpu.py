@@ -199,6 +199,7 @@ def test_bounded_wait_reports_timeout_and_recovers():
     with pytest.raises(cqsa.CqsaError) as ei:
         plan.sync()
     assert ei.value.status == cqsa.CQSA_ERR_TIMEOUT
+    assert "device forward" in str(ei.value)
     plan.debug(timeout_ns=0, stall_mma=False)
     out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
     check(out, lse, q, k, v, np.arange(N), False)
