@@ -1,9 +1,11 @@
-"""Every interleaving of the tensor-core kernels' barrier hand-offs keeps the
-parity waits sound (no wait passes early, none misses its phase, nothing
-deadlocks).  The models in barrier_model.py follow the warp roles of
-attn_tc.cu (forward) and attn_bwd_tc.cu (dq, dk/dv) for units of 0 to 7
-tiles; the planted cases check that the explorer catches each kind of
-mistake."""
+"""Every interleaving of the tensor-core kernels' hand-offs keeps the parity
+waits sound (no wait passes early, none misses its phase, nothing
+deadlocks) and every shared- and tensor-memory access free of races (each
+read finds the version it needs; nothing is overwritten while still
+needed or in use by an issued MMA or copy).  The models in barrier_model.py
+follow the warp roles of attn_tc.cu (forward) and attn_bwd_tc.cu (dq,
+dk/dv) for units of 0 to 7 tiles; the planted cases check that the
+explorer catches each kind of mistake."""
 import os
 import re
 
@@ -17,31 +19,49 @@ CSRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 @pytest.mark.parametrize("n", range(0, 6))
 def test_forward_protocol(n):
-    bm.explore(*bm.forward_model(n))
+    bm.explore(*bm.forward_model(n, data=False))
 
 
 @pytest.mark.parametrize("n", range(0, 8))
 def test_dq_protocol(n):
-    bm.explore(*bm.dq_model(n))
+    bm.explore(*bm.dq_model(n, data=False))
 
 
 @pytest.mark.parametrize("n", range(0, 8))
 def test_dkdv_protocol(n):
-    bm.explore(*bm.dkdv_model(n))
+    bm.explore(*bm.dkdv_model(n, data=False))
 
 
 @pytest.mark.parametrize("model,n", [(bm.forward_model, 3), (bm.dq_model, 4), (bm.dkdv_model, 4)])
 def test_protocols_with_three_warps(model, n):
-    bm.explore(*model(n, warps=3))
+    bm.explore(*model(n, warps=3, data=False))
+
+
+# Data: every shared- and tensor-memory region is read only when it holds
+# the version the step needs, and never written while another step still
+# needs the old one or an issued MMA / copy is using it.
+@pytest.mark.parametrize("n", range(0, 5))
+def test_forward_data_hazards(n):
+    bm.explore(*bm.forward_model(n, warps=1))
+
+
+@pytest.mark.parametrize("n", range(0, 5))
+def test_dq_data_hazards(n):
+    bm.explore(*bm.dq_model(n))
+
+
+@pytest.mark.parametrize("n", range(0, 6))
+def test_dkdv_data_hazards(n):
+    bm.explore(*bm.dkdv_model(n))
 
 
 def test_shared_handoff_pair_misses_a_phase():
     """One p_half / p_full pair for consecutive dq tiles: the elementwise
     warps can complete tile j + 1's half before the MMA warp has polled tile
     j's (the hang this kernel once had)."""
-    assert bm.explore(*bm.dq_model(1, split_handoff=False))
+    assert bm.explore(*bm.dq_model(1, split_handoff=False, data=False))
     with pytest.raises(bm.Violation, match="late: p_half"):
-        bm.explore(*bm.dq_model(2, split_handoff=False))
+        bm.explore(*bm.dq_model(2, split_handoff=False, data=False))
 
 
 def _edit(model, role, fn):
@@ -51,7 +71,7 @@ def _edit(model, role, fn):
 
 def test_planted_missing_slot_wait_is_caught():
     # producer refills a K slot without waiting for it to be released
-    m = _edit(bm.forward_model(3), "tma", lambda ops: [o for o in ops if o[:2] != ("wait", "k_empty0")])
+    m = _edit(bm.forward_model(3, data=False), "tma", lambda ops: [o for o in ops if o[:2] != ("wait", "k_empty0")])
     with pytest.raises(bm.Violation):
         bm.explore(*m)
 
@@ -62,7 +82,7 @@ def test_planted_wrong_parity_index_is_caught():
         return [("wait", o[1], 2 * o[2] + int(o[1][-1])) if o[:2] in (("wait", "s_ready0"), ("wait", "s_ready1"))
                 else o for o in ops]
     with pytest.raises(bm.Violation, match="early|late"):
-        bm.explore(*_edit(bm.dq_model(4), "elementwise", bad))
+        bm.explore(*_edit(bm.dq_model(4, data=False), "elementwise", bad))
 
 
 def test_planted_early_issue_is_caught():
@@ -74,13 +94,74 @@ def test_planted_early_issue_is_caught():
         out.insert(i, out.pop(j))
         return out
     with pytest.raises(bm.Violation, match="late"):
-        bm.explore(*_edit(bm.dkdv_model(3), "mma", bad))
+        bm.explore(*_edit(bm.dkdv_model(3, data=False), "mma", bad))
 
 
 def test_planted_missing_arrival_deadlocks():
-    m = _edit(bm.dkdv_model(2), "elementwise", lambda ops: ops[:-2] + ops[-1:])
+    m = _edit(bm.dkdv_model(2, data=False), "elementwise", lambda ops: ops[:-2] + ops[-1:])
     with pytest.raises(bm.Violation, match="deadlock"):
         bm.explore(*m)
+
+
+def _writes(op, tag):
+    return op[0] == "mma" and any(len(w) == 2 and w[1] == tag for w in op[2])
+
+
+def test_planted_overwrite_before_use_is_caught():
+    """dk/dv: S^T(1) issued (after its Q tile is in) before dV(0), so it
+    lands over P^T(0) before dV(0) has read it."""
+    def bad(ops):
+        out = list(ops)
+        b = next(i for i, o in enumerate(out) if _writes(o, ("ST", 1)))
+        moved = [out.pop(b - 1), out.pop(b - 1)]  # the qd_full wait and S^T(1)
+        a = next(i for i, o in enumerate(out) if _writes(o, ("dV", 0)))
+        out[a:a] = moved
+        return out
+    with pytest.raises(bm.Violation, match="overwrites ST"):
+        bm.explore(*_edit(bm.dkdv_model(2), "mma", bad))
+
+
+def test_planted_early_rescale_is_caught():
+    """Forward: S_0(1) issued and committed before PV_0(0), so the softmax
+    may rescale O_0 while PV_0(0) still writes it, and P_0(0) is
+    overwritten before PV_0(0) reads it."""
+    def bad(ops):
+        out = list(ops)
+        a = out.index(("wait", "p_half0", 0))
+        b = next(i for i, o in enumerate(out) if _writes(o, ("S", 0, 1)))
+        moved = [out.pop(b), out.pop(b)]  # the QK MMA and its s_full commit
+        out[a:a] = moved
+        return out
+    with pytest.raises(bm.Violation, match="stale|race"):
+        bm.explore(*_edit(bm.forward_model(2, warps=1), "mma", bad))
+
+
+def test_planted_single_s_buffer_is_caught():
+    """dq with one S buffer: S(j + 1) would land over dS(j) before dQ(j)
+    has read it."""
+    roles, counts = bm.dq_model(3)
+
+    def one(x):
+        if isinstance(x, str):
+            return x.replace("S1.", "S0.")
+        if isinstance(x, (tuple, list)):
+            return type(x)(one(y) for y in x)
+        return x
+    with pytest.raises(bm.Violation, match="stale|race"):
+        bm.explore([(r, one(ops), c) for r, ops, c in roles], counts)
+
+
+def test_planted_early_staging_is_caught():
+    """dk/dv: the TMA warp stores tile 2's lse / D before the slot is
+    released, over tile 0's, which the elementwise warps may still read."""
+    def bad(ops):
+        out = list(ops)
+        w = out.index(("wait", "qd_empty0", 0))
+        s = next(i for i, o in enumerate(out) if o[0] == "st" and o[1][0][1] == ("L", 2))
+        out.insert(w, out.pop(s))
+        return out
+    with pytest.raises(bm.Violation, match="race"):
+        bm.explore(*_edit(bm.dkdv_model(3), "tma", bad))
 
 
 def _kernel_barriers(path, struct):
@@ -107,8 +188,8 @@ def test_models_match_the_kernels(src, struct):
     """The models use the kernels' ring depths and name every barrier the
     kernels declare."""
     bars, c = _kernel_barriers(os.path.join(CSRC, src), struct)
-    model = {"Smem": lambda: bm.forward_model(3, qt=c["QT"], stages=c["STAGES"]),
-             "SmemDq": lambda: bm.dq_model(3, kst=c["KST"], vst=c["VST"]),
-             "SmemKv": lambda: bm.dkdv_model(3, stages=c["STAGES"])}[struct]
-    default = {"Smem": bm.forward_model, "SmemDq": bm.dq_model, "SmemKv": bm.dkdv_model}[struct](3)
+    model = {"Smem": lambda: bm.forward_model(3, qt=c["QT"], stages=c["STAGES"], data=False),
+             "SmemDq": lambda: bm.dq_model(3, kst=c["KST"], vst=c["VST"], data=False),
+             "SmemKv": lambda: bm.dkdv_model(3, stages=c["STAGES"], data=False)}[struct]
+    default = {"Smem": bm.forward_model, "SmemDq": bm.dq_model, "SmemKv": bm.dkdv_model}[struct](3, data=False)
     assert bars == set(model()[1]) == set(default[1])
