@@ -136,6 +136,8 @@ typedef struct {
     int debug_checked;                  /* CQSA_DEBUG set: the plan passed the brute-force checks */
     double shard_pairs;                 /* allowed (query, key) pairs of those entries, per head */
     double total_pairs;                 /* allowed pairs of all entries, per head */
+    int64_t cache_q_slots;              /* host mode: device block cache slots for query blocks */
+    int64_t cache_kv_slots;             /* host mode: slots for key blocks (one in the K pool, one in the V pool) */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */
@@ -293,6 +295,24 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info);
  * count.  INVALID_ARG when t is out of range or max_blocks is too small. */
 cqsa_status_t cqsa_plan_task_blocks(const cqsa_plan_t *plan, int64_t t, int64_t *blocks,
                                     int64_t max_blocks, int64_t *num_blocks, int *path);
+
+/* cqsa_plan_cache_task -- the streamed path's device block cache as planned
+ * for leaf task t (replayed for every head group; [B] "Implementation":
+ * stream the blocks a subsequence needs).  Copies issued before the task's
+ * kernel, in order: kinds[i] 0 for a query block (Q pool) or 1 for a key
+ * block (K and V pools, same slot), blocks[i] the global block, slots[i] the
+ * pool slot.  Slots the task's kernel reads, for each of its blocks in
+ * cqsa_plan_task_blocks order: q_slot[m] and kv_slot[m] (-1: not read).
+ * The plan never lets task t's copies evict a block task t - 1 reads (its
+ * kernel may still run); the scheduler makes a copy wait for the kernel of
+ * task t - 2 and, at a head-group boundary, for the previous kernel.
+ * Arrays hold max_copies / max_blocks entries; *num_copies / *num_blocks
+ * get the counts (arrays may be NULL to ask for the counts).  INVALID_ARG
+ * when t is out of range or an array is too small; BUDGET when the plan has
+ * no host-mode sizing. */
+cqsa_status_t cqsa_plan_cache_task(const cqsa_plan_t *plan, int64_t t, int32_t *kinds, int64_t *blocks,
+                                   int32_t *slots, int64_t max_copies, int64_t *num_copies, int32_t *q_slot,
+                                   int32_t *kv_slot, int64_t max_blocks, int64_t *num_blocks);
 
 /* cqsa_plan_entry -- entry i (0 <= i < num_entries) of the work list and its
  * key runs: runs[2r], runs[2r+1] are the first and last global key block of

@@ -41,7 +41,7 @@ EXPORTS = (
     "cqsa_plan_task_blocks", "cqsa_plan_entry", "cqsa_difference_set", "cqsa_plan_debug",
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
-    "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast",
+    "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast", "cqsa_plan_cache_task",
 )
 
 
@@ -73,7 +73,8 @@ class PlanInfo(ctypes.Structure):
                 ("merge", ctypes.c_int), ("H_kv", ctypes.c_int), ("B", ctypes.c_int),
                 ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int), ("shard_entries", ctypes.c_int64),
                 ("debug_checked", ctypes.c_int),
-                ("shard_pairs", ctypes.c_double), ("total_pairs", ctypes.c_double)]
+                ("shard_pairs", ctypes.c_double), ("total_pairs", ctypes.c_double),
+                ("cache_q_slots", ctypes.c_int64), ("cache_kv_slots", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -124,6 +125,11 @@ def load_library():
                                        ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int)]),
         "cqsa_plan_entry": (st, [P, ctypes.c_int64, ctypes.POINTER(Entry), ctypes.POINTER(ctypes.c_int64),
                                  ctypes.c_int64]),
+        "cqsa_plan_cache_task": (st, [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                      ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
         "cqsa_difference_set": (st, [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
         "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
         "cqsa_plan_profile": (st, [P, ctypes.c_int]),
@@ -180,6 +186,25 @@ class Plan:
         buf = (ctypes.c_int64 * max(1, n.value))()
         _check(lib.cqsa_plan_task_blocks(self.handle, t, buf, n.value, ctypes.byref(n), path))
         return list(buf)[: n.value], [p for p in path if p >= 0]
+
+    def cache_task(self, t: int) -> dict:
+        """The streamed path's block-cache plan for leaf task t: the copies
+        issued before its kernel, [(kind, block, slot)] (kind 0: query
+        block, 1: key/value block), and the Q and K/V slot its kernel reads
+        for each of its blocks (task_blocks order; -1: not read)."""
+        lib = load_library()
+        nc, nb = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.cqsa_plan_cache_task(self.handle, t, None, None, None, 0, ctypes.byref(nc), None, None, 0,
+                                        ctypes.byref(nb)))
+        kinds = (ctypes.c_int32 * max(1, nc.value))()
+        blocks = (ctypes.c_int64 * max(1, nc.value))()
+        slots = (ctypes.c_int32 * max(1, nc.value))()
+        qs = (ctypes.c_int32 * max(1, nb.value))()
+        ks = (ctypes.c_int32 * max(1, nb.value))()
+        _check(lib.cqsa_plan_cache_task(self.handle, t, kinds, blocks, slots, nc.value, ctypes.byref(nc), qs, ks,
+                                        nb.value, ctypes.byref(nb)))
+        return {"copies": [(kinds[i], blocks[i], slots[i]) for i in range(nc.value)],
+                "q_slot": list(qs)[: nb.value], "kv_slot": list(ks)[: nb.value]}
 
     def entry(self, i: int):
         lib = load_library()

@@ -1230,6 +1230,40 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->debug_checked = pl.debug_checked ? 1 : 0;
     info->shard_pairs = pl.shard_pairs;
     info->total_pairs = pl.total_pairs;
+    info->cache_q_slots = pl.sizing.q_slots;
+    info->cache_kv_slots = pl.sizing.kv_slots;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_cache_task(const cqsa_plan_t *plan, int64_t t, int32_t *kinds, int64_t *blocks,
+                                   int32_t *slots, int64_t max_copies, int64_t *num_copies, int32_t *q_slot,
+                                   int32_t *kv_slot, int64_t max_blocks, int64_t *num_blocks) {
+    if (!plan || !num_copies || !num_blocks) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    if (t < 0 || t >= (int64_t)pl.leaves.size()) return fail(CQSA_ERR_INVALID_ARG, "task %lld out of range", (long long)t);
+    if (pl.sizing.head_group == 0 || pl.pool.copies.size() != pl.leaves.size())
+        return fail(CQSA_ERR_BUDGET, "no host-mode sizing fits the budget; the plan has no block cache");
+    const std::vector<PoolCopy> &cp = pl.pool.copies[t];
+    const std::vector<int32_t> &qs = pl.pool.q_slot[t], &ks = pl.pool.kv_slot[t];
+    *num_copies = (int64_t)cp.size();
+    *num_blocks = (int64_t)qs.size();
+    if (kinds || blocks || slots) {
+        if (!kinds || !blocks || !slots || max_copies < (int64_t)cp.size())
+            return fail(CQSA_ERR_INVALID_ARG, "copy arrays missing or too small");
+        for (size_t i = 0; i < cp.size(); ++i) {
+            kinds[i] = cp[i].kind;
+            blocks[i] = cp[i].block;
+            slots[i] = cp[i].slot;
+        }
+    }
+    if (q_slot || kv_slot) {
+        if (!q_slot || !kv_slot || max_blocks < (int64_t)qs.size())
+            return fail(CQSA_ERR_INVALID_ARG, "slot arrays missing or too small");
+        for (size_t m = 0; m < qs.size(); ++m) {
+            q_slot[m] = qs[m];
+            kv_slot[m] = ks[m];
+        }
+    }
     return CQSA_OK;
 }
 
