@@ -336,11 +336,14 @@ cqsa_status_t cqsa_plan_debug(cqsa_plan_t *plan, uint64_t timeout_ns, int stall_
  * CQSA_FAULT_ALLOC: the nth following device allocation of the library
  * (plan arenas) fails as if cudaMalloc had run out of memory; kind =
  * CQSA_FAULT_COPY: the nth following host<->device copy of a streamed
- * forward fails.  The failing call returns CQSA_ERR_CUDA without touching
- * the GPU; work already enqueued completes, and the plan stays usable (a
- * failed allocation is retried by the next call).  nth = 0 clears; the
- * setting is process-wide and fires once.  Errors: INVALID_ARG. */
-enum { CQSA_FAULT_ALLOC = 1, CQSA_FAULT_COPY = 2 };
+ * forward fails; kind = CQSA_FAULT_SETUP: the nth following upload of a
+ * plan's tables (work lists, slot counts) into a freshly allocated arena
+ * fails.  The failing call returns CQSA_ERR_CUDA without touching the GPU;
+ * work already enqueued completes, and the plan stays usable (a setup that
+ * failed part-way releases its arena, and the next call sets it up again).
+ * nth = 0 clears; the setting is process-wide and fires once.  Errors:
+ * INVALID_ARG. */
+enum { CQSA_FAULT_ALLOC = 1, CQSA_FAULT_COPY = 2, CQSA_FAULT_SETUP = 3 };
 cqsa_status_t cqsa_debug_inject(int kind, int64_t nth);
 
 /* Per-kernel device time of a plan's launches, from CUDA events recorded

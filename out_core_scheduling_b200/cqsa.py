@@ -25,6 +25,7 @@ CQSA_ERR_NO_DEVICE = 8
 CQSA_ERR_INTERNAL = 9
 CQSA_FAULT_ALLOC = 1
 CQSA_FAULT_COPY = 2
+CQSA_FAULT_SETUP = 3
 
 CQSA_BF16 = 0
 CQSA_FP32 = 1
@@ -412,8 +413,9 @@ def cqsa_partial_cast(plan: Plan, src, dst, stream=None):
 
 
 def cqsa_debug_inject(kind: int, nth: int):
-    """Test hook: the nth following library allocation (CQSA_FAULT_ALLOC)
-    or streamed copy (CQSA_FAULT_COPY) fails on the host; 0 clears."""
+    """Test hook: the nth following library allocation (CQSA_FAULT_ALLOC),
+    streamed copy (CQSA_FAULT_COPY) or plan-table upload (CQSA_FAULT_SETUP)
+    fails on the host; 0 clears."""
     _check(load_library().cqsa_debug_inject(kind, nth))
 
 

@@ -41,9 +41,9 @@ namespace {
 thread_local std::string g_err;
 
 // Host-side fault injection for tests (cqsa_debug_inject): the n-th next
-// device allocation or streamed copy of the library reports a failure
-// instead of calling CUDA.  Process-wide, one-shot.
-std::atomic<int64_t> g_fail_alloc{0}, g_fail_copy{0};
+// device allocation, streamed copy or table upload of the library reports a
+// failure instead of calling CUDA.  Process-wide, one-shot.
+std::atomic<int64_t> g_fail_alloc{0}, g_fail_copy{0}, g_fail_setup{0};
 
 bool injected(std::atomic<int64_t> &c) {
     int64_t v = c.load();
@@ -76,6 +76,12 @@ struct NvtxRange {
 cudaError_t lib_malloc(void **ptr, size_t bytes) {
     if (injected(g_fail_alloc)) return cudaErrorMemoryAllocation;
     return cudaMalloc(ptr, bytes);
+}
+
+// Upload of a plan's tables (work lists, slot counts) into its arena.
+cudaError_t lib_upload(void *dst, const void *src, size_t bytes) {
+    if (injected(g_fail_setup)) return cudaErrorInvalidValue;
+    return cudaMemcpy(dst, src, bytes, cudaMemcpyHostToDevice);
 }
 
 cqsa_status_t fail(cqsa_status_t code, const char *fmt, ...) {
@@ -337,16 +343,26 @@ cqsa_status_t setup_device_mode_impl(cqsa_plan_t *P) {
         P->dev_part_o = reinterpret_cast<float *>(arena + o_po);
         P->dev_part_lse = reinterpret_cast<float *>(arena + o_pl);
         P->dev_nslots = reinterpret_cast<int32_t *>(arena + o_ns);
-        CK(cudaMemcpy(P->dev_nslots, pl.slots_per_block.data(), pl.slots_per_block.size() * sizeof(int32_t),
-                      cudaMemcpyHostToDevice));
+        CK(lib_upload(P->dev_nslots, pl.slots_per_block.data(), pl.slots_per_block.size() * sizeof(int32_t)));
     }
     std::vector<char> buf = pack_wl(wl);
-    if (!buf.empty()) CK(cudaMemcpy(arena + o_wl, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+    if (!buf.empty()) CK(lib_upload(arena + o_wl, buf.data(), buf.size()));
     P->dev_wl = place_wl(arena + o_wl, wl);
     return CQSA_OK;
 }
 
-cqsa_status_t setup_device_mode(cqsa_plan_t *P) { return guarded([&] { return setup_device_mode_impl(P); }); }
+// A setup that fails part-way releases what it took, so that the next call
+// starts it again instead of finding a half-initialised arena.
+cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
+    const cqsa_status_t st = guarded([&] { return setup_device_mode_impl(P); });
+    if (st != CQSA_OK && P->dev_arena) {
+        cudaFree(P->dev_arena);
+        P->dev_arena = nullptr;
+        P->dev_bytes = 0;
+        P->dev_err = nullptr;  // cqsa_plan_sync reads it
+    }
+    return st;
+}
 
 cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     if (P->host_arena) return CQSA_OK;
@@ -404,7 +420,7 @@ cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     }
     for (size_t t = 0; t < pl.leaves.size(); ++t) {
         std::vector<char> buf = pack_wl(wls[t]);
-        if (!buf.empty()) CK(cudaMemcpy(arena + o_wl[t], buf.data(), buf.size(), cudaMemcpyHostToDevice));
+        if (!buf.empty()) CK(lib_upload(arena + o_wl[t], buf.data(), buf.size()));
         P->leaves[t].wl = place_wl(arena + o_wl[t], wls[t]);
     }
     if (P->dtype == CQSA_BF16) {
@@ -428,7 +444,38 @@ cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     return CQSA_OK;
 }
 
-cqsa_status_t setup_host_mode(cqsa_plan_t *P) { return guarded([&] { return setup_host_mode_impl(P); }); }
+void release_host_mode(cqsa_plan_t *P) {
+    for (int s = 0; s < 2; ++s) {
+        cudaEvent_t *evs[4] = {&P->ev_in_ready[s], &P->ev_in_free[s], &P->ev_merged[s], &P->ev_out_free[s]};
+        for (cudaEvent_t *e : evs)
+            if (*e) {
+                cudaEventDestroy(*e);
+                *e = nullptr;
+            }
+    }
+    cudaEvent_t *evs[3] = {&P->ev_start, &P->ev_done_comp, &P->ev_done_out};
+    for (cudaEvent_t *e : evs)
+        if (*e) {
+            cudaEventDestroy(*e);
+            *e = nullptr;
+        }
+    cudaStream_t *ss[3] = {&P->s_in, &P->s_comp, &P->s_out};
+    for (cudaStream_t *s : ss)
+        if (*s) {
+            cudaStreamDestroy(*s);
+            *s = nullptr;
+        }
+    if (P->host_arena) cudaFree(P->host_arena);
+    P->host_arena = nullptr;
+    P->host_bytes = 0;
+    P->h_err = nullptr;  // cqsa_plan_sync reads it
+}
+
+cqsa_status_t setup_host_mode(cqsa_plan_t *P) {
+    const cqsa_status_t st = guarded([&] { return setup_host_mode_impl(P); });
+    if (st != CQSA_OK && P->host_arena) release_host_mode(P);
+    return st;
+}
 
 AttnParams base_params(const cqsa_plan_t *P, int *err) {
     AttnParams ap{};
@@ -520,12 +567,20 @@ cqsa_status_t setup_partial_impl(cqsa_plan_t *P) {
     CK(cudaMemset(arena, 0, a.total));
     P->part_err = reinterpret_cast<int *>(arena + o_err);
     std::vector<char> buf = pack_wl(wl);
-    if (!buf.empty()) CK(cudaMemcpy(arena + o_wl, buf.data(), buf.size(), cudaMemcpyHostToDevice));
+    if (!buf.empty()) CK(lib_upload(arena + o_wl, buf.data(), buf.size()));
     P->part_wl = place_wl(arena + o_wl, wl);
     return CQSA_OK;
 }
 
-cqsa_status_t setup_partial(cqsa_plan_t *P) { return guarded([&] { return setup_partial_impl(P); }); }
+cqsa_status_t setup_partial(cqsa_plan_t *P) {
+    const cqsa_status_t st = guarded([&] { return setup_partial_impl(P); });
+    if (st != CQSA_OK && P->part_arena) {
+        cudaFree(P->part_arena);
+        P->part_arena = nullptr;
+        P->part_err = nullptr;  // cqsa_plan_sync reads it
+    }
+    return st;
+}
 
 // This rank's entries of a sharded plan: every query block it has an entry
 // for is one work-list entry flagged SEG_FIRST only, so the epilogue leaves
@@ -624,24 +679,29 @@ cqsa_status_t setup_backward_impl(cqsa_plan_t *P, BwdState &B, bool shard) {
     if (!fused) {
         B.dq = reinterpret_cast<float *>(arena + o_dq);
         B.q_nslots = reinterpret_cast<int32_t *>(arena + o_qns);
-        CK(cudaMemcpy(B.q_nslots, q_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
+        CK(lib_upload(B.q_nslots, q_ns.data(), pl.num_blocks * sizeof(int32_t)));
     }
     if (kv_slots) {
         B.dk = reinterpret_cast<float *>(arena + o_dk);
         B.dv = reinterpret_cast<float *>(arena + o_dv);
         B.kv_nslots = reinterpret_cast<int32_t *>(arena + o_kvns);
-        CK(cudaMemcpy(B.kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t), cudaMemcpyHostToDevice));
+        CK(lib_upload(B.kv_nslots, kv_ns.data(), pl.num_blocks * sizeof(int32_t)));
     }
     std::vector<char> b1 = pack_wl(qwl), b2 = pack_wl(kvwl);
-    if (!b1.empty()) CK(cudaMemcpy(arena + o_qwl, b1.data(), b1.size(), cudaMemcpyHostToDevice));
-    if (!b2.empty()) CK(cudaMemcpy(arena + o_kvwl, b2.data(), b2.size(), cudaMemcpyHostToDevice));
+    if (!b1.empty()) CK(lib_upload(arena + o_qwl, b1.data(), b1.size()));
+    if (!b2.empty()) CK(lib_upload(arena + o_kvwl, b2.data(), b2.size()));
     B.qwl = place_wl(arena + o_qwl, qwl);
     B.kvwl = place_wl(arena + o_kvwl, kvwl);
     return CQSA_OK;
 }
 
 cqsa_status_t setup_backward(cqsa_plan_t *P, BwdState &B, bool shard) {
-    return guarded([&] { return setup_backward_impl(P, B, shard); });
+    const cqsa_status_t st = guarded([&] { return setup_backward_impl(P, B, shard); });
+    if (st != CQSA_OK && B.arena) {
+        cudaFree(B.arena);
+        B = BwdState{};
+    }
+    return st;
 }
 
 // out_elem: element bytes of dq, dk, dv (the plan's, or 4 for the fp32
@@ -1156,8 +1216,10 @@ cqsa_status_t cqsa_debug_inject(int kind, int64_t nth) {
         g_fail_alloc.store(nth);
     } else if (kind == CQSA_FAULT_COPY) {
         g_fail_copy.store(nth);
+    } else if (kind == CQSA_FAULT_SETUP) {
+        g_fail_setup.store(nth);
     } else {
-        return fail(CQSA_ERR_INVALID_ARG, "kind must be CQSA_FAULT_ALLOC or CQSA_FAULT_COPY");
+        return fail(CQSA_ERR_INVALID_ARG, "kind must be CQSA_FAULT_ALLOC, CQSA_FAULT_COPY or CQSA_FAULT_SETUP");
     }
     return CQSA_OK;
 }

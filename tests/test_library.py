@@ -273,12 +273,12 @@ def test_debug_plan_checks(monkeypatch, args):
 
 
 def test_fault_injection_arguments():
-    for kind, nth in ((0, 1), (3, 1), (cqsa.CQSA_FAULT_ALLOC, -1)):
+    for kind, nth in ((0, 1), (4, 1), (cqsa.CQSA_FAULT_ALLOC, -1), (cqsa.CQSA_FAULT_SETUP, -1)):
         with pytest.raises(cqsa.CqsaError) as ei:
             cqsa.cqsa_debug_inject(kind, nth)
         assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
-    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_ALLOC, 0)
-    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, 0)
+    for kind in (cqsa.CQSA_FAULT_ALLOC, cqsa.CQSA_FAULT_COPY, cqsa.CQSA_FAULT_SETUP):
+        cqsa.cqsa_debug_inject(kind, 0)
 
 
 def test_n_limit():

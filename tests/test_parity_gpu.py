@@ -378,6 +378,49 @@ def test_injected_allocation_failure_is_recoverable():
     check(out, lse, q, k, v, np.arange(N), True)
 
 
+@pytest.mark.parametrize("mode,nth", [("device", 1), ("device", 2), ("host", 1), ("host", 5),
+                                      ("backward", 1), ("backward", 3)])
+def test_injected_setup_failure_is_recoverable(mode, nth):
+    """An upload of the plan's tables fails after its arena was allocated:
+    the call reports CQSA_ERR_CUDA, the half-built arena is released, and
+    the next call sets it up again and is correct."""
+    N, H, d = 13 * 256, 2, 128
+    host = mode == "host"
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=62, host=host)
+    budget = int(_min_budget(N, H, d, [4], True) * 1.3) if host else 0
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True, mem_budget_bytes=budget)
+    m = cqsa.CQSA_HOST if host else cqsa.CQSA_DEVICE
+    if mode == "backward":
+        out, lse = run(plan, q, k, v, m)
+        dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=63, device=DEV)[0]
+        grads = [torch.empty_like(q) for _ in range(3)]
+        call = lambda: cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, *grads)
+    else:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory() if host else torch.empty_like(q)
+        lse = torch.empty(H, N).pin_memory() if host else torch.empty(H, N, device=DEV)
+        call = lambda: cqsa.cqsa_forward(plan, q, k, v, out, lse, m)
+    cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_SETUP, nth)
+    try:
+        with pytest.raises(cqsa.CqsaError) as ei:
+            call()
+        assert ei.value.status == cqsa.CQSA_ERR_CUDA
+    finally:
+        cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_SETUP, 0)
+    plan.sync()
+    if mode == "backward":
+        call()
+        plan.sync()
+        ref = [torch.empty_like(q) for _ in range(3)]
+        plan2 = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True)
+        cqsa.cqsa_backward(plan2, q, k, v, out, lse, dout, *ref)
+        plan2.sync()
+        for a, b in zip(grads, ref):
+            assert torch.equal(a, b)
+    else:
+        out, lse = run(plan, q, k, v, m)
+        check(out, lse, q, k, v, np.arange(N), True)
+
+
 @pytest.mark.parametrize("nth", [1, 7, 40])
 def test_injected_copy_failure_is_recoverable(nth):
     """A host<->device copy of a streamed forward fails part-way: the call
