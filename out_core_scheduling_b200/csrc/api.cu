@@ -806,6 +806,9 @@ cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const v
     CK(cudaStreamWaitEvent(P->s_in, P->ev_start, 0));
     CK(cudaStreamWaitEvent(P->s_comp, P->ev_start, 0));
     CK(cudaStreamWaitEvent(P->s_out, P->ev_start, 0));
+    // The enqueue order below (waits, copies, kernel, records per task) is
+    // modelled in tests/test_stream_schedule.py, which checks it for races
+    // over every interleaving of the three streams.
     int64_t it = 0;
     const size_t blk_stride = (size_t)B;  // pool rows per slot
     for (int h0 = 0; h0 < H; h0 += g) {

@@ -22,6 +22,14 @@ performs them:
     ("ld", reads)         tcgen05.ld / ld.shared by a warp (it waits for
                           the data before going on);
     ("st", writes)        tcgen05.st / st.shared by a warp, likewise.
+    ("ewait", ev, k)      a CUDA stream waiting on an event: blocks until
+                          record k of ``ev`` (its k-th arrival) has
+                          completed; records are not reused by parity, so
+                          neither the early nor the late rule applies;
+    ("begin", reads, writes) / ("end",)
+                          a long operation of a stream (a copy, a kernel):
+                          it holds its regions from begin to end, reads
+                          them at begin and leaves its writes at end.
 
 ``reads`` are (region, version) pairs: the data the step must find there.
 ``writes`` are (region, version) pairs, or (region, expected, version)
@@ -87,6 +95,12 @@ def explore(roles, counts, limit=3_000_000):
             rec = (kind, -1, 0, tuple(o[1]), ())
         elif kind == "st":
             rec = (kind, -1, 0, (), _norm_writes(o[1]))
+        elif kind == "ewait":
+            rec = (kind, bi[o[1]], o[2], (), ())
+        elif kind == "begin":
+            rec = (kind, -1, 0, tuple(o[1]), _norm_writes(o[2]))
+        elif kind == "end":
+            rec = (kind, -1, 0, (), ())
         else:
             raise ValueError(kind)
         for r, _ in rec[3]:
@@ -108,16 +122,18 @@ def explore(roles, counts, limit=3_000_000):
     table = [(k, b, kk, tuple((ri[r], v) for r, v in rd), tuple((ri[r], e, v) for r, e, v in wr))
              for k, b, kk, rd, wr in table]
 
-    def canon(pcs):
-        # warps of one group are interchangeable: sort their pcs
-        out, i = [], 0
+    def canon(pcs, fl):
+        # warps of one group are interchangeable: sort their (pc, in-flight)
+        out, outf, i = [], [], 0
         while i < nw:
             j = i
             while j < nw and flat[j][0] == flat[i][0]:
                 j += 1
-            out.extend(sorted(pcs[i:j]))
+            grp = sorted(zip(pcs[i:j], fl[i:j]))
+            out.extend(p for p, _ in grp)
+            outf.extend(f for _, f in grp)
             i = j
-        return tuple(out)
+        return tuple(out), tuple(outf)
 
     def desc(oid):
         k, b, kk, rd, wr = table[oid]
@@ -181,11 +197,12 @@ def explore(roles, counts, limit=3_000_000):
         return None
 
     nreg = len(regs)
-    start = (tuple([0] * nw), tuple([0] * len(bars)), tuple([0] * len(bars)), (), (), tuple([None] * nreg))
+    start = (tuple([0] * nw), tuple([0] * len(bars)), tuple([0] * len(bars)), (), (), tuple([None] * nreg),
+             tuple([-1] * nw))
     seen = {start}
     todo = deque([start])
     while todo:
-        pcs, done, pend, cq, tq, ver = todo.popleft()
+        pcs, done, pend, cq, tq, ver, fl = todo.popleft()
         succ = []
         finished = True
         for w in range(nw):
@@ -203,24 +220,24 @@ def explore(roles, counts, limit=3_000_000):
                     raise Violation(f"early: {names[w]} waits on phase {k} of {bars[b]} "
                                     f"with only {done[b]} complete")
                 if done[b] == k + 1:
-                    succ.append((npcs, done, pend, cq, tq, ver))
+                    succ.append((npcs, done, pend, cq, tq, ver, fl))
                 elif done[b] > k + 1:
                     raise Violation(f"late: {names[w]} waits on phase {k} of {bars[b]} "
                                     f"after {done[b]} completed")
             elif kind == "arrive":
                 d, p = arrive(npcs, done, pend, b)
-                succ.append((npcs, d, p, cq, tq, ver))
+                succ.append((npcs, d, p, cq, tq, ver, fl))
             elif kind == "commit":
-                succ.append((npcs, done, pend, cq + (-1 - b,), tq, ver))
+                succ.append((npcs, done, pend, cq + (-1 - b,), tq, ver, fl))
             elif kind == "mma":
-                succ.append((npcs, done, pend, cq + (oid,), tq, ver))
+                succ.append((npcs, done, pend, cq + (oid,), tq, ver, fl))
             elif kind == "tma":
                 for r, _, _ in wr:
                     why = busy(cq, tq, r, mma_writes=False)
                     if why:
                         raise Violation(f"race: {names[w]} copies into {regs[r]} while {why}")
                     check_overwrite(npcs, cq, ver, r, f"{names[w]}'s copy")
-                succ.append((npcs, done, pend, cq, tuple(sorted(tq + ((b, oid),))), ver))
+                succ.append((npcs, done, pend, cq, tuple(sorted(tq + ((b, oid),))), ver, fl))
             elif kind == "ld":
                 for r, v in rd:
                     why = busy(cq, tq, r, mma_reads=False)
@@ -228,7 +245,7 @@ def explore(roles, counts, limit=3_000_000):
                         raise Violation(f"race: {names[w]} reads {regs[r]} while {why}")
                     if ver[r] != v:
                         raise Violation(f"stale: {names[w]} reads {regs[r]} expecting {v}, finds {ver[r]}")
-                succ.append((npcs, done, pend, cq, tq, ver))
+                succ.append((npcs, done, pend, cq, tq, ver, fl))
             elif kind == "st":
                 nv = list(ver)
                 for r, e, v in wr:
@@ -239,12 +256,40 @@ def explore(roles, counts, limit=3_000_000):
                         raise Violation(f"stale: {names[w]} stores over {regs[r]} expecting {e}, finds {ver[r]}")
                     check_overwrite(npcs, cq, ver, r, names[w])
                     nv[r] = v
-                succ.append((npcs, done, pend, cq, tq, tuple(nv)))
+                succ.append((npcs, done, pend, cq, tq, tuple(nv), fl))
+            elif kind == "ewait":
+                if done[b] > k:
+                    succ.append((npcs, done, pend, cq, tq, ver, fl))
+            elif kind == "begin":
+                others = [(w2, table[fl[w2]]) for w2 in range(nw) if w2 != w and fl[w2] >= 0]
+                for r, v in rd:
+                    for w2, o2 in others:
+                        if any(rr == r for rr, _, _ in o2[4]):
+                            raise Violation(f"race: {names[w]} reads {regs[r]} while {names[w2]} writes it")
+                    if ver[r] != v:
+                        raise Violation(f"stale: {names[w]} reads {regs[r]} expecting {v}, finds {ver[r]}")
+                for r, e, v in wr:
+                    for w2, o2 in others:
+                        if any(rr == r for rr, _ in o2[3]) or any(rr == r for rr, _, _ in o2[4]):
+                            raise Violation(f"race: {names[w]} writes {regs[r]} while {names[w2]} uses it")
+                    if e is not None and ver[r] != e:
+                        raise Violation(f"stale: {names[w]} writes over {regs[r]} expecting {e}, finds {ver[r]}")
+                    check_overwrite(npcs, cq, ver, r, names[w])
+                nfl = list(fl)
+                nfl[w] = oid
+                succ.append((npcs, done, pend, cq, tq, ver, tuple(nfl)))
+            elif kind == "end":
+                nv = list(ver)
+                for r, _, v in table[fl[w]][4]:
+                    nv[r] = v
+                nfl = list(fl)
+                nfl[w] = -1
+                succ.append((npcs, done, pend, cq, tq, tuple(nv), tuple(nfl)))
         if cq:
             x = cq[0]
             if x < 0:
                 d, p = arrive(pcs, done, pend, -1 - x)
-                succ.append((pcs, d, p, cq[1:], tq, ver))
+                succ.append((pcs, d, p, cq[1:], tq, ver, fl))
             else:
                 _, _, _, rd, wr = table[x]
                 for r, v in rd:
@@ -256,7 +301,7 @@ def explore(roles, counts, limit=3_000_000):
                 for r, e, v in wr:
                     check_overwrite(pcs, cq, ver, r, "an MMA", skip_cq=0)
                     nv[r] = v
-                succ.append((pcs, done, pend, cq[1:], tq, tuple(nv)))
+                succ.append((pcs, done, pend, cq[1:], tq, tuple(nv), fl))
         for i, (b, x) in enumerate(tq):
             if i and tq[i - 1] == (b, x):
                 continue
@@ -264,14 +309,15 @@ def explore(roles, counts, limit=3_000_000):
             for r, _, v in table[x][4]:
                 nv[r] = v
             d, p = arrive(pcs, done, pend, b)
-            succ.append((pcs, d, p, cq, tq[:i] + tq[i + 1:], tuple(nv)))
+            succ.append((pcs, d, p, cq, tq[:i] + tq[i + 1:], tuple(nv), fl))
         if not succ:
             if not finished or cq or tq:
                 stuck = [f"{names[w]}@{desc(flat[w][1][pcs[w]])}" for w in range(nw) if pcs[w] < len(flat[w][1])]
                 raise Violation("deadlock: " + ", ".join(stuck))
             continue
         for s in succ:
-            s = (canon(s[0]),) + s[1:]
+            cp, cf = canon(s[0], s[6])
+            s = (cp,) + s[1:6] + (cf,)
             if s not in seen:
                 seen.add(s)
                 if len(seen) > limit:
