@@ -143,3 +143,20 @@ def test_cache_task_rejects_bad_arguments():
     with pytest.raises(cqsa.CqsaError) as ei:
         plan.cache_task(13)
     assert ei.value.status == cqsa.CQSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("N,H,d,ls,causal", CASES[:4])
+def test_cache_copies_match_planned_h2d_bytes(N, H, d, ls, causal):
+    """The planned host-to-device bytes are the exported copies: a query
+    block moves g heads, a key block g heads of K and of V, for every head
+    group."""
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, mem_budget_bytes=_min_budget(N, H, d, ls, causal))
+    info = plan.info()
+    g, B = info["head_group"], info["block_tokens"]
+    nq = nkv = 0
+    for t in range(info["num_tasks"]):
+        for kind, _, _ in plan.cache_task(t)["copies"]:
+            nq += kind == 0
+            nkv += kind == 1
+    blk = B * g * d * 2  # bf16
+    assert info["h2d_bytes"] == (nq * blk + 2 * nkv * blk) * (H // g)
