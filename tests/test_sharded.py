@@ -245,3 +245,54 @@ def test_plan_rank_must_match_group():
             forward_sharded(plan, x, x, x, x.clone(), torch.zeros(1, 7 * 64), ops=HostOps)
     finally:
         dist.destroy_process_group()
+
+
+def _rank_fail_main(rank, world, port, q):
+    """Rank 1 fails before the exchange; rank 0 enters it."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from out_core_scheduling_b200 import cqsa as lib
+    from out_core_scheduling_b200.inputs import make_qkv
+    from out_core_scheduling_b200.sharded import forward_sharded
+    from test_sharded import HostOps
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    try:
+        N, H, d = 7 * 64, 1, 64
+        qt, kt, vt = make_qkv(N, H, d, dtype=torch.float32, seed=13)
+        plan = lib.cqsa_plan_ex(N, H, d, [3], shard_rank=rank, shard_count=world)
+        if rank == 1:
+            raise RuntimeError("planted failure of rank 1 before the exchange")
+        forward_sharded(plan, qt, kt, vt, torch.empty(N, H, d), torch.empty(H, N), ops=HostOps)
+        q.put((rank, "completed"))
+    except Exception as e:  # report, then leave
+        q.put((rank, type(e).__name__))
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+def test_failed_rank_ends_the_exchange_with_an_error():
+    """A rank that fails before the exchange (host-side, no GPU) makes the
+    other rank's collective end with an error within the process group's
+    timeout instead of waiting for good."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_fail_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode is not None, "a rank did not finish"
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res[1] == "RuntimeError"
+    assert res[0] != "completed"
