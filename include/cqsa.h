@@ -69,6 +69,9 @@ enum { CQSA_DEVICE = 0, CQSA_HOST = 1 };
  *   CQSA_MERGE_SLOTS: every (task, query block) writes its partial O_j and
  *     lse_j to a slot; a merge kernel then takes the log-sum-exp over the
  *     slots.  The tasks' results are materialised as the pages describe.
+ *     At most 32 partials per query block (the merge takes one lane per
+ *     partial): deeper plans (e.g. levels 4, 3, 3: 36) report
+ *     CQSA_ERR_UNSUPPORTED from cqsa_forward and need CQSA_MERGE_FUSED.
  *   CQSA_MERGE_FUSED: one CTA walks the allowed key blocks of all the tasks
  *     of its query rows; its online softmax is the merge, and it writes the
  *     output directly (no slots, no merge launch).

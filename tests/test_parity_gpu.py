@@ -503,3 +503,17 @@ def test_forward_and_backward_in_a_cuda_graph(merge):
         ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, causal=causal)
         g_dq = dq.cpu().double().numpy()
         assert np.abs(g_dq - ref_dq).max() <= 2e-2 * np.abs(ref_dq).max()
+
+
+def test_more_than_32_partials_need_the_fused_recomposition():
+    """Three levels (4, 3, 3) give each query block 36 partials; the slots
+    merge takes one lane per partial, so a slots-mode forward reports
+    CQSA_ERR_UNSUPPORTED before launching anything."""
+    N, H, d = 637 * 4, 1, 64
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3, 3])
+    assert plan.info()["max_slots"] == 36
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=64)
+    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
+    with pytest.raises(cqsa.CqsaError) as ei:
+        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
+    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
