@@ -51,6 +51,10 @@ WORKLOADS = {
         dist="half_normal_uniform_v", budget=2 * GiB),
 }
 DEFAULT_WORKLOAD = "cqs-l4-n53248-h8-d128-bf16-device"
+# Extra keys of the default one-GPU line: one host-streamed workload and the
+# fp32 workload, each measured the same way as its own --workload line.
+STREAMED_EXTRA = "cqs-l6-n2031616-h1-d128-bf16-host-2gib"
+FP32_EXTRA = "cqs-l3-n3584-h1-d64-fp32-device"
 METRIC = "exact-attention TFLOP/s (4*N^2*H*d, halved for causal)"
 
 
@@ -196,13 +200,16 @@ class Dist:
 
 
 # ------------------------------------------------------------ sharded arm
-def run_sharded(args, W):
+def run_sharded(args, W, D=None, workload=None):
     """--shard: ONE problem of the workload split over the ranks (strong
     scaling): every rank plans with shard_rank = its rank, computes its
     (task, query block) entries with cqsa_forward_partial, and the ranks
-    exchange their log-sum-exp partials with two NCCL all-reduces
+    exchange their log-sum-exp partials over NCCL
     (out_core_scheduling_b200.sharded).  Launched without torchrun it runs
-    on a one-process NCCL group.  Device workloads only."""
+    on a one-process NCCL group.  Device workloads only.
+
+    Given D (the default run's ranks, N > 1), it returns the line as a dict
+    and leaves the process group open; otherwise rank 0 prints it."""
     import datetime
     import socket
 
@@ -214,7 +221,9 @@ def run_sharded(args, W):
 
     if W["mode"] != "device":
         raise SystemExit("--shard takes a device workload")
-    D = Dist()
+    nested = D is not None
+    workload = workload or args.workload
+    D = D or Dist()
     dev = D.local_rank
     torch.cuda.set_device(dev)
     torch_dev = f"cuda:{dev}"
@@ -275,7 +284,7 @@ def run_sharded(args, W):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
         "vs_baseline": None, "dtype": W["dtype"], "data": "synthetic (seeded torch.Generator, see inputs.py)",
-        "config": {"workload": args.workload, "N": N, "H": H, "d": d, "l": W["ls"], "causal": W["variants"],
+        "config": {"workload": workload, "N": N, "H": H, "d": d, "l": W["ls"], "causal": W["variants"],
                    "mode": "device, task shards", "parallelism": f"one problem in {world} task shards",
                    "l2": "inputs larger than L2; no flush"},
         "shard": {"rank0_entries": [i["shard_entries"] for i in infos],
@@ -286,6 +295,10 @@ def run_sharded(args, W):
         # attention (none on a rank without entries) + partial init, rescale and finish
         "gpu_launches": sum(s["attn_launches"] for s in stats) + 3 * len(plans) * args.steps,
     }
+    for p in plans:
+        p.destroy()
+    if nested:
+        return line
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist.destroy_process_group()
@@ -293,15 +306,52 @@ def run_sharded(args, W):
 
 # ------------------------------------------------------------------ our arm
 def run_ours(args, W):
+    """The default line: the workload's step, and with the default workload
+    on one GPU also the streamed l=6 workload and the fp32 workload as extra
+    keys ("streamed", "fp32_small"); with N > 1 GPUs the task-sharded step
+    of the same problem as the extra key "sharded"."""
+    import torch
+    from out_core_scheduling_b200 import cqsa
+
+    D = Dist()
+    torch.cuda.set_device(D.local_rank)
+    cqsa.load_library()  # fails loudly when the library is missing
+    result = measure(args, W, D, args.workload, args.steps, args.warmup, extras=True)
+    if result is None:  # --profile-run
+        D.close()
+        return
+    if args.workload == DEFAULT_WORKLOAD and not args.no_extra:
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        if D.world == 1:
+            sub = argparse.Namespace(**vars(args))
+            sub.no_e2e = sub.no_cpu = True
+            result["streamed"] = measure(sub, WORKLOADS[STREAMED_EXTRA], D, STREAMED_EXTRA,
+                                         args.streamed_steps, 3, extras=False)
+            torch.cuda.empty_cache()
+            result["fp32_small"] = measure(sub, WORKLOADS[FP32_EXTRA], D, FP32_EXTRA,
+                                           args.steps, max(3, args.warmup), extras=False)
+        else:
+            result["sharded"] = run_sharded(args, W, D=D, workload=args.workload)
+    if D.rank == 0:
+        print(json.dumps(result), flush=True)
+    D.close()
+
+
+def flush_l2(buf):
+    """Overwrite a buffer larger than L2, so the next launch starts cold."""
+    buf.add_(1)
+
+
+def measure(args, W, D, workload, steps, warmup, extras):
+    """One workload's line (a dict) on this rank's GPU; every rank runs its
+    own independent problem and the step time is the max over ranks."""
     import torch
     from out_core_scheduling_b200 import cqsa
     from out_core_scheduling_b200.inputs import make_qkv
 
-    D = Dist()
     dev = D.local_rank
-    torch.cuda.set_device(dev)
     torch_dev = f"cuda:{dev}"
-    cqsa.load_library()  # fails loudly when the library is missing
     N, H, d = W["N"], W["H"], W["d"]
     tdt = torch.bfloat16 if W["dtype"] == "bf16" else torch.float32
     cdt = cqsa.CQSA_BF16 if W["dtype"] == "bf16" else cqsa.CQSA_FP32
@@ -337,24 +387,29 @@ def run_ours(args, W):
         for p, o, l in zip(plans, outs, lses):
             cqsa.cqsa_forward(p, q, k, v, o, l, mode, stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     for p in plans:
         p.sync(stream)
     free_after, _ = torch.cuda.mem_get_info()
 
     if args.profile_run:
-        for _ in range(args.steps):
+        for _ in range(steps):
             step()
         if args.profile_backward and mode == cqsa.CQSA_DEVICE:
             dout = make_qkv(N, H, d, dtype=tdt, seed=1000 + D.rank, device=q.device, dist=W["dist"])[0]
             grads = tuple(torch.empty_like(q) for _ in range(3))
-            for _ in range(args.steps):  # first variant only: one backward arena on the device
+            for _ in range(steps):  # first variant only: one backward arena on the device
                 cqsa.cqsa_backward(plans[0], q, k, v, outs[0], lses[0], dout, *grads, stream=stream)
         for p in plans:
             p.sync(stream)
-        D.close()
-        return
+        return None
+
+    # Inputs smaller than L2 (the fp32 workload): each timed step starts after
+    # a write of a buffer larger than L2, outside the events that time it.
+    in_bytes = 3 * N * H * d * ebytes
+    flush = (torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=torch_dev).zero_()
+             if mode == cqsa.CQSA_DEVICE and in_bytes <= L2_BYTES else None)
 
     sampler = ClockSampler(gpu_id_for_smi(torch, dev))
     for p in plans:
@@ -362,14 +417,22 @@ def run_ours(args, W):
         p.profile(True)
     sampler.start()
     time.sleep(0.3)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps if flush is not None else 1)]
     D.barrier(dev)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
+    if flush is None:
+        evs[0][0].record(stream)
+        for _ in range(steps):
+            step()
+        evs[0][1].record(stream)
+    else:
+        for e0, e1 in evs:
+            flush_l2(flush)
+            e0.record(stream)
+            step()
+            e1.record(stream)
     torch.cuda.synchronize()
     wall1 = time.perf_counter()
     D.barrier(dev)
@@ -377,10 +440,10 @@ def run_ours(args, W):
     for p in plans:
         p.profile(False)
         p.sync(stream)
-    ms = D.max(ev0.elapsed_time(ev1), torch_dev)
+    ms = D.max(sum(e0.elapsed_time(e1) for e0, e1 in evs), torch_dev)
     stats = [p.kernel_stats(reset=True) for p in plans]
 
-    value = flops_step * args.steps * D.world / (ms * 1e-3) / 1e12
+    value = flops_step * steps * D.world / (ms * 1e-3) / 1e12
     peaks = load_peaks()
 
     # Roofline of the dominant kernel: the tile-attention launch of the first
@@ -394,7 +457,7 @@ def run_ours(args, W):
     if W["mode"] == "device":
         achieved = flops_per_forward / (launch_ms * 1e-3) / 1e12 if launch_ms > 0 else None
     else:  # one launch per task: all the forward's flops over all its launches
-        achieved = flops_per_forward * args.steps / (s0["attn_ms"] * 1e-3) / 1e12 if s0["attn_ms"] else None
+        achieved = flops_per_forward * steps / (s0["attn_ms"] * 1e-3) / 1e12 if s0["attn_ms"] else None
     if W["dtype"] == "bf16":
         # A device-mode launch is timed alone (burst peak); a streamed step
         # runs the tensor cores for seconds (sustained peak).
@@ -405,7 +468,7 @@ def run_ours(args, W):
                     "peak_source": peaks["source"] + (" bf16 dense (sustained)" if sustained
                                                       else " bf16 dense (burst)"),
                     "traffic": (profile_traffic("attn_tc.cu", "attn_tc_l4_n53248_h8_d128.md")
-                                if args.workload == DEFAULT_WORKLOAD else None),
+                                if workload == DEFAULT_WORKLOAD else None),
                     "kernel": f"attn_tc_kernel<{d}> (causal={W['variants'][0]})",
                     "avg_launch_ms": launch_ms}
     else:
@@ -432,20 +495,22 @@ def run_ours(args, W):
     arena = sum(i["device_arena_bytes"] if W["mode"] == "device" else i["host_arena_bytes"] for i in infos)
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": D.world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": W["dtype"], "data": "synthetic (seeded torch.Generator, see inputs.py)",
-        "config": {"workload": args.workload, "N": N, "H": H, "d": d, "l": W["ls"],
+        "config": {"workload": workload, "N": N, "H": H, "d": d, "l": W["ls"],
                    "c": [info["c"] for info in infos[:1]][0], "D": infos[0]["D"],
                    "causal": W["variants"], "mode": W["mode"],
                    "mem_budget_bytes": W["budget"] or None,
                    "parallelism": f"independent problem per GPU x{D.world}",
-                   "l2": f"inputs larger than L2 ({3 * N * H * d * ebytes / 1e6:.0f} MB > 126 MB); no flush"},
+                   "l2": (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB > 126 MB); no flush" if flush is None
+                          else f"inputs {in_bytes / 1e6:.1f} MB < L2: a {flush.numel() * 4 / 1e6:.0f} MB buffer "
+                               "is written before every timed step, outside its events")},
         "roofline": roofline,
         "roofline_merge": merge,
         "clocks": clocks,
         "gpu_launches": attn_launches + merge_launches,
-        "per_variant": [{"causal": c, "tflops_kernel": useful_flops(N, H, d, c) * args.steps
+        "per_variant": [{"causal": c, "tflops_kernel": useful_flops(N, H, d, c) * steps
                          / (s["attn_ms"] * 1e-3) / 1e12 if s["attn_ms"] else None,
                          "attn_ms_per_launch": s["attn_ms"] / max(1, s["attn_launches"]),
                          "merge_ms_per_launch": s["merge_ms"] / max(1, s["merge_launches"])}
@@ -457,10 +522,10 @@ def run_ours(args, W):
 
     # ---- the fused recomposition on the same device inputs (no slots, no
     # merge launch), timed the same way; the headline stays the slots path.
-    if W["mode"] == "device" and not args.no_fused:
+    if W["mode"] == "device" and extras and not args.no_fused:
         result["fused_merge"] = run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, value)
     # ---- the backward of the same problems (device mode).
-    if W["mode"] == "device" and not args.no_backward:
+    if W["mode"] == "device" and extras and not args.no_backward:
         result["backward"] = run_backward(args, W, D, plans, q, k, v, outs, lses, flops_step, stream, peaks)
 
     # ---- end to end through the public API from pinned host memory.
@@ -469,9 +534,9 @@ def run_ours(args, W):
         h2d = int(sum(i["h2d_bytes"] for i in infos))
         d2h = int(sum(i["d2h_bytes"] for i in infos))
         result["e2e"] = {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                         "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps,
+                         "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
                          "path": "cqsa_forward(CQSA_HOST), the timed path itself"}
-        result["streaming"] = streaming_report(W, infos, flops_step, ms / args.steps, peaks,
+        result["streaming"] = streaming_report(W, infos, flops_step, ms / steps, peaks,
                                                free_before, torch)
     elif not args.no_e2e:
         result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream)
@@ -482,10 +547,9 @@ def run_ours(args, W):
         rows = args.cpu_rows or max(8, min(512, int(2.5e11 / (W["H"] * W["N"] * 4 * W["d"]))))
         result["cpu_baseline"] = cpu_baseline(W, q, k, v, rows)
 
-    if D.rank == 0:
-        print(json.dumps(result), flush=True)
-    del plans
-    D.close()
+    for p in plans:
+        p.destroy()
+    return result
 
 
 def run_backward(args, W, D, plans, q, k, v, outs, lses, flops_step, stream, peaks):
@@ -749,6 +813,10 @@ def main(argv=None):
                     help="only warm-up + steps of the device path (for ncu captures)")
     ap.add_argument("--profile-backward", action="store_true",
                     help="with --profile-run: the first variant's backward after the forward steps")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default workload: skip the streamed / fp32 (one GPU) or sharded (N > 1) extra keys")
+    ap.add_argument("--streamed-steps", type=int, default=2,
+                    help="timed steps of the streamed extra workload (about 2 s each)")
     ap.add_argument("--shard", action="store_true",
                     help="one problem split over the ranks in task shards (strong scaling; not the default line)")
     args = ap.parse_args(argv)

@@ -381,21 +381,31 @@ cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *sta
  * memory, a process at its device-memory cap, or a loop that cannot afford
  * cudaMalloc's implicit device synchronisation).
  *   q, k, v, out: device pointers, [N, H, d] in the plan's dtype; lse: fp32
- *   [H, N] on the device.  The caller owns them.  The task partials, work
- *   list and error word live in one file-scope device array of
- *   CQSA_NOALLOC_SCRATCH_BYTES (64 MiB), placed by the module loader on each
- *   device that uses it and held until the process exits.
+ *   [H, N] on the device; all five on the current device, which must be the
+ *   plan's device if the plan was used before.  The caller owns them.  The
+ *   task partials, work list and error word live in one file-scope device
+ *   array of CQSA_NOALLOC_SCRATCH_BYTES (64 MiB) per device, held until the
+ *   process exits.
+ *   Set-up: the first call on a device looks up the array's address
+ *   (cudaGetSymbolAddress), which loads the library's device code there and
+ *   with it reserves the 64 MiB (under lazy module loading, the CUDA
+ *   default, not earlier).  Make that first call early, while 64 MiB are
+ *   still free (it fails with CQSA_ERR_CUDA otherwise), and before any stream
+ *   capture.  Later calls on that device reserve and allocate nothing.
  *   Limits: the plan's partials (max_slots * N * H * d * 4 bytes, plus lse)
  *   and work list must fit the array; otherwise CQSA_ERR_BUDGET with the
- *   sizes in the message, and cqsa_forward is the way.
- *   The first call on a device looks up the array's address
- *   (cudaGetSymbolAddress) and loads the library's device code; make it
- *   before any stream capture.  Calls share the array and keep the last
- *   call's contents; host callers are serialised, but work of two calls that
- *   overlaps on the GPU would race, so the call waits until its own work on
- *   `stream` has finished and then reports CQSA_ERR_TIMEOUT if a bounded
- *   device wait ran out.  Calls no cudaMalloc, cudaFree or other allocating
- *   routine.  Errors: INVALID_ARG, NO_DEVICE, BUDGET, CUDA, TIMEOUT.
+ *   sizes in the message, and cqsa_forward is the way.  A CQSA_MERGE_FUSED
+ *   plan runs as a slots plan here (partials in the array, then the merge),
+ *   so plans with more than 32 partials per query block are refused with
+ *   CQSA_ERR_UNSUPPORTED, as are batched (B > 1), grouped-query and sharded
+ *   plans.
+ *   Calls share the array and keep the last call's contents; host callers
+ *   are serialised, but work of two calls that overlaps on the GPU would
+ *   race, so every call waits until its own work on `stream` has finished
+ *   before returning, and then reports CQSA_ERR_TIMEOUT if a bounded device
+ *   wait ran out.  Calls no cudaMalloc, cudaFree or other allocating
+ *   routine.  Errors: INVALID_ARG, NO_DEVICE, BUDGET, UNSUPPORTED, CUDA,
+ *   TIMEOUT.
  */
 cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, const void *k,
                                    const void *v, void *out, float *lse, void *stream);

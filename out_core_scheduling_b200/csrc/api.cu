@@ -505,6 +505,11 @@ cqsa_status_t check_ptr(const void *p, bool want_host, const char *name) {
     } else {
         if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
             return fail(CQSA_ERR_INVALID_ARG, "%s is not device memory", name);
+        // Device memory of another GPU would be read across devices without
+        // peer access.
+        int dev = -1;
+        if (at.type == cudaMemoryTypeDevice && cudaGetDevice(&dev) == cudaSuccess && at.device != dev)
+            return fail(CQSA_ERR_INVALID_ARG, "%s is on device %d but device %d is current", name, at.device, dev);
     }
     return CQSA_OK;
 }
@@ -936,6 +941,10 @@ cqsa_status_t plan_make_map(CUtensorMap *m, const void *base, int64_t rows, int 
     return make_map(m, base, rows, heads, d);
 }
 cqsa_status_t set_error(cqsa_status_t code, const char *msg) { return fail(code, "%s", msg); }
+// Binds the plan to the current device on first use; INVALID_ARG when the
+// plan is bound to another device.
+cqsa_status_t plan_check_device(cqsa_plan_t *P) { return check_device(P); }
+cqsa_status_t plan_check_ptr(const void *p, const char *name) { return check_ptr(p, false, name); }
 
 }  // namespace cqsa
 

@@ -12,18 +12,27 @@
 // and which stays resident until the process exits.
 //
 // Rules of use (also in include/cqsa.h):
-//   * The first call on a device looks up the array's device address with
-//     cudaGetSymbolAddress (this loads the module's device image); make that
-//     first call before any stream capture.
+//   * The first call on a device is its set-up: it looks up the array's
+//     device address with cudaGetSymbolAddress, which loads this file's
+//     device image and with it reserves the 64 MiB array on that device
+//     (with lazy module loading, the CUDA default, nothing is reserved
+//     before).  Make that first call early, while the device still has the
+//     64 MiB free, and before any stream capture.  From the second call on,
+//     nothing is reserved or allocated.
 //   * Every call shares the one array and leaves its contents behind; calls
 //     whose work overlaps on the GPU race on it.  Host callers are
-//     serialised by a mutex and each call waits for its own work to finish.
+//     serialised by a mutex and each call waits for its own work to finish
+//     before it returns.
 //   * Problems whose partials and work list exceed the array are rejected
 //     with CQSA_ERR_BUDGET; nothing in this file calls cudaMalloc, cudaFree
 //     or any allocating routine.
+//   * A CQSA_MERGE_FUSED plan runs here as a slots plan (partials in the
+//     array, then the merge kernel), so a plan with more than 32 partials
+//     per query block is rejected with CQSA_ERR_UNSUPPORTED.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -41,6 +50,8 @@ int plan_dtype(const cqsa_plan_t *P);
 uint64_t plan_timeout_ns(const cqsa_plan_t *P);
 cqsa_status_t plan_make_map(CUtensorMap *m, const void *base, int64_t rows, int heads, int d);
 cqsa_status_t set_error(cqsa_status_t code, const char *msg);
+cqsa_status_t plan_check_device(cqsa_plan_t *P);
+cqsa_status_t plan_check_ptr(const void *p, const char *name);
 }  // namespace cqsa
 
 using namespace cqsa;
@@ -145,19 +156,20 @@ void write_list(const Planner &pl, int rows_per_unit, int bn, const ListSizes &n
                 if (nt > 0 && u < n.units) U[u++] = WlUnit{(int32_t)i, q0, h, nt};
             }
     }
-}
-
-cqsa_status_t check_dev_ptr(const void *p, const char *name) {
-    if (!p) return err(CQSA_ERR_INVALID_ARG, "%s is null", name);
-    cudaPointerAttributes at;
-    cudaError_t e = cudaPointerGetAttributes(&at, p);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return err(CQSA_ERR_INVALID_ARG, "%s: %s", name, cudaGetErrorString(e));
-    }
-    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
-        return err(CQSA_ERR_INVALID_ARG, "%s is not device memory", name);
-    return CQSA_OK;
+    // The launch order of cqsa_forward's device path: longest units first in
+    // classes of 32 key tiles (a short grid tail), then by head and task so
+    // the CTAs in flight share key/value blocks in L2.  Ties keep the order
+    // written above (entry, head, row), which std::sort, unlike
+    // std::stable_sort, does without a temporary buffer.
+    std::sort(U, U + u, [&](const WlUnit &a, const WlUnit &b) {
+        const int ca = a.ntiles / 32, cb = b.ntiles / 32;
+        if (ca != cb) return ca > cb;
+        if (a.head != b.head) return a.head < b.head;
+        const int64_t ta = pl.entries[a.entry].task, tb = pl.entries[b.entry].task;
+        if (ta != tb) return ta < tb;
+        if (a.entry != b.entry) return a.entry < b.entry;
+        return a.q0 < b.q0;
+    });
 }
 
 }  // namespace
@@ -166,16 +178,12 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
                                               void *out, float *lse, void *stream) {
     if (!plan) return err(CQSA_ERR_INVALID_ARG, "null plan");
     std::lock_guard<std::mutex> lock(g_mu);
+    // An sm_100 device is current and the plan is bound to it (a plan used
+    // before on another device is refused).
+    cqsa_status_t dst = plan_check_device(plan);
+    if (dst != CQSA_OK) return dst;
     int dev = -1;
-    cudaError_t ce = cudaGetDevice(&dev);
-    if (ce != cudaSuccess) {
-        cudaGetLastError();
-        return err(CQSA_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(ce));
-    }
-    int major = 0, minor = 0;
-    NA_CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
-    NA_CK(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
-    if (major != 10 || minor != 0) return err(CQSA_ERR_NO_DEVICE, "device %d is not sm_100", dev);
+    NA_CK(cudaGetDevice(&dev));
     if (dev >= kMaxDevices) return err(CQSA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
 
     const Planner &pl = plan_planner(plan);
@@ -209,7 +217,7 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     const void *ptrs[5] = {q, k, v, out, lse};
     const char *names[5] = {"q", "k", "v", "out", "lse"};
     for (int i = 0; i < 5; ++i) {
-        cqsa_status_t st = check_dev_ptr(ptrs[i], names[i]);
+        cqsa_status_t st = plan_check_ptr(ptrs[i], names[i]);  // device memory of the current device
         if (st != CQSA_OK) return st;
     }
 
@@ -261,10 +269,11 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     }
     NA_CK(launch_merge_slots(d, elem, part_o, part_lse, nslots, pl.block, N, H, out, lse, s));
 
-    // The error word is only valid once this call's work is done.
-    NA_CK(cudaStreamSynchronize(s));
+    // The error word is only valid once this call's work is done; it is read
+    // on the call's own stream, not the legacy default stream.
     int word = 0;
-    NA_CK(cudaMemcpy(&word, err_word, sizeof word, cudaMemcpyDeviceToHost));
+    NA_CK(cudaMemcpyAsync(&word, err_word, sizeof word, cudaMemcpyDeviceToHost, s));
+    NA_CK(cudaStreamSynchronize(s));
     if (word)
         return err(CQSA_ERR_TIMEOUT, "a bounded device-side wait ran out (code %d, in the allocation-free forward)", word);
     return CQSA_OK;

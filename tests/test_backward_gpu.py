@@ -14,7 +14,7 @@ import torch
 
 import oracle
 from out_core_scheduling_b200 import cqsa
-from out_core_scheduling_b200.inputs import make_qkv
+from out_core_scheduling_b200.inputs import make_qkv, sample_rows
 
 from parity import run
 
@@ -172,3 +172,60 @@ def test_backward_batch_of_sequences(causal):
         _compare(dq[b], ref_dq, torch.bfloat16, "dq")
         _compare(dk[b], ref_dk, torch.bfloat16, "dk")
         _compare(dv[b], ref_dv, torch.bfloat16, "dv")
+
+
+def _longest_entry_tiles(plan):
+    """Key tiles of 128 rows that the longest (task, query block) entry walks."""
+    info = plan.info()
+    tiles = 0
+    for i in range(info["num_entries"]):
+        e = plan.entry(i)
+        blocks = sum(b - a + 1 for a, b in e["runs"])
+        tiles = max(tiles, blocks * info["block_tokens"] // 128)
+    return tiles
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_full_size_dq_sampled_rows(causal):
+    """l=4, N=53248, H=8, d=128: dq of 256 seeded query rows against the fp64
+    oracle, every head.  A unit here walks 96 to 128 key tiles (416 with the
+    fused recomposition), so the gradient kernels' K/V rings and every
+    barrier phase wrap many times, unlike the small cases above."""
+    N, H, d = 53248, 8, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
+    dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=1000, device=DEV)[0]
+    rows = sample_rows(N)
+    qc, kc, vc, dc = (x.cpu() for x in (q, k, v, dout))
+    ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, rows=rows.numpy(), causal=causal)
+    for merge in (cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED):
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, merge=merge)
+        assert _longest_entry_tiles(plan) >= 96
+        dq, _, _ = _grads(plan, q, k, v, dout)
+        _compare(dq[rows.to(DEV)], ref_dq, torch.bfloat16, f"dq merge={merge}")
+        plan.destroy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_long_units_dkdv_sampled_keys(causal):
+    """l=4, N=13*2048, H=2, d=128: dk and dv of 256 seeded key rows against
+    the fp64 oracle (which needs every row's lse, so the size is the largest
+    whose full-lse pass stays within seconds on the host), and dq of 256
+    rows.  Units walk 48 to 64 tiles of 128 (fused: 208), so the key-
+    stationary kernel's Q/dO ring wraps many times."""
+    N, H, d = 13 * 2048, 2, 128
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=5, device=DEV)
+    dout = make_qkv(N, H, d, dtype=torch.bfloat16, seed=1005, device=DEV)[0]
+    keys = sample_rows(N, seed=4321)
+    rows = sample_rows(N)
+    qc, kc, vc, dc = (x.cpu() for x in (q, k, v, dout))
+    ref_dk, ref_dv = oracle.attention_backward_dkdv(qc, kc, vc, dc, keys=keys.numpy(), causal=causal)
+    ref_dq, _, _ = oracle.attention_backward_dq(qc, kc, vc, dc, rows=rows.numpy(), causal=causal)
+    for merge in (cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED):
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, merge=merge)
+        assert _longest_entry_tiles(plan) >= 48
+        dq, dk, dv = _grads(plan, q, k, v, dout)
+        kd = keys.to(DEV)
+        _compare(dk[kd], ref_dk, torch.bfloat16, f"dk merge={merge}")
+        _compare(dv[kd], ref_dv, torch.bfloat16, f"dv merge={merge}")
+        _compare(dq[rows.to(DEV)], ref_dq, torch.bfloat16, f"dq merge={merge}")
+        plan.destroy()

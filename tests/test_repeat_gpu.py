@@ -7,11 +7,13 @@ size make likely within a few hundred calls (the dq kernel's former shared
 P-half / P-full pair hung about one call in 250 at l = 4, N = 53248).  The
 exhaustive check of the hand-offs is the CPU model in barrier_model.py;
 this is its end-to-end counterpart on the device."""
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from out_core_scheduling_b200 import cqsa
-from out_core_scheduling_b200.inputs import make_qkv
+from out_core_scheduling_b200.inputs import make_qkv, sample_rows
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -44,3 +46,13 @@ def test_repeated_forward_and_backward(causal):
     _repeat(plan, lambda: cqsa.cqsa_backward(plan, q, k, v, out, lse, dout, *g), 300)
     for a, b in zip(g, g0):
         assert torch.equal(a, b)
+    # ... and the repeated result is the right one: dq of 64 seeded rows
+    # against the fp64 oracle (bf16 gradient tolerance, relative to the
+    # largest reference entry).
+    rows = sample_rows(N, 64, seed=77)
+    ref, _, _ = oracle.attention_backward_dq(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), rows=rows.numpy(),
+                                             causal=causal)
+    got = g[0][rows.to(DEV)].cpu().double().numpy()
+    err = np.abs(got - ref)
+    assert err.max() <= 2e-2 * np.abs(ref).max()
+    assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref)
