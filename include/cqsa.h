@@ -141,6 +141,13 @@ typedef struct {
     double total_pairs;                 /* allowed pairs of all entries, per head */
     int64_t cache_q_slots;              /* host mode: device block cache slots for query blocks */
     int64_t cache_kv_slots;             /* host mode: slots for key blocks (one in the K pool, one in the V pool) */
+    int bwd_head_group;                 /* host-mode backward: heads per group (0: none fits the budget) */
+    size_t bwd_host_arena_bytes;        /* arena of a host-mode backward (<= budget) */
+    int64_t bwd_cache_slots;            /* host-mode backward: block slots of its device cache */
+    size_t bwd_h2d_bytes;               /* planned host->device bytes of one host-mode backward */
+    size_t bwd_d2h_bytes;               /* planned device->host bytes of one host-mode backward */
+    size_t bwd_spill_host_bytes;        /* pinned host memory the host-mode backward takes for written-back sums */
+    int64_t bwd_writebacks;             /* gradient-sum write-backs per head group (0: every block stays cached) */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */
@@ -208,13 +215,30 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,
  * the exact gradients.
  *   Layouts: q, k, v, out, dout, dq, dk, dv [N, H, d] contiguous in the plan
  *     dtype; lse fp32 [H, N] as cqsa_forward wrote it.  The caller owns all.
- *   host_or_device: CQSA_DEVICE only (all ten pointers on the current
- *     device); CQSA_HOST returns UNSUPPORTED.
+ *   host_or_device = CQSA_DEVICE: all ten pointers on the current device.
+ *   host_or_device = CQSA_HOST: all ten are page-locked host pointers, and
+ *     the backward runs within the plan's mem_budget_bytes ([A]: forward and
+ *     backward past the memory limit; [B] "Precise Scaling": the backward's
+ *     peak memory).  Per group of cqsa_plan_info().bwd_head_group heads, the
+ *     lse rows are copied up and D = rowsum(dout * out) is formed block by
+ *     block; then the leaf tasks run in order, each bringing its missing
+ *     blocks' Q, K, V, dout rows into a device block cache and adding its
+ *     pairs' gradient terms into fp32 running sums kept beside them; a
+ *     block's sums leave as the finished gradients after its last task.  When
+ *     the cache holds fewer blocks than the sequence, an evicted block's sums
+ *     are written back to pinned host memory the plan allocates
+ *     (bwd_spill_host_bytes, not counted in the budget) and brought back for
+ *     its next task (cqsa_plan_bwd_cache_task).  The first host-mode call
+ *     allocates the backward's arena (bwd_host_arena_bytes); when the
+ *     streamed forward's arena and this one would exceed the budget together,
+ *     the other one is released first (and set up again by its next call).
+ *     Grouped-query plans (H_kv < H) return UNSUPPORTED in this mode.
  *   CQSA_MERGE_SLOTS plans write each (task, query block) dq partial and
  *     each (task, key block) dk / dv partial to slots of a backward arena
  *     (allocated on the first call) and sum them; CQSA_MERGE_FUSED plans
  *     walk all the tasks of a block in one CTA and write dq, dk, dv directly.
- * Asynchronous on stream.  Errors: INVALID_ARG, UNSUPPORTED, CUDA, NO_DEVICE.
+ * Asynchronous on stream.  Errors: INVALID_ARG, NOT_PINNED, BUDGET,
+ * UNSUPPORTED, CUDA, NO_DEVICE.
  */
 cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
                             const void *out, const float *lse, const void *dout, void *dq, void *dk,
@@ -316,6 +340,26 @@ cqsa_status_t cqsa_plan_task_blocks(const cqsa_plan_t *plan, int64_t t, int64_t 
 cqsa_status_t cqsa_plan_cache_task(const cqsa_plan_t *plan, int64_t t, int32_t *kinds, int64_t *blocks,
                                    int32_t *slots, int64_t max_copies, int64_t *num_copies, int32_t *q_slot,
                                    int32_t *kv_slot, int64_t max_blocks, int64_t *num_blocks);
+
+/* cqsa_plan_bwd_cache_task -- the host-mode backward's device block cache as
+ * planned for leaf task t (replayed for every head group).  A slot holds one
+ * block's Q, K, V and dO rows and its running dQ, dK, dV sums.  Copies issued
+ * before the task's kernels, in order: block blocks[i] goes into slot
+ * slots[i]; evicts[i] is the unfinished block whose sums are first written
+ * back to host memory from that slot (-1: none); reloads[i] is 1 when the
+ * block's sums come back from host memory, 0 when they start at zero.
+ * member_slot[m]: the slot of the task's m-th block (cqsa_plan_task_blocks
+ * order; -1 when the backward does not use it).  fin_blocks[j] /
+ * fin_slots[j]: the blocks whose last task is t; after its kernels their
+ * sums become the gradients (plan dtype) and go to the host.  The plan keeps
+ * the blocks of task t - 1, and the slots of blocks it finished, out of task
+ * t's copies.  Arrays may be NULL to ask for the counts.  INVALID_ARG when t
+ * is out of range or an array is too small; BUDGET when no host-mode
+ * backward fits the budget. */
+cqsa_status_t cqsa_plan_bwd_cache_task(const cqsa_plan_t *plan, int64_t t, int64_t *blocks, int32_t *slots,
+                                       int64_t *evicts, int32_t *reloads, int64_t max_copies, int64_t *num_copies,
+                                       int32_t *member_slot, int64_t max_blocks, int64_t *num_blocks,
+                                       int64_t *fin_blocks, int32_t *fin_slots, int64_t max_fin, int64_t *num_fin);
 
 /* cqsa_plan_entry -- entry i (0 <= i < num_entries) of the work list and its
  * key runs: runs[2r], runs[2r+1] are the first and last global key block of

@@ -43,6 +43,7 @@ EXPORTS = (
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
     "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast", "cqsa_plan_cache_task",
+    "cqsa_plan_bwd_cache_task",
 )
 
 
@@ -75,7 +76,11 @@ class PlanInfo(ctypes.Structure):
                 ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int), ("shard_entries", ctypes.c_int64),
                 ("debug_checked", ctypes.c_int),
                 ("shard_pairs", ctypes.c_double), ("total_pairs", ctypes.c_double),
-                ("cache_q_slots", ctypes.c_int64), ("cache_kv_slots", ctypes.c_int64)]
+                ("cache_q_slots", ctypes.c_int64), ("cache_kv_slots", ctypes.c_int64),
+                ("bwd_head_group", ctypes.c_int), ("bwd_host_arena_bytes", ctypes.c_size_t),
+                ("bwd_cache_slots", ctypes.c_int64), ("bwd_h2d_bytes", ctypes.c_size_t),
+                ("bwd_d2h_bytes", ctypes.c_size_t), ("bwd_spill_host_bytes", ctypes.c_size_t),
+                ("bwd_writebacks", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -131,6 +136,13 @@ def load_library():
                                       ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
                                       ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                       ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
+        "cqsa_plan_bwd_cache_task": (st, [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                          ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64),
+                                          ctypes.POINTER(ctypes.c_int32), ctypes.c_int64,
+                                          ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                          ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                          ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                          ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
         "cqsa_difference_set": (st, [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
         "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
         "cqsa_plan_profile": (st, [P, ctypes.c_int]),
@@ -206,6 +218,29 @@ class Plan:
                                         nb.value, ctypes.byref(nb)))
         return {"copies": [(kinds[i], blocks[i], slots[i]) for i in range(nc.value)],
                 "q_slot": list(qs)[: nb.value], "kv_slot": list(ks)[: nb.value]}
+
+    def bwd_cache_task(self, t: int) -> dict:
+        """The host-mode backward's block-cache plan for leaf task t: copies
+        [(block, slot, evicted block or -1, reload)], the slot of each of its
+        blocks (task_blocks order; -1: unused), and the blocks it finishes
+        [(block, slot)]."""
+        lib = load_library()
+        nc, nb, nf = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.cqsa_plan_bwd_cache_task(self.handle, t, None, None, None, None, 0, ctypes.byref(nc), None, 0,
+                                            ctypes.byref(nb), None, None, 0, ctypes.byref(nf)))
+        blocks = (ctypes.c_int64 * max(1, nc.value))()
+        slots = (ctypes.c_int32 * max(1, nc.value))()
+        evicts = (ctypes.c_int64 * max(1, nc.value))()
+        reloads = (ctypes.c_int32 * max(1, nc.value))()
+        ms = (ctypes.c_int32 * max(1, nb.value))()
+        fb = (ctypes.c_int64 * max(1, nf.value))()
+        fs = (ctypes.c_int32 * max(1, nf.value))()
+        _check(lib.cqsa_plan_bwd_cache_task(self.handle, t, blocks, slots, evicts, reloads, nc.value,
+                                            ctypes.byref(nc), ms, nb.value, ctypes.byref(nb), fb, fs, nf.value,
+                                            ctypes.byref(nf)))
+        return {"copies": [(blocks[i], slots[i], evicts[i], reloads[i]) for i in range(nc.value)],
+                "member_slot": list(ms)[: nb.value],
+                "finals": [(fb[j], fs[j]) for j in range(nf.value)]}
 
     def entry(self, i: int):
         lib = load_library()
@@ -320,8 +355,10 @@ def cqsa_backward(plan: Plan, q, k, v, out, lse, dout, dq, dk, dv, host_or_devic
                   stream=None):
     """Gradients dq, dk, dv of the planned attention given the forward's out
     and lse and the output gradient dout.  q, out, dout, dq: [N, H, d];
-    k, v, dk, dv: [N, H_kv, d]; contiguous device tensors in the plan's dtype;
-    lse fp32 [H, N].  Asynchronous on ``stream``."""
+    k, v, dk, dv: [N, H_kv, d]; contiguous tensors in the plan's dtype;
+    lse fp32 [H, N].  CQSA_DEVICE: device tensors.  CQSA_HOST: pinned host
+    tensors, streamed through the plan's device memory budget.
+    Asynchronous on ``stream``."""
     _check_shapes(plan, (("q", q), ("out", out), ("dout", dout), ("dq", dq)),
                   (("k", k), ("v", v), ("dk", dk), ("dv", dv)), lse)
     _check(load_library().cqsa_backward(plan.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),

@@ -209,6 +209,27 @@ struct LeafState {
     std::vector<MergeSeg> host_segs;  // query blocks of the task; SEG_LAST ones are copied out after it
 };
 
+// Streamed (host-mode) backward: its arena, block cache and streams (see
+// Planner::plan_bwd_cache).
+struct BwdHostState {
+    char *arena = nullptr;
+    size_t bytes = 0;
+    int g = 0;
+    int *err = nullptr;
+    float *lse = nullptr, *delta = nullptr;   // [g][N] of the current head group
+    char *stage_o[2] = {}, *stage_do[2] = {}; // O and dO rows of one block, two stages ([block][g][d])
+    char *pool[4] = {};                       // Q, K, V, dO block caches ([slots * block][g][d])
+    float *acc[3] = {};                       // dQ, dK, dV sums ([slots * block][g][d] fp32)
+    std::vector<DevWl> qwl, kvwl;             // per leaf task, cache coordinates
+    CUtensorMap mq, mk, mv, mdo;
+    float *spill = nullptr;                   // pinned host [3][N][g][d] fp32, when the plan writes back
+    cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> ev_slot_free;    // per slot: its write-back or gradient copy-out is done
+    std::vector<cudaEvent_t> ev_spill;        // per block: its last write-back has landed in host memory
+    cudaEvent_t ev_in_ready[2] = {}, ev_comp[2] = {}, ev_stage_ready[2] = {}, ev_stage_free[2] = {};
+    cudaEvent_t ev_start = nullptr, ev_group = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
+};
+
 }  // namespace
 
 struct cqsa_plan {
@@ -230,6 +251,8 @@ struct cqsa_plan {
     // Backward (device mode): the plan's own, and this rank's share of a
     // sharded plan (cqsa_backward_partial).
     BwdState bwd, bwd_shard;
+    // Backward from pinned host memory (host mode).
+    BwdHostState bh;
 
     // Sharded forward (cqsa_forward_partial): this rank's work list.
     char *part_arena = nullptr;
@@ -364,6 +387,8 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
     return st;
 }
 
+void release_bwd_host(cqsa_plan_t *P);
+
 cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     if (P->host_arena) return CQSA_OK;
     const Planner &pl = P->pl;
@@ -371,6 +396,8 @@ cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     if (g <= 0)
         return fail(CQSA_ERR_BUDGET, "no head group of the streamed path fits the budget of %zu bytes",
                     pl.spec.budget);
+    // The streamed backward's arena and this one may not both fit the budget.
+    if (P->bh.arena && pl.spec.budget && P->bh.bytes + pl.sizing.host_arena > pl.spec.budget) release_bwd_host(P);
     const int64_t N = pl.spec.N, R = pl.max_task_rows;
     const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
     const size_t blk = (size_t)pl.block * g * dd * e;
@@ -553,8 +580,8 @@ cqsa_status_t forward_device(cqsa_plan_t *P, const void *q, const void *k, const
     }
     if (fused) return CQSA_OK;
     LaunchTimer tm(P, stream, 1);
-    CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H, out, lse,
-                          stream));
+    CK(launch_merge_slots(d, P->elem, P->dev_part_o, P->dev_part_lse, P->dev_nslots, pl.block, N, H,
+                          (int)pl.max_slots, out, lse, stream));
     tm.stop();
     return CQSA_OK;
 }
@@ -727,7 +754,7 @@ cqsa_status_t backward_device(cqsa_plan_t *P, BwdState &B, bool shard, const voi
         if ((st = make_map(&mv, v, N, pl.spec.Hkv, d)) != CQSA_OK) return st;
         if ((st = make_map(&mo, dout, N, H, d)) != CQSA_OK) return st;
     }
-    CK(launch_bwd_delta(d, P->elem, out, dout, N, H, B.delta, stream));
+    CK(launch_bwd_delta(d, P->elem, out, dout, N, H, B.delta, N, stream));
     BwdParams bp{};
     bp.q = q;
     bp.k = k;
@@ -909,6 +936,323 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
     cudaStreamWaitEvent(stream, P->ev_start, 0);
     cudaStreamWaitEvent(stream, P->ev_done_comp, 0);
     cudaStreamWaitEvent(stream, P->ev_done_out, 0);
+}
+
+// ------------------------------------------------------------ streamed backward
+// The backward from pinned host memory under the plan's memory budget
+// ([A]: forward and backward beyond the memory limit; [B] "Precise
+// Scaling": the backward's peak memory).  Per head group: lse rows up, D =
+// rowsum(dO * O) block by block, then the leaf tasks in order, each adding
+// its pairs' gradient terms into the running sums of its blocks' cache
+// slots; a block's finished sums go back to the host after its last task.
+
+void release_bwd_host(cqsa_plan_t *P) {
+    BwdHostState &S = P->bh;
+    cudaStream_t ss[3] = {S.s_in, S.s_comp, S.s_out};
+    for (cudaStream_t st : ss)
+        if (st) cudaStreamSynchronize(st);
+    for (cudaEvent_t ev : S.ev_slot_free)
+        if (ev) cudaEventDestroy(ev);
+    for (cudaEvent_t ev : S.ev_spill)
+        if (ev) cudaEventDestroy(ev);
+    for (int i = 0; i < 2; ++i) {
+        cudaEvent_t evs[4] = {S.ev_in_ready[i], S.ev_comp[i], S.ev_stage_ready[i], S.ev_stage_free[i]};
+        for (cudaEvent_t ev : evs)
+            if (ev) cudaEventDestroy(ev);
+    }
+    cudaEvent_t evs[4] = {S.ev_start, S.ev_group, S.ev_done_comp, S.ev_done_out};
+    for (cudaEvent_t ev : evs)
+        if (ev) cudaEventDestroy(ev);
+    for (cudaStream_t st : ss)
+        if (st) cudaStreamDestroy(st);
+    if (S.arena) cudaFree(S.arena);
+    if (S.spill) cudaFreeHost(S.spill);
+    S = BwdHostState{};
+}
+
+cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
+    BwdHostState &S = P->bh;
+    if (S.arena) return CQSA_OK;
+    const Planner &pl = P->pl;
+    const BwdSizing &z = pl.bwd_sizing;
+    if (pl.spec.kv_group() != 1)
+        return fail(CQSA_ERR_UNSUPPORTED, "the streamed backward takes as many key/value heads as query heads "
+                                          "(H_kv = %d, H = %d); use device mode", pl.spec.Hkv, pl.spec.H);
+    if (z.head_group <= 0)
+        return fail(CQSA_ERR_BUDGET, "no head group of the streamed backward fits the budget of %zu bytes "
+                                     "(needs %lld block slots)", pl.spec.budget, (long long)pl.bwd_min_slots);
+    // The streamed forward's arena and this one may not both fit the budget.
+    if (P->host_arena && pl.spec.budget && P->host_bytes + z.arena > pl.spec.budget) {
+        cudaStream_t ss[3] = {P->s_in, P->s_comp, P->s_out};
+        for (cudaStream_t st : ss)
+            if (st) CK(cudaStreamSynchronize(st));
+        release_host_mode(P);
+    }
+    const int g = z.head_group;
+    const BwdCachePlan &cp = pl.bwd_cache;
+    const int64_t N = pl.spec.N;
+    const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
+    const size_t rows = (size_t)cp.slots * pl.block;
+    const int tile = P->dtype == CQSA_BF16 ? 128 : 64;
+    // Same layout steps as Planner::bwd_arena_bytes.
+    ArenaLayout a;
+    const size_t o_err = a.take(256);
+    const size_t o_lse = a.take((size_t)g * N * sizeof(float));
+    const size_t o_delta = a.take((size_t)g * N * sizeof(float));
+    size_t o_st[4], o_pool[4], o_acc[3];
+    for (int i = 0; i < 4; ++i) o_st[i] = a.take((size_t)pl.block * g * dd * e);
+    for (int i = 0; i < 4; ++i) o_pool[i] = a.take(rows * g * dd * e);
+    for (int i = 0; i < 3; ++i) o_acc[i] = a.take(rows * g * dd * sizeof(float));
+    const size_t T = pl.leaves.size();
+    std::vector<WorkList> qw(T), kw(T);
+    std::vector<size_t> o_qw(T), o_kw(T);
+    for (size_t t = 0; t < T; ++t) {
+        qw[t] = pl.leaf_bwd_q_worklist((int64_t)t, cp, tile, tile, g);
+        kw[t] = pl.leaf_bwd_kv_worklist((int64_t)t, cp, tile, tile, g);
+        o_qw[t] = a.take(wl_region(qw[t]));
+        o_kw[t] = a.take(wl_region(kw[t]));
+    }
+    if (a.total != z.arena)
+        return fail(CQSA_ERR_INTERNAL, "internal: streamed backward arena layout mismatch (%zu vs %zu)", a.total,
+                    z.arena);
+    char *arena = nullptr;
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
+    S.arena = arena;
+    S.bytes = a.total;
+    S.g = g;
+    // Zeroed once, so rows a partial tile reads past a short block are finite.
+    CK(cudaMemset(arena, 0, a.total));
+    S.err = reinterpret_cast<int *>(arena + o_err);
+    S.lse = reinterpret_cast<float *>(arena + o_lse);
+    S.delta = reinterpret_cast<float *>(arena + o_delta);
+    for (int i = 0; i < 2; ++i) {
+        S.stage_o[i] = arena + o_st[2 * i];
+        S.stage_do[i] = arena + o_st[2 * i + 1];
+    }
+    for (int i = 0; i < 4; ++i) S.pool[i] = arena + o_pool[i];
+    for (int i = 0; i < 3; ++i) S.acc[i] = reinterpret_cast<float *>(arena + o_acc[i]);
+    S.qwl.resize(T);
+    S.kvwl.resize(T);
+    for (size_t t = 0; t < T; ++t) {
+        std::vector<char> b1 = pack_wl(qw[t]), b2 = pack_wl(kw[t]);
+        if (!b1.empty()) CK(lib_upload(arena + o_qw[t], b1.data(), b1.size()));
+        if (!b2.empty()) CK(lib_upload(arena + o_kw[t], b2.data(), b2.size()));
+        S.qwl[t] = place_wl(arena + o_qw[t], qw[t]);
+        S.kvwl[t] = place_wl(arena + o_kw[t], kw[t]);
+    }
+    if (P->dtype == CQSA_BF16) {
+        cqsa_status_t st;
+        CUtensorMap *maps[4] = {&S.mq, &S.mk, &S.mv, &S.mdo};
+        for (int i = 0; i < 4; ++i)
+            if ((st = make_map(maps[i], S.pool[i], (int64_t)rows, g, pl.spec.d)) != CQSA_OK) return st;
+    }
+    if (z.spill_host) {
+        void *h = nullptr;
+        CK(cudaHostAlloc(&h, z.spill_host, cudaHostAllocDefault));
+        S.spill = static_cast<float *>(h);
+        S.ev_spill.assign((size_t)pl.num_blocks, nullptr);
+        for (auto &ev : S.ev_spill) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    }
+    CK(cudaStreamCreateWithFlags(&S.s_in, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&S.s_comp, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&S.s_out, cudaStreamNonBlocking));
+    S.ev_slot_free.assign((size_t)cp.slots, nullptr);
+    for (auto &ev : S.ev_slot_free) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    for (int i = 0; i < 2; ++i) {
+        CK(cudaEventCreateWithFlags(&S.ev_in_ready[i], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&S.ev_comp[i], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&S.ev_stage_ready[i], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&S.ev_stage_free[i], cudaEventDisableTiming));
+    }
+    CK(cudaEventCreateWithFlags(&S.ev_start, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&S.ev_group, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&S.ev_done_comp, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&S.ev_done_out, cudaEventDisableTiming));
+    return CQSA_OK;
+}
+
+cqsa_status_t setup_bwd_host(cqsa_plan_t *P) {
+    const cqsa_status_t st = guarded([&] { return setup_bwd_host_impl(P); });
+    if (st != CQSA_OK && (P->bh.arena || P->bh.s_in || P->bh.spill)) release_bwd_host(P);
+    return st;
+}
+
+// One sequence of the streamed backward; all ten pointers pinned host
+// memory ([N, H, d] in the plan dtype; lse fp32 [H, N]).
+cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const void *v, const void *out,
+                            const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                            cudaStream_t stream) {
+    cqsa_status_t st = setup_bwd_host(P);
+    if (st != CQSA_OK) return st;
+    BwdHostState &S = P->bh;
+    const Planner &pl = P->pl;
+    const BwdCachePlan &cp = pl.bwd_cache;
+    const int64_t N = pl.spec.N, Bk = pl.block;
+    const int H = pl.spec.H, d = pl.spec.d, g = S.g;
+    const size_t e = (size_t)P->elem;
+    const size_t full_row = (size_t)H * d * e, grp_row = (size_t)g * d * e, acc_row = (size_t)g * d * sizeof(float);
+    const size_t slot_rows = (size_t)Bk;
+    const char *src[4] = {static_cast<const char *>(q), static_cast<const char *>(k), static_cast<const char *>(v),
+                          static_cast<const char *>(dout)};
+    char *dst[3] = {static_cast<char *>(dq), static_cast<char *>(dk), static_cast<char *>(dv)};
+    const char *ho = static_cast<const char *>(out);
+    CK(cudaEventRecord(S.ev_start, stream));
+    cudaStream_t ss[3] = {S.s_in, S.s_comp, S.s_out};
+    for (cudaStream_t x : ss) {
+        CK(cudaStreamWaitEvent(x, S.ev_start, 0));
+        // The previous call on this plan is over before this one touches
+        // the arena (its callers' streams may differ).
+        CK(cudaStreamWaitEvent(x, S.ev_done_comp, 0));
+        CK(cudaStreamWaitEvent(x, S.ev_done_out, 0));
+    }
+    BwdParams bp{};
+    bp.lse = S.lse;
+    bp.delta = S.delta;
+    bp.N = N;
+    bp.H = g;
+    bp.Hkv = g;
+    bp.kv_group = 1;
+    bp.causal = pl.spec.causal;
+    bp.scale = 1.0f / std::sqrt((float)d);
+    bp.accum = 1;
+    bp.q = S.pool[0];
+    bp.k = S.pool[1];
+    bp.v = S.pool[2];
+    bp.dout = S.pool[3];
+    const size_t cast_n = slot_rows * g * d;  // values per slot and tensor
+    int64_t it = 0;
+    for (int h0 = 0; h0 < H; h0 += g) {
+        NvtxRange nvtx_group("cqsa streamed backward head group", h0);
+        // lse and D of this head group replace the previous group's once its
+        // kernels are done.
+        if (h0 > 0) CK(cudaStreamWaitEvent(S.s_in, S.ev_group, 0));
+        CK(cudaMemcpyAsync(S.lse, lse + (size_t)h0 * N, (size_t)g * N * sizeof(float), cudaMemcpyHostToDevice,
+                           S.s_in));
+        int ib = 0;
+        for (int64_t b = 0; b < pl.num_blocks; ++b) {
+            const size_t nr = (size_t)pl.block_rows(b);
+            if (!nr) continue;
+            const int sg = ib & 1;
+            if (ib >= 2) CK(cudaStreamWaitEvent(S.s_in, S.ev_stage_free[sg], 0));
+            const size_t off = ((size_t)b * Bk * H + h0) * d * e;
+            CK(copy_rows(S.stage_o[sg], grp_row, ho + off, full_row, grp_row, nr, cudaMemcpyHostToDevice, S.s_in));
+            CK(copy_rows(S.stage_do[sg], grp_row, src[3] + off, full_row, grp_row, nr, cudaMemcpyHostToDevice,
+                         S.s_in));
+            CK(cudaEventRecord(S.ev_stage_ready[sg], S.s_in));
+            CK(cudaStreamWaitEvent(S.s_comp, S.ev_stage_ready[sg], 0));
+            CK(launch_bwd_delta(d, P->elem, S.stage_o[sg], S.stage_do[sg], (int64_t)nr, g, S.delta + b * Bk, N,
+                                S.s_comp));
+            CK(cudaEventRecord(S.ev_stage_free[sg], S.s_comp));
+            ++ib;
+        }
+        for (size_t t = 0; t < pl.leaves.size(); ++t, ++it) {
+            NvtxRange nvtx_task("cqsa streamed backward task", (int64_t)t);
+            const int par = (int)(it & 1);
+            // -- copies into the cache: write back an evicted block's sums
+            // (after the kernels two tasks back, the last that can have
+            // touched it), then this task's missing blocks and their sums.
+            for (const BwdCopy &c : cp.copies[t]) {
+                const size_t srow = (size_t)c.slot * slot_rows;
+                if (c.evict >= 0) {
+                    if (it >= 2) CK(cudaStreamWaitEvent(S.s_out, S.ev_comp[par], 0));
+                    const size_t nr = (size_t)pl.block_rows(c.evict);
+                    for (int i = 0; i < 3; ++i)
+                        CK(copy_rows(S.spill + ((size_t)i * N + (size_t)c.evict * Bk) * g * d, acc_row,
+                                     S.acc[i] + srow * g * d, acc_row, acc_row, nr, cudaMemcpyDeviceToHost, S.s_out));
+                    CK(cudaEventRecord(S.ev_spill[c.evict], S.s_out));
+                    CK(cudaEventRecord(S.ev_slot_free[c.slot], S.s_out));
+                }
+                CK(cudaStreamWaitEvent(S.s_in, S.ev_slot_free[c.slot], 0));
+                const size_t nr = (size_t)pl.block_rows(c.block);
+                const size_t off = ((size_t)c.block * Bk * H + h0) * d * e;
+                for (int i = 0; i < 4; ++i)
+                    CK(copy_rows(S.pool[i] + srow * grp_row, grp_row, src[i] + off, full_row, grp_row, nr,
+                                 cudaMemcpyHostToDevice, S.s_in));
+                if (c.reload) {
+                    CK(cudaStreamWaitEvent(S.s_in, S.ev_spill[c.block], 0));
+                    for (int i = 0; i < 3; ++i)
+                        CK(copy_rows(S.acc[i] + srow * g * d, acc_row,
+                                     S.spill + ((size_t)i * N + (size_t)c.block * Bk) * g * d, acc_row, acc_row, nr,
+                                     cudaMemcpyHostToDevice, S.s_in));
+                } else {
+                    for (int i = 0; i < 3; ++i)
+                        CK(cudaMemsetAsync(S.acc[i] + srow * g * d, 0, slot_rows * acc_row, S.s_in));
+                }
+            }
+            CK(cudaEventRecord(S.ev_in_ready[par], S.s_in));
+            // -- the task's gradient terms, added into its blocks' sums.
+            CK(cudaStreamWaitEvent(S.s_comp, S.ev_in_ready[par], 0));
+            {
+                BwdParams pq = bp;
+                pq.entries = S.qwl[t].entries;
+                pq.runs = S.qwl[t].runs;
+                pq.units = S.qwl[t].units;
+                pq.part_a = S.acc[0];
+                LaunchTimer tm(P, S.s_comp, 2);
+                if (P->dtype == CQSA_BF16)
+                    CK(launch_bwd_dq_tc(d, S.mq, S.mk, S.mv, S.mdo, pq, S.qwl[t].num_units, P->timeout_ns, S.err,
+                                        S.s_comp));
+                else
+                    CK(launch_bwd_dq(d, P->elem, pq, S.qwl[t].num_units, S.s_comp));
+                tm.stop();
+            }
+            {
+                BwdParams pk = bp;
+                pk.entries = S.kvwl[t].entries;
+                pk.runs = S.kvwl[t].runs;
+                pk.units = S.kvwl[t].units;
+                pk.part_a = S.acc[1];
+                pk.part_b = S.acc[2];
+                LaunchTimer tm(P, S.s_comp, 2);
+                if (P->dtype == CQSA_BF16)
+                    CK(launch_bwd_dkdv_tc(d, S.mq, S.mk, S.mv, S.mdo, pk, S.kvwl[t].num_units, P->timeout_ns,
+                                          S.err, S.s_comp));
+                else
+                    CK(launch_bwd_dkdv(d, P->elem, pk, S.kvwl[t].num_units, S.s_comp));
+                tm.stop();
+            }
+            // -- blocks this task finished: their sums in the plan dtype over
+            // their Q, K, V rows (no longer needed), then to the host.
+            for (const auto &f : cp.finals[t])
+                for (int i = 0; i < 3; ++i)
+                    CK(launch_cast_out(P->elem, S.acc[i] + (size_t)f.second * slot_rows * g * d,
+                                       S.pool[i] + (size_t)f.second * slot_rows * grp_row, (int64_t)cast_n,
+                                       S.s_comp));
+            CK(cudaEventRecord(S.ev_comp[par], S.s_comp));
+            if (!cp.finals[t].empty()) {
+                CK(cudaStreamWaitEvent(S.s_out, S.ev_comp[par], 0));
+                for (const auto &f : cp.finals[t]) {
+                    const size_t nr = (size_t)pl.block_rows(f.first);
+                    const size_t off = ((size_t)f.first * Bk * H + h0) * d * e;
+                    for (int i = 0; i < 3; ++i)
+                        CK(copy_rows(dst[i] + off, full_row, S.pool[i] + (size_t)f.second * slot_rows * grp_row,
+                                     grp_row, grp_row, nr, cudaMemcpyDeviceToHost, S.s_out));
+                    CK(cudaEventRecord(S.ev_slot_free[f.second], S.s_out));
+                }
+            }
+        }
+        CK(cudaEventRecord(S.ev_group, S.s_comp));
+    }
+    CK(cudaEventRecord(S.ev_done_comp, S.s_comp));
+    CK(cudaEventRecord(S.ev_done_out, S.s_out));
+    CK(cudaStreamWaitEvent(stream, S.ev_done_comp, 0));
+    CK(cudaStreamWaitEvent(stream, S.ev_done_out, 0));
+    return CQSA_OK;
+}
+
+// After a streamed backward failed part-way: as join_after_error.
+void join_bwd_after_error(cqsa_plan_t *P, cudaStream_t stream) {
+    BwdHostState &S = P->bh;
+    if (!S.s_in || !S.s_comp || !S.s_out) return;
+    cudaEventRecord(S.ev_start, S.s_in);
+    cudaEventRecord(S.ev_done_comp, S.s_comp);
+    cudaEventRecord(S.ev_done_out, S.s_out);
+    cudaStreamWaitEvent(stream, S.ev_start, 0);
+    cudaStreamWaitEvent(stream, S.ev_done_comp, 0);
+    cudaStreamWaitEvent(stream, S.ev_done_out, 0);
+    // The next call waits for ev_done_comp: make it cover the copy stream too.
+    cudaStreamWaitEvent(S.s_comp, S.ev_start, 0);
+    cudaEventRecord(S.ev_done_comp, S.s_comp);
 }
 
 cqsa_status_t build_plan_impl(const PlanSpec &spec, int dtype, cqsa_plan_t **out) {
@@ -1099,13 +1443,34 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
                             void *stream) {
     NvtxRange nvtx("cqsa_backward");
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
-    if (host_or_device == CQSA_HOST)
-        return fail(CQSA_ERR_UNSUPPORTED, "the backward runs in device mode only");
-    if (host_or_device != CQSA_DEVICE) return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be 0 or 1");
+    if (host_or_device != CQSA_DEVICE && host_or_device != CQSA_HOST)
+        return fail(CQSA_ERR_INVALID_ARG, "host_or_device must be 0 or 1");
     if (plan->pl.spec.shard_count > 1)
         return fail(CQSA_ERR_UNSUPPORTED, "a sharded plan runs cqsa_backward_partial (shard_count = %d)",
                     plan->pl.spec.shard_count);
-    return backward_call(plan, false, q, k, v, out, lse, dout, dq, dk, dv, stream);
+    if (host_or_device == CQSA_DEVICE) return backward_call(plan, false, q, k, v, out, lse, dout, dq, dk, dv, stream);
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    const void *ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv};
+    const char *names[] = {"q", "k", "v", "out", "lse", "dout", "dq", "dk", "dv"};
+    for (int i = 0; i < 9; ++i)
+        if ((st = check_ptr(ptrs[i], true, names[i])) != CQSA_OK) return st;
+    const Planner &pl = plan->pl;
+    const size_t qs = (size_t)pl.spec.N * pl.spec.H * pl.spec.d * plan->elem, ls = (size_t)pl.spec.N * pl.spec.H;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    for (int b = 0; b < pl.spec.B; ++b) {
+        auto at = [&](const void *p) { return static_cast<const char *>(p) + b * qs; };
+        auto atw = [&](void *p) { return static_cast<char *>(p) + b * qs; };
+        st = guarded([&] {
+            return backward_host(plan, at(q), at(k), at(v), at(out), lse + b * ls, at(dout), atw(dq), atw(dk),
+                                 atw(dv), cs);
+        });
+        if (st != CQSA_OK) {
+            join_bwd_after_error(plan, cs);
+            return st;
+        }
+    }
+    return CQSA_OK;
 }
 
 cqsa_status_t cqsa_backward_partial(cqsa_plan_t *plan, const void *q, const void *k, const void *v,
@@ -1194,12 +1559,12 @@ cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
     CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-    int *words[5] = {plan->dev_err, plan->h_err, plan->bwd.err, plan->bwd_shard.err, plan->part_err};
-    static const char *const where[5] = {"device forward", "streamed forward", "backward", "partial backward",
-                                         "partial forward"};
+    int *words[6] = {plan->dev_err, plan->h_err, plan->bwd.err, plan->bwd_shard.err, plan->part_err, plan->bh.err};
+    static const char *const where[6] = {"device forward", "streamed forward", "backward", "partial backward",
+                                         "partial forward", "streamed backward"};
     int bad = 0;
     std::string sites;
-    for (int i = 0; i < 5; ++i) {
+    for (int i = 0; i < 6; ++i) {
         if (!words[i]) continue;
         int v = 0;
         CK(cudaMemcpy(&v, words[i], sizeof v, cudaMemcpyDeviceToHost));
@@ -1306,6 +1671,54 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->total_pairs = pl.total_pairs;
     info->cache_q_slots = pl.sizing.q_slots;
     info->cache_kv_slots = pl.sizing.kv_slots;
+    info->bwd_head_group = pl.bwd_sizing.head_group;
+    info->bwd_host_arena_bytes = pl.bwd_sizing.arena;
+    info->bwd_cache_slots = pl.bwd_sizing.slots;
+    info->bwd_h2d_bytes = pl.bwd_sizing.h2d;
+    info->bwd_d2h_bytes = pl.bwd_sizing.d2h;
+    info->bwd_spill_host_bytes = pl.bwd_sizing.spill_host;
+    info->bwd_writebacks = pl.bwd_cache.writebacks;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_bwd_cache_task(const cqsa_plan_t *plan, int64_t t, int64_t *blocks, int32_t *slots,
+                                       int64_t *evicts, int32_t *reloads, int64_t max_copies, int64_t *num_copies,
+                                       int32_t *member_slot, int64_t max_blocks, int64_t *num_blocks,
+                                       int64_t *fin_blocks, int32_t *fin_slots, int64_t max_fin, int64_t *num_fin) {
+    if (!plan || !num_copies || !num_blocks || !num_fin) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    if (t < 0 || t >= (int64_t)pl.leaves.size()) return fail(CQSA_ERR_INVALID_ARG, "task %lld out of range", (long long)t);
+    const BwdCachePlan &c = pl.bwd_cache;
+    if (pl.bwd_sizing.head_group == 0 || c.copies.size() != pl.leaves.size())
+        return fail(CQSA_ERR_BUDGET, "no host-mode backward sizing fits the budget; the plan has no backward cache");
+    const std::vector<BwdCopy> &cp = c.copies[t];
+    const std::vector<int32_t> &ms = c.member_slot[t];
+    const auto &fin = c.finals[t];
+    *num_copies = (int64_t)cp.size();
+    *num_blocks = (int64_t)ms.size();
+    *num_fin = (int64_t)fin.size();
+    if (blocks || slots || evicts || reloads) {
+        if (!blocks || !slots || !evicts || !reloads || max_copies < (int64_t)cp.size())
+            return fail(CQSA_ERR_INVALID_ARG, "copy arrays missing or too small");
+        for (size_t i = 0; i < cp.size(); ++i) {
+            blocks[i] = cp[i].block;
+            slots[i] = cp[i].slot;
+            evicts[i] = cp[i].evict;
+            reloads[i] = cp[i].reload;
+        }
+    }
+    if (member_slot) {
+        if (max_blocks < (int64_t)ms.size()) return fail(CQSA_ERR_INVALID_ARG, "member slot array too small");
+        for (size_t m = 0; m < ms.size(); ++m) member_slot[m] = ms[m];
+    }
+    if (fin_blocks || fin_slots) {
+        if (!fin_blocks || !fin_slots || max_fin < (int64_t)fin.size())
+            return fail(CQSA_ERR_INVALID_ARG, "final arrays missing or too small");
+        for (size_t j = 0; j < fin.size(); ++j) {
+            fin_blocks[j] = fin[j].first;
+            fin_slots[j] = fin[j].second;
+        }
+    }
     return CQSA_OK;
 }
 
@@ -1390,6 +1803,7 @@ cqsa_status_t cqsa_difference_set(int l, int *D) {
 void cqsa_plan_destroy(cqsa_plan_t *plan) {
     if (!plan) return;
     if (plan->device >= 0) {
+        release_bwd_host(plan);
         cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);

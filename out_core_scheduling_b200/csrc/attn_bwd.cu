@@ -40,7 +40,7 @@ __device__ __forceinline__ void st_out(__nv_bfloat16 *p, int64_t i, float x) { p
 template <int D, typename T>
 __global__ void __launch_bounds__(256)
     bwd_delta_kernel(const T *__restrict__ out, const T *__restrict__ dout, int64_t N, int H,
-                     float *__restrict__ delta) {
+                     float *__restrict__ delta, int64_t ldd) {
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < N * H; w += warps) {
@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256)
         for (int c = lane; c < D; c += 32) acc = fmaf(ld_f32(out, base + c), ld_f32(dout, base + c), acc);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) delta[(int64_t)h * N + r] = acc;
+        if (lane == 0) delta[(int64_t)h * ldd + r] = acc;
     }
 }
 
@@ -176,10 +176,12 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dq_kernel(const BwdParams p)
         for (int jj = 0; jj < NJ; ++jj) {
             const float g = acc[i][jj] * p.scale;
             const int c = tx + 16 * jj;
-            if (fused)
+            if (fused) {
                 st_out(static_cast<T *>(p.out_a), (orow * H + h) * D + c, g);
-            else
-                p.part_a[(((int64_t)e.slot * p.N + orow) * H + h) * D + c] = g;
+            } else {
+                float *dst = p.part_a + (((int64_t)e.slot * p.N + orow) * H + h) * D + c;
+                *dst = p.accum ? *dst + g : g;
+            }
         }
     }
 }
@@ -329,8 +331,9 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
                 st_out(static_cast<T *>(p.out_b), o, gv[i][jj]);
             } else {
                 const int64_t po = slot * p.N * Hkv * D + o;
-                p.part_a[po] = gk[i][jj] * p.scale;
-                p.part_b[po] = gv[i][jj];
+                const float a = gk[i][jj] * p.scale, b = gv[i][jj];
+                p.part_a[po] = p.accum ? p.part_a[po] + a : a;
+                p.part_b[po] = p.accum ? p.part_b[po] + b : b;
             }
         }
     }
@@ -365,9 +368,11 @@ static int grid_for_warps(int64_t warps) {
 }
 
 template <int D, typename T>
-static cudaError_t delta_t(const void *out, const void *dout, int64_t N, int H, float *delta, cudaStream_t st) {
+static cudaError_t delta_t(const void *out, const void *dout, int64_t N, int H, float *delta, int64_t ldd,
+                           cudaStream_t st) {
+    if (N <= 0) return cudaSuccess;
     bwd_delta_kernel<D, T><<<grid_for_warps(N * H), 256, 0, st>>>(static_cast<const T *>(out),
-                                                                    static_cast<const T *>(dout), N, H, delta);
+                                                                    static_cast<const T *>(dout), N, H, delta, ldd);
     return cudaGetLastError();
 }
 
@@ -403,8 +408,8 @@ static cudaError_t dkdv_t(const BwdParams &p, int units, cudaStream_t st) {
     } while (0)
 
 cudaError_t launch_bwd_delta(int d, int elem_bytes, const void *out, const void *dout, int64_t N, int H,
-                             float *delta, cudaStream_t stream) {
-#define CALL(D_, T_) delta_t<D_, T_>(out, dout, N, H, delta, stream)
+                             float *delta, int64_t ldd, cudaStream_t stream) {
+#define CALL(D_, T_) delta_t<D_, T_>(out, dout, N, H, delta, ldd, stream)
     CQSA_DISPATCH(d, elem_bytes, CALL);
 #undef CALL
 }

@@ -417,10 +417,20 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     } else {
                         float *dst = p.part_a + (((int64_t)e.slot * p.N + orow) * p.H + head) * D;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4 *>(dst + cc * 32 + i) =
-                                make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
-                                            __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
+                        for (int i = 0; i < 32; i += 4) {
+                            float4 g4 = make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                                    __uint_as_float(o[i + 2]) * p.scale,
+                                                    __uint_as_float(o[i + 3]) * p.scale);
+                            float4 *d4 = reinterpret_cast<float4 *>(dst + cc * 32 + i);
+                            if (p.accum) {  // streamed backward: add into the block's running sums
+                                const float4 a4 = *d4;
+                                g4.x += a4.x;
+                                g4.y += a4.y;
+                                g4.z += a4.z;
+                                g4.w += a4.w;
+                            }
+                            *d4 = g4;
+                        }
                     }
                 }
             }
@@ -731,10 +741,19 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                     } else {
                         float *dst = (which == 0 ? p.part_a : p.part_b) + ((slot * p.N + orow) * p.Hkv + hkv) * D;
 #pragma unroll
-                        for (int x = 0; x < 32; x += 4)
-                            *reinterpret_cast<float4 *>(dst + cc * 32 + x) =
-                                make_float4(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul,
-                                            __uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
+                        for (int x = 0; x < 32; x += 4) {
+                            float4 g4 = make_float4(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul,
+                                                    __uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
+                            float4 *d4 = reinterpret_cast<float4 *>(dst + cc * 32 + x);
+                            if (p.accum) {  // streamed backward: add into the block's running sums
+                                const float4 a4 = *d4;
+                                g4.x += a4.x;
+                                g4.y += a4.y;
+                                g4.z += a4.z;
+                                g4.w += a4.w;
+                            }
+                            *d4 = g4;
+                        }
                     }
                 }
             }

@@ -15,6 +15,14 @@
 // the tile's K and V are fetched with one vector load per four features,
 // all issued before any store.  Row maxima and sums are reduced over the 16
 // threads of a row with warp shuffles.
+//
+// Key split: a unit may be computed by a cluster of S = 1, 2 or 4 CTAs (the
+// launcher picks S so that small problems still fill every SM): CTA rank r
+// of the cluster takes the r-th contiguous share of the unit's key tiles,
+// and the cluster combines the S online-softmax states (m, l, O) through
+// distributed shared memory before rank 0 writes the unit's result, so the
+// work list, the slots and the merge are those of an unsplit unit.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -61,8 +69,17 @@ __global__ void __launch_bounds__(simt::THREADS)
     float *Vs = Kt + D * LD;    // [BN][D]
     float *Pt = Vs + BN * D;    // [BN][LD]  P transposed
 
-    const WlUnit u = p.units[blockIdx.x];
+    namespace cg = cooperative_groups;
+    const cg::cluster_group cluster = cg::this_cluster();
+    const int S = (int)cluster.num_blocks();  // CTAs sharing this unit's key tiles
+    const int rank = (int)cluster.block_rank();
+    const WlUnit u = p.units[blockIdx.x / S];
     const WlEntry e = p.entries[u.entry];
+    // This CTA's share of the unit's key tiles, in run order.
+    const int32_t ntiles = unit_key_tiles(e, p.runs, u.q0, BM, p.causal, BN);
+    const int32_t t_lo = (int32_t)((int64_t)ntiles * rank / S);
+    const int32_t t_hi = (int32_t)((int64_t)ntiles * (rank + 1) / S);
+    int32_t t_at = 0;  // index of the next key tile of the unit
     const int H = p.H;
     const int h = u.head;
     const int hkv = (h + p.hq_off) / p.kv_group - p.hk_off;  // grouped-query attention
@@ -95,11 +112,20 @@ __global__ void __launch_bounds__(simt::THREADS)
             for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = 0.f;
     }
 
-    for (int r = 0; r < e.run_count; ++r) {
+    for (int r = 0; r < e.run_count && t_at < t_hi; ++r) {
         const WlRun run = p.runs[e.run_begin + r];
         int32_t lo, hi;
         clip_run(e, run, q_end, p.causal, &lo, &hi);
-        for (int32_t ks = lo; ks < hi; ks += BN) {
+        const int32_t nt = hi > lo ? (hi - lo + BN - 1) / BN : 0;
+        if (t_at + nt <= t_lo) {  // the whole run lies before this CTA's share
+            t_at += nt;
+            continue;
+        }
+        if (t_at < t_lo) {
+            lo += (t_lo - t_at) * BN;
+            t_at = t_lo;
+        }
+        for (int32_t ks = lo; ks < hi && t_at < t_hi; ks += BN, ++t_at) {
             __syncthreads();
             float4 kr[NL], vr[NL];
 #pragma unroll
@@ -191,6 +217,51 @@ __global__ void __launch_bounds__(simt::THREADS)
         }
     }
 
+    if (S > 1) {
+        // Combine the cluster's states: ranks >= 1 leave (m, l, O) in their
+        // own shared memory, element-major so that a warp's reads are
+        // contiguous; rank 0 reads them remotely and rescales to the common
+        // maximum.  The second cluster barrier keeps the senders' shared
+        // memory alive until rank 0 has read it.
+        constexpr int NV = 8 + 16 * G;  // values per thread
+        __syncthreads();
+        float *xs = smf;
+        if (rank > 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                xs[(2 * i) * THREADS + tid] = m[i];
+                xs[(2 * i + 1) * THREADS + tid] = l[i];
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) xs[(8 + (i * G + g) * 4 + jj) * THREADS + tid] = o[i][g][jj];
+            }
+        }
+        cluster.sync();
+        if (rank == 0) {
+            for (int rr = 1; rr < S; ++rr) {
+                const float *rx = cluster.map_shared_rank(xs, rr);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float mr = rx[(2 * i) * THREADS + tid], lr = rx[(2 * i + 1) * THREADS + tid];
+                    const float mn = fmaxf(m[i], mr);
+                    const float a0 = (m[i] == -INFINITY) ? 0.f : exp2f(m[i] - mn);
+                    const float ar = (mr == -INFINITY) ? 0.f : exp2f(mr - mn);
+                    l[i] = l[i] * a0 + lr * ar;
+                    m[i] = mn;
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            o[i][g][jj] = o[i][g][jj] * a0 + rx[(8 + (i * G + g) * 4 + jj) * THREADS + tid] * ar;
+                }
+            }
+        }
+        cluster.sync();
+        if (rank > 0) return;
+        static_assert(NV * THREADS <= 2 * D * LD + BN * D + BN * LD, "combine area fits the shared tiles");
+    }
+
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int32_t row = q0 + ty * 4 + i;
@@ -236,6 +307,19 @@ __global__ void __launch_bounds__(simt::THREADS)
     }
 }
 
+// Cluster size for a launch of num_units units: the smallest S in {1, 2, 4}
+// whose num_units * S CTAs fill every SM with as many CTAs as can be
+// resident at once (fewer units than that leave SMs idle, and one CTA per
+// SM leaves the FFMA pipe waiting on shared-memory latency).
+static int simt_split(int num_units, int resident) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t target = (int64_t)sms * (resident > 0 ? resident : 1);
+    int S = 1;
+    while (S < 4 && (int64_t)num_units * S < target) S *= 2;
+    return S;
+}
+
 template <int D, typename T>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const AttnParams &p,
                                  int num_units, cudaStream_t stream) {
@@ -244,9 +328,28 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
     cudaError_t err = cudaFuncSetAttribute(attn_simt_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
-    attn_simt_kernel<D, T><<<num_units, THREADS, smem, stream>>>(
-        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), p);
-    return cudaGetLastError();
+    static int resident = 0;  // CTAs of this instantiation one SM holds (the same on every sm_100 device)
+    if (resident < 1) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_simt_kernel<D, T>, THREADS, smem) != cudaSuccess)
+            cudaGetLastError();
+        resident = n > 0 ? n : 1;
+    }
+    const int S = simt_split(num_units, resident);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)num_units * S);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_simt_kernel<D, T>, static_cast<const T *>(q), static_cast<const T *>(k),
+                              static_cast<const T *>(v), p);
 }
 
 cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k, const void *v,

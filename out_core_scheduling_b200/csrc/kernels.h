@@ -84,12 +84,14 @@ struct BwdParams {
     float scale;         // 1 / sqrt(d)
     float *part_a;       // dq, or dk
     float *part_b;       // dv
+    int accum;           // 1: add each entry's sums into part_a / part_b (streamed backward)
     void *out_a;         // dq, or dk (input dtype)
     void *out_b;         // dv
 };
 
+// delta[h * ldd + n] = <out[n][h][:], dout[n][h][:]> for n < N, h < H.
 cudaError_t launch_bwd_delta(int d, int elem_bytes, const void *out, const void *dout, int64_t N, int H,
-                             float *delta, cudaStream_t stream);
+                             float *delta, int64_t ldd, cudaStream_t stream);
 // Query-stationary: 64 query rows per unit, key tiles of 64.
 cudaError_t launch_bwd_dq(int d, int elem_bytes, const BwdParams &p, int num_units, cudaStream_t stream);
 // Key-stationary: 64 key rows per unit, query tiles of 64.
@@ -109,9 +111,10 @@ cudaError_t launch_sum_slots(int d, int elem_bytes, const float *part, const int
 
 // Log-sum-exp recomposition of a query block's partials (merge.cu).
 //   out[r][h][:] = sum_j exp(lse_j - lse) O_j,  lse = log sum_j exp(lse_j)
-// over the nslots[r / block] partials of row r.  out in the input dtype.
+// over the nslots[r / block] partials of row r (at most max_slots <= 32).
+// out in the input dtype.
 cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const float *part_lse,
-                               const int32_t *nslots, int64_t block, int64_t N, int H, void *out,
+                               const int32_t *nslots, int64_t block, int64_t N, int H, int max_slots, void *out,
                                float *lse, cudaStream_t stream);
 
 // Cross-rank exchange of a sharded forward (partial.cu).  o [N][H][d] fp32,

@@ -10,130 +10,199 @@
 // "Stream-CQSA: Breaking the Billion-Token Barrier on a Single GPU",
 // section "Implementation", step 4: aggregate).
 //
-// HBM-bound: one warp per (row, head), each lane a d/32-float vector of the
-// row, so a warp reads each partial row as one contiguous 128- or 256-float
-// segment.  Grid-stride over rows, sized to the SM count.
+// HBM-bound.  The slots of one partial are laid out [S][N][H][D], so for a
+// fixed slot consecutive (row, head) pairs are one contiguous stream.  A CTA
+// takes a tile of 128 consecutive pairs: it first stages their partial lse
+// values in shared memory and turns them into weights (one thread per
+// pair), then streams the tile's float4 chunks, each thread loading two
+// chunks of up to four slots each at once (eight 16-byte loads in flight)
+// before it sums them and stores the output chunks.  Persistent grid over
+// tiles, sized to the SM count.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include "kernels.h"
 #include "worklist.h"
 
 namespace cqsa {
 
-template <int V>
-struct VecF;
-template <>
-struct VecF<2> {
-    using T = float2;
-};
-template <>
-struct VecF<4> {
-    using T = float4;
-};
-
-template <int V>
-__device__ __forceinline__ void load_vec(const float *src, float (&x)[V]) {
-    const typename VecF<V>::T t = *reinterpret_cast<const typename VecF<V>::T *>(src);
-    const float *f = reinterpret_cast<const float *>(&t);
-#pragma unroll
-    for (int i = 0; i < V; ++i) x[i] = f[i];
-}
-
-template <int V>
-__device__ __forceinline__ void store_vec(float *dst, const float (&x)[V]) {
-    typename VecF<V>::T t;
-    float *f = reinterpret_cast<float *>(&t);
-#pragma unroll
-    for (int i = 0; i < V; ++i) f[i] = x[i];
-    *reinterpret_cast<typename VecF<V>::T *>(dst) = t;
-}
-
-template <int V>
-__device__ __forceinline__ void store_vec(__nv_bfloat16 *dst, const float (&x)[V]) {
-    if constexpr (V == 4) {
-        __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
-        __nv_bfloat162 b = __floats2bfloat162_rn(x[2], x[3]);
-        uint2 u;
-        u.x = *reinterpret_cast<uint32_t *>(&a);
-        u.y = *reinterpret_cast<uint32_t *>(&b);
-        *reinterpret_cast<uint2 *>(dst) = u;
-    } else {
-        __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]);
-        *reinterpret_cast<__nv_bfloat162 *>(dst) = a;
-    }
-}
-
 // Device mode: partials in slots [S][N][H][D], lse [S][H][N].
+constexpr int kMergePairs = 128;   // (row, head) pairs per tile
+constexpr int kMergeThreads = 256;
+constexpr int kMergeGroup = 4;     // slots loaded together per chunk (two chunks per thread at once)
+
+__device__ __forceinline__ float4 ld_stream(const float *p) {
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+}
+
+__device__ __forceinline__ void store4(float *dst, float4 x) { *reinterpret_cast<float4 *>(dst) = x; }
+
+__device__ __forceinline__ void store4(__nv_bfloat16 *dst, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(dst) = u;
+}
+
 template <int D, typename TO>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kMergeThreads, 3)
     merge_slots_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
-                       const int32_t *__restrict__ nslots, int64_t block, int64_t N, int H,
+                       const int32_t *__restrict__ nslots, int64_t block, int64_t N, int H, int smax,
                        TO *__restrict__ out, float *__restrict__ lse_out) {
-    constexpr int V = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    constexpr int CH = D / 4;  // float4 chunks per (row, head)
+    constexpr int P = kMergePairs;
+    __shared__ float s_l[32 * P];   // staged lse_j, [slot][pair]
+    __shared__ float s_w[P * 33];   // weights exp(lse_j - M), [pair][slot] (padded)
+    __shared__ float s_inv[P];      // 1 / sum of the weights
+    __shared__ int s_n[P];          // partials of the pair's row
+    const int tid = threadIdx.x;
     const int64_t total = N * H;
     const int64_t slot_stride = N * H * D;
-    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-        const int64_t r = w / H;
-        const int h = (int)(w - r * H);
-        const int n = nslots[r / block];
-        const float lj = lane < n ? part_lse[((int64_t)lane * H + h) * N + r] : -INFINITY;
-        float M = lj;
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        const float wj = (lane < n && lj != -INFINITY) ? __expf(lj - M) : 0.f;
-        float W = wj;
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
-        float acc[V];
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = 0.f;
-        const float *src = part_o + (r * H + h) * D + lane * V;
-        for (int j = 0; j < n; ++j) {
-            const float wb = __shfl_sync(0xffffffffu, wj, j);
-            if (wb == 0.f) continue;
-            float x[V];
-            load_vec<V>(src + (int64_t)j * slot_stride, x);
-#pragma unroll
-            for (int i = 0; i < V; ++i) acc[i] = fmaf(wb, x[i], acc[i]);
+    const int64_t tiles = (total + P - 1) / P;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t g0 = t * P;
+        // Stage lse_j of the tile's pairs (slot-major, so a slot's loads for
+        // consecutive rows of one head fall in the same sectors).
+        for (int idx = tid; idx < smax * P; idx += kMergeThreads) {
+            const int j = idx / P, p = idx - j * P;
+            const int64_t g = g0 + p;
+            float x = -INFINITY;
+            if (g < total) {
+                const int64_t r = g / H;
+                const int h = (int)(g - r * H);
+                if (j < nslots[r / block]) x = part_lse[((int64_t)j * H + h) * N + r];
+            }
+            s_l[j * P + p] = x;
         }
-        const float inv = 1.f / W;
+        __syncthreads();
+        if (tid < P) {
+            const int64_t g = g0 + tid;
+            int n = 0;
+            if (g < total) {
+                const int64_t r = g / H;
+                const int h = (int)(g - r * H);
+                n = nslots[r / block];
+                float M = -INFINITY;
+                for (int j = 0; j < n; ++j) M = fmaxf(M, s_l[j * P + tid]);
+                float W = 0.f;
+                for (int j = 0; j < n; ++j) {
+                    const float lj = s_l[j * P + tid];
+                    const float wj = lj != -INFINITY ? __expf(lj - M) : 0.f;
+                    s_w[tid * 33 + j] = wj;
+                    W += wj;
+                }
+                s_inv[tid] = W > 0.f ? 1.f / W : 0.f;
+                lse_out[(int64_t)h * N + r] = M + __logf(W);
+            }
+            s_n[tid] = n;
+        }
+        __syncthreads();
+        // Stream the chunks: every slot's load of a chunk is issued before
+        // any of them is used.  A zero weight (an lse of -inf) never lets
+        // its chunk into the sum.
+        const int64_t chunks = (total - g0 < P ? total - g0 : P) * CH;
+        const float *base = part_o + g0 * D;
+        TO *obase = out + g0 * D;
+        for (int64_t c0 = tid; c0 < chunks; c0 += 2 * kMergeThreads) {
+            const int64_t c[2] = {c0, c0 + kMergeThreads};
+            const bool live1 = c[1] < chunks;
+            int p[2], n[2];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] *= inv;
-        store_vec<V>(out + (r * H + h) * D + lane * V, acc);
-        if (lane == 0) lse_out[(int64_t)h * N + r] = M + __logf(W);
+            for (int i = 0; i < 2; ++i) {
+                p[i] = (int)((i == 0 || live1 ? c[i] : c0) / CH);
+                n[i] = (i == 0 || live1) ? s_n[p[i]] : 0;
+            }
+            float4 acc[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int nmax = n[0] > n[1] ? n[0] : n[1];
+            for (int j0 = 0; j0 < nmax; j0 += kMergeGroup) {
+                float4 x[2][kMergeGroup];
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int u = 0; u < kMergeGroup; ++u)
+                        if (j0 + u < n[i]) x[i][u] = ld_stream(base + c[i] * 4 + (int64_t)(j0 + u) * slot_stride);
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int u = 0; u < kMergeGroup; ++u) {
+                        if (j0 + u < n[i]) {
+                            const float w = s_w[p[i] * 33 + j0 + u];
+                            if (w != 0.f) {
+                                acc[i].x = fmaf(w, x[i][u].x, acc[i].x);
+                                acc[i].y = fmaf(w, x[i][u].y, acc[i].y);
+                                acc[i].z = fmaf(w, x[i][u].z, acc[i].z);
+                                acc[i].w = fmaf(w, x[i][u].w, acc[i].w);
+                            }
+                        }
+                    }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (i == 1 && !live1) break;
+                const float inv = s_inv[p[i]];
+                acc[i].x *= inv;
+                acc[i].y *= inv;
+                acc[i].z *= inv;
+                acc[i].w *= inv;
+                store4(obase + c[i] * 4, acc[i]);
+            }
+        }
+        __syncthreads();  // the next tile reuses the shared arrays
     }
 }
 
-static int merge_grid(int64_t warps_needed) {
+// Persistent grid: as many CTAs as fit on the device at once (or one per
+// tile when there are fewer tiles).
+template <int D, typename TO>
+static int merge_grid(int64_t tiles) {
+    static int per_sm = 0;  // the same on every device this library runs on (sm_100)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t blocks_needed = (warps_needed + 7) / 8;
-    const int64_t cap = (int64_t)sms * 8;  // 8 resident 256-thread blocks per SM
-    return (int)(blocks_needed < cap ? (blocks_needed > 0 ? blocks_needed : 1) : cap);
+    if (per_sm < 1) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_slots_kernel<D, TO>, kMergeThreads, 0) !=
+            cudaSuccess)
+            cudaGetLastError();
+        per_sm = n > 0 ? n : 1;
+    }
+    const int64_t cap = (int64_t)sms * per_sm;
+    return (int)(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
 }
 
 template <int D, typename TO>
 static cudaError_t merge_slots_t(const float *po, const float *pl, const int32_t *ns, int64_t block, int64_t N,
-                                 int H, void *out, float *lse, cudaStream_t st) {
-    merge_slots_kernel<D, TO><<<merge_grid(N * H), 256, 0, st>>>(po, pl, ns, block, N, H,
-                                                                  static_cast<TO *>(out), lse);
+                                 int H, int smax, void *out, float *lse, cudaStream_t st) {
+    const int64_t tiles = (N * H + kMergePairs - 1) / kMergePairs;
+    merge_slots_kernel<D, TO><<<merge_grid<D, TO>(tiles), kMergeThreads, 0, st>>>(po, pl, ns, block, N, H, smax,
+                                                                                   static_cast<TO *>(out), lse);
     return cudaGetLastError();
 }
 
 cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const float *part_lse,
-                               const int32_t *nslots, int64_t block, int64_t N, int H, void *out,
+                               const int32_t *nslots, int64_t block, int64_t N, int H, int max_slots, void *out,
                                float *lse, cudaStream_t stream) {
+    if (max_slots < 1 || max_slots > 32) return cudaErrorInvalidValue;
+    // Each thread stores four consecutive outputs at once, and reads float4s.
+    if ((reinterpret_cast<uintptr_t>(out) & (uintptr_t)(4 * elem_bytes - 1)) ||
+        (reinterpret_cast<uintptr_t>(part_o) & 15u))
+        return cudaErrorMisalignedAddress;
     if (elem_bytes == 4) {
-        if (d == 64) return merge_slots_t<64, float>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
-        if (d == 128) return merge_slots_t<128, float>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
+        if (d == 64)
+            return merge_slots_t<64, float>(part_o, part_lse, nslots, block, N, H, max_slots, out, lse, stream);
+        if (d == 128)
+            return merge_slots_t<128, float>(part_o, part_lse, nslots, block, N, H, max_slots, out, lse, stream);
     } else if (elem_bytes == 2) {
         if (d == 64)
-            return merge_slots_t<64, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
+            return merge_slots_t<64, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, max_slots, out, lse,
+                                                    stream);
         if (d == 128)
-            return merge_slots_t<128, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, out, lse, stream);
+            return merge_slots_t<128, __nv_bfloat16>(part_o, part_lse, nslots, block, N, H, max_slots, out, lse,
+                                                     stream);
     }
     return cudaErrorInvalidValue;
 }

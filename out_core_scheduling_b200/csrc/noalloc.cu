@@ -267,7 +267,7 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     } else {
         NA_CK(launch_attn_simt(d, elem, q, k, v, ap, (int)n.units, s));
     }
-    NA_CK(launch_merge_slots(d, elem, part_o, part_lse, nslots, pl.block, N, H, out, lse, s));
+    NA_CK(launch_merge_slots(d, elem, part_o, part_lse, nslots, pl.block, N, H, (int)pl.max_slots, out, lse, s));
 
     // The error word is only valid once this call's work is done; it is read
     // on the call's own stream, not the legacy default stream.

@@ -194,6 +194,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     for (int32_t v : slots_per_block) max_slots = std::max<int64_t>(max_slots, v);
     assign_shards();
     size_plan();
+    size_bwd();
     const char *dbg = getenv("CQSA_DEBUG");
     if (dbg && dbg[0] && !(dbg[0] == '0' && dbg[1] == 0)) {
         const std::string bad = verify();
@@ -804,6 +805,278 @@ void Planner::size_plan() {
     // A call runs the B sequences one after another on the same plan.
     sizing.h2d *= (size_t)spec.B;
     sizing.d2h *= (size_t)spec.B;
+}
+
+// ---------------------------------------------------------------------------
+// Streamed backward: block cache with running gradient sums (see planner.h).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Blocks a leaf task touches in the backward (as query or key), member order.
+std::vector<std::vector<int64_t>> bwd_task_blocks(const Planner &pl) {
+    const size_t T = pl.leaves.size();
+    std::vector<std::vector<int64_t>> out(T);
+    std::vector<char> q, kv;
+    for (size_t t = 0; t < T; ++t) {
+        pl.leaf_needs((int64_t)t, &q, &kv);
+        for (size_t m = 0; m < q.size(); ++m)
+            if (q[m] || kv[m]) out[t].push_back(pl.leaves[t].blocks[m]);
+    }
+    return out;
+}
+
+// Units of a key-stationary list: every 'rows' key rows of an entry, per
+// head, with the query tiles the causal rule leaves; longest first.
+void add_units_kv(WorkList *wl, int heads, int rows, int bn, int causal) {
+    std::vector<WlUnit> u;
+    for (int32_t ei = 0; ei < (int32_t)wl->entries.size(); ++ei) {
+        const WlEntry &e = wl->entries[ei];
+        for (int h = 0; h < heads; ++h)
+            for (int64_t k0 = e.q_lo; k0 < e.q_hi; k0 += rows) {
+                WlUnit x{ei, (int32_t)k0, h, unit_query_tiles(e, wl->runs.data(), (int32_t)k0, causal, bn)};
+                if (x.ntiles > 0) u.push_back(x);
+            }
+    }
+    std::stable_sort(u.begin(), u.end(), [](const WlUnit &a, const WlUnit &b) {
+        const int ca = a.ntiles / 32, cb = b.ntiles / 32;
+        if (ca != cb) return ca > cb;
+        return a.head < b.head;
+    });
+    wl->units.swap(u);
+}
+
+// Appends rows [lo, lo + n) with global offset goff to the entry's runs,
+// joining it to the previous run when the rows continue it.
+void push_run(WorkList *wl, int32_t run_begin, int32_t lo, int32_t n, int32_t goff) {
+    if ((int32_t)wl->runs.size() > run_begin && wl->runs.back().k_hi == lo && wl->runs.back().k_goff == goff) {
+        wl->runs.back().k_hi = lo + n;
+        return;
+    }
+    WlRun x{};
+    x.k_lo = lo;
+    x.k_hi = lo + n;
+    x.k_goff = goff;
+    wl->runs.push_back(x);
+}
+
+}  // namespace
+
+bool Planner::plan_bwd_cache(int64_t C, BwdCachePlan *out) const {
+    const std::vector<std::vector<int64_t>> tb = bwd_task_blocks(*this);
+    const int64_t T = (int64_t)tb.size();
+    std::vector<std::vector<int64_t>> uses(num_blocks);
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t b : tb[t]) uses[b].push_back(t);
+    auto next_use = [&](int64_t b, int64_t t) -> int64_t {
+        auto it = std::upper_bound(uses[b].begin(), uses[b].end(), t);
+        return it == uses[b].end() ? INT64_MAX : *it;
+    };
+    BwdCachePlan cp;
+    cp.slots = C;
+    cp.copies.assign(T, {});
+    cp.member_slot.assign(T, {});
+    cp.finals.assign(T, {});
+    std::vector<int64_t> held(C, -1);        // block whose rows the slot holds
+    std::vector<int64_t> release(C, 0);      // a finished block's slot is free from this task on
+    std::vector<char> done(num_blocks, 0), on_host(num_blocks, 0);
+    std::vector<int32_t> slot_of(num_blocks, -1);
+    for (int64_t t = 0; t < T; ++t) {
+        std::vector<int64_t> protect = tb[t];
+        if (t > 0) protect.insert(protect.end(), tb[t - 1].begin(), tb[t - 1].end());
+        std::sort(protect.begin(), protect.end());
+        for (int64_t b : tb[t]) {
+            if (slot_of[b] >= 0) continue;
+            int32_t slot = -1;
+            for (int64_t s = 0; s < C && slot < 0; ++s)
+                if (held[s] < 0 || (done[held[s]] && release[s] <= t)) slot = (int32_t)s;
+            int64_t evict = -1;
+            if (slot < 0) {
+                int64_t best = -1;
+                for (int64_t s = 0; s < C; ++s) {
+                    const int64_t ob = held[s];
+                    if (ob < 0 || done[ob] || std::binary_search(protect.begin(), protect.end(), ob)) continue;
+                    const int64_t nu = next_use(ob, t);
+                    if (nu > best) {
+                        best = nu;
+                        slot = (int32_t)s;
+                    }
+                }
+                if (slot < 0) return false;
+                evict = held[slot];
+                slot_of[evict] = -1;
+                on_host[evict] = 1;
+                ++cp.writebacks;
+            }
+            cp.copies[t].push_back(BwdCopy{b, slot, evict, on_host[b] ? 1 : 0});
+            ++cp.loads;
+            held[slot] = b;
+            slot_of[b] = slot;
+        }
+        const std::vector<int64_t> &blocks = leaves[t].blocks;
+        cp.member_slot[t].assign(blocks.size(), -1);
+        for (size_t m = 0; m < blocks.size(); ++m) cp.member_slot[t][m] = slot_of[blocks[m]];
+        for (int64_t b : tb[t])
+            if (uses[b].back() == t) {
+                done[b] = 1;
+                cp.finals[t].push_back({b, slot_of[b]});
+                release[slot_of[b]] = t + 2;
+                slot_of[b] = -1;
+            }
+    }
+    *out = std::move(cp);
+    return true;
+}
+
+WorkList Planner::leaf_bwd_q_worklist(int64_t t, const BwdCachePlan &c, int rows_per_unit, int bn,
+                                      int heads) const {
+    WorkList wl;
+    for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+        const Entry &e = entries[i];
+        const int64_t sq = c.member_slot[t][e.mq];
+        WlEntry w{};
+        w.q_lo = (int32_t)(sq * block);
+        w.q_hi = (int32_t)(sq * block + block_rows(e.qb));
+        w.q_goff = (int32_t)((e.qb - sq) * block);
+        w.slot = 0;
+        w.out_lo = w.q_lo;  // the block's dQ sums share its slot rows
+        w.flags = 0;
+        w.run_begin = (int32_t)wl.runs.size();
+        for (const KeyRun &r : e.runs)
+            for (int64_t kb = r.b0; kb <= r.b1; ++kb) {
+                const int64_t sk = c.member_slot[t][r.m0 + (kb - r.b0)];
+                push_run(&wl, w.run_begin, (int32_t)(sk * block), (int32_t)block_rows(kb),
+                         (int32_t)((kb - sk) * block));
+            }
+        w.run_count = (int32_t)wl.runs.size() - w.run_begin;
+        wl.entries.push_back(w);
+    }
+    add_units(&wl, heads, rows_per_unit, bn, spec.causal, std::vector<int64_t>(wl.entries.size(), t));
+    return wl;
+}
+
+WorkList Planner::leaf_bwd_kv_worklist(int64_t t, const BwdCachePlan &c, int rows_per_unit, int bn,
+                                       int heads) const {
+    // key member -> query members whose entries' runs hold it
+    const size_t n = leaves[t].blocks.size();
+    std::vector<std::vector<int32_t>> qs_of(n);
+    for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+        const Entry &e = entries[i];
+        for (const KeyRun &r : e.runs)
+            for (int64_t kb = r.b0; kb <= r.b1; ++kb) qs_of[r.m0 + (kb - r.b0)].push_back(e.mq);
+    }
+    WorkList wl;
+    for (size_t mk = 0; mk < n; ++mk) {
+        if (qs_of[mk].empty()) continue;
+        std::vector<int32_t> &qm = qs_of[mk];
+        std::sort(qm.begin(), qm.end());
+        const int64_t kb = leaves[t].blocks[mk], sk = c.member_slot[t][mk];
+        WlEntry w{};
+        w.q_lo = (int32_t)(sk * block);
+        w.q_hi = (int32_t)(sk * block + block_rows(kb));
+        w.q_goff = (int32_t)((kb - sk) * block);
+        w.slot = 0;
+        w.out_lo = w.q_lo;  // the block's dK / dV sums share its slot rows
+        w.flags = 0;
+        w.run_begin = (int32_t)wl.runs.size();
+        for (int32_t m : qm) {
+            const int64_t qb = leaves[t].blocks[m], sq = c.member_slot[t][m];
+            push_run(&wl, w.run_begin, (int32_t)(sq * block), (int32_t)block_rows(qb),
+                     (int32_t)((qb - sq) * block));
+        }
+        w.run_count = (int32_t)wl.runs.size() - w.run_begin;
+        wl.entries.push_back(w);
+    }
+    add_units_kv(&wl, heads, rows_per_unit, bn, spec.causal);
+    return wl;
+}
+
+size_t Planner::bwd_arena_bytes(int g, const BwdCachePlan &c) const {
+    const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d, N = (size_t)spec.N;
+    const size_t rows = (size_t)c.slots * block;
+    const int tile = spec.elem_bytes == 2 ? 128 : 64;
+    ArenaLayout a;
+    a.take(256);                                  // error word
+    a.take((size_t)g * N * sizeof(float));        // lse of the head group
+    a.take((size_t)g * N * sizeof(float));        // D = rowsum(dO * O)
+    for (int s = 0; s < 4; ++s) a.take((size_t)block * g * dd * e);  // O / dO staging, two stages
+    for (int s = 0; s < 4; ++s) a.take(rows * g * dd * e);           // Q, K, V, dO pools
+    for (int s = 0; s < 3; ++s) a.take(rows * g * dd * sizeof(float));  // dQ, dK, dV sums
+    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+        a.take(wl_bytes(leaf_bwd_q_worklist(t, c, tile, tile, g)));
+        a.take(wl_bytes(leaf_bwd_kv_worklist(t, c, tile, tile, g)));
+    }
+    return a.total;
+}
+
+void Planner::size_bwd() {
+    bwd_sizing = BwdSizing{};
+    bwd_cache = BwdCachePlan{};
+    // Grouped-query plans would need several query heads to add into one
+    // key/value head's sums within a launch; they take the device path.
+    if (spec.kv_group() != 1 || spec.shard_count > 1) return;
+    const std::vector<std::vector<int64_t>> tb = bwd_task_blocks(*this);
+    bwd_min_slots = 0;
+    std::vector<int64_t> all;
+    for (size_t t = 0; t < tb.size(); ++t) {
+        std::vector<int64_t> u = tb[t];
+        if (t > 0) u.insert(u.end(), tb[t - 1].begin(), tb[t - 1].end());
+        std::sort(u.begin(), u.end());
+        u.erase(std::unique(u.begin(), u.end()), u.end());
+        bwd_min_slots = std::max<int64_t>(bwd_min_slots, (int64_t)u.size());
+        all.insert(all.end(), tb[t].begin(), tb[t].end());
+    }
+    std::sort(all.begin(), all.end());
+    all.erase(std::unique(all.begin(), all.end()), all.end());
+    bwd_full_slots = (int64_t)all.size();
+    if (bwd_min_slots == 0) return;
+    // For each head group g dividing H: the most slots that fit the budget;
+    // keep the sizing that moves the fewest bytes over the host link (ties
+    // to the larger group).
+    double best_traffic = -1;
+    for (int g = spec.H; g >= 1; --g) {
+        if (spec.H % g) continue;
+        if (!spec.budget && g < spec.H) break;  // unlimited: all heads at once, every block cached
+        BwdCachePlan cp;
+        int64_t C = bwd_full_slots;
+        if (!plan_bwd_cache(C, &cp)) continue;
+        size_t bytes = bwd_arena_bytes(g, cp);
+        if (spec.budget && bytes > spec.budget) {
+            // Largest C in [min, full) whose arena fits (bytes grow with C).
+            int64_t lo = bwd_min_slots, hi = bwd_full_slots - 1, fit = -1;
+            while (lo <= hi) {
+                const int64_t mid = (lo + hi) / 2;
+                BwdCachePlan m;
+                if (plan_bwd_cache(mid, &m) && bwd_arena_bytes(g, m) <= spec.budget) {
+                    fit = mid;
+                    lo = mid + 1;
+                } else {
+                    hi = mid - 1;
+                }
+            }
+            if (fit < 0) continue;
+            C = fit;
+            plan_bwd_cache(C, &cp);
+            bytes = bwd_arena_bytes(g, cp);
+        }
+        const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
+        const size_t acc = (size_t)block * g * spec.d * sizeof(float);
+        const size_t groups = (size_t)(spec.H / g);
+        const size_t N = (size_t)spec.N;
+        const size_t h2d = groups * ((size_t)g * N * sizeof(float) + 2 * N * g * spec.d * spec.elem_bytes +
+                                     (size_t)cp.loads * 4 * blk + (size_t)cp.writebacks * 3 * acc);
+        const size_t d2h = groups * (3 * N * g * spec.d * spec.elem_bytes + (size_t)cp.writebacks * 3 * acc);
+        const double traffic = (double)h2d + (double)d2h;
+        if (best_traffic < 0 || traffic < best_traffic) {
+            best_traffic = traffic;
+            bwd_sizing.head_group = g;
+            bwd_sizing.arena = bytes;
+            bwd_sizing.slots = C;
+            bwd_sizing.h2d = h2d * (size_t)spec.B;
+            bwd_sizing.d2h = d2h * (size_t)spec.B;
+            bwd_sizing.spill_host = cp.writebacks ? 3 * N * g * spec.d * sizeof(float) : 0;
+            bwd_cache = std::move(cp);
+        }
+    }
 }
 
 }  // namespace cqsa

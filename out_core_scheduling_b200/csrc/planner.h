@@ -92,6 +92,40 @@ struct PoolPlan {
     int64_t q_copies = 0, kv_copies = 0;                // per head group
 };
 
+// Device block cache of the streamed backward.  A slot holds one block of
+// the current head group: its Q, K, V and dO rows ([block, g, d] each, the
+// plan dtype) and its running dQ, dK and dV sums ([block, g, d] fp32 each).
+// A block's sums start at zero on its first task, collect the terms of every
+// task that contains it, and leave as the finished gradients after its last
+// task.  The task order is fixed, so the cache is simulated at plan time
+// with Belady's rule; a block evicted between two of its tasks has its
+// sums written back to host memory and brought back on its next task.
+// Blocks of the current and the previous task stay (the previous task's
+// kernels may still run), and so does the slot of a block finished by the
+// previous task (its gradients may still be on their way to the host).
+struct BwdCopy {
+    int64_t block;    // global block brought into `slot`
+    int32_t slot;
+    int64_t evict;    // unfinished block written back from `slot` first (-1: none)
+    int32_t reload;   // 1: the block's sums come back from host memory; 0: they start at zero
+};
+
+struct BwdCachePlan {
+    int64_t slots = 0;
+    std::vector<std::vector<BwdCopy>> copies;                      // per leaf task, in copy order
+    std::vector<std::vector<int32_t>> member_slot;                 // per leaf task, per member
+    std::vector<std::vector<std::pair<int64_t, int32_t>>> finals;  // per leaf task: (block, slot) finished by it
+    int64_t loads = 0, writebacks = 0;                             // per head group
+};
+
+struct BwdSizing {
+    int head_group = 0;     // 0: no streamed backward fits the budget
+    size_t arena = 0;       // device bytes
+    int64_t slots = 0;
+    size_t h2d = 0, d2h = 0;
+    size_t spill_host = 0;  // pinned host bytes for written-back sums (0: none needed)
+};
+
 struct Sizing {
     int head_group = 0;
     size_t host_arena = 0;
@@ -186,6 +220,20 @@ public:
     // Simulate the block cache with the given capacities; false if some
     // task (with its predecessor) needs more slots than there are.
     bool plan_pool(int64_t q_slots, int64_t kv_slots, PoolPlan *out) const;
+
+    // Streamed backward: the block cache with `slots` slots (false if a task
+    // and its predecessor need more), its device arena for head group g, and
+    // the two work lists of leaf t in cache coordinates (rows of block b at
+    // slot * block): query-stationary (dq, one entry per (task, query
+    // block)) and key-stationary (dk and dv, one entry per (task, key
+    // block)); each entry's sums go to the block's own slot rows.
+    bool plan_bwd_cache(int64_t slots, BwdCachePlan *out) const;
+    size_t bwd_arena_bytes(int g, const BwdCachePlan &c) const;
+    WorkList leaf_bwd_q_worklist(int64_t t, const BwdCachePlan &c, int rows_per_unit, int bn, int heads) const;
+    WorkList leaf_bwd_kv_worklist(int64_t t, const BwdCachePlan &c, int rows_per_unit, int bn, int heads) const;
+    BwdCachePlan bwd_cache;         // cache plan of the chosen backward sizing
+    BwdSizing bwd_sizing;
+    int64_t bwd_min_slots = 0, bwd_full_slots = 0;
     PoolPlan pool;                  // cache plan of the chosen sizing
     int64_t min_q_slots = 0, min_kv_slots = 0, full_q_slots = 0, full_kv_slots = 0;
 
@@ -197,6 +245,7 @@ private:
     std::vector<int64_t> entry_begin_of_leaf_;  // first entry index of each leaf
     std::vector<int32_t> first_leaf_, last_leaf_; // per query block
     void size_plan();
+    void size_bwd();
 };
 
 // Lexicographically first perfect difference set of size l mod l(l-1)+1
