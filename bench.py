@@ -326,6 +326,8 @@ def run_ours(args, W):
         if D.world == 1:
             sub = argparse.Namespace(**vars(args))
             sub.no_e2e = sub.no_cpu = True
+            if sub.backward_host_steps < 0:
+                sub.backward_host_steps = 1
             result["streamed"] = measure(sub, WORKLOADS[STREAMED_EXTRA], D, STREAMED_EXTRA,
                                          args.streamed_steps, 3, extras=False)
             torch.cuda.empty_cache()
@@ -538,6 +540,9 @@ def measure(args, W, D, workload, steps, warmup, extras):
                          "path": "cqsa_forward(CQSA_HOST), the timed path itself"}
         result["streaming"] = streaming_report(W, infos, flops_step, ms / steps, peaks,
                                                free_before, torch)
+        if args.backward_host_steps > 0:
+            result["backward_streamed"] = run_backward_host(args, W, D, plans, infos, q, k, v, outs, lses,
+                                                            flops_step, stream, peaks, result["streaming"])
     elif not args.no_e2e:
         result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream)
 
@@ -602,6 +607,70 @@ def run_backward(args, W, D, plans, q, k, v, outs, lses, flops_step, stream, pea
             "peak": peak, "gpu_launches": sum(s["bwd_launches"] + s["merge_launches"] for s in stats),
             "path": "cqsa_backward: D = rowsum(dout * out); dq kernel over the (task, query block) list, "
                     "dk/dv kernel over the (task, key block) list, slot sums"}
+
+
+def run_backward_host(args, W, D, plans, infos, q, k, v, outs, lses, flops_step, stream, peaks, fwd_stream):
+    """cqsa_backward(CQSA_HOST) of each variant from pinned host memory under
+    the workload's budget (the forward's outputs and a seeded pinned dout):
+    2.5x the forward's useful flops per step, the bound from the sustained
+    bf16 peak and the measured host link, and the device memory it takes."""
+    import torch
+    from out_core_scheduling_b200 import cqsa
+    from out_core_scheduling_b200.inputs import make_qkv
+
+    N, H, d = W["N"], W["H"], W["d"]
+    gd = make_qkv(N, H, d, dtype=q.dtype, seed=1000 + D.rank, device=f"cuda:{D.local_rank}", dist=W["dist"])[0]
+    dout = gd.cpu().pin_memory()
+    del gd
+    grads = [tuple(torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3)) for _ in plans]
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    def step():
+        for p, o, l, g in zip(plans, outs, lses, grads):
+            cqsa.cqsa_backward(p, q, k, v, o, l, dout, *g, host_or_device=cqsa.CQSA_HOST, stream=stream)
+
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(args.backward_host_warmup):
+        step()
+    for p in plans:
+        p.sync(stream)
+    free1, _ = torch.cuda.mem_get_info()
+    sampler = ClockSampler(gpu_id_for_smi(torch, D.local_rank))
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(D.local_rank)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.backward_host_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier(D.local_rank)
+    clocks = sampler.stop()
+    for p in plans:
+        p.sync(stream)
+    ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}") / args.backward_host_steps
+    bflops = 2.5 * flops_step
+    h2d = sum(i["bwd_h2d_bytes"] for i in infos)
+    d2h = sum(i["bwd_d2h_bytes"] for i in infos)
+    t_c = bflops / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3
+    t_h = h2d / (fwd_stream["h2d_gbs"] * 1e9) * 1e3
+    t_d = d2h / (fwd_stream["d2h_gbs"] * 1e9) * 1e3
+    bound = max(t_c, t_h, t_d)
+    return {"value": bflops * D.world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "steps": args.backward_host_steps, "warmup": args.backward_host_warmup,
+            "useful_flops_per_step": bflops, "h2d_bytes": h2d, "d2h_bytes": d2h,
+            "t_compute_at_peak_ms": t_c, "t_h2d_ms": t_h, "t_d2h_ms": t_d, "t_bound_ms": bound,
+            "bound": "compute" if bound == t_c else ("h2d" if bound == t_h else "d2h"),
+            "efficiency": bound / ms, "peak_source": "sustained bf16 dense",
+            "head_group": infos[0]["bwd_head_group"], "cache_slots": infos[0]["bwd_cache_slots"],
+            "num_blocks": infos[0]["num_blocks"], "writebacks_per_head_group": infos[0]["bwd_writebacks"],
+            "library_arena_gib": max(i["bwd_host_arena_bytes"] for i in infos) / GiB,
+            "device_free_delta_gib": (free0 - free1) / GiB, "budget_gib": W["budget"] / GiB,
+            "clocks": clocks,
+            "path": "cqsa_backward(CQSA_HOST): per head group lse up, D = rowsum(dout * out) per block, then "
+                    "the leaf tasks through the backward block cache, gradient sums written back when evicted"}
 
 
 def run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, slots_value):
@@ -817,12 +886,18 @@ def main(argv=None):
                     help="default workload: skip the streamed / fp32 (one GPU) or sharded (N > 1) extra keys")
     ap.add_argument("--streamed-steps", type=int, default=2,
                     help="timed steps of the streamed extra workload (about 2 s each)")
+    ap.add_argument("--backward-host-steps", type=int, default=-1,
+                    help="host-streamed workloads: timed steps of the host-mode backward "
+                         "(default: 1 in the default run's streamed extra, 0 otherwise)")
+    ap.add_argument("--backward-host-warmup", type=int, default=1)
     ap.add_argument("--shard", action="store_true",
                     help="one problem split over the ranks in task shards (strong scaling; not the default line)")
     args = ap.parse_args(argv)
     if args.warmup < 0 or args.steps < 1:
         ap.error("need --steps >= 1 and --warmup >= 0")
     W = WORKLOADS[args.workload]
+    if args.backward_host_steps < 0 and not (args.workload == DEFAULT_WORKLOAD and not args.no_extra):
+        args.backward_host_steps = 0
     if args.impl == "reference":
         run_reference(args, W)
     elif args.shard:

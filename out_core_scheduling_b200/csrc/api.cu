@@ -258,6 +258,13 @@ struct cqsa_plan {
     char *part_arena = nullptr;
     int *part_err = nullptr;
     DevWl part_wl;
+    // Owner exchange of a sharded forward: layout and the merge's table.
+    bool shard_ready = false;
+    ShardLayout shard;
+    char *shard_arena = nullptr;
+    int32_t *shard_nsrc = nullptr;
+    int64_t *shard_offs = nullptr;
+    int shard_max_src = 1;
 
     // Streamed path.
     char *host_arena = nullptr;
@@ -938,6 +945,49 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
     cudaStreamWaitEvent(stream, P->ev_done_out, 0);
 }
 
+// ------------------------------------------------------------ owner exchange
+cqsa_status_t setup_shard_impl(cqsa_plan_t *P, bool device) {
+    if (!P->shard_ready) {
+        P->shard = P->pl.shard_layout(P->elem);
+        P->shard_ready = true;
+    }
+    if (!device || P->shard_arena) return CQSA_OK;
+    const ShardLayout &L = P->shard;
+    int max_src = 1;
+    for (const auto &o : L.own_offsets) max_src = std::max<int>(max_src, (int)o.size());
+    if (max_src > 32)
+        return fail(CQSA_ERR_UNSUPPORTED, "a query block has partials from %d ranks; the owner merge takes 32",
+                    max_src);
+    const size_t nb = (size_t)std::max<int64_t>(1, L.own_count);
+    std::vector<int32_t> ns(nb, 0);
+    std::vector<int64_t> offs(nb * max_src, 0);
+    for (int64_t i = 0; i < L.own_count; ++i) {
+        ns[i] = (int32_t)L.own_offsets[i].size();
+        for (size_t j = 0; j < L.own_offsets[i].size(); ++j) offs[i * max_src + j] = L.own_offsets[i][j];
+    }
+    ArenaLayout a;
+    const size_t o_ns = a.take(ns.size() * sizeof(int32_t));
+    const size_t o_off = a.take(offs.size() * sizeof(int64_t));
+    char *arena = nullptr;
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
+    P->shard_arena = arena;
+    P->shard_nsrc = reinterpret_cast<int32_t *>(arena + o_ns);
+    P->shard_offs = reinterpret_cast<int64_t *>(arena + o_off);
+    P->shard_max_src = max_src;
+    CK(lib_upload(P->shard_nsrc, ns.data(), ns.size() * sizeof(int32_t)));
+    CK(lib_upload(P->shard_offs, offs.data(), offs.size() * sizeof(int64_t)));
+    return CQSA_OK;
+}
+
+cqsa_status_t setup_shard(cqsa_plan_t *P, bool device) {
+    const cqsa_status_t st = guarded([&] { return setup_shard_impl(P, device); });
+    if (st != CQSA_OK && P->shard_arena) {
+        cudaFree(P->shard_arena);
+        P->shard_arena = nullptr;
+    }
+    return st;
+}
+
 // ------------------------------------------------------------ streamed backward
 // The backward from pinned host memory under the plan's memory budget
 // ([A]: forward and backward beyond the memory limit; [B] "Precise
@@ -1555,6 +1605,96 @@ cqsa_status_t cqsa_partial_finish(cqsa_plan_t *plan, const float *o_sum, const f
     return CQSA_OK;
 }
 
+cqsa_status_t cqsa_shard_layout(cqsa_plan_t *plan, int64_t *send_counts, int64_t *recv_counts, int64_t *row_lo,
+                                int64_t *rows_max, size_t *chunk_bytes) {
+    if (!plan || !send_counts || !recv_counts || !row_lo || !rows_max || !chunk_bytes)
+        return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    cqsa_status_t st = setup_shard(plan, false);
+    if (st != CQSA_OK) return st;
+    const ShardLayout &L = plan->shard;
+    for (int k = 0; k < L.G; ++k) {
+        send_counts[k] = L.send_counts[k];
+        recv_counts[k] = L.recv_counts[k];
+        row_lo[k] = L.row_lo[k];
+    }
+    row_lo[L.G] = L.row_lo[L.G];
+    *rows_max = L.rows_max;
+    *chunk_bytes = L.chunk_bytes;
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_shard_pack(cqsa_plan_t *plan, const float *o_part, const float *lse_part, float *send,
+                              void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    if ((st = setup_shard(plan, false)) != CQSA_OK) return st;
+    const ShardLayout &L = plan->shard;
+    const Planner &pl = plan->pl;
+    const int64_t N = pl.spec.N, H = pl.spec.H, d = pl.spec.d;
+    if (!L.send.empty()) {
+        const void *ptrs[3] = {o_part, lse_part, send};
+        const char *names[3] = {"o_part", "lse_part", "send"};
+        for (int i = 0; i < 3; ++i)
+            if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (const ShardPiece &pc : L.send) {
+        const int64_t nb = pl.block_rows(pc.block), r0 = pc.block * pl.block;
+        CK(cudaMemcpyAsync(send + pc.offset, o_part + r0 * H * d, (size_t)(nb * H * d) * sizeof(float),
+                           cudaMemcpyDeviceToDevice, s));
+        CK(cudaMemcpy2DAsync(send + pc.offset + nb * H * d, (size_t)nb * sizeof(float), lse_part + r0,
+                             (size_t)N * sizeof(float), (size_t)nb * sizeof(float), (size_t)H,
+                             cudaMemcpyDeviceToDevice, s));
+    }
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_shard_merge(cqsa_plan_t *plan, const float *recv, void *chunk, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    if ((st = setup_shard(plan, true)) != CQSA_OK) return st;
+    const ShardLayout &L = plan->shard;
+    const Planner &pl = plan->pl;
+    if ((st = check_ptr(chunk, false, "chunk")) != CQSA_OK) return st;
+    const int64_t lo = L.row_lo[L.me], hi = L.row_lo[L.me + 1];
+    if (hi <= lo) return CQSA_OK;
+    if ((st = check_ptr(recv, false, "recv")) != CQSA_OK) return st;
+    char *c = static_cast<char *>(chunk);
+    CK(launch_shard_merge(pl.spec.d, plan->elem, recv, plan->shard_nsrc, plan->shard_offs, plan->shard_max_src,
+                          pl.block, pl.spec.N, pl.spec.H, L.own_first, lo, hi, L.rows_max, c,
+                          reinterpret_cast<float *>(c + L.out_bytes), static_cast<cudaStream_t>(stream)));
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_shard_unpack(cqsa_plan_t *plan, const void *chunks, void *out, float *lse, void *stream) {
+    if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
+    cqsa_status_t st = check_device(plan);
+    if (st != CQSA_OK) return st;
+    if ((st = setup_shard(plan, false)) != CQSA_OK) return st;
+    const void *ptrs[3] = {chunks, out, lse};
+    const char *names[3] = {"chunks", "out", "lse"};
+    for (int i = 0; i < 3; ++i)
+        if ((st = check_ptr(ptrs[i], false, names[i])) != CQSA_OK) return st;
+    const ShardLayout &L = plan->shard;
+    const Planner &pl = plan->pl;
+    const int64_t N = pl.spec.N, H = pl.spec.H, d = pl.spec.d, e = plan->elem;
+    const char *src = static_cast<const char *>(chunks);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    for (int k = 0; k < L.G; ++k) {
+        const int64_t lo = L.row_lo[k], n = L.row_lo[k + 1] - lo;
+        if (n <= 0) continue;
+        const char *ck = src + (size_t)k * L.chunk_bytes;
+        CK(cudaMemcpyAsync(static_cast<char *>(out) + (size_t)(lo * H * d * e), ck, (size_t)(n * H * d * e),
+                           cudaMemcpyDeviceToDevice, s));
+        CK(cudaMemcpy2DAsync(lse + lo, (size_t)N * sizeof(float), ck + L.out_bytes,
+                             (size_t)L.rows_max * sizeof(float), (size_t)n * sizeof(float), (size_t)H,
+                             cudaMemcpyDeviceToDevice, s));
+    }
+    return CQSA_OK;
+}
+
 cqsa_status_t cqsa_plan_sync(cqsa_plan_t *plan, void *stream) {
     if (!plan) return fail(CQSA_ERR_INVALID_ARG, "null plan");
     if (plan->device < 0) return CQSA_OK;
@@ -1829,6 +1969,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
         if (plan->bwd.arena) cudaFree(plan->bwd.arena);
         if (plan->bwd_shard.arena) cudaFree(plan->bwd_shard.arena);
         if (plan->part_arena) cudaFree(plan->part_arena);
+        if (plan->shard_arena) cudaFree(plan->shard_arena);
         cudaGetLastError();
     }
     delete plan;

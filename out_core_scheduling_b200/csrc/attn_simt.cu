@@ -7,14 +7,17 @@
 // output and its log-sum-exp ("Stream-CQSA: Breaking the Billion-Token
 // Barrier on a Single GPU", section "Implementation", step 3).
 //
-// 256 threads as 16 x 16: thread (ty, tx) owns query rows 4ty..4ty+3, key
-// columns 4tx..4tx+3 of each 64-key tile, and output features
-// 64g + 4tx .. 64g + 4tx + 3 (g < d / 64).  Q, K and P are kept transposed in
-// shared memory ([feature or key][row], rows padded to 68 floats, 16-byte
-// aligned), so every step of both products reads one float4 per operand;
-// the tile's K and V are fetched with one vector load per four features,
-// all issued before any store.  Row maxima and sums are reduced over the 16
-// threads of a row with warp shuffles.
+// 256 threads as 16 x 16: thread (ty, tx) owns query rows 4ty..4ty+3, keys
+// tx, tx+16, tx+32, tx+48 of each 64-key tile, and output features
+// 64g + 4tx .. 64g + 4tx + 3 (g < d / 64).  Q and P are kept transposed in
+// shared memory ([feature or key][row], rows padded to 68 floats); K and V
+// tiles stay row-major (K rows padded to d + 4 floats, so the eight lanes of
+// a 16-byte load phase hit distinct banks) and arrive by cp.async in two
+// stages: the next tile's copies are in flight while the current tile is
+// computed.  Every product step reads 16-byte vectors: Q^T and K for four
+// features at a time (64 FMAs per eight loads), P^T and V for one key.  Row
+// maxima and sums are reduced over the 16 threads of a row with warp
+// shuffles.
 //
 // Key split: a unit may be computed by a cluster of S = 1, 2 or 4 CTAs (the
 // launcher picks S so that small problems still fill every SM): CTA rank r
@@ -23,7 +26,6 @@
 // distributed shared memory before rank 0 writes the unit's result, so the
 // work list, the slots and the merge are those of an unsplit unit.
 #include <cooperative_groups.h>
-#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,17 +39,17 @@ namespace simt {
 constexpr int BM = 64;
 constexpr int BN = 64;
 constexpr int THREADS = 256;
-constexpr int LD = 68;  // padded row of the transposed tiles, in floats
+constexpr int LD = 68;  // padded row of the transposed Q and P tiles, in floats
+template <int D>
+struct Layout {
+    static constexpr int KD = D + 4;  // padded K row, in floats
+    static constexpr int Q = 0;
+    static constexpr int K = Q + D * LD;          // two stages of [BN][KD]
+    static constexpr int V = K + 2 * BN * KD;     // two stages of [BN][D]
+    static constexpr int P = V + 2 * BN * D;      // [BN][LD]
+    static constexpr int FLOATS = P + BN * LD;
+};
 }  // namespace simt
-
-// Four consecutive elements as fp32 (16-byte fp32 or 8-byte bf16 load).
-__device__ __forceinline__ float4 load4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
 
 __device__ __forceinline__ void f4_split(const float4 v, float (&a)[4]) {
     a[0] = v.x;
@@ -56,18 +58,60 @@ __device__ __forceinline__ void f4_split(const float4 v, float (&a)[4]) {
     a[3] = v.w;
 }
 
-template <int D, typename T>
+// 16-byte global -> shared copy that bypasses registers; src_bytes = 0
+// fills the destination with zeros (rows past the end of a key run).
+__device__ __forceinline__ void cp_async16(float *dst, const float *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Walks the key tiles of an entry's runs in order (the same sequence on
+// every thread of the CTA).
+struct TileWalk {
+    int r = 0;
+    int32_t ks = 0, hi = 0;
+    WlRun run{};
+    bool valid = false;
+    __device__ __forceinline__ void open(const WlEntry &e, const WlRun *runs, int32_t q_end, int causal) {
+        for (; r < e.run_count; ++r) {
+            run = runs[e.run_begin + r];
+            int32_t lo;
+            clip_run(e, run, q_end, causal, &lo, &hi);
+            if (hi > lo) {
+                ks = lo;
+                valid = true;
+                return;
+            }
+        }
+        valid = false;
+    }
+    __device__ __forceinline__ void next(const WlEntry &e, const WlRun *runs, int32_t q_end, int causal) {
+        ks += simt::BN;
+        if (ks < hi) return;
+        ++r;
+        open(e, runs, q_end, causal);
+    }
+};
+
+template <int D>
 __global__ void __launch_bounds__(simt::THREADS)
-    attn_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+    attn_simt_kernel(const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v,
                      const AttnParams p) {
     using namespace simt;
+    using L = Layout<D>;
+    constexpr int KD = L::KD;
     constexpr int G = D / 64;                 // float4 groups of output features per thread
-    constexpr int NL = BN * D / 4 / THREADS;  // vector loads per thread per K (or V) tile
+    constexpr int NC = BN * D / 4 / THREADS;  // 16-byte copies per thread per K (or V) tile
     extern __shared__ __align__(16) float smf[];
-    float *Qt = smf;            // [D][LD]   Q transposed
-    float *Kt = Qt + D * LD;    // [D][LD]   K transposed
-    float *Vs = Kt + D * LD;    // [BN][D]
-    float *Pt = Vs + BN * D;    // [BN][LD]  P transposed
+    float *Qt = smf + L::Q;     // [D][LD]   Q transposed
+    float *Ks = smf + L::K;     // [2][BN][KD]
+    float *Vs = smf + L::V;     // [2][BN][D]
+    float *Pt = smf + L::P;     // [BN][LD]  P transposed
 
     namespace cg = cooperative_groups;
     const cg::cluster_group cluster = cg::this_cluster();
@@ -75,11 +119,6 @@ __global__ void __launch_bounds__(simt::THREADS)
     const int rank = (int)cluster.block_rank();
     const WlUnit u = p.units[blockIdx.x / S];
     const WlEntry e = p.entries[u.entry];
-    // This CTA's share of the unit's key tiles, in run order.
-    const int32_t ntiles = unit_key_tiles(e, p.runs, u.q0, BM, p.causal, BN);
-    const int32_t t_lo = (int32_t)((int64_t)ntiles * rank / S);
-    const int32_t t_hi = (int32_t)((int64_t)ntiles * (rank + 1) / S);
-    int32_t t_at = 0;  // index of the next key tile of the unit
     const int H = p.H;
     const int h = u.head;
     const int hkv = (h + p.hq_off) / p.kv_group - p.hk_off;  // grouped-query attention
@@ -87,13 +126,42 @@ __global__ void __launch_bounds__(simt::THREADS)
     const int32_t q0 = u.q0;
     const int32_t q_end = min(q0 + BM, e.q_hi);
     const float sl2 = p.scale_log2;
+    const int causal = p.causal;
+    // This CTA's share of the unit's key tiles, in run order.
+    const int32_t ntiles = unit_key_tiles(e, p.runs, q0, BM, causal, BN);
+    const int32_t t_lo = (int32_t)((int64_t)ntiles * rank / S);
+    const int32_t t_hi = (int32_t)((int64_t)ntiles * (rank + 1) / S);
+    const int32_t my_tiles = t_hi - t_lo;
+
+    // The copy walk runs one tile ahead of the compute walk.
+    TileWalk cw, xw;
+    cw.open(e, p.runs, q_end, causal);
+    for (int32_t i = 0; i < t_lo; ++i) cw.next(e, p.runs, q_end, causal);
+    xw = cw;
+    auto issue = [&](const TileWalk &w, int stage) {
+        float *kd = Ks + stage * BN * KD, *vd = Vs + stage * BN * D;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const int idx = 4 * (tid + j * THREADS);
+            const int rr = idx / D, c = idx % D;
+            const int32_t key = w.ks + rr;
+            const bool in = key < w.run.k_hi;
+            const int64_t off = ((int64_t)(in ? key : w.ks) * p.Hkv + hkv) * D + c;
+            cp_async16(kd + rr * KD + c, k + off, in ? 16 : 0);
+            cp_async16(vd + rr * D + c, v + off, in ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    if (my_tiles > 0) issue(cw, 0);
 
 #pragma unroll
     for (int j = 0; j < BM * D / 4 / THREADS; ++j) {
         const int idx = 4 * (tid + j * THREADS);
         const int r = idx / D, c = idx % D;
         const int32_t row = q0 + r;
-        const float4 x = row < q_end ? load4(q + ((int64_t)row * H + h) * D + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 x =
+            row < q_end ? __ldg(reinterpret_cast<const float4 *>(q + ((int64_t)row * H + h) * D + c))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
         Qt[(c + 0) * LD + r] = x.x;
         Qt[(c + 1) * LD + r] = x.y;
         Qt[(c + 2) * LD + r] = x.z;
@@ -112,109 +180,95 @@ __global__ void __launch_bounds__(simt::THREADS)
             for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = 0.f;
     }
 
-    for (int r = 0; r < e.run_count && t_at < t_hi; ++r) {
-        const WlRun run = p.runs[e.run_begin + r];
-        int32_t lo, hi;
-        clip_run(e, run, q_end, p.causal, &lo, &hi);
-        const int32_t nt = hi > lo ? (hi - lo + BN - 1) / BN : 0;
-        if (t_at + nt <= t_lo) {  // the whole run lies before this CTA's share
-            t_at += nt;
-            continue;
+    for (int32_t t = 0; t < my_tiles; ++t) {
+        const int stage = t & 1;
+        const int32_t ks = xw.ks;
+        const WlRun run = xw.run;
+        // Next tile's copies into the other stage (freed by the barrier at
+        // the end of the previous tile), then wait for this tile's.
+        if (t + 1 < my_tiles) {
+            cw.next(e, p.runs, q_end, causal);
+            issue(cw, stage ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        if (t_at < t_lo) {
-            lo += (t_lo - t_at) * BN;
-            t_at = t_lo;
-        }
-        for (int32_t ks = lo; ks < hi && t_at < t_hi; ks += BN, ++t_at) {
-            __syncthreads();
-            float4 kr[NL], vr[NL];
+        __syncthreads();
+        const float *Kc = Ks + stage * BN * KD, *Vc = Vs + stage * BN * D;
+        float sacc[4][4];
 #pragma unroll
-            for (int j = 0; j < NL; ++j) {
-                const int idx = 4 * (tid + j * THREADS);
-                const int rr = idx / D, c = idx % D;
-                const int32_t key = ks + rr;
-                const int64_t off = ((int64_t)key * p.Hkv + hkv) * D + c;
-                const bool in = key < run.k_hi;
-                kr[j] = in ? load4(k + off) : make_float4(0.f, 0.f, 0.f, 0.f);
-                vr[j] = in ? load4(v + off) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < NL; ++j) {
-                const int idx = 4 * (tid + j * THREADS);
-                const int rr = idx / D, c = idx % D;
-                Kt[(c + 0) * LD + rr] = kr[j].x;
-                Kt[(c + 1) * LD + rr] = kr[j].y;
-                Kt[(c + 2) * LD + rr] = kr[j].z;
-                Kt[(c + 3) * LD + rr] = kr[j].w;
-                *reinterpret_cast<float4 *>(Vs + rr * D + c) = vr[j];
-            }
-            __syncthreads();
-            float sacc[4][4];
+            for (int mm = 0; mm < 4; ++mm) sacc[i][mm] = 0.f;
+#pragma unroll 2
+        for (int kk = 0; kk < D; kk += 4) {
+            float qa[4][4], ka[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int u4 = 0; u4 < 4; ++u4) f4_split(*reinterpret_cast<const float4 *>(Qt + (kk + u4) * LD + 4 * ty), qa[u4]);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) sacc[i][jj] = 0.f;
-#pragma unroll 8
-            for (int kk = 0; kk < D; ++kk) {
-                float qa[4], ka[4];
-                f4_split(*reinterpret_cast<const float4 *>(Qt + kk * LD + 4 * ty), qa);
-                f4_split(*reinterpret_cast<const float4 *>(Kt + kk * LD + 4 * tx), ka);
+            for (int mm = 0; mm < 4; ++mm)
+                f4_split(*reinterpret_cast<const float4 *>(Kc + (tx + 16 * mm) * KD + kk), ka[mm]);
+#pragma unroll
+            for (int u4 = 0; u4 < 4; ++u4)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) sacc[i][jj] = fmaf(qa[i], ka[jj], sacc[i][jj]);
-            }
-            float pm[4][4];
+                    for (int mm = 0; mm < 4; ++mm) sacc[i][mm] = fmaf(qa[u4][i], ka[mm][u4], sacc[i][mm]);
+        }
+        float pm[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float x[4];
-                float mx = -INFINITY;
+        for (int i = 0; i < 4; ++i) {
+            float x[4];
+            float mx = -INFINITY;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int32_t key = ks + 4 * tx + jj;
-                    const bool keep = key < run.k_hi && (!p.causal || (int64_t)key + run.k_goff <= qg[i]);
-                    x[jj] = keep ? sacc[i][jj] * sl2 : -INFINITY;
-                    mx = fmaxf(mx, x[jj]);
-                }
-#pragma unroll
-                for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                const float m_new = fmaxf(m[i], mx);
-                const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m[i] - m_new);
-                float sum = 0.f;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    pm[i][jj] = (m_new == -INFINITY) ? 0.f : exp2f(x[jj] - m_new);
-                    sum += pm[i][jj];
-                }
-#pragma unroll
-                for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                l[i] = l[i] * alpha + sum;
-                m[i] = m_new;
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) o[i][g][jj] *= alpha;
+            for (int mm = 0; mm < 4; ++mm) {
+                const int32_t key = ks + tx + 16 * mm;
+                const bool keep = key < run.k_hi && (!causal || (int64_t)key + run.k_goff <= qg[i]);
+                x[mm] = keep ? sacc[i][mm] * sl2 : -INFINITY;
+                mx = fmaxf(mx, x[mm]);
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                *reinterpret_cast<float4 *>(Pt + (4 * tx + jj) * LD + 4 * ty) =
-                    make_float4(pm[0][jj], pm[1][jj], pm[2][jj], pm[3][jj]);
-            __syncthreads();
+            for (int off = 8; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float m_new = fmaxf(m[i], mx);
+            const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m[i] - m_new);
+            float sum = 0.f;
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+                pm[i][mm] = (m_new == -INFINITY) ? 0.f : exp2f(x[mm] - m_new);
+                sum += pm[i][mm];
+            }
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            l[i] = l[i] * alpha + sum;
+            m[i] = m_new;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) o[i][g][jj] *= alpha;
+        }
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm)
+            *reinterpret_cast<float4 *>(Pt + (tx + 16 * mm) * LD + 4 * ty) =
+                make_float4(pm[0][mm], pm[1][mm], pm[2][mm], pm[3][mm]);
+        __syncthreads();
 #pragma unroll 4
-            for (int c = 0; c < BN; ++c) {
-                float pa[4];
-                f4_split(*reinterpret_cast<const float4 *>(Pt + c * LD + 4 * ty), pa);
+        for (int c = 0; c < BN; ++c) {
+            float pa[4];
+            f4_split(*reinterpret_cast<const float4 *>(Pt + c * LD + 4 * ty), pa);
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float va[4];
-                    f4_split(*reinterpret_cast<const float4 *>(Vs + c * D + 64 * g + 4 * tx), va);
+            for (int g = 0; g < G; ++g) {
+                float va[4];
+                f4_split(*reinterpret_cast<const float4 *>(Vc + c * D + 64 * g + 4 * tx), va);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = fmaf(pa[i], va[jj], o[i][g][jj]);
-                }
+                    for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = fmaf(pa[i], va[jj], o[i][g][jj]);
             }
         }
+        // Everyone is done with this stage and with P before the next tile
+        // overwrites them.
+        __syncthreads();
+        xw = cw;
     }
 
     if (S > 1) {
@@ -259,7 +313,7 @@ __global__ void __launch_bounds__(simt::THREADS)
         }
         cluster.sync();
         if (rank > 0) return;
-        static_assert(NV * THREADS <= 2 * D * LD + BN * D + BN * LD, "combine area fits the shared tiles");
+        static_assert(NV * THREADS <= L::FLOATS, "combine area fits the shared tiles");
     }
 
 #pragma unroll
@@ -277,7 +331,7 @@ __global__ void __launch_bounds__(simt::THREADS)
             FoldWeights w{0.f, 1.f, lse_n};
             if (!first) w = fold_weights(p.acc_lse[(int64_t)h * p.acc_rows + grow], lse_n);
             float *acc = p.acc_o + (grow * H + h) * D;
-            T *dst = static_cast<T *>(p.out) + (out_row * H + h) * D;
+            float *dst = static_cast<float *>(p.out) + (out_row * H + h) * D;
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -320,18 +374,18 @@ static int simt_split(int num_units, int resident) {
     return S;
 }
 
-template <int D, typename T>
+template <int D>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const AttnParams &p,
                                  int num_units, cudaStream_t stream) {
     using namespace simt;
-    const size_t smem = sizeof(float) * (size_t)(D * LD + D * LD + BN * D + BN * LD);
-    cudaError_t err = cudaFuncSetAttribute(attn_simt_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = sizeof(float) * (size_t)Layout<D>::FLOATS;
+    cudaError_t err = cudaFuncSetAttribute(attn_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
     static int resident = 0;  // CTAs of this instantiation one SM holds (the same on every sm_100 device)
     if (resident < 1) {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_simt_kernel<D, T>, THREADS, smem) != cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_simt_kernel<D>, THREADS, smem) != cudaSuccess)
             cudaGetLastError();
         resident = n > 0 ? n : 1;
     }
@@ -348,24 +402,21 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attn_simt_kernel<D, T>, static_cast<const T *>(q), static_cast<const T *>(k),
-                              static_cast<const T *>(v), p);
+    return cudaLaunchKernelEx(&cfg, attn_simt_kernel<D>, static_cast<const float *>(q),
+                              static_cast<const float *>(k), static_cast<const float *>(v), p);
 }
 
 cudaError_t launch_attn_simt(int d, int elem_bytes, const void *q, const void *k, const void *v,
                              const AttnParams &p, int num_units, cudaStream_t stream) {
     if (num_units <= 0) return cudaSuccess;
-    // The kernel reads four consecutive elements per load.
+    // fp32 only (bf16 plans run the tensor-core kernel); the kernel copies
+    // 16-byte vectors.
+    if (elem_bytes != 4) return cudaErrorInvalidValue;
     const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                           reinterpret_cast<uintptr_t>(v)) & (uintptr_t)(4 * elem_bytes - 1);
+                           reinterpret_cast<uintptr_t>(v)) & (uintptr_t)15;
     if (mis) return cudaErrorMisalignedAddress;
-    if (elem_bytes == 4) {
-        if (d == 64) return launch_simt_t<64, float>(q, k, v, p, num_units, stream);
-        if (d == 128) return launch_simt_t<128, float>(q, k, v, p, num_units, stream);
-    } else if (elem_bytes == 2) {
-        if (d == 64) return launch_simt_t<64, __nv_bfloat16>(q, k, v, p, num_units, stream);
-        if (d == 128) return launch_simt_t<128, __nv_bfloat16>(q, k, v, p, num_units, stream);
-    }
+    if (d == 64) return launch_simt_t<64>(q, k, v, p, num_units, stream);
+    if (d == 128) return launch_simt_t<128>(q, k, v, p, num_units, stream);
     return cudaErrorInvalidValue;
 }
 

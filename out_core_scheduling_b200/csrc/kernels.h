@@ -127,4 +127,12 @@ cudaError_t launch_partial_finish(int d, int elem_bytes, const float *o_sum, con
                                   const float *lse_max, void *out, float *lse, int64_t N, int H,
                                   cudaStream_t stream);
 
+// Owner exchange of a sharded forward (partial.cu): merge of the partials a
+// rank received for its rows [row_lo, row_hi) into out [rows][H][d] (plan
+// dtype) and lse [H][rows_max]; per owned block ib: nsrc[ib] partials at
+// receive offsets offs[ib * max_src + j] (floats).
+cudaError_t launch_shard_merge(int d, int elem_bytes, const float *recv, const int32_t *nsrc, const int64_t *offs,
+                               int max_src, int64_t block, int64_t N, int H, int64_t own_first, int64_t row_lo,
+                               int64_t row_hi, int64_t rows_max, void *out, float *lse, cudaStream_t stream);
+
 }  // namespace cqsa

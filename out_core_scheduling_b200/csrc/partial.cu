@@ -156,4 +156,81 @@ cudaError_t launch_partial_finish(int d, int elem_bytes, const float *o_sum, con
     return cudaGetLastError();
 }
 
+// Owner exchange: the log-sum-exp merge of the partials a rank received
+// for the rows it owns.  One warp per (row, head); lane j reads the lse of
+// partial j, lanes then cover the d features (float4 or float2).
+// The receive buffer holds, per partial of block b (offset off): o rows
+// [n_b][H][D], then lse [H][n_b].
+template <int D, typename TO>
+__global__ void __launch_bounds__(kThreads)
+    shard_merge_kernel(const float *__restrict__ recv, const int32_t *__restrict__ nsrc,
+                       const int64_t *__restrict__ offs, int max_src, int64_t block, int64_t N, int H,
+                       int64_t own_first, int64_t row_lo, int64_t row_hi, int64_t rows_max, TO *__restrict__ out,
+                       float *__restrict__ lse_out) {
+    constexpr int V = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t total = (row_hi - row_lo) * H;
+    for (int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < total; w += warps) {
+        const int64_t r = row_lo + w / H;
+        const int h = (int)(w % H);
+        const int64_t b = r / block, rl = r - b * block;
+        const int64_t nb = (N - b * block) < block ? (N - b * block) : block;
+        const int64_t ib = b - own_first;
+        const int n = nsrc[ib];
+        const int64_t *off = offs + ib * max_src;
+        const float lj = lane < n ? recv[off[lane] + nb * H * D + (int64_t)h * nb + rl] : -INFINITY;
+        float M = lj;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float wj = (lane < n && lj != -INFINITY) ? __expf(lj - M) : 0.f;
+        float W = wj;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = 0.f;
+        for (int j = 0; j < n; ++j) {
+            const float wb = __shfl_sync(0xffffffffu, wj, j);
+            if (wb == 0.f) continue;
+            const float *src = recv + off[j] + (rl * H + h) * D + lane * V;
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[i] = fmaf(wb, src[i], acc[i]);
+        }
+        const float inv = W > 0.f ? 1.f / W : 0.f;
+        TO *dst = out + ((r - row_lo) * H + h) * D + lane * V;
+#pragma unroll
+        for (int i = 0; i < V; ++i) store_out(dst + i, acc[i] * inv);
+        if (lane == 0) lse_out[(int64_t)h * rows_max + (r - row_lo)] = W > 0.f ? M + __logf(W) : -INFINITY;
+    }
+}
+
+template <int D, typename TO>
+static cudaError_t shard_merge_t(const float *recv, const int32_t *nsrc, const int64_t *offs, int max_src,
+                                 int64_t block, int64_t N, int H, int64_t own_first, int64_t row_lo, int64_t row_hi,
+                                 int64_t rows_max, void *out, float *lse, cudaStream_t st) {
+    const int64_t warps = (row_hi - row_lo) * H;
+    if (warps <= 0) return cudaSuccess;
+    shard_merge_kernel<D, TO><<<grid_for(warps, kThreads / 32), kThreads, 0, st>>>(
+        recv, nsrc, offs, max_src, block, N, H, own_first, row_lo, row_hi, rows_max, static_cast<TO *>(out), lse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shard_merge(int d, int elem_bytes, const float *recv, const int32_t *nsrc, const int64_t *offs,
+                               int max_src, int64_t block, int64_t N, int H, int64_t own_first, int64_t row_lo,
+                               int64_t row_hi, int64_t rows_max, void *out, float *lse, cudaStream_t stream) {
+    if (max_src < 1 || max_src > 32) return cudaErrorInvalidValue;
+#define SM_CALL(D_, T_) \
+    shard_merge_t<D_, T_>(recv, nsrc, offs, max_src, block, N, H, own_first, row_lo, row_hi, rows_max, out, lse, stream)
+    if (elem_bytes == 4) {
+        if (d == 64) return SM_CALL(64, float);
+        if (d == 128) return SM_CALL(128, float);
+    } else if (elem_bytes == 2) {
+        if (d == 64) return SM_CALL(64, __nv_bfloat16);
+        if (d == 128) return SM_CALL(128, __nv_bfloat16);
+    }
+#undef SM_CALL
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace cqsa

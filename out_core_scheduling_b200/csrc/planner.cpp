@@ -1079,4 +1079,56 @@ void Planner::size_bwd() {
     }
 }
 
+ShardLayout Planner::shard_layout(int elem_bytes) const {
+    ShardLayout L;
+    L.G = std::max(1, spec.shard_count);
+    L.me = spec.shard_rank;
+    const int G = L.G;
+    const int64_t H = spec.H, d = spec.d;
+    L.owner.resize(num_blocks);
+    for (int64_t b = 0; b < num_blocks; ++b) L.owner[b] = (int32_t)(b * G / num_blocks);
+    L.row_lo.assign(G + 1, spec.N);
+    for (int64_t b = num_blocks - 1; b >= 0; --b) L.row_lo[L.owner[b]] = std::min<int64_t>(b * block, spec.N);
+    for (int k = G - 1; k >= 0; --k) L.row_lo[k] = std::min(L.row_lo[k], L.row_lo[k + 1]);
+    for (int k = 0; k < G; ++k) L.rows_max = std::max(L.rows_max, L.row_lo[k + 1] - L.row_lo[k]);
+    // touched[r * num_blocks + b]: rank r has an entry for query block b.
+    std::vector<char> touched((size_t)G * num_blocks, 0);
+    for (size_t i = 0; i < entries.size(); ++i) touched[(size_t)entry_rank[i] * num_blocks + entries[i].qb] = 1;
+    // o rows, then lse padded to four floats: every piece starts 16-byte aligned.
+    auto piece = [&](int64_t b) { return block_rows(b) * H * d + ((block_rows(b) * H + 3) & ~int64_t(3)); };
+    L.send_counts.assign(G, 0);
+    L.recv_counts.assign(G, 0);
+    int64_t off = 0;
+    for (int k = 0; k < G; ++k)
+        for (int64_t b = 0; b < num_blocks; ++b)
+            if (L.owner[b] == k && touched[(size_t)L.me * num_blocks + b] && block_rows(b) > 0) {
+                L.send.push_back(ShardPiece{b, off});
+                off += piece(b);
+                L.send_counts[k] += piece(b);
+            }
+    L.own_first = num_blocks;
+    for (int64_t b = 0; b < num_blocks; ++b)
+        if (L.owner[b] == L.me) {
+            L.own_first = std::min(L.own_first, b);
+            ++L.own_count;
+        }
+    if (L.own_count == 0) L.own_first = 0;
+    L.own_offsets.assign(L.own_count, {});
+    off = 0;
+    for (int r = 0; r < G; ++r)
+        for (int64_t i = 0; i < L.own_count; ++i) {
+            const int64_t b = L.own_first + i;
+            if (touched[(size_t)r * num_blocks + b] && block_rows(b) > 0) {
+                L.own_offsets[i].push_back(off);
+                off += piece(b);
+                L.recv_counts[r] += piece(b);
+            }
+        }
+    auto up16 = [](size_t x) { return (x + 15) & ~size_t(15); };
+    L.out_bytes = up16((size_t)L.rows_max * H * d * elem_bytes);
+    L.chunk_bytes = L.out_bytes + up16((size_t)H * L.rows_max * sizeof(float));
+    if (L.chunk_bytes == 0) L.chunk_bytes = 16;
+    return L;
+}
+
 }  // namespace cqsa

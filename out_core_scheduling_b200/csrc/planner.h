@@ -126,6 +126,31 @@ struct BwdSizing {
     size_t spill_host = 0;  // pinned host bytes for written-back sums (0: none needed)
 };
 
+// Exchange of a sharded forward to the query blocks' owners.  Query block b
+// belongs to rank floor(b * G / num_blocks), so each rank owns a contiguous
+// range of rows.  A rank sends, to each owner in rank order, the partials
+// (o rows [n_b][H][d] fp32, then lse [H][n_b] fp32 padded to a multiple of
+// four floats) of the owner's blocks it
+// has an entry for, in increasing block order; the owner merges the
+// partials it receives (sources in rank order) and the ranks all-gather the
+// merged rows.
+struct ShardPiece {
+    int64_t block;
+    int64_t offset;  // floats into the send (or receive) buffer
+};
+
+struct ShardLayout {
+    int G = 1, me = 0;
+    std::vector<int32_t> owner;                 // per block
+    std::vector<int64_t> row_lo;                // G + 1: rows [row_lo[k], row_lo[k + 1]) belong to rank k
+    int64_t rows_max = 0;                       // most rows a rank owns
+    std::vector<int64_t> send_counts, recv_counts;  // floats to / from each rank
+    std::vector<ShardPiece> send;               // this rank's pieces, in send order
+    int64_t own_first = 0, own_count = 0;       // this rank's blocks [own_first, own_first + own_count)
+    std::vector<std::vector<int64_t>> own_offsets;  // per owned block: its partials' receive offsets
+    size_t out_bytes = 0, chunk_bytes = 0;      // gathered chunk: out rows, then lse [H][rows_max]
+};
+
 struct Sizing {
     int head_group = 0;
     size_t host_arena = 0;
@@ -197,6 +222,9 @@ public:
                                     int64_t *max_kv_slots) const;
     // Entries of this rank (all entries when the plan is not sharded).
     std::vector<char> shard_use() const;
+    // Owner exchange of this rank (see ShardLayout); elem_bytes of the
+    // gathered output rows.
+    ShardLayout shard_layout(int elem_bytes) const;
     // Work list of leaf t reading Q, K, V from the block pools of `pool`.
     WorkList leaf_worklist(int64_t t, const PoolPlan &pool, int rows_per_unit, int bn, int heads) const;
     // Merge segments of leaf t in host mode (one per query block with an

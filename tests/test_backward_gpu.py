@@ -100,7 +100,9 @@ def test_backward_gradient_identities_full_size():
         assert torch.isfinite(dq.float()).all()
 
 
-def test_backward_rejects_host_mode():
+def test_backward_host_mode_rejects_device_pointers():
+    """Host mode streams from page-locked host memory; device tensors are
+    refused (the streamed backward itself: test_backward_streamed_gpu.py)."""
     N, H, d = 7 * 64, 1, 64
     q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=0, device=DEV)
     plan = cqsa.cqsa_plan(N, H, d, 3)
@@ -108,7 +110,7 @@ def test_backward_rejects_host_mode():
     g = [torch.empty_like(q) for _ in range(3)]
     with pytest.raises(cqsa.CqsaError) as ei:
         cqsa.cqsa_backward(plan, q, k, v, out, lse, q, *g, host_or_device=cqsa.CQSA_HOST)
-    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+    assert ei.value.status == cqsa.CQSA_ERR_NOT_PINNED
 
 
 @pytest.mark.parametrize("merge", [cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED], ids=["slots", "fused"])

@@ -149,8 +149,8 @@ def test_streamed_backward_rejects_pageable_and_grouped_query():
     kv = torch.zeros(N, 2, d, dtype=torch.bfloat16).pin_memory()
     l4 = torch.zeros(4, N).pin_memory()
     with pytest.raises(cqsa.CqsaError) as ei:
-        cqsa.cqsa_backward(gplan, q, kv, kv, q, l4, q, q.clone(), kv.clone(), kv.clone(),
-                           host_or_device=cqsa.CQSA_HOST)
+        cqsa.cqsa_backward(gplan, q, kv, kv, q, l4, q, q.clone().pin_memory(), kv.clone().pin_memory(),
+                           kv.clone().pin_memory(), host_or_device=cqsa.CQSA_HOST)
     assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
 
 
