@@ -204,7 +204,8 @@ def run_sharded(args, W, D=None, workload=None):
     """--shard: ONE problem of the workload split over the ranks (strong
     scaling): every rank plans with shard_rank = its rank, computes its
     (task, query block) entries with cqsa_forward_partial, and the ranks
-    exchange their log-sum-exp partials over NCCL
+    exchange their log-sum-exp partials over NCCL: an all-to-all to each
+    query block's owner, the owner's merge, an all-gather of the merged rows
     (out_core_scheduling_b200.sharded).  Launched without torchrun it runs
     on a one-process NCCL group.  Device workloads only.
 
@@ -279,7 +280,9 @@ def run_sharded(args, W, D=None, workload=None):
     ms = D.max(ev0.elapsed_time(ev1), torch_dev)
     value = flops_step * args.steps / (ms * 1e-3) / 1e12
     infos = [p.info() for p in plans]
-    exch = sum(N * H * (d + 2) * 4 for _ in plans)
+    from out_core_scheduling_b200.sharded import exchange_bytes
+    exch = sum(exchange_bytes(p) for p in plans)
+    exch_ar = sum(exchange_bytes(p, "allreduce") for p in plans)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
@@ -289,11 +292,14 @@ def run_sharded(args, W, D=None, workload=None):
                    "l2": "inputs larger than L2; no flush"},
         "shard": {"rank0_entries": [i["shard_entries"] for i in infos],
                   "rank0_pair_share": [i["shard_pairs"] / i["total_pairs"] for i in infos],
+                  "exchange": "owners: all-to-all of partials to each query block's owner, owner-side "
+                              "log-sum-exp merge, all-gather of the merged rows",
                   "exchange_bytes_per_rank_per_step": exch,
+                  "exchange_bytes_two_all_reduces": exch_ar,
                   "collectives_per_step": 2 * len(plans)},
         "clocks": clocks,
-        # attention (none on a rank without entries) + partial init, rescale and finish
-        "gpu_launches": sum(s["attn_launches"] for s in stats) + 3 * len(plans) * args.steps,
+        # attention (none on a rank without entries) + partial init + owner merge
+        "gpu_launches": sum(s["attn_launches"] for s in stats) + 2 * len(plans) * args.steps,
     }
     for p in plans:
         p.destroy()

@@ -287,6 +287,52 @@ cqsa_status_t cqsa_partial_rescale(cqsa_plan_t *plan, float *o_part, const float
 cqsa_status_t cqsa_partial_finish(cqsa_plan_t *plan, const float *o_sum, const float *w_sum,
                                   const float *lse_max, void *out, float *lse, void *stream);
 
+/*
+ * Owner exchange (the alternative to steps 2-5 above, and what the Python
+ * binding uses by default).  Query block b belongs to rank
+ * floor(b * G / num_blocks), so rank k owns the contiguous rows
+ * [row_lo[k], row_lo[k + 1]).  Per sequence:
+ *   2'. cqsa_shard_pack: for each rank k in order, for each block b that k
+ *       owns and this rank has an entry for, in increasing b: o_part rows of
+ *       b ([n_b][H][d] fp32) then lse_part of b ([H][n_b] fp32, padded to a
+ *       multiple of four floats) into `send`.
+ *   3'. all-to-all (caller): send_counts[k] floats to rank k; the received
+ *       pieces concatenated in source-rank order (recv_counts[r] from r).
+ *   4'. cqsa_shard_merge: for each row this rank owns, the log-sum-exp merge
+ *       of its received partials ([A] recomposition) into `chunk`: out rows
+ *       [rows_max][H][d] in the plan dtype, then lse [H][rows_max] fp32,
+ *       each part padded to 16 bytes (chunk_bytes in all).
+ *   5'. all-gather (caller): the G chunks in rank order.
+ *   6'. cqsa_shard_unpack: out [N][H][d] and lse [H][N] from the chunks.
+ * A block has entries on at most l ranks, so a rank sends about (l - 1) / G
+ * of the partial rows rather than all of them twice; the all-gather moves the
+ * output once, in the plan dtype.  All four calls take one sequence; device
+ * pointers on the current device; asynchronous on stream.
+ */
+
+/* cqsa_shard_layout -- host only: send_counts[G], recv_counts[G] (fp32
+ * values to and from each rank), row_lo[G + 1], *rows_max and *chunk_bytes
+ * of this rank's plan.  Errors: INVALID_ARG. */
+cqsa_status_t cqsa_shard_layout(cqsa_plan_t *plan, int64_t *send_counts, int64_t *recv_counts, int64_t *row_lo,
+                                int64_t *rows_max, size_t *chunk_bytes);
+
+/* cqsa_shard_pack -- step 2': o_part fp32 [N, H, d], lse_part fp32 [H, N]
+ * (cqsa_forward_partial's outputs for one sequence) into send (fp32, the sum
+ * of send_counts).  Errors: INVALID_ARG, CUDA. */
+cqsa_status_t cqsa_shard_pack(cqsa_plan_t *plan, const float *o_part, const float *lse_part, float *send,
+                              void *stream);
+
+/* cqsa_shard_merge -- step 4': recv (fp32, the sum of recv_counts, as the
+ * all-to-all left it) into chunk (chunk_bytes).  The first call allocates a
+ * small table of the owned blocks' partial offsets.  Errors: INVALID_ARG,
+ * UNSUPPORTED (a block with partials from more than 32 ranks), CUDA. */
+cqsa_status_t cqsa_shard_merge(cqsa_plan_t *plan, const float *recv, void *chunk, void *stream);
+
+/* cqsa_shard_unpack -- step 6': the G chunks (G * chunk_bytes, rank order)
+ * into out [N, H, d] (plan dtype) and lse [H, N] fp32.  Errors:
+ * INVALID_ARG, CUDA. */
+cqsa_status_t cqsa_shard_unpack(cqsa_plan_t *plan, const void *chunks, void *out, float *lse, void *stream);
+
 /* cqsa_backward_partial -- this rank's part of the backward of a sharded
  * plan (any plan: with one rank it is the whole backward).  Every allowed
  * pair's gradient terms depend only on the pair and the row statistics

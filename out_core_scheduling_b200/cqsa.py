@@ -43,7 +43,7 @@ EXPORTS = (
     "cqsa_plan_profile", "cqsa_plan_kernel_stats", "cqsa_forward_noalloc", "cqsa_plan_destroy",
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
     "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast", "cqsa_plan_cache_task",
-    "cqsa_plan_bwd_cache_task",
+    "cqsa_plan_bwd_cache_task", "cqsa_shard_layout", "cqsa_shard_pack", "cqsa_shard_merge", "cqsa_shard_unpack",
 )
 
 
@@ -143,6 +143,12 @@ def load_library():
                                           ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
                                           ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
                                           ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
+        "cqsa_shard_layout": (st, [P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                   ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                   ctypes.POINTER(ctypes.c_size_t)]),
+        "cqsa_shard_pack": (st, [P, P, P, P, P]),
+        "cqsa_shard_merge": (st, [P, P, P, P]),
+        "cqsa_shard_unpack": (st, [P, P, P, P, P]),
         "cqsa_difference_set": (st, [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
         "cqsa_plan_debug": (st, [P, ctypes.c_uint64, ctypes.c_int]),
         "cqsa_plan_profile": (st, [P, ctypes.c_int]),
@@ -418,6 +424,64 @@ def cqsa_partial_finish(plan: Plan, o_sum, w_sum, lse_max, out, lse, stream=None
     _check(load_library().cqsa_partial_finish(plan.handle, o_sum.data_ptr(), w_sum.data_ptr(),
                                               lse_max.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def shard_layout(plan: Plan) -> dict:
+    """The owner exchange of a sharded plan (host only): floats this rank
+    sends to and receives from each rank, each rank's first row (and N),
+    the most rows a rank owns, and the bytes of one gathered chunk."""
+    info = plan.info()
+    G = info["shard_count"]
+    sc, rc = (ctypes.c_int64 * G)(), (ctypes.c_int64 * G)()
+    lo = (ctypes.c_int64 * (G + 1))()
+    rmax, cb = ctypes.c_int64(), ctypes.c_size_t()
+    _check(load_library().cqsa_shard_layout(plan.handle, sc, rc, lo, ctypes.byref(rmax), ctypes.byref(cb)))
+    return {"send_counts": list(sc), "recv_counts": list(rc), "row_lo": list(lo), "rows_max": rmax.value,
+            "chunk_bytes": cb.value}
+
+
+def cqsa_shard_pack(plan: Plan, o_part, lse_part, send, stream=None):
+    """This rank's partials of the blocks each owner receives, into ``send``
+    (fp32, sum of shard_layout()["send_counts"] values)."""
+    info = plan.info()
+    N, H, d = info["N"], info["H"], info["d"]
+    for name, t, want in (("o_part", o_part, (N, H, d)), ("lse_part", lse_part, (H, N)), ("send", send, None)):
+        if t.dtype != _float32() or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 tensor")
+        if want is not None and tuple(t.shape) != want:
+            raise ValueError(f"{name} must be {want} (one sequence)")
+    _check(load_library().cqsa_shard_pack(plan.handle, o_part.data_ptr(), lse_part.data_ptr(), send.data_ptr(),
+                                          ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_shard_merge(plan: Plan, recv, chunk, stream=None):
+    """The rows this rank owns, merged from the partials in ``recv`` (as the
+    all-to-all delivered them), into ``chunk`` (uint8, chunk_bytes)."""
+    if recv.dtype != _float32() or not recv.is_contiguous() or not chunk.is_contiguous():
+        raise ValueError("recv must be contiguous float32 and chunk contiguous")
+    _check(load_library().cqsa_shard_merge(plan.handle, recv.data_ptr(), chunk.data_ptr(),
+                                           ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def cqsa_shard_unpack(plan: Plan, chunks, out, lse, stream=None):
+    """out [N, H, d] and lse [H, N] (one sequence) from the all-gathered chunks."""
+    import torch
+    info = plan.info()
+    N, H, d = info["N"], info["H"], info["d"]
+    want = torch.bfloat16 if info["dtype"] == CQSA_BF16 else torch.float32
+    if tuple(out.shape) != (N, H, d) or out.dtype != want or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {want} tensor of shape {(N, H, d)}")
+    if tuple(lse.shape) != (H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError(f"lse must be a contiguous float32 tensor of shape {(H, N)}")
+    if not chunks.is_contiguous():
+        raise ValueError("chunks must be contiguous")
+    _check(load_library().cqsa_shard_unpack(plan.handle, chunks.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                            ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def _float32():
+    import torch
+    return torch.float32
 
 
 def cqsa_backward_partial(plan: Plan, q, k, v, out, lse, dout, dq_part, dk_part, dv_part, stream=None):

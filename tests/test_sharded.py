@@ -164,6 +164,171 @@ HostOps.backward_partial = staticmethod(_host_backward_partial)
 HostOps.partial_cast = staticmethod(lambda plan, src, dst: dst.copy_(src.to(dst.dtype)))
 
 
+# ------------------------------------------------------------ owner exchange
+def host_layout(plan):
+    """The owner exchange as the header describes it, derived here from the
+    plan's entries: owner(b) = floor(b G / num_blocks); a rank sends, owner
+    by owner, the blocks it has an entry for in increasing order, each piece
+    o rows [n_b][H][d] then lse [H][n_b] padded to four floats; the owner's
+    receive buffer holds the pieces by source rank, blocks in order."""
+    info = plan.info()
+    G, me, nb_all, blk, N = (info["shard_count"], info["shard_rank"], info["num_blocks"], info["block_tokens"],
+                             info["N"])
+    H, d = info["H"], info["d"]
+    owner = [b * G // nb_all for b in range(nb_all)]
+    rows = [max(0, min((b + 1) * blk, N) - b * blk) for b in range(nb_all)]
+    touched = set()
+    for i in range(info["num_entries"]):
+        e = plan.entry(i)
+        touched.add((e["shard"], e["q_block"]))
+    piece = [rows[b] * H * d + (rows[b] * H + 3) // 4 * 4 for b in range(nb_all)]
+    send, send_counts, off = [], [0] * G, 0
+    for k in range(G):
+        for b in range(nb_all):
+            if owner[b] == k and (me, b) in touched and rows[b]:
+                send.append((b, off))
+                off += piece[b]
+                send_counts[k] += piece[b]
+    recv, recv_counts, off = {}, [0] * G, 0
+    for r in range(G):
+        for b in range(nb_all):
+            if owner[b] == me and (r, b) in touched and rows[b]:
+                recv.setdefault(b, []).append(off)
+                off += piece[b]
+                recv_counts[r] += piece[b]
+    row_lo = [N] * (G + 1)
+    for b in range(nb_all - 1, -1, -1):
+        row_lo[owner[b]] = min(b * blk, N)
+    for k in range(G - 1, -1, -1):
+        row_lo[k] = min(row_lo[k], row_lo[k + 1])
+    rows_max = max(row_lo[k + 1] - row_lo[k] for k in range(G))
+    return {"send": send, "recv": recv, "send_counts": send_counts, "recv_counts": recv_counts,
+            "row_lo": row_lo, "rows_max": rows_max, "rows": rows}
+
+
+def _host_shard_layout(plan):
+    lay = host_layout(plan)
+    lib = cqsa.shard_layout(plan)
+    for key in ("send_counts", "recv_counts", "row_lo", "rows_max"):
+        assert lay[key] == lib[key], (key, lay[key], lib[key])
+    # One chunk: out rows [rows_max][H][d] in the plan dtype, then lse
+    # [H][rows_max] fp32, each padded to 16 bytes.
+    info = plan.info()
+    assert lib["chunk_bytes"] == max(16, _up16(lay["rows_max"] * info["H"] * info["d"] * _elem(plan)) +
+                                     _up16(info["H"] * lay["rows_max"] * 4))
+    return lib
+
+
+def _up16(x):
+    return (x + 15) // 16 * 16
+
+
+def _elem(plan):
+    return 4 if plan.info()["dtype"] == cqsa.CQSA_FP32 else 2
+
+
+def _tdtype(plan):
+    import torch
+    return torch.float32 if plan.info()["dtype"] == cqsa.CQSA_FP32 else torch.bfloat16
+
+
+def _host_shard_pack(plan, o_part, lse_part, send):
+    info = plan.info()
+    H, d, blk = info["H"], info["d"], info["block_tokens"]
+    lay = host_layout(plan)
+    for b, off in lay["send"]:
+        n = lay["rows"][b]
+        send[off:off + n * H * d] = o_part[b * blk:b * blk + n].reshape(-1)
+        send[off + n * H * d:off + n * H * d + H * n] = lse_part[:, b * blk:b * blk + n].reshape(-1)
+
+
+def _host_shard_merge(plan, recv, chunk):
+    import torch
+    info = plan.info()
+    H, d, blk, me = info["H"], info["d"], info["block_tokens"], info["shard_rank"]
+    lay = host_layout(plan)
+    R, lo = lay["rows_max"], lay["row_lo"][me]
+    out = np.zeros((max(R, 1), H, d))
+    lse = np.full((H, max(R, 1)), -np.inf)
+    rv = recv.double().numpy()
+    for b, offs in lay["recv"].items():
+        n = lay["rows"][b]
+        o = np.stack([rv[x:x + n * H * d].reshape(n, H, d) for x in offs])               # [S, n, H, d]
+        l = np.stack([rv[x + n * H * d:x + n * H * d + H * n].reshape(H, n) for x in offs])  # [S, H, n]
+        M = l.max(0)
+        w = np.where(np.isinf(l), 0.0, np.exp(l - M))
+        W = w.sum(0)
+        r0 = b * blk - lo
+        out[r0:r0 + n] = np.einsum("shn,snhd->nhd", w, o) / W.T[..., None]
+        lse[:, r0:r0 + n] = M + np.log(W)
+    ob = torch.from_numpy(out[:R]).to(_tdtype(plan)).reshape(-1).view(torch.uint8)
+    lb = torch.from_numpy(lse[:, :R].astype(np.float32)).reshape(-1).view(torch.uint8)
+    chunk.zero_()
+    chunk[:ob.numel()] = ob
+    ofs = _up16(R * H * d * _elem(plan))
+    chunk[ofs:ofs + lb.numel()] = lb
+
+
+def _host_shard_unpack(plan, chunks, out, lse):
+    import torch
+    info = plan.info()
+    G, H, d = info["shard_count"], info["H"], info["d"]
+    lay = host_layout(plan)
+    R = lay["rows_max"]
+    cb = cqsa.shard_layout(plan)["chunk_bytes"]
+    e = _elem(plan)
+    for k in range(G):
+        lo, hi = lay["row_lo"][k], lay["row_lo"][k + 1]
+        if hi <= lo:
+            continue
+        c = chunks[k * cb:(k + 1) * cb]
+        o = c[:R * H * d * e].view(_tdtype(plan)).reshape(R, H, d)
+        ofs = _up16(R * H * d * e)
+        l = c[ofs:ofs + H * R * 4].view(torch.float32).reshape(H, R)
+        out[lo:hi] = o[:hi - lo].to(out.dtype)
+        lse[:, lo:hi] = l[:, :hi - lo]
+
+
+HostOps.shard_layout = staticmethod(_host_shard_layout)
+HostOps.shard_pack = staticmethod(_host_shard_pack)
+HostOps.shard_merge = staticmethod(_host_shard_merge)
+HostOps.shard_unpack = staticmethod(_host_shard_unpack)
+
+
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: f"n{c[0]}-l{c[3]}-{'c' if c[4] else 'nc'}")
+def test_owner_exchange_layout(cfg, G):
+    """The library's layout (cqsa_shard_layout) equals the one derived from
+    the header's rules; every block's partials reach its owner; the pieces
+    the ranks send to an owner are exactly what it expects."""
+    N, H, d, ls, causal = cfg
+    plans = [cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cqsa.CQSA_FP32, shard_rank=r, shard_count=G)
+             for r in range(G)]
+    lays = [host_layout(p) for p in plans]
+    for p, lay in zip(plans, lays):
+        lib = cqsa.shard_layout(p)
+        for key in ("send_counts", "recv_counts", "row_lo", "rows_max"):
+            assert lay[key] == lib[key], key
+    for k in range(G):
+        for r in range(G):
+            assert lays[r]["send_counts"][k] == lays[k]["recv_counts"][r]
+    info = plans[0].info()
+    for b in range(info["num_blocks"]):
+        if lays[0]["rows"][b]:
+            k = b * G // info["num_blocks"]
+            assert b in lays[k]["recv"], f"block {b} reaches no owner"
+
+
+def test_owner_exchange_moves_less_than_the_all_reduces():
+    """l=4, 13 blocks of 4096, H=8, d=128 over 8 ranks: bytes a rank sends
+    per forward in the owner exchange against the two all-reduces."""
+    from out_core_scheduling_b200.sharded import exchange_bytes
+    G = 8
+    own = [exchange_bytes(cqsa.cqsa_plan_ex(53248, 8, 128, [4], shard_rank=r, shard_count=G)) for r in range(G)]
+    ar = exchange_bytes(cqsa.cqsa_plan_ex(53248, 8, 128, [4], shard_rank=0, shard_count=G), "allreduce")
+    assert max(own) < 0.6 * ar, (own, ar)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -189,13 +354,16 @@ def _rank_main(rank, world, port, cfg, q):
     try:
         N, H, d, ls, causal = cfg
         qt, kt, vt = make_qkv(N, H, d, dtype=torch.float32, seed=11)
-        plan = lib.cqsa_plan_ex(N, H, d, ls, causal=causal, shard_rank=rank, shard_count=world)
-        out = torch.empty(N, H, d)
-        lse = torch.empty(H, N)
-        forward_sharded(plan, qt, kt, vt, out, lse, ops=HostOps)
+        plan = lib.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=lib.CQSA_FP32, shard_rank=rank,
+                                shard_count=world)
         ref_o, ref_l = oracle.attention_rows(qt, kt, vt, causal=causal)
-        e_o = float(np.abs(out.double().numpy() - ref_o).max())
-        e_l = float(np.abs(lse.double().numpy().T - ref_l).max())
+        e_o = e_l = 0.0
+        for exchange in ("owners", "allreduce"):
+            out = torch.empty(N, H, d)
+            lse = torch.empty(H, N)
+            forward_sharded(plan, qt, kt, vt, out, lse, ops=HostOps, exchange=exchange)
+            e_o = max(e_o, float(np.abs(out.double().numpy() - ref_o).max()))
+            e_l = max(e_l, float(np.abs(lse.double().numpy().T - ref_l).max()))
         # The backward from the exchanged out and lse.
         dout = make_qkv(N, H, d, dtype=torch.float32, seed=12)[0]
         dq, dk, dv = (torch.empty(N, H, d) for _ in range(3))
@@ -212,8 +380,10 @@ def _rank_main(rank, world, port, cfg, q):
 @pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("cfg", [CONFIGS[1], CONFIGS[3], CONFIGS[4]], ids=["l3-c", "l43-nc", "l43-ragged-c"])
 def test_forward_sharded_gloo(cfg, world):
-    """Every rank ends with the full attention (fp32 buffers: 1e-5) and,
-    after backward_sharded, the full gradients (1e-4 of the largest)."""
+    """Every rank ends with the full attention after either exchange (the
+    owners' all-to-all and all-gather, or the two all-reduces; fp32
+    buffers: 1e-5) and, after backward_sharded, the full gradients (1e-4 of
+    the largest)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -266,7 +436,7 @@ def _rank_fail_main(rank, world, port, q):
     try:
         N, H, d = 7 * 64, 1, 64
         qt, kt, vt = make_qkv(N, H, d, dtype=torch.float32, seed=13)
-        plan = lib.cqsa_plan_ex(N, H, d, [3], shard_rank=rank, shard_count=world)
+        plan = lib.cqsa_plan_ex(N, H, d, [3], dtype=lib.CQSA_FP32, shard_rank=rank, shard_count=world)
         if rank == 1:
             raise RuntimeError("planted failure of rank 1 before the exchange")
         forward_sharded(plan, qt, kt, vt, torch.empty(N, H, d), torch.empty(H, N), ops=HostOps)

@@ -83,6 +83,65 @@ def test_sharded_forward_matches_oracle(case):
     check(out, lse, q, k, v, np.arange(N) if N <= 3000 else sample_rows(N, 512), causal)
 
 
+def _owners(N, H, d, ls, causal, dtype, G, seed=0):
+    """The owner exchange with G emulated ranks: each rank's partial forward
+    and cqsa_shard_pack; the all-to-all stood in for by slicing the send
+    buffers by the exported counts; each owner's cqsa_shard_merge; the
+    all-gather by concatenating the chunks; cqsa_shard_unpack on every rank,
+    which must all give the same result."""
+    cdt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    q, k, v = make_qkv(N, H, d, dtype=dtype, seed=seed, device=DEV)
+    plans = [cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=cdt, shard_rank=r, shard_count=G)
+             for r in range(G)]
+    lays = [cqsa.shard_layout(p) for p in plans]
+    sends = []
+    for p, lay in zip(plans, lays):
+        o = torch.empty(N, H, d, device=DEV)
+        l = torch.empty(H, N, device=DEV)
+        cqsa.cqsa_forward_partial(p, q, k, v, o, l)
+        send = torch.full((max(1, sum(lay["send_counts"])),), float("nan"), device=DEV)
+        cqsa.cqsa_shard_pack(p, o, l, send)
+        sends.append(send)
+    chunks = []
+    for kk, (p, lay) in enumerate(zip(plans, lays)):
+        parts = []
+        for r in range(G):
+            c = lays[r]["send_counts"]
+            off = sum(c[:kk])
+            parts.append(sends[r][off:off + c[kk]])
+            assert c[kk] == lay["recv_counts"][r]
+        recv = torch.cat(parts) if sum(lay["recv_counts"]) else torch.zeros(1, device=DEV)
+        chunk = torch.zeros(lay["chunk_bytes"], dtype=torch.uint8, device=DEV)
+        cqsa.cqsa_shard_merge(p, recv, chunk)
+        chunks.append(chunk)
+    gathered = torch.cat(chunks)
+    results = []
+    for p in plans:
+        out = torch.full((N, H, d), float("nan"), device=DEV, dtype=dtype)
+        lse = torch.full((H, N), float("nan"), device=DEV)
+        cqsa.cqsa_shard_unpack(p, gathered, out, lse)
+        p.sync()
+        results.append((out, lse))
+    for out, lse in results[1:]:
+        assert torch.equal(out, results[0][0]) and torch.equal(lse, results[0][1])
+    return q, k, v, results[0][0], results[0][1]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"n{c[0]}-d{c[2]}-l{c[3]}-{'c' if c[4] else 'nc'}-"
+                                                      f"{str(c[5])[6:]}-g{c[6]}")
+def test_owner_exchange_matches_oracle(case):
+    N, H, d, ls, causal, dtype, G = case
+    q, k, v, out, lse = _owners(N, H, d, ls, causal, dtype, G, seed=50)
+    check(out, lse, q, k, v, np.arange(N) if N <= 3000 else sample_rows(N, 512), causal)
+
+
+def test_owner_exchange_more_ranks_than_blocks():
+    """G above the block count: some ranks own no rows (empty chunks)."""
+    N, H, d = 7 * 64, 1, 64
+    q, k, v, out, lse = _owners(N, H, d, [3], False, torch.bfloat16, 9, seed=51)
+    check(out, lse, q, k, v, np.arange(N), False)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_sharded_grouped_query_and_batch(causal):
     N, H, Hkv, d, B, G = 7 * 128, 4, 2, 128, 2, 3
