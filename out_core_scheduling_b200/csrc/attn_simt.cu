@@ -362,13 +362,15 @@ __global__ void __launch_bounds__(simt::THREADS)
 }
 
 // Cluster size for a launch of num_units units: the smallest S in {1, 2, 4}
-// whose num_units * S CTAs fill every SM with as many CTAs as can be
-// resident at once (fewer units than that leave SMs idle, and one CTA per
-// SM leaves the FFMA pipe waiting on shared-memory latency).
+// whose num_units * S CTAs fill every SM twice over with as many CTAs as
+// can be resident at once: fewer units than that leave SMs idle or give a
+// long last wave.  Measured on the l=3, N=3584, d=64 workload (168 units,
+// two resident CTAs per SM): S = 2 19.4 TFLOP/s, S = 4 21.5, S = 8 19.2
+// (shorter CTAs pay their Q load and the cluster combine more often).
 static int simt_split(int num_units, int resident) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t target = (int64_t)sms * (resident > 0 ? resident : 1);
+    const int64_t target = 2 * (int64_t)sms * (resident > 0 ? resident : 1);
     int S = 1;
     while (S < 4 && (int64_t)num_units * S < target) S *= 2;
     return S;
