@@ -63,6 +63,17 @@ def useful_flops(N: int, H: int, d: int, causal: bool) -> float:
     return 4.0 * N * N * H * d * (0.5 if causal else 1.0)
 
 
+def merge_bytes(plan, info, ebytes: int) -> float:
+    """HBM bytes the slots merge must move for one forward: every partial of
+    every query block read once (O_j fp32 and lse_j), out and lse written."""
+    N, H, d, blk = info["N"], info["H"], info["d"], info["block_tokens"]
+    parts = 0
+    for i in range(info["num_entries"]):
+        b = plan.entry(i)["q_block"]
+        parts += max(0, min((b + 1) * blk, N) - b * blk)
+    return float(parts) * H * (4 * d + 4) + float(N) * H * (ebytes * d + 4)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -492,13 +503,13 @@ def measure(args, W, D, workload, steps, warmup, extras):
     merge_launches = sum(s["merge_launches"] for s in stats)
     if W["mode"] == "device" and merge_ms > 0:
         mb = 0.0
-        for info, s in zip(infos, stats):
-            S = info["max_slots"]
-            mb += N * H * (S * (4 * d + 4) + ebytes * d + 4) * s["merge_launches"]
+        for p, info, s in zip(plans, infos, stats):
+            mb += merge_bytes(p, info, ebytes) * s["merge_launches"]
         merge = {"bound": "hbm", "achieved": mb / (merge_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                  "unit": "GB/s", "frac": mb / (merge_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                  "bytes_per_launch": mb / max(1, merge_launches), "kernel": "merge_slots_kernel",
-                 "note": "upper bound: assumes every block holds max_slots partials"}
+                 "note": "algorithmic bytes: each query block's partials (4d+4 B per row and head each, "
+                         "as many as the block has entries) read once, the output and lse written once"}
 
     arena = sum(i["device_arena_bytes"] if W["mode"] == "device" else i["host_arena_bytes"] for i in infos)
     result = {
