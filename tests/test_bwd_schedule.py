@@ -139,7 +139,8 @@ CASES = [
     (13 * 128, 2, 64, [4], False, 1.0),
     (13 * 128, 2, 64, [4], True, 1.0),
     (21 * 64, 2, 64, [5], False, 1.0),
-    (91 * 32, 2, 64, [4, 3], True, None),
+    (49 * 32, 1, 64, [3, 3], True, None),        # two levels, 49 tasks
+    (49 * 32, 1, 64, [3, 3], False, 1.0),
 ]
 
 
