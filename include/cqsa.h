@@ -232,7 +232,10 @@ cqsa_status_t cqsa_forward(cqsa_plan_t *plan, const void *q, const void *k,
  *     allocates the backward's arena (bwd_host_arena_bytes); when the
  *     streamed forward's arena and this one would exceed the budget together,
  *     the other one is released first (and set up again by its next call).
- *     Grouped-query plans (H_kv < H) return UNSUPPORTED in this mode.
+ *     With grouped-query attention a head group holds whole key/value
+ *     groups, and the key-stationary gradients run one launch per query
+ *     head residue modulo the group size, so that the query heads of a
+ *     group add into their key/value head's sums one launch at a time.
  *   CQSA_MERGE_SLOTS plans write each (task, query block) dq partial and
  *     each (task, key block) dk / dv partial to slots of a backward arena
  *     (allocated on the first call) and sum them; CQSA_MERGE_FUSED plans

@@ -218,11 +218,13 @@ struct BwdHostState {
     int *err = nullptr;
     float *lse = nullptr, *delta = nullptr;   // [g][N] of the current head group
     char *stage_o[2] = {}, *stage_do[2] = {}; // O and dO rows of one block, two stages ([block][g][d])
-    char *pool[4] = {};                       // Q, K, V, dO block caches ([slots * block][g][d])
-    float *acc[3] = {};                       // dQ, dK, dV sums ([slots * block][g][d] fp32)
+    int gk = 0;                               // key/value heads of a head group (g / kv_group)
+    char *pool[4] = {};                       // Q, K, V, dO block caches ([slots * block][g or gk][d])
+    float *acc[3] = {};                       // dQ, dK, dV sums ([slots * block][g or gk][d] fp32)
     std::vector<DevWl> qwl, kvwl;             // per leaf task, cache coordinates
+    std::vector<std::vector<int>> kv_split;   // per leaf task: unit offsets of each query-head residue
     CUtensorMap mq, mk, mv, mdo;
-    float *spill = nullptr;                   // pinned host [3][N][g][d] fp32, when the plan writes back
+    float *spill = nullptr;                   // pinned host dQ [N][g][d], dK, dV [N][gk][d] fp32, when the plan writes back
     cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
     std::vector<cudaEvent_t> ev_slot_free;    // per slot: its write-back or gradient copy-out is done
     std::vector<cudaEvent_t> ev_spill;        // per block: its last write-back has landed in host memory
@@ -1025,9 +1027,6 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
     if (S.arena) return CQSA_OK;
     const Planner &pl = P->pl;
     const BwdSizing &z = pl.bwd_sizing;
-    if (pl.spec.kv_group() != 1)
-        return fail(CQSA_ERR_UNSUPPORTED, "the streamed backward takes as many key/value heads as query heads "
-                                          "(H_kv = %d, H = %d); use device mode", pl.spec.Hkv, pl.spec.H);
     if (z.head_group <= 0)
         return fail(CQSA_ERR_BUDGET, "no head group of the streamed backward fits the budget of %zu bytes "
                                      "(needs %lld block slots)", pl.spec.budget, (long long)pl.bwd_min_slots);
@@ -1039,11 +1038,13 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
         release_host_mode(P);
     }
     const int g = z.head_group;
+    const int kvg = pl.spec.kv_group(), gk = g / kvg;
     const BwdCachePlan &cp = pl.bwd_cache;
     const int64_t N = pl.spec.N;
     const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
     const size_t rows = (size_t)cp.slots * pl.block;
     const int tile = P->dtype == CQSA_BF16 ? 128 : 64;
+    const int heads[4] = {g, gk, gk, g};  // Q, K, V, dO
     // Same layout steps as Planner::bwd_arena_bytes.
     ArenaLayout a;
     const size_t o_err = a.take(256);
@@ -1051,8 +1052,8 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
     const size_t o_delta = a.take((size_t)g * N * sizeof(float));
     size_t o_st[4], o_pool[4], o_acc[3];
     for (int i = 0; i < 4; ++i) o_st[i] = a.take((size_t)pl.block * g * dd * e);
-    for (int i = 0; i < 4; ++i) o_pool[i] = a.take(rows * g * dd * e);
-    for (int i = 0; i < 3; ++i) o_acc[i] = a.take(rows * g * dd * sizeof(float));
+    for (int i = 0; i < 4; ++i) o_pool[i] = a.take(rows * heads[i] * dd * e);
+    for (int i = 0; i < 3; ++i) o_acc[i] = a.take(rows * heads[i] * dd * sizeof(float));
     const size_t T = pl.leaves.size();
     std::vector<WorkList> qw(T), kw(T);
     std::vector<size_t> o_qw(T), o_kw(T);
@@ -1070,6 +1071,7 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
     S.arena = arena;
     S.bytes = a.total;
     S.g = g;
+    S.gk = gk;
     // Zeroed once, so rows a partial tile reads past a short block are finite.
     CK(cudaMemset(arena, 0, a.total));
     S.err = reinterpret_cast<int *>(arena + o_err);
@@ -1083,7 +1085,11 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
     for (int i = 0; i < 3; ++i) S.acc[i] = reinterpret_cast<float *>(arena + o_acc[i]);
     S.qwl.resize(T);
     S.kvwl.resize(T);
+    S.kv_split.assign(T, std::vector<int>(kvg + 1, 0));
     for (size_t t = 0; t < T; ++t) {
+        // Units come ordered by query head modulo the group size.
+        for (const WlUnit &u : kw[t].units) ++S.kv_split[t][u.head % kvg + 1];
+        for (int j = 0; j < kvg; ++j) S.kv_split[t][j + 1] += S.kv_split[t][j];
         std::vector<char> b1 = pack_wl(qw[t]), b2 = pack_wl(kw[t]);
         if (!b1.empty()) CK(lib_upload(arena + o_qw[t], b1.data(), b1.size()));
         if (!b2.empty()) CK(lib_upload(arena + o_kw[t], b2.data(), b2.size()));
@@ -1094,7 +1100,7 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
         cqsa_status_t st;
         CUtensorMap *maps[4] = {&S.mq, &S.mk, &S.mv, &S.mdo};
         for (int i = 0; i < 4; ++i)
-            if ((st = make_map(maps[i], S.pool[i], (int64_t)rows, g, pl.spec.d)) != CQSA_OK) return st;
+            if ((st = make_map(maps[i], S.pool[i], (int64_t)rows, heads[i], pl.spec.d)) != CQSA_OK) return st;
     }
     if (z.spill_host) {
         void *h = nullptr;
@@ -1138,14 +1144,21 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
     const Planner &pl = P->pl;
     const BwdCachePlan &cp = pl.bwd_cache;
     const int64_t N = pl.spec.N, Bk = pl.block;
-    const int H = pl.spec.H, d = pl.spec.d, g = S.g;
+    const int H = pl.spec.H, Hkv = pl.spec.Hkv, d = pl.spec.d, g = S.g, gk = S.gk, kvg = pl.spec.kv_group();
     const size_t e = (size_t)P->elem;
-    const size_t full_row = (size_t)H * d * e, grp_row = (size_t)g * d * e, acc_row = (size_t)g * d * sizeof(float);
     const size_t slot_rows = (size_t)Bk;
+    // Per tensor: heads in the caller's rows and in a head group.  Q, K, V, dO
+    // (pools) and dQ, dK, dV (sums, gradients) follow Q, K, V's head counts.
+    const int full_h[4] = {H, Hkv, Hkv, H}, grp_h[4] = {g, gk, gk, g};
+    auto row_bytes = [&](int heads) { return (size_t)heads * d * e; };
+    auto acc_row = [&](int heads) { return (size_t)heads * d * sizeof(float); };
     const char *src[4] = {static_cast<const char *>(q), static_cast<const char *>(k), static_cast<const char *>(v),
                           static_cast<const char *>(dout)};
     char *dst[3] = {static_cast<char *>(dq), static_cast<char *>(dk), static_cast<char *>(dv)};
     const char *ho = static_cast<const char *>(out);
+    // Written-back sums on the host: dQ [N][g][d], then dK and dV [N][gk][d].
+    float *spill_of[3] = {S.spill, S.spill ? S.spill + (size_t)N * g * d : nullptr,
+                          S.spill ? S.spill + (size_t)N * (g + gk) * d : nullptr};
     CK(cudaEventRecord(S.ev_start, stream));
     cudaStream_t ss[3] = {S.s_in, S.s_comp, S.s_out};
     for (cudaStream_t x : ss) {
@@ -1160,8 +1173,8 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
     bp.delta = S.delta;
     bp.N = N;
     bp.H = g;
-    bp.Hkv = g;
-    bp.kv_group = 1;
+    bp.Hkv = gk;
+    bp.kv_group = kvg;
     bp.causal = pl.spec.causal;
     bp.scale = 1.0f / std::sqrt((float)d);
     bp.accum = 1;
@@ -1169,10 +1182,10 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
     bp.k = S.pool[1];
     bp.v = S.pool[2];
     bp.dout = S.pool[3];
-    const size_t cast_n = slot_rows * g * d;  // values per slot and tensor
     int64_t it = 0;
     for (int h0 = 0; h0 < H; h0 += g) {
         NvtxRange nvtx_group("cqsa streamed backward head group", h0);
+        const int hh[4] = {h0, h0 / kvg, h0 / kvg, h0};  // first head of the group per tensor
         // lse and D of this head group replace the previous group's once its
         // kernels are done.
         if (h0 > 0) CK(cudaStreamWaitEvent(S.s_in, S.ev_group, 0));
@@ -1185,9 +1198,10 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
             const int sg = ib & 1;
             if (ib >= 2) CK(cudaStreamWaitEvent(S.s_in, S.ev_stage_free[sg], 0));
             const size_t off = ((size_t)b * Bk * H + h0) * d * e;
-            CK(copy_rows(S.stage_o[sg], grp_row, ho + off, full_row, grp_row, nr, cudaMemcpyHostToDevice, S.s_in));
-            CK(copy_rows(S.stage_do[sg], grp_row, src[3] + off, full_row, grp_row, nr, cudaMemcpyHostToDevice,
-                         S.s_in));
+            CK(copy_rows(S.stage_o[sg], row_bytes(g), ho + off, row_bytes(H), row_bytes(g), nr,
+                         cudaMemcpyHostToDevice, S.s_in));
+            CK(copy_rows(S.stage_do[sg], row_bytes(g), src[3] + off, row_bytes(H), row_bytes(g), nr,
+                         cudaMemcpyHostToDevice, S.s_in));
             CK(cudaEventRecord(S.ev_stage_ready[sg], S.s_in));
             CK(cudaStreamWaitEvent(S.s_comp, S.ev_stage_ready[sg], 0));
             CK(launch_bwd_delta(d, P->elem, S.stage_o[sg], S.stage_do[sg], (int64_t)nr, g, S.delta + b * Bk, N,
@@ -1206,27 +1220,33 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
                 if (c.evict >= 0) {
                     if (it >= 2) CK(cudaStreamWaitEvent(S.s_out, S.ev_comp[par], 0));
                     const size_t nr = (size_t)pl.block_rows(c.evict);
-                    for (int i = 0; i < 3; ++i)
-                        CK(copy_rows(S.spill + ((size_t)i * N + (size_t)c.evict * Bk) * g * d, acc_row,
-                                     S.acc[i] + srow * g * d, acc_row, acc_row, nr, cudaMemcpyDeviceToHost, S.s_out));
+                    for (int i = 0; i < 3; ++i) {
+                        const int gh = grp_h[i];
+                        CK(copy_rows(spill_of[i] + (size_t)c.evict * Bk * gh * d, acc_row(gh),
+                                     S.acc[i] + srow * gh * d, acc_row(gh), acc_row(gh), nr, cudaMemcpyDeviceToHost,
+                                     S.s_out));
+                    }
                     CK(cudaEventRecord(S.ev_spill[c.evict], S.s_out));
                     CK(cudaEventRecord(S.ev_slot_free[c.slot], S.s_out));
                 }
                 CK(cudaStreamWaitEvent(S.s_in, S.ev_slot_free[c.slot], 0));
                 const size_t nr = (size_t)pl.block_rows(c.block);
-                const size_t off = ((size_t)c.block * Bk * H + h0) * d * e;
-                for (int i = 0; i < 4; ++i)
-                    CK(copy_rows(S.pool[i] + srow * grp_row, grp_row, src[i] + off, full_row, grp_row, nr,
-                                 cudaMemcpyHostToDevice, S.s_in));
+                for (int i = 0; i < 4; ++i) {
+                    const size_t off = ((size_t)c.block * Bk * full_h[i] + hh[i]) * d * e;
+                    CK(copy_rows(S.pool[i] + srow * row_bytes(grp_h[i]), row_bytes(grp_h[i]), src[i] + off,
+                                 row_bytes(full_h[i]), row_bytes(grp_h[i]), nr, cudaMemcpyHostToDevice, S.s_in));
+                }
                 if (c.reload) {
                     CK(cudaStreamWaitEvent(S.s_in, S.ev_spill[c.block], 0));
-                    for (int i = 0; i < 3; ++i)
-                        CK(copy_rows(S.acc[i] + srow * g * d, acc_row,
-                                     S.spill + ((size_t)i * N + (size_t)c.block * Bk) * g * d, acc_row, acc_row, nr,
+                    for (int i = 0; i < 3; ++i) {
+                        const int gh = grp_h[i];
+                        CK(copy_rows(S.acc[i] + srow * gh * d, acc_row(gh),
+                                     spill_of[i] + (size_t)c.block * Bk * gh * d, acc_row(gh), acc_row(gh), nr,
                                      cudaMemcpyHostToDevice, S.s_in));
+                    }
                 } else {
                     for (int i = 0; i < 3; ++i)
-                        CK(cudaMemsetAsync(S.acc[i] + srow * g * d, 0, slot_rows * acc_row, S.s_in));
+                        CK(cudaMemsetAsync(S.acc[i] + srow * grp_h[i] * d, 0, slot_rows * acc_row(grp_h[i]), S.s_in));
                 }
             }
             CK(cudaEventRecord(S.ev_in_ready[par], S.s_in));
@@ -1246,37 +1266,44 @@ cqsa_status_t backward_host(cqsa_plan_t *P, const void *q, const void *k, const 
                     CK(launch_bwd_dq(d, P->elem, pq, S.qwl[t].num_units, S.s_comp));
                 tm.stop();
             }
-            {
+            // One launch per query-head residue modulo the key/value group,
+            // so no two CTAs of a launch add into one key/value head's sums.
+            for (int j = 0; j < kvg; ++j) {
+                const int u0 = S.kv_split[t][j], nu = S.kv_split[t][j + 1] - u0;
+                if (nu <= 0) continue;
                 BwdParams pk = bp;
                 pk.entries = S.kvwl[t].entries;
                 pk.runs = S.kvwl[t].runs;
-                pk.units = S.kvwl[t].units;
+                pk.units = S.kvwl[t].units + u0;
                 pk.part_a = S.acc[1];
                 pk.part_b = S.acc[2];
                 LaunchTimer tm(P, S.s_comp, 2);
                 if (P->dtype == CQSA_BF16)
-                    CK(launch_bwd_dkdv_tc(d, S.mq, S.mk, S.mv, S.mdo, pk, S.kvwl[t].num_units, P->timeout_ns,
-                                          S.err, S.s_comp));
+                    CK(launch_bwd_dkdv_tc(d, S.mq, S.mk, S.mv, S.mdo, pk, nu, P->timeout_ns, S.err, S.s_comp));
                 else
-                    CK(launch_bwd_dkdv(d, P->elem, pk, S.kvwl[t].num_units, S.s_comp));
+                    CK(launch_bwd_dkdv(d, P->elem, pk, nu, S.s_comp));
                 tm.stop();
             }
             // -- blocks this task finished: their sums in the plan dtype over
             // their Q, K, V rows (no longer needed), then to the host.
             for (const auto &f : cp.finals[t])
-                for (int i = 0; i < 3; ++i)
-                    CK(launch_cast_out(P->elem, S.acc[i] + (size_t)f.second * slot_rows * g * d,
-                                       S.pool[i] + (size_t)f.second * slot_rows * grp_row, (int64_t)cast_n,
-                                       S.s_comp));
+                for (int i = 0; i < 3; ++i) {
+                    const int gh = grp_h[i];
+                    CK(launch_cast_out(P->elem, S.acc[i] + (size_t)f.second * slot_rows * gh * d,
+                                       S.pool[i] + (size_t)f.second * slot_rows * row_bytes(gh),
+                                       (int64_t)(slot_rows * gh * d), S.s_comp));
+                }
             CK(cudaEventRecord(S.ev_comp[par], S.s_comp));
             if (!cp.finals[t].empty()) {
                 CK(cudaStreamWaitEvent(S.s_out, S.ev_comp[par], 0));
                 for (const auto &f : cp.finals[t]) {
                     const size_t nr = (size_t)pl.block_rows(f.first);
-                    const size_t off = ((size_t)f.first * Bk * H + h0) * d * e;
-                    for (int i = 0; i < 3; ++i)
-                        CK(copy_rows(dst[i] + off, full_row, S.pool[i] + (size_t)f.second * slot_rows * grp_row,
-                                     grp_row, grp_row, nr, cudaMemcpyDeviceToHost, S.s_out));
+                    for (int i = 0; i < 3; ++i) {
+                        const size_t off = ((size_t)f.first * Bk * full_h[i] + hh[i]) * d * e;
+                        CK(copy_rows(dst[i] + off, row_bytes(full_h[i]),
+                                     S.pool[i] + (size_t)f.second * slot_rows * row_bytes(grp_h[i]),
+                                     row_bytes(grp_h[i]), row_bytes(grp_h[i]), nr, cudaMemcpyDeviceToHost, S.s_out));
+                    }
                     CK(cudaEventRecord(S.ev_slot_free[f.second], S.s_out));
                 }
             }
@@ -1507,13 +1534,14 @@ cqsa_status_t cqsa_backward(cqsa_plan_t *plan, const void *q, const void *k, con
         if ((st = check_ptr(ptrs[i], true, names[i])) != CQSA_OK) return st;
     const Planner &pl = plan->pl;
     const size_t qs = (size_t)pl.spec.N * pl.spec.H * pl.spec.d * plan->elem, ls = (size_t)pl.spec.N * pl.spec.H;
+    const size_t kvs = (size_t)pl.spec.N * pl.spec.Hkv * pl.spec.d * plan->elem;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     for (int b = 0; b < pl.spec.B; ++b) {
-        auto at = [&](const void *p) { return static_cast<const char *>(p) + b * qs; };
-        auto atw = [&](void *p) { return static_cast<char *>(p) + b * qs; };
+        auto at = [&](const void *p, size_t stride) { return static_cast<const char *>(p) + b * stride; };
+        auto atw = [&](void *p, size_t stride) { return static_cast<char *>(p) + b * stride; };
         st = guarded([&] {
-            return backward_host(plan, at(q), at(k), at(v), at(out), lse + b * ls, at(dout), atw(dq), atw(dk),
-                                 atw(dv), cs);
+            return backward_host(plan, at(q, qs), at(k, kvs), at(v, kvs), at(out, qs), lse + b * ls, at(dout, qs),
+                                 atw(dq, qs), atw(dk, kvs), atw(dv, kvs), cs);
         });
         if (st != CQSA_OK) {
             join_bwd_after_error(plan, cs);

@@ -316,7 +316,9 @@ __global__ void __launch_bounds__(bwd::THREADS) bwd_dkdv_kernel(const BwdParams 
 
     // Direct writes only when one query head owns the key/value head.
     const bool direct = p.kv_group == 1 && (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
-    const int64_t slot = (int64_t)e.slot * p.kv_group + h % p.kv_group;
+    // Streamed backward: one launch never holds two query heads of a
+    // key/value group, so they all add into the one set of sums.
+    const int64_t slot = p.accum ? 0 : (int64_t)e.slot * p.kv_group + h % p.kv_group;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int32_t row = k0 + ty * 4 + i;

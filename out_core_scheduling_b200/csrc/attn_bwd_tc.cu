@@ -715,7 +715,9 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             const bool fused = p.kv_group == 1 && (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
             const int64_t orow = (int64_t)e.out_lo + (k_local - e.q_lo);
             const int hkv = head / p.kv_group;
-            const int64_t slot = (int64_t)e.slot * p.kv_group + head % p.kv_group;
+            // Streamed backward: one launch never holds two query heads of a
+            // key/value group, so they all add into the one set of sums.
+            const int64_t slot = p.accum ? 0 : (int64_t)e.slot * p.kv_group + head % p.kv_group;
             // Warps of columns 0-63 write dK, those of 64-127 dV.
             {
                 const int which = hf;

@@ -987,20 +987,33 @@ WorkList Planner::leaf_bwd_kv_worklist(int64_t t, const BwdCachePlan &c, int row
         wl.entries.push_back(w);
     }
     add_units_kv(&wl, heads, rows_per_unit, bn, spec.causal);
+    // Grouped-query attention: units by query head modulo the group size, so
+    // that each launch takes the query heads of one residue and no two of a
+    // launch's CTAs add into the same key/value head's sums.
+    const int kvg = spec.kv_group();
+    if (kvg > 1)
+        std::stable_sort(wl.units.begin(), wl.units.end(),
+                         [kvg](const WlUnit &a, const WlUnit &b) { return a.head % kvg < b.head % kvg; });
     return wl;
 }
 
 size_t Planner::bwd_arena_bytes(int g, const BwdCachePlan &c) const {
     const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d, N = (size_t)spec.N;
     const size_t rows = (size_t)c.slots * block;
+    const size_t gk = (size_t)(g / spec.kv_group());  // key/value heads of the group
     const int tile = spec.elem_bytes == 2 ? 128 : 64;
     ArenaLayout a;
     a.take(256);                                  // error word
     a.take((size_t)g * N * sizeof(float));        // lse of the head group
     a.take((size_t)g * N * sizeof(float));        // D = rowsum(dO * O)
     for (int s = 0; s < 4; ++s) a.take((size_t)block * g * dd * e);  // O / dO staging, two stages
-    for (int s = 0; s < 4; ++s) a.take(rows * g * dd * e);           // Q, K, V, dO pools
-    for (int s = 0; s < 3; ++s) a.take(rows * g * dd * sizeof(float));  // dQ, dK, dV sums
+    a.take(rows * g * dd * e);                    // Q pool
+    a.take(rows * gk * dd * e);                   // K pool
+    a.take(rows * gk * dd * e);                   // V pool
+    a.take(rows * g * dd * e);                    // dO pool
+    a.take(rows * g * dd * sizeof(float));        // dQ sums
+    a.take(rows * gk * dd * sizeof(float));       // dK sums
+    a.take(rows * gk * dd * sizeof(float));       // dV sums
     for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
         a.take(wl_bytes(leaf_bwd_q_worklist(t, c, tile, tile, g)));
         a.take(wl_bytes(leaf_bwd_kv_worklist(t, c, tile, tile, g)));
@@ -1011,9 +1024,10 @@ size_t Planner::bwd_arena_bytes(int g, const BwdCachePlan &c) const {
 void Planner::size_bwd() {
     bwd_sizing = BwdSizing{};
     bwd_cache = BwdCachePlan{};
-    // Grouped-query plans would need several query heads to add into one
-    // key/value head's sums within a launch; they take the device path.
-    if (spec.kv_group() != 1 || spec.shard_count > 1) return;
+    // Head groups cover whole key/value groups, so that a key/value head's
+    // sums collect all of its query heads' terms within one head group.
+    if (spec.shard_count > 1) return;
+    const int kvg = spec.kv_group();
     const std::vector<std::vector<int64_t>> tb = bwd_task_blocks(*this);
     bwd_min_slots = 0;
     std::vector<int64_t> all;
@@ -1034,7 +1048,7 @@ void Planner::size_bwd() {
     // to the larger group).
     double best_traffic = -1;
     for (int g = spec.H; g >= 1; --g) {
-        if (spec.H % g) continue;
+        if (spec.H % g || g % kvg) continue;
         if (!spec.budget && g < spec.H) break;  // unlimited: all heads at once, every block cached
         BwdCachePlan cp;
         int64_t C = bwd_full_slots;
@@ -1058,13 +1072,15 @@ void Planner::size_bwd() {
             plan_bwd_cache(C, &cp);
             bytes = bwd_arena_bytes(g, cp);
         }
-        const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
-        const size_t acc = (size_t)block * g * spec.d * sizeof(float);
+        const size_t gh = (size_t)g + (size_t)(g / kvg);  // heads of (Q, dO) and of (K, V): per pair
+        const size_t blk = (size_t)block * spec.d * spec.elem_bytes;     // one head of one block
+        const size_t acc = (size_t)block * spec.d * sizeof(float);
         const size_t groups = (size_t)(spec.H / g);
         const size_t N = (size_t)spec.N;
+        const size_t sums = (size_t)g + 2 * (size_t)(g / kvg);             // heads of dQ, dK, dV
         const size_t h2d = groups * ((size_t)g * N * sizeof(float) + 2 * N * g * spec.d * spec.elem_bytes +
-                                     (size_t)cp.loads * 4 * blk + (size_t)cp.writebacks * 3 * acc);
-        const size_t d2h = groups * (3 * N * g * spec.d * spec.elem_bytes + (size_t)cp.writebacks * 3 * acc);
+                                     (size_t)cp.loads * 2 * gh * blk + (size_t)cp.writebacks * sums * acc);
+        const size_t d2h = groups * (N * sums * spec.d * spec.elem_bytes + (size_t)cp.writebacks * sums * acc);
         const double traffic = (double)h2d + (double)d2h;
         if (best_traffic < 0 || traffic < best_traffic) {
             best_traffic = traffic;
@@ -1073,7 +1089,7 @@ void Planner::size_bwd() {
             bwd_sizing.slots = C;
             bwd_sizing.h2d = h2d * (size_t)spec.B;
             bwd_sizing.d2h = d2h * (size_t)spec.B;
-            bwd_sizing.spill_host = cp.writebacks ? 3 * N * g * spec.d * sizeof(float) : 0;
+            bwd_sizing.spill_host = cp.writebacks ? N * sums * spec.d * sizeof(float) : 0;
             bwd_cache = std::move(cp);
         }
     }

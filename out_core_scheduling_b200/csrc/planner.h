@@ -254,7 +254,9 @@ public:
     // the two work lists of leaf t in cache coordinates (rows of block b at
     // slot * block): query-stationary (dq, one entry per (task, query
     // block)) and key-stationary (dk and dv, one entry per (task, key
-    // block)); each entry's sums go to the block's own slot rows.
+    // block)); each entry's sums go to the block's own slot rows.  With
+    // grouped-query attention the key-stationary list's units are ordered
+    // by query head modulo the group size (one launch per residue).
     bool plan_bwd_cache(int64_t slots, BwdCachePlan *out) const;
     size_t bwd_arena_bytes(int g, const BwdCachePlan &c) const;
     WorkList leaf_bwd_q_worklist(int64_t t, const BwdCachePlan &c, int rows_per_unit, int bn, int heads) const;

@@ -136,7 +136,7 @@ def test_streamed_backward_batch():
         _compare(dv[b], ref_dv, torch.bfloat16, "dv")
 
 
-def test_streamed_backward_rejects_pageable_and_grouped_query():
+def test_streamed_backward_rejects_pageable():
     N, H, d = 7 * 64, 2, 64
     plan = cqsa.cqsa_plan_ex(N, H, d, [3], mem_budget_bytes=1 << 30)
     x = torch.zeros(N, H, d, dtype=torch.bfloat16)
@@ -144,14 +144,51 @@ def test_streamed_backward_rejects_pageable_and_grouped_query():
     with pytest.raises(cqsa.CqsaError) as ei:
         cqsa.cqsa_backward(plan, x, x, x, x, lse, x, x, x, x, host_or_device=cqsa.CQSA_HOST)
     assert ei.value.status == cqsa.CQSA_ERR_NOT_PINNED
-    gplan = cqsa.cqsa_plan_ex(N, 4, d, [3], H_kv=2, mem_budget_bytes=1 << 30)
-    q = torch.zeros(N, 4, d, dtype=torch.bfloat16).pin_memory()
-    kv = torch.zeros(N, 2, d, dtype=torch.bfloat16).pin_memory()
-    l4 = torch.zeros(4, N).pin_memory()
-    with pytest.raises(cqsa.CqsaError) as ei:
-        cqsa.cqsa_backward(gplan, q, kv, kv, q, l4, q, q.clone().pin_memory(), kv.clone().pin_memory(),
-                           kv.clone().pin_memory(), host_or_device=cqsa.CQSA_HOST)
-    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("tight", [False, True], ids=["roomy", "tight"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", [(13 * 128, 4, 2, 128, [4], torch.bfloat16), (7 * 100, 8, 2, 64, [3], torch.bfloat16),
+                                  (7 * 128, 4, 1, 64, [3], torch.float32)],
+                         ids=lambda c: f"n{c[0]}-h{c[1]}-kv{c[2]}-d{c[3]}-{str(c[5])[6:]}")
+def test_streamed_backward_grouped_query(case, causal, tight):
+    """dk, dv of a key/value head sum the terms of its query heads; the
+    streamed path adds them in one launch per query-head residue."""
+    N, H, Hkv, d, ls, dtype = case
+    g = H // Hkv
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    budget = 1 << 34
+    if tight:
+        lo, hi = 1 << 20, 1 << 36
+        while hi - lo > hi // 100:
+            mid = (lo + hi) // 2
+            try:
+                i = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, H_kv=Hkv, mem_budget_bytes=mid).info()
+                ok = i["bwd_head_group"] and i["head_group"]
+            except cqsa.CqsaError:
+                ok = 0
+            lo, hi = (lo, mid) if ok else (mid, hi)
+        budget = hi
+    q = make_qkv(N, H, d, dtype=dtype, seed=74, device=DEV)[0]
+    _, k, v = make_qkv(N, Hkv, d, dtype=dtype, seed=75, device=DEV)
+    dout = make_qkv(N, H, d, dtype=dtype, seed=76, device=DEV)[0]
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, H_kv=Hkv, mem_budget_bytes=budget)
+    assert plan.info()["bwd_host_arena_bytes"] <= budget
+    hq, hk, hv, hd = _pinned(q, k, v, dout)
+    out = torch.empty(hq.shape, dtype=dtype).pin_memory()
+    lse = torch.empty(H, N).pin_memory()
+    cqsa.cqsa_forward(plan, hq, hk, hv, out, lse, cqsa.CQSA_HOST)
+    gq = torch.empty(hq.shape, dtype=dtype).pin_memory()
+    gk, gv = (torch.empty(hk.shape, dtype=dtype).pin_memory() for _ in range(2))
+    cqsa.cqsa_backward(plan, hq, hk, hv, out, lse, hd, gq, gk, gv, host_or_device=cqsa.CQSA_HOST)
+    plan.sync()
+    ke = k.repeat_interleave(g, dim=1).contiguous().cpu()
+    ve = v.repeat_interleave(g, dim=1).contiguous().cpu()
+    ref_dq, _, _ = oracle.attention_backward_dq(q.cpu(), ke, ve, dout.cpu(), causal=causal)
+    ref_dk, ref_dv = oracle.attention_backward_dkdv(q.cpu(), ke, ve, dout.cpu(), causal=causal)
+    _compare(gq, ref_dq, dtype, "dq")
+    _compare(gk, ref_dk.reshape(N, Hkv, g, d).sum(2), dtype, "dk")
+    _compare(gv, ref_dv.reshape(N, Hkv, g, d).sum(2), dtype, "dv")
 
 
 def test_l5_n688128_h8_streamed_backward_2gib():

@@ -155,9 +155,34 @@ def test_workload_budgets():
         assert info["bwd_host_arena_bytes"] <= budget
 
 
-def test_grouped_query_plans_have_no_streamed_backward():
-    info = cqsa.cqsa_plan_ex(7 * 64, 4, 64, [3], H_kv=2, mem_budget_bytes=1 << 30).info()
-    assert info["bwd_head_group"] == 0
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (8, 2), (4, 1)])
+def test_grouped_query_head_groups_cover_whole_groups(H, Hkv):
+    """A key/value head's sums collect every query head of its group inside
+    one head group, so head groups are whole multiples of the group size,
+    also under a budget that forces small groups."""
+    N, d, ls = 13 * 128, 64, [4]
+    for budget in (1 << 34, _min_budget_gqa(N, H, Hkv, d, ls)):
+        plan = cqsa.cqsa_plan_ex(N, H, d, ls, H_kv=Hkv, mem_budget_bytes=budget)
+        info = plan.info()
+        g = info["bwd_head_group"]
+        assert g >= H // Hkv and g % (H // Hkv) == 0 and H % g == 0
+        assert info["bwd_host_arena_bytes"] <= budget
+        replay(plan)
+
+
+def _min_budget_gqa(N, H, Hkv, d, ls):
+    lo, hi = 1 << 20, 1 << 36
+    while hi - lo > hi // 100:
+        mid = (lo + hi) // 2
+        try:
+            ok = cqsa.cqsa_plan_ex(N, H, d, ls, H_kv=Hkv, mem_budget_bytes=mid).info()["bwd_head_group"]
+        except cqsa.CqsaError:
+            ok = 0
+        if ok:
+            hi = mid
+        else:
+            lo = mid
+    return hi
 
 
 def _tight_plan():
