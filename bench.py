@@ -561,7 +561,7 @@ def measure(args, W, D, workload, steps, warmup, extras):
             result["backward_streamed"] = run_backward_host(args, W, D, plans, infos, q, k, v, outs, lses,
                                                             flops_step, stream, peaks, result["streaming"])
     elif not args.no_e2e:
-        result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream)
+        result["e2e"] = run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream, extras)
 
     # ---- oracle on the host cores (rank 0, N = 1 only).
     if D.rank == 0 and D.world == 1 and not args.no_cpu:
@@ -726,7 +726,11 @@ def run_fused(args, W, D, q, k, v, outs, lses, flops_step, stream, slots_value):
                     "key runs of all the tasks of its rows and writes out and lse; no slots, no merge launch"}
 
 
-def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream):
+def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream, extras=True):
+    """The step through cqsa_forward(CQSA_HOST) from pinned host inputs to
+    pinned host outputs.  The plans fit every block, so the resident
+    schedule runs; with extras, the task-by-task schedule of the same plans
+    is timed beside it."""
     import torch
     from out_core_scheduling_b200 import cqsa
 
@@ -738,31 +742,47 @@ def run_e2e(args, W, D, plans, infos, q, k, v, flops_step, stream):
     outs = [torch.empty(hq.shape, dtype=hq.dtype).pin_memory() for _ in plans]
     lses = [torch.empty(H, N, dtype=torch.float32).pin_memory() for _ in plans]
 
-    def step():
-        for p, o, l in zip(plans, outs, lses):
-            cqsa.cqsa_forward(p, hq, hk, hv, o, l, cqsa.CQSA_HOST, stream)
+    def timed(ps):
+        def step():
+            for p, o, l in zip(ps, outs, lses):
+                cqsa.cqsa_forward(p, hq, hk, hv, o, l, cqsa.CQSA_HOST, stream)
 
-    for _ in range(max(1, min(args.warmup, 3))):
-        step()
-    torch.cuda.synchronize()
-    steps = max(1, min(args.steps, args.e2e_steps))
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    D.barrier(D.local_rank)
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for _ in range(steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    D.barrier(D.local_rank)
-    for p in plans:
-        p.sync(stream)
-    ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}")
-    return {"value": flops_step * steps * D.world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": int(sum(i["h2d_bytes"] for i in infos)),
-            "d2h_bytes_per_step": int(sum(i["d2h_bytes"] for i in infos)),
-            "steps": steps, "ms_per_step": ms / steps,
-            "path": "cqsa_forward(CQSA_HOST): pinned host q,k,v -> streamed tasks -> pinned host out,lse"}
+        for _ in range(max(1, min(args.warmup, 3))):
+            step()
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, args.e2e_steps))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier(D.local_rank)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        D.barrier(D.local_rank)
+        for p in ps:
+            p.sync(stream)
+        ms = D.max(ev0.elapsed_time(ev1), f"cuda:{D.local_rank}")
+        return steps, ms
+
+    steps, ms = timed(plans)
+    hinfo = [p.info() for p in plans]
+    res = {"value": flops_step * steps * D.world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(sum(i["h2d_bytes"] for i in hinfo)),
+           "d2h_bytes_per_step": int(sum(i["d2h_bytes"] for i in hinfo)),
+           "steps": steps, "ms_per_step": ms / steps,
+           "schedule": "resident" if all(i["host_resident"] for i in hinfo) else "tasks",
+           "path": "cqsa_forward(CQSA_HOST): pinned host q,k,v -> device block pools -> pinned host out,lse"}
+    if extras and res["schedule"] == "resident":
+        tp = [cqsa.cqsa_plan_ex(N, H, W["d"], W["ls"], causal=i["causal"], dtype=i["dtype"], host_tasks=True)
+              for i in hinfo]
+        steps_t, ms_t = timed(tp)
+        res["tasks_schedule"] = {"value": flops_step * steps_t * D.world / (ms_t * 1e-3) / 1e12,
+                                 "ms_per_step": ms_t / steps_t,
+                                 "path": "the same call, task by task (cqsa_plan_ex(host_tasks=True))"}
+        for p in tp:
+            p.destroy()
+    return res
 
 
 def host_link_gbs(torch, nbytes=1 << 30):

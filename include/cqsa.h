@@ -110,6 +110,10 @@ typedef struct {
                         computes the entries of shard_rank with
                         cqsa_forward_partial (see there). */
     int shard_count;
+    int host_tasks;  /* host mode: run the streamed forward task by task even
+                        when every block of a head group fits the budget
+                        (0: the resident schedule then, see
+                        cqsa_plan_host_launch). */
 } cqsa_plan_desc_t;
 
 /* What a plan decided (for logging, tests and the benchmark). */
@@ -148,6 +152,9 @@ typedef struct {
     size_t bwd_d2h_bytes;               /* planned device->host bytes of one host-mode backward */
     size_t bwd_spill_host_bytes;        /* pinned host memory the host-mode backward takes for written-back sums */
     int64_t bwd_writebacks;             /* gradient-sum write-backs per head group (0: every block stays cached) */
+    int host_resident;                  /* host-mode forward runs the resident schedule (1) or task by task (0) */
+    int64_t host_launches;              /* launches of the resident schedule per head group (0: task by task) */
+    int64_t arrival_blocks;             /* resident schedule: blocks per arrival group of the copy-in */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */
@@ -385,7 +392,9 @@ cqsa_status_t cqsa_plan_task_blocks(const cqsa_plan_t *plan, int64_t t, int64_t 
  * Arrays hold max_copies / max_blocks entries; *num_copies / *num_blocks
  * get the counts (arrays may be NULL to ask for the counts).  INVALID_ARG
  * when t is out of range or an array is too small; BUDGET when the plan has
- * no host-mode sizing. */
+ * no host-mode sizing.  A plan with info.host_resident set runs the resident
+ * schedule instead (cqsa_plan_host_launch); this is then the cache the
+ * task-by-task schedule would use with every block cached. */
 cqsa_status_t cqsa_plan_cache_task(const cqsa_plan_t *plan, int64_t t, int32_t *kinds, int64_t *blocks,
                                    int32_t *slots, int64_t max_copies, int64_t *num_copies, int32_t *q_slot,
                                    int32_t *kv_slot, int64_t max_blocks, int64_t *num_blocks);
@@ -409,6 +418,24 @@ cqsa_status_t cqsa_plan_bwd_cache_task(const cqsa_plan_t *plan, int64_t t, int64
                                        int64_t *evicts, int32_t *reloads, int64_t max_copies, int64_t *num_copies,
                                        int32_t *member_slot, int64_t max_blocks, int64_t *num_blocks,
                                        int64_t *fin_blocks, int32_t *fin_slots, int64_t max_fin, int64_t *num_fin);
+
+/* cqsa_plan_host_launch -- launch i (0 <= i < info.host_launches) of the
+ * streamed forward's resident schedule, used when every block of a head
+ * group fits the budget ([B] "Implementation": stream the blocks the tasks
+ * need; here each block crosses the host link once per head group).  The
+ * blocks are copied in increasing order; the copy stream marks every
+ * info.arrival_blocks consecutive blocks.  The launch waits for the mark of
+ * the group holding *need (the last block it reads), runs on internal
+ * compute stream *stream (0 or 1), and first waits for launch *after of the
+ * other stream (-1: none).  It takes the plan's (query block, key block)
+ * pairs pairs[2p], pairs[2p + 1], p < *num_pairs, in query-block order;
+ * flags[p] is its entry's SEG flags for that query block (1: the block's
+ * first launch, starts its accumulator; 2: its last, writes its finished
+ * rows, which then go to the host).  Arrays may be NULL to ask for the
+ * count.  INVALID_ARG when i is out of range or an array is too small. */
+cqsa_status_t cqsa_plan_host_launch(const cqsa_plan_t *plan, int64_t i, int64_t *need, int32_t *stream,
+                                    int32_t *after, int64_t *pairs, int32_t *flags, int64_t max_pairs,
+                                    int64_t *num_pairs);
 
 /* cqsa_plan_entry -- entry i (0 <= i < num_entries) of the work list and its
  * key runs: runs[2r], runs[2r+1] are the first and last global key block of

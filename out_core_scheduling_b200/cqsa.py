@@ -44,6 +44,7 @@ EXPORTS = (
     "cqsa_last_error", "cqsa_forward_partial", "cqsa_partial_rescale", "cqsa_partial_finish",
     "cqsa_debug_inject", "cqsa_backward_partial", "cqsa_partial_cast", "cqsa_plan_cache_task",
     "cqsa_plan_bwd_cache_task", "cqsa_shard_layout", "cqsa_shard_pack", "cqsa_shard_merge", "cqsa_shard_unpack",
+    "cqsa_plan_host_launch",
 )
 
 
@@ -58,7 +59,8 @@ class PlanDesc(ctypes.Structure):
                 ("levels", ctypes.c_int), ("l", ctypes.c_int * MAX_LEVELS),
                 ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("mem_budget_bytes", ctypes.c_size_t), ("merge", ctypes.c_int), ("H_kv", ctypes.c_int),
-                ("B", ctypes.c_int), ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int)]
+                ("B", ctypes.c_int), ("shard_rank", ctypes.c_int), ("shard_count", ctypes.c_int),
+                ("host_tasks", ctypes.c_int)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -80,7 +82,8 @@ class PlanInfo(ctypes.Structure):
                 ("bwd_head_group", ctypes.c_int), ("bwd_host_arena_bytes", ctypes.c_size_t),
                 ("bwd_cache_slots", ctypes.c_int64), ("bwd_h2d_bytes", ctypes.c_size_t),
                 ("bwd_d2h_bytes", ctypes.c_size_t), ("bwd_spill_host_bytes", ctypes.c_size_t),
-                ("bwd_writebacks", ctypes.c_int64)]
+                ("bwd_writebacks", ctypes.c_int64), ("host_resident", ctypes.c_int),
+                ("host_launches", ctypes.c_int64), ("arrival_blocks", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         out = {}
@@ -143,6 +146,10 @@ def load_library():
                                           ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
                                           ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
                                           ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
+        "cqsa_plan_host_launch": (st, [P, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
         "cqsa_shard_layout": (st, [P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
                                    ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
                                    ctypes.POINTER(ctypes.c_size_t)]),
@@ -248,6 +255,23 @@ class Plan:
                 "member_slot": list(ms)[: nb.value],
                 "finals": [(fb[j], fs[j]) for j in range(nf.value)]}
 
+    def host_launch(self, i: int) -> dict:
+        """Launch i of the streamed forward's resident schedule: the last
+        block it reads (need), its compute stream, the launch of the other
+        stream it waits for (after, -1: none), and its (query block, key
+        block) pairs with their entries' SEG flags."""
+        lib = load_library()
+        need, n = ctypes.c_int64(), ctypes.c_int64()
+        stream, after = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.cqsa_plan_host_launch(self.handle, i, ctypes.byref(need), ctypes.byref(stream),
+                                         ctypes.byref(after), None, None, 0, ctypes.byref(n)))
+        pairs = (ctypes.c_int64 * (2 * max(1, n.value)))()
+        flags = (ctypes.c_int32 * max(1, n.value))()
+        _check(lib.cqsa_plan_host_launch(self.handle, i, None, None, None, pairs, flags, n.value, ctypes.byref(n)))
+        return {"need": need.value, "stream": stream.value, "after": after.value,
+                "pairs": [(pairs[2 * p], pairs[2 * p + 1]) for p in range(n.value)],
+                "flags": list(flags)[: n.value]}
+
     def entry(self, i: int):
         lib = load_library()
         e = Entry()
@@ -294,7 +318,7 @@ def cqsa_plan(N: int, H: int, d: int, l: int, levels: int = 1, causal: bool = Fa
 
 def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = CQSA_BF16,
                  mem_budget_bytes: int = 0, merge: int = CQSA_MERGE_SLOTS, H_kv: int = 0, B: int = 1,
-                 shard_rank: int = 0, shard_count: int = 1) -> Plan:
+                 shard_rank: int = 0, shard_count: int = 1, host_tasks: bool = False) -> Plan:
     desc = PlanDesc()
     desc.N, desc.H, desc.d = N, H, d
     desc.levels = len(ls)
@@ -307,6 +331,7 @@ def cqsa_plan_ex(N: int, H: int, d: int, ls, causal: bool = False, dtype: int = 
     desc.H_kv = H_kv
     desc.B = B
     desc.shard_rank, desc.shard_count = shard_rank, shard_count
+    desc.host_tasks = int(bool(host_tasks))
     h = ctypes.c_void_p()
     _check(load_library().cqsa_plan_ex(ctypes.byref(desc), ctypes.byref(h)))
     return Plan(h.value)

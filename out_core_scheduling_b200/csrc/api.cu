@@ -282,6 +282,13 @@ struct cqsa_plan {
     cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
     cudaEvent_t ev_in_ready[2] = {}, ev_in_free[2] = {}, ev_merged[2] = {}, ev_out_free[2] = {};
     cudaEvent_t ev_start = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
+    // Resident schedule (Planner::host_sched): per launch its work list, a
+    // second compute stream, a mark per arrival group and per launch, and
+    // the ends of a head group on the compute and copy-out streams.
+    std::vector<DevWl> res_wl;
+    cudaStream_t s_comp2 = nullptr;
+    std::vector<cudaEvent_t> ev_arrive, ev_launch;
+    cudaEvent_t ev_comp_end[2] = {}, ev_out_end = nullptr;
 
     // Kernel timing (cqsa_plan_profile): event pairs not yet read, a pool of
     // spare events, and the totals read so far.
@@ -398,6 +405,74 @@ cqsa_status_t setup_device_mode(cqsa_plan_t *P) {
 
 void release_bwd_host(cqsa_plan_t *P);
 
+// Arena, work lists, streams and events of the resident schedule.
+cqsa_status_t setup_resident(cqsa_plan_t *P) {
+    const Planner &pl = P->pl;
+    const std::vector<HostLaunch> &LS = pl.host_sched;
+    const int g = pl.sizing.head_group, gk = pl.spec.kv_heads_of(g);
+    const int64_t N = pl.spec.N, rows = pl.num_blocks * pl.block;
+    const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
+    // Same layout steps as Planner::resident_arena_bytes.
+    ArenaLayout a;
+    const size_t o_err = a.take(256);
+    const size_t o_acc = a.take((size_t)N * g * dd * sizeof(float));
+    const size_t o_accl = a.take((size_t)g * N * sizeof(float));
+    const size_t o_pq = a.take((size_t)rows * g * dd * e);
+    const size_t o_pk = a.take((size_t)rows * gk * dd * e);
+    const size_t o_pv = a.take((size_t)rows * gk * dd * e);
+    const size_t o_out = a.take((size_t)N * g * dd * e);
+    const size_t o_lse = a.take((size_t)g * N * sizeof(float));
+    std::vector<size_t> o_wl(LS.size());
+    for (size_t i = 0; i < LS.size(); ++i) o_wl[i] = a.take(wl_region(LS[i].wl));
+    if (a.total != pl.sizing.host_arena)
+        return fail(CQSA_ERR_CUDA, "internal: resident arena layout mismatch (%zu vs %zu)", a.total,
+                    pl.sizing.host_arena);
+    char *arena = nullptr;
+    CK(lib_malloc(reinterpret_cast<void **>(&arena), a.total));
+    P->host_arena = arena;
+    P->host_bytes = a.total;
+    P->g = g;
+    // Zeroed once, so rows a partial key tile reads past the last block are finite.
+    CK(cudaMemset(arena, 0, a.total));
+    P->h_err = reinterpret_cast<int *>(arena + o_err);
+    P->acc_o = reinterpret_cast<float *>(arena + o_acc);
+    P->acc_lse = reinterpret_cast<float *>(arena + o_accl);
+    P->pool_q = arena + o_pq;
+    P->pool_k = arena + o_pk;
+    P->pool_v = arena + o_pv;
+    P->out_st[0] = arena + o_out;
+    P->lse_st[0] = reinterpret_cast<float *>(arena + o_lse);
+    P->out_st[1] = nullptr;
+    P->lse_st[1] = nullptr;
+    P->res_wl.assign(LS.size(), DevWl());
+    for (size_t i = 0; i < LS.size(); ++i) {
+        std::vector<char> buf = pack_wl(LS[i].wl);
+        if (!buf.empty()) CK(lib_upload(arena + o_wl[i], buf.data(), buf.size()));
+        P->res_wl[i] = place_wl(arena + o_wl[i], LS[i].wl);
+    }
+    if (P->dtype == CQSA_BF16) {
+        cqsa_status_t st;
+        if ((st = make_map(&P->mq, P->pool_q, rows, g, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mk, P->pool_k, rows, gk, pl.spec.d)) != CQSA_OK) return st;
+        if ((st = make_map(&P->mv, P->pool_v, rows, gk, pl.spec.d)) != CQSA_OK) return st;
+    }
+    CK(cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&P->s_comp2, cudaStreamNonBlocking));
+    CK(cudaStreamCreateWithFlags(&P->s_out, cudaStreamNonBlocking));
+    const int64_t A = pl.arrival_blocks();
+    P->ev_arrive.assign((size_t)((pl.num_blocks + A - 1) / A), nullptr);
+    P->ev_launch.assign(LS.size(), nullptr);
+    for (cudaEvent_t &ev : P->ev_arrive) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    for (cudaEvent_t &ev : P->ev_launch) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    for (int s = 0; s < 2; ++s) CK(cudaEventCreateWithFlags(&P->ev_comp_end[s], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_out_end, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_start, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_done_comp, cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&P->ev_done_out, cudaEventDisableTiming));
+    return CQSA_OK;
+}
+
 cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     if (P->host_arena) return CQSA_OK;
     const Planner &pl = P->pl;
@@ -412,6 +487,7 @@ cqsa_status_t setup_host_mode_impl(cqsa_plan_t *P) {
     const size_t blk = (size_t)pl.block * g * dd * e;
     const int gk = pl.spec.kv_heads_of(g);  // key/value heads of a head group
     const size_t blk_kv = (size_t)pl.block * gk * dd * e;
+    if (pl.sizing.resident) return setup_resident(P);
     const PoolPlan &pp = pl.pool;
     // Same layout steps as Planner::host_arena_bytes.
     ArenaLayout a;
@@ -489,13 +565,20 @@ void release_host_mode(cqsa_plan_t *P) {
                 *e = nullptr;
             }
     }
-    cudaEvent_t *evs[3] = {&P->ev_start, &P->ev_done_comp, &P->ev_done_out};
+    cudaEvent_t *evs[6] = {&P->ev_start, &P->ev_done_comp, &P->ev_done_out, &P->ev_comp_end[0],
+                           &P->ev_comp_end[1], &P->ev_out_end};
     for (cudaEvent_t *e : evs)
         if (*e) {
             cudaEventDestroy(*e);
             *e = nullptr;
         }
-    cudaStream_t *ss[3] = {&P->s_in, &P->s_comp, &P->s_out};
+    for (std::vector<cudaEvent_t> *v : {&P->ev_arrive, &P->ev_launch}) {
+        for (cudaEvent_t e : *v)
+            if (e) cudaEventDestroy(e);
+        v->clear();
+    }
+    P->res_wl.clear();
+    cudaStream_t *ss[4] = {&P->s_in, &P->s_comp, &P->s_comp2, &P->s_out};
     for (cudaStream_t *s : ss)
         if (*s) {
             cudaStreamDestroy(*s);
@@ -829,10 +912,116 @@ cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, 
     return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, kind, s);
 }
 
+// The resident schedule (Planner::host_sched): per head group, every block
+// to its own pool slot in increasing order with a mark per arrival group;
+// each launch on its compute stream after its blocks' mark and the launch of
+// the other stream it depends on; the rows it finishes to the host.  The
+// enqueue order is modelled in tests/test_resident_schedule.py over every
+// interleaving of the four streams.
+cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k, const void *v, void *out,
+                                    float *lse, cudaStream_t stream) {
+    const Planner &pl = P->pl;
+    const std::vector<HostLaunch> &LS = pl.host_sched;
+    const int64_t N = pl.spec.N, Bk = pl.block, A = pl.arrival_blocks(), nb = pl.num_blocks;
+    const int H = pl.spec.H, d = pl.spec.d, g = P->g;
+    const int Hkv = pl.spec.Hkv, kvg = pl.spec.kv_group(), gk = pl.spec.kv_heads_of(g);
+    const size_t e = (size_t)P->elem;
+    const size_t full_row = (size_t)H * d * e, grp_row = (size_t)g * d * e;
+    const size_t full_kv_row = (size_t)Hkv * d * e, grp_kv_row = (size_t)gk * d * e;
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
+               *hv = static_cast<const char *>(v);
+    char *ho = static_cast<char *>(out);
+    cudaStream_t sc[2] = {P->s_comp, P->s_comp2};
+    CK(cudaEventRecord(P->ev_start, stream));
+    for (cudaStream_t x : {P->s_in, sc[0], sc[1], P->s_out}) CK(cudaStreamWaitEvent(x, P->ev_start, 0));
+    for (int h0 = 0; h0 < H; h0 += g) {
+        NvtxRange nvtx_group("cqsa resident head group", h0);
+        if (h0 > 0) {
+            // The pools change once the previous group's launches are done;
+            // its accumulators and finished rows once its launches and
+            // copy-out are.
+            CK(cudaStreamWaitEvent(P->s_in, P->ev_comp_end[0], 0));
+            CK(cudaStreamWaitEvent(P->s_in, P->ev_comp_end[1], 0));
+            for (int s = 0; s < 2; ++s) {
+                CK(cudaStreamWaitEvent(sc[s], P->ev_comp_end[1 - s], 0));
+                CK(cudaStreamWaitEvent(sc[s], P->ev_out_end, 0));
+            }
+        }
+        // -- H2D: block b to pool rows b * Bk.
+        for (int64_t b = 0; b < nb; ++b) {
+            const size_t rows = (size_t)pl.block_rows(b);
+            if (rows) {
+                const size_t src = ((size_t)b * Bk * H + h0) * d * e;
+                const size_t src_kv = ((size_t)b * Bk * Hkv + h0 / kvg) * d * e;
+                CK(copy_rows(P->pool_q + (size_t)b * Bk * grp_row, grp_row, hq + src, full_row, grp_row, rows,
+                             cudaMemcpyHostToDevice, P->s_in));
+                CK(copy_rows(P->pool_k + (size_t)b * Bk * grp_kv_row, grp_kv_row, hk + src_kv, full_kv_row,
+                             grp_kv_row, rows, cudaMemcpyHostToDevice, P->s_in));
+                CK(copy_rows(P->pool_v + (size_t)b * Bk * grp_kv_row, grp_kv_row, hv + src_kv, full_kv_row,
+                             grp_kv_row, rows, cudaMemcpyHostToDevice, P->s_in));
+            }
+            if ((b + 1) % A == 0 || b == nb - 1) CK(cudaEventRecord(P->ev_arrive[(size_t)(b / A)], P->s_in));
+        }
+        for (size_t i = 0; i < LS.size(); ++i) {
+            const HostLaunch &L = LS[i];
+            cudaStream_t s = sc[L.stream];
+            CK(cudaStreamWaitEvent(s, P->ev_arrive[(size_t)(L.need / A)], 0));
+            if (L.after >= 0) CK(cudaStreamWaitEvent(s, P->ev_launch[(size_t)L.after], 0));
+            AttnParams ap = base_params(P, P->h_err);
+            ap.entries = P->res_wl[i].entries;
+            ap.runs = P->res_wl[i].runs;
+            ap.units = P->res_wl[i].units;
+            ap.H = g;
+            ap.Hkv = gk;
+            ap.hq_off = h0;
+            ap.hk_off = h0 / kvg;
+            ap.epi = EPI_MERGE;
+            ap.acc_o = P->acc_o;
+            ap.acc_lse = P->acc_lse;
+            ap.acc_rows = N;
+            ap.out = P->out_st[0];
+            ap.out_lse = P->lse_st[0];
+            ap.out_rows = N;
+            {
+                LaunchTimer tm(P, s, 0);
+                if (P->dtype == CQSA_BF16)
+                    CK(launch_attn_tc(d, P->mq, P->mk, P->mv, ap, P->res_wl[i].num_units, s));
+                else
+                    CK(launch_attn_simt(d, P->elem, P->pool_q, P->pool_k, P->pool_v, ap, P->res_wl[i].num_units,
+                                        s));
+                tm.stop();
+            }
+            CK(cudaEventRecord(P->ev_launch[i], s));
+            if (L.finish.empty()) continue;
+            // -- D2H of the finished query blocks, consecutive ones together.
+            CK(cudaStreamWaitEvent(P->s_out, P->ev_launch[i], 0));
+            for (size_t j = 0; j < L.finish.size();) {
+                size_t j1 = j + 1;
+                while (j1 < L.finish.size() && L.finish[j1] == L.finish[j1 - 1] + 1) ++j1;
+                const int64_t r0 = L.finish[j] * Bk, r1 = pl.block_end(L.finish[j1 - 1]);
+                CK(copy_rows(ho + ((size_t)r0 * H + h0) * d * e, full_row, P->out_st[0] + (size_t)r0 * grp_row,
+                             grp_row, grp_row, (size_t)(r1 - r0), cudaMemcpyDeviceToHost, P->s_out));
+                CK(cudaMemcpy2DAsync(lse + (size_t)h0 * N + r0, (size_t)N * sizeof(float), P->lse_st[0] + r0,
+                                     (size_t)N * sizeof(float), (size_t)(r1 - r0) * sizeof(float), (size_t)g,
+                                     cudaMemcpyDeviceToHost, P->s_out));
+                j = j1;
+            }
+        }
+        CK(cudaEventRecord(P->ev_comp_end[0], sc[0]));
+        CK(cudaEventRecord(P->ev_comp_end[1], sc[1]));
+        CK(cudaEventRecord(P->ev_out_end, P->s_out));
+    }
+    CK(cudaStreamWaitEvent(stream, P->ev_comp_end[0], 0));
+    CK(cudaStreamWaitEvent(stream, P->ev_comp_end[1], 0));
+    CK(cudaStreamWaitEvent(stream, P->ev_out_end, 0));
+    return CQSA_OK;
+}
+
 cqsa_status_t forward_host(cqsa_plan_t *P, const void *q, const void *k, const void *v, void *out, float *lse,
                            cudaStream_t stream) {
     cqsa_status_t st = setup_host_mode(P);
     if (st != CQSA_OK) return st;
+    if (P->pl.sizing.resident) return forward_host_resident(P, q, k, v, out, lse, stream);
     const Planner &pl = P->pl;
     const int64_t N = pl.spec.N, R = pl.max_task_rows, B = pl.block;
     const int H = pl.spec.H, d = pl.spec.d, g = P->g;
@@ -945,6 +1134,10 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
     cudaStreamWaitEvent(stream, P->ev_start, 0);
     cudaStreamWaitEvent(stream, P->ev_done_comp, 0);
     cudaStreamWaitEvent(stream, P->ev_done_out, 0);
+    if (P->s_comp2 && P->ev_comp_end[1]) {
+        cudaEventRecord(P->ev_comp_end[1], P->s_comp2);
+        cudaStreamWaitEvent(stream, P->ev_comp_end[1], 0);
+    }
 }
 
 // ------------------------------------------------------------ owner exchange
@@ -1032,7 +1225,7 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
                                      "(needs %lld block slots)", pl.spec.budget, (long long)pl.bwd_min_slots);
     // The streamed forward's arena and this one may not both fit the budget.
     if (P->host_arena && pl.spec.budget && P->host_bytes + z.arena > pl.spec.budget) {
-        cudaStream_t ss[3] = {P->s_in, P->s_comp, P->s_out};
+        cudaStream_t ss[4] = {P->s_in, P->s_comp, P->s_comp2, P->s_out};
         for (cudaStream_t st : ss)
             if (st) CK(cudaStreamSynchronize(st));
         release_host_mode(P);
@@ -1395,6 +1588,7 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out) {
     if (desc->merge != CQSA_MERGE_SLOTS && desc->merge != CQSA_MERGE_FUSED)
         return fail(CQSA_ERR_INVALID_ARG, "merge must be CQSA_MERGE_SLOTS or CQSA_MERGE_FUSED");
     s.fused = desc->merge == CQSA_MERGE_FUSED;
+    s.host_tasks = desc->host_tasks ? 1 : 0;
     cqsa_plan_t *P = nullptr;
     cqsa_status_t st = build_plan(s, desc->dtype, &P);
     if (st != CQSA_OK) return st;
@@ -1846,6 +2040,38 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->bwd_d2h_bytes = pl.bwd_sizing.d2h;
     info->bwd_spill_host_bytes = pl.bwd_sizing.spill_host;
     info->bwd_writebacks = pl.bwd_cache.writebacks;
+    info->host_resident = pl.sizing.resident ? 1 : 0;
+    info->host_launches = (int64_t)pl.host_sched.size();
+    info->arrival_blocks = pl.arrival_blocks();
+    return CQSA_OK;
+}
+
+cqsa_status_t cqsa_plan_host_launch(const cqsa_plan_t *plan, int64_t i, int64_t *need, int32_t *stream,
+                                    int32_t *after, int64_t *pairs, int32_t *flags, int64_t max_pairs,
+                                    int64_t *num_pairs) {
+    if (!plan || !num_pairs) return fail(CQSA_ERR_INVALID_ARG, "null argument");
+    const Planner &pl = plan->pl;
+    if (i < 0 || i >= (int64_t)pl.host_sched.size())
+        return fail(CQSA_ERR_INVALID_ARG, "launch %lld out of range (%zu launches)", (long long)i, pl.host_sched.size());
+    const HostLaunch &L = pl.host_sched[i];
+    if (need) *need = L.need;
+    if (stream) *stream = L.stream;
+    if (after) *after = L.after;
+    int64_t n = 0;
+    for (const WlEntry &e : L.wl.entries)
+        for (int32_t r = 0; r < e.run_count; ++r) {
+            const WlRun &x = L.wl.runs[e.run_begin + r];
+            for (int64_t kb = x.k_lo / pl.block; kb * pl.block < x.k_hi; ++kb) {
+                if (pairs || flags) {
+                    if (!pairs || !flags || n >= max_pairs) return fail(CQSA_ERR_INVALID_ARG, "pair arrays too small");
+                    pairs[2 * n] = e.q_lo / pl.block;
+                    pairs[2 * n + 1] = kb;
+                    flags[n] = e.flags;
+                }
+                ++n;
+            }
+        }
+    *num_pairs = n;
     return CQSA_OK;
 }
 
@@ -1972,28 +2198,17 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
     if (!plan) return;
     if (plan->device >= 0) {
         release_bwd_host(plan);
-        cudaStream_t ss[3] = {plan->s_in, plan->s_comp, plan->s_out};
+        cudaStream_t ss[4] = {plan->s_in, plan->s_comp, plan->s_comp2, plan->s_out};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);
         if (plan->dev_arena || plan->bwd.arena || plan->bwd_shard.arena || plan->part_arena) cudaDeviceSynchronize();
-        for (int s = 0; s < 2; ++s) {
-            if (plan->ev_in_ready[s]) cudaEventDestroy(plan->ev_in_ready[s]);
-            if (plan->ev_in_free[s]) cudaEventDestroy(plan->ev_in_free[s]);
-            if (plan->ev_merged[s]) cudaEventDestroy(plan->ev_merged[s]);
-            if (plan->ev_out_free[s]) cudaEventDestroy(plan->ev_out_free[s]);
-        }
         for (const auto &t : plan->pending) {
             cudaEventDestroy(t.a);
             cudaEventDestroy(t.b);
         }
         for (cudaEvent_t e : plan->spare) cudaEventDestroy(e);
-        if (plan->ev_start) cudaEventDestroy(plan->ev_start);
-        if (plan->ev_done_comp) cudaEventDestroy(plan->ev_done_comp);
-        if (plan->ev_done_out) cudaEventDestroy(plan->ev_done_out);
-        for (cudaStream_t s : ss)
-            if (s) cudaStreamDestroy(s);
+        release_host_mode(plan);  // its events, streams and arena
         if (plan->dev_arena) cudaFree(plan->dev_arena);
-        if (plan->host_arena) cudaFree(plan->host_arena);
         if (plan->bwd.arena) cudaFree(plan->bwd.arena);
         if (plan->bwd_shard.arena) cudaFree(plan->bwd_shard.arena);
         if (plan->part_arena) cudaFree(plan->part_arena);

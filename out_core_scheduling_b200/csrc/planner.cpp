@@ -740,8 +740,120 @@ size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
     return a.total;
 }
 
+// ---------------------------------------------------------------------------
+// Resident schedule of the streamed forward (see planner.h, HostLaunch).
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int64_t kArrivalGroups = 16;  // copy-in marks per head group (fewer when there are fewer blocks)
+}
+
+int64_t Planner::arrival_blocks() const {
+    return std::max<int64_t>(1, (num_blocks + kArrivalGroups - 1) / kArrivalGroups);
+}
+
+std::vector<HostLaunch> Planner::host_launches(int rows_per_unit, int bn, int heads) const {
+    const int64_t A = arrival_blocks();
+    const int64_t G = (num_blocks + A - 1) / A;
+    // Pairs needing one of the last quarter of the arrival groups are taken
+    // query group by query group (the finishing phase).
+    const int64_t cut = G - (G + 3) / 4;
+    // Launch slots in order: for k < cut, [2k] = earlier query groups x keys
+    // of group k, [2k + 1] = query group k x keys of groups <= k; then
+    // [2 cut + j] = query group j's pairs of the finishing phase.  Per slot
+    // and query block, the key blocks as inclusive intervals.
+    const int64_t slots = 2 * cut + G;
+    using Runs = std::vector<std::pair<int64_t, int64_t>>;
+    std::vector<std::map<int64_t, Runs>> pairs(slots);
+    for (const Entry &e : entries) {
+        const int64_t gq = e.qb / A;
+        for (const KeyRun &r : e.runs)
+            for (int64_t b0 = r.b0; b0 <= r.b1;) {
+                // the part of the run inside one arrival group
+                const int64_t gk = b0 / A, b1 = std::min(r.b1, (gk + 1) * A - 1), w = std::max(gq, gk);
+                const int64_t slot = w < cut ? 2 * w + (gq == w ? 1 : 0) : 2 * cut + gq;
+                pairs[slot][e.qb].push_back({b0, b1});
+                b0 = b1 + 1;
+            }
+    }
+    std::vector<HostLaunch> out;
+    std::vector<int64_t> last(num_blocks, -1);  // latest launch that touched a query block
+    std::vector<std::pair<int64_t, int32_t>> last_entry(num_blocks, {-1, -1});  // (launch, entry)
+    for (int64_t sl = 0; sl < slots; ++sl) {
+        if (pairs[sl].empty()) continue;
+        HostLaunch L;
+        L.stream = (int32_t)(out.size() & 1);
+        for (auto &qk : pairs[sl]) {
+            const int64_t qb = qk.first;
+            Runs &kr = qk.second;
+            std::sort(kr.begin(), kr.end());
+            const int64_t prev = last[qb];
+            if (prev >= 0 && out[prev].stream != L.stream) L.after = std::max<int32_t>(L.after, (int32_t)prev);
+            WlEntry w{};
+            w.q_lo = (int32_t)(qb * block);
+            w.q_hi = (int32_t)block_end(qb);
+            w.q_goff = 0;
+            w.slot = 0;
+            w.out_lo = w.q_lo;
+            w.flags = prev < 0 ? SEG_FIRST : 0;
+            w.run_begin = (int32_t)L.wl.runs.size();
+            L.need = std::max(L.need, qb);
+            for (size_t i = 0; i < kr.size(); ++i) {
+                L.need = std::max(L.need, kr[i].second);
+                if (i > 0 && kr[i].first == kr[i - 1].second + 1) {
+                    L.wl.runs.back().k_hi = (int32_t)block_end(kr[i].second);
+                } else {
+                    WlRun x{};
+                    x.k_lo = (int32_t)(kr[i].first * block);
+                    x.k_hi = (int32_t)block_end(kr[i].second);
+                    L.wl.runs.push_back(x);
+                }
+            }
+            w.run_count = (int32_t)L.wl.runs.size() - w.run_begin;
+            last[qb] = (int64_t)out.size();
+            last_entry[qb] = {(int64_t)out.size(), (int32_t)L.wl.entries.size()};
+            L.wl.entries.push_back(w);
+        }
+        out.push_back(std::move(L));
+    }
+    // The last launch of each query block finishes it; units once the flags
+    // are final.
+    for (int64_t qb = 0; qb < num_blocks; ++qb) {
+        if (last_entry[qb].first < 0) continue;
+        HostLaunch &L = out[last_entry[qb].first];
+        L.wl.entries[last_entry[qb].second].flags |= SEG_LAST;
+        L.finish.push_back(qb);
+    }
+    for (HostLaunch &L : out) {
+        std::vector<int64_t> group;
+        for (const WlEntry &e : L.wl.entries) group.push_back(e.q_lo / block);
+        add_units(&L.wl, heads, rows_per_unit, bn, spec.causal, group);
+    }
+    return out;
+}
+
+size_t Planner::resident_arena_bytes(int g, std::vector<HostLaunch> *launches) const {
+    const int64_t N = spec.N, rows = num_blocks * block;
+    const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
+    const size_t gk = (size_t)spec.kv_heads_of(g);
+    ArenaLayout a;
+    a.take(256);                                        // error word
+    a.take((size_t)N * g * dd * sizeof(float));         // accumulator O
+    a.take((size_t)g * N * sizeof(float));              // accumulator lse
+    a.take((size_t)rows * g * dd * e);                  // Q pool, one slot per block
+    a.take((size_t)rows * gk * dd * e);                 // K pool
+    a.take((size_t)rows * gk * dd * e);                 // V pool
+    a.take((size_t)N * g * dd * e);                     // finished out rows
+    a.take((size_t)g * N * sizeof(float));              // finished lse rows
+    launches->clear();
+    if (spec.budget && a.total > spec.budget) return a.total;  // does not fit: no need for the launches
+    *launches = host_launches(unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
+    for (const HostLaunch &L : *launches) a.take(wl_bytes(L.wl));
+    return a.total;
+}
+
 void Planner::size_plan() {
     sizing = Sizing{};
+    host_sched.clear();
     sizing.device_arena = device_arena_bytes();
     // Smallest and largest useful pools (a task and its predecessor must fit).
     std::vector<std::vector<int64_t>> nq, nkv;
@@ -765,7 +877,29 @@ void Planner::size_plan() {
     span(nkv, &min_kv_slots, &full_kv_slots);
 
     const int kvg = spec.kv_group();
-    for (int g = spec.H; g >= 1; --g) {
+    // The resident schedule at the largest head group whose arena fits
+    // (every block of the group on the device: each crosses the host link
+    // once per group, and the copies overlap the launches pair by pair).
+    for (int g = spec.H; g >= 1 && !spec.host_tasks; --g) {
+        if (spec.H % g || (g % kvg != 0 && kvg % g != 0)) continue;
+        std::vector<HostLaunch> sched;
+        const size_t rb = resident_arena_bytes(g, &sched);
+        PoolPlan pp;
+        if ((spec.budget && rb > spec.budget) || !plan_pool(full_q_slots, full_kv_slots, &pp)) continue;
+        const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
+        const size_t blk_kv = (size_t)block * spec.kv_heads_of(g) * spec.d * spec.elem_bytes;
+        int64_t nb_rows = 0;
+        for (int64_t b = 0; b < num_blocks; ++b) nb_rows += block_rows(b) > 0;
+        host_sched = std::move(sched);
+        sizing.head_group = g;
+        sizing.host_arena = rb;
+        sizing.q_slots = sizing.kv_slots = num_blocks;
+        sizing.resident = true;
+        sizing.h2d = (size_t)nb_rows * (blk + 2 * blk_kv) * (size_t)(spec.H / g);
+        pool = std::move(pp);
+        break;
+    }
+    for (int g = spec.H; g >= 1 && !sizing.resident; --g) {
         if (spec.H % g) continue;
         // A head group covers whole key/value groups, or lies inside one.
         if (g % kvg != 0 && kvg % g != 0) continue;

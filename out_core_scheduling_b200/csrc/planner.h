@@ -67,6 +67,7 @@ struct PlanSpec {
     int Hkv = 0;                            // key/value heads (grouped-query attention); 0 = H
     int B = 1;                              // independent sequences of N tokens per call
     int shard_rank = 0, shard_count = 1;    // task sharding over processes
+    int host_tasks = 0;                     // streamed forward: task by task even when every block fits
     int kv_group() const { return H / (Hkv > 0 ? Hkv : H); }
     // Key/value heads a streamed head group of g query heads reads.
     int kv_heads_of(int g) const { return g >= kv_group() ? g / kv_group() : 1; }
@@ -157,6 +158,33 @@ struct Sizing {
     size_t device_arena = 0;
     size_t h2d = 0, d2h = 0;
     int64_t q_slots = 0, kv_slots = 0;
+    bool resident = false;  // the streamed forward runs the resident schedule (HostLaunch)
+};
+
+// Streamed forward when the device holds every block of a head group at
+// once (the resident schedule).  The blocks are copied in increasing order,
+// block b to pool rows [b * block, ...), and the copy stream marks each
+// arrival group of consecutive blocks.  A launch takes the plan's (query
+// block, key block) pairs whose blocks have arrived: one entry per query
+// block with the union of those pairs' key blocks as maximal runs, folded
+// into the block's running accumulator by the epilogue merge; the launch
+// that takes a query block's last pairs writes its finished rows.  Every
+// pair of every entry of the plan is taken exactly once.  While blocks
+// arrive, launch pairs come in two kinds per arrival group k: the new
+// query blocks of group k against keys of groups <= k, and the query
+// blocks of earlier groups against the keys of group k.  Pairs that need
+// one of the last arrival groups are taken query group by query group, so
+// that finished rows go to the host while the rest still computes.
+// Launches alternate between two compute streams; a launch waits for the
+// latest launch on the other stream that touched one of its query blocks
+// (launches on one stream run in order), so the merges of a query block
+// happen in launch order and launches of disjoint query blocks overlap.
+struct HostLaunch {
+    WorkList wl;                  // global rows (slot b holds block b)
+    int64_t need = 0;             // last block it reads
+    int32_t stream = 0;           // compute stream 0 or 1
+    int32_t after = -1;           // launch on the other stream it waits for (-1: none)
+    std::vector<int64_t> finish;  // query blocks whose rows it finishes, increasing
 };
 
 class Planner {
@@ -270,6 +298,12 @@ public:
     // Arena bytes of each mode for a head group g (host) / all heads (device).
     size_t host_arena_bytes(int g, const PoolPlan &pool) const;
     size_t device_arena_bytes() const;
+    // The resident schedule (see HostLaunch): blocks per arrival group, the
+    // launches, and its arena for a head group g.
+    int64_t arrival_blocks() const;
+    std::vector<HostLaunch> host_launches(int rows_per_unit, int bn, int heads) const;
+    size_t resident_arena_bytes(int g, std::vector<HostLaunch> *launches) const;
+    std::vector<HostLaunch> host_sched;  // the chosen resident schedule (empty: task by task)
 
 private:
     std::vector<int64_t> entry_begin_of_leaf_;  // first entry index of each leaf

@@ -93,18 +93,61 @@ def test_repeated_forward_is_deterministic():
 
 
 # ---------------------------------------------------------------- streamed
+@pytest.mark.parametrize("tasks", [False, True], ids=["resident", "tasks"])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_streamed_head_groups(causal, dtype):
+def test_streamed_head_groups(causal, dtype, tasks):
     """Host-resident inputs under a budget that forces head groups < H."""
     N, H, d = 7 * 256, 4, 128
     q, k, v = _inputs(N, H, d, dtype, seed=7, host=True)
     dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
-    full = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt).info()["host_arena_bytes"]
-    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt, mem_budget_bytes=full // 2)
-    assert plan.info()["head_group"] < H
+    full = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt, host_tasks=tasks).info()["host_arena_bytes"]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=causal, dtype=dt, mem_budget_bytes=full // 2, host_tasks=tasks)
+    info = plan.info()
+    assert info["head_group"] < H and info["host_resident"] == (not tasks)
     out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
     check(out, lse, q, k, v, np.arange(N), causal)
+
+
+SCHEDULE_CASES = [
+    # (N, H, d, levels, dtype)
+    (7 * 256, 2, 128, [3], torch.bfloat16),
+    (13 * 256, 2, 64, [4], torch.bfloat16),
+    (7 * 100 + 3, 2, 128, [3], torch.bfloat16),   # ragged: a short last block
+    (31 * 64, 1, 128, [6], torch.bfloat16),       # arrival groups of two blocks
+    (49 * 64, 2, 128, [3, 3], torch.bfloat16),    # two levels, arrival groups of four
+    (7 * 128, 2, 64, [3], torch.float32),
+    (13 * 128, 1, 128, [4], torch.float32),
+]
+
+
+@pytest.mark.parametrize("tasks", [False, True], ids=["resident", "tasks"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", SCHEDULE_CASES, ids=lambda c: f"n{c[0]}-h{c[1]}-d{c[2]}-l{c[3]}-{str(c[4])[6:]}")
+def test_streamed_schedules_every_row(case, causal, tasks):
+    """Both schedules of the streamed forward (every block on the device at
+    once, and task by task) on every row."""
+    N, H, d, ls, dtype = case
+    dt = cqsa.CQSA_BF16 if dtype == torch.bfloat16 else cqsa.CQSA_FP32
+    q, k, v = _inputs(N, H, d, dtype, seed=30, host=True)
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dt, host_tasks=tasks)
+    assert plan.info()["host_resident"] == (not tasks)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_resident_repeat_is_deterministic(causal):
+    """The resident schedule's two compute streams never share a query
+    block, so the merge order, and the result, are fixed."""
+    N, H, d = 13 * 256, 2, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=31, host=True)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal)
+    assert plan.info()["host_resident"] == 1
+    a, la = run(plan, q, k, v, cqsa.CQSA_HOST)
+    for _ in range(3):
+        b, lb = run(plan, q, k, v, cqsa.CQSA_HOST)
+        assert torch.equal(a, b) and torch.equal(la, lb)
 
 
 @pytest.mark.parametrize("causal", [False, True])

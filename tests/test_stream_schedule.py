@@ -89,7 +89,9 @@ CASES = [
 @pytest.mark.parametrize("N,H,d,ls,causal,f", CASES)
 def test_streamed_schedule_is_race_free(N, H, d, ls, causal, f):
     budget = 0 if f is None else int(_min_budget(N, H, d, ls, causal) * f)
-    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, mem_budget_bytes=budget)
+    # Unlimited: every block fits, which runs task by task only on request.
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, mem_budget_bytes=budget, host_tasks=f is None)
+    assert plan.info()["host_resident"] == 0
     groups = min(2, H // plan.info()["head_group"])
     assert bm.explore(*streamed_model(plan, groups))
 
