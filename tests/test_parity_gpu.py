@@ -421,17 +421,18 @@ def test_injected_allocation_failure_is_recoverable():
     check(out, lse, q, k, v, np.arange(N), True)
 
 
-@pytest.mark.parametrize("mode,nth", [("device", 1), ("device", 2), ("host", 1), ("host", 5),
-                                      ("backward", 1), ("backward", 3)])
+@pytest.mark.parametrize("mode,nth", [("device", 1), ("device", 2), ("host", 1), ("host", 5), ("resident", 1),
+                                      ("resident", 9), ("backward", 1), ("backward", 3)])
 def test_injected_setup_failure_is_recoverable(mode, nth):
     """An upload of the plan's tables fails after its arena was allocated:
     the call reports CQSA_ERR_CUDA, the half-built arena is released, and
     the next call sets it up again and is correct."""
     N, H, d = 13 * 256, 2, 128
-    host = mode == "host"
+    host = mode in ("host", "resident")
     q, k, v = _inputs(N, H, d, torch.bfloat16, seed=62, host=host)
-    budget = int(_min_budget(N, H, d, [4], True) * 1.3) if host else 0
+    budget = int(_min_budget(N, H, d, [4], True) * 1.3) if mode == "host" else 0
     plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True, mem_budget_bytes=budget)
+    assert plan.info()["host_resident"] == (mode == "resident") or not host
     m = cqsa.CQSA_HOST if host else cqsa.CQSA_DEVICE
     if mode == "backward":
         out, lse = run(plan, q, k, v, m)
@@ -464,14 +465,17 @@ def test_injected_setup_failure_is_recoverable(mode, nth):
         check(out, lse, q, k, v, np.arange(N), True)
 
 
+@pytest.mark.parametrize("resident", [False, True], ids=["tasks", "resident"])
 @pytest.mark.parametrize("nth", [1, 7, 40])
-def test_injected_copy_failure_is_recoverable(nth):
+def test_injected_copy_failure_is_recoverable(nth, resident):
     """A host<->device copy of a streamed forward fails part-way: the call
     reports CQSA_ERR_CUDA, the work already enqueued completes, and the next
     forward on the same plan is correct."""
     N, H, d = 13 * 256, 2, 128
     q, k, v = _inputs(N, H, d, torch.bfloat16, seed=61, host=True)
-    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=False, mem_budget_bytes=int(_min_budget(N, H, d, [4], False) * 1.3))
+    budget = 0 if resident else int(_min_budget(N, H, d, [4], False) * 1.3)
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=False, mem_budget_bytes=budget)
+    assert plan.info()["host_resident"] == resident
     out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     lse = torch.empty(H, N).pin_memory()
     cqsa.cqsa_debug_inject(cqsa.CQSA_FAULT_COPY, nth)
