@@ -69,9 +69,10 @@ enum { CQSA_DEVICE = 0, CQSA_HOST = 1 };
  *   CQSA_MERGE_SLOTS: every (task, query block) writes its partial O_j and
  *     lse_j to a slot; a merge kernel then takes the log-sum-exp over the
  *     slots.  The tasks' results are materialised as the pages describe.
- *     At most 32 partials per query block (the merge takes one lane per
- *     partial): deeper plans (e.g. levels 4, 3, 3: 36) report
- *     CQSA_ERR_UNSUPPORTED from cqsa_forward and need CQSA_MERGE_FUSED.
+ *     Up to 1024 partials per query block (levels 4, 3, 3 give 36; the
+ *     merge stages a tile's lse values and weights in shared memory, with
+ *     fewer rows per tile as the partials grow); beyond that cqsa_forward
+ *     reports CQSA_ERR_UNSUPPORTED and the plan needs CQSA_MERGE_FUSED.
  *   CQSA_MERGE_FUSED: one CTA walks the allowed key blocks of all the tasks
  *     of its query rows; its online softmax is the merge, and it writes the
  *     output directly (no slots, no merge launch).
@@ -516,7 +517,7 @@ cqsa_status_t cqsa_plan_kernel_stats(cqsa_plan_t *plan, cqsa_kernel_stats_t *sta
  *   and work list must fit the array; otherwise CQSA_ERR_BUDGET with the
  *   sizes in the message, and cqsa_forward is the way.  A CQSA_MERGE_FUSED
  *   plan runs as a slots plan here (partials in the array, then the merge),
- *   so plans with more than 32 partials per query block are refused with
+ *   so plans with more than 1024 partials per query block are refused with
  *   CQSA_ERR_UNSUPPORTED, as are batched (B > 1), grouped-query and sharded
  *   plans.
  *   Calls share the array and keep the last call's contents; host callers

@@ -356,7 +356,9 @@ cqsa_status_t setup_device_mode_impl(cqsa_plan_t *P) {
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
     const bool fused = pl.spec.fused != 0;
-    if (!fused && pl.max_slots > 32) return fail(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
+    if (!fused && pl.max_slots > 1024)
+        return fail(CQSA_ERR_UNSUPPORTED, "%lld partials per query block (the merge takes 1024)",
+                    (long long)pl.max_slots);
     WorkList wl = pl.device_worklist(unit_rows_for(P->elem), key_tile_for(P->elem), H);
     ArenaLayout a;
     const size_t o_err = a.take(256);

@@ -12,7 +12,8 @@
 //
 // HBM-bound.  The slots of one partial are laid out [S][N][H][D], so for a
 // fixed slot consecutive (row, head) pairs are one contiguous stream.  A CTA
-// takes a tile of 128 consecutive pairs: it first stages their partial lse
+// takes a tile of consecutive pairs (128 with up to 32 partials per row,
+// fewer beyond, up to 1024 partials): it first stages their partial lse
 // values in shared memory and turns them into weights (one thread per
 // pair), then streams the tile's float4 chunks, each thread loading two
 // chunks of up to four slots each at once (eight 16-byte loads in flight)
@@ -28,9 +29,25 @@
 namespace cqsa {
 
 // Device mode: partials in slots [S][N][H][D], lse [S][H][N].
-constexpr int kMergePairs = 128;   // (row, head) pairs per tile
+constexpr int kMergePairs = 128;   // (row, head) pairs per tile with at most 32 partials
 constexpr int kMergeThreads = 256;
 constexpr int kMergeGroup = 4;     // slots loaded together per chunk (two chunks per thread at once)
+constexpr int kMergeMaxSlots = 1024;
+
+// Pairs per tile for a plan with up to smax partials per row: 128 up to 32
+// partials, then fewer (a multiple of 8), so the staged lse and weights
+// stay near 33 KB of shared memory.
+__host__ __device__ __forceinline__ int merge_pairs(int smax) {
+    if (smax <= 32) return kMergePairs;
+    const int p = (kMergePairs * 32 / smax) & ~7;
+    return p < 8 ? 8 : p;
+}
+
+__host__ __device__ __forceinline__ size_t merge_smem(int smax) {
+    const int P = merge_pairs(smax);
+    // s_l [smax][P], s_w [P][smax + 1], s_inv [P], s_n [P]
+    return sizeof(float) * ((size_t)smax * P + (size_t)P * (smax + 1) + P) + sizeof(int) * (size_t)P;
+}
 
 __device__ __forceinline__ float4 ld_stream(const float *p) {
     return __ldcs(reinterpret_cast<const float4 *>(p));
@@ -53,11 +70,13 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
                        const int32_t *__restrict__ nslots, int64_t block, int64_t N, int H, int smax,
                        TO *__restrict__ out, float *__restrict__ lse_out) {
     constexpr int CH = D / 4;  // float4 chunks per (row, head)
-    constexpr int P = kMergePairs;
-    __shared__ float s_l[32 * P];   // staged lse_j, [slot][pair]
-    __shared__ float s_w[P * 33];   // weights exp(lse_j - M), [pair][slot] (padded)
-    __shared__ float s_inv[P];      // 1 / sum of the weights
-    __shared__ int s_n[P];          // partials of the pair's row
+    const int P = merge_pairs(smax);
+    const int WS = smax + 1;   // padded row of the weights
+    extern __shared__ __align__(16) float smerge[];
+    float *s_l = smerge;                      // staged lse_j, [slot][pair]
+    float *s_w = s_l + (size_t)smax * P;      // weights exp(lse_j - M), [pair][slot]
+    float *s_inv = s_w + (size_t)P * WS;      // 1 / sum of the weights
+    int *s_n = reinterpret_cast<int *>(s_inv + P);  // partials of the pair's row
     const int tid = threadIdx.x;
     const int64_t total = N * H;
     const int64_t slot_stride = N * H * D;
@@ -91,7 +110,7 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
                 for (int j = 0; j < n; ++j) {
                     const float lj = s_l[j * P + tid];
                     const float wj = lj != -INFINITY ? __expf(lj - M) : 0.f;
-                    s_w[tid * 33 + j] = wj;
+                    s_w[tid * WS + j] = wj;
                     W += wj;
                 }
                 s_inv[tid] = W > 0.f ? 1.f / W : 0.f;
@@ -131,7 +150,7 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
 #pragma unroll
                     for (int u = 0; u < kMergeGroup; ++u) {
                         if (j0 + u < n[i]) {
-                            const float w = s_w[p[i] * 33 + j0 + u];
+                            const float w = s_w[p[i] * WS + j0 + u];
                             if (w != 0.f) {
                                 acc[i].x = fmaf(w, x[i][u].x, acc[i].x);
                                 acc[i].y = fmaf(w, x[i][u].y, acc[i].y);
@@ -157,18 +176,21 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
 }
 
 // Persistent grid: as many CTAs as fit on the device at once (or one per
-// tile when there are fewer tiles).
+// tile when there are fewer tiles).  Occupancy is looked up once per
+// shared-memory size.
 template <int D, typename TO>
-static int merge_grid(int64_t tiles) {
+static int merge_grid(int64_t tiles, size_t smem) {
+    static size_t cached_smem = 0;
     static int per_sm = 0;  // the same on every device this library runs on (sm_100)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (per_sm < 1) {
+    if (per_sm < 1 || cached_smem != smem) {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_slots_kernel<D, TO>, kMergeThreads, 0) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_slots_kernel<D, TO>, kMergeThreads, smem) !=
             cudaSuccess)
             cudaGetLastError();
         per_sm = n > 0 ? n : 1;
+        cached_smem = smem;
     }
     const int64_t cap = (int64_t)sms * per_sm;
     return (int)(tiles < cap ? (tiles > 0 ? tiles : 1) : cap);
@@ -177,16 +199,22 @@ static int merge_grid(int64_t tiles) {
 template <int D, typename TO>
 static cudaError_t merge_slots_t(const float *po, const float *pl, const int32_t *ns, int64_t block, int64_t N,
                                  int H, int smax, void *out, float *lse, cudaStream_t st) {
-    const int64_t tiles = (N * H + kMergePairs - 1) / kMergePairs;
-    merge_slots_kernel<D, TO><<<merge_grid<D, TO>(tiles), kMergeThreads, 0, st>>>(po, pl, ns, block, N, H, smax,
-                                                                                   static_cast<TO *>(out), lse);
+    const size_t smem = merge_smem(smax);
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(merge_slots_kernel<D, TO>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t tiles = (N * H + merge_pairs(smax) - 1) / merge_pairs(smax);
+    merge_slots_kernel<D, TO><<<merge_grid<D, TO>(tiles, smem), kMergeThreads, smem, st>>>(
+        po, pl, ns, block, N, H, smax, static_cast<TO *>(out), lse);
     return cudaGetLastError();
 }
 
 cudaError_t launch_merge_slots(int d, int elem_bytes, const float *part_o, const float *part_lse,
                                const int32_t *nslots, int64_t block, int64_t N, int H, int max_slots, void *out,
                                float *lse, cudaStream_t stream) {
-    if (max_slots < 1 || max_slots > 32) return cudaErrorInvalidValue;
+    if (max_slots < 1 || max_slots > kMergeMaxSlots) return cudaErrorInvalidValue;
     // Each thread stores four consecutive outputs at once, and reads float4s.
     if ((reinterpret_cast<uintptr_t>(out) & (uintptr_t)(4 * elem_bytes - 1)) ||
         (reinterpret_cast<uintptr_t>(part_o) & 15u))

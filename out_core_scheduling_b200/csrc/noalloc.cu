@@ -27,8 +27,8 @@
 //     with CQSA_ERR_BUDGET; nothing in this file calls cudaMalloc, cudaFree
 //     or any allocating routine.
 //   * A CQSA_MERGE_FUSED plan runs here as a slots plan (partials in the
-//     array, then the merge kernel), so a plan with more than 32 partials
-//     per query block is rejected with CQSA_ERR_UNSUPPORTED.
+//     array, then the merge kernel); the merge takes up to 1024 partials
+//     per query block (CQSA_ERR_UNSUPPORTED beyond).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -192,7 +192,7 @@ extern "C" cqsa_status_t cqsa_forward_noalloc(cqsa_plan_t *plan, const void *q, 
     const int64_t N = pl.spec.N;
     const int H = pl.spec.H, d = pl.spec.d;
     const int rows = unit_rows_for(elem), bn = key_tile_for(elem);
-    if (pl.max_slots > 32) return err(CQSA_ERR_UNSUPPORTED, "more than 32 partials per query block");
+    if (pl.max_slots > 1024) return err(CQSA_ERR_UNSUPPORTED, "more than 1024 partials per query block");
     if (pl.spec.B != 1) return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes one sequence (B = 1)");
     if (pl.spec.shard_count != 1) return err(CQSA_ERR_UNSUPPORTED, "the allocation-free forward takes no sharded plan");
     if (pl.spec.Hkv != pl.spec.H)

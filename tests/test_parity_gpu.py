@@ -552,15 +552,25 @@ def test_forward_and_backward_in_a_cuda_graph(merge):
         assert np.abs(g_dq - ref_dq).max() <= 2e-2 * np.abs(ref_dq).max()
 
 
-def test_more_than_32_partials_need_the_fused_recomposition():
-    """Three levels (4, 3, 3) give each query block 36 partials; the slots
-    merge takes one lane per partial, so a slots-mode forward reports
-    CQSA_ERR_UNSUPPORTED before launching anything."""
-    N, H, d = 637 * 4, 1, 64
-    plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3, 3])
-    assert plan.info()["max_slots"] == 36
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("ls,N,H,d", [([4, 3, 3], 637 * 4, 2, 64), ([4, 3, 3], 637 * 16 + 5, 1, 128),
+                                      ([3, 3, 3, 3], 2401 * 2, 1, 64)],
+                         ids=["l433-n2548", "l433-ragged", "l3333-n4802"])
+def test_more_than_32_partials_slots_merge(ls, N, H, d, causal):
+    """Three and four levels give each query block 36 and 81 partials: the
+    slots merge stages fewer rows per tile, with every row against the
+    oracle, in both dtypes' tile kernels' slot layouts (bf16 here)."""
+    plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal)
+    assert plan.info()["max_slots"] > 32
     q, k, v = _inputs(N, H, d, torch.bfloat16, seed=64)
-    out, lse = torch.empty_like(q), torch.empty(H, N, device=DEV)
-    with pytest.raises(cqsa.CqsaError) as ei:
-        cqsa.cqsa_forward(plan, q, k, v, out, lse, cqsa.CQSA_DEVICE)
-    assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), causal)
+
+
+def test_more_than_32_partials_fp32():
+    N, H, d = 637 * 2, 1, 64
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3, 3], dtype=cqsa.CQSA_FP32)
+    assert plan.info()["max_slots"] == 36
+    q, k, v = _inputs(N, H, d, torch.float32, seed=65)
+    out, lse = run(plan, q, k, v, cqsa.CQSA_DEVICE)
+    check(out, lse, q, k, v, np.arange(N), False)

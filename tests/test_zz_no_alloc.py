@@ -81,16 +81,17 @@ def test_noalloc_rejects_plans_beyond_its_array():
     assert str(64 << 20) in str(ei.value)
 
 
-def test_noalloc_rejects_more_than_32_partials():
-    """Levels 4, 3, 3 give a query block 36 partials; the merge of the
-    allocation-free path takes at most 32, fused plan or not."""
+def test_noalloc_more_than_32_partials():
+    """Levels 4, 3, 3 give a query block 36 partials; the allocation-free
+    path merges them (fused plan or not), every row against the oracle."""
     N, H, d = 13 * 7 * 7 * 2, 1, 64
+    q, k, v = make_qkv(N, H, d, dtype=torch.bfloat16, seed=66, device=DEV)
     for merge in (cqsa.CQSA_MERGE_SLOTS, cqsa.CQSA_MERGE_FUSED):
-        plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3, 3], merge=merge)
+        plan = cqsa.cqsa_plan_ex(N, H, d, [4, 3, 3], merge=merge, causal=True)
         assert plan.info()["max_slots"] > 32
-        x = torch.zeros(N, H, d, device=DEV, dtype=torch.bfloat16)
+        out = torch.empty_like(q)
         lse = torch.empty(H, N, device=DEV, dtype=torch.float32)
-        with pytest.raises(cqsa.CqsaError) as ei:
-            cqsa.cqsa_forward_noalloc(plan, x, x, x, torch.empty_like(x), lse)
-        assert ei.value.status == cqsa.CQSA_ERR_UNSUPPORTED
+        cqsa.cqsa_forward_noalloc(plan, q, k, v, out, lse)
+        torch.cuda.synchronize()
+        check(out, lse, q, k, v, np.arange(N), True)
         plan.destroy()
