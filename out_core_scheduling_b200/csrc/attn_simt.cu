@@ -9,15 +9,16 @@
 //
 // 256 threads as 16 x 16: thread (ty, tx) owns query rows 4ty..4ty+3, keys
 // tx, tx+16, tx+32, tx+48 of each 64-key tile, and output features
-// 64g + 4tx .. 64g + 4tx + 3 (g < d / 64).  Q and P are kept transposed in
-// shared memory ([feature or key][row], rows padded to 68 floats); K and V
-// tiles stay row-major (K rows padded to d + 4 floats, so the eight lanes of
-// a 16-byte load phase hit distinct banks) and arrive by cp.async in two
-// stages: the next tile's copies are in flight while the current tile is
-// computed.  Every product step reads 16-byte vectors: Q^T and K for four
-// features at a time (64 FMAs per eight loads), P^T and V for one key.  Row
-// maxima and sums are reduced over the 16 threads of a row with warp
-// shuffles.
+// 64g + 4tx .. 64g + 4tx + 3 (g < d / 64).  Q and K rows are row-major in
+// shared memory (padded to d + 4 floats, so the eight lanes of a 16-byte
+// load phase hit distinct banks); Q arrives by cp.async with the first K / V
+// tile, and K and V tiles by cp.async in two stages: the next tile's copies
+// are in flight while the current tile is computed.  P is kept transposed
+// ([key][row], rows padded to 68 floats).  The products run on packed f32x2
+// FMAs: S pairs consecutive features of a Q row and a K row (both 16-byte
+// vectors; the two halves of each accumulator are added at the end), O += P V
+// pairs consecutive rows of a P^T vector with one V value.  Row maxima and
+// sums are reduced over the 16 threads of a row with warp shuffles.
 //
 // Key split: a unit may be computed by a cluster of S = 1, 2 or 4 CTAs (the
 // launcher picks S so that small problems still fill every SM): CTA rank r
@@ -39,12 +40,12 @@ namespace simt {
 constexpr int BM = 64;
 constexpr int BN = 64;
 constexpr int THREADS = 256;
-constexpr int LD = 68;  // padded row of the transposed Q and P tiles, in floats
+constexpr int LD = 68;  // padded row of the transposed P tile, in floats
 template <int D>
 struct Layout {
-    static constexpr int KD = D + 4;  // padded K row, in floats
-    static constexpr int Q = 0;
-    static constexpr int K = Q + D * LD;          // two stages of [BN][KD]
+    static constexpr int KD = D + 4;  // padded K and Q rows, in floats
+    static constexpr int Q = 0;                   // [BM][KD], row-major
+    static constexpr int K = Q + BM * KD;         // two stages of [BN][KD]
     static constexpr int V = K + 2 * BN * KD;     // two stages of [BN][D]
     static constexpr int P = V + 2 * BN * D;      // [BN][LD]
     static constexpr int FLOATS = P + BN * LD;
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(simt::THREADS)
     constexpr int G = D / 64;                 // float4 groups of output features per thread
     constexpr int NC = BN * D / 4 / THREADS;  // 16-byte copies per thread per K (or V) tile
     extern __shared__ __align__(16) float smf[];
-    float *Qt = smf + L::Q;     // [D][LD]   Q transposed
+    float *Qs = smf + L::Q;     // [BM][KD]  Q rows
     float *Ks = smf + L::K;     // [2][BN][KD]
     float *Vs = smf + L::V;     // [2][BN][D]
     float *Pt = smf + L::P;     // [BN][LD]  P transposed
@@ -152,33 +153,38 @@ __global__ void __launch_bounds__(simt::THREADS)
         }
         cp_async_commit();
     };
-    if (my_tiles > 0) issue(cw, 0);
-
+    // Q rows by cp.async (zero rows past the entry), in the same group as the
+    // first K / V tile, so the two loads overlap.
 #pragma unroll
     for (int j = 0; j < BM * D / 4 / THREADS; ++j) {
         const int idx = 4 * (tid + j * THREADS);
         const int r = idx / D, c = idx % D;
         const int32_t row = q0 + r;
-        const float4 x =
-            row < q_end ? __ldg(reinterpret_cast<const float4 *>(q + ((int64_t)row * H + h) * D + c))
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        Qt[(c + 0) * LD + r] = x.x;
-        Qt[(c + 1) * LD + r] = x.y;
-        Qt[(c + 2) * LD + r] = x.z;
-        Qt[(c + 3) * LD + r] = x.w;
+        const bool in = row < q_end;
+        cp_async16(Qs + r * KD + c, q + ((int64_t)(in ? row : q0) * H + h) * D + c, in ? 16 : 0);
     }
-    float m[4], l[4], o[4][G][4];
+    if (my_tiles > 0) {
+        issue(cw, 0);
+    } else {
+        cp_async_commit();
+    }
+    float m[4], l[4];
+    // O as row pairs (rows 2 pp, 2 pp + 1 of the thread's four) for the
+    // packed f32x2 FMAs: o2[pp][g][jj] holds feature 64 g + 4 tx + jj.
+    uint64_t o2[2][G][4];
     int64_t qg[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         m[i] = -INFINITY;
         l[i] = 0.f;
         qg[i] = (int64_t)(q0 + ty * 4 + i) + e.q_goff;
+    }
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = 0.f;
-    }
+            for (int jj = 0; jj < 4; ++jj) o2[pp][g][jj] = 0ull;
 
     for (int32_t t = 0; t < my_tiles; ++t) {
         const int stage = t & 1;
@@ -195,27 +201,42 @@ __global__ void __launch_bounds__(simt::THREADS)
         }
         __syncthreads();
         const float *Kc = Ks + stage * BN * KD, *Vc = Vs + stage * BN * D;
+        // S on packed f32x2 FMAs over feature pairs: a Q row vector and a K
+        // row vector hold four consecutive features each, so features (0, 1)
+        // and (2, 3) are register pairs on both sides; the two halves of each
+        // accumulator are added at the end.
+        uint64_t s2[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) s2[i][mm] = 0ull;
+#pragma unroll 2
+        for (int kk = 0; kk < D; kk += 4) {
+            float4 qv[4], kv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4 *>(Qs + (4 * ty + i) * KD + kk);
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) kv[mm] = *reinterpret_cast<const float4 *>(Kc + (tx + 16 * mm) * KD + kk);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint64_t qa = f2_pack(qv[i].x, qv[i].y), qb = f2_pack(qv[i].z, qv[i].w);
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    s2[i][mm] = f2_fma(qa, f2_pack(kv[mm].x, kv[mm].y), s2[i][mm]);
+                    s2[i][mm] = f2_fma(qb, f2_pack(kv[mm].z, kv[mm].w), s2[i][mm]);
+                }
+            }
+        }
         float sacc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int mm = 0; mm < 4; ++mm) sacc[i][mm] = 0.f;
-#pragma unroll 2
-        for (int kk = 0; kk < D; kk += 4) {
-            float qa[4][4], ka[4][4];
-#pragma unroll
-            for (int u4 = 0; u4 < 4; ++u4) f4_split(*reinterpret_cast<const float4 *>(Qt + (kk + u4) * LD + 4 * ty), qa[u4]);
-#pragma unroll
-            for (int mm = 0; mm < 4; ++mm)
-                f4_split(*reinterpret_cast<const float4 *>(Kc + (tx + 16 * mm) * KD + kk), ka[mm]);
-#pragma unroll
-            for (int u4 = 0; u4 < 4; ++u4)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int mm = 0; mm < 4; ++mm) sacc[i][mm] = fmaf(qa[u4][i], ka[mm][u4], sacc[i][mm]);
-        }
-        float pm[4][4];
+            for (int mm = 0; mm < 4; ++mm) {
+                float a, b;
+                f2_unpack(s2[i][mm], a, b);
+                sacc[i][mm] = a + b;
+            }
+        float pm[4][4], alph[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float x[4];
@@ -241,28 +262,40 @@ __global__ void __launch_bounds__(simt::THREADS)
             for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
             l[i] = l[i] * alpha + sum;
             m[i] = m_new;
+            alph[i] = alpha;
+        }
+        {
+            const uint64_t a01 = f2_pack(alph[0], alph[1]), a23 = f2_pack(alph[2], alph[3]);
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) o[i][g][jj] *= alpha;
+                for (int jj = 0; jj < 4; ++jj) {
+                    o2[0][g][jj] = f2_fma(o2[0][g][jj], a01, 0ull);
+                    o2[1][g][jj] = f2_fma(o2[1][g][jj], a23, 0ull);
+                }
         }
 #pragma unroll
         for (int mm = 0; mm < 4; ++mm)
             *reinterpret_cast<float4 *>(Pt + (tx + 16 * mm) * LD + 4 * ty) =
                 make_float4(pm[0][mm], pm[1][mm], pm[2][mm], pm[3][mm]);
         __syncthreads();
+        // O += P V on packed f32x2 FMAs: a P^T vector holds four consecutive
+        // rows of one key, so rows (0, 1) and (2, 3) pair up; each V value is
+        // paired with itself.
 #pragma unroll 4
         for (int c = 0; c < BN; ++c) {
-            float pa[4];
-            f4_split(*reinterpret_cast<const float4 *>(Pt + c * LD + 4 * ty), pa);
+            const float4 pv = *reinterpret_cast<const float4 *>(Pt + c * LD + 4 * ty);
+            const uint64_t p01 = f2_pack(pv.x, pv.y), p23 = f2_pack(pv.z, pv.w);
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float va[4];
-                f4_split(*reinterpret_cast<const float4 *>(Vc + c * D + 64 * g + 4 * tx), va);
+                const float4 vv = *reinterpret_cast<const float4 *>(Vc + c * D + 64 * g + 4 * tx);
+                const float va[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = fmaf(pa[i], va[jj], o[i][g][jj]);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint64_t v2 = f2_pack(va[jj], va[jj]);
+                    o2[0][g][jj] = f2_fma(p01, v2, o2[0][g][jj]);
+                    o2[1][g][jj] = f2_fma(p23, v2, o2[1][g][jj]);
+                }
             }
         }
         // Everyone is done with this stage and with P before the next tile
@@ -271,6 +304,16 @@ __global__ void __launch_bounds__(simt::THREADS)
         xw = cw;
     }
 
+    // A CTA without key tiles still has its Q copy in flight.
+    cp_async_wait<0>();
+    float o[4][G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            f2_unpack(o2[0][g][jj], o[0][g][jj], o[1][g][jj]);
+            f2_unpack(o2[1][g][jj], o[2][g][jj], o[3][g][jj]);
+        }
     if (S > 1) {
         // Combine the cluster's states: ranks >= 1 leave (m, l, O) in their
         // own shared memory, element-major so that a warp's reads are
