@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <map>
 #include <numeric>
+#include <queue>
 #include <unordered_map>
 
 namespace cqsa {
@@ -193,6 +194,7 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     max_slots = 0;
     for (int32_t v : slots_per_block) max_slots = std::max<int64_t>(max_slots, v);
     assign_shards();
+    count_leaves();
     size_plan();
     size_bwd();
     const char *dbg = getenv("CQSA_DEBUG");
@@ -207,6 +209,8 @@ std::string Planner::build(const PlanSpec &s, int *code) {
     *code = 0;
     return "";
 }
+
+static size_t wl_bytes(const WorkList &wl);
 
 std::string Planner::verify() const {
     const int64_t P = num_blocks;
@@ -223,6 +227,22 @@ std::string Planner::verify() const {
     }
     for (int64_t b = 0; b < P; ++b)
         if (seen_slots[b] != slots_per_block[b]) return "slot count mismatch";
+    // The counted work-list sizes of the sizing loops equal the built lists'.
+    if (sizing.head_group > 0 && !sizing.resident)
+        for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+            const int rpu = unit_rows_for(spec.elem_bytes);
+            if (leaf_wl_bytes(t, pool, rpu, sizing.head_group) !=
+                wl_bytes(leaf_worklist(t, pool, rpu, key_tile_for(spec.elem_bytes), sizing.head_group)))
+                return "counted streamed work-list size differs from the built list";
+        }
+    if (bwd_sizing.head_group > 0)
+        for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+            const int tile = spec.elem_bytes == 2 ? 128 : 64, g = bwd_sizing.head_group;
+            if (leaf_bwd_wl_bytes(t, bwd_cache, tile, g) !=
+                wl_bytes(leaf_bwd_q_worklist(t, bwd_cache, tile, tile, g)) +
+                    wl_bytes(leaf_bwd_kv_worklist(t, bwd_cache, tile, tile, g)))
+                return "counted backward work-list size differs from the built lists";
+        }
     // Exactly-once coverage of the allowed block pairs.
     if (P <= 4096) {
         std::vector<uint8_t> hits((size_t)P * P, 0);
@@ -607,44 +627,67 @@ void task_needs(const Planner &pl, std::vector<std::vector<int64_t>> *nq, std::v
 
 // One cache of `cap` slots over the task sequence; fills slot_of[t][block]
 // and the copies.  False when a task and its predecessor need more than cap.
+// A miss takes the lowest slot never used, else evicts, among the slots
+// whose block neither this task nor the previous one needs, the block used
+// again farthest ahead (the lowest slot on a tie).  The candidates sit in a
+// max-heap keyed by (next use, -slot), kept lazily: an entry counts only
+// while its slot still holds a block with that key and is unprotected; a
+// protected slot rejoins the heap when its protection ends.
 bool simulate(const std::vector<std::vector<int64_t>> &need, int64_t cap, int kind,
               std::vector<std::unordered_map<int64_t, int32_t>> *slot_of, std::vector<std::vector<PoolCopy>> *copies,
               int64_t *ncopies) {
     const size_t T = need.size();
-    std::map<int64_t, std::vector<int64_t>> uses;  // block -> tasks using it, increasing
+    std::unordered_map<int64_t, std::vector<int64_t>> uses;  // block -> tasks using it, increasing
     for (size_t t = 0; t < T; ++t)
-        for (int64_t b : need[t]) uses[b].push_back((int64_t)t);
+        for (int64_t b : need[t]) {
+            std::vector<int64_t> &u = uses[b];
+            if (u.empty() || u.back() != (int64_t)t) u.push_back((int64_t)t);
+        }
     auto next_use = [&](int64_t b, int64_t t) -> int64_t {
         const std::vector<int64_t> &u = uses[b];
         auto it = std::upper_bound(u.begin(), u.end(), t);
         return it == u.end() ? INT64_MAX : *it;
     };
-    std::vector<int64_t> slot_block(cap, -1);
+    std::vector<int64_t> slot_block(cap, -1), key(cap, -1), guard(cap, -1);  // guard: protected through this task
     std::unordered_map<int64_t, int32_t> where;
+    std::priority_queue<std::pair<int64_t, int64_t>> heap;  // (next use, -slot)
+    std::vector<std::vector<int32_t>> rejoin(T + 2);       // slots whose protection ends before task t
+    int64_t next_free = 0;
     slot_of->assign(T, {});
+    auto protect = [&](int32_t sl, int64_t b, int64_t t) {
+        guard[sl] = t + 1;  // needed by task t: protected in tasks t and t + 1
+        key[sl] = next_use(b, t);
+        rejoin[t + 2].push_back(sl);
+    };
     for (size_t t = 0; t < T; ++t) {
-        std::vector<int64_t> protect = need[t];
-        if (t > 0) protect.insert(protect.end(), need[t - 1].begin(), need[t - 1].end());
-        std::sort(protect.begin(), protect.end());
+        for (int32_t sl : rejoin[t])
+            if (slot_block[sl] >= 0 && guard[sl] == (int64_t)t - 1) heap.push({key[sl], -(int64_t)sl});
+        for (int64_t b : need[t]) {
+            auto hit = where.find(b);
+            if (hit != where.end()) protect(hit->second, b, (int64_t)t);
+        }
         for (int64_t b : need[t]) {
             auto hit = where.find(b);
             if (hit == where.end()) {
                 int32_t slot = -1;
-                for (int64_t sl = 0; sl < cap; ++sl)
-                    if (slot_block[sl] < 0) { slot = (int32_t)sl; break; }
-                if (slot < 0) {
-                    int64_t best = -1;
-                    for (int64_t sl = 0; sl < cap; ++sl) {
-                        const int64_t ob = slot_block[sl];
-                        if (std::binary_search(protect.begin(), protect.end(), ob)) continue;
-                        const int64_t nu = next_use(ob, (int64_t)t);
-                        if (nu > best) { best = nu; slot = (int32_t)sl; }
+                if (next_free < cap) {
+                    slot = (int32_t)next_free++;
+                } else {
+                    while (!heap.empty()) {
+                        const std::pair<int64_t, int64_t> top = heap.top();
+                        heap.pop();
+                        const int32_t sl = (int32_t)(-top.second);
+                        if (slot_block[sl] >= 0 && key[sl] == top.first && guard[sl] < (int64_t)t) {
+                            slot = sl;
+                            break;
+                        }
                     }
                     if (slot < 0) return false;
                     where.erase(slot_block[slot]);
                 }
                 slot_block[slot] = b;
                 where[b] = slot;
+                protect(slot, b, (int64_t)t);
                 (*copies)[t].push_back(PoolCopy{kind, b, slot});
                 ++*ncopies;
                 hit = where.find(b);
@@ -658,8 +701,7 @@ bool simulate(const std::vector<std::vector<int64_t>> &need, int64_t cap, int ki
 }  // namespace
 
 bool Planner::plan_pool(int64_t q_slots, int64_t kv_slots, PoolPlan *out) const {
-    std::vector<std::vector<int64_t>> nq, nkv;
-    task_needs(*this, &nq, &nkv);
+    const std::vector<std::vector<int64_t>> &nq = need_q_, &nkv = need_kv_;
     PoolPlan pp;
     pp.q_slots = q_slots;
     pp.kv_slots = kv_slots;
@@ -717,6 +759,117 @@ size_t Planner::device_arena_bytes() const {
     return a.total;
 }
 
+namespace {
+size_t wl_sizes(size_t entries, size_t runs, size_t units) {
+    ArenaLayout a;
+    a.take(entries * sizeof(WlEntry));
+    a.take(runs * sizeof(WlRun));
+    a.take(units * sizeof(WlUnit));
+    return a.total;
+}
+
+// Runs left after joining rows that continue the previous run (the rule of
+// leaf_worklist and push_run): rows [lo, lo + n) with offset goff.
+struct RunCount {
+    size_t n = 0;
+    bool have = false;
+    int64_t hi = 0, goff = 0;
+    void add(int64_t lo, int64_t rows, int64_t g) {
+        if (!(have && hi == lo && goff == g)) {
+            ++n;
+            have = true;
+            goff = g;
+        }
+        hi = lo + rows;
+    }
+};
+}  // namespace
+
+namespace {
+std::vector<std::vector<int64_t>> bwd_task_blocks(const Planner &pl);
+}  // namespace
+
+void Planner::count_leaves() {
+    task_needs(*this, &need_q_, &need_kv_);
+    bwd_blocks_ = bwd_task_blocks(*this);
+    const int rpus[3] = {64, 128, 256};
+    leaf_counts_.assign(leaves.size(), LeafCount{});
+    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
+        LeafCount &c = leaf_counts_[t];
+        const size_t n = leaves[t].blocks.size();
+        std::vector<int32_t> adj_q(n, 0), adj_kv(n, 0);
+        std::vector<std::vector<int32_t>> qs_of(n);
+        for (int64_t i = entry_begin_of_leaf_[t]; i < entry_begin_of_leaf_[t + 1]; ++i) {
+            const Entry &e = entries[i];
+            ++c.ne_q;
+            for (const KeyRun &r : e.runs) {
+                c.keys_q += r.b1 - r.b0 + 1;
+                for (int64_t kb = r.b0; kb < r.b1; ++kb) ++adj_q[r.m0 + (kb - r.b0)];
+                for (int64_t kb = r.b0; kb <= r.b1; ++kb) qs_of[r.m0 + (kb - r.b0)].push_back(e.mq);
+            }
+            // A chunk is a unit when the entry's first key is at or before its last query.
+            const int64_t q_lo = e.qb * block, q_hi = q_lo + block_rows(e.qb), k_first = e.runs.front().b0 * block;
+            for (int x = 0; x < 3; ++x)
+                for (int64_t q0 = q_lo; q0 < q_hi; q0 += rpus[x])
+                    if (!spec.causal || k_first <= std::min<int64_t>(q0 + rpus[x], q_hi) - 1) ++c.nu_q[x];
+        }
+        for (size_t mk = 0; mk < n; ++mk) {
+            std::vector<int32_t> &qm = qs_of[mk];
+            if (qm.empty()) continue;
+            std::sort(qm.begin(), qm.end());
+            ++c.ne_kv;
+            c.qrys_kv += (int64_t)qm.size();
+            int64_t q_end = 0;  // one past the last query row (global)
+            for (size_t j = 0; j < qm.size(); ++j) {
+                const int64_t qb = leaves[t].blocks[qm[j]];
+                q_end = std::max<int64_t>(q_end, qb * block + block_rows(qb));
+                // Consecutive members with consecutive blocks (members need not hold consecutive blocks).
+                if (j > 0 && qm[j] == qm[j - 1] + 1 && qb == leaves[t].blocks[qm[j - 1]] + 1) ++adj_kv[qm[j - 1]];
+            }
+            // A chunk of keys is a unit when some query is at or after its first key.
+            const int64_t kb = leaves[t].blocks[mk], k_lo = kb * block, k_hi = k_lo + block_rows(kb);
+            for (int x = 0; x < 3; ++x)
+                for (int64_t k0 = k_lo; k0 < k_hi; k0 += rpus[x])
+                    if (!spec.causal || q_end > k0) ++c.nu_kv[x];
+        }
+        for (size_t m = 0; m < n; ++m) {
+            if (adj_q[m]) c.adj_q.push_back({(int32_t)m, adj_q[m]});
+            if (adj_kv[m]) c.adj_kv.push_back({(int32_t)m, adj_kv[m]});
+        }
+    }
+}
+
+namespace {
+int rpu_index(int rows) { return rows == 64 ? 0 : rows == 128 ? 1 : 2; }
+}  // namespace
+
+size_t Planner::leaf_wl_bytes(int64_t t, const PoolPlan &pool, int rows_per_unit, int heads) const {
+    const LeafCount &c = leaf_counts_[t];
+    // Members m and m + 1 listed here hold consecutive blocks; a run
+    // continues across them when their slots are adjacent and block m is full.
+    int64_t joins = 0;
+    for (const auto &a : c.adj_q) {
+        const int32_t m = a.first;
+        if (pool.kv_slot[t][m + 1] == pool.kv_slot[t][m] + 1 && block_rows(leaves[t].blocks[m]) == block)
+            joins += a.second;
+    }
+    return wl_sizes((size_t)c.ne_q, (size_t)(c.keys_q - joins), (size_t)c.nu_q[rpu_index(rows_per_unit)] * heads);
+}
+
+size_t Planner::leaf_bwd_wl_bytes(int64_t t, const BwdCachePlan &cp, int rows_per_unit, int heads) const {
+    const LeafCount &c = leaf_counts_[t];
+    const std::vector<int32_t> &ms = cp.member_slot[t];
+    auto joined = [&](const std::vector<std::pair<int32_t, int32_t>> &adj) {
+        int64_t j = 0;
+        for (const auto &a : adj)
+            if (ms[a.first + 1] == ms[a.first] + 1 && block_rows(leaves[t].blocks[a.first]) == block) j += a.second;
+        return j;
+    };
+    const int x = rpu_index(rows_per_unit);
+    return wl_sizes((size_t)c.ne_q, (size_t)(c.keys_q - joined(c.adj_q)), (size_t)c.nu_q[x] * heads) +
+           wl_sizes((size_t)c.ne_kv, (size_t)(c.qrys_kv - joined(c.adj_kv)), (size_t)c.nu_kv[x] * heads);
+}
+
 size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
     const int64_t N = spec.N, R = max_task_rows;
     const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
@@ -733,10 +886,7 @@ size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
         a.take((size_t)R * g * dd * e);                 // finished out rows
         a.take((size_t)g * R * sizeof(float));          // finished lse rows
     }
-    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
-        WorkList wl = leaf_worklist(t, pl, unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
-        a.take(wl_bytes(wl));
-    }
+    for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) a.take(leaf_wl_bytes(t, pl, unit_rows_for(spec.elem_bytes), g));
     return a.total;
 }
 
@@ -996,7 +1146,7 @@ void push_run(WorkList *wl, int32_t run_begin, int32_t lo, int32_t n, int32_t go
 }  // namespace
 
 bool Planner::plan_bwd_cache(int64_t C, BwdCachePlan *out) const {
-    const std::vector<std::vector<int64_t>> tb = bwd_task_blocks(*this);
+    const std::vector<std::vector<int64_t>> &tb = bwd_blocks_;
     const int64_t T = (int64_t)tb.size();
     std::vector<std::vector<int64_t>> uses(num_blocks);
     for (int64_t t = 0; t < T; ++t)
@@ -1011,28 +1161,45 @@ bool Planner::plan_bwd_cache(int64_t C, BwdCachePlan *out) const {
     cp.member_slot.assign(T, {});
     cp.finals.assign(T, {});
     std::vector<int64_t> held(C, -1);        // block whose rows the slot holds
-    std::vector<int64_t> release(C, 0);      // a finished block's slot is free from this task on
     std::vector<char> done(num_blocks, 0), on_host(num_blocks, 0);
     std::vector<int32_t> slot_of(num_blocks, -1);
+    // Free slots: the lowest index first (a finished block's slot is free
+    // from two tasks after its last one).  Eviction candidates: as in the
+    // forward cache (simulate above), a lazy max-heap of (next use, -slot)
+    // over the slots of unfinished blocks neither this task nor the
+    // previous one touches.
+    std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> free_slots;
+    for (int64_t sl = 0; sl < C; ++sl) free_slots.push(sl);
+    std::vector<std::vector<int32_t>> freed(T + 2), rejoin(T + 2);
+    std::vector<int64_t> key(C, -1), guard(C, -1);
+    std::priority_queue<std::pair<int64_t, int64_t>> heap;
+    auto protect = [&](int32_t sl, int64_t b, int64_t t) {
+        guard[sl] = t + 1;
+        key[sl] = next_use(b, t);
+        rejoin[t + 2].push_back(sl);
+    };
     for (int64_t t = 0; t < T; ++t) {
-        std::vector<int64_t> protect = tb[t];
-        if (t > 0) protect.insert(protect.end(), tb[t - 1].begin(), tb[t - 1].end());
-        std::sort(protect.begin(), protect.end());
+        for (int32_t sl : freed[t]) free_slots.push(sl);
+        for (int32_t sl : rejoin[t])
+            if (held[sl] >= 0 && !done[held[sl]] && guard[sl] == t - 1) heap.push({key[sl], -(int64_t)sl});
+        for (int64_t b : tb[t])
+            if (slot_of[b] >= 0) protect(slot_of[b], b, t);
         for (int64_t b : tb[t]) {
             if (slot_of[b] >= 0) continue;
             int32_t slot = -1;
-            for (int64_t s = 0; s < C && slot < 0; ++s)
-                if (held[s] < 0 || (done[held[s]] && release[s] <= t)) slot = (int32_t)s;
             int64_t evict = -1;
-            if (slot < 0) {
-                int64_t best = -1;
-                for (int64_t s = 0; s < C; ++s) {
-                    const int64_t ob = held[s];
-                    if (ob < 0 || done[ob] || std::binary_search(protect.begin(), protect.end(), ob)) continue;
-                    const int64_t nu = next_use(ob, t);
-                    if (nu > best) {
-                        best = nu;
-                        slot = (int32_t)s;
+            if (!free_slots.empty()) {
+                slot = (int32_t)free_slots.top();
+                free_slots.pop();
+            } else {
+                while (!heap.empty()) {
+                    const std::pair<int64_t, int64_t> top = heap.top();
+                    heap.pop();
+                    const int32_t sl = (int32_t)(-top.second);
+                    const int64_t ob = held[sl];
+                    if (ob >= 0 && !done[ob] && key[sl] == top.first && guard[sl] < t) {
+                        slot = sl;
+                        break;
                     }
                 }
                 if (slot < 0) return false;
@@ -1045,6 +1212,7 @@ bool Planner::plan_bwd_cache(int64_t C, BwdCachePlan *out) const {
             ++cp.loads;
             held[slot] = b;
             slot_of[b] = slot;
+            protect(slot, b, t);
         }
         const std::vector<int64_t> &blocks = leaves[t].blocks;
         cp.member_slot[t].assign(blocks.size(), -1);
@@ -1053,7 +1221,7 @@ bool Planner::plan_bwd_cache(int64_t C, BwdCachePlan *out) const {
             if (uses[b].back() == t) {
                 done[b] = 1;
                 cp.finals[t].push_back({b, slot_of[b]});
-                release[slot_of[b]] = t + 2;
+                freed[t + 2].push_back(slot_of[b]);
                 slot_of[b] = -1;
             }
     }
@@ -1149,8 +1317,9 @@ size_t Planner::bwd_arena_bytes(int g, const BwdCachePlan &c) const {
     a.take(rows * gk * dd * sizeof(float));       // dK sums
     a.take(rows * gk * dd * sizeof(float));       // dV sums
     for (int64_t t = 0; t < (int64_t)leaves.size(); ++t) {
-        a.take(wl_bytes(leaf_bwd_q_worklist(t, c, tile, tile, g)));
-        a.take(wl_bytes(leaf_bwd_kv_worklist(t, c, tile, tile, g)));
+        // The two lists are laid out one after the other; each ArenaLayout
+        // step is 256-aligned, so their sum is the same as two takes.
+        a.take(leaf_bwd_wl_bytes(t, c, tile, g));
     }
     return a.total;
 }

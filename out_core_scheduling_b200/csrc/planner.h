@@ -306,6 +306,33 @@ public:
     std::vector<HostLaunch> host_sched;  // the chosen resident schedule (empty: task by task)
 
 private:
+    // Bytes of leaf_worklist(t, pool, rows_per_unit, *, heads) and of the two
+    // streamed-backward lists of leaf t, counted without building them (the
+    // sizing loops try many caches): the same entries, the same runs after
+    // joining rows that continue each other, and one unit per head and
+    // chunk of an entry's rows that some key (query) of its runs reaches
+    // under the causal rule.  verify() checks them against the built lists.
+    size_t leaf_wl_bytes(int64_t t, const PoolPlan &pool, int rows_per_unit, int heads) const;
+    size_t leaf_bwd_wl_bytes(int64_t t, const BwdCachePlan &c, int rows_per_unit, int heads) const;
+    // What those counts need that does not depend on the cache, per leaf:
+    // entries; units per head for chunks of 64, 128 and 256 rows; key
+    // blocks over all entries (runs before joining), and for each member m
+    // how many entries list the key blocks of members m and m + 1 one after
+    // the other when those blocks are consecutive (a run joins there when
+    // their slots are adjacent); the same for the key-stationary list (per
+    // key member, its query members).
+    struct LeafCount {
+        int64_t ne_q = 0, nu_q[3] = {0, 0, 0}, keys_q = 0;
+        std::vector<std::pair<int32_t, int32_t>> adj_q;
+        int64_t ne_kv = 0, nu_kv[3] = {0, 0, 0}, qrys_kv = 0;
+        std::vector<std::pair<int32_t, int32_t>> adj_kv;
+    };
+    std::vector<LeafCount> leaf_counts_;
+    // Blocks each leaf task needs as Q and as K/V (forward), and touches
+    // (backward), in member order: fixed by the plan, used by every cache
+    // simulation of the sizing loops.
+    std::vector<std::vector<int64_t>> need_q_, need_kv_, bwd_blocks_;
+    void count_leaves();
     std::vector<int64_t> entry_begin_of_leaf_;  // first entry index of each leaf
     std::vector<int32_t> first_leaf_, last_leaf_; // per query block
     void size_plan();

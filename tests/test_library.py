@@ -272,6 +272,39 @@ def test_debug_plan_checks(monkeypatch, args):
     assert cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, H_kv=Hkv).info()["debug_checked"] == 0
 
 
+def _smallest_budget(N, H, d, ls, causal, dtype, Hkv):
+    lo, hi = 1 << 16, 1 << 36
+    while hi - lo > hi // 64:
+        mid = (lo + hi) // 2
+        try:
+            i = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dtype, H_kv=Hkv, mem_budget_bytes=mid,
+                                  host_tasks=True).info()
+            ok = i["head_group"] > 0 and i["bwd_head_group"] > 0
+        except cqsa.CqsaError:
+            ok = False
+        lo, hi = (lo, mid) if ok else (mid, hi)
+    return hi
+
+
+@pytest.mark.parametrize("args", [
+    (21 * 64, 4, 64, [5], False, 0), (21 * 64, 4, 64, [5], True, 0), (91 * 16 + 5, 2, 64, [4, 3], True, 0),
+    (7 * 100 + 3, 2, 128, [3], False, 0), (13 * 64, 4, 64, [4], True, 2), (343 * 8, 1, 64, [3, 3, 3], False, 0)])
+def test_debug_counted_work_list_sizes(monkeypatch, args):
+    """The sizing loops count the streamed work lists' bytes instead of
+    building them; under CQSA_DEBUG every plan compares those counts with
+    the built lists of its chosen caches (forward task by task and backward),
+    here at budgets that force evictions and write-backs."""
+    N, H, d, ls, causal, Hkv = args
+    for dtype in (cqsa.CQSA_BF16, cqsa.CQSA_FP32):
+        b = _smallest_budget(N, H, d, ls, causal, dtype, Hkv)
+        monkeypatch.setenv("CQSA_DEBUG", "1")
+        for f in (1.0, 1.3, 2.0):
+            i = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal, dtype=dtype, H_kv=Hkv, mem_budget_bytes=int(b * f),
+                                  host_tasks=True).info()
+            assert i["debug_checked"] == 1 and i["head_group"] > 0 and i["bwd_head_group"] > 0
+        monkeypatch.setenv("CQSA_DEBUG", "0")
+
+
 def test_fault_injection_arguments():
     for kind, nth in ((0, 1), (4, 1), (cqsa.CQSA_FAULT_ALLOC, -1), (cqsa.CQSA_FAULT_SETUP, -1)):
         with pytest.raises(cqsa.CqsaError) as ei:
