@@ -156,6 +156,8 @@ typedef struct {
     int host_resident;                  /* host-mode forward runs the resident schedule (1) or task by task (0) */
     int64_t host_launches;              /* launches of the resident schedule per head group (0: task by task) */
     int64_t arrival_blocks;             /* resident schedule: blocks per arrival group of the copy-in */
+    int host_sets;                      /* resident schedule: head groups whose device buffers coexist
+                                           (2: the next group's copies overlap this group's launches) */
 } cqsa_plan_info_t;
 
 /* One (leaf task, query block) entry of the work list, in global blocks. */
@@ -425,7 +427,10 @@ cqsa_status_t cqsa_plan_bwd_cache_task(const cqsa_plan_t *plan, int64_t t, int64
  * group fits the budget ([B] "Implementation": stream the blocks the tasks
  * need; here each block crosses the host link once per head group).  The
  * blocks are copied in increasing order; the copy stream marks every
- * info.arrival_blocks consecutive blocks.  The launch waits for the mark of
+ * info.arrival_blocks consecutive blocks.  With info.host_sets = 2 the
+ * head groups alternate between two sets of device buffers, so one group's
+ * copies run while the previous group's launches do; a group waits only for
+ * the group before last (the same set).  The launch waits for the mark of
  * the group holding *need (the last block it reads), runs on internal
  * compute stream *stream (0 or 1), and first waits for launch *after of the
  * other stream (-1: none).  It takes the plan's (query block, key block)

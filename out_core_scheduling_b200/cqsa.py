@@ -83,7 +83,7 @@ class PlanInfo(ctypes.Structure):
                 ("bwd_cache_slots", ctypes.c_int64), ("bwd_h2d_bytes", ctypes.c_size_t),
                 ("bwd_d2h_bytes", ctypes.c_size_t), ("bwd_spill_host_bytes", ctypes.c_size_t),
                 ("bwd_writebacks", ctypes.c_int64), ("host_resident", ctypes.c_int),
-                ("host_launches", ctypes.c_int64), ("arrival_blocks", ctypes.c_int64)]
+                ("host_launches", ctypes.c_int64), ("arrival_blocks", ctypes.c_int64), ("host_sets", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         out = {}

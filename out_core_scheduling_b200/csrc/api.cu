@@ -283,12 +283,21 @@ struct cqsa_plan {
     cudaEvent_t ev_in_ready[2] = {}, ev_in_free[2] = {}, ev_merged[2] = {}, ev_out_free[2] = {};
     cudaEvent_t ev_start = nullptr, ev_done_comp = nullptr, ev_done_out = nullptr;
     // Resident schedule (Planner::host_sched): per launch its work list, a
-    // second compute stream, a mark per arrival group and per launch, and
-    // the ends of a head group on the compute and copy-out streams.
+    // second compute stream, and per buffer set (head groups in flight, see
+    // Sizing::sets) its accumulators, block pools, finished rows, tensor
+    // maps, a mark per arrival group and per launch, and the ends of its
+    // latest head group on the compute and copy-out streams.
+    struct ResidentSet {
+        float *acc_o = nullptr, *acc_lse = nullptr, *lse = nullptr;
+        char *pool_q = nullptr, *pool_k = nullptr, *pool_v = nullptr, *out = nullptr;
+        CUtensorMap mq, mk, mv;
+        std::vector<cudaEvent_t> ev_arrive, ev_launch;
+        cudaEvent_t ev_comp_end[2] = {}, ev_out_end = nullptr;
+    };
+    ResidentSet rs[2];
+    int nsets = 0;
     std::vector<DevWl> res_wl;
     cudaStream_t s_comp2 = nullptr;
-    std::vector<cudaEvent_t> ev_arrive, ev_launch;
-    cudaEvent_t ev_comp_end[2] = {}, ev_out_end = nullptr;
 
     // Kernel timing (cqsa_plan_profile): event pairs not yet read, a pool of
     // spare events, and the totals read so far.
@@ -414,16 +423,20 @@ cqsa_status_t setup_resident(cqsa_plan_t *P) {
     const int g = pl.sizing.head_group, gk = pl.spec.kv_heads_of(g);
     const int64_t N = pl.spec.N, rows = pl.num_blocks * pl.block;
     const size_t e = (size_t)P->elem, dd = (size_t)pl.spec.d;
+    const int nsets = pl.sizing.sets;
     // Same layout steps as Planner::resident_arena_bytes.
     ArenaLayout a;
     const size_t o_err = a.take(256);
-    const size_t o_acc = a.take((size_t)N * g * dd * sizeof(float));
-    const size_t o_accl = a.take((size_t)g * N * sizeof(float));
-    const size_t o_pq = a.take((size_t)rows * g * dd * e);
-    const size_t o_pk = a.take((size_t)rows * gk * dd * e);
-    const size_t o_pv = a.take((size_t)rows * gk * dd * e);
-    const size_t o_out = a.take((size_t)N * g * dd * e);
-    const size_t o_lse = a.take((size_t)g * N * sizeof(float));
+    size_t o_acc[2], o_accl[2], o_pq[2], o_pk[2], o_pv[2], o_out[2], o_lse[2];
+    for (int st = 0; st < nsets; ++st) {
+        o_acc[st] = a.take((size_t)N * g * dd * sizeof(float));
+        o_accl[st] = a.take((size_t)g * N * sizeof(float));
+        o_pq[st] = a.take((size_t)rows * g * dd * e);
+        o_pk[st] = a.take((size_t)rows * gk * dd * e);
+        o_pv[st] = a.take((size_t)rows * gk * dd * e);
+        o_out[st] = a.take((size_t)N * g * dd * e);
+        o_lse[st] = a.take((size_t)g * N * sizeof(float));
+    }
     std::vector<size_t> o_wl(LS.size());
     for (size_t i = 0; i < LS.size(); ++i) o_wl[i] = a.take(wl_region(LS[i].wl));
     if (a.total != pl.sizing.host_arena)
@@ -437,38 +450,43 @@ cqsa_status_t setup_resident(cqsa_plan_t *P) {
     // Zeroed once, so rows a partial key tile reads past the last block are finite.
     CK(cudaMemset(arena, 0, a.total));
     P->h_err = reinterpret_cast<int *>(arena + o_err);
-    P->acc_o = reinterpret_cast<float *>(arena + o_acc);
-    P->acc_lse = reinterpret_cast<float *>(arena + o_accl);
-    P->pool_q = arena + o_pq;
-    P->pool_k = arena + o_pk;
-    P->pool_v = arena + o_pv;
-    P->out_st[0] = arena + o_out;
-    P->lse_st[0] = reinterpret_cast<float *>(arena + o_lse);
-    P->out_st[1] = nullptr;
-    P->lse_st[1] = nullptr;
+    P->nsets = nsets;
+    for (int st = 0; st < nsets; ++st) {
+        cqsa_plan_t::ResidentSet &R = P->rs[st];
+        R.acc_o = reinterpret_cast<float *>(arena + o_acc[st]);
+        R.acc_lse = reinterpret_cast<float *>(arena + o_accl[st]);
+        R.pool_q = arena + o_pq[st];
+        R.pool_k = arena + o_pk[st];
+        R.pool_v = arena + o_pv[st];
+        R.out = arena + o_out[st];
+        R.lse = reinterpret_cast<float *>(arena + o_lse[st]);
+        if (P->dtype == CQSA_BF16) {
+            cqsa_status_t st2;
+            if ((st2 = make_map(&R.mq, R.pool_q, rows, g, pl.spec.d)) != CQSA_OK) return st2;
+            if ((st2 = make_map(&R.mk, R.pool_k, rows, gk, pl.spec.d)) != CQSA_OK) return st2;
+            if ((st2 = make_map(&R.mv, R.pool_v, rows, gk, pl.spec.d)) != CQSA_OK) return st2;
+        }
+    }
     P->res_wl.assign(LS.size(), DevWl());
     for (size_t i = 0; i < LS.size(); ++i) {
         std::vector<char> buf = pack_wl(LS[i].wl);
         if (!buf.empty()) CK(lib_upload(arena + o_wl[i], buf.data(), buf.size()));
         P->res_wl[i] = place_wl(arena + o_wl[i], LS[i].wl);
     }
-    if (P->dtype == CQSA_BF16) {
-        cqsa_status_t st;
-        if ((st = make_map(&P->mq, P->pool_q, rows, g, pl.spec.d)) != CQSA_OK) return st;
-        if ((st = make_map(&P->mk, P->pool_k, rows, gk, pl.spec.d)) != CQSA_OK) return st;
-        if ((st = make_map(&P->mv, P->pool_v, rows, gk, pl.spec.d)) != CQSA_OK) return st;
-    }
     CK(cudaStreamCreateWithFlags(&P->s_in, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_comp2, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_out, cudaStreamNonBlocking));
     const int64_t A = pl.arrival_blocks();
-    P->ev_arrive.assign((size_t)((pl.num_blocks + A - 1) / A), nullptr);
-    P->ev_launch.assign(LS.size(), nullptr);
-    for (cudaEvent_t &ev : P->ev_arrive) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
-    for (cudaEvent_t &ev : P->ev_launch) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
-    for (int s = 0; s < 2; ++s) CK(cudaEventCreateWithFlags(&P->ev_comp_end[s], cudaEventDisableTiming));
-    CK(cudaEventCreateWithFlags(&P->ev_out_end, cudaEventDisableTiming));
+    for (int st = 0; st < nsets; ++st) {
+        cqsa_plan_t::ResidentSet &R = P->rs[st];
+        R.ev_arrive.assign((size_t)((pl.num_blocks + A - 1) / A), nullptr);
+        R.ev_launch.assign(LS.size(), nullptr);
+        for (cudaEvent_t &ev : R.ev_arrive) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+        for (cudaEvent_t &ev : R.ev_launch) CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+        for (int x = 0; x < 2; ++x) CK(cudaEventCreateWithFlags(&R.ev_comp_end[x], cudaEventDisableTiming));
+        CK(cudaEventCreateWithFlags(&R.ev_out_end, cudaEventDisableTiming));
+    }
     CK(cudaEventCreateWithFlags(&P->ev_start, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&P->ev_done_comp, cudaEventDisableTiming));
     CK(cudaEventCreateWithFlags(&P->ev_done_out, cudaEventDisableTiming));
@@ -567,18 +585,25 @@ void release_host_mode(cqsa_plan_t *P) {
                 *e = nullptr;
             }
     }
-    cudaEvent_t *evs[6] = {&P->ev_start, &P->ev_done_comp, &P->ev_done_out, &P->ev_comp_end[0],
-                           &P->ev_comp_end[1], &P->ev_out_end};
+    cudaEvent_t *evs[3] = {&P->ev_start, &P->ev_done_comp, &P->ev_done_out};
     for (cudaEvent_t *e : evs)
         if (*e) {
             cudaEventDestroy(*e);
             *e = nullptr;
         }
-    for (std::vector<cudaEvent_t> *v : {&P->ev_arrive, &P->ev_launch}) {
-        for (cudaEvent_t e : *v)
-            if (e) cudaEventDestroy(e);
-        v->clear();
+    for (cqsa_plan_t::ResidentSet &R : P->rs) {
+        for (std::vector<cudaEvent_t> *v : {&R.ev_arrive, &R.ev_launch}) {
+            for (cudaEvent_t e : *v)
+                if (e) cudaEventDestroy(e);
+            v->clear();
+        }
+        for (cudaEvent_t *e : {&R.ev_comp_end[0], &R.ev_comp_end[1], &R.ev_out_end})
+            if (*e) {
+                cudaEventDestroy(*e);
+                *e = nullptr;
+            }
     }
+    P->nsets = 0;
     P->res_wl.clear();
     cudaStream_t *ss[4] = {&P->s_in, &P->s_comp, &P->s_comp2, &P->s_out};
     for (cudaStream_t *s : ss)
@@ -936,17 +961,20 @@ cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k
     cudaStream_t sc[2] = {P->s_comp, P->s_comp2};
     CK(cudaEventRecord(P->ev_start, stream));
     for (cudaStream_t x : {P->s_in, sc[0], sc[1], P->s_out}) CK(cudaStreamWaitEvent(x, P->ev_start, 0));
-    for (int h0 = 0; h0 < H; h0 += g) {
+    int gi = 0;
+    for (int h0 = 0; h0 < H; h0 += g, ++gi) {
         NvtxRange nvtx_group("cqsa resident head group", h0);
-        if (h0 > 0) {
-            // The pools change once the previous group's launches are done;
-            // its accumulators and finished rows once its launches and
-            // copy-out are.
-            CK(cudaStreamWaitEvent(P->s_in, P->ev_comp_end[0], 0));
-            CK(cudaStreamWaitEvent(P->s_in, P->ev_comp_end[1], 0));
+        cqsa_plan_t::ResidentSet &R = P->rs[gi % P->nsets];
+        if (gi >= P->nsets) {
+            // The set's previous head group: its pools change once that
+            // group's launches are done; its accumulators and finished rows
+            // once its launches and copy-out are.  The group between them
+            // (the other set) is independent of this one.
+            CK(cudaStreamWaitEvent(P->s_in, R.ev_comp_end[0], 0));
+            CK(cudaStreamWaitEvent(P->s_in, R.ev_comp_end[1], 0));
             for (int s = 0; s < 2; ++s) {
-                CK(cudaStreamWaitEvent(sc[s], P->ev_comp_end[1 - s], 0));
-                CK(cudaStreamWaitEvent(sc[s], P->ev_out_end, 0));
+                CK(cudaStreamWaitEvent(sc[s], R.ev_comp_end[1 - s], 0));
+                CK(cudaStreamWaitEvent(sc[s], R.ev_out_end, 0));
             }
         }
         // -- H2D: block b to pool rows b * Bk.
@@ -955,20 +983,20 @@ cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k
             if (rows) {
                 const size_t src = ((size_t)b * Bk * H + h0) * d * e;
                 const size_t src_kv = ((size_t)b * Bk * Hkv + h0 / kvg) * d * e;
-                CK(copy_rows(P->pool_q + (size_t)b * Bk * grp_row, grp_row, hq + src, full_row, grp_row, rows,
+                CK(copy_rows(R.pool_q + (size_t)b * Bk * grp_row, grp_row, hq + src, full_row, grp_row, rows,
                              cudaMemcpyHostToDevice, P->s_in));
-                CK(copy_rows(P->pool_k + (size_t)b * Bk * grp_kv_row, grp_kv_row, hk + src_kv, full_kv_row,
+                CK(copy_rows(R.pool_k + (size_t)b * Bk * grp_kv_row, grp_kv_row, hk + src_kv, full_kv_row,
                              grp_kv_row, rows, cudaMemcpyHostToDevice, P->s_in));
-                CK(copy_rows(P->pool_v + (size_t)b * Bk * grp_kv_row, grp_kv_row, hv + src_kv, full_kv_row,
+                CK(copy_rows(R.pool_v + (size_t)b * Bk * grp_kv_row, grp_kv_row, hv + src_kv, full_kv_row,
                              grp_kv_row, rows, cudaMemcpyHostToDevice, P->s_in));
             }
-            if ((b + 1) % A == 0 || b == nb - 1) CK(cudaEventRecord(P->ev_arrive[(size_t)(b / A)], P->s_in));
+            if ((b + 1) % A == 0 || b == nb - 1) CK(cudaEventRecord(R.ev_arrive[(size_t)(b / A)], P->s_in));
         }
         for (size_t i = 0; i < LS.size(); ++i) {
             const HostLaunch &L = LS[i];
             cudaStream_t s = sc[L.stream];
-            CK(cudaStreamWaitEvent(s, P->ev_arrive[(size_t)(L.need / A)], 0));
-            if (L.after >= 0) CK(cudaStreamWaitEvent(s, P->ev_launch[(size_t)L.after], 0));
+            CK(cudaStreamWaitEvent(s, R.ev_arrive[(size_t)(L.need / A)], 0));
+            if (L.after >= 0) CK(cudaStreamWaitEvent(s, R.ev_launch[(size_t)L.after], 0));
             AttnParams ap = base_params(P, P->h_err);
             ap.entries = P->res_wl[i].entries;
             ap.runs = P->res_wl[i].runs;
@@ -978,44 +1006,45 @@ cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k
             ap.hq_off = h0;
             ap.hk_off = h0 / kvg;
             ap.epi = EPI_MERGE;
-            ap.acc_o = P->acc_o;
-            ap.acc_lse = P->acc_lse;
+            ap.acc_o = R.acc_o;
+            ap.acc_lse = R.acc_lse;
             ap.acc_rows = N;
-            ap.out = P->out_st[0];
-            ap.out_lse = P->lse_st[0];
+            ap.out = R.out;
+            ap.out_lse = R.lse;
             ap.out_rows = N;
             {
                 LaunchTimer tm(P, s, 0);
                 if (P->dtype == CQSA_BF16)
-                    CK(launch_attn_tc(d, P->mq, P->mk, P->mv, ap, P->res_wl[i].num_units, s));
+                    CK(launch_attn_tc(d, R.mq, R.mk, R.mv, ap, P->res_wl[i].num_units, s));
                 else
-                    CK(launch_attn_simt(d, P->elem, P->pool_q, P->pool_k, P->pool_v, ap, P->res_wl[i].num_units,
-                                        s));
+                    CK(launch_attn_simt(d, P->elem, R.pool_q, R.pool_k, R.pool_v, ap, P->res_wl[i].num_units, s));
                 tm.stop();
             }
-            CK(cudaEventRecord(P->ev_launch[i], s));
+            CK(cudaEventRecord(R.ev_launch[i], s));
             if (L.finish.empty()) continue;
             // -- D2H of the finished query blocks, consecutive ones together.
-            CK(cudaStreamWaitEvent(P->s_out, P->ev_launch[i], 0));
+            CK(cudaStreamWaitEvent(P->s_out, R.ev_launch[i], 0));
             for (size_t j = 0; j < L.finish.size();) {
                 size_t j1 = j + 1;
                 while (j1 < L.finish.size() && L.finish[j1] == L.finish[j1 - 1] + 1) ++j1;
                 const int64_t r0 = L.finish[j] * Bk, r1 = pl.block_end(L.finish[j1 - 1]);
-                CK(copy_rows(ho + ((size_t)r0 * H + h0) * d * e, full_row, P->out_st[0] + (size_t)r0 * grp_row,
-                             grp_row, grp_row, (size_t)(r1 - r0), cudaMemcpyDeviceToHost, P->s_out));
-                CK(cudaMemcpy2DAsync(lse + (size_t)h0 * N + r0, (size_t)N * sizeof(float), P->lse_st[0] + r0,
+                CK(copy_rows(ho + ((size_t)r0 * H + h0) * d * e, full_row, R.out + (size_t)r0 * grp_row, grp_row,
+                             grp_row, (size_t)(r1 - r0), cudaMemcpyDeviceToHost, P->s_out));
+                CK(cudaMemcpy2DAsync(lse + (size_t)h0 * N + r0, (size_t)N * sizeof(float), R.lse + r0,
                                      (size_t)N * sizeof(float), (size_t)(r1 - r0) * sizeof(float), (size_t)g,
                                      cudaMemcpyDeviceToHost, P->s_out));
                 j = j1;
             }
         }
-        CK(cudaEventRecord(P->ev_comp_end[0], sc[0]));
-        CK(cudaEventRecord(P->ev_comp_end[1], sc[1]));
-        CK(cudaEventRecord(P->ev_out_end, P->s_out));
+        CK(cudaEventRecord(R.ev_comp_end[0], sc[0]));
+        CK(cudaEventRecord(R.ev_comp_end[1], sc[1]));
+        CK(cudaEventRecord(R.ev_out_end, P->s_out));
     }
-    CK(cudaStreamWaitEvent(stream, P->ev_comp_end[0], 0));
-    CK(cudaStreamWaitEvent(stream, P->ev_comp_end[1], 0));
-    CK(cudaStreamWaitEvent(stream, P->ev_out_end, 0));
+    for (int st = 0; st < std::min(gi, P->nsets); ++st) {
+        CK(cudaStreamWaitEvent(stream, P->rs[st].ev_comp_end[0], 0));
+        CK(cudaStreamWaitEvent(stream, P->rs[st].ev_comp_end[1], 0));
+        CK(cudaStreamWaitEvent(stream, P->rs[st].ev_out_end, 0));
+    }
     return CQSA_OK;
 }
 
@@ -1136,9 +1165,9 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
     cudaStreamWaitEvent(stream, P->ev_start, 0);
     cudaStreamWaitEvent(stream, P->ev_done_comp, 0);
     cudaStreamWaitEvent(stream, P->ev_done_out, 0);
-    if (P->s_comp2 && P->ev_comp_end[1]) {
-        cudaEventRecord(P->ev_comp_end[1], P->s_comp2);
-        cudaStreamWaitEvent(stream, P->ev_comp_end[1], 0);
+    if (P->s_comp2 && P->rs[0].ev_comp_end[1]) {
+        cudaEventRecord(P->rs[0].ev_comp_end[1], P->s_comp2);
+        cudaStreamWaitEvent(stream, P->rs[0].ev_comp_end[1], 0);
     }
 }
 
@@ -2043,6 +2072,7 @@ cqsa_status_t cqsa_plan_info(const cqsa_plan_t *plan, cqsa_plan_info_t *info) {
     info->bwd_spill_host_bytes = pl.bwd_sizing.spill_host;
     info->bwd_writebacks = pl.bwd_cache.writebacks;
     info->host_resident = pl.sizing.resident ? 1 : 0;
+    info->host_sets = pl.sizing.resident ? pl.sizing.sets : 0;
     info->host_launches = (int64_t)pl.host_sched.size();
     info->arrival_blocks = pl.arrival_blocks();
     return CQSA_OK;

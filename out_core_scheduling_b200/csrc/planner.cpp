@@ -981,19 +981,21 @@ std::vector<HostLaunch> Planner::host_launches(int rows_per_unit, int bn, int he
     return out;
 }
 
-size_t Planner::resident_arena_bytes(int g, std::vector<HostLaunch> *launches) const {
+size_t Planner::resident_arena_bytes(int g, int sets, std::vector<HostLaunch> *launches) const {
     const int64_t N = spec.N, rows = num_blocks * block;
     const size_t e = (size_t)spec.elem_bytes, dd = (size_t)spec.d;
     const size_t gk = (size_t)spec.kv_heads_of(g);
     ArenaLayout a;
     a.take(256);                                        // error word
-    a.take((size_t)N * g * dd * sizeof(float));         // accumulator O
-    a.take((size_t)g * N * sizeof(float));              // accumulator lse
-    a.take((size_t)rows * g * dd * e);                  // Q pool, one slot per block
-    a.take((size_t)rows * gk * dd * e);                 // K pool
-    a.take((size_t)rows * gk * dd * e);                 // V pool
-    a.take((size_t)N * g * dd * e);                     // finished out rows
-    a.take((size_t)g * N * sizeof(float));              // finished lse rows
+    for (int st = 0; st < sets; ++st) {                 // one buffer set per head group in flight
+        a.take((size_t)N * g * dd * sizeof(float));     // accumulator O
+        a.take((size_t)g * N * sizeof(float));          // accumulator lse
+        a.take((size_t)rows * g * dd * e);              // Q pool, one slot per block
+        a.take((size_t)rows * gk * dd * e);             // K pool
+        a.take((size_t)rows * gk * dd * e);             // V pool
+        a.take((size_t)N * g * dd * e);                 // finished out rows
+        a.take((size_t)g * N * sizeof(float));          // finished lse rows
+    }
     launches->clear();
     if (spec.budget && a.total > spec.budget) return a.total;  // does not fit: no need for the launches
     *launches = host_launches(unit_rows_for(spec.elem_bytes), key_tile_for(spec.elem_bytes), g);
@@ -1027,13 +1029,19 @@ void Planner::size_plan() {
     span(nkv, &min_kv_slots, &full_kv_slots);
 
     const int kvg = spec.kv_group();
-    // The resident schedule at the largest head group whose arena fits
-    // (every block of the group on the device: each crosses the host link
-    // once per group, and the copies overlap the launches pair by pair).
-    for (int g = spec.H; g >= 1 && !spec.host_tasks; --g) {
+    // The resident schedule (every block of a head group on the device:
+    // each crosses the host link once per group, and the copies overlap the
+    // launches pair by pair).  First with two buffer sets at the largest
+    // head group of at most half the heads whose arena fits (the next
+    // group's copies overlap this group's launches, and the first launches
+    // wait for half the bytes), else with one set at the largest group.
+    for (int pass = 0; pass < 2 && !spec.host_tasks && !sizing.resident; ++pass)
+        for (int g = spec.H; g >= 1; --g) {
         if (spec.H % g || (g % kvg != 0 && kvg % g != 0)) continue;
+        const int sets = pass == 0 ? 2 : 1;
+        if (sets == 2 && spec.H / g < 2) continue;
         std::vector<HostLaunch> sched;
-        const size_t rb = resident_arena_bytes(g, &sched);
+        const size_t rb = resident_arena_bytes(g, sets, &sched);
         PoolPlan pp;
         if ((spec.budget && rb > spec.budget) || !plan_pool(full_q_slots, full_kv_slots, &pp)) continue;
         const size_t blk = (size_t)block * g * spec.d * spec.elem_bytes;
@@ -1045,10 +1053,11 @@ void Planner::size_plan() {
         sizing.host_arena = rb;
         sizing.q_slots = sizing.kv_slots = num_blocks;
         sizing.resident = true;
+        sizing.sets = sets;
         sizing.h2d = (size_t)nb_rows * (blk + 2 * blk_kv) * (size_t)(spec.H / g);
         pool = std::move(pp);
         break;
-    }
+        }
     for (int g = spec.H; g >= 1 && !sizing.resident; --g) {
         if (spec.H % g) continue;
         // A head group covers whole key/value groups, or lies inside one.

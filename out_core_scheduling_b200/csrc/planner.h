@@ -159,6 +159,7 @@ struct Sizing {
     size_t h2d = 0, d2h = 0;
     int64_t q_slots = 0, kv_slots = 0;
     bool resident = false;  // the streamed forward runs the resident schedule (HostLaunch)
+    int sets = 1;           // resident schedule: head groups whose buffers coexist (copies of the next overlap this one)
 };
 
 // Streamed forward when the device holds every block of a head group at
@@ -302,7 +303,7 @@ public:
     // launches, and its arena for a head group g.
     int64_t arrival_blocks() const;
     std::vector<HostLaunch> host_launches(int rows_per_unit, int bn, int heads) const;
-    size_t resident_arena_bytes(int g, std::vector<HostLaunch> *launches) const;
+    size_t resident_arena_bytes(int g, int sets, std::vector<HostLaunch> *launches) const;
     std::vector<HostLaunch> host_sched;  // the chosen resident schedule (empty: task by task)
 
 private:

@@ -93,12 +93,14 @@ def check_schedule(plan, launches=None):
     return L, A
 
 
-def resident_model(plan, groups=2, drop=()):
+def resident_model(plan, groups=2, drop=(), sets=None):
     """Roles and event counts of ``groups`` head groups of the resident
-    schedule; ``drop`` removes waits by name (planted mistakes)."""
+    schedule, alternating over ``sets`` buffer sets (default: the plan's);
+    ``drop`` removes waits by name (planted mistakes)."""
     info = plan.info()
     L = _launches(plan)
     A, nb = info["arrival_blocks"], info["num_blocks"]
+    sets = sets or info["host_sets"]
     s_in, s_c, s_out = [], [[], []], []
     rec = defaultdict(int)
 
@@ -115,46 +117,47 @@ def resident_model(plan, groups=2, drop=()):
 
     acc = {}
     for g in range(groups):
-        if g:
-            wait(s_in, "comp_end0", "pools_after_launches")
-            wait(s_in, "comp_end1", "pools_after_launches")
+        z = g % sets  # the group's buffer set
+        if g >= sets:
+            wait(s_in, f"comp_end{z}_0", "pools_after_launches")
+            wait(s_in, f"comp_end{z}_1", "pools_after_launches")
             for s in (0, 1):
-                wait(s_c[s], f"comp_end{1 - s}", "group_after_other_stream")
-                wait(s_c[s], "out_end", "group_after_copy_out")
+                wait(s_c[s], f"comp_end{z}_{1 - s}", "group_after_other_stream")
+                wait(s_c[s], f"out_end{z}", "group_after_copy_out")
         for b in range(nb):
-            op(s_in, [], [(f"Q{b}", (g, b)), (f"KV{b}", (g, b))])
+            op(s_in, [], [(f"Q{z}_{b}", (g, b)), (f"KV{z}_{b}", (g, b))])
             if (b + 1) % A == 0 or b == nb - 1:
-                record(s_in, f"arrive{b // A}")
+                record(s_in, f"arrive{z}_{b // A}")
         for i, x in enumerate(L):
             s = x["stream"]
-            wait(s_c[s], f"arrive{x['need'] // A}", "arrival")
+            wait(s_c[s], f"arrive{z}_{x['need'] // A}", "arrival")
             if x["after"] >= 0:
-                wait(s_c[s], f"launch{x['after']}", "after")
+                wait(s_c[s], f"launch{z}_{x['after']}", "after")
             reads, writes = [], []
             flags = dict(zip([p[0] for p in x["pairs"]], x["flags"]))
             keys = defaultdict(set)
             for q, kb in x["pairs"]:
                 keys[q].add(kb)
             for q, f in flags.items():
-                reads.append((f"Q{q}", (g, q)))
-                reads += [(f"KV{kb}", (g, kb)) for kb in sorted(keys[q])]
+                reads.append((f"Q{z}_{q}", (g, q)))
+                reads += [(f"KV{z}_{kb}", (g, kb)) for kb in sorted(keys[q])]
                 n = 0 if f & 1 else acc[(g, q)]
                 if not f & 1:
-                    reads.append((f"acc{q}", (g, q, n)))
+                    reads.append((f"acc{z}_{q}", (g, q, n)))
                 acc[(g, q)] = n + len(keys[q])
                 if f & 2:
-                    writes.append((f"out{q}", (g, q, "final")))
+                    writes.append((f"out{z}_{q}", (g, q, "final")))
                 else:
-                    writes.append((f"acc{q}", (g, q, acc[(g, q)])))
+                    writes.append((f"acc{z}_{q}", (g, q, acc[(g, q)])))
             op(s_c[s], reads, writes)
-            record(s_c[s], f"launch{i}")
+            record(s_c[s], f"launch{z}_{i}")
             fin = [q for q, f in flags.items() if f & 2]
             if fin:
-                wait(s_out, f"launch{i}", "copy_out_after_launch")
-                op(s_out, [(f"out{q}", (g, q, "final")) for q in fin], [])
-        record(s_c[0], "comp_end0")
-        record(s_c[1], "comp_end1")
-        record(s_out, "out_end")
+                wait(s_out, f"launch{z}_{i}", "copy_out_after_launch")
+                op(s_out, [(f"out{z}_{q}", (g, q, "final")) for q in fin], [])
+        record(s_c[0], f"comp_end{z}_0")
+        record(s_c[1], f"comp_end{z}_1")
+        record(s_out, f"out_end{z}")
     counts = {name: 1 for name in rec}
     return [("copy-in", s_in, 1), ("compute0", s_c[0], 1), ("compute1", s_c[1], 1),
             ("copy-out", s_out, 1)], counts
@@ -217,8 +220,17 @@ def test_planted_schedule_mistake_is_caught(what):
 
 @pytest.mark.parametrize("N,H,d,ls,causal", CASES[:4] + CASES[5:6])
 def test_resident_schedule_is_race_free(N, H, d, ls, causal):
+    """One buffer set over two head groups (each waits for the last)."""
     plan = cqsa.cqsa_plan_ex(N, H, d, ls, causal=causal)
-    assert bm.explore(*resident_model(plan, groups=2))
+    assert bm.explore(*resident_model(plan, groups=2, sets=1))
+
+
+def test_two_buffer_sets_are_race_free():
+    """Two buffer sets over three head groups: the second group overlaps the
+    first, the third reuses the first's buffers."""
+    plan = cqsa.cqsa_plan_ex(7 * 128, 2, 64, [3], causal=True)
+    assert plan.info()["host_sets"] == 2
+    assert bm.explore(*resident_model(plan, groups=3))
 
 
 @pytest.mark.parametrize("drop", ["pools_after_launches", "group_after_copy_out", "arrival", "after",
@@ -226,20 +238,23 @@ def test_resident_schedule_is_race_free(N, H, d, ls, causal):
 def test_planted_missing_wait_is_caught(drop):
     plan = cqsa.cqsa_plan_ex(7 * 128, 2, 64, [3], causal=False)
     with pytest.raises(bm.Violation):
-        bm.explore(*resident_model(plan, groups=2, drop=(drop,)))
+        bm.explore(*resident_model(plan, groups=2, drop=(drop,), sets=1))
+    if drop not in ("after",):  # the causal plan's launches need no other-stream waits
+        with pytest.raises(bm.Violation):
+            bm.explore(*resident_model(cqsa.cqsa_plan_ex(7 * 128, 2, 64, [3], causal=True), groups=3,
+                                       drop=(drop,), sets=2))
 
 
 def test_budget_below_the_resident_arena_runs_task_by_task():
     N, H, d = 13 * 256, 2, 128
     full = cqsa.cqsa_plan_ex(N, H, d, [4]).info()
-    assert full["host_resident"] == 1 and full["head_group"] == H
-    plan = cqsa.cqsa_plan_ex(N, H, d, [4], mem_budget_bytes=full["host_arena_bytes"] - 1)
+    # Unlimited: two head groups of one head, in two buffer sets.
+    assert full["host_resident"] == 1 and full["head_group"] == H // 2 and full["host_sets"] == 2
+    one = cqsa.cqsa_plan_ex(N, H, d, [4], mem_budget_bytes=full["host_arena_bytes"] - 1).info()
+    assert one["host_resident"] == 1 and one["host_sets"] == 1   # one set still fits every block
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], mem_budget_bytes=one["host_arena_bytes"] - 1)
     info = plan.info()
-    assert info["host_resident"] in (0, 1)
-    if info["host_resident"]:
-        assert info["head_group"] < H          # a smaller head group still fits every block
-    else:
-        assert info["host_launches"] == 0
+    assert info["host_resident"] == 0 and info["host_launches"] == 0
     forced = cqsa.cqsa_plan_ex(N, H, d, [4], host_tasks=True).info()
     assert forced["host_resident"] == 0 and forced["host_launches"] == 0
     assert forced["host_arena_bytes"] <= full["host_arena_bytes"]
@@ -247,13 +262,13 @@ def test_budget_below_the_resident_arena_runs_task_by_task():
 
 
 def test_resident_head_groups_replay_the_schedule():
-    """A budget between the resident arenas of H and H / 2 heads: two head
-    groups, each with every block on the device."""
-    N, H, d = 13 * 256, 4, 128
-    full = cqsa.cqsa_plan_ex(N, H, d, [4]).info()["host_arena_bytes"]
-    plan = cqsa.cqsa_plan_ex(N, H, d, [4], mem_budget_bytes=full * 3 // 4)
+    """A budget below the unlimited resident arena: smaller head groups,
+    each with every block on the device."""
+    N, H, d = 7 * 128, 4, 64
+    full = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True).info()
+    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True, mem_budget_bytes=full["host_arena_bytes"] * 3 // 4)
     info = plan.info()
-    assert info["host_resident"] == 1 and info["head_group"] < H
-    assert info["host_arena_bytes"] <= full * 3 // 4
+    assert info["host_resident"] == 1 and info["head_group"] < full["head_group"]
+    assert info["host_arena_bytes"] <= full["host_arena_bytes"] * 3 // 4
     check_schedule(plan)
-    assert bm.explore(*resident_model(plan, groups=H // info["head_group"]))
+    assert bm.explore(*resident_model(plan, groups=min(info["host_sets"] + 1, H // info["head_group"])))
