@@ -49,6 +49,14 @@ constexpr uint32_t BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizz
 constexpr float LOG2_RESCALE_THRESHOLD = 8.0f;
 constexpr int P_HALF_LEAD = 8;  // pairs of the second P half computed before the p_half arrival
 
+// Epilogue staging: a softmax warp's 32 output rows in fp32, in the operand
+// buffers (free once the last MMA is done), rows padded by 16 bytes so that
+// both the row-per-lane writes and the row-by-row reads are conflict-free.
+template <int D>
+struct EpiStride {
+    static constexpr int value = D + 4;
+};
+
 template <int D>
 struct Smem {
     static constexpr int KB = D / 64;
@@ -131,6 +139,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     Smem<D> &s = *reinterpret_cast<Smem<D> *>(smem_raw + pad);
+    constexpr int EPI_STRIDE = EpiStride<D>::value;
+    static_assert(offsetof(Smem<D>, k) == offsetof(Smem<D>, q) + sizeof(Smem<D>::q) &&
+                      offsetof(Smem<D>, v) == offsetof(Smem<D>, k) + sizeof(Smem<D>::k),
+                  "the epilogue stages rows across the q, k and v buffers");
+    static_assert(8 * 32 * EPI_STRIDE * sizeof(float) <=
+                      sizeof(Smem<D>::q) + sizeof(Smem<D>::k) + sizeof(Smem<D>::v),
+                  "epilogue staging exceeds the operand buffers");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -444,79 +459,86 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
             }
         }
         if (ok) ok = warp_wait(&s.o_full, 0, abort, tmo);
-        if (ok && p.epi == EPI_MERGE) {
-            // Fold this task's row into the running accumulator, or write
-            // the finished row (see epilogue.cuh).
+        if (ok) {
+            // o_full follows the last PV, so every operand buffer is free:
+            // each warp stages its 32 normalised rows there (one row per
+            // lane, as tensor memory hands them out), then writes them back
+            // row by row, a whole row per store instruction.
             tc_fence_after();
             const bool valid = q_local < e.q_hi;
             const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
             const float lse_n = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-            const bool first = (e.flags & SEG_FIRST) != 0, last = (e.flags & SEG_LAST) != 0;
-            const int64_t grow = (int64_t)q_local + e.q_goff;
-            const int64_t orow = (int64_t)e.out_lo + (q_local - e.q_lo);
-            FoldWeights w{0.f, 1.f, lse_n};
-            if (valid && !first) w = fold_weights(p.acc_lse[(int64_t)head * p.acc_rows + grow], lse_n);
-            float *acc = p.acc_o + (grow * p.H + head) * D;
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out) + (orow * p.H + head) * D;
+            float *stage = reinterpret_cast<float *>(&s.q[0][0][0]) + (size_t)warp * 32 * EPI_STRIDE;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
                 tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
                 tmem_wait_ld();
                 reg_fence32(o);
-                if (valid) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float4 v4 = make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(stage + lane * EPI_STRIDE + cc * 32 + i) =
+                        make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                    __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            }
+            __syncwarp();
+            constexpr int CH = D / 4;      // float4 chunks per row
+            constexpr int RPI = 32 / CH;   // rows per store instruction
+            const int rsub = lane / CH, c4 = (lane % CH) * 4;
+            const int32_t wq0 = q0 + t * BM + quarter * 32;  // local query row of lane 0
+            const int nrows = max(0, min(32, e.q_hi - wq0));
+            const int64_t orow0 = (int64_t)e.out_lo + (wq0 - e.q_lo);
+            const int64_t rstride = (int64_t)p.H * D;
+            if (p.epi == EPI_MERGE) {
+                // Fold this task's rows into the running accumulator, or
+                // write the finished rows (see epilogue.cuh).
+                const bool first = (e.flags & SEG_FIRST) != 0, last = (e.flags & SEG_LAST) != 0;
+                const int64_t grow0 = (int64_t)wq0 + e.q_goff;
+                FoldWeights w{0.f, 1.f, lse_n};
+                if (valid && !first) w = fold_weights(p.acc_lse[(int64_t)head * p.acc_rows + grow0 + lane], lse_n);
+                float *acc0 = p.acc_o + (grow0 * p.H + head) * D;
+                __nv_bfloat16 *dst0 = static_cast<__nv_bfloat16 *>(p.out) + (orow0 * p.H + head) * D;
+#pragma unroll 4
+                for (int r0 = 0; r0 < 32; r0 += RPI) {
+                    const int r = r0 + rsub;
+                    const float wa = __shfl_sync(0xffffffffu, w.wa, r);
+                    const float wn = __shfl_sync(0xffffffffu, w.wn, r);
+                    if (r < nrows) {
+                        float4 v4 = *reinterpret_cast<const float4 *>(stage + r * EPI_STRIDE + c4);
+                        float *arow = acc0 + r * rstride + c4;
                         if (!first) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(acc + cc * 32 + i);
-                            v4.x = w.wa * a4.x + w.wn * v4.x;
-                            v4.y = w.wa * a4.y + w.wn * v4.y;
-                            v4.z = w.wa * a4.z + w.wn * v4.z;
-                            v4.w = w.wa * a4.w + w.wn * v4.w;
+                            const float4 a4 = *reinterpret_cast<const float4 *>(arow);
+                            v4.x = wa * a4.x + wn * v4.x;
+                            v4.y = wa * a4.y + wn * v4.y;
+                            v4.z = wa * a4.z + wn * v4.z;
+                            v4.w = wa * a4.w + wn * v4.w;
                         }
                         if (last) {
-                            uint2 u;
-                            u.x = pack_bf16x2(v4.x, v4.y);
-                            u.y = pack_bf16x2(v4.z, v4.w);
-                            *reinterpret_cast<uint2 *>(dst + cc * 32 + i) = u;
+                            uint2 u2;
+                            u2.x = pack_bf16x2(v4.x, v4.y);
+                            u2.y = pack_bf16x2(v4.z, v4.w);
+                            *reinterpret_cast<uint2 *>(dst0 + r * rstride + c4) = u2;
                         } else {
-                            *reinterpret_cast<float4 *>(acc + cc * 32 + i) = v4;
+                            *reinterpret_cast<float4 *>(arow) = v4;
                         }
                     }
                 }
-            }
-            if (valid) {
-                if (last)
-                    p.out_lse[(int64_t)head * p.out_rows + orow] = w.lse;
-                else
-                    p.acc_lse[(int64_t)head * p.acc_rows + grow] = w.lse;
-            }
-        } else if (ok) {
-            tc_fence_after();
-            const bool valid = q_local < e.q_hi;
-            const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            const int64_t out_row = (int64_t)e.out_lo + (q_local - e.q_lo);
-            float *dst = p.part_o + (((int64_t)e.slot * p.part_rows + out_row) * p.H + head) * D;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(o_addr + (uint32_t)(cc * 32), o);
-                tmem_wait_ld();
-                reg_fence32(o);
                 if (valid) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float4 v4 = make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                        *reinterpret_cast<float4 *>(dst + cc * 32 + i) = v4;
-                    }
+                    if (last)
+                        p.out_lse[(int64_t)head * p.out_rows + orow0 + lane] = w.lse;
+                    else
+                        p.acc_lse[(int64_t)head * p.acc_rows + grow0 + lane] = w.lse;
                 }
-            }
-            if (valid) {
-                const float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-                p.part_lse[((int64_t)e.slot * p.H + head) * p.part_rows + out_row] = lse;
+            } else {
+                float *dst0 = p.part_o + (((int64_t)e.slot * p.part_rows + orow0) * p.H + head) * D;
+#pragma unroll 4
+                for (int r0 = 0; r0 < 32; r0 += RPI) {
+                    const int r = r0 + rsub;
+                    if (r < nrows)
+                        *reinterpret_cast<float4 *>(dst0 + r * rstride + c4) =
+                            *reinterpret_cast<const float4 *>(stage + r * EPI_STRIDE + c4);
+                }
+                if (valid) p.part_lse[((int64_t)e.slot * p.H + head) * p.part_rows + orow0 + lane] = lse_n;
             }
         } else {
             if (lane == 0) atomicExch(p.err, DEV_TIMEOUT);

@@ -129,7 +129,9 @@ def test_configs_plan():
     assert p1.info()["block_tokens"] == 512 and p1.info()["D"] == [[0, 1, 3]]
     p2 = cqsa.cqsa_plan(53248, 8, 128, 4, 1, False, 0)
     i2 = p2.info()
-    assert i2["block_tokens"] == 4096 and i2["num_tasks"] == 13 and i2["head_group"] == 8
+    # Unlimited memory: the resident host schedule with two buffer sets of half the heads.
+    assert i2["block_tokens"] == 4096 and i2["num_tasks"] == 13 and i2["head_group"] == 4
+    assert i2["host_resident"] == 1 and i2["host_sets"] == 2
     assert i2["useful_flops"] == 4.0 * 53248 ** 2 * 8 * 128
     p3 = cqsa.cqsa_plan(688128, 8, 128, 5, 1, False, 2 * GiB)
     i3 = p3.info()
