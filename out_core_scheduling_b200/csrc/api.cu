@@ -298,6 +298,11 @@ struct cqsa_plan {
     int nsets = 0;
     std::vector<DevWl> res_wl;
     cudaStream_t s_comp2 = nullptr;
+    // The second buffer set's two compute streams: with their own streams
+    // one head group's launches overlap the other's instead of queueing
+    // behind them.
+    cudaStream_t s_set1[2] = {nullptr, nullptr};
+    cudaStream_t res_stream(int set, int s) const { return set == 0 ? (s == 0 ? s_comp : s_comp2) : s_set1[s]; }
 
     // Kernel timing (cqsa_plan_profile): event pairs not yet read, a pool of
     // spare events, and the totals read so far.
@@ -477,6 +482,8 @@ cqsa_status_t setup_resident(cqsa_plan_t *P) {
     CK(cudaStreamCreateWithFlags(&P->s_comp, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_comp2, cudaStreamNonBlocking));
     CK(cudaStreamCreateWithFlags(&P->s_out, cudaStreamNonBlocking));
+    if (nsets > 1)
+        for (cudaStream_t &x : P->s_set1) CK(cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking));
     const int64_t A = pl.arrival_blocks();
     for (int st = 0; st < nsets; ++st) {
         cqsa_plan_t::ResidentSet &R = P->rs[st];
@@ -605,7 +612,7 @@ void release_host_mode(cqsa_plan_t *P) {
     }
     P->nsets = 0;
     P->res_wl.clear();
-    cudaStream_t *ss[4] = {&P->s_in, &P->s_comp, &P->s_comp2, &P->s_out};
+    cudaStream_t *ss[6] = {&P->s_in, &P->s_comp, &P->s_comp2, &P->s_out, &P->s_set1[0], &P->s_set1[1]};
     for (cudaStream_t *s : ss)
         if (*s) {
             cudaStreamDestroy(*s);
@@ -958,13 +965,15 @@ cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k
     const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
                *hv = static_cast<const char *>(v);
     char *ho = static_cast<char *>(out);
-    cudaStream_t sc[2] = {P->s_comp, P->s_comp2};
     CK(cudaEventRecord(P->ev_start, stream));
-    for (cudaStream_t x : {P->s_in, sc[0], sc[1], P->s_out}) CK(cudaStreamWaitEvent(x, P->ev_start, 0));
+    for (cudaStream_t x : {P->s_in, P->s_out}) CK(cudaStreamWaitEvent(x, P->ev_start, 0));
+    for (int z = 0; z < P->nsets; ++z)
+        for (int s = 0; s < 2; ++s) CK(cudaStreamWaitEvent(P->res_stream(z, s), P->ev_start, 0));
     int gi = 0;
     for (int h0 = 0; h0 < H; h0 += g, ++gi) {
         NvtxRange nvtx_group("cqsa resident head group", h0);
         cqsa_plan_t::ResidentSet &R = P->rs[gi % P->nsets];
+        const cudaStream_t sc[2] = {P->res_stream(gi % P->nsets, 0), P->res_stream(gi % P->nsets, 1)};
         if (gi >= P->nsets) {
             // The set's previous head group: its pools change once that
             // group's launches are done; its accumulators and finished rows
@@ -1169,6 +1178,11 @@ void join_after_error(cqsa_plan_t *P, cudaStream_t stream) {
         cudaEventRecord(P->rs[0].ev_comp_end[1], P->s_comp2);
         cudaStreamWaitEvent(stream, P->rs[0].ev_comp_end[1], 0);
     }
+    for (int s = 0; s < 2; ++s)
+        if (P->s_set1[s] && P->rs[1].ev_comp_end[s]) {
+            cudaEventRecord(P->rs[1].ev_comp_end[s], P->s_set1[s]);
+            cudaStreamWaitEvent(stream, P->rs[1].ev_comp_end[s], 0);
+        }
 }
 
 // ------------------------------------------------------------ owner exchange
@@ -1256,7 +1270,7 @@ cqsa_status_t setup_bwd_host_impl(cqsa_plan_t *P) {
                                      "(needs %lld block slots)", pl.spec.budget, (long long)pl.bwd_min_slots);
     // The streamed forward's arena and this one may not both fit the budget.
     if (P->host_arena && pl.spec.budget && P->host_bytes + z.arena > pl.spec.budget) {
-        cudaStream_t ss[4] = {P->s_in, P->s_comp, P->s_comp2, P->s_out};
+        cudaStream_t ss[6] = {P->s_in, P->s_comp, P->s_comp2, P->s_out, P->s_set1[0], P->s_set1[1]};
         for (cudaStream_t st : ss)
             if (st) CK(cudaStreamSynchronize(st));
         release_host_mode(P);
@@ -2230,7 +2244,7 @@ void cqsa_plan_destroy(cqsa_plan_t *plan) {
     if (!plan) return;
     if (plan->device >= 0) {
         release_bwd_host(plan);
-        cudaStream_t ss[4] = {plan->s_in, plan->s_comp, plan->s_comp2, plan->s_out};
+        cudaStream_t ss[6] = {plan->s_in, plan->s_comp, plan->s_comp2, plan->s_out, plan->s_set1[0], plan->s_set1[1]};
         for (cudaStream_t s : ss)
             if (s) cudaStreamSynchronize(s);
         if (plan->dev_arena || plan->bwd.arena || plan->bwd_shard.arena || plan->part_arena) cudaDeviceSynchronize();

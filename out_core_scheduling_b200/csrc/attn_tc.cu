@@ -321,6 +321,13 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         const uint32_t s_addr = lane_base + (uint32_t)t * 128u;
         const uint32_t o_addr = lane_base + 256u + (uint32_t)(t * D);
         const float sl2 = p.scale_log2;
+        if (p.epi == EPI_MERGE && !(e.flags & SEG_FIRST) && q_local < e.q_hi) {
+            // The running row this unit folds into at the end: fetch it into
+            // L2 now, so the epilogue does not wait on HBM.
+            const char *arow = reinterpret_cast<const char *>(p.acc_o + (q_glob * p.H + head) * D);
+#pragma unroll
+            for (int c = 0; c < D * 4; c += 128) prefetch_l2(arow + c);
+        }
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         int j = 0;
@@ -498,28 +505,38 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                 if (valid && !first) w = fold_weights(p.acc_lse[(int64_t)head * p.acc_rows + grow0 + lane], lse_n);
                 float *acc0 = p.acc_o + (grow0 * p.H + head) * D;
                 __nv_bfloat16 *dst0 = static_cast<__nv_bfloat16 *>(p.out) + (orow0 * p.H + head) * D;
-#pragma unroll 4
-                for (int r0 = 0; r0 < 32; r0 += RPI) {
-                    const int r = r0 + rsub;
-                    const float wa = __shfl_sync(0xffffffffu, w.wa, r);
-                    const float wn = __shfl_sync(0xffffffffu, w.wn, r);
-                    if (r < nrows) {
-                        float4 v4 = *reinterpret_cast<const float4 *>(stage + r * EPI_STRIDE + c4);
-                        float *arow = acc0 + r * rstride + c4;
-                        if (!first) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(arow);
-                            v4.x = wa * a4.x + wn * v4.x;
-                            v4.y = wa * a4.y + wn * v4.y;
-                            v4.z = wa * a4.z + wn * v4.z;
-                            v4.w = wa * a4.w + wn * v4.w;
-                        }
-                        if (last) {
-                            uint2 u2;
-                            u2.x = pack_bf16x2(v4.x, v4.y);
-                            u2.y = pack_bf16x2(v4.z, v4.w);
-                            *reinterpret_cast<uint2 *>(dst0 + r * rstride + c4) = u2;
-                        } else {
-                            *reinterpret_cast<float4 *>(arow) = v4;
+                // Eight rows per batch: their accumulator loads are all in
+                // flight before the first fold.
+                constexpr int RB = 8;
+                for (int r0 = 0; r0 < 32; r0 += RB * RPI) {
+                    float4 a4[RB];
+#pragma unroll
+                    for (int b = 0; b < RB; ++b) {
+                        const int r = r0 + b * RPI + rsub;
+                        a4[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (!first && r < nrows) a4[b] = *reinterpret_cast<const float4 *>(acc0 + r * rstride + c4);
+                    }
+#pragma unroll
+                    for (int b = 0; b < RB; ++b) {
+                        const int r = r0 + b * RPI + rsub;
+                        const float wa = __shfl_sync(0xffffffffu, w.wa, r);
+                        const float wn = __shfl_sync(0xffffffffu, w.wn, r);
+                        if (r < nrows) {
+                            float4 v4 = *reinterpret_cast<const float4 *>(stage + r * EPI_STRIDE + c4);
+                            if (!first) {
+                                v4.x = wa * a4[b].x + wn * v4.x;
+                                v4.y = wa * a4[b].y + wn * v4.y;
+                                v4.z = wa * a4[b].z + wn * v4.z;
+                                v4.w = wa * a4[b].w + wn * v4.w;
+                            }
+                            if (last) {
+                                uint2 u2;
+                                u2.x = pack_bf16x2(v4.x, v4.y);
+                                u2.y = pack_bf16x2(v4.z, v4.w);
+                                *reinterpret_cast<uint2 *>(dst0 + r * rstride + c4) = u2;
+                            } else {
+                                *reinterpret_cast<float4 *>(acc0 + r * rstride + c4) = v4;
+                            }
                         }
                     }
                 }

@@ -1,15 +1,17 @@
 """The streamed forward's resident schedule (every block of a head group on
 the device at once): its launches take every allowed pair exactly once, in
-an order that keeps each query block's merges sequential, and its four
-streams are race-free over every interleaving.
+an order that keeps each query block's merges sequential, and its streams
+are race-free over every interleaving.
 
-forward_host_resident (csrc/api.cu) enqueues, per head group:
+forward_host_resident (csrc/api.cu) enqueues, per head group, with z the
+group's buffer set (groups alternate over the sets; each set has its own
+two compute streams, the copy streams are shared):
 
-    copy stream     (after the previous group's launches: comp_end of both
-                    compute streams) every block's Q, K, V rows into its
-                    own pool slot, in increasing order; record arrive[a]
-                    after the last block of arrival group a
-    compute s       (after the previous group: comp_end of the other
+    copy stream     (after the set's previous group's launches: comp_end of
+                    both its compute streams) every block's Q, K, V rows
+                    into its own pool slot, in increasing order; record
+                    arrive[a] after the last block of arrival group a
+    compute (z, s)  (after the set's previous group: comp_end of the other
                     stream, out_end) per launch on s, in launch order: wait
                     arrive[group of need]; wait launch[after] (other
                     stream); the kernel reads its query and key blocks and
@@ -18,8 +20,8 @@ forward_host_resident (csrc/api.cu) enqueues, per head group:
     copy-out stream per launch that finishes query blocks: wait launch[i];
                     their rows to the host
 
-and records comp_end on both compute streams and out_end on the copy-out
-stream after the group.  A CUDA event wait refers to the latest record
+and records comp_end on both of the set's compute streams and out_end on
+the copy-out stream after the group.  A CUDA event wait refers to the latest record
 enqueued before it.  Dropping a wait is caught, except a compute stream's
 wait for the other stream's comp_end at a group boundary: every launch is
 followed, on its query blocks' chains, by the launch that finishes one of
@@ -101,7 +103,8 @@ def resident_model(plan, groups=2, drop=(), sets=None):
     L = _launches(plan)
     A, nb = info["arrival_blocks"], info["num_blocks"]
     sets = sets or info["host_sets"]
-    s_in, s_c, s_out = [], [[], []], []
+    s_in, s_out = [], []
+    s_cs = [[[], []] for _ in range(sets)]  # per buffer set, its two compute streams
     rec = defaultdict(int)
 
     def record(stream, name):
@@ -118,6 +121,7 @@ def resident_model(plan, groups=2, drop=(), sets=None):
     acc = {}
     for g in range(groups):
         z = g % sets  # the group's buffer set
+        s_c = s_cs[z]
         if g >= sets:
             wait(s_in, f"comp_end{z}_0", "pools_after_launches")
             wait(s_in, f"comp_end{z}_1", "pools_after_launches")
@@ -159,8 +163,8 @@ def resident_model(plan, groups=2, drop=(), sets=None):
         record(s_c[1], f"comp_end{z}_1")
         record(s_out, f"out_end{z}")
     counts = {name: 1 for name in rec}
-    return [("copy-in", s_in, 1), ("compute0", s_c[0], 1), ("compute1", s_c[1], 1),
-            ("copy-out", s_out, 1)], counts
+    comp = [(f"compute{z}_{s}", s_cs[z][s], 1) for z in range(sets) for s in (0, 1)]
+    return [("copy-in", s_in, 1)] + comp + [("copy-out", s_out, 1)], counts
 
 
 CASES = [
@@ -227,8 +231,10 @@ def test_resident_schedule_is_race_free(N, H, d, ls, causal):
 
 def test_two_buffer_sets_are_race_free():
     """Two buffer sets over three head groups: the second group overlaps the
-    first, the third reuses the first's buffers."""
-    plan = cqsa.cqsa_plan_ex(7 * 128, 2, 64, [3], causal=True)
+    first (on its own compute streams), the third reuses the first's
+    buffers.  Six streams: the smallest plan whose launches need
+    other-stream waits keeps the exploration in seconds."""
+    plan = cqsa.cqsa_plan_ex(3 * 128, 2, 64, [2], causal=False)
     assert plan.info()["host_sets"] == 2
     assert bm.explore(*resident_model(plan, groups=3))
 
@@ -241,7 +247,7 @@ def test_planted_missing_wait_is_caught(drop):
         bm.explore(*resident_model(plan, groups=2, drop=(drop,), sets=1))
     if drop not in ("after",):  # the causal plan's launches need no other-stream waits
         with pytest.raises(bm.Violation):
-            bm.explore(*resident_model(cqsa.cqsa_plan_ex(7 * 128, 2, 64, [3], causal=True), groups=3,
+            bm.explore(*resident_model(cqsa.cqsa_plan_ex(3 * 128, 2, 64, [2], causal=True), groups=3,
                                        drop=(drop,), sets=2))
 
 
