@@ -895,6 +895,7 @@ size_t Planner::host_arena_bytes(int g, const PoolPlan &pl) const {
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int64_t kArrivalGroups = 16;  // copy-in marks per head group (fewer when there are fewer blocks)
+constexpr int64_t kSms = 148;           // streaming multiprocessors of the B200
 }
 
 int64_t Planner::arrival_blocks() const {
@@ -925,14 +926,56 @@ std::vector<HostLaunch> Planner::host_launches(int rows_per_unit, int bn, int he
                 b0 = b1 + 1;
             }
     }
+    // Finishing slots that need the same block go m query groups to a
+    // launch, so that the two launches in flight (one per compute stream)
+    // cover the SMs; slots that become ready at different arrivals (causal
+    // plans) stay apart.
+    const int64_t unit_per_group =
+        (int64_t)heads * ((A * block + rows_per_unit - 1) / rows_per_unit);
+    const int64_t m = std::max<int64_t>(1, (kSms / 2 + unit_per_group - 1) / unit_per_group);
+    // Among slots ready at the same arrival, the longest chains of key
+    // blocks go first, so that the phase ends on short ones.
+    struct Fin {
+        int64_t need, chain, sl;
+    };
+    std::vector<Fin> fin;
+    for (int64_t sl = 2 * cut; sl < slots; ++sl) {
+        if (pairs[sl].empty()) continue;
+        Fin f{0, 0, sl};
+        for (const auto &qk : pairs[sl]) {
+            int64_t chain = 0;
+            for (const auto &r : qk.second) {
+                f.need = std::max(f.need, std::max(qk.first, r.second));
+                chain += r.second - r.first + 1;
+            }
+            f.chain = std::max(f.chain, chain);
+        }
+        fin.push_back(f);
+    }
+    std::stable_sort(fin.begin(), fin.end(), [](const Fin &a, const Fin &b) {
+        return a.need != b.need ? a.need < b.need : a.chain > b.chain;
+    });
+    std::vector<std::map<int64_t, Runs>> launch_pairs(pairs.begin(), pairs.begin() + 2 * cut);
+    int64_t in_launch = 0, launch_need = -1;
+    for (const Fin &f : fin) {
+        const int64_t sl = f.sl, need = f.need;
+        if (in_launch > 0 && in_launch < m && need == launch_need) {
+            launch_pairs.back().insert(pairs[sl].begin(), pairs[sl].end());
+            ++in_launch;
+        } else {
+            launch_pairs.push_back(std::move(pairs[sl]));
+            in_launch = 1;
+            launch_need = need;
+        }
+    }
     std::vector<HostLaunch> out;
     std::vector<int64_t> last(num_blocks, -1);  // latest launch that touched a query block
     std::vector<std::pair<int64_t, int32_t>> last_entry(num_blocks, {-1, -1});  // (launch, entry)
-    for (int64_t sl = 0; sl < slots; ++sl) {
-        if (pairs[sl].empty()) continue;
+    for (auto &lp : launch_pairs) {
+        if (lp.empty()) continue;
         HostLaunch L;
         L.stream = (int32_t)(out.size() & 1);
-        for (auto &qk : pairs[sl]) {
+        for (auto &qk : lp) {
             const int64_t qb = qk.first;
             Runs &kr = qk.second;
             std::sort(kr.begin(), kr.end());

@@ -269,10 +269,11 @@ def test_budget_below_the_resident_arena_runs_task_by_task():
 
 def test_resident_head_groups_replay_the_schedule():
     """A budget below the unlimited resident arena: smaller head groups,
-    each with every block on the device."""
-    N, H, d = 7 * 128, 4, 64
-    full = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True).info()
-    plan = cqsa.cqsa_plan_ex(N, H, d, [3], causal=True, mem_budget_bytes=full["host_arena_bytes"] * 3 // 4)
+    each with every block on the device (three groups over the two buffer
+    sets: six streams, so a three-block plan)."""
+    N, H, d = 3 * 128, 4, 64
+    full = cqsa.cqsa_plan_ex(N, H, d, [2], causal=True).info()
+    plan = cqsa.cqsa_plan_ex(N, H, d, [2], causal=True, mem_budget_bytes=full["host_arena_bytes"] * 3 // 4)
     info = plan.info()
     assert info["host_resident"] == 1 and info["head_group"] < full["head_group"]
     assert info["host_arena_bytes"] <= full["host_arena_bytes"] * 3 // 4
