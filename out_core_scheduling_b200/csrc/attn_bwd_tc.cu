@@ -86,6 +86,60 @@ struct SmemKv {
     int abort;
 };
 
+// Epilogue stores of one warp's 32 stationary rows.  The lanes hold their
+// own rows (as tensor memory hands them out); staged in shared memory (rows
+// padded by 16 bytes, so both the row-per-lane writes and the row-by-row
+// reads are conflict-free), they leave row-contiguous: CH lanes per row,
+// 32 / CH rows per store instruction.
+template <int COLS>
+__device__ __forceinline__ void store_rows_f32(const float *stage, int str, int nrows, int lane, float *dst0,
+                                               int64_t rstride, bool accum) {
+    constexpr int CH = COLS / 4;
+    constexpr int RPI = 32 / CH;
+    constexpr int RB = 8;  // rows in flight per batch when adding into running sums
+    const int rsub = lane / CH, c4 = (lane % CH) * 4;
+    for (int r0 = 0; r0 < 32; r0 += RB * RPI) {
+        float4 a4[RB];
+#pragma unroll
+        for (int b = 0; b < RB; ++b) {
+            const int r = r0 + b * RPI + rsub;
+            a4[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (accum && r < nrows) a4[b] = *reinterpret_cast<const float4 *>(dst0 + r * rstride + c4);
+        }
+#pragma unroll
+        for (int b = 0; b < RB; ++b) {
+            const int r = r0 + b * RPI + rsub;
+            if (r < nrows) {
+                float4 v = *reinterpret_cast<const float4 *>(stage + r * str + c4);
+                v.x += a4[b].x;
+                v.y += a4[b].y;
+                v.z += a4[b].z;
+                v.w += a4[b].w;
+                *reinterpret_cast<float4 *>(dst0 + r * rstride + c4) = v;
+            }
+        }
+    }
+}
+
+template <int COLS>
+__device__ __forceinline__ void store_rows_bf16(const float *stage, int str, int nrows, int lane,
+                                                __nv_bfloat16 *dst0, int64_t rstride) {
+    constexpr int CH = COLS / 4;
+    constexpr int RPI = 32 / CH;
+    const int rsub = lane / CH, c4 = (lane % CH) * 4;
+#pragma unroll 4
+    for (int r0 = 0; r0 < 32; r0 += RPI) {
+        const int r = r0 + rsub;
+        if (r < nrows) {
+            const float4 v = *reinterpret_cast<const float4 *>(stage + r * str + c4);
+            uint2 w;
+            w.x = pack_bf16x2(v.x, v.y);
+            w.y = pack_bf16x2(v.z, v.w);
+            *reinterpret_cast<uint2 *>(dst0 + r * rstride + c4) = w;
+        }
+    }
+}
+
 // Four floats from shared memory, kept in program order (not hoisted ahead
 // of the arithmetic that precedes them, which would raise register pressure).
 __device__ __forceinline__ float4 lds_f4(const float *p) {
@@ -392,10 +446,17 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
         }
         if (ok) ok = warp_wait_b(&s.o_full, 0, abort, tmo);
         if (ok) {
+            // o_full follows the last dQ MMA, so the operand buffers are
+            // free: each warp stages its rows' D/2 features there.
             tc_fence_after();
             const bool fused = (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
-            const int64_t orow = (int64_t)e.out_lo + (q_local - e.q_lo);
-            // This warp writes features hf * D/2 .. of its row.
+            constexpr int HC = D / 2, STR = HC + 4;
+            static_assert(offsetof(SmemDq<D>, dout) == offsetof(SmemDq<D>, q) + sizeof(SmemDq<D>::q) &&
+                              offsetof(SmemDq<D>, k) == offsetof(SmemDq<D>, dout) + sizeof(SmemDq<D>::dout) &&
+                              EW_WARPS * 32 * STR * sizeof(float) <=
+                                  sizeof(SmemDq<D>::q) + sizeof(SmemDq<D>::dout) + sizeof(SmemDq<D>::k),
+                          "dq epilogue staging exceeds the q, dout and k buffers");
+            float *stage = reinterpret_cast<float *>(&s.q[0][0]) + (size_t)warp * 32 * STR;
 #pragma unroll
             for (int ch = 0; ch < D / 64; ++ch) {
                 const int cc = hf * (D / 64) + ch;
@@ -403,37 +464,25 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
                 tmem_ld32(lane_base + 256u + (uint32_t)(cc * 32), o);
                 tmem_wait_ld();
                 fence_regs32(o);
-                if (valid) {
-                    if (fused) {
-                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.out_a) + (orow * p.H + head) * D;
 #pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            uint2 w;
-                            w.x = pack_bf16x2(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale);
-                            w.y = pack_bf16x2(__uint_as_float(o[i + 2]) * p.scale,
-                                              __uint_as_float(o[i + 3]) * p.scale);
-                            *reinterpret_cast<uint2 *>(dst + cc * 32 + i) = w;
-                        }
-                    } else {
-                        float *dst = p.part_a + (((int64_t)e.slot * p.N + orow) * p.H + head) * D;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4) {
-                            float4 g4 = make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
-                                                    __uint_as_float(o[i + 2]) * p.scale,
-                                                    __uint_as_float(o[i + 3]) * p.scale);
-                            float4 *d4 = reinterpret_cast<float4 *>(dst + cc * 32 + i);
-                            if (p.accum) {  // streamed backward: add into the block's running sums
-                                const float4 a4 = *d4;
-                                g4.x += a4.x;
-                                g4.y += a4.y;
-                                g4.z += a4.z;
-                                g4.w += a4.w;
-                            }
-                            *d4 = g4;
-                        }
-                    }
-                }
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(stage + lane * STR + ch * 32 + i) =
+                        make_float4(__uint_as_float(o[i]) * p.scale, __uint_as_float(o[i + 1]) * p.scale,
+                                    __uint_as_float(o[i + 2]) * p.scale, __uint_as_float(o[i + 3]) * p.scale);
             }
+            __syncwarp();
+            const int32_t wq0 = q0 + quarter * 32;  // local query row of lane 0
+            const int nrows = max(0, min(32, q_end - wq0));
+            const int64_t orow0 = (int64_t)e.out_lo + (wq0 - e.q_lo);
+            const int64_t rstride = (int64_t)p.H * D;
+            if (fused)
+                store_rows_bf16<HC>(stage, STR, nrows, lane,
+                                    static_cast<__nv_bfloat16 *>(p.out_a) + (orow0 * p.H + head) * D + hf * HC,
+                                    rstride);
+            else
+                store_rows_f32<HC>(stage, STR, nrows, lane,
+                                   p.part_a + (((int64_t)e.slot * p.N + orow0) * p.H + head) * D + hf * HC, rstride,
+                                   p.accum != 0);
         } else if (lane == 0) {
             atomicExch(err, DEV_TIMEOUT);
         }
@@ -713,52 +762,49 @@ __global__ void __launch_bounds__(btc::THREADS, 1)
             // Direct writes only when one query head owns the key/value head;
             // otherwise each query head of the group has its own slot.
             const bool fused = p.kv_group == 1 && (e.flags & (SEG_FIRST | SEG_LAST)) == (SEG_FIRST | SEG_LAST);
-            const int64_t orow = (int64_t)e.out_lo + (k_local - e.q_lo);
             const int hkv = head / p.kv_group;
             // Streamed backward: one launch never holds two query heads of a
             // key/value group, so they all add into the one set of sums.
             const int64_t slot = p.accum ? 0 : (int64_t)e.slot * p.kv_group + head % p.kv_group;
-            // Warps of columns 0-63 write dK, those of 64-127 dV.
-            {
-                const int which = hf;
-                const uint32_t col = which == 0 ? COL_DK : COL_DV;
-                const float mul = which == 0 ? p.scale : 1.f;
+            // Warps of columns 0-63 write dK, those of 64-127 dV, staged
+            // through the operand buffers (free once o_full is in).
+            const int which = hf;
+            const uint32_t col = which == 0 ? COL_DK : COL_DV;
+            const float mul = which == 0 ? p.scale : 1.f;
+            constexpr int STR = D + 4;
+            static_assert(offsetof(SmemKv<D>, v) == offsetof(SmemKv<D>, k) + sizeof(SmemKv<D>::k) &&
+                              offsetof(SmemKv<D>, q) == offsetof(SmemKv<D>, v) + sizeof(SmemKv<D>::v) &&
+                              offsetof(SmemKv<D>, dout) == offsetof(SmemKv<D>, q) + sizeof(SmemKv<D>::q) &&
+                              EW_WARPS * 32 * STR * sizeof(float) <= sizeof(SmemKv<D>::k) + sizeof(SmemKv<D>::v) +
+                                                                        sizeof(SmemKv<D>::q) + sizeof(SmemKv<D>::dout),
+                          "dk/dv epilogue staging exceeds the operand buffers");
+            float *stage = reinterpret_cast<float *>(&s.k[0][0]) + (size_t)warp * 32 * STR;
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + col + (uint32_t)(cc * 32), o);
-                    tmem_wait_ld();
-                    fence_regs32(o);
-                    if (!valid) continue;
-                    if (fused) {
-                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? p.out_a : p.out_b) +
-                                             (orow * p.Hkv + hkv) * D;
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + col + (uint32_t)(cc * 32), o);
+                tmem_wait_ld();
+                fence_regs32(o);
 #pragma unroll
-                        for (int x = 0; x < 32; x += 4) {
-                            uint2 w;
-                            w.x = pack_bf16x2(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul);
-                            w.y = pack_bf16x2(__uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
-                            *reinterpret_cast<uint2 *>(dst + cc * 32 + x) = w;
-                        }
-                    } else {
-                        float *dst = (which == 0 ? p.part_a : p.part_b) + ((slot * p.N + orow) * p.Hkv + hkv) * D;
-#pragma unroll
-                        for (int x = 0; x < 32; x += 4) {
-                            float4 g4 = make_float4(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul,
-                                                    __uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
-                            float4 *d4 = reinterpret_cast<float4 *>(dst + cc * 32 + x);
-                            if (p.accum) {  // streamed backward: add into the block's running sums
-                                const float4 a4 = *d4;
-                                g4.x += a4.x;
-                                g4.y += a4.y;
-                                g4.z += a4.z;
-                                g4.w += a4.w;
-                            }
-                            *d4 = g4;
-                        }
-                    }
-                }
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4 *>(stage + lane * STR + cc * 32 + x) =
+                        make_float4(__uint_as_float(o[x]) * mul, __uint_as_float(o[x + 1]) * mul,
+                                    __uint_as_float(o[x + 2]) * mul, __uint_as_float(o[x + 3]) * mul);
             }
+            __syncwarp();
+            const int32_t wk0 = k0 + quarter * 32;  // local key row of lane 0
+            const int nrows = max(0, min(32, k_end - wk0));
+            const int64_t orow0 = (int64_t)e.out_lo + (wk0 - e.q_lo);
+            const int64_t rstride = (int64_t)p.Hkv * D;
+            if (fused)
+                store_rows_bf16<D>(stage, STR, nrows, lane,
+                                   static_cast<__nv_bfloat16 *>(which == 0 ? p.out_a : p.out_b) +
+                                       (orow0 * p.Hkv + hkv) * D,
+                                   rstride);
+            else
+                store_rows_f32<D>(stage, STR, nrows, lane,
+                                  (which == 0 ? p.part_a : p.part_b) + ((slot * p.N + orow0) * p.Hkv + hkv) * D,
+                                  rstride, p.accum != 0);
         } else if (lane == 0) {
             atomicExch(err, DEV_TIMEOUT);
         }
