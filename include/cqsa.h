@@ -195,7 +195,10 @@ cqsa_status_t cqsa_plan_ex(const cqsa_plan_desc_t *desc, cqsa_plan_t **out);
  *     task's missing Q/K/V blocks are copied into a device block cache on a
  *     copy stream, computed, folded into device-resident accumulators of the
  *     current head group in the kernel's epilogue, and finished blocks are
- *     copied back.
+ *     copied back.  When every block of a head group fits the budget
+ *     (info.host_resident), the resident schedule runs instead: each block
+ *     is copied once per head group and each pair of blocks computed as soon
+ *     as both have arrived (cqsa_plan_host_launch).
  *   stream: a cudaStream_t (0 = legacy default stream) the call is ordered
  *     after and that is ordered after all of its work.
  * Asynchronous: returns once all work is enqueued.  The first call on a plan
@@ -430,10 +433,11 @@ cqsa_status_t cqsa_plan_bwd_cache_task(const cqsa_plan_t *plan, int64_t t, int64
  * info.arrival_blocks consecutive blocks.  With info.host_sets = 2 the
  * head groups alternate between two sets of device buffers, so one group's
  * copies run while the previous group's launches do; a group waits only for
- * the group before last (the same set).  The launch waits for the mark of
- * the group holding *need (the last block it reads), runs on internal
- * compute stream *stream (0 or 1), and first waits for launch *after of the
- * other stream (-1: none).  It takes the plan's (query block, key block)
+ * the group before last (the same set).  Each set has its own two internal
+ * compute streams, so the launches of consecutive groups also overlap.  The
+ * launch waits for the mark of the group holding *need (the last block it
+ * reads), runs on its set's compute stream *stream (0 or 1), and first
+ * waits for launch *after of the other stream (-1: none).  It takes the plan's (query block, key block)
  * pairs pairs[2p], pairs[2p + 1], p < *num_pairs, in query-block order;
  * flags[p] is its entry's SEG flags for that query block (1: the block's
  * first launch, starts its accumulator; 2: its last, writes its finished
