@@ -150,6 +150,30 @@ def test_resident_repeat_is_deterministic(causal):
         assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+def test_two_plans_on_two_streams_host():
+    """Two independent streamed forwards in flight at once, each plan on a
+    stream of its own (the pattern of bench.py's end-to-end step): each
+    result is bit-identical to the same call run alone, and within the
+    tolerances of the oracle on every row."""
+    N, H, d = 13 * 256, 4, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=37, host=True)
+    plans = [cqsa.cqsa_plan_ex(N, H, d, [4], causal=c) for c in (False, True)]
+    assert all(p.info()["host_resident"] == 1 and p.info()["host_sets"] == 2 for p in plans)
+    alone = [run(p, q, k, v, cqsa.CQSA_HOST) for p in plans]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [(torch.empty(q.shape, dtype=q.dtype).pin_memory(), torch.empty(H, N, dtype=torch.float32).pin_memory())
+            for _ in plans]
+    for _ in range(3):
+        for p, (o, l), st in zip(plans, outs, streams):
+            cqsa.cqsa_forward(p, q, k, v, o, l, cqsa.CQSA_HOST, st)
+        torch.cuda.synchronize()
+        for p, (o, l), (ao, al) in zip(plans, outs, alone):
+            p.sync()
+            assert torch.equal(o, ao) and torch.equal(l, al)
+    for (o, l), c in zip(outs, (False, True)):
+        check(o, l, q, k, v, np.arange(N), c)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_streamed_two_level(causal):
     N, H, d = 91 * 128, 2, 128
