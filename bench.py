@@ -496,7 +496,9 @@ def measure(args, W, D, workload, steps, warmup, extras):
         roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak if achieved else None,
                     "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 x 1965 MHz",
-                    "traffic": None, "kernel": f"attn_simt_kernel<{d}>",
+                    "traffic": (profile_traffic("attn_simt.cu", "attn_simt_l3_n3584_h1_d64_fp32.md")
+                                if workload == FP32_EXTRA else None),
+                    "kernel": f"attn_simt_kernel<{d}>",
                     "avg_launch_ms": launch_ms}
     merge = None
     merge_ms = sum(s["merge_ms"] for s in stats)
