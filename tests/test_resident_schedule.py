@@ -279,3 +279,29 @@ def test_resident_head_groups_replay_the_schedule():
     assert info["host_arena_bytes"] <= full["host_arena_bytes"] * 3 // 4
     check_schedule(plan)
     assert bm.explore(*resident_model(plan, groups=min(info["host_sets"] + 1, H // info["head_group"])))
+
+
+def test_finishing_launches_fill_the_sms():
+    """The finishing phase of the default workload's non-causal plan: launches
+    of two query blocks (two launches in flight, one per compute stream,
+    then hold 2 x 2 x 64 units for 148 SMs), the longest key chains first;
+    the causal plan's finishing launches become ready at different arrivals
+    and stay one query block each."""
+    N, H, d = 53248, 8, 128
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=False)
+    info = plan.info()
+    assert info["head_group"] == 4 and info["arrival_blocks"] == 1
+    L, _ = check_schedule(plan)
+    fin = [x for x in L if x["need"] == info["num_blocks"] - 1]
+    chains = []
+    for x in fin:
+        per_q = defaultdict(int)
+        for q, _ in x["pairs"]:
+            per_q[q] += 1
+        assert len(per_q) <= 2
+        chains.append(max(per_q.values()))
+    assert sum(len({q for q, _ in x["pairs"]}) == 2 for x in fin) >= len(fin) - 1
+    assert chains == sorted(chains, reverse=True)
+    causal = cqsa.cqsa_plan_ex(N, H, d, [4], causal=True)
+    Lc, _ = check_schedule(causal)
+    assert all(len({q for q, _ in x["pairs"]}) == 1 for x in Lc)
