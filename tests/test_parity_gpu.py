@@ -150,6 +150,23 @@ def test_resident_repeat_is_deterministic(causal):
         assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_resident_buffer_sets_reused(causal):
+    """Four head groups over two buffer sets, so the third and fourth groups
+    reuse the first two's device buffers (and their compute streams): every
+    row against the oracle, and bit-identical on a repeat."""
+    N, H, d = 13 * 256, 8, 128
+    q, k, v = _inputs(N, H, d, torch.bfloat16, seed=41, host=True)
+    full = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal).info()["host_arena_bytes"]
+    plan = cqsa.cqsa_plan_ex(N, H, d, [4], causal=causal, mem_budget_bytes=full - 1)
+    info = plan.info()
+    assert info["host_resident"] == 1 and info["host_sets"] == 2 and H // info["head_group"] == 4
+    out, lse = run(plan, q, k, v, cqsa.CQSA_HOST)
+    check(out, lse, q, k, v, np.arange(N), causal)
+    out2, lse2 = run(plan, q, k, v, cqsa.CQSA_HOST)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
 def test_two_plans_on_two_streams_host():
     """Two independent streamed forwards in flight at once, each plan on a
     stream of its own (the pattern of bench.py's end-to-end step): each
