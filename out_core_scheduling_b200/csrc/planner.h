@@ -174,8 +174,10 @@ struct Sizing {
 // arrive, launch pairs come in two kinds per arrival group k: the new
 // query blocks of group k against keys of groups <= k, and the query
 // blocks of earlier groups against the keys of group k.  Pairs that need
-// one of the last arrival groups are taken query group by query group, so
-// that finished rows go to the host while the rest still computes.
+// one of the last arrival groups are taken a few query groups at a time
+// (enough for two launches in flight to cover the SMs; groups ready at the
+// same arrival only, longest key chains first), so that finished rows go
+// to the host while the rest still computes.
 // Launches alternate between two compute streams; a launch waits for the
 // latest launch on the other stream that touched one of its query blocks
 // (launches on one stream run in order), so the merges of a query block
