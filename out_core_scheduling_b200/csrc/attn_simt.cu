@@ -24,8 +24,9 @@
 // launcher picks S so that small problems still fill every SM): CTA rank r
 // of the cluster takes the r-th contiguous share of the unit's key tiles,
 // and the cluster combines the S online-softmax states (m, l, O) through
-// distributed shared memory before rank 0 writes the unit's result, so the
-// work list, the slots and the merge are those of an unsplit unit.
+// distributed shared memory, each rank finishing and writing a share of
+// the unit's rows, so the work list, the slots and the merge are those of
+// an unsplit unit.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -314,30 +315,47 @@ __global__ void __launch_bounds__(simt::THREADS)
             f2_unpack(o2[0][g][jj], o[0][g][jj], o[1][g][jj]);
             f2_unpack(o2[1][g][jj], o[2][g][jj], o[3][g][jj]);
         }
+    // With a key split, each rank finishes a share of the rows: rank r takes
+    // the threads of rows 4 ty .. 4 ty + 3 for ty in [16 r / S, 16 (r + 1) / S).
+    const bool finisher = ty >= (16 * rank) / S && ty < (16 * (rank + 1)) / S;
     if (S > 1) {
-        // Combine the cluster's states: ranks >= 1 leave (m, l, O) in their
+        // Combine the cluster's states: every rank leaves (m, l, O) in its
         // own shared memory, element-major so that a warp's reads are
-        // contiguous; rank 0 reads them remotely and rescales to the common
-        // maximum.  The second cluster barrier keeps the senders' shared
-        // memory alive until rank 0 has read it.
+        // contiguous; each rank's finishing threads fold the states of their
+        // rows in rank order (rank 0's, then 1, 2, ...: the same order, and
+        // so the same result, whichever rank finishes them), reading the
+        // other ranks' remotely and rescaling to the common maximum, so the
+        // ranks combine and write their shares in parallel.  The second
+        // cluster barrier keeps every rank's shared memory alive until the
+        // others have read it.
         constexpr int NV = 8 + 16 * G;  // values per thread
         __syncthreads();
         float *xs = smf;
-        if (rank > 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                xs[(2 * i) * THREADS + tid] = m[i];
-                xs[(2 * i + 1) * THREADS + tid] = l[i];
+        for (int i = 0; i < 4; ++i) {
+            xs[(2 * i) * THREADS + tid] = m[i];
+            xs[(2 * i + 1) * THREADS + tid] = l[i];
 #pragma unroll
-                for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) xs[(8 + (i * G + g) * 4 + jj) * THREADS + tid] = o[i][g][jj];
-            }
+                for (int jj = 0; jj < 4; ++jj) xs[(8 + (i * G + g) * 4 + jj) * THREADS + tid] = o[i][g][jj];
         }
         cluster.sync();
-        if (rank == 0) {
+        if (finisher) {
+            if (rank != 0) {
+                const float *r0 = cluster.map_shared_rank(xs, 0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    m[i] = r0[(2 * i) * THREADS + tid];
+                    l[i] = r0[(2 * i + 1) * THREADS + tid];
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) o[i][g][jj] = r0[(8 + (i * G + g) * 4 + jj) * THREADS + tid];
+                }
+            }
             for (int rr = 1; rr < S; ++rr) {
-                const float *rx = cluster.map_shared_rank(xs, rr);
+                const float *rx = cluster.map_shared_rank(xs, rr);  // this rank's own state when rr == rank
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float mr = rx[(2 * i) * THREADS + tid], lr = rx[(2 * i + 1) * THREADS + tid];
@@ -355,9 +373,9 @@ __global__ void __launch_bounds__(simt::THREADS)
             }
         }
         cluster.sync();
-        if (rank > 0) return;
         static_assert(NV * THREADS <= L::FLOATS, "combine area fits the shared tiles");
     }
+    if (!finisher) return;
 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
