@@ -948,10 +948,12 @@ cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, 
 
 // The resident schedule (Planner::host_sched): per head group, every block
 // to its own pool slot in increasing order with a mark per arrival group;
-// each launch on its compute stream after its blocks' mark and the launch of
-// the other stream it depends on; the rows it finishes to the host.  The
-// enqueue order is modelled in tests/test_resident_schedule.py over every
-// interleaving of the four streams.
+// each launch on its buffer set's compute stream after its blocks' mark and
+// the launch of the set's other stream it depends on; the rows it finishes
+// to the host.  Head groups alternate over the buffer sets, each set with
+// its own two compute streams; the copy streams are shared.  The enqueue
+// order is modelled in tests/test_resident_schedule.py over every
+// interleaving of the streams.
 cqsa_status_t forward_host_resident(cqsa_plan_t *P, const void *q, const void *k, const void *v, void *out,
                                     float *lse, cudaStream_t stream) {
     const Planner &pl = P->pl;
