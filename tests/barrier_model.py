@@ -335,11 +335,14 @@ def _cols(prefix, warps):
     return [f"{prefix}.w{w}.{c}" for w in range(warps) for c in ("c0", "c1", "rest")]
 
 
-def forward_model(n, warps=2, qt=2, stages=2, data=True):
+def forward_model(n, warps=2, qt=2, stages=2, data=True, stage_epilogue=True):
     """Forward tile kernel: TMA producer, MMA issuer, ``warps`` softmax warps
     (lane quarters) per query tile (the kernel has 4).  The softmax always
-    takes the lazy O rescale branch (a superset of the kernel's accesses)."""
+    takes the lazy O rescale branch (a superset of the kernel's accesses).
+    With ``stage_epilogue``, each softmax warp's epilogue then stores into
+    the Q, K and V buffers (its staging rows)."""
     D = data
+    fwd_operands = [f"q{t}" for t in range(qt)] + [f"{x}{s}" for x in ("k", "v") for s in range(stages)]
     tma = [("tma", "bar_q", [(f"q{t}", "Q") for t in range(qt)] if D else [])]
     for j in range(n):
         st = j % stages
@@ -400,11 +403,15 @@ def forward_model(n, warps=2, qt=2, stages=2, data=True):
             sm += [("wait", "o_full", 0)]
             if D and n > 0:
                 sm += [("ld", [(f"O{t}.w{w}", ("O", t, n - 1))])]
+            if D and stage_epilogue:
+                # The epilogue stages the warp's rows in the operand buffers
+                # (modelled as a store to all of them).
+                sm += [("st", [(r, None, ("E", t, w)) for r in fwd_operands])]
             roles.append((f"softmax{t}.{w}", sm, 1) if D else (f"softmax{t}", sm, warps))
     return roles, counts
 
 
-def dq_model(n, warps=2, kst=3, vst=2, split_handoff=True, data=True):
+def dq_model(n, warps=2, kst=3, vst=2, split_handoff=True, data=True, stage_epilogue=True):
     """dq gradient kernel; ``warps`` elementwise warps, each owning one
     column half (the kernel's 8 are 4 lane quarters x 2 halves).
     ``split_handoff=False`` is the earlier form with one p_half / p_full
@@ -467,6 +474,8 @@ def dq_model(n, warps=2, kst=3, vst=2, split_handoff=True, data=True):
         ew += [("wait", "o_full", 0)]
         if D and n > 0:
             ew += [("ld", [(f"dQ.w{w}", ("dQ", n - 1, 1))])]
+        if D and stage_epilogue:  # dQ rows staged in the Q, dO and K buffers
+            ew += [("st", [(r, None, ("E", w)) for r in ["q", "dout"] + [f"k{i}" for i in range(kst)]])]
         roles.append((f"elementwise{w}", ew, 1) if D else ("elementwise", ew, warps))
     counts = {"bar_q": 1, "s_ready0": 1, "s_ready1": 1, "dp_ready": 1, "dp_free": warps, "o_full": 1,
               "drain": 1}
@@ -482,7 +491,7 @@ def dq_model(n, warps=2, kst=3, vst=2, split_handoff=True, data=True):
     return roles, counts
 
 
-def dkdv_model(n, warps=2, stages=2, data=True):
+def dkdv_model(n, warps=2, stages=2, data=True, stage_epilogue=True):
     """dk/dv gradient kernel (the loop runs over query tiles).  A Q / dO
     stage completes on two arrivals: the copy's expect_tx (issued first) and
     the TMA warp's arrival once it has stored the tile's lse and D (region
@@ -542,6 +551,9 @@ def dkdv_model(n, warps=2, stages=2, data=True):
         ew += [("wait", "o_full", 0)]
         if D and n > 0:  # warps of columns 0-63 write dK, those of 64-127 dV
             ew += [("ld", [("dK", ("dK", n - 1))] if w % 2 == 0 else [("dV", ("dV", n - 1))])]
+        if D and stage_epilogue:  # dK / dV rows staged in the K, V, Q and dO buffers
+            ew += [("st", [(r, None, ("E", w)) for r in ["k", "v"] + [f"{x}{s}" for x in ("q", "dout")
+                                                                     for s in range(stages)]])]
         roles.append((f"elementwise{w}", ew, 1) if D else ("elementwise", ew, warps))
     counts = {"bar_kv": 1, "st_full": 1, "dp_full": 1, "pt_full": warps, "ds_full": warps, "o_full": 1,
               "drain": 1}

@@ -193,3 +193,19 @@ def test_models_match_the_kernels(src, struct):
              "SmemKv": lambda: bm.dkdv_model(3, stages=c["STAGES"], data=False)}[struct]
     default = {"Smem": bm.forward_model, "SmemDq": bm.dq_model, "SmemKv": bm.dkdv_model}[struct](3, data=False)
     assert bars == set(model()[1]) == set(default[1])
+
+
+@pytest.mark.parametrize("model,n", [(bm.forward_model, 2), (bm.dq_model, 2), (bm.dkdv_model, 2)])
+def test_epilogue_staging_before_o_full_is_caught(model, n):
+    """The epilogues stage rows in the operand buffers, which is safe only
+    once o_full says every MMA (and so every copy it consumed) is done:
+    staging before that wait races with an issued MMA or a copy."""
+    roles, counts = model(n, warps=1)
+
+    def early(ops):
+        i = ops.index(("wait", "o_full", 0))
+        return ops[:i] + [ops[-1]] + ops[i:-1]  # the staging store is the role's last op
+
+    edited = [(r, early(ops) if r.startswith(("softmax", "elementwise")) else ops, c) for r, ops, c in roles]
+    with pytest.raises(bm.Violation):
+        bm.explore(edited, counts)
